@@ -1,0 +1,323 @@
+// Lightning Attention forward -- plain fp64 CPU oracle.
+//
+// TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and bench.py's
+// cpu_baseline / reference arm may load or run this code.  It shares no code,
+// header, table or helper with the CUDA library, and it never routes product calls.
+//
+// Sources (web pages; cited by title and section):
+//   [Tut64]  "六十四：MiniMax-01" (LLM tutorial, lesson 64), section 3 "Lightning Attention 的定位":
+//            linear attention as a running state, S_t = S_{t-1} + phi(k_t) v_t^T, and the
+//            output read from the state, phi(q_t)^T S_t (sum over i <= t: causal, inclusive).
+//   [Arch]   "MiniMax-Text-01 405B MoE模型架构与训练策略解析", section 2.1 "Lightning Attention-2":
+//            Q, K, V = SiLU(X);  Y = Q * (K^T * V);  output = RMSNorm(Y) * sigmoid(X).
+//   [Ops]    "MiniMax-01技术报告解读（二）计算优化", section 3: lightning_attention_chunk_size 256 and
+//            lightning_attention_pad_options [32, 64, 128] (block size and tail padding).
+//
+// Readings taken where the pages are silent or disagree (each is listed in the design doc):
+//   * phi = SiLU on q and k only; v is used raw (the workload statement applies SiLU to Q, K).
+//   * No normaliser z and no denominator: [Arch] feeds Y straight into RMSNorm.
+//   * No decay factor and no 1/sqrt(d) scaling (neither appears in the linear form).
+//   * Causal mask inclusive (i <= t); a decode step updates S first, then reads it.
+//   * RMSNorm over the concatenation of all heads of a token (H*D values), eps inside the
+//     square root: r = 1/sqrt(mean(y^2) + eps); then multiply by weight w and sigmoid(g).
+//
+// Every function computes in fp64 from the exact widening of the stored inputs
+// (bf16 bits or fp32).  Layouts: q, k, v [tokens, H, D]; g and out [tokens, H*D];
+// states [seq, H, D(k), D(v)] row-major.
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+#include <algorithm>
+
+namespace {
+
+enum { DT_F32 = 0, DT_BF16 = 1 };
+enum { PHI_SILU = 0, PHI_IDENTITY = 1 };
+enum { MODE_RAW = 0, MODE_RMSNORM = 1, MODE_RMSNORM_GATE = 2 };
+
+inline double widen(const void* base, int dtype, int64_t i) {
+  if (dtype == DT_BF16) {
+    uint32_t u = static_cast<uint32_t>(static_cast<const uint16_t*>(base)[i]) << 16;
+    float f;
+    std::memcpy(&f, &u, 4);
+    return static_cast<double>(f);
+  }
+  return static_cast<double>(static_cast<const float*>(base)[i]);
+}
+
+// [Arch] 2.1: SiLU(x) = x * sigmoid(x) = x / (1 + e^-x).
+inline double silu(double x) { return x / (1.0 + std::exp(-x)); }
+inline double sigmoid(double x) { return 1.0 / (1.0 + std::exp(-x)); }
+inline double feature(double x, int phi) { return phi == PHI_SILU ? silu(x) : x; }
+
+// Token-by-token recurrence for one head over rows [row0, row0 + n) of the packed
+// [tokens, H, D] inputs.  S (D x D, fp64) enters as the state before the first
+// token and leaves as the state after the last.  y receives, for each token, the
+// D values phi(q_t)^T S_t at y[(t * H + h) * D + j]  ([Tut64] section 3).
+void recur_head(const void* q, const void* k, const void* v, int dtype, int64_t row0, int64_t n,
+                int H, int D, int h, int phi, double* S, double* y) {
+  std::vector<double> fq(D), fk(D), vv(D), acc(D);
+  for (int64_t t = 0; t < n; ++t) {
+    const int64_t base = ((row0 + t) * H + h) * static_cast<int64_t>(D);
+    for (int i = 0; i < D; ++i) {
+      fq[i] = feature(widen(q, dtype, base + i), phi);
+      fk[i] = feature(widen(k, dtype, base + i), phi);
+      vv[i] = widen(v, dtype, base + i);
+      acc[i] = 0.0;
+    }
+    // S_t = S_{t-1} + phi(k_t) v_t^T, then y_t = phi(q_t)^T S_t.
+    for (int i = 0; i < D; ++i) {
+      double* Si = S + static_cast<int64_t>(i) * D;
+      const double a = fk[i], b = fq[i];
+      for (int j = 0; j < D; ++j) {
+        Si[j] += a * vv[j];
+        acc[j] += b * Si[j];
+      }
+    }
+    double* yt = y + (t * H + h) * static_cast<int64_t>(D);
+    for (int j = 0; j < D; ++j) yt[j] = acc[j];
+  }
+}
+
+// Output transform of one token ([Arch] 2.1): concatenate the H heads (index h*D + j),
+// then RAW: o = y; RMSNORM: o = y * r * w; RMSNORM_GATE: o = y * r * w * sigmoid(g),
+// with r = 1 / sqrt(mean(y^2) + eps) over the H*D values.
+void transform_token(const double* y, int HD, int mode, double eps, const float* w,
+                     const void* g, int dtype, int64_t grow, double* o) {
+  if (mode == MODE_RAW) {
+    for (int c = 0; c < HD; ++c) o[c] = y[c];
+    return;
+  }
+  double ss = 0.0;
+  for (int c = 0; c < HD; ++c) ss += y[c] * y[c];
+  const double r = 1.0 / std::sqrt(ss / HD + eps);
+  for (int c = 0; c < HD; ++c) {
+    double val = y[c] * r * (w ? static_cast<double>(w[c]) : 1.0);
+    if (mode == MODE_RMSNORM_GATE) val *= sigmoid(widen(g, dtype, grow * HD + c));
+    o[c] = val;
+  }
+}
+
+// Comparison accumulator for the streaming check of a candidate output.
+struct Cmp {
+  double max_ref = 0.0, max_err = 0.0;
+  int64_t argmax = -1, nonfinite = 0;
+};
+
+inline void cmp_update(Cmp& c, double ref, double cand, int64_t idx) {
+  if (!std::isfinite(cand)) { c.nonfinite++; return; }
+  c.max_ref = std::max(c.max_ref, std::fabs(ref));
+  double e = std::fabs(ref - cand);
+  if (e > c.max_err) { c.max_err = e; c.argmax = idx; }
+}
+
+// One packed sequence: rows [row0, row0 + L).  The H recurrences run in parallel
+// over token chunks; each chunk's outputs are transformed and either stored
+// (out != nullptr) or compared against `cand` (a dtype tensor [tokens, H*D]).
+void run_sequence(const void* q, const void* k, const void* v, const void* g, int dtype,
+                  int64_t row0, int64_t L, int H, int D, int phi, int mode, double eps,
+                  const float* w, std::vector<double>& states /* H*D*D, in/out */,
+                  double* out, const void* cand, Cmp* cmp) {
+  const int HD = H * D;
+  const int64_t CH = 256;
+  std::vector<double> y(static_cast<size_t>(CH) * HD);
+  std::vector<double> o(static_cast<size_t>(CH) * HD);
+  for (int64_t c0 = 0; c0 < L; c0 += CH) {
+    const int64_t n = std::min(CH, L - c0);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h)
+      recur_head(q, k, v, dtype, row0 + c0, n, H, D, h, phi,
+                 states.data() + static_cast<size_t>(h) * D * D, y.data());
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < n; ++t) {
+      double* ot = out ? out + (row0 + c0 + t) * HD : o.data() + t * HD;
+      transform_token(y.data() + t * HD, HD, mode, eps, w, g, dtype, row0 + c0 + t, ot);
+    }
+    if (cand) {
+      Cmp local;
+      for (int64_t t = 0; t < n; ++t) {
+        const int64_t grow = row0 + c0 + t;
+        const double* ot = out ? out + grow * HD : o.data() + t * HD;
+        for (int c = 0; c < HD; ++c)
+          cmp_update(local, ot[c], widen(cand, dtype, grow * HD + c), grow * HD + c);
+      }
+      cmp->max_ref = std::max(cmp->max_ref, local.max_ref);
+      cmp->nonfinite += local.nonfinite;
+      if (local.max_err > cmp->max_err) { cmp->max_err = local.max_err; cmp->argmax = local.argmax; }
+    }
+  }
+}
+
+void load_states(std::vector<double>& st, const float* state_in, int64_t seq, int H, int D) {
+  const int64_t n = static_cast<int64_t>(H) * D * D;
+  st.assign(n, 0.0);
+  if (state_in)
+    for (int64_t i = 0; i < n; ++i) st[i] = static_cast<double>(state_in[seq * n + i]);
+}
+
+void finish_states(const std::vector<double>& st, int64_t seq, int H, int D, double* state_out,
+                   const float* cand_state, Cmp* scmp) {
+  const int64_t n = static_cast<int64_t>(H) * D * D;
+  if (state_out)
+    for (int64_t i = 0; i < n; ++i) state_out[seq * n + i] = st[i];
+  if (cand_state && scmp)
+    for (int64_t i = 0; i < n; ++i)
+      cmp_update(*scmp, st[i], static_cast<double>(cand_state[seq * n + i]), seq * n + i);
+}
+
+void write_stats(double* stats, const Cmp& o, const Cmp& s) {
+  if (!stats) return;
+  stats[0] = o.max_ref; stats[1] = o.max_err; stats[2] = static_cast<double>(o.argmax);
+  stats[3] = static_cast<double>(o.nonfinite);
+  stats[4] = s.max_ref; stats[5] = s.max_err; stats[6] = static_cast<double>(s.argmax);
+  stats[7] = static_cast<double>(s.nonfinite);
+}
+
+}  // namespace
+
+extern "C" {
+
+// Packed-sequence forward ([Tut64] section 3 recurrence, [Arch] 2.1 output transform).
+// cu: N + 1 row offsets into the packed tensors (sequence s = rows cu[s] .. cu[s+1]).
+// Each sequence starts from state_in[s] (zeros if state_in is null); its final state
+// goes to state_out[s].  If `out` is non-null the fp64 result [tokens, H*D] is stored.
+// If `cand_out` / `cand_state` are non-null they are compared instead (streaming: no
+// fp64 copy of the output is kept) and stats[0..7] receive
+// {max|o_ref|, max|o_ref - o_cand|, argmax, nonfinite, same four for the state}.
+int oracle_forward_packed(const void* q, const void* k, const void* v, const void* g, int dtype,
+                          const int32_t* cu, int N, int H, int D, const float* state_in, int phi,
+                          int mode, double eps, const float* w, double* out, double* state_out,
+                          const void* cand_out, const float* cand_state, double* stats) {
+  if (N < 0 || H <= 0 || D <= 0) return 1;
+  if (mode == MODE_RMSNORM_GATE && !g) return 1;
+  Cmp ocmp, scmp;
+  std::vector<double> st;
+  for (int s = 0; s < N; ++s) {
+    const int64_t L = static_cast<int64_t>(cu[s + 1]) - cu[s];
+    if (L < 0) return 1;
+    load_states(st, state_in, s, H, D);
+    run_sequence(q, k, v, g, dtype, cu[s], L, H, D, phi, mode, eps, w, st, out, cand_out, &ocmp);
+    finish_states(st, s, H, D, state_out, cand_state, &scmp);
+  }
+  write_stats(stats, ocmp, scmp);
+  return 0;
+}
+
+// Fixed-length batch [B, T, H, D]: the packed form with cu[b] = b * T.
+int oracle_prefill(const void* q, const void* k, const void* v, const void* g, int dtype, int B,
+                   int T, int H, int D, const float* state_in, int phi, int mode, double eps,
+                   const float* w, double* out, double* state_out, const void* cand_out,
+                   const float* cand_state, double* stats) {
+  if (B < 0 || T < 0) return 1;
+  std::vector<int32_t> cu(B + 1);
+  for (int b = 0; b <= B; ++b) cu[b] = b * T;
+  return oracle_forward_packed(q, k, v, g, dtype, cu.data(), B, H, D, state_in, phi, mode, eps, w,
+                               out, state_out, cand_out, cand_state, stats);
+}
+
+// One decode step for B sequences: q, k, v [B, H, D], g [B, H*D], state [B, H, D, D] fp32.
+// [Tut64] section 3: each new token only updates the state, S <- S + phi(k) v^T, and is
+// read from it, y = phi(q)^T S; then the [Arch] 2.1 output transform.
+int oracle_decode(const void* q, const void* k, const void* v, const void* g, int dtype, int B, int H,
+                  int D, const float* state_in, int phi, int mode, double eps, const float* w,
+                  double* out, double* state_out, const void* cand_out, const float* cand_state,
+                  double* stats) {
+  return oracle_prefill(q, k, v, g, dtype, B, 1, H, D, state_in, phi, mode, eps, w, out, state_out,
+                        cand_out, cand_state, stats);
+}
+
+// Independent restatement R1 ([Tut64] section 3, the sum form before it is folded into
+// a state): y_t = sum_{i <= t} (phi(q_t) . phi(k_i)) v_i, i.e. Y = (phi(Q) phi(K)^T (.) M) V
+// with M_ti = [i <= t].  O(T^2 D) per head; tiny inputs only.  One sequence [T, H, D];
+// y receives the raw (untransformed) [T, H, D] result.
+int oracle_quadratic(const void* q, const void* k, const void* v, int dtype, int T, int H, int D,
+                     int phi, double* y) {
+  if (T < 0 || H <= 0 || D <= 0) return 1;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int h = 0; h < H; ++h) {
+    std::vector<double> fq(static_cast<size_t>(T) * D), fk(static_cast<size_t>(T) * D),
+        vv(static_cast<size_t>(T) * D);
+    for (int t = 0; t < T; ++t)
+      for (int i = 0; i < D; ++i) {
+        const int64_t idx = (static_cast<int64_t>(t) * H + h) * D + i;
+        fq[static_cast<size_t>(t) * D + i] = feature(widen(q, dtype, idx), phi);
+        fk[static_cast<size_t>(t) * D + i] = feature(widen(k, dtype, idx), phi);
+        vv[static_cast<size_t>(t) * D + i] = widen(v, dtype, idx);
+      }
+    for (int t = 0; t < T; ++t) {
+      double* yt = y + (static_cast<int64_t>(t) * H + h) * D;
+      for (int j = 0; j < D; ++j) yt[j] = 0.0;
+      for (int i = 0; i <= t; ++i) {
+        double p = 0.0;
+        for (int c = 0; c < D; ++c) p += fq[static_cast<size_t>(t) * D + c] * fk[static_cast<size_t>(i) * D + c];
+        for (int j = 0; j < D; ++j) yt[j] += p * vv[static_cast<size_t>(i) * D + j];
+      }
+    }
+  }
+  return 0;
+}
+
+// Independent restatement R2: the block-wise form with block size C (any C >= 1).
+// For each block of C tokens (the last one may be shorter):
+//   intra:  y_t = sum_{i in block, i <= t} (phi(q_t) . phi(k_i)) v_i
+//   inter:  y_t += phi(q_t)^T S_prev            (S_prev = state before the block)
+//   carry:  S_prev += sum_{i in block} phi(k_i) v_i^T
+// [Ops] section 3 fixes the block size the deployment uses (256).  One sequence
+// [T, H, D] starting from s0 [H, D, D] (zeros if null); y receives the raw result and
+// state_out [H, D, D] the final state.
+int oracle_chunked(const void* q, const void* k, const void* v, int dtype, int T, int H, int D, int C,
+                   int phi, const double* s0, double* y, double* state_out) {
+  if (T < 0 || H <= 0 || D <= 0 || C < 1) return 1;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int h = 0; h < H; ++h) {
+    std::vector<double> S(static_cast<size_t>(D) * D, 0.0);
+    if (s0)
+      for (int i = 0; i < D * D; ++i) S[i] = s0[static_cast<size_t>(h) * D * D + i];
+    std::vector<double> fq(static_cast<size_t>(C) * D), fk(static_cast<size_t>(C) * D),
+        vv(static_cast<size_t>(C) * D);
+    for (int b0 = 0; b0 < T; b0 += C) {
+      const int n = std::min(C, T - b0);
+      for (int t = 0; t < n; ++t)
+        for (int i = 0; i < D; ++i) {
+          const int64_t idx = (static_cast<int64_t>(b0 + t) * H + h) * D + i;
+          fq[static_cast<size_t>(t) * D + i] = feature(widen(q, dtype, idx), phi);
+          fk[static_cast<size_t>(t) * D + i] = feature(widen(k, dtype, idx), phi);
+          vv[static_cast<size_t>(t) * D + i] = widen(v, dtype, idx);
+        }
+      for (int t = 0; t < n; ++t) {
+        double* yt = y + (static_cast<int64_t>(b0 + t) * H + h) * D;
+        for (int j = 0; j < D; ++j) {
+          double inter = 0.0;
+          for (int i = 0; i < D; ++i) inter += fq[static_cast<size_t>(t) * D + i] * S[static_cast<size_t>(i) * D + j];
+          yt[j] = inter;
+        }
+        for (int i = 0; i <= t; ++i) {
+          double p = 0.0;
+          for (int c = 0; c < D; ++c) p += fq[static_cast<size_t>(t) * D + c] * fk[static_cast<size_t>(i) * D + c];
+          for (int j = 0; j < D; ++j) yt[j] += p * vv[static_cast<size_t>(i) * D + j];
+        }
+      }
+      for (int t = 0; t < n; ++t)
+        for (int i = 0; i < D; ++i) {
+          const double a = fk[static_cast<size_t>(t) * D + i];
+          for (int j = 0; j < D; ++j) S[static_cast<size_t>(i) * D + j] += a * vv[static_cast<size_t>(t) * D + j];
+        }
+    }
+    if (state_out)
+      for (int i = 0; i < D * D; ++i) state_out[static_cast<size_t>(h) * D * D + i] = S[i];
+  }
+  return 0;
+}
+
+// The output transform alone ([Arch] 2.1), for tests of the norm and gate on given y.
+int oracle_transform(const double* y, int64_t tokens, int H, int D, int mode, double eps,
+                     const float* w, const void* g, int dtype, double* out) {
+  const int HD = H * D;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < tokens; ++t) transform_token(y + t * HD, HD, mode, eps, w, g, dtype, t, out + t * HD);
+  return 0;
+}
+
+}  // extern "C"
