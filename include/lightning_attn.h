@@ -1,0 +1,176 @@
+/*
+ * lightning_attn.h -- C ABI of the Lightning Attention forward on B200 (sm_100a).
+ *
+ * What the library computes (sources are web pages, cited by title and section):
+ *
+ *   "六十四：MiniMax-01" (LLM tutorial, lesson 64), section 3 "Lightning Attention 的定位":
+ *     linear attention keeps a running state per head,
+ *         S_t = S_{t-1} + phi(k_t) v_t^T,        y_t = phi(q_t)^T S_t,
+ *     (the sum runs over i <= t: causal, diagonal included), and a decode step only
+ *     updates the state and reads it.
+ *   "MiniMax-Text-01 405B MoE模型架构与训练策略解析", section 2.1 "Lightning Attention-2":
+ *     phi = SiLU, Y = Q (K^T V), output = RMSNorm(Y) * sigmoid(gate).
+ *   "MiniMax-01技术报告解读（二）计算优化", section 3: the block (chunk) size is 256 and the
+ *     tail block is padded to one of 32 / 64 / 128 rows; section 6: prefill and decode run
+ *     as separate paths on separate CUDA streams.
+ *
+ * Readings where the pages are silent: phi is applied to q and k only (v raw); there is
+ * no normaliser denominator, no decay and no 1/sqrt(d) scale; the RMSNorm runs over the
+ * concatenation of the H heads of a token (H*D values) with eps inside the square root,
+ *     o = y * rsqrt(mean(y^2) + eps) * w * sigmoid(g).
+ * The block size changes rounding and work, not the exact result.
+ *
+ * Tensor layouts (all row-major, contiguous, device memory unless stated):
+ *   q, k, v   [B, T, H, D] (prefill), [total_tokens, H, D] (varlen), [B, H, D] (decode)
+ *   g, out    [B, T, H*D],            [total_tokens, H*D],             [B, H*D]
+ *   states    fp32 [B or N, H, D, D]: state[s][h][i][j] multiplies phi(q)[i] to give y[j]
+ * q, k, v, g and out share one element type (la_dtype); states are always fp32.
+ * All device pointers must be 16-byte aligned.
+ *
+ * Calls are asynchronous on `stream`.  Arguments are validated on the host before any
+ * launch; a rejected call launches nothing and returns its status.  Failures detected
+ * on the device (a bounded wait that ran out, decreasing cu_seqlens) are recorded in
+ * the workspace and reported by lightning_attn_check().  Ownership: the caller owns
+ * every buffer, including the workspace; the library allocates nothing and keeps no
+ * per-call state, so calls on different streams with different workspaces are
+ * independent.  Calls that share a workspace must be ordered on one stream.
+ */
+#ifndef LIGHTNING_ATTN_H_
+#define LIGHTNING_ATTN_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (the same type as cudaStream_t / CUstream). NULL = legacy stream. */
+typedef struct CUstream_st* la_stream_t;
+
+typedef enum {
+  LA_OK = 0,
+  LA_ERR_INVALID_ARG = 1,  /* a pointer, size, alignment or enum value is invalid          */
+  LA_ERR_UNSUPPORTED = 2,  /* valid, but no kernel of this build handles the combination   */
+  LA_ERR_CUDA = 3,         /* a CUDA runtime/driver call or a kernel launch failed         */
+  LA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out (reported by _check)      */
+  LA_ERR_DEVICE = 5        /* a device-side argument check failed (reported by _check)     */
+} la_status;
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+
+/* RAW: out = y.  RMSNORM: out = y * r * w.  RMSNORM_GATE: out = y * r * w * sigmoid(g). */
+typedef enum { LA_OUT_RAW = 0, LA_OUT_RMSNORM = 1, LA_OUT_RMSNORM_GATE = 2 } la_out_mode;
+
+/* SILU: phi(x) = x * sigmoid(x) on q and k.  IDENTITY: phi(x) = x (exact-integer tests). */
+typedef enum { LA_PHI_SILU = 0, LA_PHI_IDENTITY = 1 } la_feature_map;
+
+typedef enum { LA_OP_PREFILL = 0, LA_OP_PREFILL_VARLEN = 1, LA_OP_DECODE = 2 } la_op;
+
+/*
+ * Causal block-wise prefill of B sequences of T tokens each.
+ * Source: "六十四：MiniMax-01" section 3 (recurrence), "MiniMax-Text-01 405B MoE模型架构与训练
+ * 策略解析" section 2.1 (SiLU, RMSNorm * sigmoid gate), "MiniMax-01技术报告解读（二）计算优化"
+ * section 3 (block size 256, tail pads 32/64/128).
+ *
+ *   q, k, v      [B, T, H, D], dtype; read only.
+ *   g            [B, T, H*D], dtype; required iff mode == LA_OUT_RMSNORM_GATE, else ignored.
+ *   out          [B, T, H*D], dtype; written.  May not alias any input.
+ *   state_in     fp32 [B, H, D, D] initial state per sequence, or NULL for zeros.
+ *   state_out    fp32 [B, H, D, D] final state, or NULL.  May equal state_in (in place).
+ *   B, T         B >= 1, T >= 0 (T == 0: no output; state_out = state_in or zeros).
+ *   H, D         H >= 1; D in {64, 128}.  The RMSNorm modes need H*D <= 16384.
+ *   block_size   the block (chunk) size C, 1..1024.  bf16 with D = 128 and C in {128, 256} runs
+ *                on the tcgen05 tensor-core kernel; every other valid combination runs on the
+ *                CUDA-core kernel (fp32 arithmetic).  lightning_attn_last_path() names the one used.
+ *   eps          RMSNorm epsilon (> 0 for the norm modes).
+ *   norm_weight  fp32 [H*D] RMSNorm weight, or NULL for ones.
+ *   workspace    device scratch of >= lightning_attn_workspace_size(LA_OP_PREFILL, ...)
+ *                bytes, 256-byte aligned.  Its first 256 bytes hold the error record
+ *                (words 0-3: status, site, index, detail -- read and cleared by
+ *                lightning_attn_check; word 4: bounded-wait limit in ms, 0 = default 4 s;
+ *                word 5: fault-injection selector for failure tests, 0 = none).  The call
+ *                clears the rest of the workspace itself.
+ * Returns LA_OK after enqueueing, or an error status with nothing enqueued.
+ */
+LA_API la_status lightning_attn_prefill(const void* q, const void* k, const void* v, const void* g, void* out,
+                                 const float* state_in, float* state_out, int B, int T, int H, int D,
+                                 int block_size, la_dtype dtype, la_feature_map phi, la_out_mode mode,
+                                 float eps, const float* norm_weight, void* workspace,
+                                 size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * Prefill of N variable-length sequences packed along the token axis.
+ * Source: as lightning_attn_prefill; packing with cu_seqlens follows the varlen
+ * treatment of "MiniMax-01系列大模型：超长上下文与多模态能力深度解析与部署指南" section 2.1.3.
+ *
+ *   q, k, v      [total_tokens, H, D]; g, out [total_tokens, H*D].
+ *   cu_seqlens   DEVICE int32 [N + 1], cu_seqlens[0] == 0, non-decreasing,
+ *                cu_seqlens[N] == total_tokens.  Sequence s is rows cu[s] .. cu[s+1]-1.
+ *                Violations found on the device are reported by lightning_attn_check.
+ *   state_in / state_out  fp32 [N, H, D, D] or NULL.  Each sequence starts from its own
+ *                state (zeros if NULL) -- states never flow between sequences.
+ *   max_seqlen   an upper bound on every sequence length (sizes the workspace).
+ *   Tail blocks are padded to the smallest of 32 / 64 / 128 that fits.
+ * Other arguments as lightning_attn_prefill.
+ */
+LA_API la_status lightning_attn_prefill_varlen(const void* q, const void* k, const void* v, const void* g,
+                                        void* out, const float* state_in, float* state_out,
+                                        const int* cu_seqlens, int num_seqs, int max_seqlen,
+                                        int total_tokens, int H, int D, int block_size,
+                                        la_dtype dtype, la_feature_map phi, la_out_mode mode,
+                                        float eps, const float* norm_weight, void* workspace,
+                                        size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * One decode step for B sequences, one new token each.
+ * Source: "六十四：MiniMax-01" section 3 (each new token only updates the state and is
+ * read from it: S <- S + phi(k) v^T, y = phi(q)^T S -- update first, then read), and
+ * "MiniMax-Text-01 405B MoE模型架构与训练策略解析" section 2.1 (output transform).
+ *
+ *   q, k, v      [B, H, D]; g, out [B, H*D].
+ *   state        fp32 [B, H, D, D], updated IN PLACE.
+ *   workspace    >= lightning_attn_workspace_size(LA_OP_DECODE, ...) bytes, 256-byte aligned,
+ *                zero-filled before its first use; every completed call leaves it zeroed.
+ * Other arguments as lightning_attn_prefill.
+ */
+LA_API la_status lightning_attn_decode_step(const void* q, const void* k, const void* v, const void* g,
+                                     void* out, float* state, int B, int H, int D, la_dtype dtype,
+                                     la_feature_map phi, la_out_mode mode, float eps,
+                                     const float* norm_weight, void* workspace, size_t workspace_bytes,
+                                     la_stream_t stream);
+
+/*
+ * Workspace bytes needed by one call (0 on invalid arguments).
+ *   op == LA_OP_PREFILL:         B_or_N = B, T_or_max = T, total_tokens ignored.
+ *   op == LA_OP_PREFILL_VARLEN:  B_or_N = N, T_or_max = max_seqlen, total_tokens.
+ *   op == LA_OP_DECODE:          B_or_N = B, the rest ignored except H, D, dtype, mode.
+ * The size depends on the kernel the call will select (which depends on the device), so
+ * query it with the target device current.
+ */
+LA_API size_t lightning_attn_workspace_size(la_op op, int B_or_N, int T_or_max, int total_tokens, int H, int D,
+                                     int block_size, la_dtype dtype, la_out_mode mode);
+
+/*
+ * Synchronises `stream`, then reads and clears the error record in `workspace`.
+ * Returns LA_OK, LA_ERR_TIMEOUT, LA_ERR_DEVICE, or LA_ERR_CUDA (stream error).
+ * `detail` (may be NULL) receives 4 words: {status, site, index, extra}.
+ */
+LA_API la_status lightning_attn_check(void* workspace, la_stream_t stream, unsigned int* detail);
+
+/* Static, human-readable name of a status. */
+LA_API const char* lightning_attn_status_string(la_status s);
+
+/* Name of the kernel path the last successful call on this thread selected (diagnostic). */
+LA_API const char* lightning_attn_last_path(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIGHTNING_ATTN_H_ */

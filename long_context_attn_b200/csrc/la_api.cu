@@ -1,0 +1,209 @@
+// C ABI of the Lightning Attention library: argument validation, kernel selection,
+// workspace carving and the device error record.  Every compute step runs in the
+// kernels of la_decode.cu, la_simt.cu and la_prefill_tc.cu; there is no CPU path.
+#include <cstdint>
+#include <cstring>
+
+#include "la_common.cuh"
+#include "la_prefill_tc.h"
+
+namespace la {
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, void* out, float* state,
+                          int B, int H, int D, la_dtype dt, int phi_identity, int mode, float eps,
+                          const float* w, void* workspace, cudaStream_t stream);
+size_t decode_workspace_bytes(int B, int H, int D);
+cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, void* out, float* y_ws,
+                                const float* state_in, float* state_out, const int* cu, int nseq, int T,
+                                int H, int D, int C, la_dtype dt, int phi_identity, int64_t total_rows,
+                                ErrRec* err, cudaStream_t stream);
+cudaError_t launch_norm_gate(const float* y, const void* g, void* out, int64_t tokens, int HD, int mode,
+                             float eps, const float* w, la_dtype dt, cudaStream_t stream);
+}  // namespace la
+
+namespace {
+
+thread_local const char* g_last_path = "none";
+
+constexpr size_t kErrBytes = sizeof(la::ErrRec);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool valid_enums(la_dtype dt, la_feature_map phi, la_out_mode mode) {
+  return (dt == LA_F32 || dt == LA_BF16) && (phi == LA_PHI_SILU || phi == LA_PHI_IDENTITY) &&
+         (mode == LA_OUT_RAW || mode == LA_OUT_RMSNORM || mode == LA_OUT_RMSNORM_GATE);
+}
+
+bool valid_head(int H, int D, la_out_mode mode, float eps) {
+  if (H < 1 || (D != 64 && D != 128)) return false;
+  if (mode != LA_OUT_RAW && (static_cast<int64_t>(H) * D > la::kMaxNormWidth || !(eps > 0.0f))) return false;
+  return true;
+}
+
+int current_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+bool device_is_sm100() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
+  return major == 10 && minor == 0;
+}
+
+// Which prefill kernel a call takes.
+enum class Path { kTc, kSimt };
+
+Path choose_path(la_dtype dt, int H, int D, int C, la_out_mode mode) {
+  la::TcShape s{H, D, C, dt == LA_BF16, static_cast<int>(mode)};
+  if (device_is_sm100() && la::tc_eligible(s, current_sm_count())) return Path::kTc;
+  return Path::kSimt;
+}
+
+size_t prefill_ws_bytes(Path p, int nseq, int max_len, int64_t tokens, int H, int D, int C, la_out_mode mode) {
+  if (p == Path::kTc) return kErrBytes + la::tc_workspace_bytes(nseq, max_len, tokens, H, D, C);
+  size_t y = (mode == LA_OUT_RAW) ? 0 : up256(sizeof(float) * static_cast<size_t>(tokens) * H * D);
+  return kErrBytes + y;
+}
+
+la_status common_prefill(const void* q, const void* k, const void* v, const void* g, void* out,
+                         const float* state_in, float* state_out, const int* cu, int nseq, int T_fixed,
+                         int max_len, int64_t tokens, int H, int D, int C, la_dtype dt, la_feature_map phi,
+                         la_out_mode mode, float eps, const float* w, void* workspace, size_t ws_bytes,
+                         cudaStream_t stream) {
+  if (!valid_enums(dt, phi, mode) || !valid_head(H, D, mode, eps)) return LA_ERR_INVALID_ARG;
+  if (C < 1 || C > 1024 || nseq < 1 || tokens < 0 || max_len < 0) return LA_ERR_INVALID_ARG;
+  if (tokens > 0) {
+    if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_INVALID_ARG;
+    if (mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g))) return LA_ERR_INVALID_ARG;
+  }
+  if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)) ||
+      (w && !aligned16(w)))
+    return LA_ERR_INVALID_ARG;
+  if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;
+
+  const Path path = choose_path(dt, H, D, C, mode);
+  if (ws_bytes < prefill_ws_bytes(path, nseq, max_len, tokens, H, D, C, mode)) return LA_ERR_INVALID_ARG;
+  la::ErrRec* err = static_cast<la::ErrRec*>(workspace);
+  char* ws = static_cast<char*>(workspace) + kErrBytes;
+  const int phi_id = (phi == LA_PHI_IDENTITY) ? 1 : 0;
+  cudaError_t e;
+  if (path == Path::kTc) {
+    la::TcArgs a{};
+    a.q = q; a.k = k; a.v = v; a.g = g; a.out = out;
+    a.state_in = state_in; a.state_out = state_out; a.cu = cu;
+    a.nseq = nseq; a.T = T_fixed; a.max_len = max_len; a.tokens = tokens;
+    a.H = H; a.D = D; a.C = C; a.phi_identity = phi_id; a.mode = static_cast<int>(mode);
+    a.eps = eps; a.w = w; a.err = err; a.ws = ws;
+    e = la::launch_tc_prefill(a, current_sm_count(), stream);
+    g_last_path = "tcgen05";
+  } else {
+    float* y_ws = (mode == LA_OUT_RAW) ? nullptr : reinterpret_cast<float*>(ws);
+    e = la::launch_simt_prefill(q, k, v, out, y_ws, state_in, state_out, cu, nseq, T_fixed, H, D, C, dt, phi_id,
+                                tokens, err, stream);
+    if (e == cudaSuccess && y_ws)
+      e = la::launch_norm_gate(y_ws, g, out, tokens, H * D, static_cast<int>(mode), eps, w, dt, stream);
+    g_last_path = "simt";
+  }
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+la_status lightning_attn_prefill(const void* q, const void* k, const void* v, const void* g, void* out,
+                                 const float* state_in, float* state_out, int B, int T, int H, int D,
+                                 int block_size, la_dtype dtype, la_feature_map phi, la_out_mode mode,
+                                 float eps, const float* norm_weight, void* workspace, size_t workspace_bytes,
+                                 la_stream_t stream) {
+  if (B < 1 || T < 0) return LA_ERR_INVALID_ARG;
+  const int64_t tokens = static_cast<int64_t>(B) * T;
+  if (tokens > INT32_MAX) return LA_ERR_UNSUPPORTED;
+  return common_prefill(q, k, v, g, out, state_in, state_out, nullptr, B, T, T, tokens, H, D, block_size, dtype,
+                        phi, mode, eps, norm_weight, workspace, workspace_bytes,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status lightning_attn_prefill_varlen(const void* q, const void* k, const void* v, const void* g, void* out,
+                                        const float* state_in, float* state_out, const int* cu_seqlens,
+                                        int num_seqs, int max_seqlen, int total_tokens, int H, int D,
+                                        int block_size, la_dtype dtype, la_feature_map phi, la_out_mode mode,
+                                        float eps, const float* norm_weight, void* workspace,
+                                        size_t workspace_bytes, la_stream_t stream) {
+  if (num_seqs < 1 || !cu_seqlens || !aligned16(cu_seqlens) || total_tokens < 0 || max_seqlen < 0)
+    return LA_ERR_INVALID_ARG;
+  return common_prefill(q, k, v, g, out, state_in, state_out, cu_seqlens, num_seqs, 0, max_seqlen, total_tokens,
+                        H, D, block_size, dtype, phi, mode, eps, norm_weight, workspace, workspace_bytes,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status lightning_attn_decode_step(const void* q, const void* k, const void* v, const void* g, void* out,
+                                     float* state, int B, int H, int D, la_dtype dtype, la_feature_map phi,
+                                     la_out_mode mode, float eps, const float* norm_weight, void* workspace,
+                                     size_t workspace_bytes, la_stream_t stream) {
+  if (!valid_enums(dtype, phi, mode) || !valid_head(H, D, mode, eps) || B < 1) return LA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * H > INT32_MAX / 2) return LA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !out || !state) return LA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state))
+    return LA_ERR_INVALID_ARG;
+  if (mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g))) return LA_ERR_INVALID_ARG;
+  if (norm_weight && !aligned16(norm_weight)) return LA_ERR_INVALID_ARG;
+  if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;
+  if (workspace_bytes < la::decode_workspace_bytes(B, H, D)) return LA_ERR_INVALID_ARG;
+  cudaError_t e = la::launch_decode(q, k, v, g, out, state, B, H, D, dtype, phi == LA_PHI_IDENTITY ? 1 : 0,
+                                    static_cast<int>(mode), eps, norm_weight, workspace,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  g_last_path = "decode";
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+size_t lightning_attn_workspace_size(la_op op, int B_or_N, int T_or_max, int total_tokens, int H, int D,
+                                     int block_size, la_dtype dtype, la_out_mode mode) {
+  if (B_or_N < 1 || T_or_max < 0 || H < 1 || (D != 64 && D != 128)) return 0;
+  if (op == LA_OP_DECODE) return la::decode_workspace_bytes(B_or_N, H, D);
+  if (block_size < 1 || block_size > 1024) return 0;
+  const Path path = choose_path(dtype, H, D, block_size, mode);
+  if (op == LA_OP_PREFILL)
+    return prefill_ws_bytes(path, B_or_N, T_or_max, static_cast<int64_t>(B_or_N) * T_or_max, H, D, block_size,
+                            mode);
+  if (op == LA_OP_PREFILL_VARLEN) {
+    if (total_tokens < 0) return 0;
+    return prefill_ws_bytes(path, B_or_N, T_or_max, total_tokens, H, D, block_size, mode);
+  }
+  return 0;
+}
+
+la_status lightning_attn_check(void* workspace, la_stream_t stream, unsigned int* detail) {
+  if (!workspace) return LA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LA_ERR_CUDA;
+  unsigned int rec[4] = {0, 0, 0, 0};
+  if (cudaMemcpy(rec, workspace, sizeof(rec), cudaMemcpyDeviceToHost) != cudaSuccess) return LA_ERR_CUDA;
+  if (detail) std::memcpy(detail, rec, sizeof(rec));
+  if (rec[0] == 0) return LA_OK;
+  if (cudaMemset(workspace, 0, sizeof(rec)) != cudaSuccess) return LA_ERR_CUDA;
+  return static_cast<la_status>(rec[0]);
+}
+
+const char* lightning_attn_status_string(la_status s) {
+  switch (s) {
+    case LA_OK: return "LA_OK";
+    case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG";
+    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED";
+    case LA_ERR_CUDA: return "LA_ERR_CUDA";
+    case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT";
+    case LA_ERR_DEVICE: return "LA_ERR_DEVICE";
+  }
+  return "LA_ERR_UNKNOWN";
+}
+
+const char* lightning_attn_last_path(void) { return g_last_path; }
+
+}  // extern "C"

@@ -1,0 +1,169 @@
+// Single-token decode step of Lightning Attention (sm_100a).
+//
+// "六十四：MiniMax-01", section 3: a new token only updates the running state and reads
+// it -- S <- S + phi(k) v^T, y = phi(q)^T S (update first, so the token sees itself).
+// "MiniMax-Text-01 405B MoE模型架构与训练策略解析", section 2.1: o = RMSNorm(y) * sigmoid(g),
+// the norm taken over the concatenation of all heads of the sequence.
+//
+// The step is bound by HBM: per (sequence, head) the D x D fp32 state is read and written
+// once (128 KiB at D = 128) against ~1 KiB of token data.  One CTA owns one (b, h) state;
+// each warp streams whole 512-byte rows with 128-bit accesses, every thread keeps all
+// of its rows in flight at once, and the update and the read happen in the same pass.
+// The cross-head norm needs all H heads of a sequence: each CTA publishes its y and its
+// sum of squares, and the last CTA of the sequence to arrive (a counter per sequence)
+// normalises the whole H*D row.  Nobody waits, so no co-residency is needed, and the
+// counter is reset by that last CTA, which leaves the workspace zeroed.
+#include "la_common.cuh"
+
+namespace la {
+
+struct DecodeWs {
+  int* count;      // [B] arrivals per sequence (zero between calls)
+  float* y;        // [B, H, D] raw outputs
+  float* part;     // [B, H] per-head sums of squares
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                   const T* __restrict__ g, T* __restrict__ out, float* __restrict__ state, int B,
+                   int H, int phi_identity, int mode, float eps, const float* __restrict__ norm_w,
+                   DecodeWs ws) {
+  constexpr int kThreads = 256;
+  constexpr int kVecPerRow = D / 4;                  // float4 per state row
+  constexpr int kRowsPerPass = kThreads / kVecPerRow;
+  constexpr int kPasses = D / kRowsPerPass;          // rows each thread owns
+  static_assert(kThreads % kVecPerRow == 0 && D % kRowsPerPass == 0, "tiling");
+
+  __shared__ float s_fq[D], s_fk[D], s_v[D];
+  __shared__ float s_red[kRowsPerPass][D];
+  __shared__ float s_ss[kThreads / 32];
+  __shared__ int s_last;
+
+  const int bh = blockIdx.x;            // b * H + h
+  const int b = bh / H;
+  const int tid = threadIdx.x;
+  const int64_t tok = static_cast<int64_t>(bh) * D;
+
+  for (int i = tid; i < D; i += kThreads) {
+    const float xq = load_elem<T>(q, tok + i), xk = load_elem<T>(k, tok + i);
+    s_fq[i] = phi_identity ? xq : silu_accurate(xq);
+    s_fk[i] = phi_identity ? xk : silu_accurate(xk);
+    s_v[i] = load_elem<T>(v, tok + i);
+  }
+
+  // Issue every state load of this thread before the first use.
+  const int c4 = tid % kVecPerRow;
+  const int r0 = tid / kVecPerRow;
+  float4* S = reinterpret_cast<float4*>(state + static_cast<int64_t>(bh) * D * D);
+  float4 s[kPasses];
+#pragma unroll
+  for (int p = 0; p < kPasses; ++p) s[p] = __ldcs(&S[(r0 + p * kRowsPerPass) * kVecPerRow + c4]);
+  __syncthreads();
+
+  const float4 vv = make_float4(s_v[4 * c4], s_v[4 * c4 + 1], s_v[4 * c4 + 2], s_v[4 * c4 + 3]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int p = 0; p < kPasses; ++p) {
+    const int row = r0 + p * kRowsPerPass;
+    const float a = s_fk[row], c = s_fq[row];
+    s[p].x = fmaf(a, vv.x, s[p].x); s[p].y = fmaf(a, vv.y, s[p].y);
+    s[p].z = fmaf(a, vv.z, s[p].z); s[p].w = fmaf(a, vv.w, s[p].w);
+    acc.x = fmaf(c, s[p].x, acc.x); acc.y = fmaf(c, s[p].y, acc.y);
+    acc.z = fmaf(c, s[p].z, acc.z); acc.w = fmaf(c, s[p].w, acc.w);
+    __stcs(&S[row * kVecPerRow + c4], s[p]);
+  }
+  s_red[r0][4 * c4 + 0] = acc.x; s_red[r0][4 * c4 + 1] = acc.y;
+  s_red[r0][4 * c4 + 2] = acc.z; s_red[r0][4 * c4 + 3] = acc.w;
+  __syncthreads();
+
+  // y[j] = sum over the row groups, in a fixed order.
+  float y = 0.f;
+  if (tid < D) {
+#pragma unroll
+    for (int r = 0; r < kRowsPerPass; ++r) y += s_red[r][tid];
+  }
+  const int HD = H * D;
+  if (mode == LA_OUT_RAW) {
+    if (tid < D) store_elem<T>(out, static_cast<int64_t>(b) * HD + (bh % H) * D + tid, y);
+    return;
+  }
+
+  // Publish y and this head's sum of squares (fixed-order reduction).
+  float sq = (tid < D) ? y * y : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  if ((tid & 31) == 0) s_ss[tid >> 5] = sq;
+  if (tid < D) ws.y[tok + tid] = y;
+  __syncthreads();
+  if (tid == 0) {
+    float t = 0.f;
+    for (int w = 0; w < kThreads / 32; ++w) t += s_ss[w];
+    ws.part[bh] = t;
+    __threadfence();
+    const int prev = atomicAdd(&ws.count[b], 1);
+    s_last = (prev == H - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+
+  // Last arriver of sequence b: normalise the whole H*D row.
+  __threadfence();
+  if (tid == 0) {
+    float t = 0.f;
+    for (int h = 0; h < H; ++h) t += __ldcg(&ws.part[b * H + h]);
+    s_ss[0] = 1.0f / sqrtf(t / static_cast<float>(HD) + eps);
+    ws.count[b] = 0;  // leave the workspace zeroed for the next call
+  }
+  __syncthreads();
+  const float r = s_ss[0];
+  const int64_t row = static_cast<int64_t>(b) * HD;
+  for (int c = tid; c < HD; c += kThreads) {
+    float o = __ldcg(&ws.y[row + c]) * r;
+    if (norm_w) o *= norm_w[c];
+    if (mode == LA_OUT_RMSNORM_GATE) o *= sigmoid_accurate(load_elem<T>(g, row + c));
+    store_elem<T>(out, row + c, o);
+  }
+}
+
+size_t decode_workspace_bytes(int B, int H, int D) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  return 256 + up(sizeof(int) * size_t(B)) + up(sizeof(float) * size_t(B) * H * D) +
+         up(sizeof(float) * size_t(B) * H);
+}
+
+static DecodeWs carve_decode_ws(void* workspace, int B, int H, int D) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  char* p = static_cast<char*>(workspace) + 256;
+  DecodeWs ws;
+  ws.count = reinterpret_cast<int*>(p);
+  p += up(sizeof(int) * size_t(B));
+  ws.y = reinterpret_cast<float*>(p);
+  p += up(sizeof(float) * size_t(B) * H * D);
+  ws.part = reinterpret_cast<float*>(p);
+  return ws;
+}
+
+template <typename T, int D>
+static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* g, void* out,
+                                   float* state, int B, int H, int phi_identity, int mode, float eps,
+                                   const float* w, void* workspace, cudaStream_t stream) {
+  DecodeWs ws = carve_decode_ws(workspace, B, H, D);
+  decode_step_kernel<T, D><<<B * H, 256, 0, stream>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+      static_cast<const T*>(g), static_cast<T*>(out), state, B, H, phi_identity, mode, eps, w, ws);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, void* out, float* state,
+                          int B, int H, int D, la_dtype dt, int phi_identity, int mode, float eps,
+                          const float* w, void* workspace, cudaStream_t stream) {
+  if (dt == LA_BF16) {
+    if (D == 128) return launch_decode_t<uint16_t, 128>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace, stream);
+    return launch_decode_t<uint16_t, 64>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace, stream);
+  }
+  if (D == 128) return launch_decode_t<float, 128>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace, stream);
+  return launch_decode_t<float, 64>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace, stream);
+}
+
+}  // namespace la

@@ -1,0 +1,38 @@
+// Host interface of the tcgen05 (5th-generation tensor core) prefill kernel.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "la_common.cuh"
+
+namespace la {
+
+struct TcShape {
+  int H, D, C;
+  bool bf16;
+  int mode;
+};
+
+struct TcArgs {
+  const void *q, *k, *v, *g;
+  void* out;
+  const float* state_in;
+  float* state_out;
+  const int* cu;       // device cu_seqlens (varlen) or nullptr (fixed length T)
+  int nseq, T, max_len;
+  int64_t tokens;
+  int H, D, C, phi_identity, mode;
+  float eps;
+  const float* w;
+  ErrRec* err;
+  char* ws;            // workspace after the error record
+};
+
+// True when the tensor-core kernel handles this shape on a GPU with `num_sms` SMs.
+bool tc_eligible(const TcShape& s, int num_sms);
+// Workspace bytes after the 256-byte error record.
+size_t tc_workspace_bytes(int nseq, int max_len, int64_t tokens, int H, int D, int C);
+cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream);
+
+}  // namespace la

@@ -1,0 +1,179 @@
+"""Thin ctypes binding of liblightning_attn.so (argument marshalling only).
+
+The functions carry the names of the C ABI in include/lightning_attn.h.  They take
+torch tensors (device memory and streams come from PyTorch), pass raw pointers and
+sizes to the library, and raise LightningAttnError on a non-OK status.  Every step of
+the computation runs in the library's CUDA kernels; there is no Python or CPU path, and
+a missing library raises at import.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblightning_attn.so")
+
+LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT, LA_ERR_DEVICE = range(6)
+LA_F32, LA_BF16 = 0, 1
+LA_OUT_RAW, LA_OUT_RMSNORM, LA_OUT_RMSNORM_GATE = 0, 1, 2
+LA_PHI_SILU, LA_PHI_IDENTITY = 0, 1
+LA_OP_PREFILL, LA_OP_PREFILL_VARLEN, LA_OP_DECODE = 0, 1, 2
+
+# The symbols include/lightning_attn.h declares (checked by tests/test_abi.py).
+EXPORTED = (
+    "lightning_attn_prefill",
+    "lightning_attn_prefill_varlen",
+    "lightning_attn_decode_step",
+    "lightning_attn_workspace_size",
+    "lightning_attn_check",
+    "lightning_attn_status_string",
+    "lightning_attn_last_path",
+)
+
+
+class LightningAttnError(RuntimeError):
+    def __init__(self, status: int, where: str, detail=None):
+        self.status = status
+        self.detail = detail
+        super().__init__(f"{where}: {status_string(status)}" + (f" detail={detail}" if detail else ""))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m long_context_attn_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.lightning_attn_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                           f32, vp, vp, sz, vp]
+    lib.lightning_attn_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                                  i32, i32, i32, f32, vp, vp, sz, vp]
+    lib.lightning_attn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp,
+                                               sz, vp]
+    lib.lightning_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
+    lib.lightning_attn_workspace_size.restype = sz
+    lib.lightning_attn_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint * 4)]
+    lib.lightning_attn_status_string.argtypes = [i32]
+    lib.lightning_attn_status_string.restype = ctypes.c_char_p
+    lib.lightning_attn_last_path.argtypes = []
+    lib.lightning_attn_last_path.restype = ctypes.c_char_p
+    for f in ("lightning_attn_prefill", "lightning_attn_prefill_varlen", "lightning_attn_decode_step",
+              "lightning_attn_check"):
+        getattr(lib, f).restype = i32
+    return lib
+
+
+_lib = _load()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return LA_BF16
+    if t.dtype == torch.float32:
+        return LA_F32
+    raise TypeError(f"q/k/v/g/out must be bfloat16 or float32, got {t.dtype}")
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _f32_or_none(t):
+    if t is None:
+        return None
+    if t.dtype != torch.float32 or not t.is_contiguous():
+        raise TypeError("states and norm_weight must be contiguous float32 tensors")
+    return t
+
+
+def _check_contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def status_string(status: int) -> str:
+    return _lib.lightning_attn_status_string(int(status)).decode()
+
+
+def lightning_attn_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def lightning_attn_last_path() -> str:
+    return _lib.lightning_attn_last_path().decode()
+
+
+def lightning_attn_workspace_size(op: int, B_or_N: int, T_or_max: int, total_tokens: int, H: int, D: int,
+                                  block_size: int, dtype: int, mode: int) -> int:
+    return int(_lib.lightning_attn_workspace_size(op, B_or_N, T_or_max, total_tokens, H, D, block_size, dtype,
+                                                  mode))
+
+
+def new_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zero-filled uint8 device buffer (the caching allocator aligns it to >= 512 bytes)."""
+    ws = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    assert ws.data_ptr() % 256 == 0
+    return ws
+
+
+def lightning_attn_prefill(q, k, v, g, out, state_in=None, state_out=None, block_size=256,
+                           phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE, eps=1e-6, norm_weight=None,
+                           workspace=None, stream=None):
+    """q, k, v [B, T, H, D]; g, out [B, T, H*D]; states fp32 [B, H, D, D]."""
+    B, T, H, D = q.shape
+    _check_contig(q, k, v, g, out)
+    st = _lib.lightning_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(out), _ptr(_f32_or_none(state_in)),
+                                     _ptr(_f32_or_none(state_out)), B, T, H, D, block_size, _dtype(q), phi, mode,
+                                     eps, _ptr(_f32_or_none(norm_weight)), _ptr(workspace),
+                                     0 if workspace is None else workspace.numel(), _stream(stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_prefill")
+
+
+def lightning_attn_prefill_varlen(q, k, v, g, out, cu_seqlens, max_seqlen, state_in=None, state_out=None,
+                                  block_size=256, phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE, eps=1e-6,
+                                  norm_weight=None, workspace=None, stream=None):
+    """q, k, v [total, H, D]; g, out [total, H*D]; cu_seqlens int32 device [N + 1]."""
+    total, H, D = q.shape
+    _check_contig(q, k, v, g, out, cu_seqlens)
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    n = cu_seqlens.numel() - 1
+    st = _lib.lightning_attn_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(out),
+                                            _ptr(_f32_or_none(state_in)), _ptr(_f32_or_none(state_out)),
+                                            _ptr(cu_seqlens), n, int(max_seqlen), total, H, D, block_size, _dtype(q),
+                                            phi, mode, eps, _ptr(_f32_or_none(norm_weight)), _ptr(workspace),
+                                            0 if workspace is None else workspace.numel(), _stream(stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_prefill_varlen")
+
+
+def lightning_attn_decode_step(q, k, v, g, out, state, phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE, eps=1e-6,
+                               norm_weight=None, workspace=None, stream=None):
+    """q, k, v [B, H, D]; g, out [B, H*D]; state fp32 [B, H, D, D] updated in place."""
+    B, H, D = q.shape
+    _check_contig(q, k, v, g, out, state)
+    st = _lib.lightning_attn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(out), _ptr(_f32_or_none(state)),
+                                         B, H, D, _dtype(q), phi, mode, eps, _ptr(_f32_or_none(norm_weight)),
+                                         _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                         _stream(stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_decode_step")
+
+
+def lightning_attn_check(workspace, stream=None, raise_on_error=True):
+    """Synchronise the stream and read/clear the device error record of `workspace`."""
+    detail = (ctypes.c_uint * 4)()
+    st = _lib.lightning_attn_check(_ptr(workspace), _stream(stream), ctypes.byref(detail))
+    if st != LA_OK and raise_on_error:
+        raise LightningAttnError(st, "lightning_attn_check", tuple(detail))
+    return st, tuple(detail)

@@ -1,0 +1,91 @@
+"""The C ABI on the host (no GPU): the library loads, exports every symbol the header
+declares, and rejects invalid arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(HEADER_DIR):
+        if fn.endswith(".h"):
+            src = open(os.path.join(HEADER_DIR, fn)).read()
+            names |= set(re.findall(r"LA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_attn_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert {"lightning_attn_prefill", "lightning_attn_prefill_varlen", "lightning_attn_decode_step"} <= names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_binding_names_match_header(lib):
+    from long_context_attn_b200 import lightning_attn as la
+    assert set(la.EXPORTED) == _declared()
+    for n in la.EXPORTED:
+        assert callable(getattr(la, n))
+
+
+def test_status_strings(lib):
+    lib.lightning_attn_status_string.restype = ctypes.c_char_p
+    assert lib.lightning_attn_status_string(0) == b"LA_OK"
+    assert lib.lightning_attn_status_string(4) == b"LA_ERR_TIMEOUT"
+    assert lib.lightning_attn_status_string(99) == b"LA_ERR_UNKNOWN"
+
+
+def test_decode_workspace_size_is_host_only(lib):
+    lib.lightning_attn_workspace_size.restype = ctypes.c_size_t
+    n = lib.lightning_attn_workspace_size(2, 256, 0, 0, 64, 128, 0, 1, 2)
+    # error record + counters + y [B, H, D] fp32 + per-head partial sums
+    assert n >= 256 + 256 * 64 * 128 * 4 + 256 * 64 * 4
+    assert lib.lightning_attn_workspace_size(2, 0, 0, 0, 64, 128, 0, 1, 2) == 0
+    assert lib.lightning_attn_workspace_size(2, 4, 0, 0, 64, 96, 0, 1, 2) == 0  # D not supported
+
+
+def test_invalid_arguments_rejected_before_launch(lib):
+    f = lib.lightning_attn_prefill
+    vp = ctypes.c_void_p
+    f.argtypes = [vp, vp, vp, vp, vp, vp, vp] + [ctypes.c_int] * 8 + [ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
+    fake = vp(0x1000)
+    odd = vp(0x1008)
+    ws = vp(0x100000)
+    args = dict(q=fake, k=fake, v=fake, g=fake, out=fake, si=None, so=None, B=1, T=8, H=2, D=128, C=256,
+                dt=1, phi=0, mode=2, eps=1e-6, w=None, ws=ws, wsb=1 << 30, st=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(a["q"], a["k"], a["v"], a["g"], a["out"], a["si"], a["so"], a["B"], a["T"], a["H"], a["D"],
+                 a["C"], a["dt"], a["phi"], a["mode"], a["eps"], a["w"], a["ws"], a["wsb"], a["st"])
+
+    assert call(D=96) == 1          # unsupported head dim
+    assert call(q=None) == 1        # missing input
+    assert call(g=None) == 1        # gate required in RMSNORM_GATE mode
+    assert call(k=odd) == 1         # misaligned
+    assert call(dt=7) == 1          # bad enum
+    assert call(mode=1, eps=0.0) == 1   # norm needs eps > 0
+    assert call(B=0) == 1
+    assert call(C=0) == 1
+    assert call(H=200) == 1         # H*D > 16384 with a norm mode
+    assert call(ws=None) == 1
+    assert call(ws=vp(0x100010)) == 1   # workspace not 256-byte aligned
+
+    d = lib.lightning_attn_decode_step
+    d.argtypes = [vp, vp, vp, vp, vp, vp] + [ctypes.c_int] * 6 + [ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
+    assert d(fake, fake, fake, fake, fake, None, 4, 2, 128, 1, 0, 2, ctypes.c_float(1e-6), None, ws, 1 << 20,
+             None) == 1  # missing state
+    assert d(fake, fake, fake, fake, fake, fake, 4, 2, 128, 1, 0, 2, ctypes.c_float(1e-6), None, ws, 16,
+             None) == 1  # workspace too small
