@@ -1,8 +1,852 @@
-// Placeholder: the tcgen05 prefill kernel is not built yet; every call takes the SIMT path.
+// Lightning Attention prefill on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// What is computed ("六十四：MiniMax-01", section 3; "MiniMax-Text-01 405B MoE模型架构与
+// 训练策略解析", section 2.1; "MiniMax-01技术报告解读（二）计算优化", section 3):
+// causal linear attention with phi = SiLU on q and k, evaluated block by block with the
+// block size C (256 in the deployment config).  For block j with rows Q_j, K_j, V_j:
+//     O_j = (phi(Q_j) phi(K_j)^T (.) M) V_j + phi(Q_j) S_{j-1}          (intra + inter)
+//     S_j = S_{j-1} + phi(K_j)^T V_j                                    (fp32 state carry)
+// followed by o = RMSNorm over the H*D head concatenation of a token times sigmoid(g).
+//
+// Design (B200, sm_100a):
+//  * One CTA owns one (head, 64-column slice of d_v) chain and walks all sequences.  With
+//    H = 64 that is 128 CTAs, one per SM, all resident at once.
+//  * Work is tiled in 128-row tiles (the tcgen05 M).  C = 256 is two tiles per block: the
+//    second tile multiplies by the first tile's keys densely and by its own keys under the
+//    causal mask; the all-zero upper-right quarter of the 256 x 256 block is never issued.
+//  * TMA loads Q, K (128 x 128) and V, G (128 x 64) tiles with the 128-byte swizzle into a
+//    two-slot ring.  A transform warpgroup applies SiLU in place (and zeroes tail rows).
+//  * One thread issues all MMAs (bf16 in, fp32 accumulate in TMEM):
+//      P   = phi(Q) phi(K)^T          SS, M128 x N(<=128) x K128, into TMEM
+//      O   = phi(Q) S_snap            SS, M128 x N64 x K128 (S_snap = bf16 copy of S)
+//      O  += P_bf16 V                 TS (P read back from TMEM), M128 x N64 x K(<=128)
+//      S  += phi(K)^T V               SS (both operands MN-major), M128 x N64 x K(<=128)
+//    The fp32 state S stays in TMEM for the whole sequence.
+//  * A conversion warpgroup turns P (fp32, TMEM) into masked bf16 in place and, at each
+//    block end, copies S into the bf16 snapshot the next block's inter product reads.
+//  * The epilogue warpgroup reads O, publishes the per-token sum of squares of its slice,
+//    and one tile later -- once all H * 2 CTAs have published that tile -- scales by the
+//    token's rsqrt(mean(y^2) + eps), the norm weight and sigmoid(g), and stores bf16 O
+//    with TMA.  The last CTA to publish a tile reduces the partial sums (fixed order).
+//  * Every wait is bounded (globaltimer); a wait that runs out records LA_ERR_TIMEOUT in
+//    the workspace and the CTA drains its async work, frees TMEM and exits.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "la_common.cuh"
 #include "la_prefill_tc.h"
+#include "la_sm100.cuh"
 
 namespace la {
-bool tc_eligible(const TcShape&, int) { return false; }
-size_t tc_workspace_bytes(int, int, int64_t, int, int, int) { return 0; }
-cudaError_t launch_tc_prefill(const TcArgs&, int, cudaStream_t) { return cudaErrorNotSupported; }
+using namespace sm100;
+
+namespace {
+
+constexpr int kD = 128;          // head dim (d_k = d_v)
+constexpr int kDV = 64;          // d_v slice per CTA
+constexpr int kNdv = kD / kDV;   // CTAs per head
+constexpr int kTile = 128;       // rows per tile (MMA M)
+constexpr int kThreads = 512;
+
+constexpr uint32_t kQBytes = kTile * kD * 2;     // 32 KiB (two 64-column swizzled boxes)
+constexpr uint32_t kKBytes = kQBytes;
+constexpr uint32_t kVBytes = kTile * kDV * 2;    // 16 KiB
+constexpr uint32_t kGBytes = kVBytes;
+constexpr uint32_t kSnapBytes = kD * kDV * 2;    // 16 KiB
+constexpr uint32_t kBoxBytes = kTile * 64 * 2;   // one 128-row x 64-column box
+
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = OFF_Q + 2 * kQBytes;
+constexpr uint32_t OFF_V = OFF_K + 2 * kKBytes;
+constexpr uint32_t OFF_G = OFF_V + 2 * kVBytes;
+constexpr uint32_t OFF_SNAP = OFF_G + 2 * kGBytes;
+constexpr uint32_t OFF_BARS = OFF_SNAP + kSnapBytes;
+
+// TMEM columns (512 allocated; 128 lanes each)
+constexpr uint32_t TM_S = 0;      // fp32 state slice, 64 columns
+constexpr uint32_t TM_O = 64;     // 3 output accumulators x 64 columns
+constexpr uint32_t TM_P = 256;    // 2 score tiles x 128 columns
+constexpr uint32_t kTmemCols = 512;
+
+struct Bars {
+  uint64_t full_qkv[2], xformed[2], empty[2], full_g[2], empty_g[2];
+  uint64_t p_full, p_conv, pv_done;
+  uint64_t o_full[3], o_empty[3];
+  uint64_t s_done, snap_ready, final_bar;
+  uint64_t wg3_bar;      // epilogue warpgroup sync (bounded, unlike bar.sync)
+  uint32_t tmem_base;
+  int abort_flag;
+  int last_flag;
+  int go_flag;
+  float w[kDV];
+};
+
+constexpr uint32_t kSmemBytes = OFF_BARS + sizeof(Bars) + 1024;  // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+struct TcParams {
+  const float* state_in;
+  float* state_out;
+  const int* cu;
+  int nseq, T, H, C, phi_identity, mode, max_tiles;
+  int64_t tokens;
+  float eps;
+  const float* w;
+  ErrRec* err;
+  unsigned int* cnt;
+  float* part;
+  float* rnorm;
+  uint16_t* out;
+};
+
+constexpr uint32_t kIdescQS = make_idesc_bf16(128, kDV, 0, 1);
+constexpr uint32_t kIdescPV = make_idesc_bf16(128, kDV, 0, 1);
+constexpr uint32_t kIdescDS = make_idesc_bf16(128, kDV, 1, 1);
+
+__device__ __forceinline__ int pad_rows(int vr) { return vr <= 32 ? 32 : (vr <= 64 ? 64 : 128); }
+
+// Rows [row0, row0 + L) of sequence s.  Invalid cu_seqlens entries are reported and the
+// sequence is treated as empty (every role and every CTA reaches the same decision).
+__device__ __forceinline__ void seq_range(const TcParams& p, int s, int64_t& row0, int& L) {
+  if (p.cu) {
+    const int a = __ldg(p.cu + s), b = __ldg(p.cu + s + 1);
+    row0 = a;
+    L = b - a;
+    if (a < 0 || L < 0 || static_cast<int64_t>(b) > p.tokens || ((L + kTile - 1) / kTile) > p.max_tiles) {
+      if (threadIdx.x == 0) report(p.err, LA_ERR_DEVICE, SITE_VARLEN_CU, s, 0);
+      L = 0;
+    }
+  } else {
+    row0 = static_cast<int64_t>(s) * p.T;
+    L = p.T;
+  }
+}
+
+__device__ __forceinline__ bool aborted(Bars& B) { return *reinterpret_cast<volatile int*>(&B.abort_flag) != 0; }
+
+// Bounded wait for phase `parity` of an mbarrier.  Returns false (after recording a
+// timeout, or because another role already did) when the CTA is aborting.
+__device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars& B, const TcParams& p, uint32_t site,
+                                      uint32_t index) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  const uint64_t lim = wait_limit_ns(p.err);
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 31u) == 0) {
+      if (aborted(B)) return false;
+      if (globaltimer_ns() - t0 > lim) {
+        report(p.err, LA_ERR_TIMEOUT, site, index, parity);
+        *reinterpret_cast<volatile int*>(&B.abort_flag) = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Short bounded wait used while draining at exit (never records an error).
+__device__ __noinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) return;
+  }
+}
+
+// The same wait taken by every lane of a warp: the outcome is made warp-uniform so that
+// the .sync.aligned tcgen05 instructions that follow always see a converged warp.
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, Bars& B, const TcParams& p,
+                                              uint32_t site, uint32_t index) {
+  const bool ok = wait_bar(bar, parity, B, p, site, index);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// Bounded barrier of a 128-thread warpgroup on an mbarrier (count 128).  A lane that has
+// left never hangs the others: they give up when the CTA aborts or the limit runs out.
+__device__ __forceinline__ bool wg_sync(uint64_t* bar, uint32_t& phase, Bars& B, const TcParams& p, uint32_t site,
+                                        uint32_t index) {
+  mbar_arrive(bar);
+  const bool ok = wait_bar_warp(bar, phase, B, p, site, index);
+  phase ^= 1u;
+  return ok;
+}
+
+__device__ __forceinline__ uint32_t silu_bf16x2(uint32_t x) {
+  const float lo = __uint_as_float(x << 16), hi = __uint_as_float(x & 0xFFFF0000u);
+  return pack_bf16x2(silu_fast(lo), silu_fast(hi));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// ======================================================================================
+// The kernel
+// ======================================================================================
+__global__ void __launch_bounds__(kThreads, 1)
+lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                            const __grid_constant__ CUtensorMap tm_o, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw_addr);
+  Bars& B = *reinterpret_cast<Bars*>(smem + OFF_BARS);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int h = blockIdx.x / kNdv;
+  const int dvt = blockIdx.x % kNdv;
+  const int tpb = p.C / kTile;           // tiles per block (1 or 2)
+  const bool norm = p.mode != LA_OUT_RAW;
+  const bool gate = p.mode == LA_OUT_RMSNORM_GATE;
+  const int W = p.H * kNdv;              // CTAs contributing to one token's norm
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&B.full_qkv[i], 1);
+      mbar_init(&B.xformed[i], 128);
+      mbar_init(&B.empty[i], 1);
+      mbar_init(&B.full_g[i], 1);
+      mbar_init(&B.empty_g[i], 1);
+    }
+    mbar_init(&B.p_full, 1);
+    mbar_init(&B.p_conv, 128);
+    mbar_init(&B.pv_done, 1);
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&B.o_full[i], 1);
+      mbar_init(&B.o_empty[i], 128);
+    }
+    mbar_init(&B.s_done, 1);
+    mbar_init(&B.snap_ready, 128);
+    mbar_init(&B.final_bar, 1);
+    mbar_init(&B.wg3_bar, 128);
+    B.abort_flag = 0;
+    B.last_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc<kTmemCols>(&B.tmem_base);
+  if (tid >= 384 && tid < 384 + kDV) B.w[tid - 384] = p.w ? p.w[h * kD + dvt * kDV + (tid - 384)] : 1.0f;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = B.tmem_base;
+
+  // ------------------------------------------------------------------------------------
+  // Warp 0: TMA producer
+  // ------------------------------------------------------------------------------------
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      if (gate) prefetch_tmap(&tm_g);
+      const uint64_t pol = policy_evict_first();
+      uint32_t uses[2] = {0, 0}, guses[2] = {0, 0};
+      int t = 0;
+      bool have_prev = false;
+      int prev_t = 0;
+      int64_t prev_row = 0;
+      bool ok = true;
+      auto load_g = [&](int tt, int64_t row) -> bool {
+        const int gs = tt & 1;
+        if (guses[gs] > 0 && !wait_bar(&B.empty_g[gs], (guses[gs] - 1) & 1, B, p, SITE_TC_PRODUCER, tt)) return false;
+        mbar_arrive_expect_tx(&B.full_g[gs], kGBytes);
+        tma_load_2d(smem + OFF_G + gs * kGBytes, &tm_g, h * kD + dvt * kDV, static_cast<int32_t>(row), &B.full_g[gs],
+                    pol);
+        guses[gs]++;
+        return true;
+      };
+      for (int s = 0; s < p.nseq && ok; ++s) {
+        int64_t row0;
+        int L;
+        seq_range(p, s, row0, L);
+        const int nt = (L + kTile - 1) / kTile;
+        for (int i = 0; i < nt; ++i) {
+          const int slot = (tpb == 2) ? (i & 1) : (t & 1);
+          if (uses[slot] > 0 && !wait_bar(&B.empty[slot], (uses[slot] - 1) & 1, B, p, SITE_TC_PRODUCER, t)) {
+            ok = false;
+            break;
+          }
+          const int32_t row = static_cast<int32_t>(row0 + static_cast<int64_t>(i) * kTile);
+          mbar_arrive_expect_tx(&B.full_qkv[slot], kQBytes + kKBytes + kVBytes);
+          uint8_t* q = smem + OFF_Q + slot * kQBytes;
+          uint8_t* k = smem + OFF_K + slot * kKBytes;
+          tma_load_2d(q, &tm_q, h * kD, row, &B.full_qkv[slot], pol);
+          tma_load_2d(q + kBoxBytes, &tm_q, h * kD + 64, row, &B.full_qkv[slot], pol);
+          tma_load_2d(k, &tm_k, h * kD, row, &B.full_qkv[slot], pol);
+          tma_load_2d(k + kBoxBytes, &tm_k, h * kD + 64, row, &B.full_qkv[slot], pol);
+          tma_load_2d(smem + OFF_V + slot * kVBytes, &tm_v, h * kD + dvt * kDV, row, &B.full_qkv[slot], pol);
+          uses[slot]++;
+          if (gate) {
+            if (have_prev && !load_g(prev_t, prev_row)) {
+              ok = false;
+              break;
+            }
+            have_prev = true;
+            prev_t = t;
+            prev_row = row;
+          }
+          ++t;
+        }
+      }
+      if (ok && gate && have_prev) load_g(prev_t, prev_row);
+      // Drain: every issued load must have landed before the CTA may exit.
+      for (int i = 0; i < 2; ++i) {
+        if (uses[i] > 0) drain_bar(&B.full_qkv[i], (uses[i] - 1) & 1);
+        if (guses[i] > 0) drain_bar(&B.full_g[i], (guses[i] - 1) & 1);
+      }
+    }
+  }
+  // ------------------------------------------------------------------------------------
+  // Warp 1: MMA issuer (one thread)
+  // ------------------------------------------------------------------------------------
+  else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t uses[2] = {0, 0};
+      uint32_t snap_waits = 0;
+      int t = 0;
+      bool ok = true;
+      for (int s = 0; s < p.nseq && ok; ++s) {
+        int64_t row0;
+        int L;
+        seq_range(p, s, row0, L);
+        const int nt = (L + kTile - 1) / kTile;
+        for (int i = 0; i < nt; ++i) {
+          const int u = i % tpb;
+          const int slot = (tpb == 2) ? (i & 1) : (t & 1);
+          const int ob = t % 3;
+          const int vr = min(kTile, L - i * kTile);
+          const int nk = pad_rows(vr);
+          if (!wait_bar(&B.xformed[slot], uses[slot] & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
+          uses[slot]++;
+          tc_fence_after();
+          if (t > 0 && !wait_bar(&B.pv_done, (t - 1) & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t qa = sbase + OFF_Q + slot * kQBytes;
+          // P[kt] = phi(Q_i) phi(K_kt)^T
+          for (int kt = 0; kt <= u; ++kt) {
+            const int kslot = (tpb == 2) ? kt : slot;
+            const uint32_t n = (kt == u) ? static_cast<uint32_t>(nk) : 128u;
+            const uint32_t kb = sbase + OFF_K + kslot * kKBytes;
+            const uint32_t idesc = make_idesc_bf16(128, n, 0, 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
+              mma_ss(tmem + TM_P + 128 * kt, make_sdesc(qa + off, 16, 1024), make_sdesc(kb + off, 16, 1024), idesc,
+                     k > 0);
+            }
+          }
+          mma_commit(&B.p_full);
+          // O = phi(Q_i) S_snap
+          if (u == 0) {
+            if (!wait_bar(&B.snap_ready, snap_waits & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
+            snap_waits++;
+            tc_fence_after();
+          }
+          if (t >= 3) {
+            if (!wait_bar(&B.o_empty[ob], ((t / 3) - 1) & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
+            tc_fence_after();
+          }
+          const uint32_t od = tmem + TM_O + kDV * ob;
+          const uint32_t snap = sbase + OFF_SNAP;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
+            mma_ss(od, make_sdesc(qa + off, 16, 1024), make_sdesc(snap + k * 2048, kBoxBytes, 1024), kIdescQS, k > 0);
+          }
+          // O += P_bf16 V
+          if (!wait_bar(&B.p_conv, t & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
+          tc_fence_after();
+          for (int kt = 0; kt <= u; ++kt) {
+            const int kslot = (tpb == 2) ? kt : slot;
+            const int kext = (kt == u) ? nk : 128;
+            const uint32_t vb = sbase + OFF_V + kslot * kVBytes;
+            for (int k = 0; k < kext / 16; ++k)
+              mma_ts(od, tmem + TM_P + 128 * kt + 8 * k, make_sdesc(vb + k * 2048, kBoxBytes, 1024), kIdescPV, 1);
+          }
+          mma_commit(&B.o_full[ob]);
+          mma_commit(&B.pv_done);
+          // S += phi(K_i)^T V_i
+          {
+            const uint32_t kb = sbase + OFF_K + slot * kKBytes;
+            const uint32_t vb = sbase + OFF_V + slot * kVBytes;
+            for (int k = 0; k < nk / 16; ++k)
+              mma_ss(tmem + TM_S, make_sdesc(kb + k * 2048, kBoxBytes, 1024), make_sdesc(vb + k * 2048, kBoxBytes, 1024),
+                     kIdescDS, 1);
+          }
+          const bool blk_end = (u == tpb - 1) || (i == nt - 1);
+          if (tpb == 1) {
+            mma_commit(&B.empty[slot]);
+          } else if (blk_end) {
+            mma_commit(&B.empty[0]);
+            if (u == 1) mma_commit(&B.empty[1]);
+          }
+          if (blk_end) mma_commit(&B.s_done);
+          ++t;
+        }
+      }
+      // Drain: all MMAs complete before TMEM is released.
+      mma_commit(&B.final_bar);
+      drain_bar(&B.final_bar, 0);
+    }
+  }
+  // ------------------------------------------------------------------------------------
+  // Warps 4-7: SiLU transform of Q and K in shared memory; zero tail rows of K and V
+  // ------------------------------------------------------------------------------------
+  else if (warp >= 4 && warp < 8) {
+    const int wt = tid - 128;
+    uint32_t uses[2] = {0, 0};
+    int t = 0;
+    bool ok = true;
+    for (int s = 0; s < p.nseq && ok; ++s) {
+      int64_t row0;
+      int L;
+      seq_range(p, s, row0, L);
+      const int nt = (L + kTile - 1) / kTile;
+      for (int i = 0; i < nt; ++i) {
+        const int slot = (tpb == 2) ? (i & 1) : (t & 1);
+        if (!wait_bar_warp(&B.full_qkv[slot], uses[slot] & 1, B, p, SITE_TC_TRANSFORM, t)) { ok = false; break; }
+        uses[slot]++;
+        const int vr = min(kTile, L - i * kTile);
+        const uint32_t qa = sbase + OFF_Q + slot * kQBytes;
+        const uint32_t ka = sbase + OFF_K + slot * kKBytes;
+#pragma unroll 4
+        for (int m = 0; m < 16; ++m) {
+          const uint32_t off = static_cast<uint32_t>(wt + 128 * m) * 16u;
+          const int row = static_cast<int>((off & (kBoxBytes - 1)) >> 7);
+          uint4 kv = lds128(ka + off);
+          if (row >= vr) {
+            kv = make_uint4(0, 0, 0, 0);
+          } else if (!p.phi_identity) {
+            kv.x = silu_bf16x2(kv.x); kv.y = silu_bf16x2(kv.y); kv.z = silu_bf16x2(kv.z); kv.w = silu_bf16x2(kv.w);
+          }
+          sts128(ka + off, kv);
+          if (!p.phi_identity) {
+            uint4 qv = lds128(qa + off);
+            qv.x = silu_bf16x2(qv.x); qv.y = silu_bf16x2(qv.y); qv.z = silu_bf16x2(qv.z); qv.w = silu_bf16x2(qv.w);
+            sts128(qa + off, qv);
+          }
+        }
+        if (vr < kTile) {
+          const uint32_t va = sbase + OFF_V + slot * kVBytes;
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const uint32_t off = static_cast<uint32_t>(wt + 128 * m) * 16u;
+            if (static_cast<int>(off >> 7) >= vr) sts128(va + off, make_uint4(0, 0, 0, 0));
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&B.xformed[slot]);
+        ++t;
+      }
+    }
+  }
+  // ------------------------------------------------------------------------------------
+  // Warps 8-11: P conversion (fp32 -> masked bf16, in TMEM) and the state snapshot
+  // ------------------------------------------------------------------------------------
+  else if (warp >= 8 && warp < 12) {
+    const int wt = tid - 256;                      // TMEM lane = row
+    const uint32_t lane_off = static_cast<uint32_t>(wt & ~31) << 16;
+    const uint32_t snap = sbase + OFF_SNAP;
+    int t = 0;
+    uint32_t blk = 0;
+    bool ok = true;
+    for (int s = 0; s < p.nseq && ok; ++s) {
+      int64_t row0;
+      int L;
+      seq_range(p, s, row0, L);
+      const int nt = (L + kTile - 1) / kTile;
+      // Initial state: S0 (or zeros) into TMEM and the bf16 snapshot.
+      const int64_t st_row = ((static_cast<int64_t>(s) * p.H + h) * kD + wt) * kD + dvt * kDV;
+      {
+        float v[kDV];
+#pragma unroll
+        for (int c = 0; c < kDV; c += 4) {
+          float4 x = p.state_in ? *reinterpret_cast<const float4*>(p.state_in + st_row + c) : make_float4(0, 0, 0, 0);
+          v[c] = x.x; v[c + 1] = x.y; v[c + 2] = x.z; v[c + 3] = x.w;
+        }
+        if (nt == 0) {
+          if (p.state_out)
+            for (int c = 0; c < kDV; c += 4)
+              *reinterpret_cast<float4*>(p.state_out + st_row + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+          continue;
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < kDV; c0 += 16) {
+          uint32_t r[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(v[c0 + e]);
+          tmem_st16(tmem + lane_off + TM_S + c0, r);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 pk = make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]), pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                                pack_bf16x2(v[8 * c + 4], v[8 * c + 5]), pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+          sts128(snap + sw128_offset(wt, c), pk);
+        }
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&B.snap_ready);
+      }
+      for (int i = 0; i < nt; ++i) {
+        const int u = i % tpb;
+        const int vr = min(kTile, L - i * kTile);
+        const int nk = pad_rows(vr);
+        if (!wait_bar_warp(&B.p_full, t & 1, B, p, SITE_TC_CONVERT, t)) { ok = false; break; }
+        tc_fence_after();
+        for (int kt = 0; kt <= u; ++kt) {
+          const bool diag = (kt == u);
+          const int ncols = diag ? nk : 128;
+          const uint32_t base = tmem + lane_off + TM_P + 128 * kt;
+          for (int c = 0; c < ncols / 32; ++c) {
+            uint32_t x[32];
+            tmem_ld32(base + 32 * c, x);
+            tmem_ld_wait();
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int j = 32 * c + 2 * e;
+              float a = __uint_as_float(x[2 * e]), b = __uint_as_float(x[2 * e + 1]);
+              if (diag) {
+                a = (j <= wt) ? a : 0.f;
+                b = (j + 1 <= wt) ? b : 0.f;
+              }
+              pk[e] = pack_bf16x2(a, b);
+            }
+            tmem_st16(base + 16 * c, pk);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&B.p_conv);
+        const bool blk_end = (u == tpb - 1) || (i == nt - 1);
+        if (blk_end) {
+          if (!wait_bar_warp(&B.s_done, blk & 1, B, p, SITE_TC_CONVERT, t)) { ok = false; break; }
+          blk++;
+          tc_fence_after();
+          uint32_t x0[32], x1[32];
+          tmem_ld32(tmem + lane_off + TM_S, x0);
+          tmem_ld32(tmem + lane_off + TM_S + 32, x1);
+          tmem_ld_wait();
+          if (i == nt - 1) {
+            if (p.state_out) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 4) {
+                *reinterpret_cast<float4*>(p.state_out + st_row + c) =
+                    make_float4(__uint_as_float(x0[c]), __uint_as_float(x0[c + 1]), __uint_as_float(x0[c + 2]),
+                                __uint_as_float(x0[c + 3]));
+                *reinterpret_cast<float4*>(p.state_out + st_row + 32 + c) =
+                    make_float4(__uint_as_float(x1[c]), __uint_as_float(x1[c + 1]), __uint_as_float(x1[c + 2]),
+                                __uint_as_float(x1[c + 3]));
+              }
+            }
+            tc_fence_before();
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint32_t* a = x0 + 8 * c;
+              const uint32_t* b = x1 + 8 * c;
+              sts128(snap + sw128_offset(wt, c),
+                     make_uint4(pack_bf16x2(__uint_as_float(a[0]), __uint_as_float(a[1])),
+                                pack_bf16x2(__uint_as_float(a[2]), __uint_as_float(a[3])),
+                                pack_bf16x2(__uint_as_float(a[4]), __uint_as_float(a[5])),
+                                pack_bf16x2(__uint_as_float(a[6]), __uint_as_float(a[7]))));
+              sts128(snap + sw128_offset(wt, c + 4),
+                     make_uint4(pack_bf16x2(__uint_as_float(b[0]), __uint_as_float(b[1])),
+                                pack_bf16x2(__uint_as_float(b[2]), __uint_as_float(b[3])),
+                                pack_bf16x2(__uint_as_float(b[4]), __uint_as_float(b[5])),
+                                pack_bf16x2(__uint_as_float(b[6]), __uint_as_float(b[7]))));
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&B.snap_ready);
+          }
+        }
+        ++t;
+      }
+    }
+  }
+  // ------------------------------------------------------------------------------------
+  // Warps 12-15: epilogue (sum of squares, cross-head norm exchange, gate, store)
+  // ------------------------------------------------------------------------------------
+  else if (warp >= 12) {
+    const int wt = tid - 384;                      // TMEM lane = row of the tile
+    const uint32_t lane_off = static_cast<uint32_t>(wt & ~31) << 16;
+    const int HD = p.H * kD;
+    uint32_t guses[2] = {0, 0};
+    uint32_t sph = 0;                              // phase of the warpgroup barrier
+    bool ok = true;
+
+    struct Pend {
+      int t, s, i, vr;
+      int64_t row;
+    };
+    Pend pend{};
+    bool have_pend = false;
+
+    // Scale, gate and store one tile whose O is still in TMEM.
+    auto finalize = [&](const Pend& q) -> bool {
+      const int ob = q.t % 3;
+      const int gs = q.t & 1;
+      const int64_t grow = q.row + wt;
+      const uint32_t tix = static_cast<uint32_t>(q.t);
+      float rn = 1.0f;
+      if (norm) {
+        unsigned int* c = p.cnt + static_cast<int64_t>(q.s) * p.max_tiles + q.i;
+        if (wt == 0) {
+          int go = 1;
+          const uint64_t t0 = globaltimer_ns();
+          const uint64_t lim = wait_limit_ns(p.err);
+          while (ld_acquire_gpu(c) < static_cast<uint32_t>(W + 1)) {
+            if (aborted(B)) { go = 0; break; }
+            if (globaltimer_ns() - t0 > lim) {
+              report(p.err, LA_ERR_TIMEOUT, SITE_TC_NORM_WAIT, static_cast<uint32_t>(q.s * p.max_tiles + q.i),
+                     ld_acquire_gpu(c));
+              *reinterpret_cast<volatile int*>(&B.abort_flag) = 1;
+              go = 0;
+              break;
+            }
+            __nanosleep(64);
+          }
+          B.go_flag = go;
+        }
+        if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix)) return false;
+        if (!__all_sync(0xFFFFFFFFu, B.go_flag != 0)) return false;
+        (void)ld_acquire_gpu(c);
+        if (wt < q.vr) rn = __ldcg(p.rnorm + grow);
+      }
+      if (gate) {
+        if (!wait_bar_warp(&B.full_g[gs], guses[gs] & 1, B, p, SITE_TC_EPILOGUE, tix)) return false;
+        guses[gs]++;
+      }
+      const uint32_t stg = sbase + OFF_G + gs * kGBytes;
+      const uint32_t obase = tmem + lane_off + TM_O + kDV * ob;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t x[32];
+        tmem_ld32(obase + 32 * half, x);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = 4 * half + c;
+          const uint32_t addr = stg + sw128_offset(wt, chunk);
+          uint4 gv = make_uint4(0, 0, 0, 0);
+          if (gate) gv = lds128(addr);
+          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+          uint32_t ow[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = 8 * chunk + 2 * e;
+            float a = __uint_as_float(x[8 * c + 2 * e]) * rn;
+            float b = __uint_as_float(x[8 * c + 2 * e + 1]) * rn;
+            if (norm) {
+              a *= B.w[col];
+              b *= B.w[col + 1];
+            }
+            if (gate) {
+              a *= sigmoid_fast(__uint_as_float(gw[e] << 16));
+              b *= sigmoid_fast(__uint_as_float(gw[e] & 0xFFFF0000u));
+            }
+            ow[e] = pack_bf16x2(a, b);
+          }
+          sts128(addr, make_uint4(ow[0], ow[1], ow[2], ow[3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&B.o_empty[ob]);
+      fence_proxy_async_smem();
+      if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix)) return false;
+      if (q.vr == kTile) {
+        if (wt == 0) {
+          tma_store_2d(&tm_o, smem + OFF_G + gs * kGBytes, h * kD + dvt * kDV, static_cast<int32_t>(q.row));
+          bulk_commit();
+          bulk_wait_read0();
+          if (gate) mbar_arrive(&B.empty_g[gs]);
+        }
+      } else {
+        if (wt < q.vr) {
+          uint16_t* dst = p.out + grow * HD + h * kD + dvt * kDV;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + 8 * c) = lds128(stg + sw128_offset(wt, c));
+        }
+        if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix)) return false;
+        if (wt == 0 && gate) mbar_arrive(&B.empty_g[gs]);
+      }
+      // The staging buffer is free again once thread 0 has seen the store read it.
+      return wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix);
+    };
+
+    int t = 0;
+    for (int s = 0; s < p.nseq && ok; ++s) {
+      int64_t row0;
+      int L;
+      seq_range(p, s, row0, L);
+      const int nt = (L + kTile - 1) / kTile;
+      for (int i = 0; i < nt; ++i) {
+        const int ob = t % 3;
+        const int vr = min(kTile, L - i * kTile);
+        const int64_t row = row0 + static_cast<int64_t>(i) * kTile;
+        if (!wait_bar_warp(&B.o_full[ob], (t / 3) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+        tc_fence_after();
+        Pend cur{t, s, i, vr, row};
+        if (norm) {
+          // Sum of squares of this row's 64 outputs (fixed order).
+          float ss = 0.f;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t x[32];
+            tmem_ld32(tmem + lane_off + TM_O + kDV * ob + 32 * half, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(x[e]), __uint_as_float(x[e]), ss);
+          }
+          const int64_t grow = row + wt;
+          if (wt < vr) p.part[grow * W + h * kNdv + dvt] = ss;
+          __threadfence();
+          if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+          unsigned int* c = p.cnt + static_cast<int64_t>(s) * p.max_tiles + i;
+          if (wt == 0) {
+            const bool skip = (p.err->inject == INJECT_SKIP_PUBLISH) && blockIdx.x == 0;
+            B.last_flag = skip ? 0 : (atom_add_acq_rel_gpu(c, 1u) == static_cast<uint32_t>(W - 1));
+          }
+          if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+          if (B.last_flag) {
+            // Last CTA of this tile: reduce the W partial sums of every token in order.
+            __threadfence();
+            if (wt < vr) {
+              const float2* src = reinterpret_cast<const float2*>(p.part + grow * W);
+              float acc = 0.f;
+              for (int j = 0; j < W / 2; ++j) {
+                const float2 v = __ldcg(src + j);
+                acc += v.x;
+                acc += v.y;
+              }
+              p.rnorm[grow] = 1.0f / sqrtf(acc / static_cast<float>(HD) + p.eps);
+            }
+            __threadfence();
+            if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+            if (wt == 0) atom_add_acq_rel_gpu(c, 1u);
+          }
+          if (have_pend && !finalize(pend)) { ok = false; break; }
+          pend = cur;
+          have_pend = true;
+        } else {
+          if (!finalize(cur)) { ok = false; break; }
+        }
+        ++t;
+      }
+    }
+    if (ok && have_pend) finalize(pend);
+    if (wt == 0) bulk_wait0();
+  }
+
+  // Teardown: all roles are done (or aborted with their async work drained).
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc<kTmemCols>(tmem);
+}
+
+// ======================================================================================
+// Host side
+// ======================================================================================
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [rows, cols] bf16 row-major, box 64 columns x 128 rows, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTile)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+bool tc_eligible(const TcShape& s, int num_sms) {
+  if (!s.bf16 || s.D != kD || (s.C != 128 && s.C != 256) || s.H < 1) return false;
+  // The cross-head norm exchange needs every CTA of a token resident at once.
+  if (s.mode != LA_OUT_RAW && s.H * kNdv > num_sms) return false;
+  return true;
+}
+
+size_t tc_workspace_bytes(int nseq, int max_len, int64_t tokens, int H, int D, int C) {
+  (void)D;
+  (void)C;
+  const size_t max_tiles = (static_cast<size_t>(max_len) + kTile - 1) / kTile;
+  return up256(sizeof(unsigned int) * static_cast<size_t>(nseq) * (max_tiles ? max_tiles : 1)) +
+         up256(sizeof(float) * static_cast<size_t>(tokens) * H * kNdv) + up256(sizeof(float) * static_cast<size_t>(tokens));
+}
+
+cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream) {
+  (void)num_sms;
+  const int max_tiles = (a.max_len + kTile - 1) / kTile;
+  const size_t cnt_bytes = up256(sizeof(unsigned int) * static_cast<size_t>(a.nseq) * (max_tiles ? max_tiles : 1));
+  const size_t part_bytes = up256(sizeof(float) * static_cast<size_t>(a.tokens) * a.H * kNdv);
+  TcParams p{};
+  p.state_in = a.state_in;
+  p.state_out = a.state_out;
+  p.cu = a.cu;
+  p.nseq = a.nseq;
+  p.T = a.T;
+  p.H = a.H;
+  p.C = a.C;
+  p.phi_identity = a.phi_identity;
+  p.mode = a.mode;
+  p.max_tiles = max_tiles;
+  p.tokens = a.tokens;
+  p.eps = a.eps;
+  p.w = a.w;
+  p.err = a.err;
+  p.cnt = reinterpret_cast<unsigned int*>(a.ws);
+  p.part = reinterpret_cast<float*>(a.ws + cnt_bytes);
+  p.rnorm = reinterpret_cast<float*>(a.ws + cnt_bytes + part_bytes);
+  p.out = static_cast<uint16_t*>(a.out);
+
+  const int64_t cols = static_cast<int64_t>(a.H) * kD;
+  CUtensorMap mq, mk, mv, mg, mo;
+  if (!make_map(&mq, a.q, a.tokens, cols) || !make_map(&mk, a.k, a.tokens, cols) ||
+      !make_map(&mv, a.v, a.tokens, cols) || !make_map(&mo, a.out, a.tokens, cols))
+    return cudaErrorInvalidValue;
+  if (a.mode == LA_OUT_RMSNORM_GATE) {
+    if (!make_map(&mg, a.g, a.tokens, cols)) return cudaErrorInvalidValue;
+  } else {
+    mg = mq;  // never read
+  }
+  cudaError_t e = cudaMemsetAsync(a.ws, 0, cnt_bytes, stream);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(lightning_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  lightning_prefill_tc_kernel<<<a.H * kNdv, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, p);
+  return cudaGetLastError();
+}
+
 }  // namespace la
