@@ -1,0 +1,483 @@
+#!/usr/bin/env python
+"""Benchmark of the Lightning Attention forward on B200 (one JSON line on rank 0).
+
+Default workload: prefill of one 131072-token sequence, 64 heads of 128, bf16, block 256,
+RMSNorm over the head concatenation times sigmoid(gate), final fp32 state returned.
+A step is one lightning_attn_prefill call over that batch (the whole hot path: SiLU,
+intra- and inter-block products, the fp32 state carry, the norm and the gate).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+* value: tokens/s of the whole job (N ranks, each an independent replica of the workload:
+  the sequences/heads of the path are independent, so there is no data-path collective),
+  timed with CUDA events on the launching stream, inputs resident in HBM, max over ranks.
+  Inputs are larger than L2 (10.7 GB per step at 128K), so no L2 flush is needed.
+* roofline: the prefill kernel is bound by HBM; achieved = algorithmic bytes per launch
+  (q, k, v, g read + out written, bf16: 5 * H * D * 2 bytes per token, plus the state)
+  / mean launch duration from events around each call in the timed region.
+* e2e: the same metric through the C ABI with pinned host buffers; every step copies
+  q, k, v, g host->device and reads out (and the state) back.
+* cpu_baseline: the fp64 oracle timed on this host's cores on a bounded sample.
+* --impl reference: the oracle timed as the reference arm (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "lightning-attn prefill tokens/s @128K,H64,d128; % tensor/HBM roofline"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ----------------------------------------------------------------------------------------------
+_CLK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={_CLK_FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.text = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.text, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.text, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(self.text)) if len(r) >= 10]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x.strip())
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows]
+        util = [num(r[4]) for r in rows]
+        loaded = [s for s, u in zip(sm, util) if s is not None and (u or 0) >= 50] or [s for s in sm if s]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in rows for j in range(4) if r[6 + j].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": num(rows[0][2]),
+                "reasons": reasons, "samples": len(rows), "power_w_max": max((num(r[3]) or 0) for r in rows)}
+
+
+# ----------------------------------------------------------------------------------------------
+# Workloads
+# ----------------------------------------------------------------------------------------------
+def _bytes_per_token(H, D):
+    return 5 * H * D * 2  # q, k, v, g read + out written, bf16
+
+
+def _flops_per_token(H, D, C):
+    """(algorithmic, issued) FLOPs per token over all heads.
+
+    algorithmic: 2 d (C + 1) for the masked intra block (averaged over a block) plus 4 d^2
+    for the inter read phi(q)^T S and the state carry phi(k) v^T.
+    issued by the tensor-core kernel: 128-row tiles; a query tile multiplies by the key
+    tiles of its block up to the diagonal (the zero quarter of a 256-block is skipped),
+    and the two CTAs of a head (64 columns of d_v each) both compute the scores.
+    """
+    algo = H * (2 * D * (C + 1) + 4 * D * D)
+    tiles = C // 128
+    keys = 128 * (tiles + 1) / 2          # mean keys per query row multiplied
+    n_dv = 2
+    issued = H * (2 * keys * D * n_dv     # P = phi(Q) phi(K)^T, once per d_v slice
+                  + 2 * keys * D          # O += P V over both slices
+                  + 2 * D * D             # O += phi(Q) S
+                  + 2 * D * D)            # S += phi(K)^T V
+    return algo, issued
+
+
+class PrefillCase:
+    def __init__(self, name, w, device, rank):
+        import torch
+        from long_context_attn_b200 import lightning_attn as la
+        self.la, self.w = la, w
+        self.T, self.H, self.D, self.C = w.T, w.H, w.D, w.block_size
+        assert w.dtype == "bf16"
+        t0 = time.time()
+        q, k, v, g = synth.prefill_inputs(w.seed + 1000 * rank, w.T, w.H, w.D, "bf16", w.qkv_scale, True)
+        self.gen_s = time.time() - t0
+
+        def pin(a):
+            t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+            return t.pin_memory()
+
+        self.h_q, self.h_k, self.h_v, self.h_g = (pin(a) for a in (q, k, v, g))
+        del q, k, v, g
+        T, H, D = w.T, w.H, w.D
+        self.q = self.h_q.to(device).view(1, T, H, D)
+        self.k = self.h_k.to(device).view(1, T, H, D)
+        self.v = self.h_v.to(device).view(1, T, H, D)
+        self.g = self.h_g.to(device).view(1, T, H * D)
+        self.out = torch.empty((1, T, H * D), dtype=torch.bfloat16, device=device)
+        self.state = torch.empty((1, H, D, D), dtype=torch.float32, device=device)
+        self.h_out = torch.empty((1, T, H * D), dtype=torch.bfloat16).pin_memory()
+        self.h_state = torch.empty((1, H, D, D), dtype=torch.float32).pin_memory()
+        nbytes = la.lightning_attn_workspace_size(la.LA_OP_PREFILL, 1, T, 0, H, D, self.C, la.LA_BF16,
+                                                  la.LA_OUT_RMSNORM_GATE)
+        self.ws = la.new_workspace(nbytes, device)
+        self.tokens = T
+        self.alg_bytes = T * _bytes_per_token(H, D) + H * D * D * 4
+        self.alg_flops, self.issued_flops = (x * T for x in _flops_per_token(H, D, self.C))
+        self.h2d = sum(t.numel() * t.element_size() for t in (self.h_q, self.h_k, self.h_v, self.h_g))
+        self.d2h = self.h_out.numel() * 2 + self.h_state.numel() * 4
+
+    def step(self):
+        self.la.lightning_attn_prefill(self.q, self.k, self.v, self.g, self.out, None, self.state,
+                                       block_size=self.C, workspace=self.ws)
+
+    def e2e_step(self):
+        self.q.view(-1).copy_(self.h_q.view(-1), non_blocking=True)
+        self.k.view(-1).copy_(self.h_k.view(-1), non_blocking=True)
+        self.v.view(-1).copy_(self.h_v.view(-1), non_blocking=True)
+        self.g.view(-1).copy_(self.h_g.view(-1), non_blocking=True)
+        self.step()
+        self.h_out.copy_(self.out, non_blocking=True)
+        self.h_state.copy_(self.state, non_blocking=True)
+
+    def check(self):
+        self.la.lightning_attn_check(self.ws)
+
+    def oracle_sample(self, tokens):
+        """fp64 oracle on the first `tokens` rows of the same workload (all heads)."""
+        import oracle
+        w = self.w
+        q, k, v, g = synth.prefill_inputs(w.seed, tokens, w.H, w.D, "bf16", w.qkv_scale, True)
+        t0 = time.perf_counter()
+        oracle.prefill(q[None], k[None], v[None], g[None], store=False)
+        return time.perf_counter() - t0
+
+    def describe(self):
+        return {"workload": self.w.name, "B": 1, "T": self.T, "H": self.H, "D": self.D, "block_size": self.C,
+                "mode": "rmsnorm_gate", "state_out": True,
+                "l2": "inputs larger than L2 (%.1f GB per step), no flush" % (self.alg_bytes / 1e9)}
+
+
+class DecodeCase:
+    """256 sequences x 64 heads, one token each; S (1 GiB fp32) updated in place."""
+
+    def __init__(self, name, w, device, rank):
+        import torch
+        from long_context_attn_b200 import lightning_attn as la
+        self.la, self.w = la, w
+        B, H, D = w.B, w.H, w.D
+        t0 = time.time()
+        S = synth.decode_state(w.seed + 1000 * rank, B, H, D)
+        ring = [synth.decode_tokens(w.seed, s, B, H, D, "bf16", w.qkv_scale) for s in range(16)]
+        self.gen_s = time.time() - t0
+        self.S = torch.from_numpy(S).to(device)
+
+        def dev(a):
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+
+        self.ring = [tuple(dev(a) for a in r) for r in ring]
+        self.h_ring = [tuple(torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in r)
+                       for r in ring]
+        self.out = torch.empty((B, H * D), dtype=torch.bfloat16, device=device)
+        self.h_out = torch.empty((B, H * D), dtype=torch.bfloat16).pin_memory()
+        self.ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_DECODE, B, 0, 0, H, D, 0, la.LA_BF16,
+                                                                    la.LA_OUT_RMSNORM_GATE), device)
+        self.i = 0
+        self.tokens = B
+        self.alg_bytes = B * H * (2 * D * D * 4 + 5 * D * 2)
+        self.alg_flops = B * H * 4 * D * D
+        self.issued_flops = self.alg_flops
+        self.h2d = sum(a.numel() * 2 for a in self.h_ring[0])
+        self.d2h = self.h_out.numel() * 2
+
+    def step(self):
+        q, k, v, g = self.ring[self.i % 16]
+        self.i += 1
+        self.la.lightning_attn_decode_step(q, k, v, g, self.out, self.S, workspace=self.ws)
+
+    def e2e_step(self):
+        q, k, v, g = self.ring[self.i % 16]
+        hq, hk, hv, hg = self.h_ring[self.i % 16]
+        for d, h in ((q, hq), (k, hk), (v, hv), (g, hg)):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        self.h_out.copy_(self.out, non_blocking=True)
+
+    def check(self):
+        self.la.lightning_attn_check(self.ws)
+
+    def oracle_sample(self, seqs):
+        import oracle
+        w = self.w
+        q, k, v, g = synth.decode_tokens(w.seed, 0, w.B, w.H, w.D, "bf16", w.qkv_scale)
+        S = synth.decode_state(w.seed, w.B, w.H, w.D)
+        t0 = time.perf_counter()
+        oracle.decode(q[:seqs], k[:seqs], v[:seqs], g[:seqs], S[:seqs])
+        return time.perf_counter() - t0
+
+    def describe(self):
+        return {"workload": self.w.name, "B": self.w.B, "H": self.w.H, "D": self.w.D, "mode": "rmsnorm_gate",
+                "state": "fp32 [256,64,128,128] in place (1 GiB)",
+                "l2": "state larger than L2 (1 GiB read + written per step), no flush"}
+
+
+def _make_case(name, device, rank):
+    w = synth.WORKLOADS[name]
+    if w.kind == "prefill" and w.dtype == "bf16":
+        return PrefillCase(name, w, device, rank)
+    if w.kind == "decode":
+        return DecodeCase(name, w, device, rank)
+    raise SystemExit(f"workload {name} is not a bench workload")
+
+
+# ----------------------------------------------------------------------------------------------
+# Arms
+# ----------------------------------------------------------------------------------------------
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    case = _make_case(args.workload, device, rank)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        case.step()
+    case.check()
+    torch.cuda.synchronize()
+
+    # ---- device-resident timing ----
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            case.step()
+            ends[i].record(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    case.check()
+    elapsed_ms = e0.elapsed_time(e1)
+    launch_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    t = torch.tensor([elapsed_ms, launch_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms, launch_ms = float(t[0]), float(t[1])
+
+    # ---- end-to-end through the C ABI with pinned host buffers ----
+    for _ in range(min(2, args.warmup)):
+        case.e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        case.e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    case.check()
+    t = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t[0])
+
+    if rank == 0:
+        peaks = _peaks()
+        tokens_total = case.tokens * args.steps * world
+        value = tokens_total / (elapsed_ms / 1e3)
+        achieved_gbs = case.alg_bytes / (launch_ms / 1e3) / 1e9
+        line = {
+            "metric": METRIC if args.workload == "prefill_128k" else f"lightning-attn {args.workload} tokens/s",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded SplitMix64/Box-Muller)",
+            "config": dict(case.describe(), parallelism=f"replicas x{world} (independent sequences, no collective)"),
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": _traffic(args.workload),
+                         "peak_source": peaks["source"], "launch_ms": launch_ms,
+                         "algorithmic_bytes_per_launch": case.alg_bytes},
+            "tensor": {"algorithmic_tflops": case.alg_flops / (launch_ms / 1e3) / 1e12,
+                       "issued_tflops": case.issued_flops / (launch_ms / 1e3) / 1e12,
+                       "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                       "frac_algorithmic": case.alg_flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                       "frac_issued": case.issued_flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
+            "e2e": {"value": case.tokens * args.steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": case.h2d, "d2h_bytes_per_step": case.d2h},
+            "gpu_launches": args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = _cpu_baseline(case)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# Source files each measured kernel is built from (a traffic figure is tied to their hash).
+KERNEL_SOURCES = {
+    "prefill": ("la_prefill_tc.cu", "la_sm100.cuh", "la_common.cuh"),
+    "decode": ("la_decode.cu", "la_common.cuh"),
+}
+
+
+def kernel_source_hash(kind):
+    """Hash of the CUDA sources of one kernel; committed DRAM traffic is used only while it matches."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "long_context_attn_b200", "csrc")
+    for fn in KERNEL_SOURCES[kind]:
+        h.update(fn.encode())
+        h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(workload):
+    """DRAM bytes per launch of the dominant kernel (from ncu), or None once the kernel changed."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    entry = json.load(open(path)).get(workload)
+    kind = "decode" if workload.startswith("decode") else "prefill"
+    if not entry or entry.get("kernel_source_hash") != kernel_source_hash(kind):
+        return None
+    return entry["bytes_per_launch"]
+
+
+def _cpu_baseline(case):
+    import oracle
+    if isinstance(case, PrefillCase):
+        n = 4096
+        dt = case.oracle_sample(n)
+        return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                "sample": f"first {n} tokens of the {case.w.name} workload, all {case.H} heads, fp64, "
+                          f"recurrence + norm + gate ({dt:.1f} s)"}
+    n = 64
+    dt = case.oracle_sample(n)
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {n} of {case.w.B} sequences of one decode step, all heads, fp64 ({dt:.1f} s)"}
+
+
+def run_reference(args):
+    """The reference arm: the fp64 oracle on the host cores, on bounded samples of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w = synth.WORKLOADS[args.workload]
+    if w.kind == "prefill":
+        n = 1024
+        q, k, v, g = synth.prefill_inputs(w.seed, n, w.H, w.D, w.dtype, w.qkv_scale, True)
+
+        def step():
+            oracle.prefill(q[None], k[None], v[None], g[None], store=False)
+        unit_per_step = n
+        sample = f"first {n} tokens of {w.name} (all {w.H} heads) per step, fp64 recurrence + norm + gate"
+    else:
+        n = 16
+        q, k, v, g = synth.decode_tokens(w.seed, 0, w.B, w.H, w.D, "bf16", w.qkv_scale)
+        S = synth.decode_state(w.seed, n, w.H, w.D)
+
+        def step():
+            oracle.decode(q[:n], k[:n], v[:n], g[:n], S)
+        unit_per_step = n
+        sample = f"{n} of {w.B} sequences of one decode step per step, fp64"
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = unit_per_step * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC if args.workload == "prefill_128k" else f"lightning-attn {args.workload} tokens/s",
+        "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded SplitMix64/Box-Muller)",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "D": w.D, "block_size": w.block_size},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill_128k", choices=["prefill_8k", "prefill_128k", "decode_256"])
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        print("note: fewer than 3 warm-up steps; this run is not a valid bench line", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

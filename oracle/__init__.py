@@ -62,6 +62,8 @@ def _get():
         lib.oracle_quadratic.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
         lib.oracle_chunked.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
         lib.oracle_transform.argtypes = [vp, i64, i32, i32, i32, dbl, vp, vp, i32, vp]
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = ctypes.c_int
         for f in (lib.oracle_forward_packed, lib.oracle_prefill, lib.oracle_decode,
                   lib.oracle_quadratic, lib.oracle_chunked, lib.oracle_transform):
             f.restype = ctypes.c_int
@@ -167,6 +169,11 @@ def chunked(q, k, v, C, phi=PHI_SILU, s0=None):
                              _ptr(_c(s0, np.float64)), _ptr(y), _ptr(st)) != 0:
         raise ValueError("oracle_chunked rejected its arguments")
     return y, st
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle uses (the `cores` of a CPU timing)."""
+    return int(_get().oracle_num_threads())
 
 
 def transform(y, mode, eps=1e-6, norm_weight=None, g=None):

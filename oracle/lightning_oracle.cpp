@@ -25,6 +25,8 @@
 // (bf16 bits or fp32).  Layouts: q, k, v [tokens, H, D]; g and out [tokens, H*D];
 // states [seq, H, D(k), D(v)] row-major.
 
+#include <omp.h>
+
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -319,5 +321,8 @@ int oracle_transform(const double* y, int64_t tokens, int H, int D, int mode, do
   for (int64_t t = 0; t < tokens; ++t) transform_token(y + t * HD, HD, mode, eps, w, g, dtype, t, out + t * HD);
   return 0;
 }
+
+// Number of OpenMP threads the oracle's parallel loops use (reported with CPU timings).
+int oracle_num_threads() { return omp_get_max_threads(); }
 
 }  // extern "C"
