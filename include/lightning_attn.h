@@ -145,6 +145,36 @@ LA_API la_status lightning_attn_decode_step(const void* q, const void* k, const 
                                      const float* norm_weight, void* workspace, size_t workspace_bytes,
                                      la_stream_t stream);
 
+/* Size of the scratch array compiled into the library for
+ * lightning_attn_decode_step_noalloc (8.25 MiB: enough for B*H*D up to 2^21, e.g. 256
+ * sequences x 64 heads x 128). */
+#define LA_DECODE_NOALLOC_SCRATCH_BYTES 8650752u
+
+/*
+ * Decode step that allocates nothing and takes no workspace (the pages have no
+ * counterpart: this entry point exists for callers of this library that cannot allocate).
+ * It is for callers whose device memory is owned entirely by another allocator (e.g. a
+ * serving engine that reserves nearly all of HBM for its cache and state pools, where an
+ * extra cudaMalloc fails or fragments the pool) and for latency-critical decode loops in
+ * which cudaMalloc, which can synchronise the device, is not allowed.
+ *
+ * Same computation, arguments and results as lightning_attn_decode_step, without
+ * `workspace` / `workspace_bytes`.  Its scratch is a fixed array of
+ * LA_DECODE_NOALLOC_SCRATCH_BYTES bytes inside the library (one copy per GPU that loads the
+ * library, held until the process exits):
+ *   - The first call on each device looks up the array's device address (with that device
+ *     current); make that first call before any stream capture.
+ *   - Every call shares the array: each call clears the per-sequence counters on its stream,
+ *     and calls that overlap on the GPU (other streams, unordered host threads) race.
+ *   - Batches whose scratch would exceed the array (decode_workspace bytes > the size above)
+ *     return LA_ERR_UNSUPPORTED with nothing enqueued.
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+LA_API la_status lightning_attn_decode_step_noalloc(const void* q, const void* k, const void* v, const void* g,
+                                                    void* out, float* state, int B, int H, int D, la_dtype dtype,
+                                                    la_feature_map phi, la_out_mode mode, float eps,
+                                                    const float* norm_weight, la_stream_t stream);
+
 /*
  * Workspace bytes needed by one call (0 on invalid arguments).
  *   op == LA_OP_PREFILL:         B_or_N = B, T_or_max = T, total_tokens ignored.

@@ -27,6 +27,7 @@ EXPORTED = (
     "lightning_attn_prefill",
     "lightning_attn_prefill_varlen",
     "lightning_attn_decode_step",
+    "lightning_attn_decode_step_noalloc",
     "lightning_attn_workspace_size",
     "lightning_attn_check",
     "lightning_attn_status_string",
@@ -52,6 +53,8 @@ def _load():
                                                   i32, i32, i32, f32, vp, vp, sz, vp]
     lib.lightning_attn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp,
                                                sz, vp]
+    lib.lightning_attn_decode_step_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32,
+                                                       vp, vp]
     lib.lightning_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
     lib.lightning_attn_workspace_size.restype = sz
     lib.lightning_attn_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint * 4)]
@@ -60,7 +63,7 @@ def _load():
     lib.lightning_attn_last_path.argtypes = []
     lib.lightning_attn_last_path.restype = ctypes.c_char_p
     for f in ("lightning_attn_prefill", "lightning_attn_prefill_varlen", "lightning_attn_decode_step",
-              "lightning_attn_check"):
+              "lightning_attn_decode_step_noalloc", "lightning_attn_check"):
         getattr(lib, f).restype = i32
     return lib
 
@@ -168,6 +171,23 @@ def lightning_attn_decode_step(q, k, v, g, out, state, phi=LA_PHI_SILU, mode=LA_
                                          _stream(stream))
     if st != LA_OK:
         raise LightningAttnError(st, "lightning_attn_decode_step")
+
+
+def lightning_attn_decode_step_noalloc(q, k, v, g, out, state, phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE,
+                                       eps=1e-6, norm_weight=None, stream=None):
+    """Decode step without a workspace, for callers that cannot allocate device memory.
+
+    Same arguments and results as lightning_attn_decode_step; the scratch is a fixed array
+    inside the library shared by every call (calls that overlap on the GPU race), and
+    batches that do not fit it raise with LA_ERR_UNSUPPORTED.
+    """
+    B, H, D = q.shape
+    _check_contig(q, k, v, g, out, state)
+    st = _lib.lightning_attn_decode_step_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(out),
+                                                 _ptr(_f32_or_none(state)), B, H, D, _dtype(q), phi, mode, eps,
+                                                 _ptr(_f32_or_none(norm_weight)), _stream(stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_decode_step_noalloc")
 
 
 def lightning_attn_check(workspace, stream=None, raise_on_error=True):
