@@ -14,20 +14,24 @@
 //  * Work is tiled in 128-row tiles (the tcgen05 M).  C = 256 is two tiles per block: the
 //    second tile multiplies by the first tile's keys densely and by its own keys under the
 //    causal mask; the all-zero upper-right quarter of the 256 x 256 block is never issued.
-//  * TMA loads Q, K (128 x 128) and V, G (128 x 64) tiles with the 128-byte swizzle into a
-//    two-slot ring.  A transform warpgroup applies SiLU in place (and zeroes tail rows).
-//  * One thread issues all MMAs (bf16 in, fp32 accumulate in TMEM):
+//  * TMA loads Q, K (128 x 128) and V, G (128 x 64) tiles with the 128-byte swizzle into
+//    rings in shared memory; six transform warps apply SiLU in place (and zero tail rows).
+//  * One thread issues all MMAs (bf16 in, fp32 accumulate in TMEM), per tile:
 //      P   = phi(Q) phi(K)^T          SS, M128 x N(<=128) x K128, into TMEM
-//      O   = phi(Q) S_snap            SS, M128 x N64 x K128 (S_snap = bf16 copy of S)
-//      O  += P_bf16 V                 TS (P read back from TMEM), M128 x N64 x K(<=128)
+//      O   = P_bf16 V                 TS (P read back from TMEM), M128 x N64 x K(<=128)
+//      O  += phi(Q) S_snap            SS, M128 x N64 x K128 (S_snap = bf16 copy of S)
 //      S  += phi(K)^T V               SS (both operands MN-major), M128 x N64 x K(<=128)
-//    The fp32 state S stays in TMEM for the whole sequence.
+//    The fp32 state S stays in TMEM for the whole sequence; the inter product comes last
+//    so the snapshot of S taken at the previous block end is ready by then.
 //  * A conversion warpgroup turns P (fp32, TMEM) into masked bf16 in place and, at each
 //    block end, copies S into the bf16 snapshot the next block's inter product reads.
-//  * The epilogue warpgroup reads O, publishes the per-token sum of squares of its slice,
-//    and one tile later -- once all H * 2 CTAs have published that tile -- scales by the
-//    token's rsqrt(mean(y^2) + eps), the norm weight and sigmoid(g), and stores bf16 O
-//    with TMA.  The last CTA to publish a tile reduces the partial sums (fixed order).
+//  * The epilogue warpgroup reads O once: it adds each row's sum of squares into an fp64
+//    per-token accumulator in global memory (red.add; the fp64 sum of the fp32 partials is
+//    exact whenever a token's partials span less than 2^22, so the result does not depend
+//    on the order the additions land in), bumps the tile's arrival counter, and parks
+//    z = y * w * sigmoid(g) as bf16 in place of the gate tile.  Two tiles later, once all
+//    H * 2 CTAs have arrived for that tile, it scales z by rsqrt(mean(y^2) + eps) and
+//    stores the bf16 output with TMA.  The TMEM accumulator is free right after the read.
 //  * Every wait is bounded (globaltimer); a wait that runs out records LA_ERR_TIMEOUT in
 //    the workspace and the CTA drains its async work, frees TMEM and exits.
 #include <cudaTypedefs.h>
@@ -48,6 +52,10 @@ constexpr int kDV = 64;          // d_v slice per CTA
 constexpr int kNdv = kD / kDV;   // CTAs per head
 constexpr int kTile = 128;       // rows per tile (MMA M)
 constexpr int kThreads = 512;
+constexpr int kXfWarp0 = 2;      // transform warps 2..7
+constexpr int kXfThreads = 192;
+constexpr int kNG = 3;           // gate / output staging slots
+constexpr int kLag = 2;          // tiles between reading O and storing the normalised output
 
 constexpr uint32_t kQBytes = kTile * kD * 2;     // 32 KiB (two 64-column swizzled boxes)
 constexpr uint32_t kKBytes = kQBytes;
@@ -60,25 +68,26 @@ constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + 2 * kQBytes;
 constexpr uint32_t OFF_V = OFF_K + 2 * kKBytes;
 constexpr uint32_t OFF_G = OFF_V + 2 * kVBytes;
-constexpr uint32_t OFF_SNAP = OFF_G + 2 * kGBytes;
+constexpr uint32_t OFF_SNAP = OFF_G + kNG * kGBytes;
 constexpr uint32_t OFF_BARS = OFF_SNAP + kSnapBytes;
 
 // TMEM columns (512 allocated; 128 lanes each)
 constexpr uint32_t TM_S = 0;      // fp32 state slice, 64 columns
-constexpr uint32_t TM_O = 64;     // 3 output accumulators x 64 columns
+constexpr uint32_t TM_O = 64;     // 2 output accumulators x 64 columns
 constexpr uint32_t TM_P = 256;    // 2 score tiles x 128 columns
 constexpr uint32_t kTmemCols = 512;
 
 struct Bars {
-  uint64_t full_qkv[2], xformed[2], empty[2], full_g[2], empty_g[2];
+  uint64_t full_qkv[2], xformed[2], empty[2];
+  uint64_t full_g[kNG], empty_g[kNG];
   uint64_t p_full, p_conv, pv_done;
-  uint64_t o_full[3], o_empty[3];
+  uint64_t o_full[2], o_empty[2];
   uint64_t s_done, snap_ready, final_bar;
   uint64_t wg3_bar;      // epilogue warpgroup sync (bounded, unlike bar.sync)
   uint32_t tmem_base;
   int abort_flag;
-  int last_flag;
   int go_flag;
+  int pad;
   float w[kDV];
 };
 
@@ -94,9 +103,8 @@ struct TcParams {
   float eps;
   const float* w;
   ErrRec* err;
-  unsigned int* cnt;
-  float* part;
-  float* rnorm;
+  unsigned int* cnt;   // [nseq * max_tiles] arrivals per tile
+  double* ss;          // [tokens] sum of squares over the head concatenation
   uint16_t* out;
 };
 
@@ -185,6 +193,14 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
 }
+__device__ __forceinline__ double ld_cg_f64(const double* p) {
+  double v;
+  asm volatile("ld.global.cg.f64 %0, [%1];" : "=d"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_add_release_gpu(unsigned int* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 // ======================================================================================
 // The kernel
@@ -212,24 +228,24 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&B.full_qkv[i], 1);
-      mbar_init(&B.xformed[i], 128);
+      mbar_init(&B.xformed[i], kXfThreads);
       mbar_init(&B.empty[i], 1);
+      mbar_init(&B.o_full[i], 1);
+      mbar_init(&B.o_empty[i], 128);
+    }
+    for (int i = 0; i < kNG; ++i) {
       mbar_init(&B.full_g[i], 1);
       mbar_init(&B.empty_g[i], 1);
     }
     mbar_init(&B.p_full, 1);
     mbar_init(&B.p_conv, 128);
     mbar_init(&B.pv_done, 1);
-    for (int i = 0; i < 3; ++i) {
-      mbar_init(&B.o_full[i], 1);
-      mbar_init(&B.o_empty[i], 128);
-    }
     mbar_init(&B.s_done, 1);
     mbar_init(&B.snap_ready, 128);
     mbar_init(&B.final_bar, 1);
     mbar_init(&B.wg3_bar, 128);
     B.abort_flag = 0;
-    B.last_flag = 0;
+    B.go_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc<kTmemCols>(&B.tmem_base);
@@ -240,30 +256,18 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   const uint32_t tmem = B.tmem_base;
 
   // ------------------------------------------------------------------------------------
-  // Warp 0: TMA producer
+  // Warp 0: TMA producers.  Lane 0 streams Q/K/V tiles into the two-slot ring; lane 1
+  // streams gate tiles into the three-slot staging ring, running ahead on its own.
   // ------------------------------------------------------------------------------------
   if (warp == 0) {
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      if (gate) prefetch_tmap(&tm_g);
       const uint64_t pol = policy_evict_first();
-      uint32_t uses[2] = {0, 0}, guses[2] = {0, 0};
+      uint32_t uses[2] = {0, 0};
       int t = 0;
-      bool have_prev = false;
-      int prev_t = 0;
-      int64_t prev_row = 0;
       bool ok = true;
-      auto load_g = [&](int tt, int64_t row) -> bool {
-        const int gs = tt & 1;
-        if (guses[gs] > 0 && !wait_bar(&B.empty_g[gs], (guses[gs] - 1) & 1, B, p, SITE_TC_PRODUCER, tt)) return false;
-        mbar_arrive_expect_tx(&B.full_g[gs], kGBytes);
-        tma_load_2d(smem + OFF_G + gs * kGBytes, &tm_g, h * kD + dvt * kDV, static_cast<int32_t>(row), &B.full_g[gs],
-                    pol);
-        guses[gs]++;
-        return true;
-      };
       for (int s = 0; s < p.nseq && ok; ++s) {
         int64_t row0;
         int L;
@@ -285,24 +289,38 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           tma_load_2d(k + kBoxBytes, &tm_k, h * kD + 64, row, &B.full_qkv[slot], pol);
           tma_load_2d(smem + OFF_V + slot * kVBytes, &tm_v, h * kD + dvt * kDV, row, &B.full_qkv[slot], pol);
           uses[slot]++;
-          if (gate) {
-            if (have_prev && !load_g(prev_t, prev_row)) {
-              ok = false;
-              break;
-            }
-            have_prev = true;
-            prev_t = t;
-            prev_row = row;
-          }
           ++t;
         }
       }
-      if (ok && gate && have_prev) load_g(prev_t, prev_row);
       // Drain: every issued load must have landed before the CTA may exit.
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < 2; ++i)
         if (uses[i] > 0) drain_bar(&B.full_qkv[i], (uses[i] - 1) & 1);
-        if (guses[i] > 0) drain_bar(&B.full_g[i], (guses[i] - 1) & 1);
+    } else if (lane == 1 && gate) {
+      prefetch_tmap(&tm_g);
+      const uint64_t pol = policy_evict_first();
+      uint32_t guses[kNG] = {0, 0, 0};
+      int t = 0;
+      bool ok = true;
+      for (int s = 0; s < p.nseq && ok; ++s) {
+        int64_t row0;
+        int L;
+        seq_range(p, s, row0, L);
+        const int nt = (L + kTile - 1) / kTile;
+        for (int i = 0; i < nt; ++i) {
+          const int gs = t % kNG;
+          if (guses[gs] > 0 && !wait_bar(&B.empty_g[gs], (guses[gs] - 1) & 1, B, p, SITE_TC_PRODUCER, t)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&B.full_g[gs], kGBytes);
+          tma_load_2d(smem + OFF_G + gs * kGBytes, &tm_g, h * kD + dvt * kDV,
+                      static_cast<int32_t>(row0 + static_cast<int64_t>(i) * kTile), &B.full_g[gs], pol);
+          guses[gs]++;
+          ++t;
+        }
       }
+      for (int i = 0; i < kNG; ++i)
+        if (guses[i] > 0) drain_bar(&B.full_g[i], (guses[i] - 1) & 1);
     }
   }
   // ------------------------------------------------------------------------------------
@@ -322,7 +340,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         for (int i = 0; i < nt; ++i) {
           const int u = i % tpb;
           const int slot = (tpb == 2) ? (i & 1) : (t & 1);
-          const int ob = t % 3;
+          const int ob = t & 1;
           const int vr = min(kTile, L - i * kTile);
           const int nk = pad_rows(vr);
           if (!wait_bar(&B.xformed[slot], uses[slot] & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
@@ -345,32 +363,35 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             }
           }
           mma_commit(&B.p_full);
-          // O = phi(Q_i) S_snap
+          // O = P_bf16 V  (the accumulator is free once the epilogue read tile t - 2)
+          if (t >= 2) {
+            if (!wait_bar(&B.o_empty[ob], ((t >> 1) - 1) & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
+            tc_fence_after();
+          }
+          const uint32_t od = tmem + TM_O + kDV * ob;
+          if (!wait_bar(&B.p_conv, t & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t acc = 0;
+          for (int kt = 0; kt <= u; ++kt) {
+            const int kslot = (tpb == 2) ? kt : slot;
+            const int kext = (kt == u) ? nk : 128;
+            const uint32_t vb = sbase + OFF_V + kslot * kVBytes;
+            for (int k = 0; k < kext / 16; ++k) {
+              mma_ts(od, tmem + TM_P + 128 * kt + 8 * k, make_sdesc(vb + k * 2048, kBoxBytes, 1024), kIdescPV, acc);
+              acc = 1;
+            }
+          }
+          // O += phi(Q_i) S_snap
           if (u == 0) {
             if (!wait_bar(&B.snap_ready, snap_waits & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
             snap_waits++;
             tc_fence_after();
           }
-          if (t >= 3) {
-            if (!wait_bar(&B.o_empty[ob], ((t / 3) - 1) & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
-            tc_fence_after();
-          }
-          const uint32_t od = tmem + TM_O + kDV * ob;
           const uint32_t snap = sbase + OFF_SNAP;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
-            mma_ss(od, make_sdesc(qa + off, 16, 1024), make_sdesc(snap + k * 2048, kBoxBytes, 1024), kIdescQS, k > 0);
-          }
-          // O += P_bf16 V
-          if (!wait_bar(&B.p_conv, t & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
-          tc_fence_after();
-          for (int kt = 0; kt <= u; ++kt) {
-            const int kslot = (tpb == 2) ? kt : slot;
-            const int kext = (kt == u) ? nk : 128;
-            const uint32_t vb = sbase + OFF_V + kslot * kVBytes;
-            for (int k = 0; k < kext / 16; ++k)
-              mma_ts(od, tmem + TM_P + 128 * kt + 8 * k, make_sdesc(vb + k * 2048, kBoxBytes, 1024), kIdescPV, 1);
+            mma_ss(od, make_sdesc(qa + off, 16, 1024), make_sdesc(snap + k * 2048, kBoxBytes, 1024), kIdescQS, 1);
           }
           mma_commit(&B.o_full[ob]);
           mma_commit(&B.pv_done);
@@ -399,10 +420,10 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     }
   }
   // ------------------------------------------------------------------------------------
-  // Warps 4-7: SiLU transform of Q and K in shared memory; zero tail rows of K and V
+  // Warps 2-7: SiLU transform of Q and K in shared memory; zero tail rows of K and V
   // ------------------------------------------------------------------------------------
-  else if (warp >= 4 && warp < 8) {
-    const int wt = tid - 128;
+  else if (warp >= kXfWarp0 && warp < kXfWarp0 + kXfThreads / 32) {
+    const int wt = tid - 32 * kXfWarp0;
     uint32_t uses[2] = {0, 0};
     int t = 0;
     bool ok = true;
@@ -418,28 +439,28 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         const int vr = min(kTile, L - i * kTile);
         const uint32_t qa = sbase + OFF_Q + slot * kQBytes;
         const uint32_t ka = sbase + OFF_K + slot * kKBytes;
-#pragma unroll 4
-        for (int m = 0; m < 16; ++m) {
-          const uint32_t off = static_cast<uint32_t>(wt + 128 * m) * 16u;
+        // Chunks 0..2047 are Q, 2048..4095 are K (16 bytes = 8 bf16 each).
+        constexpr int kChunks = 2 * (kQBytes / 16);
+#pragma unroll 2
+        for (int c = wt; c < kChunks; c += kXfThreads) {
+          const bool is_k = c >= kChunks / 2;
+          const uint32_t off = static_cast<uint32_t>(is_k ? c - kChunks / 2 : c) * 16u;
+          const uint32_t addr = (is_k ? ka : qa) + off;
           const int row = static_cast<int>((off & (kBoxBytes - 1)) >> 7);
-          uint4 kv = lds128(ka + off);
-          if (row >= vr) {
-            kv = make_uint4(0, 0, 0, 0);
+          uint4 v = lds128(addr);
+          if (is_k && row >= vr) {
+            v = make_uint4(0, 0, 0, 0);
           } else if (!p.phi_identity) {
-            kv.x = silu_bf16x2(kv.x); kv.y = silu_bf16x2(kv.y); kv.z = silu_bf16x2(kv.z); kv.w = silu_bf16x2(kv.w);
+            v.x = silu_bf16x2(v.x); v.y = silu_bf16x2(v.y); v.z = silu_bf16x2(v.z); v.w = silu_bf16x2(v.w);
+          } else if (!is_k) {
+            continue;  // identity feature map: Q stays as loaded
           }
-          sts128(ka + off, kv);
-          if (!p.phi_identity) {
-            uint4 qv = lds128(qa + off);
-            qv.x = silu_bf16x2(qv.x); qv.y = silu_bf16x2(qv.y); qv.z = silu_bf16x2(qv.z); qv.w = silu_bf16x2(qv.w);
-            sts128(qa + off, qv);
-          }
+          sts128(addr, v);
         }
         if (vr < kTile) {
           const uint32_t va = sbase + OFF_V + slot * kVBytes;
-#pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const uint32_t off = static_cast<uint32_t>(wt + 128 * m) * 16u;
+          for (int c = wt; c < static_cast<int>(kVBytes / 16); c += kXfThreads) {
+            const uint32_t off = static_cast<uint32_t>(c) * 16u;
             if (static_cast<int>(off >> 7) >= vr) sts128(va + off, make_uint4(0, 0, 0, 0));
           }
         }
@@ -576,13 +597,14 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     }
   }
   // ------------------------------------------------------------------------------------
-  // Warps 12-15: epilogue (sum of squares, cross-head norm exchange, gate, store)
+  // Warps 12-15: epilogue
   // ------------------------------------------------------------------------------------
   else if (warp >= 12) {
     const int wt = tid - 384;                      // TMEM lane = row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(wt & ~31) << 16;
     const int HD = p.H * kD;
-    uint32_t guses[2] = {0, 0};
+    const float inv_hd = 1.0f / static_cast<float>(HD);
+    uint32_t guses[kNG] = {0, 0, 0};
     uint32_t sph = 0;                              // phase of the warpgroup barrier
     bool ok = true;
 
@@ -590,79 +612,51 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       int t, s, i, vr;
       int64_t row;
     };
-    Pend pend{};
-    bool have_pend = false;
+    Pend pend[kLag];
+    int npend = 0;
 
-    // Scale, gate and store one tile whose O is still in TMEM.
+    // Scale the parked z tile by the token's norm factor and store it.
     auto finalize = [&](const Pend& q) -> bool {
-      const int ob = q.t % 3;
-      const int gs = q.t & 1;
-      const int64_t grow = q.row + wt;
+      const int gs = q.t % kNG;
       const uint32_t tix = static_cast<uint32_t>(q.t);
-      float rn = 1.0f;
+      const uint32_t stg = sbase + OFF_G + gs * kGBytes;
       if (norm) {
         unsigned int* c = p.cnt + static_cast<int64_t>(q.s) * p.max_tiles + q.i;
         if (wt == 0) {
           int go = 1;
-          const uint64_t t0 = globaltimer_ns();
-          const uint64_t lim = wait_limit_ns(p.err);
-          while (ld_acquire_gpu(c) < static_cast<uint32_t>(W + 1)) {
-            if (aborted(B)) { go = 0; break; }
-            if (globaltimer_ns() - t0 > lim) {
-              report(p.err, LA_ERR_TIMEOUT, SITE_TC_NORM_WAIT, static_cast<uint32_t>(q.s * p.max_tiles + q.i),
-                     ld_acquire_gpu(c));
-              *reinterpret_cast<volatile int*>(&B.abort_flag) = 1;
-              go = 0;
-              break;
+          if (ld_acquire_gpu(c) < static_cast<uint32_t>(W)) {
+            const uint64_t t0 = globaltimer_ns();
+            const uint64_t lim = wait_limit_ns(p.err);
+            while (ld_acquire_gpu(c) < static_cast<uint32_t>(W)) {
+              if (aborted(B)) { go = 0; break; }
+              if (globaltimer_ns() - t0 > lim) {
+                report(p.err, LA_ERR_TIMEOUT, SITE_TC_NORM_WAIT, static_cast<uint32_t>(q.s * p.max_tiles + q.i),
+                       ld_acquire_gpu(c));
+                *reinterpret_cast<volatile int*>(&B.abort_flag) = 1;
+                go = 0;
+                break;
+              }
             }
-            __nanosleep(64);
           }
           B.go_flag = go;
         }
         if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix)) return false;
         if (!__all_sync(0xFFFFFFFFu, B.go_flag != 0)) return false;
         (void)ld_acquire_gpu(c);
-        if (wt < q.vr) rn = __ldcg(p.rnorm + grow);
-      }
-      if (gate) {
-        if (!wait_bar_warp(&B.full_g[gs], guses[gs] & 1, B, p, SITE_TC_EPILOGUE, tix)) return false;
-        guses[gs]++;
-      }
-      const uint32_t stg = sbase + OFF_G + gs * kGBytes;
-      const uint32_t obase = tmem + lane_off + TM_O + kDV * ob;
+        const float rn = (wt < q.vr) ? 1.0f / sqrtf(static_cast<float>(ld_cg_f64(p.ss + q.row + wt)) * inv_hd + p.eps)
+                                     : 0.0f;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t x[32];
-        tmem_ld32(obase + 32 * half, x);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int chunk = 4 * half + c;
+        for (int chunk = 0; chunk < 8; ++chunk) {
           const uint32_t addr = stg + sw128_offset(wt, chunk);
-          uint4 gv = make_uint4(0, 0, 0, 0);
-          if (gate) gv = lds128(addr);
-          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+          const uint4 zv = lds128(addr);
+          const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
           uint32_t ow[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = 8 * chunk + 2 * e;
-            float a = __uint_as_float(x[8 * c + 2 * e]) * rn;
-            float b = __uint_as_float(x[8 * c + 2 * e + 1]) * rn;
-            if (norm) {
-              a *= B.w[col];
-              b *= B.w[col + 1];
-            }
-            if (gate) {
-              a *= sigmoid_fast(__uint_as_float(gw[e] << 16));
-              b *= sigmoid_fast(__uint_as_float(gw[e] & 0xFFFF0000u));
-            }
-            ow[e] = pack_bf16x2(a, b);
-          }
+          for (int e = 0; e < 4; ++e)
+            ow[e] = pack_bf16x2(__uint_as_float(zw[e] << 16) * rn, __uint_as_float(zw[e] & 0xFFFF0000u) * rn);
           sts128(addr, make_uint4(ow[0], ow[1], ow[2], ow[3]));
         }
       }
-      tc_fence_before();
-      mbar_arrive(&B.o_empty[ob]);
       fence_proxy_async_smem();
       if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix)) return false;
       if (q.vr == kTile) {
@@ -674,14 +668,14 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         }
       } else {
         if (wt < q.vr) {
-          uint16_t* dst = p.out + grow * HD + h * kD + dvt * kDV;
+          uint16_t* dst = p.out + (q.row + wt) * HD + h * kD + dvt * kDV;
 #pragma unroll
           for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + 8 * c) = lds128(stg + sw128_offset(wt, c));
         }
         if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix)) return false;
         if (wt == 0 && gate) mbar_arrive(&B.empty_g[gs]);
       }
-      // The staging buffer is free again once thread 0 has seen the store read it.
+      // The staging slot is free again once thread 0 has seen the store read it.
       return wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix);
     };
 
@@ -692,60 +686,76 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       seq_range(p, s, row0, L);
       const int nt = (L + kTile - 1) / kTile;
       for (int i = 0; i < nt; ++i) {
-        const int ob = t % 3;
+        const int ob = t & 1;
+        const int gs = t % kNG;
         const int vr = min(kTile, L - i * kTile);
         const int64_t row = row0 + static_cast<int64_t>(i) * kTile;
-        if (!wait_bar_warp(&B.o_full[ob], (t / 3) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+        const uint32_t stg = sbase + OFF_G + gs * kGBytes;
+        if (!wait_bar_warp(&B.o_full[ob], (t >> 1) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+        if (gate) {
+          if (!wait_bar_warp(&B.full_g[gs], guses[gs] & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+          guses[gs]++;
+        }
         tc_fence_after();
+        // Read O once: sum of squares of the row, and z = y * w * sigmoid(g) parked as bf16.
+        float ss = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t x[32];
+          tmem_ld32(tmem + lane_off + TM_O + kDV * ob + 32 * half, x);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int chunk = 4 * half + c;
+            const uint32_t addr = stg + sw128_offset(wt, chunk);
+            uint4 gv = make_uint4(0, 0, 0, 0);
+            if (gate) gv = lds128(addr);
+            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t zw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int col = 8 * chunk + 2 * e;
+              float a = __uint_as_float(x[8 * c + 2 * e]);
+              float b = __uint_as_float(x[8 * c + 2 * e + 1]);
+              ss = fmaf(a, a, ss);
+              ss = fmaf(b, b, ss);
+              if (norm) {
+                a *= B.w[col];
+                b *= B.w[col + 1];
+              }
+              if (gate) {
+                a *= sigmoid_fast(__uint_as_float(gw[e] << 16));
+                b *= sigmoid_fast(__uint_as_float(gw[e] & 0xFFFF0000u));
+              }
+              zw[e] = pack_bf16x2(a, b);
+            }
+            sts128(addr, make_uint4(zw[0], zw[1], zw[2], zw[3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&B.o_empty[ob]);
         Pend cur{t, s, i, vr, row};
         if (norm) {
-          // Sum of squares of this row's 64 outputs (fixed order).
-          float ss = 0.f;
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t x[32];
-            tmem_ld32(tmem + lane_off + TM_O + kDV * ob + 32 * half, x);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(x[e]), __uint_as_float(x[e]), ss);
-          }
-          const int64_t grow = row + wt;
-          if (wt < vr) p.part[grow * W + h * kNdv + dvt] = ss;
+          if (wt < vr) atomicAdd(p.ss + row + wt, static_cast<double>(ss));
           __threadfence();
           if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
-          unsigned int* c = p.cnt + static_cast<int64_t>(s) * p.max_tiles + i;
           if (wt == 0) {
             const bool skip = (p.err->inject == INJECT_SKIP_PUBLISH) && blockIdx.x == 0;
-            B.last_flag = skip ? 0 : (atom_add_acq_rel_gpu(c, 1u) == static_cast<uint32_t>(W - 1));
+            if (!skip) red_add_release_gpu(p.cnt + static_cast<int64_t>(s) * p.max_tiles + i, 1u);
           }
-          if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
-          if (B.last_flag) {
-            // Last CTA of this tile: reduce the W partial sums of every token in order.
-            __threadfence();
-            if (wt < vr) {
-              const float2* src = reinterpret_cast<const float2*>(p.part + grow * W);
-              float acc = 0.f;
-              for (int j = 0; j < W / 2; ++j) {
-                const float2 v = __ldcg(src + j);
-                acc += v.x;
-                acc += v.y;
-              }
-              p.rnorm[grow] = 1.0f / sqrtf(acc / static_cast<float>(HD) + p.eps);
-            }
-            __threadfence();
-            if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
-            if (wt == 0) atom_add_acq_rel_gpu(c, 1u);
+          if (npend == kLag) {
+            if (!finalize(pend[0])) { ok = false; break; }
+            for (int j = 0; j + 1 < kLag; ++j) pend[j] = pend[j + 1];
+            npend--;
           }
-          if (have_pend && !finalize(pend)) { ok = false; break; }
-          pend = cur;
-          have_pend = true;
+          pend[npend++] = cur;
         } else {
           if (!finalize(cur)) { ok = false; break; }
         }
         ++t;
       }
     }
-    if (ok && have_pend) finalize(pend);
+    for (int j = 0; ok && j < npend; ++j) ok = finalize(pend[j]);
     if (wt == 0) bulk_wait0();
   }
 
@@ -800,16 +810,17 @@ bool tc_eligible(const TcShape& s, int num_sms) {
 size_t tc_workspace_bytes(int nseq, int max_len, int64_t tokens, int H, int D, int C) {
   (void)D;
   (void)C;
+  (void)H;
   const size_t max_tiles = (static_cast<size_t>(max_len) + kTile - 1) / kTile;
   return up256(sizeof(unsigned int) * static_cast<size_t>(nseq) * (max_tiles ? max_tiles : 1)) +
-         up256(sizeof(float) * static_cast<size_t>(tokens) * H * kNdv) + up256(sizeof(float) * static_cast<size_t>(tokens));
+         up256(sizeof(double) * static_cast<size_t>(tokens > 0 ? tokens : 1));
 }
 
 cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream) {
   (void)num_sms;
   const int max_tiles = (a.max_len + kTile - 1) / kTile;
   const size_t cnt_bytes = up256(sizeof(unsigned int) * static_cast<size_t>(a.nseq) * (max_tiles ? max_tiles : 1));
-  const size_t part_bytes = up256(sizeof(float) * static_cast<size_t>(a.tokens) * a.H * kNdv);
+  const size_t ss_bytes = up256(sizeof(double) * static_cast<size_t>(a.tokens > 0 ? a.tokens : 1));
   TcParams p{};
   p.state_in = a.state_in;
   p.state_out = a.state_out;
@@ -826,8 +837,7 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
   p.w = a.w;
   p.err = a.err;
   p.cnt = reinterpret_cast<unsigned int*>(a.ws);
-  p.part = reinterpret_cast<float*>(a.ws + cnt_bytes);
-  p.rnorm = reinterpret_cast<float*>(a.ws + cnt_bytes + part_bytes);
+  p.ss = reinterpret_cast<double*>(a.ws + cnt_bytes);
   p.out = static_cast<uint16_t*>(a.out);
 
   const int64_t cols = static_cast<int64_t>(a.H) * kD;
@@ -840,7 +850,8 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
   } else {
     mg = mq;  // never read
   }
-  cudaError_t e = cudaMemsetAsync(a.ws, 0, cnt_bytes, stream);
+  // Arrival counters and the fp64 sums start at zero on every call.
+  cudaError_t e = cudaMemsetAsync(a.ws, 0, cnt_bytes + (a.mode != LA_OUT_RAW ? ss_bytes : 0), stream);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(lightning_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kSmemBytes));
