@@ -51,11 +51,12 @@ constexpr int kD = 128;          // head dim (d_k = d_v)
 constexpr int kDV = 64;          // d_v slice per CTA
 constexpr int kNdv = kD / kDV;   // CTAs per head
 constexpr int kTile = 128;       // rows per tile (MMA M)
-constexpr int kThreads = 512;
+constexpr int kThreads = 576;  // 18 warps
 constexpr int kXfWarp0 = 2;      // transform warps 2..7
 constexpr int kXfThreads = 192;
 constexpr int kNG = 3;           // gate / output staging slots
-constexpr int kLag = 2;          // tiles between reading O and storing the normalised output
+constexpr int kReadWarp0 = 12;   // epilogue readers: warps 12..15
+constexpr int kStoreWarp0 = 16;  // epilogue storers: warps 16..17 (alternate tiles)
 
 constexpr uint32_t kQBytes = kTile * kD * 2;     // 32 KiB (two 64-column swizzled boxes)
 constexpr uint32_t kKBytes = kQBytes;
@@ -83,11 +84,9 @@ struct Bars {
   uint64_t p_full, p_conv, pv_done;
   uint64_t o_full[2], o_empty[2];
   uint64_t s_done, snap_ready, final_bar;
-  uint64_t wg3_bar;      // epilogue warpgroup sync (bounded, unlike bar.sync)
+  uint64_t z_ready[kNG], stg_free[kNG];
   uint32_t tmem_base;
   int abort_flag;
-  int go_flag;
-  int pad;
   float w[kDV];
 };
 
@@ -169,19 +168,15 @@ __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, Ba
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
-// Bounded barrier of a 128-thread warpgroup on an mbarrier (count 128).  A lane that has
-// left never hangs the others: they give up when the CTA aborts or the limit runs out.
-__device__ __forceinline__ bool wg_sync(uint64_t* bar, uint32_t& phase, Bars& B, const TcParams& p, uint32_t site,
-                                        uint32_t index) {
-  mbar_arrive(bar);
-  const bool ok = wait_bar_warp(bar, phase, B, p, site, index);
-  phase ^= 1u;
-  return ok;
-}
-
+// SiLU of two packed bf16 values in packed bf16 arithmetic, from sigmoid(x) =
+// (1 + tanh(x/2)) / 2:  h = x/2 (exact), t = tanh(h) (one MUFU op for both halves),
+// SiLU(x) = h + h t (one fused multiply-add, rounded once to bf16).
 __device__ __forceinline__ uint32_t silu_bf16x2(uint32_t x) {
-  const float lo = __uint_as_float(x << 16), hi = __uint_as_float(x & 0xFFFF0000u);
-  return pack_bf16x2(silu_fast(lo), silu_fast(hi));
+  uint32_t h, t, r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(h) : "r"(x), "r"(0x3F003F00u));
+  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(h));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(h), "r"(t), "r"(h));
+  return r;
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -200,6 +195,9 @@ __device__ __forceinline__ double ld_cg_f64(const double* p) {
 }
 __device__ __forceinline__ void red_add_release_gpu(unsigned int* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_f64(double* p, double v) {
+  asm volatile("red.relaxed.gpu.global.add.f64 [%0], %1;" ::"l"(p), "d"(v) : "memory");
 }
 
 // ======================================================================================
@@ -223,7 +221,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   const int tpb = p.C / kTile;           // tiles per block (1 or 2)
   const bool norm = p.mode != LA_OUT_RAW;
   const bool gate = p.mode == LA_OUT_RMSNORM_GATE;
-  const int W = p.H * kNdv;              // CTAs contributing to one token's norm
+  const int W = p.H * kNdv * 4;          // reader warps contributing to one tile's norm
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -243,13 +241,16 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     mbar_init(&B.s_done, 1);
     mbar_init(&B.snap_ready, 128);
     mbar_init(&B.final_bar, 1);
-    mbar_init(&B.wg3_bar, 128);
+    for (int i = 0; i < kNG; ++i) {
+      mbar_init(&B.z_ready[i], 128);
+      mbar_init(&B.stg_free[i], 1);
+    }
     B.abort_flag = 0;
-    B.go_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc<kTmemCols>(&B.tmem_base);
-  if (tid >= 384 && tid < 384 + kDV) B.w[tid - 384] = p.w ? p.w[h * kD + dvt * kDV + (tid - 384)] : 1.0f;
+  if (tid >= 32 * kReadWarp0 && tid < 32 * kReadWarp0 + kDV)
+    B.w[tid - 32 * kReadWarp0] = p.w ? p.w[h * kD + dvt * kDV + (tid - 32 * kReadWarp0)] : 1.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -597,88 +598,14 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     }
   }
   // ------------------------------------------------------------------------------------
-  // Warps 12-15: epilogue
+  // Warps 12-15: epilogue readers.  Read O once, release the TMEM accumulator, add the
+  // rows' sums of squares into the fp64 per-token totals, park z = y * w * sigmoid(g).
   // ------------------------------------------------------------------------------------
-  else if (warp >= 12) {
-    const int wt = tid - 384;                      // TMEM lane = row of the tile
+  else if (warp >= kReadWarp0 && warp < kStoreWarp0) {
+    const int wt = tid - 32 * kReadWarp0;          // TMEM lane = row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(wt & ~31) << 16;
-    const int HD = p.H * kD;
-    const float inv_hd = 1.0f / static_cast<float>(HD);
-    uint32_t guses[kNG] = {0, 0, 0};
-    uint32_t sph = 0;                              // phase of the warpgroup barrier
+    const bool skip_publish = (p.err->inject == INJECT_SKIP_PUBLISH) && blockIdx.x == 0;
     bool ok = true;
-
-    struct Pend {
-      int t, s, i, vr;
-      int64_t row;
-    };
-    Pend pend[kLag];
-    int npend = 0;
-
-    // Scale the parked z tile by the token's norm factor and store it.
-    auto finalize = [&](const Pend& q) -> bool {
-      const int gs = q.t % kNG;
-      const uint32_t tix = static_cast<uint32_t>(q.t);
-      const uint32_t stg = sbase + OFF_G + gs * kGBytes;
-      if (norm) {
-        unsigned int* c = p.cnt + static_cast<int64_t>(q.s) * p.max_tiles + q.i;
-        if (wt == 0) {
-          int go = 1;
-          if (ld_acquire_gpu(c) < static_cast<uint32_t>(W)) {
-            const uint64_t t0 = globaltimer_ns();
-            const uint64_t lim = wait_limit_ns(p.err);
-            while (ld_acquire_gpu(c) < static_cast<uint32_t>(W)) {
-              if (aborted(B)) { go = 0; break; }
-              if (globaltimer_ns() - t0 > lim) {
-                report(p.err, LA_ERR_TIMEOUT, SITE_TC_NORM_WAIT, static_cast<uint32_t>(q.s * p.max_tiles + q.i),
-                       ld_acquire_gpu(c));
-                *reinterpret_cast<volatile int*>(&B.abort_flag) = 1;
-                go = 0;
-                break;
-              }
-            }
-          }
-          B.go_flag = go;
-        }
-        if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix)) return false;
-        if (!__all_sync(0xFFFFFFFFu, B.go_flag != 0)) return false;
-        (void)ld_acquire_gpu(c);
-        const float rn = (wt < q.vr) ? 1.0f / sqrtf(static_cast<float>(ld_cg_f64(p.ss + q.row + wt)) * inv_hd + p.eps)
-                                     : 0.0f;
-#pragma unroll
-        for (int chunk = 0; chunk < 8; ++chunk) {
-          const uint32_t addr = stg + sw128_offset(wt, chunk);
-          const uint4 zv = lds128(addr);
-          const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
-          uint32_t ow[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            ow[e] = pack_bf16x2(__uint_as_float(zw[e] << 16) * rn, __uint_as_float(zw[e] & 0xFFFF0000u) * rn);
-          sts128(addr, make_uint4(ow[0], ow[1], ow[2], ow[3]));
-        }
-      }
-      fence_proxy_async_smem();
-      if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix)) return false;
-      if (q.vr == kTile) {
-        if (wt == 0) {
-          tma_store_2d(&tm_o, smem + OFF_G + gs * kGBytes, h * kD + dvt * kDV, static_cast<int32_t>(q.row));
-          bulk_commit();
-          bulk_wait_read0();
-          if (gate) mbar_arrive(&B.empty_g[gs]);
-        }
-      } else {
-        if (wt < q.vr) {
-          uint16_t* dst = p.out + (q.row + wt) * HD + h * kD + dvt * kDV;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + 8 * c) = lds128(stg + sw128_offset(wt, c));
-        }
-        if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix)) return false;
-        if (wt == 0 && gate) mbar_arrive(&B.empty_g[gs]);
-      }
-      // The staging slot is free again once thread 0 has seen the store read it.
-      return wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, tix);
-    };
-
     int t = 0;
     for (int s = 0; s < p.nseq && ok; ++s) {
       int64_t row0;
@@ -693,11 +620,11 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         const uint32_t stg = sbase + OFF_G + gs * kGBytes;
         if (!wait_bar_warp(&B.o_full[ob], (t >> 1) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
         if (gate) {
-          if (!wait_bar_warp(&B.full_g[gs], guses[gs] & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
-          guses[gs]++;
+          if (!wait_bar_warp(&B.full_g[gs], (t / kNG) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+        } else if (t >= kNG) {
+          if (!wait_bar_warp(&B.stg_free[gs], ((t / kNG) - 1) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
         }
         tc_fence_after();
-        // Read O once: sum of squares of the row, and z = y * w * sigmoid(g) parked as bf16.
         float ss = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -734,29 +661,103 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         }
         tc_fence_before();
         mbar_arrive(&B.o_empty[ob]);
-        Pend cur{t, s, i, vr, row};
         if (norm) {
-          if (wt < vr) atomicAdd(p.ss + row + wt, static_cast<double>(ss));
-          __threadfence();
-          if (!wg_sync(&B.wg3_bar, sph, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
-          if (wt == 0) {
-            const bool skip = (p.err->inject == INJECT_SKIP_PUBLISH) && blockIdx.x == 0;
-            if (!skip) red_add_release_gpu(p.cnt + static_cast<int64_t>(s) * p.max_tiles + i, 1u);
-          }
-          if (npend == kLag) {
-            if (!finalize(pend[0])) { ok = false; break; }
-            for (int j = 0; j + 1 < kLag; ++j) pend[j] = pend[j + 1];
-            npend--;
-          }
-          pend[npend++] = cur;
-        } else {
-          if (!finalize(cur)) { ok = false; break; }
+          if (wt < vr) red_add_f64(p.ss + row + wt, static_cast<double>(ss));
+          __syncwarp();
+          // One release per warp orders the warp's additions before the arrival count.
+          if (lane == 0 && !skip_publish) red_add_release_gpu(p.cnt + static_cast<int64_t>(s) * p.max_tiles + i, 1u);
         }
+        mbar_arrive(&B.z_ready[gs]);
         ++t;
       }
     }
-    for (int j = 0; ok && j < npend; ++j) ok = finalize(pend[j]);
-    if (wt == 0) bulk_wait0();
+  }
+  // ------------------------------------------------------------------------------------
+  // Warps 16-17: epilogue storers, alternating tiles.  Wait until every reader warp of
+  // every CTA has added its sums for the tile, scale z by rsqrt(mean(y^2) + eps), store.
+  // ------------------------------------------------------------------------------------
+  else if (warp >= kStoreWarp0) {
+    const int sw = warp - kStoreWarp0;
+    const int HD = p.H * kD;
+    const float inv_hd = 1.0f / static_cast<float>(HD);
+    bool ok = true;
+    int t = 0;
+    for (int s = 0; s < p.nseq && ok; ++s) {
+      int64_t row0;
+      int L;
+      seq_range(p, s, row0, L);
+      const int nt = (L + kTile - 1) / kTile;
+      for (int i = 0; i < nt; ++i, ++t) {
+        if ((t & 1) != sw) continue;
+        const int gs = t % kNG;
+        const int vr = min(kTile, L - i * kTile);
+        const int64_t row = row0 + static_cast<int64_t>(i) * kTile;
+        const uint32_t stg = sbase + OFF_G + gs * kGBytes;
+        if (!wait_bar_warp(&B.z_ready[gs], (t / kNG) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+        if (norm) {
+          unsigned int* c = p.cnt + static_cast<int64_t>(s) * p.max_tiles + i;
+          int go = 1;
+          if (lane == 0 && ld_acquire_gpu(c) < static_cast<uint32_t>(W)) {
+            const uint64_t t0 = globaltimer_ns();
+            const uint64_t lim = wait_limit_ns(p.err);
+            while (ld_acquire_gpu(c) < static_cast<uint32_t>(W)) {
+              if (aborted(B)) { go = 0; break; }
+              if (globaltimer_ns() - t0 > lim) {
+                report(p.err, LA_ERR_TIMEOUT, SITE_TC_NORM_WAIT, static_cast<uint32_t>(s * p.max_tiles + i),
+                       ld_acquire_gpu(c));
+                *reinterpret_cast<volatile int*>(&B.abort_flag) = 1;
+                go = 0;
+                break;
+              }
+            }
+          }
+          if (!__shfl_sync(0xFFFFFFFFu, go, 0)) { ok = false; break; }
+          (void)ld_acquire_gpu(c);
+          float rn[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int r = lane + 32 * m;
+            rn[m] = (r < vr) ? 1.0f / sqrtf(static_cast<float>(ld_cg_f64(p.ss + row + r)) * inv_hd + p.eps) : 0.0f;
+          }
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int r = lane + 32 * m;
+#pragma unroll
+            for (int chunk = 0; chunk < 8; ++chunk) {
+              const uint32_t addr = stg + sw128_offset(r, chunk);
+              const uint4 zv = lds128(addr);
+              const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
+              uint32_t ow[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                ow[e] = pack_bf16x2(__uint_as_float(zw[e] << 16) * rn[m], __uint_as_float(zw[e] & 0xFFFF0000u) * rn[m]);
+              sts128(addr, make_uint4(ow[0], ow[1], ow[2], ow[3]));
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (vr == kTile) {
+          if (lane == 0) {
+            tma_store_2d(&tm_o, smem + OFF_G + gs * kGBytes, h * kD + dvt * kDV, static_cast<int32_t>(row));
+            bulk_commit();
+            bulk_wait_read0();
+          }
+        } else {
+          for (int m = 0; m < 4; ++m) {
+            const int r = lane + 32 * m;
+            if (r < vr) {
+              uint16_t* dst = p.out + (row + r) * HD + h * kD + dvt * kDV;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + 8 * c) = lds128(stg + sw128_offset(r, c));
+            }
+          }
+          __syncwarp();
+        }
+        if (lane == 0) mbar_arrive(gate ? &B.empty_g[gs] : &B.stg_free[gs]);
+      }
+    }
+    if (lane == 0) bulk_wait0();
   }
 
   // Teardown: all roles are done (or aborted with their async work drained).
