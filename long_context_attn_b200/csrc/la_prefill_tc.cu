@@ -14,8 +14,11 @@
 //  * Work is tiled in 128-row tiles (the tcgen05 M).  C = 256 is two tiles per block: the
 //    second tile multiplies by the first tile's keys densely and by its own keys under the
 //    causal mask; the all-zero upper-right quarter of the 256 x 256 block is never issued.
-//  * TMA loads Q, K (128 x 128) and V, G (128 x 64) tiles with the 128-byte swizzle into
-//    rings in shared memory; six transform warps apply SiLU in place (and zero tail rows).
+//  * The two CTAs of a head form a cluster.  Each loads (TMA, 128-byte swizzle) its own
+//    64-column box of the Q and K tiles plus its V and gate slices, applies SiLU to its
+//    boxes with six transform warps, and writes the result both into its own shared memory
+//    and into its partner's (distributed shared memory), so each SiLU is computed once per
+//    head and both CTAs end up with the full phi(Q), phi(K) tiles.
 //  * One thread issues all MMAs (bf16 in, fp32 accumulate in TMEM), per tile:
 //      P   = phi(Q) phi(K)^T          SS, M128 x N(<=128) x K128, into TMEM
 //      O   = P_bf16 V                 TS (P read back from TMEM), M128 x N64 x K(<=128)
@@ -23,9 +26,11 @@
 //      S  += phi(K)^T V               SS (both operands MN-major), M128 x N64 x K(<=128)
 //    The fp32 state S stays in TMEM for the whole sequence; the inter product comes last
 //    so the snapshot of S taken at the previous block end is ready by then.
-//  * A conversion warpgroup turns P (fp32, TMEM) into masked bf16 in place and, at each
-//    block end, copies S into the bf16 snapshot the next block's inter product reads.
-//  * The epilogue warpgroup reads O once: it adds each row's sum of squares into an fp64
+//    Score tiles alternate between two TMEM regions so that P of the next key/query tile
+//    is computed while the current one is being converted.
+//  * A conversion warpgroup turns P (fp32, TMEM) into masked bf16 in place.
+//  * The epilogue reader warpgroup owns the state (S0 in, the bf16 snapshot of S at each
+//    block end, the final state out) and reads O once: it adds each row's sum of squares into an fp64
 //    per-token accumulator in global memory (red.add; the fp64 sum of the fp32 partials is
 //    exact whenever a token's partials span less than 2^22, so the result does not depend
 //    on the order the additions land in), bumps the tile's arrival counter, and parks
@@ -81,7 +86,7 @@ constexpr uint32_t kTmemCols = 512;
 struct Bars {
   uint64_t full_qkv[2], xformed[2], empty[2];
   uint64_t full_g[kNG], empty_g[kNG];
-  uint64_t p_full, p_conv, pv_done;
+  uint64_t p_full[2], p_conv[2], pv_done[2];   // per TMEM score region
   uint64_t o_full[2], o_empty[2];
   uint64_t s_done, snap_ready, final_bar;
   uint64_t z_ready[kNG], stg_free[kNG];
@@ -128,6 +133,45 @@ __device__ __forceinline__ void seq_range(const TcParams& p, int s, int64_t& row
     row0 = static_cast<int64_t>(s) * p.T;
     L = p.T;
   }
+}
+
+// The (sequence, tile) order every role walks; empty sequences have no tiles.
+struct TileIter {
+  int s, i, nt, L;
+  int64_t row0;
+  bool valid;
+};
+__device__ __forceinline__ void tile_next(const TcParams& p, TileIter& it) {
+  if (it.valid && it.i + 1 < it.nt) {
+    ++it.i;
+    return;
+  }
+  for (int s = it.s + 1; s < p.nseq; ++s) {
+    int64_t r0;
+    int L;
+    seq_range(p, s, r0, L);
+    const int nt = (L + kTile - 1) / kTile;
+    if (nt > 0) {
+      it.s = s;
+      it.i = 0;
+      it.nt = nt;
+      it.L = L;
+      it.row0 = r0;
+      it.valid = true;
+      return;
+    }
+  }
+  it.s = p.nseq;
+  it.valid = false;
+}
+__device__ __forceinline__ void tile_first(const TcParams& p, TileIter& it) {
+  it.s = -1;
+  it.i = 0;
+  it.nt = 0;
+  it.L = 0;
+  it.row0 = 0;
+  it.valid = false;
+  tile_next(p, it);
 }
 
 __device__ __forceinline__ bool aborted(Bars& B) { return *reinterpret_cast<volatile int*>(&B.abort_flag) != 0; }
@@ -217,7 +261,8 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int h = blockIdx.x / kNdv;
-  const int dvt = blockIdx.x % kNdv;
+  const int dvt = static_cast<int>(cluster_ctarank());   // == blockIdx.x % 2 (cluster of 2)
+  const uint32_t partner = static_cast<uint32_t>(dvt ^ 1);
   const int tpb = p.C / kTile;           // tiles per block (1 or 2)
   const bool norm = p.mode != LA_OUT_RAW;
   const bool gate = p.mode == LA_OUT_RMSNORM_GATE;
@@ -226,8 +271,8 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&B.full_qkv[i], 1);
-      mbar_init(&B.xformed[i], kXfThreads);
-      mbar_init(&B.empty[i], 1);
+      mbar_init(&B.xformed[i], 2 * kXfThreads);   // both CTAs' transform threads
+      mbar_init(&B.empty[i], 2);                  // both CTAs' MMAs released the slot
       mbar_init(&B.o_full[i], 1);
       mbar_init(&B.o_empty[i], 128);
     }
@@ -235,9 +280,11 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       mbar_init(&B.full_g[i], 1);
       mbar_init(&B.empty_g[i], 1);
     }
-    mbar_init(&B.p_full, 1);
-    mbar_init(&B.p_conv, 128);
-    mbar_init(&B.pv_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&B.p_full[i], 1);
+      mbar_init(&B.p_conv[i], 128);
+      mbar_init(&B.pv_done[i], 1);
+    }
     mbar_init(&B.s_done, 1);
     mbar_init(&B.snap_ready, 128);
     mbar_init(&B.final_bar, 1);
@@ -253,6 +300,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     B.w[tid - 32 * kReadWarp0] = p.w ? p.w[h * kD + dvt * kDV + (tid - 32 * kReadWarp0)] : 1.0f;
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // the partner may arrive on these barriers from now on
   tc_fence_after();
   const uint32_t tmem = B.tmem_base;
 
@@ -281,13 +329,13 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             break;
           }
           const int32_t row = static_cast<int32_t>(row0 + static_cast<int64_t>(i) * kTile);
-          mbar_arrive_expect_tx(&B.full_qkv[slot], kQBytes + kKBytes + kVBytes);
-          uint8_t* q = smem + OFF_Q + slot * kQBytes;
-          uint8_t* k = smem + OFF_K + slot * kKBytes;
-          tma_load_2d(q, &tm_q, h * kD, row, &B.full_qkv[slot], pol);
-          tma_load_2d(q + kBoxBytes, &tm_q, h * kD + 64, row, &B.full_qkv[slot], pol);
-          tma_load_2d(k, &tm_k, h * kD, row, &B.full_qkv[slot], pol);
-          tma_load_2d(k + kBoxBytes, &tm_k, h * kD + 64, row, &B.full_qkv[slot], pol);
+          // This CTA's 64-column boxes of Q and K (the partner supplies the other box) and
+          // its V slice.
+          mbar_arrive_expect_tx(&B.full_qkv[slot], 2 * kBoxBytes + kVBytes);
+          uint8_t* q = smem + OFF_Q + slot * kQBytes + dvt * kBoxBytes;
+          uint8_t* k = smem + OFF_K + slot * kKBytes + dvt * kBoxBytes;
+          tma_load_2d(q, &tm_q, h * kD + dvt * 64, row, &B.full_qkv[slot], pol);
+          tma_load_2d(k, &tm_k, h * kD + dvt * 64, row, &B.full_qkv[slot], pol);
           tma_load_2d(smem + OFF_V + slot * kVBytes, &tm_v, h * kD + dvt * kDV, row, &B.full_qkv[slot], pol);
           uses[slot]++;
           ++t;
@@ -325,95 +373,147 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     }
   }
   // ------------------------------------------------------------------------------------
-  // Warp 1: MMA issuer (one thread)
+  // Warp 1: MMA issuer (one thread).  Score tiles ("jobs": one per query tile and key
+  // tile of its block) alternate between two TMEM regions; P of the next job is issued
+  // while the conversion warps still work on the current one, so the tensor core is not
+  // idle while scores are converted.
   // ------------------------------------------------------------------------------------
   else if (warp == 1) {
     if (lane == 0) {
-      uint32_t uses[2] = {0, 0};
+      uint32_t uses[2] = {0, 0};       // xformed phases consumed per slot
       uint32_t snap_waits = 0;
+      uint32_t k = 0;                  // next job to consume (PV)
+      uint32_t kp = 0;                 // next job whose P is issued
+      int xf_tile = -1;                // last tile whose transformed data was waited for
       int t = 0;
       bool ok = true;
-      for (int s = 0; s < p.nseq && ok; ++s) {
-        int64_t row0;
-        int L;
-        seq_range(p, s, row0, L);
-        const int nt = (L + kTile - 1) / kTile;
-        for (int i = 0; i < nt; ++i) {
-          const int u = i % tpb;
-          const int slot = (tpb == 2) ? (i & 1) : (t & 1);
-          const int ob = t & 1;
-          const int vr = min(kTile, L - i * kTile);
-          const int nk = pad_rows(vr);
-          if (!wait_bar(&B.xformed[slot], uses[slot] & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
-          uses[slot]++;
+      TileIter cur, nxt;
+      tile_first(p, cur);
+      nxt = cur;
+      tile_next(p, nxt);
+
+      auto slot_of = [&](const TileIter& it, int tt) { return (tpb == 2) ? (it.i & 1) : (tt & 1); };
+      // Wait (blocking) or test (non-blocking) for the transformed data of tile tt.
+      auto take_xf = [&](const TileIter& it, int tt, bool block) -> int {
+        if (xf_tile >= tt) return 1;
+        const int slot = slot_of(it, tt);
+        if (block) {
+          if (!wait_bar(&B.xformed[slot], uses[slot] & 1, B, p, SITE_TC_MMA, tt)) return -1;
+        } else if (!mbar_try_wait(&B.xformed[slot], uses[slot] & 1)) {
+          return 0;
+        }
+        uses[slot]++;
+        xf_tile = tt;
+        tc_fence_after();
+        return 1;
+      };
+      // P of job `job` = (tile it / tt, key tile kt) into region job & 1.
+      auto issue_p = [&](const TileIter& it, int tt, int kt, uint32_t job) -> bool {
+        const uint32_t r = job & 1u;
+        if (job >= 2) {
+          if (!wait_bar(&B.pv_done[r], ((job - 2) >> 1) & 1, B, p, SITE_TC_MMA, tt)) return false;
           tc_fence_after();
-          if (t > 0 && !wait_bar(&B.pv_done, (t - 1) & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t qa = sbase + OFF_Q + slot * kQBytes;
-          // P[kt] = phi(Q_i) phi(K_kt)^T
-          for (int kt = 0; kt <= u; ++kt) {
-            const int kslot = (tpb == 2) ? kt : slot;
-            const uint32_t n = (kt == u) ? static_cast<uint32_t>(nk) : 128u;
-            const uint32_t kb = sbase + OFF_K + kslot * kKBytes;
-            const uint32_t idesc = make_idesc_bf16(128, n, 0, 0);
+        }
+        const int u = it.i % tpb;
+        const int slot = slot_of(it, tt);
+        const int vr = min(kTile, it.L - it.i * kTile);
+        const int kslot = (tpb == 2) ? kt : slot;
+        const uint32_t n = (kt == u) ? static_cast<uint32_t>(pad_rows(vr)) : 128u;
+        const uint32_t qa = sbase + OFF_Q + slot * kQBytes;
+        const uint32_t kb = sbase + OFF_K + kslot * kKBytes;
+        const uint32_t idesc = make_idesc_bf16(128, n, 0, 0);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
-              mma_ss(tmem + TM_P + 128 * kt, make_sdesc(qa + off, 16, 1024), make_sdesc(kb + off, 16, 1024), idesc,
-                     k > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          mma_ss(tmem + TM_P + 128 * r, make_sdesc(qa + off, 16, 1024), make_sdesc(kb + off, 16, 1024), idesc,
+                 kk > 0);
+        }
+        mma_commit(&B.p_full[r]);
+        return true;
+      };
+
+      while (ok && cur.valid) {
+        const int u = cur.i % tpb;
+        const int slot = slot_of(cur, t);
+        const int ob = t & 1;
+        const int vr = min(kTile, cur.L - cur.i * kTile);
+        const int nk = pad_rows(vr);
+        const uint32_t k0 = k;
+        if (kp == k0) {  // P of this tile's first job was not issued ahead
+          if (take_xf(cur, t, true) < 0 || !issue_p(cur, t, 0, kp)) { ok = false; break; }
+          ++kp;
+        }
+        const uint32_t od = tmem + TM_O + kDV * ob;
+        for (int kt = 0; kt <= u && ok; ++kt) {
+          // Issue the next job's P ahead: the next key tile of this tile, or the first
+          // job of the next tile if its data is already transformed.
+          if (kp == k + 1) {
+            if (kt < u) {
+              if (!issue_p(cur, t, kt + 1, kp)) { ok = false; break; }
+              ++kp;
+            } else if (nxt.valid) {
+              const int got = take_xf(nxt, t + 1, false);
+              if (got > 0) {
+                if (!issue_p(nxt, t + 1, 0, kp)) { ok = false; break; }
+                ++kp;
+              }
             }
           }
-          mma_commit(&B.p_full);
-          // O = P_bf16 V  (the accumulator is free once the epilogue read tile t - 2)
-          if (t >= 2) {
+          if (kt == 0 && t >= 2) {
             if (!wait_bar(&B.o_empty[ob], ((t >> 1) - 1) & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
             tc_fence_after();
           }
-          const uint32_t od = tmem + TM_O + kDV * ob;
-          if (!wait_bar(&B.p_conv, t & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
+          const uint32_t r = k & 1u;
+          if (!wait_bar(&B.p_conv[r], (k >> 1) & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
           tc_fence_after();
-          uint32_t acc = 0;
-          for (int kt = 0; kt <= u; ++kt) {
-            const int kslot = (tpb == 2) ? kt : slot;
-            const int kext = (kt == u) ? nk : 128;
-            const uint32_t vb = sbase + OFF_V + kslot * kVBytes;
-            for (int k = 0; k < kext / 16; ++k) {
-              mma_ts(od, tmem + TM_P + 128 * kt + 8 * k, make_sdesc(vb + k * 2048, kBoxBytes, 1024), kIdescPV, acc);
-              acc = 1;
-            }
-          }
-          // O += phi(Q_i) S_snap
-          if (u == 0) {
-            if (!wait_bar(&B.snap_ready, snap_waits & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
-            snap_waits++;
-            tc_fence_after();
-          }
-          const uint32_t snap = sbase + OFF_SNAP;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
-            mma_ss(od, make_sdesc(qa + off, 16, 1024), make_sdesc(snap + k * 2048, kBoxBytes, 1024), kIdescQS, 1);
-          }
-          mma_commit(&B.o_full[ob]);
-          mma_commit(&B.pv_done);
-          // S += phi(K_i)^T V_i
-          {
-            const uint32_t kb = sbase + OFF_K + slot * kKBytes;
-            const uint32_t vb = sbase + OFF_V + slot * kVBytes;
-            for (int k = 0; k < nk / 16; ++k)
-              mma_ss(tmem + TM_S, make_sdesc(kb + k * 2048, kBoxBytes, 1024), make_sdesc(vb + k * 2048, kBoxBytes, 1024),
-                     kIdescDS, 1);
-          }
-          const bool blk_end = (u == tpb - 1) || (i == nt - 1);
-          if (tpb == 1) {
-            mma_commit(&B.empty[slot]);
-          } else if (blk_end) {
-            mma_commit(&B.empty[0]);
-            if (u == 1) mma_commit(&B.empty[1]);
-          }
-          if (blk_end) mma_commit(&B.s_done);
-          ++t;
+          // O (+)= P_bf16 V over this key tile
+          const int kslot = (tpb == 2) ? kt : slot;
+          const int kext = (kt == u) ? nk : 128;
+          const uint32_t vb = sbase + OFF_V + kslot * kVBytes;
+          for (int kk = 0; kk < kext / 16; ++kk)
+            mma_ts(od, tmem + TM_P + 128 * r + 8 * kk, make_sdesc(vb + kk * 2048, kBoxBytes, 1024), kIdescPV,
+                   (kt > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&B.pv_done[r]);
+          // The first tile's keys and values of a 256-block have no reader after this.
+          if (tpb == 2 && u == 1 && kt == 0) mma_commit_multicast(&B.empty[0], 0x3);
+          ++k;
         }
+        if (!ok) break;
+        // O += phi(Q) S_snap
+        if (u == 0) {
+          if (!wait_bar(&B.snap_ready, snap_waits & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
+          snap_waits++;
+          tc_fence_after();
+        }
+        const uint32_t qa = sbase + OFF_Q + slot * kQBytes;
+        const uint32_t snap = sbase + OFF_SNAP;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          mma_ss(od, make_sdesc(qa + off, 16, 1024), make_sdesc(snap + kk * 2048, kBoxBytes, 1024), kIdescQS, 1);
+        }
+        mma_commit(&B.o_full[ob]);
+        // S += phi(K)^T V
+        {
+          const uint32_t kb = sbase + OFF_K + slot * kKBytes;
+          const uint32_t vb = sbase + OFF_V + slot * kVBytes;
+          for (int kk = 0; kk < nk / 16; ++kk)
+            mma_ss(tmem + TM_S, make_sdesc(kb + kk * 2048, kBoxBytes, 1024), make_sdesc(vb + kk * 2048, kBoxBytes, 1024),
+                   kIdescDS, 1);
+        }
+        const bool blk_end = (u == tpb - 1) || (cur.i == cur.nt - 1);
+        // Slot release goes to both CTAs: the partner writes its transformed box here.
+        if (tpb == 1) {
+          mma_commit_multicast(&B.empty[slot], 0x3);
+        } else if (u == 1) {
+          mma_commit_multicast(&B.empty[1], 0x3);
+        } else if (blk_end) {
+          mma_commit_multicast(&B.empty[0], 0x3);  // a block of one tile (sequence tail)
+        }
+        if (blk_end) mma_commit(&B.s_done);
+        ++t;
+        cur = nxt;
+        tile_next(p, nxt);
       }
       // Drain: all MMAs complete before TMEM is released.
       mma_commit(&B.final_bar);
@@ -421,7 +521,8 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     }
   }
   // ------------------------------------------------------------------------------------
-  // Warps 2-7: SiLU transform of Q and K in shared memory; zero tail rows of K and V
+  // Warps 2-7: SiLU of this CTA's Q and K boxes, written to both CTAs of the pair; zero
+  // tail rows of K (both copies) and of this CTA's V slice.
   // ------------------------------------------------------------------------------------
   else if (warp >= kXfWarp0 && warp < kXfWarp0 + kXfThreads / 32) {
     const int wt = tid - 32 * kXfWarp0;
@@ -438,25 +539,24 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         if (!wait_bar_warp(&B.full_qkv[slot], uses[slot] & 1, B, p, SITE_TC_TRANSFORM, t)) { ok = false; break; }
         uses[slot]++;
         const int vr = min(kTile, L - i * kTile);
-        const uint32_t qa = sbase + OFF_Q + slot * kQBytes;
-        const uint32_t ka = sbase + OFF_K + slot * kKBytes;
-        // Chunks 0..2047 are Q, 2048..4095 are K (16 bytes = 8 bf16 each).
-        constexpr int kChunks = 2 * (kQBytes / 16);
+        const uint32_t qa = sbase + OFF_Q + slot * kQBytes + dvt * kBoxBytes;
+        const uint32_t ka = sbase + OFF_K + slot * kKBytes + dvt * kBoxBytes;
+        // Chunks 0..1023 are this CTA's Q box, 1024..2047 its K box (16 bytes = 8 bf16).
+        constexpr int kBoxChunks = kBoxBytes / 16;
 #pragma unroll 2
-        for (int c = wt; c < kChunks; c += kXfThreads) {
-          const bool is_k = c >= kChunks / 2;
-          const uint32_t off = static_cast<uint32_t>(is_k ? c - kChunks / 2 : c) * 16u;
+        for (int c = wt; c < 2 * kBoxChunks; c += kXfThreads) {
+          const bool is_k = c >= kBoxChunks;
+          const uint32_t off = static_cast<uint32_t>(is_k ? c - kBoxChunks : c) * 16u;
           const uint32_t addr = (is_k ? ka : qa) + off;
-          const int row = static_cast<int>((off & (kBoxBytes - 1)) >> 7);
+          const int row = static_cast<int>(off >> 7);
           uint4 v = lds128(addr);
           if (is_k && row >= vr) {
             v = make_uint4(0, 0, 0, 0);
           } else if (!p.phi_identity) {
             v.x = silu_bf16x2(v.x); v.y = silu_bf16x2(v.y); v.z = silu_bf16x2(v.z); v.w = silu_bf16x2(v.w);
-          } else if (!is_k) {
-            continue;  // identity feature map: Q stays as loaded
           }
           sts128(addr, v);
+          st_cluster128(mapa_shared(addr, partner), v);
         }
         if (vr < kTile) {
           const uint32_t va = sbase + OFF_V + slot * kVBytes;
@@ -465,22 +565,76 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             if (static_cast<int>(off >> 7) >= vr) sts128(va + off, make_uint4(0, 0, 0, 0));
           }
         }
-        fence_proxy_async_smem();
+        // Local and remote writes become visible to both tensor cores before the arrivals.
+        fence_proxy_async_cluster();
         mbar_arrive(&B.xformed[slot]);
+        mbar_arrive_cluster(mapa_shared(smem_u32(&B.xformed[slot]), partner));
         ++t;
       }
     }
   }
   // ------------------------------------------------------------------------------------
-  // Warps 8-11: P conversion (fp32 -> masked bf16, in TMEM) and the state snapshot
+  // Warps 8-11: score conversion (fp32 -> masked bf16, in place in TMEM), job by job.
   // ------------------------------------------------------------------------------------
   else if (warp >= 8 && warp < 12) {
     const int wt = tid - 256;                      // TMEM lane = row
     const uint32_t lane_off = static_cast<uint32_t>(wt & ~31) << 16;
+    uint32_t k = 0;
+    bool ok = true;
+    for (int s = 0; s < p.nseq && ok; ++s) {
+      int64_t row0;
+      int L;
+      seq_range(p, s, row0, L);
+      const int nt = (L + kTile - 1) / kTile;
+      for (int i = 0; i < nt && ok; ++i) {
+        const int u = i % tpb;
+        const int vr = min(kTile, L - i * kTile);
+        const int nk = pad_rows(vr);
+        for (int kt = 0; kt <= u; ++kt, ++k) {
+          const uint32_t r = k & 1u;
+          if (!wait_bar_warp(&B.p_full[r], (k >> 1) & 1, B, p, SITE_TC_CONVERT, k)) { ok = false; break; }
+          tc_fence_after();
+          const bool diag = (kt == u);
+          const int ncols = diag ? nk : 128;
+          const uint32_t base = tmem + lane_off + TM_P + 128 * r;
+          for (int c = 0; c < ncols / 32; ++c) {
+            uint32_t x[32];
+            tmem_ld32(base + 32 * c, x);
+            tmem_ld_wait();
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int j = 32 * c + 2 * e;
+              float a = __uint_as_float(x[2 * e]), b = __uint_as_float(x[2 * e + 1]);
+              if (diag) {
+                a = (j <= wt) ? a : 0.f;
+                b = (j + 1 <= wt) ? b : 0.f;
+              }
+              pk[e] = pack_bf16x2(a, b);
+            }
+            tmem_st16(base + 16 * c, pk);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&B.p_conv[r]);
+        }
+      }
+    }
+  }
+  // ------------------------------------------------------------------------------------
+  // Warps 12-15: epilogue readers.  Read O once, release the TMEM accumulator, add the
+  // rows' sums of squares into the fp64 per-token totals, park z = y * w * sigmoid(g).
+  // They also own the state: S0 into TMEM at each sequence start, the bf16 snapshot of S
+  // at each block end, and the final state.
+  // ------------------------------------------------------------------------------------
+  else if (warp >= kReadWarp0 && warp < kStoreWarp0) {
+    const int wt = tid - 32 * kReadWarp0;          // TMEM lane = row of the tile / of S
+    const uint32_t lane_off = static_cast<uint32_t>(wt & ~31) << 16;
     const uint32_t snap = sbase + OFF_SNAP;
+    const bool skip_publish = (p.err->inject == INJECT_SKIP_PUBLISH) && blockIdx.x == 0;
+    bool ok = true;
     int t = 0;
     uint32_t blk = 0;
-    bool ok = true;
     for (int s = 0; s < p.nseq && ok; ++s) {
       int64_t row0;
       int L;
@@ -520,101 +674,9 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         mbar_arrive(&B.snap_ready);
       }
       for (int i = 0; i < nt; ++i) {
-        const int u = i % tpb;
-        const int vr = min(kTile, L - i * kTile);
-        const int nk = pad_rows(vr);
-        if (!wait_bar_warp(&B.p_full, t & 1, B, p, SITE_TC_CONVERT, t)) { ok = false; break; }
-        tc_fence_after();
-        for (int kt = 0; kt <= u; ++kt) {
-          const bool diag = (kt == u);
-          const int ncols = diag ? nk : 128;
-          const uint32_t base = tmem + lane_off + TM_P + 128 * kt;
-          for (int c = 0; c < ncols / 32; ++c) {
-            uint32_t x[32];
-            tmem_ld32(base + 32 * c, x);
-            tmem_ld_wait();
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int j = 32 * c + 2 * e;
-              float a = __uint_as_float(x[2 * e]), b = __uint_as_float(x[2 * e + 1]);
-              if (diag) {
-                a = (j <= wt) ? a : 0.f;
-                b = (j + 1 <= wt) ? b : 0.f;
-              }
-              pk[e] = pack_bf16x2(a, b);
-            }
-            tmem_st16(base + 16 * c, pk);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&B.p_conv);
-        const bool blk_end = (u == tpb - 1) || (i == nt - 1);
-        if (blk_end) {
-          if (!wait_bar_warp(&B.s_done, blk & 1, B, p, SITE_TC_CONVERT, t)) { ok = false; break; }
-          blk++;
-          tc_fence_after();
-          uint32_t x0[32], x1[32];
-          tmem_ld32(tmem + lane_off + TM_S, x0);
-          tmem_ld32(tmem + lane_off + TM_S + 32, x1);
-          tmem_ld_wait();
-          if (i == nt - 1) {
-            if (p.state_out) {
-#pragma unroll
-              for (int c = 0; c < 32; c += 4) {
-                *reinterpret_cast<float4*>(p.state_out + st_row + c) =
-                    make_float4(__uint_as_float(x0[c]), __uint_as_float(x0[c + 1]), __uint_as_float(x0[c + 2]),
-                                __uint_as_float(x0[c + 3]));
-                *reinterpret_cast<float4*>(p.state_out + st_row + 32 + c) =
-                    make_float4(__uint_as_float(x1[c]), __uint_as_float(x1[c + 1]), __uint_as_float(x1[c + 2]),
-                                __uint_as_float(x1[c + 3]));
-              }
-            }
-            tc_fence_before();
-          } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint32_t* a = x0 + 8 * c;
-              const uint32_t* b = x1 + 8 * c;
-              sts128(snap + sw128_offset(wt, c),
-                     make_uint4(pack_bf16x2(__uint_as_float(a[0]), __uint_as_float(a[1])),
-                                pack_bf16x2(__uint_as_float(a[2]), __uint_as_float(a[3])),
-                                pack_bf16x2(__uint_as_float(a[4]), __uint_as_float(a[5])),
-                                pack_bf16x2(__uint_as_float(a[6]), __uint_as_float(a[7]))));
-              sts128(snap + sw128_offset(wt, c + 4),
-                     make_uint4(pack_bf16x2(__uint_as_float(b[0]), __uint_as_float(b[1])),
-                                pack_bf16x2(__uint_as_float(b[2]), __uint_as_float(b[3])),
-                                pack_bf16x2(__uint_as_float(b[4]), __uint_as_float(b[5])),
-                                pack_bf16x2(__uint_as_float(b[6]), __uint_as_float(b[7]))));
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&B.snap_ready);
-          }
-        }
-        ++t;
-      }
-    }
-  }
-  // ------------------------------------------------------------------------------------
-  // Warps 12-15: epilogue readers.  Read O once, release the TMEM accumulator, add the
-  // rows' sums of squares into the fp64 per-token totals, park z = y * w * sigmoid(g).
-  // ------------------------------------------------------------------------------------
-  else if (warp >= kReadWarp0 && warp < kStoreWarp0) {
-    const int wt = tid - 32 * kReadWarp0;          // TMEM lane = row of the tile
-    const uint32_t lane_off = static_cast<uint32_t>(wt & ~31) << 16;
-    const bool skip_publish = (p.err->inject == INJECT_SKIP_PUBLISH) && blockIdx.x == 0;
-    bool ok = true;
-    int t = 0;
-    for (int s = 0; s < p.nseq && ok; ++s) {
-      int64_t row0;
-      int L;
-      seq_range(p, s, row0, L);
-      const int nt = (L + kTile - 1) / kTile;
-      for (int i = 0; i < nt; ++i) {
         const int ob = t & 1;
         const int gs = t % kNG;
+        const int u = i % tpb;
         const int vr = min(kTile, L - i * kTile);
         const int64_t row = row0 + static_cast<int64_t>(i) * kTile;
         const uint32_t stg = sbase + OFF_G + gs * kGBytes;
@@ -668,6 +730,49 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           if (lane == 0 && !skip_publish) red_add_release_gpu(p.cnt + static_cast<int64_t>(s) * p.max_tiles + i, 1u);
         }
         mbar_arrive(&B.z_ready[gs]);
+        // Block end: snapshot S for the next block's inter product, or emit the final state.
+        if (u == tpb - 1 || i == nt - 1) {
+          if (!wait_bar_warp(&B.s_done, blk & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+          blk++;
+          tc_fence_after();
+          uint32_t x0[32], x1[32];
+          tmem_ld32(tmem + lane_off + TM_S, x0);
+          tmem_ld32(tmem + lane_off + TM_S + 32, x1);
+          tmem_ld_wait();
+          if (i == nt - 1) {
+            if (p.state_out) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 4) {
+                *reinterpret_cast<float4*>(p.state_out + st_row + c) =
+                    make_float4(__uint_as_float(x0[c]), __uint_as_float(x0[c + 1]), __uint_as_float(x0[c + 2]),
+                                __uint_as_float(x0[c + 3]));
+                *reinterpret_cast<float4*>(p.state_out + st_row + 32 + c) =
+                    make_float4(__uint_as_float(x1[c]), __uint_as_float(x1[c + 1]), __uint_as_float(x1[c + 2]),
+                                __uint_as_float(x1[c + 3]));
+              }
+            }
+            tc_fence_before();
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint32_t* a = x0 + 8 * c;
+              const uint32_t* b = x1 + 8 * c;
+              sts128(snap + sw128_offset(wt, c),
+                     make_uint4(pack_bf16x2(__uint_as_float(a[0]), __uint_as_float(a[1])),
+                                pack_bf16x2(__uint_as_float(a[2]), __uint_as_float(a[3])),
+                                pack_bf16x2(__uint_as_float(a[4]), __uint_as_float(a[5])),
+                                pack_bf16x2(__uint_as_float(a[6]), __uint_as_float(a[7]))));
+              sts128(snap + sw128_offset(wt, c + 4),
+                     make_uint4(pack_bf16x2(__uint_as_float(b[0]), __uint_as_float(b[1])),
+                                pack_bf16x2(__uint_as_float(b[2]), __uint_as_float(b[3])),
+                                pack_bf16x2(__uint_as_float(b[4]), __uint_as_float(b[5])),
+                                pack_bf16x2(__uint_as_float(b[6]), __uint_as_float(b[7]))));
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&B.snap_ready);
+          }
+        }
         ++t;
       }
     }
@@ -760,9 +865,12 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     if (lane == 0) bulk_wait0();
   }
 
-  // Teardown: all roles are done (or aborted with their async work drained).
+  // Teardown: all roles are done (or aborted with their async work drained).  The cluster
+  // barrier keeps this CTA's shared memory alive until the partner has stopped writing to
+  // it and arriving on its barriers.
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   tc_fence_after();
   if (warp == 1) tmem_dealloc<kTmemCols>(tmem);
 }
@@ -801,10 +909,40 @@ inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+// Clusters (head pairs) that fit on the current device at once; cached per device.
+int max_active_clusters() {
+  static int cache[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    if (cudaFuncSetAttribute(lightning_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+      return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kNdv);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kNdv;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, lightning_prefill_tc_kernel, &cfg) != cudaSuccess) n = -1;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 bool tc_eligible(const TcShape& s, int num_sms) {
+  (void)num_sms;
   if (!s.bf16 || s.D != kD || (s.C != 128 && s.C != 256) || s.H < 1) return false;
-  // The cross-head norm exchange needs every CTA of a token resident at once.
-  if (s.mode != LA_OUT_RAW && s.H * kNdv > num_sms) return false;
+  // The cross-head norm exchange needs every head's CTA pair resident at once.
+  if (s.mode != LA_OUT_RAW && s.H > max_active_clusters()) return false;
   return true;
 }
 
@@ -857,7 +995,20 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
   e = cudaFuncSetAttribute(lightning_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  lightning_prefill_tc_kernel<<<a.H * kNdv, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mg, mo, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.H * kNdv);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kNdv;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, lightning_prefill_tc_kernel, mq, mk, mv, mg, mo, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
