@@ -112,6 +112,22 @@ struct TcParams {
   uint16_t* out;
 };
 
+// Shared-memory descriptor templates with start address 0; an operand at shared address a
+// is template + ((a >> 4) & 0x3FFF) (the 14-bit start field; adding in-tile offsets to it
+// never carries out of the field because every operand lies below 256 KiB).
+// Building descriptors this way keeps the single MMA-issuing thread at a few instructions
+// per MMA, which is what lets small-N MMAs run at the tensor pipe's rate.
+constexpr uint64_t sdesc_template(uint32_t lbo, uint32_t sbo) {
+  return (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) | (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
+constexpr uint64_t kDescK = sdesc_template(16, 1024);          // K-major, 128-byte swizzle
+constexpr uint64_t kDescMN = sdesc_template(kBoxBytes, 1024);  // MN-major, 64-element chunks kBoxBytes apart
+// Descriptor of the operand at shared address `a`.  Only the low 18 address bits enter
+// the 14-bit start field: in a cluster the shared address of a CTA other than rank 0 has
+// higher bits set, which must not spill into the leading-byte-offset field.
+__device__ __forceinline__ uint64_t desc_at(uint64_t tmpl, uint32_t a) { return tmpl + ((a >> 4) & 0x3FFFu); }
+
 constexpr uint32_t kIdescQS = make_idesc_bf16(128, kDV, 0, 1);
 constexpr uint32_t kIdescPV = make_idesc_bf16(128, kDV, 0, 1);
 constexpr uint32_t kIdescDS = make_idesc_bf16(128, kDV, 1, 1);
@@ -419,14 +435,14 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         const int vr = min(kTile, it.L - it.i * kTile);
         const int kslot = (tpb == 2) ? kt : slot;
         const uint32_t n = (kt == u) ? static_cast<uint32_t>(pad_rows(vr)) : 128u;
-        const uint32_t qa = sbase + OFF_Q + slot * kQBytes;
-        const uint32_t kb = sbase + OFF_K + kslot * kKBytes;
+        const uint64_t qd = desc_at(kDescK, sbase + OFF_Q + slot * kQBytes);
+        const uint64_t kd = desc_at(kDescK, sbase + OFF_K + kslot * kKBytes);
         const uint32_t idesc = make_idesc_bf16(128, n, 0, 0);
+        const uint32_t dst = tmem + TM_P + 128 * r;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + TM_P + 128 * r, make_sdesc(qa + off, 16, 1024), make_sdesc(kb + off, 16, 1024), idesc,
-                 kk > 0);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4);
+          mma_ss(dst, qd + off, kd + off, idesc, kk > 0);
         }
         mma_commit(&B.p_full[r]);
         return true;
@@ -468,11 +484,12 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           tc_fence_after();
           // O (+)= P_bf16 V over this key tile
           const int kslot = (tpb == 2) ? kt : slot;
-          const int kext = (kt == u) ? nk : 128;
-          const uint32_t vb = sbase + OFF_V + kslot * kVBytes;
-          for (int kk = 0; kk < kext / 16; ++kk)
-            mma_ts(od, tmem + TM_P + 128 * r + 8 * kk, make_sdesc(vb + kk * 2048, kBoxBytes, 1024), kIdescPV,
-                   (kt > 0 || kk > 0) ? 1u : 0u);
+          const int ksteps = ((kt == u) ? nk : 128) / 16;
+          const uint64_t vd = desc_at(kDescMN, sbase + OFF_V + kslot * kVBytes);
+          const uint32_t pa = tmem + TM_P + 128 * r;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            if (kk < ksteps) mma_ts(od, pa + 8 * kk, vd + 128 * kk, kIdescPV, (kt > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&B.pv_done[r]);
           // The first tile's keys and values of a 256-block have no reader after this.
           if (tpb == 2 && u == 1 && kt == 0) mma_commit_multicast(&B.empty[0], 0x3);
@@ -485,21 +502,23 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           snap_waits++;
           tc_fence_after();
         }
-        const uint32_t qa = sbase + OFF_Q + slot * kQBytes;
-        const uint32_t snap = sbase + OFF_SNAP;
+        {
+          const uint64_t qd = desc_at(kDescK, sbase + OFF_Q + slot * kQBytes);
+          const uint64_t sd = desc_at(kDescMN, sbase + OFF_SNAP);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_ss(od, make_sdesc(qa + off, 16, 1024), make_sdesc(snap + kk * 2048, kBoxBytes, 1024), kIdescQS, 1);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(od, qd + static_cast<uint64_t>(((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4), sd + 128 * kk,
+                   kIdescQS, 1);
         }
         mma_commit(&B.o_full[ob]);
         // S += phi(K)^T V
         {
-          const uint32_t kb = sbase + OFF_K + slot * kKBytes;
-          const uint32_t vb = sbase + OFF_V + slot * kVBytes;
-          for (int kk = 0; kk < nk / 16; ++kk)
-            mma_ss(tmem + TM_S, make_sdesc(kb + kk * 2048, kBoxBytes, 1024), make_sdesc(vb + kk * 2048, kBoxBytes, 1024),
-                   kIdescDS, 1);
+          const uint64_t kd = desc_at(kDescMN, sbase + OFF_K + slot * kKBytes);
+          const uint64_t vd = desc_at(kDescMN, sbase + OFF_V + slot * kVBytes);
+          const int ksteps = nk / 16;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            if (kk < ksteps) mma_ss(tmem + TM_S, kd + 128 * kk, vd + 128 * kk, kIdescDS, 1);
         }
         const bool blk_end = (u == tpb - 1) || (cur.i == cur.nt - 1);
         // Slot release goes to both CTAs: the partner writes its transformed box here.
