@@ -30,13 +30,14 @@
 //    is computed while the current one is being converted.
 //  * A conversion warpgroup turns P (fp32, TMEM) into masked bf16 in place.
 //  * The epilogue reader warpgroup owns the state (S0 in, the bf16 snapshot of S at each
-//    block end, the final state out) and reads O once: it adds each row's sum of squares into an fp64
-//    per-token accumulator in global memory (red.add; the fp64 sum of the fp32 partials is
-//    exact whenever a token's partials span less than 2^22, so the result does not depend
-//    on the order the additions land in), bumps the tile's arrival counter, and parks
-//    z = y * w * sigmoid(g) as bf16 in place of the gate tile.  Two tiles later, once all
-//    H * 2 CTAs have arrived for that tile, it scales z by rsqrt(mean(y^2) + eps) and
-//    stores the bf16 output with TMA.  The TMEM accumulator is free right after the read.
+//    block end, the final state out) and reads O once, releasing the accumulator at once:
+//    it parks z = y * w * sigmoid(g) as bf16 pairs in two spare TMEM tiles (which frees the
+//    gate slot straight away), adds each row's sum of squares into an fp64 per-token
+//    accumulator in global memory (red.add; the fp64 sum of the fp32 partials is exact
+//    whenever a token's partials span less than 2^22, so the result does not depend on the
+//    order the additions land in) and bumps the tile's arrival counter.  Four storer warps,
+//    one per TMEM lane quarter, wait until all H * 2 CTAs have arrived for the tile, scale
+//    their rows of z by rsqrt(mean(y^2) + eps) in registers and store 32-row boxes with TMA.
 //  * Every wait is bounded (globaltimer); a wait that runs out records LA_ERR_TIMEOUT in
 //    the workspace and the CTA drains its async work, frees TMEM and exits.
 #include <cudaTypedefs.h>
@@ -56,12 +57,13 @@ constexpr int kD = 128;          // head dim (d_k = d_v)
 constexpr int kDV = 64;          // d_v slice per CTA
 constexpr int kNdv = kD / kDV;   // CTAs per head
 constexpr int kTile = 128;       // rows per tile (MMA M)
-constexpr int kThreads = 576;  // 18 warps
+constexpr int kThreads = 640;    // 20 warps
 constexpr int kXfWarp0 = 2;      // transform warps 2..7
 constexpr int kXfThreads = 192;
-constexpr int kNG = 3;           // gate / output staging slots
-constexpr int kReadWarp0 = 12;   // epilogue readers: warps 12..15
-constexpr int kStoreWarp0 = 16;  // epilogue storers: warps 16..17 (alternate tiles)
+constexpr int kNG = 2;           // gate slots
+constexpr int kReadWarp0 = 12;   // epilogue readers: warps 12..15 (TMEM lane quarters 0..3)
+constexpr int kStoreWarp0 = 16;  // epilogue storers: warps 16..19 (TMEM lane quarters 0..3)
+constexpr int kQuarterRows = 32; // rows of a tile one reader / storer warp owns
 
 constexpr uint32_t kQBytes = kTile * kD * 2;     // 32 KiB (two 64-column swizzled boxes)
 constexpr uint32_t kKBytes = kQBytes;
@@ -69,17 +71,20 @@ constexpr uint32_t kVBytes = kTile * kDV * 2;    // 16 KiB
 constexpr uint32_t kGBytes = kVBytes;
 constexpr uint32_t kSnapBytes = kD * kDV * 2;    // 16 KiB
 constexpr uint32_t kBoxBytes = kTile * 64 * 2;   // one 128-row x 64-column box
+constexpr uint32_t kStgBytes = kQuarterRows * kDV * 2;   // 4 KiB output staging per storer warp
 
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + 2 * kQBytes;
 constexpr uint32_t OFF_V = OFF_K + 2 * kKBytes;
 constexpr uint32_t OFF_G = OFF_V + 2 * kVBytes;
-constexpr uint32_t OFF_SNAP = OFF_G + kNG * kGBytes;
+constexpr uint32_t OFF_STG = OFF_G + kNG * kGBytes;
+constexpr uint32_t OFF_SNAP = OFF_STG + 4 * kStgBytes;
 constexpr uint32_t OFF_BARS = OFF_SNAP + kSnapBytes;
 
 // TMEM columns (512 allocated; 128 lanes each)
 constexpr uint32_t TM_S = 0;      // fp32 state slice, 64 columns
 constexpr uint32_t TM_O = 64;     // 2 output accumulators x 64 columns
+constexpr uint32_t TM_Z = 192;    // 2 parked z tiles x 32 columns (bf16 pairs)
 constexpr uint32_t TM_P = 256;    // 2 score tiles x 128 columns
 constexpr uint32_t kTmemCols = 512;
 
@@ -89,7 +94,7 @@ struct Bars {
   uint64_t p_full[2], p_conv[2], pv_done[2];   // per TMEM score region
   uint64_t o_full[2], o_empty[2];
   uint64_t s_done, snap_ready, final_bar;
-  uint64_t z_ready[kNG], stg_free[kNG];
+  uint64_t z_full[2][4], z_free[2][4];   // per parked-z slot and TMEM lane quarter
   uint32_t tmem_base;
   int abort_flag;
   float w[kDV];
@@ -294,7 +299,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     }
     for (int i = 0; i < kNG; ++i) {
       mbar_init(&B.full_g[i], 1);
-      mbar_init(&B.empty_g[i], 1);
+      mbar_init(&B.empty_g[i], 128);   // every reader thread has read its row of the gate
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&B.p_full[i], 1);
@@ -304,10 +309,11 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     mbar_init(&B.s_done, 1);
     mbar_init(&B.snap_ready, 128);
     mbar_init(&B.final_bar, 1);
-    for (int i = 0; i < kNG; ++i) {
-      mbar_init(&B.z_ready[i], 128);
-      mbar_init(&B.stg_free[i], 1);
-    }
+    for (int i = 0; i < 2; ++i)
+      for (int q = 0; q < 4; ++q) {
+        mbar_init(&B.z_full[i][q], 32);
+        mbar_init(&B.z_free[i][q], 32);
+      }
     B.abort_flag = 0;
     fence_mbar_init();
   }
@@ -322,7 +328,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
 
   // ------------------------------------------------------------------------------------
   // Warp 0: TMA producers.  Lane 0 streams Q/K/V tiles into the two-slot ring; lane 1
-  // streams gate tiles into the three-slot staging ring, running ahead on its own.
+  // streams gate tiles into the two-slot gate ring, running ahead on its own.
   // ------------------------------------------------------------------------------------
   if (warp == 0) {
     if (lane == 0) {
@@ -363,7 +369,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     } else if (lane == 1 && gate) {
       prefetch_tmap(&tm_g);
       const uint64_t pol = policy_evict_first();
-      uint32_t guses[kNG] = {0, 0, 0};
+      uint32_t guses[kNG] = {0, 0};
       int t = 0;
       bool ok = true;
       for (int s = 0; s < p.nseq && ok; ++s) {
@@ -648,6 +654,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   // ------------------------------------------------------------------------------------
   else if (warp >= kReadWarp0 && warp < kStoreWarp0) {
     const int wt = tid - 32 * kReadWarp0;          // TMEM lane = row of the tile / of S
+    const int q = warp - kReadWarp0;               // lane quarter
     const uint32_t lane_off = static_cast<uint32_t>(wt & ~31) << 16;
     const uint32_t snap = sbase + OFF_SNAP;
     const bool skip_publish = (p.err->inject == INJECT_SKIP_PUBLISH) && blockIdx.x == 0;
@@ -695,60 +702,64 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       for (int i = 0; i < nt; ++i) {
         const int ob = t & 1;
         const int gs = t % kNG;
+        const int zs = t & 1;
         const int u = i % tpb;
         const int vr = min(kTile, L - i * kTile);
         const int64_t row = row0 + static_cast<int64_t>(i) * kTile;
-        const uint32_t stg = sbase + OFF_G + gs * kGBytes;
         if (!wait_bar_warp(&B.o_full[ob], (t >> 1) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
-        if (gate) {
-          if (!wait_bar_warp(&B.full_g[gs], (t / kNG) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
-        } else if (t >= kNG) {
-          if (!wait_bar_warp(&B.stg_free[gs], ((t / kNG) - 1) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+        if (t >= 2 && !wait_bar_warp(&B.z_free[zs][q], ((t >> 1) - 1) & 1, B, p, SITE_TC_EPILOGUE, t)) {
+          ok = false;
+          break;
         }
+        if (gate && !wait_bar_warp(&B.full_g[gs], (t / kNG) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
         tc_fence_after();
-        float ss = 0.f;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t x[32];
-          tmem_ld32(tmem + lane_off + TM_O + kDV * ob + 32 * half, x);
-          tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int chunk = 4 * half + c;
-            const uint32_t addr = stg + sw128_offset(wt, chunk);
-            uint4 gv = make_uint4(0, 0, 0, 0);
-            if (gate) gv = lds128(addr);
-            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-            uint32_t zw[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int col = 8 * chunk + 2 * e;
-              float a = __uint_as_float(x[8 * c + 2 * e]);
-              float b = __uint_as_float(x[8 * c + 2 * e + 1]);
-              ss = fmaf(a, a, ss);
-              ss = fmaf(b, b, ss);
-              if (norm) {
-                a *= B.w[col];
-                b *= B.w[col + 1];
-              }
-              if (gate) {
-                a *= sigmoid_fast(__uint_as_float(gw[e] << 16));
-                b *= sigmoid_fast(__uint_as_float(gw[e] & 0xFFFF0000u));
-              }
-              zw[e] = pack_bf16x2(a, b);
-            }
-            sts128(addr, make_uint4(zw[0], zw[1], zw[2], zw[3]));
-          }
-        }
+        // O of this row, then the accumulator goes straight back to the MMA warp.
+        uint32_t x[2 * 32];
+        tmem_ld32(tmem + lane_off + TM_O + kDV * ob, *reinterpret_cast<uint32_t(*)[32]>(x));
+        tmem_ld32(tmem + lane_off + TM_O + kDV * ob + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+        tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&B.o_empty[ob]);
+        // z = y * w * sigmoid(g), parked as bf16 pairs in TMEM for the storer of this quarter.
+        const uint8_t* grow = smem + OFF_G + gs * kGBytes;
+        float ss = 0.f;
+        uint32_t z[32];
+#pragma unroll
+        for (int chunk = 0; chunk < 8; ++chunk) {
+          uint4 gv = make_uint4(0, 0, 0, 0);
+          if (gate) gv = *reinterpret_cast<const uint4*>(grow + sw128_offset(wt, chunk));
+          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = 8 * chunk + 2 * e;
+            float a = __uint_as_float(x[col]);
+            float b = __uint_as_float(x[col + 1]);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+            if (norm) {
+              a *= B.w[col];
+              b *= B.w[col + 1];
+            }
+            if (gate) {
+              a *= sigmoid_fast(__uint_as_float(gw[e] << 16));
+              b *= sigmoid_fast(__uint_as_float(gw[e] & 0xFFFF0000u));
+            }
+            z[4 * chunk + e] = pack_bf16x2(a, b);
+          }
+        }
+        if (gate) mbar_arrive(&B.empty_g[gs]);
+        const uint32_t zt = tmem + lane_off + TM_Z + 32 * zs;
+        tmem_st16(zt, *reinterpret_cast<const uint32_t(*)[16]>(z));
+        tmem_st16(zt + 16, *reinterpret_cast<const uint32_t(*)[16]>(z + 16));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&B.z_full[zs][q]);
         if (norm) {
           if (wt < vr) red_add_f64(p.ss + row + wt, static_cast<double>(ss));
           __syncwarp();
           // One release per warp orders the warp's additions before the arrival count.
           if (lane == 0 && !skip_publish) red_add_release_gpu(p.cnt + static_cast<int64_t>(s) * p.max_tiles + i, 1u);
         }
-        mbar_arrive(&B.z_ready[gs]);
         // Block end: snapshot S for the next block's inter product, or emit the final state.
         if (u == tpb - 1 || i == nt - 1) {
           if (!wait_bar_warp(&B.s_done, blk & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
@@ -797,11 +808,14 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     }
   }
   // ------------------------------------------------------------------------------------
-  // Warps 16-17: epilogue storers, alternating tiles.  Wait until every reader warp of
-  // every CTA has added its sums for the tile, scale z by rsqrt(mean(y^2) + eps), store.
+  // Warps 16-19: epilogue storers, one per TMEM lane quarter (32 rows of every tile).
+  // Wait until every reader warp of every CTA has added its sums for the tile, read the
+  // parked z, scale it by rsqrt(mean(y^2) + eps) and store the quarter.
   // ------------------------------------------------------------------------------------
   else if (warp >= kStoreWarp0) {
-    const int sw = warp - kStoreWarp0;
+    const int q = warp - kStoreWarp0;              // == warp % 4: the lane quarter it may access
+    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+    const uint32_t stg = sbase + OFF_STG + q * kStgBytes;
     const int HD = p.H * kD;
     const float inv_hd = 1.0f / static_cast<float>(HD);
     bool ok = true;
@@ -812,12 +826,17 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       seq_range(p, s, row0, L);
       const int nt = (L + kTile - 1) / kTile;
       for (int i = 0; i < nt; ++i, ++t) {
-        if ((t & 1) != sw) continue;
-        const int gs = t % kNG;
+        const int zs = t & 1;
         const int vr = min(kTile, L - i * kTile);
+        const int r = kQuarterRows * q + lane;     // row of the tile
         const int64_t row = row0 + static_cast<int64_t>(i) * kTile;
-        const uint32_t stg = sbase + OFF_G + gs * kGBytes;
-        if (!wait_bar_warp(&B.z_ready[gs], (t / kNG) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+        if (!wait_bar_warp(&B.z_full[zs][q], (t >> 1) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t z[32];
+        tmem_ld32(tmem + lane_off + TM_Z + 32 * zs, z);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&B.z_free[zs][q]);
         if (norm) {
           unsigned int* c = p.cnt + static_cast<int64_t>(s) * p.max_tiles + i;
           int go = 1;
@@ -837,48 +856,30 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           }
           if (!__shfl_sync(0xFFFFFFFFu, go, 0)) { ok = false; break; }
           (void)ld_acquire_gpu(c);
-          float rn[4];
+          const float rn = (r < vr) ? 1.0f / sqrtf(static_cast<float>(ld_cg_f64(p.ss + row + r)) * inv_hd + p.eps) : 0.0f;
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const int r = lane + 32 * m;
-            rn[m] = (r < vr) ? 1.0f / sqrtf(static_cast<float>(ld_cg_f64(p.ss + row + r)) * inv_hd + p.eps) : 0.0f;
-          }
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const int r = lane + 32 * m;
-#pragma unroll
-            for (int chunk = 0; chunk < 8; ++chunk) {
-              const uint32_t addr = stg + sw128_offset(r, chunk);
-              const uint4 zv = lds128(addr);
-              const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
-              uint32_t ow[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                ow[e] = pack_bf16x2(__uint_as_float(zw[e] << 16) * rn[m], __uint_as_float(zw[e] & 0xFFFF0000u) * rn[m]);
-              sts128(addr, make_uint4(ow[0], ow[1], ow[2], ow[3]));
-            }
-          }
+          for (int e = 0; e < 32; ++e)
+            z[e] = pack_bf16x2(__uint_as_float(z[e] << 16) * rn, __uint_as_float(z[e] & 0xFFFF0000u) * rn);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (vr == kTile) {
-          if (lane == 0) {
-            tma_store_2d(&tm_o, smem + OFF_G + gs * kGBytes, h * kD + dvt * kDV, static_cast<int32_t>(row));
-            bulk_commit();
-            bulk_wait_read0();
-          }
-        } else {
-          for (int m = 0; m < 4; ++m) {
-            const int r = lane + 32 * m;
-            if (r < vr) {
-              uint16_t* dst = p.out + (row + r) * HD + h * kD + dvt * kDV;
-#pragma unroll
-              for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + 8 * c) = lds128(stg + sw128_offset(r, c));
-            }
-          }
+        if (kQuarterRows * (q + 1) <= vr) {
+          // The staging buffer is free once this warp's previous store has read it.
+          if (lane == 0) bulk_wait_read0();
           __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            sts128(stg + sw128_offset(lane, c), make_uint4(z[4 * c], z[4 * c + 1], z[4 * c + 2], z[4 * c + 3]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_o, smem + OFF_STG + q * kStgBytes, h * kD + dvt * kDV,
+                         static_cast<int32_t>(row + kQuarterRows * q));
+            bulk_commit();
+          }
+        } else if (r < vr) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (row + r) * HD + h * kD + dvt * kDV);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) dst[c] = make_uint4(z[4 * c], z[4 * c + 1], z[4 * c + 2], z[4 * c + 3]);
         }
-        if (lane == 0) mbar_arrive(gate ? &B.empty_g[gs] : &B.stg_free[gs]);
       }
     }
     if (lane == 0) bulk_wait0();
@@ -910,13 +911,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [rows, cols] bf16 row-major, box 64 columns x 128 rows, 128-byte swizzle, zero fill.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
+// [rows, cols] bf16 row-major, box 64 columns x box_rows rows, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows = kTile) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTile)};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1001,7 +1002,7 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
   const int64_t cols = static_cast<int64_t>(a.H) * kD;
   CUtensorMap mq, mk, mv, mg, mo;
   if (!make_map(&mq, a.q, a.tokens, cols) || !make_map(&mk, a.k, a.tokens, cols) ||
-      !make_map(&mv, a.v, a.tokens, cols) || !make_map(&mo, a.out, a.tokens, cols))
+      !make_map(&mv, a.v, a.tokens, cols) || !make_map(&mo, a.out, a.tokens, cols, kQuarterRows))
     return cudaErrorInvalidValue;
   if (a.mode == LA_OUT_RMSNORM_GATE) {
     if (!make_map(&mg, a.g, a.tokens, cols)) return cudaErrorInvalidValue;
