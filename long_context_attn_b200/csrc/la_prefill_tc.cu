@@ -15,10 +15,13 @@
 //    second tile multiplies by the first tile's keys densely and by its own keys under the
 //    causal mask; the all-zero upper-right quarter of the 256 x 256 block is never issued.
 //  * The two CTAs of a head form a cluster.  Each loads (TMA, 128-byte swizzle) its own
-//    64-column box of the Q and K tiles plus its V and gate slices, applies SiLU to its
-//    boxes with six transform warps, and writes the result both into its own shared memory
-//    and into its partner's (distributed shared memory), so each SiLU is computed once per
-//    head and both CTAs end up with the full phi(Q), phi(K) tiles.
+//    64-column box of the Q and K tiles plus its V slice, applies SiLU to its boxes with
+//    six transform warps, and writes the result both into its own shared memory and into
+//    its partner's (distributed shared memory), so each SiLU is computed once per head and
+//    both CTAs end up with the full phi(Q), phi(K) tiles.  Q tiles use a two-slot ring and
+//    K/V tiles a three-slot ring, so the next block's first tile loads while the second
+//    tile of a 256-block still reads the first tile's keys and values.  The gate tile is
+//    only prefetched into L2.
 //  * One thread issues all MMAs (bf16 in, fp32 accumulate in TMEM), per tile:
 //      P   = phi(Q) phi(K)^T          SS, M128 x N(<=128) x K128, into TMEM
 //      O   = P_bf16 V                 TS (P read back from TMEM), M128 x N64 x K(<=128)
@@ -31,13 +34,14 @@
 //  * A conversion warpgroup turns P (fp32, TMEM) into masked bf16 in place.
 //  * The epilogue reader warpgroup owns the state (S0 in, the bf16 snapshot of S at each
 //    block end, the final state out) and reads O once, releasing the accumulator at once:
-//    it parks z = y * w * sigmoid(g) as bf16 pairs in two spare TMEM tiles (which frees the
-//    gate slot straight away), adds each row's sum of squares into an fp64 per-token
-//    accumulator in global memory (red.add; the fp64 sum of the fp32 partials is exact
-//    whenever a token's partials span less than 2^22, so the result does not depend on the
-//    order the additions land in) and bumps the tile's arrival counter.  Four storer warps,
-//    one per TMEM lane quarter, wait until all H * 2 CTAs have arrived for the tile, scale
-//    their rows of z by rsqrt(mean(y^2) + eps) in registers and store 32-row boxes with TMA.
+//    it parks z = y * w as bf16 pairs in two spare TMEM tiles, adds each row's sum of
+//    squares into an fp64 per-token accumulator in global memory (red.add; the fp64 sum of
+//    the fp32 partials is exact whenever a token's partials span less than 2^22, so the
+//    result does not depend on the order the additions land in) and bumps the tile's
+//    arrival counter.  Four storer warps, one per TMEM lane quarter, load their rows of the
+//    gate, wait until all H * 2 CTAs have arrived for the tile (the gate loads are in
+//    flight meanwhile), scale z by rsqrt(mean(y^2) + eps) * sigmoid(g) in registers and
+//    store each row's 128 bytes straight from registers.
 //  * Every wait is bounded (globaltimer); a wait that runs out records LA_ERR_TIMEOUT in
 //    the workspace and the CTA drains its async work, frees TMEM and exits.
 #include <cudaTypedefs.h>
@@ -60,7 +64,8 @@ constexpr int kTile = 128;       // rows per tile (MMA M)
 constexpr int kThreads = 640;    // 20 warps
 constexpr int kXfWarp0 = 2;      // transform warps 2..7
 constexpr int kXfThreads = 192;
-constexpr int kNG = 2;           // gate slots
+constexpr int kNQ = 2;           // Q slots
+constexpr int kNKV = 3;          // K / V slots (a 256-block's first tile stays while the next loads)
 constexpr int kReadWarp0 = 12;   // epilogue readers: warps 12..15 (TMEM lane quarters 0..3)
 constexpr int kStoreWarp0 = 16;  // epilogue storers: warps 16..19 (TMEM lane quarters 0..3)
 constexpr int kQuarterRows = 32; // rows of a tile one reader / storer warp owns
@@ -68,17 +73,13 @@ constexpr int kQuarterRows = 32; // rows of a tile one reader / storer warp owns
 constexpr uint32_t kQBytes = kTile * kD * 2;     // 32 KiB (two 64-column swizzled boxes)
 constexpr uint32_t kKBytes = kQBytes;
 constexpr uint32_t kVBytes = kTile * kDV * 2;    // 16 KiB
-constexpr uint32_t kGBytes = kVBytes;
 constexpr uint32_t kSnapBytes = kD * kDV * 2;    // 16 KiB
 constexpr uint32_t kBoxBytes = kTile * 64 * 2;   // one 128-row x 64-column box
-constexpr uint32_t kStgBytes = kQuarterRows * kDV * 2;   // 4 KiB output staging per storer warp
 
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + 2 * kQBytes;
-constexpr uint32_t OFF_V = OFF_K + 2 * kKBytes;
-constexpr uint32_t OFF_G = OFF_V + 2 * kVBytes;
-constexpr uint32_t OFF_STG = OFF_G + kNG * kGBytes;
-constexpr uint32_t OFF_SNAP = OFF_STG + 4 * kStgBytes;
+constexpr uint32_t OFF_K = OFF_Q + kNQ * kQBytes;
+constexpr uint32_t OFF_V = OFF_K + kNKV * kKBytes;
+constexpr uint32_t OFF_SNAP = OFF_V + kNKV * kVBytes;
 constexpr uint32_t OFF_BARS = OFF_SNAP + kSnapBytes;
 
 // TMEM columns (512 allocated; 128 lanes each)
@@ -89,8 +90,7 @@ constexpr uint32_t TM_P = 256;    // 2 score tiles x 128 columns
 constexpr uint32_t kTmemCols = 512;
 
 struct Bars {
-  uint64_t full_qkv[2], xformed[2], empty[2];
-  uint64_t full_g[kNG], empty_g[kNG];
+  uint64_t full_qkv[kNKV], xformed[kNKV], kv_empty[kNKV], q_empty[kNQ];
   uint64_t p_full[2], p_conv[2], pv_done[2];   // per TMEM score region
   uint64_t o_full[2], o_empty[2];
   uint64_t s_done, snap_ready, final_bar;
@@ -111,6 +111,7 @@ struct TcParams {
   int64_t tokens;
   float eps;
   const float* w;
+  const uint16_t* g;   // gate [tokens, H * D] (gated mode)
   ErrRec* err;
   unsigned int* cnt;   // [nseq * max_tiles] arrivals per tile
   double* ss;          // [tokens] sum of squares over the head concatenation
@@ -199,7 +200,7 @@ __device__ __forceinline__ bool aborted(Bars& B) { return *reinterpret_cast<vola
 
 // Bounded wait for phase `parity` of an mbarrier.  Returns false (after recording a
 // timeout, or because another role already did) when the CTA is aborting.
-__device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars& B, const TcParams& p, uint32_t site,
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars& B, const TcParams& p, uint32_t site,
                                       uint32_t index) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -244,6 +245,20 @@ __device__ __forceinline__ uint32_t silu_bf16x2(uint32_t x) {
   return r;
 }
 
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v);
+// Columns 16j .. 16j + 15 of one row of S (fp32 bits) into the bf16 snapshot: two
+// 16-byte chunks of the row's 128-byte-swizzled line.
+__device__ __forceinline__ void store_snap16(uint32_t snap, int row, int j, const uint32_t (&r)[16]) {
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    const uint32_t* a = r + 8 * h2;
+    sts128(snap + sw128_offset(row, 2 * j + h2),
+           make_uint4(pack_bf16x2(__uint_as_float(a[0]), __uint_as_float(a[1])),
+                      pack_bf16x2(__uint_as_float(a[2]), __uint_as_float(a[3])),
+                      pack_bf16x2(__uint_as_float(a[4]), __uint_as_float(a[5])),
+                      pack_bf16x2(__uint_as_float(a[6]), __uint_as_float(a[7]))));
+  }
+}
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -251,6 +266,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 }
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+// Streaming 16-byte store that does not allocate in L1.
+__device__ __forceinline__ void st_global_na(uint4* p, uint4 v) {
+  asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
                : "memory");
 }
 __device__ __forceinline__ double ld_cg_f64(const double* p) {
@@ -271,7 +292,7 @@ __device__ __forceinline__ void red_add_f64(double* p, double v) {
 __global__ void __launch_bounds__(kThreads, 1)
 lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                            const __grid_constant__ CUtensorMap tm_o, const TcParams p) {
+                            const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
@@ -290,16 +311,15 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   const int W = p.H * kNdv * 4;          // reader warps contributing to one tile's norm
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNKV; ++i) {
       mbar_init(&B.full_qkv[i], 1);
       mbar_init(&B.xformed[i], 2 * kXfThreads);   // both CTAs' transform threads
-      mbar_init(&B.empty[i], 2);                  // both CTAs' MMAs released the slot
+      mbar_init(&B.kv_empty[i], 2);               // both CTAs' MMAs released the slot
+    }
+    for (int i = 0; i < kNQ; ++i) mbar_init(&B.q_empty[i], 2);
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&B.o_full[i], 1);
       mbar_init(&B.o_empty[i], 128);
-    }
-    for (int i = 0; i < kNG; ++i) {
-      mbar_init(&B.full_g[i], 1);
-      mbar_init(&B.empty_g[i], 128);   // every reader thread has read its row of the gate
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&B.p_full[i], 1);
@@ -327,16 +347,18 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   const uint32_t tmem = B.tmem_base;
 
   // ------------------------------------------------------------------------------------
-  // Warp 0: TMA producers.  Lane 0 streams Q/K/V tiles into the two-slot ring; lane 1
-  // streams gate tiles into the two-slot gate ring, running ahead on its own.
+  // Warp 0, lane 0: TMA producer.  Tile t's Q box goes to Q slot t % 2, its K box and V
+  // slice to K/V slot t % 3; the gate tile is only prefetched into L2 (the readers load
+  // their rows of it straight from global memory).
   // ------------------------------------------------------------------------------------
   if (warp == 0) {
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
+      if (gate) prefetch_tmap(&tm_g);
       const uint64_t pol = policy_evict_first();
-      uint32_t uses[2] = {0, 0};
+      uint32_t qu[kNQ] = {0, 0}, ku[kNKV] = {0, 0, 0};
       int t = 0;
       bool ok = true;
       for (int s = 0; s < p.nseq && ok; ++s) {
@@ -345,53 +367,33 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         seq_range(p, s, row0, L);
         const int nt = (L + kTile - 1) / kTile;
         for (int i = 0; i < nt; ++i) {
-          const int slot = (tpb == 2) ? (i & 1) : (t & 1);
-          if (uses[slot] > 0 && !wait_bar(&B.empty[slot], (uses[slot] - 1) & 1, B, p, SITE_TC_PRODUCER, t)) {
+          const int qs = t % kNQ, ks = t % kNKV;
+          if (qu[qs] > 0 && !wait_bar(&B.q_empty[qs], (qu[qs] - 1) & 1, B, p, SITE_TC_PRODUCER, t)) {
+            ok = false;
+            break;
+          }
+          if (ku[ks] > 0 && !wait_bar(&B.kv_empty[ks], (ku[ks] - 1) & 1, B, p, SITE_TC_PRODUCER, t)) {
             ok = false;
             break;
           }
           const int32_t row = static_cast<int32_t>(row0 + static_cast<int64_t>(i) * kTile);
           // This CTA's 64-column boxes of Q and K (the partner supplies the other box) and
           // its V slice.
-          mbar_arrive_expect_tx(&B.full_qkv[slot], 2 * kBoxBytes + kVBytes);
-          uint8_t* q = smem + OFF_Q + slot * kQBytes + dvt * kBoxBytes;
-          uint8_t* k = smem + OFF_K + slot * kKBytes + dvt * kBoxBytes;
-          tma_load_2d(q, &tm_q, h * kD + dvt * 64, row, &B.full_qkv[slot], pol);
-          tma_load_2d(k, &tm_k, h * kD + dvt * 64, row, &B.full_qkv[slot], pol);
-          tma_load_2d(smem + OFF_V + slot * kVBytes, &tm_v, h * kD + dvt * kDV, row, &B.full_qkv[slot], pol);
-          uses[slot]++;
+          mbar_arrive_expect_tx(&B.full_qkv[ks], 2 * kBoxBytes + kVBytes);
+          uint8_t* qd = smem + OFF_Q + qs * kQBytes + dvt * kBoxBytes;
+          uint8_t* kd = smem + OFF_K + ks * kKBytes + dvt * kBoxBytes;
+          tma_load_2d(qd, &tm_q, h * kD + dvt * 64, row, &B.full_qkv[ks], pol);
+          tma_load_2d(kd, &tm_k, h * kD + dvt * 64, row, &B.full_qkv[ks], pol);
+          tma_load_2d(smem + OFF_V + ks * kVBytes, &tm_v, h * kD + dvt * kDV, row, &B.full_qkv[ks], pol);
+          if (gate) tma_prefetch_l2_2d(&tm_g, h * kD + dvt * kDV, row);
+          qu[qs]++;
+          ku[ks]++;
           ++t;
         }
       }
       // Drain: every issued load must have landed before the CTA may exit.
-      for (int i = 0; i < 2; ++i)
-        if (uses[i] > 0) drain_bar(&B.full_qkv[i], (uses[i] - 1) & 1);
-    } else if (lane == 1 && gate) {
-      prefetch_tmap(&tm_g);
-      const uint64_t pol = policy_evict_first();
-      uint32_t guses[kNG] = {0, 0};
-      int t = 0;
-      bool ok = true;
-      for (int s = 0; s < p.nseq && ok; ++s) {
-        int64_t row0;
-        int L;
-        seq_range(p, s, row0, L);
-        const int nt = (L + kTile - 1) / kTile;
-        for (int i = 0; i < nt; ++i) {
-          const int gs = t % kNG;
-          if (guses[gs] > 0 && !wait_bar(&B.empty_g[gs], (guses[gs] - 1) & 1, B, p, SITE_TC_PRODUCER, t)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&B.full_g[gs], kGBytes);
-          tma_load_2d(smem + OFF_G + gs * kGBytes, &tm_g, h * kD + dvt * kDV,
-                      static_cast<int32_t>(row0 + static_cast<int64_t>(i) * kTile), &B.full_g[gs], pol);
-          guses[gs]++;
-          ++t;
-        }
-      }
-      for (int i = 0; i < kNG; ++i)
-        if (guses[i] > 0) drain_bar(&B.full_g[i], (guses[i] - 1) & 1);
+      for (int i = 0; i < kNKV; ++i)
+        if (ku[i] > 0) drain_bar(&B.full_qkv[i], (ku[i] - 1) & 1);
     }
   }
   // ------------------------------------------------------------------------------------
@@ -402,7 +404,6 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   // ------------------------------------------------------------------------------------
   else if (warp == 1) {
     if (lane == 0) {
-      uint32_t uses[2] = {0, 0};       // xformed phases consumed per slot
       uint32_t snap_waits = 0;
       uint32_t k = 0;                  // next job to consume (PV)
       uint32_t kp = 0;                 // next job whose P is issued
@@ -414,21 +415,22 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       nxt = cur;
       tile_next(p, nxt);
 
-      auto slot_of = [&](const TileIter& it, int tt) { return (tpb == 2) ? (it.i & 1) : (tt & 1); };
       // Wait (blocking) or test (non-blocking) for the transformed data of tile tt.
-      auto take_xf = [&](const TileIter& it, int tt, bool block) -> int {
+      auto take_xf = [&](int tt, bool block) -> int {
         if (xf_tile >= tt) return 1;
-        const int slot = slot_of(it, tt);
+        uint64_t* bar = &B.xformed[tt % kNKV];
+        const uint32_t par = static_cast<uint32_t>(tt / kNKV) & 1u;
         if (block) {
-          if (!wait_bar(&B.xformed[slot], uses[slot] & 1, B, p, SITE_TC_MMA, tt)) return -1;
-        } else if (!mbar_try_wait(&B.xformed[slot], uses[slot] & 1)) {
+          if (!wait_bar(bar, par, B, p, SITE_TC_MMA, tt)) return -1;
+        } else if (!mbar_try_wait(bar, par)) {
           return 0;
         }
-        uses[slot]++;
         xf_tile = tt;
         tc_fence_after();
         return 1;
       };
+      // K/V slot of key tile kt of the block that tile tt (position u in it) belongs to.
+      auto kv_slot = [&](int tt, int u, int kt) { return (kt == u ? tt : tt - 1) % kNKV; };
       // P of job `job` = (tile it / tt, key tile kt) into region job & 1.
       auto issue_p = [&](const TileIter& it, int tt, int kt, uint32_t job) -> bool {
         const uint32_t r = job & 1u;
@@ -437,12 +439,10 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           tc_fence_after();
         }
         const int u = it.i % tpb;
-        const int slot = slot_of(it, tt);
         const int vr = min(kTile, it.L - it.i * kTile);
-        const int kslot = (tpb == 2) ? kt : slot;
         const uint32_t n = (kt == u) ? static_cast<uint32_t>(pad_rows(vr)) : 128u;
-        const uint64_t qd = desc_at(kDescK, sbase + OFF_Q + slot * kQBytes);
-        const uint64_t kd = desc_at(kDescK, sbase + OFF_K + kslot * kKBytes);
+        const uint64_t qd = desc_at(kDescK, sbase + OFF_Q + (tt % kNQ) * kQBytes);
+        const uint64_t kd = desc_at(kDescK, sbase + OFF_K + kv_slot(tt, u, kt) * kKBytes);
         const uint32_t idesc = make_idesc_bf16(128, n, 0, 0);
         const uint32_t dst = tmem + TM_P + 128 * r;
 #pragma unroll
@@ -456,13 +456,13 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
 
       while (ok && cur.valid) {
         const int u = cur.i % tpb;
-        const int slot = slot_of(cur, t);
+        const int qs = t % kNQ, ks = t % kNKV;
         const int ob = t & 1;
         const int vr = min(kTile, cur.L - cur.i * kTile);
         const int nk = pad_rows(vr);
         const uint32_t k0 = k;
         if (kp == k0) {  // P of this tile's first job was not issued ahead
-          if (take_xf(cur, t, true) < 0 || !issue_p(cur, t, 0, kp)) { ok = false; break; }
+          if (take_xf(t, true) < 0 || !issue_p(cur, t, 0, kp)) { ok = false; break; }
           ++kp;
         }
         const uint32_t od = tmem + TM_O + kDV * ob;
@@ -474,7 +474,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
               if (!issue_p(cur, t, kt + 1, kp)) { ok = false; break; }
               ++kp;
             } else if (nxt.valid) {
-              const int got = take_xf(nxt, t + 1, false);
+              const int got = take_xf(t + 1, false);
               if (got > 0) {
                 if (!issue_p(nxt, t + 1, 0, kp)) { ok = false; break; }
                 ++kp;
@@ -489,16 +489,16 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           if (!wait_bar(&B.p_conv[r], (k >> 1) & 1, B, p, SITE_TC_MMA, t)) { ok = false; break; }
           tc_fence_after();
           // O (+)= P_bf16 V over this key tile
-          const int kslot = (tpb == 2) ? kt : slot;
           const int ksteps = ((kt == u) ? nk : 128) / 16;
-          const uint64_t vd = desc_at(kDescMN, sbase + OFF_V + kslot * kVBytes);
+          const uint64_t vd = desc_at(kDescMN, sbase + OFF_V + kv_slot(t, u, kt) * kVBytes);
           const uint32_t pa = tmem + TM_P + 128 * r;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             if (kk < ksteps) mma_ts(od, pa + 8 * kk, vd + 128 * kk, kIdescPV, (kt > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&B.pv_done[r]);
           // The first tile's keys and values of a 256-block have no reader after this.
-          if (tpb == 2 && u == 1 && kt == 0) mma_commit_multicast(&B.empty[0], 0x3);
+          // Slot releases go to both CTAs: the partner writes its transformed boxes here.
+          if (kt < u) mma_commit_multicast(&B.kv_empty[kv_slot(t, u, kt)], 0x3);
           ++k;
         }
         if (!ok) break;
@@ -509,7 +509,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           tc_fence_after();
         }
         {
-          const uint64_t qd = desc_at(kDescK, sbase + OFF_Q + slot * kQBytes);
+          const uint64_t qd = desc_at(kDescK, sbase + OFF_Q + qs * kQBytes);
           const uint64_t sd = desc_at(kDescMN, sbase + OFF_SNAP);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -517,24 +517,19 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
                    kIdescQS, 1);
         }
         mma_commit(&B.o_full[ob]);
+        mma_commit_multicast(&B.q_empty[qs], 0x3);   // phi(Q) of this tile has no reader after this
         // S += phi(K)^T V
         {
-          const uint64_t kd = desc_at(kDescMN, sbase + OFF_K + slot * kKBytes);
-          const uint64_t vd = desc_at(kDescMN, sbase + OFF_V + slot * kVBytes);
+          const uint64_t kd = desc_at(kDescMN, sbase + OFF_K + ks * kKBytes);
+          const uint64_t vd = desc_at(kDescMN, sbase + OFF_V + ks * kVBytes);
           const int ksteps = nk / 16;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             if (kk < ksteps) mma_ss(tmem + TM_S, kd + 128 * kk, vd + 128 * kk, kIdescDS, 1);
         }
         const bool blk_end = (u == tpb - 1) || (cur.i == cur.nt - 1);
-        // Slot release goes to both CTAs: the partner writes its transformed box here.
-        if (tpb == 1) {
-          mma_commit_multicast(&B.empty[slot], 0x3);
-        } else if (u == 1) {
-          mma_commit_multicast(&B.empty[1], 0x3);
-        } else if (blk_end) {
-          mma_commit_multicast(&B.empty[0], 0x3);  // a block of one tile (sequence tail)
-        }
+        // This tile's keys and values are done unless the second tile of its block follows.
+        if (blk_end) mma_commit_multicast(&B.kv_empty[ks], 0x3);
         if (blk_end) mma_commit(&B.s_done);
         ++t;
         cur = nxt;
@@ -551,7 +546,6 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   // ------------------------------------------------------------------------------------
   else if (warp >= kXfWarp0 && warp < kXfWarp0 + kXfThreads / 32) {
     const int wt = tid - 32 * kXfWarp0;
-    uint32_t uses[2] = {0, 0};
     int t = 0;
     bool ok = true;
     for (int s = 0; s < p.nseq && ok; ++s) {
@@ -560,12 +554,11 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       seq_range(p, s, row0, L);
       const int nt = (L + kTile - 1) / kTile;
       for (int i = 0; i < nt; ++i) {
-        const int slot = (tpb == 2) ? (i & 1) : (t & 1);
-        if (!wait_bar_warp(&B.full_qkv[slot], uses[slot] & 1, B, p, SITE_TC_TRANSFORM, t)) { ok = false; break; }
-        uses[slot]++;
+        const int qs = t % kNQ, ks = t % kNKV;
+        if (!wait_bar_warp(&B.full_qkv[ks], (t / kNKV) & 1, B, p, SITE_TC_TRANSFORM, t)) { ok = false; break; }
         const int vr = min(kTile, L - i * kTile);
-        const uint32_t qa = sbase + OFF_Q + slot * kQBytes + dvt * kBoxBytes;
-        const uint32_t ka = sbase + OFF_K + slot * kKBytes + dvt * kBoxBytes;
+        const uint32_t qa = sbase + OFF_Q + qs * kQBytes + dvt * kBoxBytes;
+        const uint32_t ka = sbase + OFF_K + ks * kKBytes + dvt * kBoxBytes;
         // Chunks 0..1023 are this CTA's Q box, 1024..2047 its K box (16 bytes = 8 bf16).
         constexpr int kBoxChunks = kBoxBytes / 16;
 #pragma unroll 2
@@ -584,7 +577,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           st_cluster128(mapa_shared(addr, partner), v);
         }
         if (vr < kTile) {
-          const uint32_t va = sbase + OFF_V + slot * kVBytes;
+          const uint32_t va = sbase + OFF_V + ks * kVBytes;
           for (int c = wt; c < static_cast<int>(kVBytes / 16); c += kXfThreads) {
             const uint32_t off = static_cast<uint32_t>(c) * 16u;
             if (static_cast<int>(off >> 7) >= vr) sts128(va + off, make_uint4(0, 0, 0, 0));
@@ -592,8 +585,8 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         }
         // Local and remote writes become visible to both tensor cores before the arrivals.
         fence_proxy_async_cluster();
-        mbar_arrive(&B.xformed[slot]);
-        mbar_arrive_cluster(mapa_shared(smem_u32(&B.xformed[slot]), partner));
+        mbar_arrive(&B.xformed[ks]);
+        mbar_arrive_cluster(mapa_shared(smem_u32(&B.xformed[ks]), partner));
         ++t;
       }
     }
@@ -648,7 +641,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   }
   // ------------------------------------------------------------------------------------
   // Warps 12-15: epilogue readers.  Read O once, release the TMEM accumulator, add the
-  // rows' sums of squares into the fp64 per-token totals, park z = y * w * sigmoid(g).
+  // rows' sums of squares into the fp64 per-token totals, park z = y * w.
   // They also own the state: S0 into TMEM at each sequence start, the bf16 snapshot of S
   // at each block end, and the final state.
   // ------------------------------------------------------------------------------------
@@ -669,31 +662,30 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       // Initial state: S0 (or zeros) into TMEM and the bf16 snapshot.
       const int64_t st_row = ((static_cast<int64_t>(s) * p.H + h) * kD + wt) * kD + dvt * kDV;
       {
-        float v[kDV];
+        // 16 columns at a time: TMEM copy (fp32) and snapshot chunks 2j, 2j + 1 (bf16).
 #pragma unroll
-        for (int c = 0; c < kDV; c += 4) {
-          float4 x = p.state_in ? *reinterpret_cast<const float4*>(p.state_in + st_row + c) : make_float4(0, 0, 0, 0);
-          v[c] = x.x; v[c + 1] = x.y; v[c + 2] = x.z; v[c + 3] = x.w;
-        }
-        if (nt == 0) {
-          if (p.state_out)
-            for (int c = 0; c < kDV; c += 4)
-              *reinterpret_cast<float4*>(p.state_out + st_row + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-          continue;
-        }
-#pragma unroll
-        for (int c0 = 0; c0 < kDV; c0 += 16) {
+        for (int j = 0; j < kDV / 16; ++j) {
           uint32_t r[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(v[c0 + e]);
-          tmem_st16(tmem + lane_off + TM_S + c0, r);
-        }
+          for (int c = 0; c < 16; c += 4) {
+            const float4 x = p.state_in ? *reinterpret_cast<const float4*>(p.state_in + st_row + 16 * j + c)
+                                        : make_float4(0, 0, 0, 0);
+            r[c] = __float_as_uint(x.x); r[c + 1] = __float_as_uint(x.y);
+            r[c + 2] = __float_as_uint(x.z); r[c + 3] = __float_as_uint(x.w);
+          }
+          if (nt == 0) {
+            if (p.state_out)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 pk = make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]), pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
-                                pack_bf16x2(v[8 * c + 4], v[8 * c + 5]), pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
-          sts128(snap + sw128_offset(wt, c), pk);
+              for (int c = 0; c < 16; c += 4)
+                *reinterpret_cast<float4*>(p.state_out + st_row + 16 * j + c) =
+                    make_float4(__uint_as_float(r[c]), __uint_as_float(r[c + 1]), __uint_as_float(r[c + 2]),
+                                __uint_as_float(r[c + 3]));
+            continue;
+          }
+          tmem_st16(tmem + lane_off + TM_S + 16 * j, r);
+          store_snap16(snap, wt, j, r);
         }
+        if (nt == 0) continue;
         tmem_st_wait();
         fence_proxy_async_smem();
         tc_fence_before();
@@ -701,7 +693,6 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       }
       for (int i = 0; i < nt; ++i) {
         const int ob = t & 1;
-        const int gs = t % kNG;
         const int zs = t & 1;
         const int u = i % tpb;
         const int vr = min(kTile, L - i * kTile);
@@ -711,46 +702,40 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           ok = false;
           break;
         }
-        if (gate && !wait_bar_warp(&B.full_g[gs], (t / kNG) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
         tc_fence_after();
-        // O of this row, then the accumulator goes straight back to the MMA warp.
-        uint32_t x[2 * 32];
-        tmem_ld32(tmem + lane_off + TM_O + kDV * ob, *reinterpret_cast<uint32_t(*)[32]>(x));
-        tmem_ld32(tmem + lane_off + TM_O + kDV * ob + 32, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(&B.o_empty[ob]);
-        // z = y * w * sigmoid(g), parked as bf16 pairs in TMEM for the storer of this quarter.
-        const uint8_t* grow = smem + OFF_G + gs * kGBytes;
+        // z = y * w, parked as bf16 pairs in TMEM for the storer of this quarter; the
+        // accumulator goes back to the MMA warp as soon as it has been read.
         float ss = 0.f;
-        uint32_t z[32];
-#pragma unroll
-        for (int chunk = 0; chunk < 8; ++chunk) {
-          uint4 gv = make_uint4(0, 0, 0, 0);
-          if (gate) gv = *reinterpret_cast<const uint4*>(grow + sw128_offset(wt, chunk));
-          const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = 8 * chunk + 2 * e;
-            float a = __uint_as_float(x[col]);
-            float b = __uint_as_float(x[col + 1]);
-            ss = fmaf(a, a, ss);
-            ss = fmaf(b, b, ss);
-            if (norm) {
-              a *= B.w[col];
-              b *= B.w[col + 1];
-            }
-            if (gate) {
-              a *= sigmoid_fast(__uint_as_float(gw[e] << 16));
-              b *= sigmoid_fast(__uint_as_float(gw[e] & 0xFFFF0000u));
-            }
-            z[4 * chunk + e] = pack_bf16x2(a, b);
-          }
-        }
-        if (gate) mbar_arrive(&B.empty_g[gs]);
         const uint32_t zt = tmem + lane_off + TM_Z + 32 * zs;
-        tmem_st16(zt, *reinterpret_cast<const uint32_t(*)[16]>(z));
-        tmem_st16(zt + 16, *reinterpret_cast<const uint32_t(*)[16]>(z + 16));
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t zh[16];
+#pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            const int c0 = 32 * half + 16 * sub;   // first column of this group of 16
+            uint32_t x[16];
+            tmem_ld16(tmem + lane_off + TM_O + kDV * ob + c0, x);
+            tmem_ld_wait();
+            if (c0 == kDV - 16) {
+              tc_fence_before();
+              mbar_arrive(&B.o_empty[ob]);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int col = c0 + 2 * e;
+              float a = __uint_as_float(x[2 * e]);
+              float b = __uint_as_float(x[2 * e + 1]);
+              ss = fmaf(a, a, ss);
+              ss = fmaf(b, b, ss);
+              if (norm) {
+                a *= B.w[col];
+                b *= B.w[col + 1];
+              }
+              zh[8 * sub + e] = pack_bf16x2(a, b);
+            }
+          }
+          tmem_st16(zt + 16 * half, zh);
+        }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&B.z_full[zs][q]);
@@ -765,39 +750,26 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           if (!wait_bar_warp(&B.s_done, blk & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
           blk++;
           tc_fence_after();
-          uint32_t x0[32], x1[32];
-          tmem_ld32(tmem + lane_off + TM_S, x0);
-          tmem_ld32(tmem + lane_off + TM_S + 32, x1);
-          tmem_ld_wait();
-          if (i == nt - 1) {
-            if (p.state_out) {
+          const bool last = (i == nt - 1);
 #pragma unroll
-              for (int c = 0; c < 32; c += 4) {
-                *reinterpret_cast<float4*>(p.state_out + st_row + c) =
-                    make_float4(__uint_as_float(x0[c]), __uint_as_float(x0[c + 1]), __uint_as_float(x0[c + 2]),
-                                __uint_as_float(x0[c + 3]));
-                *reinterpret_cast<float4*>(p.state_out + st_row + 32 + c) =
-                    make_float4(__uint_as_float(x1[c]), __uint_as_float(x1[c + 1]), __uint_as_float(x1[c + 2]),
-                                __uint_as_float(x1[c + 3]));
-              }
+          for (int j = 0; j < kDV / 16; ++j) {
+            uint32_t r[16];
+            tmem_ld16(tmem + lane_off + TM_S + 16 * j, r);
+            tmem_ld_wait();
+            if (last) {
+              if (p.state_out)
+#pragma unroll
+                for (int c = 0; c < 16; c += 4)
+                  *reinterpret_cast<float4*>(p.state_out + st_row + 16 * j + c) =
+                      make_float4(__uint_as_float(r[c]), __uint_as_float(r[c + 1]), __uint_as_float(r[c + 2]),
+                                  __uint_as_float(r[c + 3]));
+            } else {
+              store_snap16(snap, wt, j, r);
             }
+          }
+          if (last) {
             tc_fence_before();
           } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint32_t* a = x0 + 8 * c;
-              const uint32_t* b = x1 + 8 * c;
-              sts128(snap + sw128_offset(wt, c),
-                     make_uint4(pack_bf16x2(__uint_as_float(a[0]), __uint_as_float(a[1])),
-                                pack_bf16x2(__uint_as_float(a[2]), __uint_as_float(a[3])),
-                                pack_bf16x2(__uint_as_float(a[4]), __uint_as_float(a[5])),
-                                pack_bf16x2(__uint_as_float(a[6]), __uint_as_float(a[7]))));
-              sts128(snap + sw128_offset(wt, c + 4),
-                     make_uint4(pack_bf16x2(__uint_as_float(b[0]), __uint_as_float(b[1])),
-                                pack_bf16x2(__uint_as_float(b[2]), __uint_as_float(b[3])),
-                                pack_bf16x2(__uint_as_float(b[4]), __uint_as_float(b[5])),
-                                pack_bf16x2(__uint_as_float(b[6]), __uint_as_float(b[7]))));
-            }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&B.snap_ready);
@@ -809,14 +781,14 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   }
   // ------------------------------------------------------------------------------------
   // Warps 16-19: epilogue storers, one per TMEM lane quarter (32 rows of every tile).
-  // Wait until every reader warp of every CTA has added its sums for the tile, read the
-  // parked z, scale it by rsqrt(mean(y^2) + eps) and store the quarter.
+  // Load the rows' gate values, read the parked z, wait until every reader warp of every
+  // CTA has added its sums for the tile, scale z by rsqrt(mean(y^2) + eps) * sigmoid(g)
+  // and store the rows from registers.
   // ------------------------------------------------------------------------------------
   else if (warp >= kStoreWarp0) {
     const int q = warp - kStoreWarp0;              // == warp % 4: the lane quarter it may access
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
-    const uint32_t stg = sbase + OFF_STG + q * kStgBytes;
-    const int HD = p.H * kD;
+    const int64_t HD = static_cast<int64_t>(p.H) * kD;
     const float inv_hd = 1.0f / static_cast<float>(HD);
     bool ok = true;
     int t = 0;
@@ -830,6 +802,22 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         const int vr = min(kTile, L - i * kTile);
         const int r = kQuarterRows * q + lane;     // row of the tile
         const int64_t row = row0 + static_cast<int64_t>(i) * kTile;
+        // This row's 64 gate values (bf16 pairs), loaded before the waits so that their
+        // latency overlaps them; the producer has prefetched the tile into L2.
+        uint32_t gq[32];
+        if (gate) {
+          if (r < vr) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.g + (row + r) * HD + h * kD + dvt * kDV);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint4 v = __ldg(src + c);
+              gq[4 * c] = v.x; gq[4 * c + 1] = v.y; gq[4 * c + 2] = v.z; gq[4 * c + 3] = v.w;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) gq[c] = 0;
+          }
+        }
         if (!wait_bar_warp(&B.z_full[zs][q], (t >> 1) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
         tc_fence_after();
         uint32_t z[32];
@@ -857,32 +845,26 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           if (!__shfl_sync(0xFFFFFFFFu, go, 0)) { ok = false; break; }
           (void)ld_acquire_gpu(c);
           const float rn = (r < vr) ? 1.0f / sqrtf(static_cast<float>(ld_cg_f64(p.ss + row + r)) * inv_hd + p.eps) : 0.0f;
+          if (gate) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            z[e] = pack_bf16x2(__uint_as_float(z[e] << 16) * rn, __uint_as_float(z[e] & 0xFFFF0000u) * rn);
-        }
-        if (kQuarterRows * (q + 1) <= vr) {
-          // The staging buffer is free once this warp's previous store has read it.
-          if (lane == 0) bulk_wait_read0();
-          __syncwarp();
+            for (int e = 0; e < 32; ++e)
+              z[e] = pack_bf16x2(__uint_as_float(z[e] << 16) * (rn * sigmoid_fast(__uint_as_float(gq[e] << 16))),
+                                 __uint_as_float(z[e] & 0xFFFF0000u) *
+                                     (rn * sigmoid_fast(__uint_as_float(gq[e] & 0xFFFF0000u))));
+          } else {
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            sts128(stg + sw128_offset(lane, c), make_uint4(z[4 * c], z[4 * c + 1], z[4 * c + 2], z[4 * c + 3]));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tm_o, smem + OFF_STG + q * kStgBytes, h * kD + dvt * kDV,
-                         static_cast<int32_t>(row + kQuarterRows * q));
-            bulk_commit();
+            for (int e = 0; e < 32; ++e)
+              z[e] = pack_bf16x2(__uint_as_float(z[e] << 16) * rn, __uint_as_float(z[e] & 0xFFFF0000u) * rn);
           }
-        } else if (r < vr) {
+        }
+        // Each lane writes its row's 128 contiguous bytes (the 64-column slice of the head).
+        if (r < vr) {
           uint4* dst = reinterpret_cast<uint4*>(p.out + (row + r) * HD + h * kD + dvt * kDV);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) dst[c] = make_uint4(z[4 * c], z[4 * c + 1], z[4 * c + 2], z[4 * c + 3]);
+          for (int c = 0; c < 8; ++c) st_global_na(dst + c, make_uint4(z[4 * c], z[4 * c + 1], z[4 * c + 2], z[4 * c + 3]));
         }
       }
     }
-    if (lane == 0) bulk_wait0();
   }
 
   // Teardown: all roles are done (or aborted with their async work drained).  The cluster
@@ -911,13 +893,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [rows, cols] bf16 row-major, box 64 columns x box_rows rows, 128-byte swizzle, zero fill.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows = kTile) {
+// [rows, cols] bf16 row-major, box 64 columns x 128 rows, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTile)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -994,15 +976,16 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
   p.tokens = a.tokens;
   p.eps = a.eps;
   p.w = a.w;
+  p.g = static_cast<const uint16_t*>(a.g);
   p.err = a.err;
   p.cnt = reinterpret_cast<unsigned int*>(a.ws);
   p.ss = reinterpret_cast<double*>(a.ws + cnt_bytes);
   p.out = static_cast<uint16_t*>(a.out);
 
   const int64_t cols = static_cast<int64_t>(a.H) * kD;
-  CUtensorMap mq, mk, mv, mg, mo;
+  CUtensorMap mq, mk, mv, mg;
   if (!make_map(&mq, a.q, a.tokens, cols) || !make_map(&mk, a.k, a.tokens, cols) ||
-      !make_map(&mv, a.v, a.tokens, cols) || !make_map(&mo, a.out, a.tokens, cols, kQuarterRows))
+      !make_map(&mv, a.v, a.tokens, cols))
     return cudaErrorInvalidValue;
   if (a.mode == LA_OUT_RMSNORM_GATE) {
     if (!make_map(&mg, a.g, a.tokens, cols)) return cudaErrorInvalidValue;
@@ -1027,7 +1010,7 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, lightning_prefill_tc_kernel, mq, mk, mv, mg, mo, p);
+  e = cudaLaunchKernelEx(&cfg, lightning_prefill_tc_kernel, mq, mk, mv, mg, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
