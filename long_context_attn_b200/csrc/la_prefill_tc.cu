@@ -90,7 +90,7 @@ constexpr uint32_t TM_P = 256;    // 2 score tiles x 128 columns
 constexpr uint32_t kTmemCols = 512;
 
 struct Bars {
-  uint64_t full_qkv[kNKV], xformed[kNKV], kv_empty[kNKV], q_empty[kNQ];
+  uint64_t full_q[kNQ], q_empty[kNQ], full_kv[kNKV], kv_empty[kNKV], xformed[kNKV];
   uint64_t p_full[2], p_conv[2], pv_done[2];   // per TMEM score region
   uint64_t o_full[2], o_empty[2];
   uint64_t s_done, snap_ready, final_bar;
@@ -312,11 +312,14 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
 
   if (tid == 0) {
     for (int i = 0; i < kNKV; ++i) {
-      mbar_init(&B.full_qkv[i], 1);
+      mbar_init(&B.full_kv[i], 1);
       mbar_init(&B.xformed[i], 2 * kXfThreads);   // both CTAs' transform threads
       mbar_init(&B.kv_empty[i], 2);               // both CTAs' MMAs released the slot
     }
-    for (int i = 0; i < kNQ; ++i) mbar_init(&B.q_empty[i], 2);
+    for (int i = 0; i < kNQ; ++i) {
+      mbar_init(&B.full_q[i], 1);
+      mbar_init(&B.q_empty[i], 2);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&B.o_full[i], 1);
       mbar_init(&B.o_empty[i], 128);
@@ -347,18 +350,25 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   const uint32_t tmem = B.tmem_base;
 
   // ------------------------------------------------------------------------------------
-  // Warp 0, lane 0: TMA producer.  Tile t's Q box goes to Q slot t % 2, its K box and V
-  // slice to K/V slot t % 3; the gate tile is only prefetched into L2 (the readers load
-  // their rows of it straight from global memory).
+  // Warp 0: TMA producers.  Lane 0 streams this CTA's 64-column Q boxes into Q slot
+  // t % 2; lane 1 streams its K boxes and V slices into K/V slot t % 3 and prefetches the
+  // gate tile into L2 (the storers load their rows of it straight from global memory).
+  // The partner CTA supplies the other box of Q and K.  The two rings run independently,
+  // so keys and values run ahead of the queries whenever their slots free up earlier.
   // ------------------------------------------------------------------------------------
   if (warp == 0) {
-    if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      if (gate) prefetch_tmap(&tm_g);
+    if (lane < 2) {
+      const bool is_q = lane == 0;
+      if (is_q) {
+        prefetch_tmap(&tm_q);
+      } else {
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        if (gate) prefetch_tmap(&tm_g);
+      }
       const uint64_t pol = policy_evict_first();
-      uint32_t qu[kNQ] = {0, 0}, ku[kNKV] = {0, 0, 0};
+      const int nslots = is_q ? kNQ : kNKV;
+      uint32_t uses[kNKV] = {0, 0, 0};
       int t = 0;
       bool ok = true;
       for (int s = 0; s < p.nseq && ok; ++s) {
@@ -367,33 +377,31 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         seq_range(p, s, row0, L);
         const int nt = (L + kTile - 1) / kTile;
         for (int i = 0; i < nt; ++i) {
-          const int qs = t % kNQ, ks = t % kNKV;
-          if (qu[qs] > 0 && !wait_bar(&B.q_empty[qs], (qu[qs] - 1) & 1, B, p, SITE_TC_PRODUCER, t)) {
-            ok = false;
-            break;
-          }
-          if (ku[ks] > 0 && !wait_bar(&B.kv_empty[ks], (ku[ks] - 1) & 1, B, p, SITE_TC_PRODUCER, t)) {
+          const int sl = t % nslots;
+          uint64_t* empty = is_q ? &B.q_empty[sl] : &B.kv_empty[sl];
+          if (uses[sl] > 0 && !wait_bar(empty, (uses[sl] - 1) & 1, B, p, SITE_TC_PRODUCER, t)) {
             ok = false;
             break;
           }
           const int32_t row = static_cast<int32_t>(row0 + static_cast<int64_t>(i) * kTile);
-          // This CTA's 64-column boxes of Q and K (the partner supplies the other box) and
-          // its V slice.
-          mbar_arrive_expect_tx(&B.full_qkv[ks], 2 * kBoxBytes + kVBytes);
-          uint8_t* qd = smem + OFF_Q + qs * kQBytes + dvt * kBoxBytes;
-          uint8_t* kd = smem + OFF_K + ks * kKBytes + dvt * kBoxBytes;
-          tma_load_2d(qd, &tm_q, h * kD + dvt * 64, row, &B.full_qkv[ks], pol);
-          tma_load_2d(kd, &tm_k, h * kD + dvt * 64, row, &B.full_qkv[ks], pol);
-          tma_load_2d(smem + OFF_V + ks * kVBytes, &tm_v, h * kD + dvt * kDV, row, &B.full_qkv[ks], pol);
-          if (gate) tma_prefetch_l2_2d(&tm_g, h * kD + dvt * kDV, row);
-          qu[qs]++;
-          ku[ks]++;
+          if (is_q) {
+            mbar_arrive_expect_tx(&B.full_q[sl], kBoxBytes);
+            tma_load_2d(smem + OFF_Q + sl * kQBytes + dvt * kBoxBytes, &tm_q, h * kD + dvt * 64, row, &B.full_q[sl],
+                        pol);
+          } else {
+            mbar_arrive_expect_tx(&B.full_kv[sl], kBoxBytes + kVBytes);
+            tma_load_2d(smem + OFF_K + sl * kKBytes + dvt * kBoxBytes, &tm_k, h * kD + dvt * 64, row, &B.full_kv[sl],
+                        pol);
+            tma_load_2d(smem + OFF_V + sl * kVBytes, &tm_v, h * kD + dvt * kDV, row, &B.full_kv[sl], pol);
+            if (gate) tma_prefetch_l2_2d(&tm_g, h * kD + dvt * kDV, row);
+          }
+          uses[sl]++;
           ++t;
         }
       }
       // Drain: every issued load must have landed before the CTA may exit.
-      for (int i = 0; i < kNKV; ++i)
-        if (ku[i] > 0) drain_bar(&B.full_qkv[i], (ku[i] - 1) & 1);
+      for (int i = 0; i < nslots; ++i)
+        if (uses[i] > 0) drain_bar(is_q ? &B.full_q[i] : &B.full_kv[i], (uses[i] - 1) & 1);
     }
   }
   // ------------------------------------------------------------------------------------
@@ -542,53 +550,80 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   }
   // ------------------------------------------------------------------------------------
   // Warps 2-7: SiLU of this CTA's Q and K boxes, written to both CTAs of the pair; zero
-  // tail rows of K (both copies) and of this CTA's V slice.
+  // tail rows of K (both copies) and of this CTA's V slice.  Keys are transformed as soon
+  // as they land (one tile ahead when possible), so only the query box stands between a
+  // query slot's load and the MMAs that free it.
   // ------------------------------------------------------------------------------------
   else if (warp >= kXfWarp0 && warp < kXfWarp0 + kXfThreads / 32) {
     const int wt = tid - 32 * kXfWarp0;
-    int t = 0;
-    bool ok = true;
-    for (int s = 0; s < p.nseq && ok; ++s) {
-      int64_t row0;
-      int L;
-      seq_range(p, s, row0, L);
-      const int nt = (L + kTile - 1) / kTile;
-      for (int i = 0; i < nt; ++i) {
-        const int qs = t % kNQ, ks = t % kNKV;
-        if (!wait_bar_warp(&B.full_qkv[ks], (t / kNKV) & 1, B, p, SITE_TC_TRANSFORM, t)) { ok = false; break; }
-        const int vr = min(kTile, L - i * kTile);
-        const uint32_t qa = sbase + OFF_Q + qs * kQBytes + dvt * kBoxBytes;
-        const uint32_t ka = sbase + OFF_K + ks * kKBytes + dvt * kBoxBytes;
-        // Chunks 0..1023 are this CTA's Q box, 1024..2047 its K box (16 bytes = 8 bf16).
-        constexpr int kBoxChunks = kBoxBytes / 16;
-#pragma unroll 2
-        for (int c = wt; c < 2 * kBoxChunks; c += kXfThreads) {
-          const bool is_k = c >= kBoxChunks;
-          const uint32_t off = static_cast<uint32_t>(is_k ? c - kBoxChunks : c) * 16u;
-          const uint32_t addr = (is_k ? ka : qa) + off;
-          const int row = static_cast<int>(off >> 7);
-          uint4 v = lds128(addr);
-          if (is_k && row >= vr) {
-            v = make_uint4(0, 0, 0, 0);
-          } else if (!p.phi_identity) {
-            v.x = silu_bf16x2(v.x); v.y = silu_bf16x2(v.y); v.z = silu_bf16x2(v.z); v.w = silu_bf16x2(v.w);
-          }
-          sts128(addr, v);
-          st_cluster128(mapa_shared(addr, partner), v);
+    constexpr int kBoxChunks = static_cast<int>(kBoxBytes / 16);   // 16 bytes = 8 bf16
+    // The partner's shared window maps this CTA's offsets one to one.
+    const uint32_t remote = mapa_shared(sbase, partner);
+    // SiLU of one 128 x 64 box in place, mirrored into the partner; rows >= zero_from are
+    // zeroed instead.  Four chunks per thread are loaded before any is stored.
+    auto xf_box = [&](uint32_t off0, int zero_from) {
+      for (int c0 = wt; c0 < kBoxChunks; c0 += 4 * kXfThreads) {
+        uint4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = c0 + j * kXfThreads;
+          v[j] = (c < kBoxChunks) ? lds128(sbase + off0 + 16u * c) : make_uint4(0, 0, 0, 0);
         }
-        if (vr < kTile) {
-          const uint32_t va = sbase + OFF_V + ks * kVBytes;
-          for (int c = wt; c < static_cast<int>(kVBytes / 16); c += kXfThreads) {
-            const uint32_t off = static_cast<uint32_t>(c) * 16u;
-            if (static_cast<int>(off >> 7) >= vr) sts128(va + off, make_uint4(0, 0, 0, 0));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = c0 + j * kXfThreads;
+          if (c < kBoxChunks) {
+            uint4 x = v[j];
+            if ((c >> 3) >= zero_from) {
+              x = make_uint4(0, 0, 0, 0);
+            } else if (!p.phi_identity) {
+              x.x = silu_bf16x2(x.x); x.y = silu_bf16x2(x.y); x.z = silu_bf16x2(x.z); x.w = silu_bf16x2(x.w);
+            }
+            sts128(sbase + off0 + 16u * c, x);
+            st_cluster128(remote + off0 + 16u * c, x);
           }
         }
-        // Local and remote writes become visible to both tensor cores before the arrivals.
-        fence_proxy_async_cluster();
-        mbar_arrive(&B.xformed[ks]);
-        mbar_arrive_cluster(mapa_shared(smem_u32(&B.xformed[ks]), partner));
-        ++t;
       }
+    };
+    // Keys (and the zeroed tail of the values) of tile tt.
+    auto xf_keys = [&](const TileIter& it, int tt) {
+      const int ks = tt % kNKV;
+      const int vr = min(kTile, it.L - it.i * kTile);
+      xf_box(OFF_K + ks * kKBytes + dvt * kBoxBytes, vr);
+      if (vr < kTile) {
+        const uint32_t va = sbase + OFF_V + ks * kVBytes;
+        for (int c = wt; c < static_cast<int>(kVBytes / 16); c += kXfThreads)
+          if ((c >> 3) >= vr) sts128(va + 16u * c, make_uint4(0, 0, 0, 0));
+      }
+    };
+    TileIter cur, nxt;
+    tile_first(p, cur);
+    nxt = cur;
+    tile_next(p, nxt);
+    int t = 0;
+    int k_done = -1;   // last tile whose keys this thread has transformed
+    while (cur.valid) {
+      const int qs = t % kNQ, ks = t % kNKV;
+      if (k_done < t) {
+        if (!wait_bar_warp(&B.full_kv[ks], (t / kNKV) & 1, B, p, SITE_TC_TRANSFORM, t)) break;
+        xf_keys(cur, t);
+        k_done = t;
+      }
+      if (!wait_bar_warp(&B.full_q[qs], (t / kNQ) & 1, B, p, SITE_TC_TRANSFORM, t)) break;
+      xf_box(OFF_Q + qs * kQBytes + dvt * kBoxBytes, kTile);
+      // Local and remote writes become visible to both tensor cores before the arrivals.
+      fence_proxy_async_cluster();
+      mbar_arrive(&B.xformed[ks]);
+      mbar_arrive_cluster(mapa_shared(smem_u32(&B.xformed[ks]), partner));
+      // The next tile's keys, if they have landed already.
+      if (nxt.valid &&
+          __all_sync(0xFFFFFFFFu, mbar_test_wait(&B.full_kv[(t + 1) % kNKV], ((t + 1) / kNKV) & 1))) {
+        xf_keys(nxt, t + 1);
+        k_done = t + 1;
+      }
+      ++t;
+      cur = nxt;
+      tile_next(p, nxt);
     }
   }
   // ------------------------------------------------------------------------------------
