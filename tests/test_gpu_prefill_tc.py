@@ -136,3 +136,34 @@ def test_tc_config_8k(cuda_device):
     assert stats["out_nonfinite"] == 0 and stats["state_nonfinite"] == 0
     assert stats["out_max_err"] <= 2e-2 * stats["out_max_ref"], stats
     assert stats["state_max_err"] <= 2e-2 * stats["state_max_ref"], stats
+
+
+@pytest.mark.slow
+def test_tc_config_128k_full(cuda_device):
+    """B1 H64 T131072 D128 bf16, block 256, gated concat RMSNorm, final state: every output
+    element and every state element against the fp64 oracle (streamed, not stored)."""
+    w = synth.WORKLOADS["prefill_128k"]
+    q, k, v, g = synth.prefill_inputs(w.seed, w.T, w.H, w.D, "bf16", w.qkv_scale, True)
+    o, st, _ = run_prefill(q[None], k[None], v[None], g[None], w.block_size, oracle.MODE_RMSNORM_GATE,
+                           want_state=True, expect_path="tcgen05")
+    _, _, stats = oracle.prefill(q[None], k[None], v[None], g[None], store=False, cand_out=o, cand_state=st)
+    assert stats["out_nonfinite"] == 0 and stats["state_nonfinite"] == 0
+    assert stats["out_max_err"] <= 2e-2 * stats["out_max_ref"], stats
+    assert stats["state_max_err"] <= 2e-2 * stats["state_max_ref"], stats
+
+
+@pytest.mark.slow
+def test_tc_config_varlen16_full(cuda_device):
+    """16 packed sequences, lengths ~ U{1000..32768}, block 256 with 32/64/128 tail pads,
+    gated concat RMSNorm, per-sequence final states: full compare against the oracle."""
+    w = synth.WORKLOADS["varlen_16"]
+    lens = synth.varlen_lengths(w)
+    tot = int(lens.sum())
+    q, k, v, g = synth.prefill_inputs(w.seed, tot, w.H, w.D, "bf16", w.qkv_scale, True)
+    o, st, _ = run_varlen(q, k, v, g, lens, w.block_size, oracle.MODE_RMSNORM_GATE, want_state=True,
+                          expect_path="tcgen05")
+    _, _, stats = oracle.forward_packed(q, k, v, g, synth.cu_seqlens_of(lens), w.H, w.D, store=False,
+                                        cand_out=o, cand_state=st)
+    assert stats["out_nonfinite"] == 0 and stats["state_nonfinite"] == 0
+    assert stats["out_max_err"] <= 2e-2 * stats["out_max_ref"], stats
+    assert stats["state_max_err"] <= 2e-2 * stats["state_max_ref"], stats
