@@ -263,10 +263,95 @@ class DecodeCase:
                 "l2": "state larger than L2 (1 GiB read + written per step), no flush"}
 
 
+class VarlenCase:
+    """16 packed sequences (lengths ~ U{1000..32768}), cu_seqlens on the device, block 256
+    with 32/64/128 tail pads, gated concat RMSNorm, per-sequence final states."""
+
+    def __init__(self, name, w, device, rank):
+        import torch
+        from long_context_attn_b200 import lightning_attn as la
+        self.la, self.w = la, w
+        H, D = w.H, w.D
+        self.lens = synth.varlen_lengths(w)
+        self.n = len(self.lens)
+        self.total = int(self.lens.sum())
+        self.max_len = int(self.lens.max())
+        t0 = time.time()
+        q, k, v, g = synth.prefill_inputs(w.seed + 1000 * rank, self.total, H, D, "bf16", w.qkv_scale, True)
+        self.gen_s = time.time() - t0
+
+        def pin(a):
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+        self.h_q, self.h_k, self.h_v, self.h_g = (pin(a) for a in (q, k, v, g))
+        del q, k, v, g
+        self.q = self.h_q.to(device).view(self.total, H, D)
+        self.k = self.h_k.to(device).view(self.total, H, D)
+        self.v = self.h_v.to(device).view(self.total, H, D)
+        self.g = self.h_g.to(device).view(self.total, H * D)
+        self.cu = torch.from_numpy(synth.cu_seqlens_of(self.lens)).to(device)
+        self.out = torch.empty((self.total, H * D), dtype=torch.bfloat16, device=device)
+        self.state = torch.empty((self.n, H, D, D), dtype=torch.float32, device=device)
+        self.h_out = torch.empty((self.total, H * D), dtype=torch.bfloat16).pin_memory()
+        self.h_state = torch.empty((self.n, H, D, D), dtype=torch.float32).pin_memory()
+        self.ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_PREFILL_VARLEN, self.n, self.max_len,
+                                                                    self.total, H, D, w.block_size, la.LA_BF16,
+                                                                    la.LA_OUT_RMSNORM_GATE), device)
+        self.tokens = self.total
+        self.alg_bytes = self.total * _bytes_per_token(H, D) + self.n * H * D * D * 4
+        self.alg_flops, self.issued_flops = (x * self.total for x in _flops_per_token(H, D, w.block_size))
+        self.h2d = sum(t.numel() * t.element_size() for t in (self.h_q, self.h_k, self.h_v, self.h_g))
+        self.d2h = self.h_out.numel() * 2 + self.h_state.numel() * 4
+        # Rows the tail pads add (per sequence: the last block's r = L mod C rows run at the
+        # smallest of 32/64/128 that holds them, else at C).
+        C = w.block_size
+        pad = 0
+        for L in self.lens.tolist():
+            r = L % C
+            if r:
+                p = next((x for x in (32, 64, 128) if x >= r and x < C), C)
+                pad += p - r
+        self.padded_rows = pad
+
+    def step(self):
+        self.la.lightning_attn_prefill_varlen(self.q, self.k, self.v, self.g, self.out, self.cu, self.max_len,
+                                              None, self.state, block_size=self.w.block_size, workspace=self.ws)
+
+    def e2e_step(self):
+        self.q.view(-1).copy_(self.h_q.view(-1), non_blocking=True)
+        self.k.view(-1).copy_(self.h_k.view(-1), non_blocking=True)
+        self.v.view(-1).copy_(self.h_v.view(-1), non_blocking=True)
+        self.g.view(-1).copy_(self.h_g.view(-1), non_blocking=True)
+        self.step()
+        self.h_out.copy_(self.out, non_blocking=True)
+        self.h_state.copy_(self.state, non_blocking=True)
+
+    def check(self):
+        self.la.lightning_attn_check(self.ws)
+
+    def oracle_sample(self, tokens):
+        """fp64 oracle on the first `tokens` rows of the first sequence (all heads)."""
+        import oracle
+        w = self.w
+        n = min(tokens, int(self.lens[0]))
+        q, k, v, g = synth.prefill_inputs(w.seed, n, w.H, w.D, "bf16", w.qkv_scale, True)
+        t0 = time.perf_counter()
+        oracle.prefill(q[None], k[None], v[None], g[None], store=False)
+        return time.perf_counter() - t0, n
+
+    def describe(self):
+        return {"workload": self.w.name, "N": self.n, "total_tokens": self.total, "max_len": self.max_len,
+                "H": self.w.H, "D": self.w.D, "block_size": self.w.block_size, "mode": "rmsnorm_gate",
+                "state_out": True, "padded_rows": self.padded_rows,
+                "l2": "inputs larger than L2 (%.1f GB per step), no flush" % (self.alg_bytes / 1e9)}
+
+
 def _make_case(name, device, rank):
     w = synth.WORKLOADS[name]
     if w.kind == "prefill" and w.dtype == "bf16":
         return PrefillCase(name, w, device, rank)
+    if w.kind == "varlen":
+        return VarlenCase(name, w, device, rank)
     if w.kind == "decode":
         return DecodeCase(name, w, device, rank)
     raise SystemExit(f"workload {name} is not a bench workload")
@@ -407,11 +492,16 @@ def _traffic(workload):
 def _cpu_baseline(case):
     import oracle
     if isinstance(case, PrefillCase):
-        n = 4096
+        n = 65536
         dt = case.oracle_sample(n)
         return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
                 "sample": f"first {n} tokens of the {case.w.name} workload, all {case.H} heads, fp64, "
                           f"recurrence + norm + gate ({dt:.1f} s)"}
+    if isinstance(case, VarlenCase):
+        dt, n = case.oracle_sample(65536)
+        return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                "sample": f"first {n} tokens of sequence 0 of the {case.w.name} workload, all {case.w.H} heads, "
+                          f"fp64, recurrence + norm + gate ({dt:.1f} s)"}
     n = 64
     dt = case.oracle_sample(n)
     return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
@@ -425,7 +515,7 @@ def run_reference(args):
         return
     import oracle
     w = synth.WORKLOADS[args.workload]
-    if w.kind == "prefill":
+    if w.kind in ("prefill", "varlen"):
         n = 1024
         q, k, v, g = synth.prefill_inputs(w.seed, n, w.H, w.D, w.dtype, w.qkv_scale, True)
 
@@ -467,7 +557,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="prefill_128k", choices=["prefill_8k", "prefill_128k", "decode_256"])
+    ap.add_argument("--workload", default="prefill_128k",
+                    choices=["prefill_8k", "prefill_128k", "varlen_16", "decode_256"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     args = ap.parse_args()
