@@ -358,6 +358,24 @@ def _make_case(name, device, rank):
 
 
 # ----------------------------------------------------------------------------------------------
+# Multi-rank helpers (one process per GPU; the job's time is its slowest rank's)
+# ----------------------------------------------------------------------------------------------
+def _max_over_ranks(vals, world, device=None):
+    """Element-wise maximum of `vals` over all ranks of the default process group."""
+    import torch
+    t = torch.tensor([float(x) for x in vals], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def _job_value(units_per_rank_step, steps, world, elapsed_ms):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank_step * steps * world / (elapsed_ms / 1e3)
+
+
+# ----------------------------------------------------------------------------------------------
 # Arms
 # ----------------------------------------------------------------------------------------------
 def run_gpu(args):
@@ -404,10 +422,7 @@ def run_gpu(args):
     case.check()
     elapsed_ms = e0.elapsed_time(e1)
     launch_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
-    t = torch.tensor([elapsed_ms, launch_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, launch_ms = float(t[0]), float(t[1])
+    elapsed_ms, launch_ms = _max_over_ranks([elapsed_ms, launch_ms], world, device)
 
     # ---- end-to-end through the C ABI with pinned host buffers ----
     for _ in range(min(2, args.warmup)):
@@ -422,15 +437,11 @@ def run_gpu(args):
     torch.cuda.synchronize()
     barrier()
     case.check()
-    t = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t[0])
+    e2e_ms = _max_over_ranks([f0.elapsed_time(f1)], world, device)[0]
 
     if rank == 0:
         peaks = _peaks()
-        tokens_total = case.tokens * args.steps * world
-        value = tokens_total / (elapsed_ms / 1e3)
+        value = _job_value(case.tokens, args.steps, world, elapsed_ms)
         achieved_gbs = case.alg_bytes / (launch_ms / 1e3) / 1e9
         line = {
             "metric": METRIC if args.workload == "prefill_128k" else f"lightning-attn {args.workload} tokens/s",
@@ -447,7 +458,7 @@ def run_gpu(args):
                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                        "frac_algorithmic": case.alg_flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
                        "frac_issued": case.issued_flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
-            "e2e": {"value": case.tokens * args.steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
+            "e2e": {"value": _job_value(case.tokens, args.steps, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": case.h2d, "d2h_bytes_per_step": case.d2h},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
