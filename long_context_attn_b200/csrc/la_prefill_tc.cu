@@ -32,9 +32,10 @@
 //    Score tiles alternate between two TMEM regions so that P of the next key/query tile
 //    is computed while the current one is being converted.
 //  * A conversion warpgroup turns P (fp32, TMEM) into masked bf16 in place.
-//  * The epilogue reader warpgroup owns the state (S0 in, the bf16 snapshot of S at each
-//    block end, the final state out) and reads O once, releasing the accumulator at once:
-//    it parks z = y * w as bf16 pairs in two spare TMEM tiles, adds each row's sum of
+//  * The kernel is instantiated per output mode.  The epilogue reader warpgroup owns the
+//    state (S0 in, the bf16 snapshot of S at each block end, the final state out) and reads
+//    O once, releasing the accumulator at once.  In the raw mode it stores y directly.  In
+//    the norm modes it parks z = y * w as bf16 pairs in two spare TMEM tiles, adds each row's sum of
 //    squares into an fp64 per-token accumulator in global memory (red.add; the fp64 sum of
 //    the fp32 partials is exact whenever a token's partials span less than 2^22, so the
 //    result does not depend on the order the additions land in) and bumps the tile's
@@ -289,6 +290,9 @@ __device__ __forceinline__ void red_add_f64(double* p, double v) {
 // ======================================================================================
 // The kernel
 // ======================================================================================
+// One instantiation per output mode (la_out_mode), so that each mode's roles compile to
+// straight-line code.
+template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
 lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -306,8 +310,8 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   const int dvt = static_cast<int>(cluster_ctarank());   // == blockIdx.x % 2 (cluster of 2)
   const uint32_t partner = static_cast<uint32_t>(dvt ^ 1);
   const int tpb = p.C / kTile;           // tiles per block (1 or 2)
-  const bool norm = p.mode != LA_OUT_RAW;
-  const bool gate = p.mode == LA_OUT_RMSNORM_GATE;
+  constexpr bool norm = kMode != LA_OUT_RAW;
+  constexpr bool gate = kMode == LA_OUT_RMSNORM_GATE;
   const int W = p.H * kNdv * 4;          // reader warps contributing to one tile's norm
 
   if (tid == 0) {
@@ -685,6 +689,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     const int q = warp - kReadWarp0;               // lane quarter
     const uint32_t lane_off = static_cast<uint32_t>(wt & ~31) << 16;
     const uint32_t snap = sbase + OFF_SNAP;
+    const int64_t HD = static_cast<int64_t>(p.H) * kD;
     const bool skip_publish = (p.err->inject == INJECT_SKIP_PUBLISH) && blockIdx.x == 0;
     bool ok = true;
     int t = 0;
@@ -733,15 +738,17 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         const int vr = min(kTile, L - i * kTile);
         const int64_t row = row0 + static_cast<int64_t>(i) * kTile;
         if (!wait_bar_warp(&B.o_full[ob], (t >> 1) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
-        if (t >= 2 && !wait_bar_warp(&B.z_free[zs][q], ((t >> 1) - 1) & 1, B, p, SITE_TC_EPILOGUE, t)) {
+        if (norm && t >= 2 && !wait_bar_warp(&B.z_free[zs][q], ((t >> 1) - 1) & 1, B, p, SITE_TC_EPILOGUE, t)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        // z = y * w, parked as bf16 pairs in TMEM for the storer of this quarter; the
-        // accumulator goes back to the MMA warp as soon as it has been read.
+        // Norm modes: z = y * w, parked as bf16 pairs in TMEM for the storer of this
+        // quarter.  Raw mode: y is the output and goes straight from here to global memory.
+        // The accumulator goes back to the MMA warp as soon as it has been read.
         float ss = 0.f;
         const uint32_t zt = tmem + lane_off + TM_Z + 32 * zs;
+        uint4* zdst = reinterpret_cast<uint4*>(p.out + (row + wt) * HD + h * kD + dvt * kDV);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t zh[16];
@@ -769,11 +776,19 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
               zh[8 * sub + e] = pack_bf16x2(a, b);
             }
           }
-          tmem_st16(zt + 16 * half, zh);
+          if (norm) {
+            tmem_st16(zt + 16 * half, zh);
+          } else if (wt < vr) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              zdst[4 * half + c] = make_uint4(zh[4 * c], zh[4 * c + 1], zh[4 * c + 2], zh[4 * c + 3]);
+          }
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&B.z_full[zs][q]);
+        if (norm) {
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&B.z_full[zs][q]);
+        }
         if (norm) {
           if (wt < vr) red_add_f64(p.ss + row + wt, static_cast<double>(ss));
           __syncwarp();
@@ -815,12 +830,12 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     }
   }
   // ------------------------------------------------------------------------------------
-  // Warps 16-19: epilogue storers, one per TMEM lane quarter (32 rows of every tile).
+  // Warps 16-19 (norm modes): epilogue storers, one per TMEM lane quarter (32 rows of every tile).
   // Load the rows' gate values, read the parked z, wait until every reader warp of every
   // CTA has added its sums for the tile, scale z by rsqrt(mean(y^2) + eps) * sigmoid(g)
   // and store the rows from registers.
   // ------------------------------------------------------------------------------------
-  else if (warp >= kStoreWarp0) {
+  else if (warp >= kStoreWarp0 && norm) {
     const int q = warp - kStoreWarp0;              // == warp % 4: the lane quarter it may access
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
     const int64_t HD = static_cast<int64_t>(p.H) * kD;
@@ -954,7 +969,7 @@ int max_active_clusters() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   std::lock_guard<std::mutex> lock(mu);
   if (cache[dev] == 0) {
-    if (cudaFuncSetAttribute(lightning_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess)
       return 0;
     cudaLaunchConfig_t cfg = {};
@@ -969,7 +984,8 @@ int max_active_clusters() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, lightning_prefill_tc_kernel, &cfg) != cudaSuccess) n = -1;
+    if (cudaOccupancyMaxActiveClusters(&n, lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE>, &cfg) != cudaSuccess)
+      n = -1;
     cache[dev] = n;
   }
   return cache[dev];
@@ -1030,8 +1046,10 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
   // Arrival counters and the fp64 sums start at zero on every call.
   cudaError_t e = cudaMemsetAsync(a.ws, 0, cnt_bytes + (a.mode != LA_OUT_RAW ? ss_bytes : 0), stream);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(lightning_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kSmemBytes));
+  auto kernel = a.mode == LA_OUT_RAW       ? lightning_prefill_tc_kernel<LA_OUT_RAW>
+                : a.mode == LA_OUT_RMSNORM ? lightning_prefill_tc_kernel<LA_OUT_RMSNORM>
+                                           : lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE>;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.H * kNdv);
@@ -1045,7 +1063,7 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, lightning_prefill_tc_kernel, mq, mk, mv, mg, p);
+  e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mv, mg, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
