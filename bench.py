@@ -503,13 +503,13 @@ def _traffic(workload):
 def _cpu_baseline(case):
     import oracle
     if isinstance(case, PrefillCase):
-        n = 65536
+        n = min(131072, case.T)
         dt = case.oracle_sample(n)
         return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
                 "sample": f"first {n} tokens of the {case.w.name} workload, all {case.H} heads, fp64, "
                           f"recurrence + norm + gate ({dt:.1f} s)"}
     if isinstance(case, VarlenCase):
-        dt, n = case.oracle_sample(65536)
+        dt, n = case.oracle_sample(131072)
         return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
                 "sample": f"first {n} tokens of sequence 0 of the {case.w.name} workload, all {case.w.H} heads, "
                           f"fp64, recurrence + norm + gate ({dt:.1f} s)"}
