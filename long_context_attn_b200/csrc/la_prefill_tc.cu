@@ -290,9 +290,9 @@ __device__ __forceinline__ void red_add_f64(double* p, double v) {
 // ======================================================================================
 // The kernel
 // ======================================================================================
-// One instantiation per output mode (la_out_mode), so that each mode's roles compile to
-// straight-line code.
-template <int kMode>
+// One instantiation per output mode (la_out_mode) and block size (128 or 256 rows), so
+// that each variant's roles compile to straight-line code.
+template <int kMode, int kC>
 __global__ void __launch_bounds__(kThreads, 1)
 lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -309,7 +309,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   const int h = blockIdx.x / kNdv;
   const int dvt = static_cast<int>(cluster_ctarank());   // == blockIdx.x % 2 (cluster of 2)
   const uint32_t partner = static_cast<uint32_t>(dvt ^ 1);
-  const int tpb = p.C / kTile;           // tiles per block (1 or 2)
+  constexpr int tpb = kC / kTile;        // tiles per block (1 or 2)
   constexpr bool norm = kMode != LA_OUT_RAW;
   constexpr bool gate = kMode == LA_OUT_RMSNORM_GATE;
   const int W = p.H * kNdv * 4;          // reader warps contributing to one tile's norm
@@ -969,7 +969,8 @@ int max_active_clusters() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   std::lock_guard<std::mutex> lock(mu);
   if (cache[dev] == 0) {
-    if (cudaFuncSetAttribute(lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 256>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess)
       return 0;
     cudaLaunchConfig_t cfg = {};
@@ -984,7 +985,8 @@ int max_active_clusters() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE>, &cfg) != cudaSuccess)
+    if (cudaOccupancyMaxActiveClusters(&n, lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 256>, &cfg) !=
+        cudaSuccess)
       n = -1;
     cache[dev] = n;
   }
@@ -1046,9 +1048,12 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
   // Arrival counters and the fp64 sums start at zero on every call.
   cudaError_t e = cudaMemsetAsync(a.ws, 0, cnt_bytes + (a.mode != LA_OUT_RAW ? ss_bytes : 0), stream);
   if (e != cudaSuccess) return e;
-  auto kernel = a.mode == LA_OUT_RAW       ? lightning_prefill_tc_kernel<LA_OUT_RAW>
-                : a.mode == LA_OUT_RMSNORM ? lightning_prefill_tc_kernel<LA_OUT_RMSNORM>
-                                           : lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE>;
+  using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, TcParams);
+  static const Kernel kernels[3][2] = {
+      {lightning_prefill_tc_kernel<LA_OUT_RAW, 128>, lightning_prefill_tc_kernel<LA_OUT_RAW, 256>},
+      {lightning_prefill_tc_kernel<LA_OUT_RMSNORM, 128>, lightning_prefill_tc_kernel<LA_OUT_RMSNORM, 256>},
+      {lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 128>, lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 256>}};
+  const Kernel kernel = kernels[a.mode == LA_OUT_RAW ? 0 : (a.mode == LA_OUT_RMSNORM ? 1 : 2)][a.C == 256 ? 1 : 0];
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
