@@ -200,23 +200,46 @@ __device__ __forceinline__ void tile_first(const TcParams& p, TileIter& it) {
 __device__ __forceinline__ bool aborted(Bars& B) { return *reinterpret_cast<volatile int*>(&B.abort_flag) != 0; }
 
 // Bounded wait for phase `parity` of an mbarrier.  Returns false (after recording a
-// timeout, or because another role already did) when the CTA is aborting.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars& B, const TcParams& p, uint32_t site,
-                                      uint32_t index) {
-  if (mbar_try_wait(bar, parity)) return true;
+// timeout, or because another role already did) when the CTA is aborting.  The polling
+// loop is out of line: only the first test is inlined at each of the many wait sites,
+// which keeps the kernel's code (and its instruction-cache footprint) small.
+__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, int* abort_flag, ErrRec* err,
+                                           uint32_t site, uint32_t index) {
   const uint64_t t0 = globaltimer_ns();
-  const uint64_t lim = wait_limit_ns(p.err);
+  const uint64_t lim = wait_limit_ns(err);
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 31u) == 0) {
-      if (aborted(B)) return false;
+      if (*reinterpret_cast<volatile int*>(abort_flag) != 0) return false;
       if (globaltimer_ns() - t0 > lim) {
-        report(p.err, LA_ERR_TIMEOUT, site, index, parity);
-        *reinterpret_cast<volatile int*>(&B.abort_flag) = 1;
+        report(err, LA_ERR_TIMEOUT, site, index, parity);
+        *reinterpret_cast<volatile int*>(abort_flag) = 1;
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars& B, const TcParams& p, uint32_t site,
+                                      uint32_t index) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_bar_slow(bar, parity, &B.abort_flag, p.err, site, index);
+}
+
+// Bounded poll (one thread) until the arrival count at c reaches W, out of line for the
+// same reason; false when the CTA is aborting or the wait ran out (recorded).
+__device__ __noinline__ bool poll_count_slow(unsigned int* c, uint32_t W, int* abort_flag, ErrRec* err,
+                                             uint32_t index) {
+  const uint64_t t0 = globaltimer_ns();
+  const uint64_t lim = wait_limit_ns(err);
+  while (ld_acquire_gpu(c) < W) {
+    if (*reinterpret_cast<volatile int*>(abort_flag) != 0) return false;
+    if (globaltimer_ns() - t0 > lim) {
+      report(err, LA_ERR_TIMEOUT, SITE_TC_NORM_WAIT, index, ld_acquire_gpu(c));
+      *reinterpret_cast<volatile int*>(abort_flag) = 1;
+      return false;
+    }
+  }
+  return true;
 }
 
 // Short bounded wait used while draining at exit (never records an error).
@@ -878,20 +901,9 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         if (norm) {
           unsigned int* c = p.cnt + static_cast<int64_t>(s) * p.max_tiles + i;
           int go = 1;
-          if (lane == 0 && ld_acquire_gpu(c) < static_cast<uint32_t>(W)) {
-            const uint64_t t0 = globaltimer_ns();
-            const uint64_t lim = wait_limit_ns(p.err);
-            while (ld_acquire_gpu(c) < static_cast<uint32_t>(W)) {
-              if (aborted(B)) { go = 0; break; }
-              if (globaltimer_ns() - t0 > lim) {
-                report(p.err, LA_ERR_TIMEOUT, SITE_TC_NORM_WAIT, static_cast<uint32_t>(s * p.max_tiles + i),
-                       ld_acquire_gpu(c));
-                *reinterpret_cast<volatile int*>(&B.abort_flag) = 1;
-                go = 0;
-                break;
-              }
-            }
-          }
+          if (lane == 0 && ld_acquire_gpu(c) < static_cast<uint32_t>(W))
+            go = poll_count_slow(c, static_cast<uint32_t>(W), &B.abort_flag, p.err,
+                                 static_cast<uint32_t>(s * p.max_tiles + i)) ? 1 : 0;
           if (!__shfl_sync(0xFFFFFFFFu, go, 0)) { ok = false; break; }
           (void)ld_acquire_gpu(c);
           const float rn = (r < vr) ? 1.0f / sqrtf(static_cast<float>(ld_cg_f64(p.ss + row + r)) * inv_hd + p.eps) : 0.0f;
