@@ -812,14 +812,18 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           tc_fence_before();
           mbar_arrive(&B.z_full[zs][q]);
         }
+        const bool blk_end = (u == tpb - 1 || i == nt - 1);
         if (norm) {
           if (wt < vr) red_add_f64(p.ss + row + wt, static_cast<double>(ss));
-          __syncwarp();
-          // One release per warp orders the warp's additions before the arrival count.
-          if (lane == 0 && !skip_publish) red_add_release_gpu(p.cnt + static_cast<int64_t>(s) * p.max_tiles + i, 1u);
+          if (!blk_end) {
+            __syncwarp();
+            // One release per warp orders the warp's additions before the arrival count.
+            if (lane == 0 && !skip_publish) red_add_release_gpu(p.cnt + static_cast<int64_t>(s) * p.max_tiles + i, 1u);
+          }
         }
-        // Block end: snapshot S for the next block's inter product, or emit the final state.
-        if (u == tpb - 1 || i == nt - 1) {
+        // Block end: snapshot S for the next block's inter product, or emit the final state;
+        // the release of this tile's sums waits until the snapshot is out.
+        if (blk_end) {
           if (!wait_bar_warp(&B.s_done, blk & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
           blk++;
           tc_fence_after();
@@ -846,6 +850,10 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&B.snap_ready);
+          }
+          if (norm) {
+            __syncwarp();
+            if (lane == 0 && !skip_publish) red_add_release_gpu(p.cnt + static_cast<int64_t>(s) * p.max_tiles + i, 1u);
           }
         }
         ++t;
