@@ -32,14 +32,15 @@
 //    Score tiles alternate between two TMEM regions so that P of the next key/query tile
 //    is computed while the current one is being converted.
 //  * A conversion warpgroup turns P (fp32, TMEM) into masked bf16 in place.
-//  * The kernel is instantiated per output mode.  The epilogue reader warpgroup owns the
-//    state (S0 in, the bf16 snapshot of S at each block end, the final state out) and reads
-//    O once, releasing the accumulator at once.  In the raw mode it stores y directly.  In
-//    the norm modes it parks z = y * w as bf16 pairs in two spare TMEM tiles, adds each row's sum of
-//    squares into an fp64 per-token accumulator in global memory (red.add; the fp64 sum of
-//    the fp32 partials is exact whenever a token's partials span less than 2^22, so the
-//    result does not depend on the order the additions land in) and bumps the tile's
-//    arrival counter.  Four storer warps, one per TMEM lane quarter, load their rows of the
+//  * The kernel is instantiated per output mode and block size.  The epilogue reader
+//    warpgroup owns the state (S0 in, the bf16 snapshot of S at each block end, the final
+//    state out) and reads O once, releasing the accumulator at once.  In the raw mode it
+//    stores y directly.  In the norm modes it parks z = y * w as bf16 pairs in two spare
+//    TMEM tiles, adds each row's sum of squares into an fp64 per-token accumulator in
+//    global memory (red.add; the fp64 sum of the fp32 partials is exact whenever a token's
+//    partials span less than 2^22, so the result does not depend on the order the
+//    additions land in) and bumps the tile's arrival counter (at a block end only after
+//    the state snapshot is out, since the release waits for the additions).  Four storer warps, one per TMEM lane quarter, load their rows of the
 //    gate, wait until all H * 2 CTAs have arrived for the tile (the gate loads are in
 //    flight meanwhile), scale z by rsqrt(mean(y^2) + eps) * sigmoid(g) in registers and
 //    store each row's 128 bytes straight from registers.
