@@ -70,7 +70,7 @@ typedef enum { LA_OUT_RAW = 0, LA_OUT_RMSNORM = 1, LA_OUT_RMSNORM_GATE = 2 } la_
 /* SILU: phi(x) = x * sigmoid(x) on q and k.  IDENTITY: phi(x) = x (exact-integer tests). */
 typedef enum { LA_PHI_SILU = 0, LA_PHI_IDENTITY = 1 } la_feature_map;
 
-typedef enum { LA_OP_PREFILL = 0, LA_OP_PREFILL_VARLEN = 1, LA_OP_DECODE = 2 } la_op;
+typedef enum { LA_OP_PREFILL = 0, LA_OP_PREFILL_VARLEN = 1, LA_OP_DECODE = 2, LA_OP_MIXED = 3 } la_op;
 
 /*
  * Causal block-wise prefill of B sequences of T tokens each.
@@ -176,10 +176,43 @@ LA_API la_status lightning_attn_decode_step_noalloc(const void* q, const void* k
                                                     const float* norm_weight, la_stream_t stream);
 
 /*
+ * Mixed serving step over N sequences packed back to back: "MiniMax-01技术报告解读（二）
+ * 计算优化", sections 3 and 6 (chunked prefill; prefill and decode on separate streams).
+ * A sequence with exactly one new token is decoded (lightning_attn_decode_step: S is
+ * updated, then read); a sequence with more new tokens is prefilled as a continuation
+ * (lightning_attn_prefill_varlen with S0 = its current state, which is then replaced by
+ * the state after its last token).  Results are those of the two calls.
+ *   q, k, v          packed [total, H, D] device; g, out packed [total, H*D] (g when gated)
+ *   cu_seqlens       [N+1] int32 device: token offsets of the sequences (non-decreasing)
+ *   cu_seqlens_host  [N+1] int32 host: the same values (they decide the split and sizes)
+ *   state_pool       fp32 device [P, H, D, D]: the caller's state pool, updated in place
+ *   state_slot       [N] int32 device: pool slot of each sequence; slots must be distinct
+ *   prefill_stream   runs the prefill kernel; decode_stream runs the decode kernels (the
+ *                    two may be the same stream).  Nothing is ordered between them: the
+ *                    caller synchronises both before reading the results or reusing
+ *                    `workspace`.
+ *   workspace        >= lightning_attn_workspace_size(LA_OP_MIXED, N, max_prefill_len,
+ *                    total, ...) bytes, 256-byte aligned; the error record is shared by
+ *                    both streams (read it with lightning_attn_check after syncing both).
+ * Only the tensor-core configuration (bf16, D = 128, block 128 or 256, and for the norm
+ * modes all heads' CTA pairs resident at once) is supported, else LA_ERR_UNSUPPORTED with
+ * nothing enqueued; sequences of length 0 are allowed and left alone.  Invalid arguments
+ * (including host cu_seqlens that decrease) return LA_ERR_INVALID_ARG and enqueue nothing.
+ */
+LA_API la_status lightning_attn_mixed_step(const void* q, const void* k, const void* v, const void* g, void* out,
+                                           const int* cu_seqlens, const int* cu_seqlens_host, float* state_pool,
+                                           const int* state_slot, int num_seqs, int H, int D, int block_size,
+                                           la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
+                                           const float* norm_weight, void* workspace, size_t workspace_bytes,
+                                           la_stream_t prefill_stream, la_stream_t decode_stream);
+
+/*
  * Workspace bytes needed by one call (0 on invalid arguments).
  *   op == LA_OP_PREFILL:         B_or_N = B, T_or_max = T, total_tokens ignored.
  *   op == LA_OP_PREFILL_VARLEN:  B_or_N = N, T_or_max = max_seqlen, total_tokens.
  *   op == LA_OP_DECODE:          B_or_N = B, the rest ignored except H, D, dtype, mode.
+ *   op == LA_OP_MIXED:           B_or_N = N, T_or_max = longest sequence with more than
+ *                                one token (0 if none), total_tokens = all packed tokens.
  * The size depends on the kernel the call will select (which depends on the device), so
  * query it with the target device current.
  */

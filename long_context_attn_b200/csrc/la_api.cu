@@ -10,8 +10,11 @@
 namespace la {
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, void* out, float* state,
                           int B, int H, int D, la_dtype dt, int phi_identity, int mode, float eps,
-                          const float* w, void* workspace, cudaStream_t stream);
+                          const float* w, void* workspace, cudaStream_t stream,
+                          const int* row_index = nullptr, const int* state_index = nullptr);
 size_t decode_workspace_bytes(int B, int H, int D);
+cudaError_t launch_gather_single_token(const int* cu, const int* state_slot, int n, int* row_index,
+                                       int* state_index, cudaStream_t stream);
 cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, void* out, float* y_ws,
                                 const float* state_in, float* state_out, const int* cu, int nseq, int T,
                                 int H, int D, int C, la_dtype dt, int phi_identity, int64_t total_rows,
@@ -114,6 +117,20 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
+// Mixed step workspace: [prefill part (error record + counters + sums)] [decode part]
+// [decode item token rows] [decode item state slots].  Sized for N decode items at most.
+struct MixedLayout {
+  size_t pre, dec, idx, total;
+};
+MixedLayout mixed_layout(int n, int max_pre, int64_t total, int H, int D, int C, la_out_mode mode) {
+  MixedLayout m{};
+  m.pre = max_pre > 1 ? prefill_ws_bytes(Path::kTc, n, max_pre, total, H, D, C, mode) : kErrBytes;
+  m.dec = la::decode_workspace_bytes(n, H, D);
+  m.idx = 2 * up256(sizeof(int) * static_cast<size_t>(n));
+  m.total = m.pre + m.dec + m.idx;
+  return m;
+}
+
 }  // namespace
 
 extern "C" {
@@ -164,10 +181,78 @@ la_status lightning_attn_decode_step(const void* q, const void* k, const void* v
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
+la_status lightning_attn_mixed_step(const void* q, const void* k, const void* v, const void* g, void* out,
+                                    const int* cu_seqlens, const int* cu_seqlens_host, float* state_pool,
+                                    const int* state_slot, int num_seqs, int H, int D, int block_size,
+                                    la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
+                                    const float* norm_weight, void* workspace, size_t workspace_bytes,
+                                    la_stream_t prefill_stream, la_stream_t decode_stream) {
+  if (!valid_enums(dtype, phi, mode) || !valid_head(H, D, mode, eps)) return LA_ERR_INVALID_ARG;
+  if (num_seqs < 1 || !cu_seqlens || !cu_seqlens_host || !state_pool || !state_slot || !aligned16(cu_seqlens) ||
+      !aligned16(state_pool))
+    return LA_ERR_INVALID_ARG;
+  if (block_size < 1 || block_size > 1024) return LA_ERR_INVALID_ARG;
+  // The split: one-token sequences decode, longer ones prefill.
+  int n_dec = 0, max_pre = 0;
+  if (cu_seqlens_host[0] < 0) return LA_ERR_INVALID_ARG;
+  for (int s = 0; s < num_seqs; ++s) {
+    const int L = cu_seqlens_host[s + 1] - cu_seqlens_host[s];
+    if (L < 0) return LA_ERR_INVALID_ARG;
+    if (L == 1) ++n_dec;
+    if (L > max_pre) max_pre = L;
+  }
+  const int64_t total = cu_seqlens_host[num_seqs];
+  if (total > 0) {
+    if (!q || !k || !v || !out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LA_ERR_INVALID_ARG;
+    if (mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g))) return LA_ERR_INVALID_ARG;
+  }
+  if (norm_weight && !aligned16(norm_weight)) return LA_ERR_INVALID_ARG;
+  if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;
+  if (choose_path(dtype, H, D, block_size, mode) != Path::kTc) return LA_ERR_UNSUPPORTED;
+  const MixedLayout lay = mixed_layout(num_seqs, max_pre, total, H, D, block_size, mode);
+  if (workspace_bytes < lay.total) return LA_ERR_INVALID_ARG;
+
+  char* base = static_cast<char*>(workspace);
+  la::ErrRec* err = reinterpret_cast<la::ErrRec*>(base);
+  const int phi_id = (phi == LA_PHI_IDENTITY) ? 1 : 0;
+  cudaStream_t ps = reinterpret_cast<cudaStream_t>(prefill_stream);
+  cudaStream_t ds = reinterpret_cast<cudaStream_t>(decode_stream);
+  cudaError_t e = cudaSuccess;
+  if (max_pre > 1) {
+    la::TcArgs a{};
+    a.q = q; a.k = k; a.v = v; a.g = g; a.out = out;
+    a.state_in = state_pool; a.state_out = state_pool; a.cu = cu_seqlens;
+    a.nseq = num_seqs; a.T = 0; a.max_len = max_pre; a.tokens = total;
+    a.H = H; a.D = D; a.C = block_size; a.phi_identity = phi_id; a.mode = static_cast<int>(mode);
+    a.eps = eps; a.w = norm_weight; a.err = err; a.ws = base + kErrBytes;
+    a.state_index = state_slot;
+    a.skip_single = 1;
+    e = la::launch_tc_prefill(a, current_sm_count(), ps);
+  }
+  if (e == cudaSuccess && n_dec > 0) {
+    char* dws = base + lay.pre;
+    int* rows = reinterpret_cast<int*>(base + lay.pre + lay.dec);
+    int* slots = reinterpret_cast<int*>(base + lay.pre + lay.dec + lay.idx / 2);
+    // The decode counters live where the previous step's layout may have left other data.
+    e = cudaMemsetAsync(dws, 0, lay.dec, ds);
+    if (e == cudaSuccess) e = la::launch_gather_single_token(cu_seqlens, state_slot, num_seqs, rows, slots, ds);
+    if (e == cudaSuccess)
+      e = la::launch_decode(q, k, v, g, out, state_pool, n_dec, H, D, dtype, phi_id, static_cast<int>(mode), eps,
+                            norm_weight, dws, ds, rows, slots);
+  }
+  g_last_path = "mixed";
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
 size_t lightning_attn_workspace_size(la_op op, int B_or_N, int T_or_max, int total_tokens, int H, int D,
                                      int block_size, la_dtype dtype, la_out_mode mode) {
   if (B_or_N < 1 || T_or_max < 0 || H < 1 || (D != 64 && D != 128)) return 0;
   if (op == LA_OP_DECODE) return la::decode_workspace_bytes(B_or_N, H, D);
+  if (op == LA_OP_MIXED) {
+    if (total_tokens < 0 || block_size < 1 || block_size > 1024) return 0;
+    return mixed_layout(B_or_N, T_or_max, total_tokens, H, D, block_size, mode).total;
+  }
   if (block_size < 1 || block_size > 1024) return 0;
   const Path path = choose_path(dtype, H, D, block_size, mode);
   if (op == LA_OP_PREFILL)

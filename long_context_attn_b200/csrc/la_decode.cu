@@ -21,6 +21,8 @@ struct DecodeWs {
   int* count;      // [B] arrivals per sequence (zero between calls)
   float* y;        // [B, H, D] raw outputs
   float* part;     // [B, H] per-head sums of squares
+  const int* row_index;    // optional [B]: token row of item b in q, k, v, g, out (else b)
+  const int* state_index;  // optional [B]: state slot of item b (else b)
 };
 
 template <typename T, int D>
@@ -42,8 +44,12 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 
   const int bh = blockIdx.x;            // b * H + h
   const int b = bh / H;
+  const int h = bh % H;
   const int tid = threadIdx.x;
-  const int64_t tok = static_cast<int64_t>(bh) * D;
+  // Item b's token row and state slot (a mixed step gathers its one-token sequences).
+  const int64_t trow = ws.row_index ? __ldg(ws.row_index + b) : b;
+  const int64_t slot = ws.state_index ? __ldg(ws.state_index + b) : b;
+  const int64_t tok = (trow * H + h) * D;
 
   for (int i = tid; i < D; i += kThreads) {
     const float xq = load_elem<T>(q, tok + i), xk = load_elem<T>(k, tok + i);
@@ -55,7 +61,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
   // Issue every state load of this thread before the first use.
   const int c4 = tid % kVecPerRow;
   const int r0 = tid / kVecPerRow;
-  float4* S = reinterpret_cast<float4*>(state + static_cast<int64_t>(bh) * D * D);
+  float4* S = reinterpret_cast<float4*>(state + (slot * H + h) * D * D);
   float4 s[kPasses];
 #pragma unroll
   for (int p = 0; p < kPasses; ++p) s[p] = __ldcs(&S[(r0 + p * kRowsPerPass) * kVecPerRow + c4]);
@@ -85,7 +91,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
   }
   const int HD = H * D;
   if (mode == LA_OUT_RAW) {
-    if (tid < D) store_elem<T>(out, static_cast<int64_t>(b) * HD + (bh % H) * D + tid, y);
+    if (tid < D) store_elem<T>(out, trow * HD + h * D + tid, y);
     return;
   }
 
@@ -94,7 +100,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
   if ((tid & 31) == 0) s_ss[tid >> 5] = sq;
-  if (tid < D) ws.y[tok + tid] = y;
+  if (tid < D) ws.y[static_cast<int64_t>(bh) * D + tid] = y;
   __syncthreads();
   if (tid == 0) {
     float t = 0.f;
@@ -117,9 +123,10 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
   }
   __syncthreads();
   const float r = s_ss[0];
-  const int64_t row = static_cast<int64_t>(b) * HD;
+  const int64_t yrow = static_cast<int64_t>(b) * HD;
+  const int64_t row = trow * HD;
   for (int c = tid; c < HD; c += kThreads) {
-    float o = __ldcg(&ws.y[row + c]) * r;
+    float o = __ldcg(&ws.y[yrow + c]) * r;
     if (norm_w) o *= norm_w[c];
     if (mode == LA_OUT_RMSNORM_GATE) o *= sigmoid_accurate(load_elem<T>(g, row + c));
     store_elem<T>(out, row + c, o);
@@ -132,7 +139,8 @@ size_t decode_workspace_bytes(int B, int H, int D) {
          up(sizeof(float) * size_t(B) * H);
 }
 
-static DecodeWs carve_decode_ws(void* workspace, int B, int H, int D) {
+static DecodeWs carve_decode_ws(void* workspace, int B, int H, int D, const int* row_index,
+                                const int* state_index) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   char* p = static_cast<char*>(workspace) + 256;
   DecodeWs ws;
@@ -141,14 +149,17 @@ static DecodeWs carve_decode_ws(void* workspace, int B, int H, int D) {
   ws.y = reinterpret_cast<float*>(p);
   p += up(sizeof(float) * size_t(B) * H * D);
   ws.part = reinterpret_cast<float*>(p);
+  ws.row_index = row_index;
+  ws.state_index = state_index;
   return ws;
 }
 
 template <typename T, int D>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* g, void* out,
                                    float* state, int B, int H, int phi_identity, int mode, float eps,
-                                   const float* w, void* workspace, cudaStream_t stream) {
-  DecodeWs ws = carve_decode_ws(workspace, B, H, D);
+                                   const float* w, void* workspace, const int* row_index,
+                                   const int* state_index, cudaStream_t stream) {
+  DecodeWs ws = carve_decode_ws(workspace, B, H, D, row_index, state_index);
   decode_step_kernel<T, D><<<B * H, 256, 0, stream>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
       static_cast<const T*>(g), static_cast<T*>(out), state, B, H, phi_identity, mode, eps, w, ws);
@@ -157,13 +168,62 @@ static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, 
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, void* out, float* state,
                           int B, int H, int D, la_dtype dt, int phi_identity, int mode, float eps,
-                          const float* w, void* workspace, cudaStream_t stream) {
+                          const float* w, void* workspace, cudaStream_t stream, const int* row_index,
+                          const int* state_index) {
   if (dt == LA_BF16) {
-    if (D == 128) return launch_decode_t<uint16_t, 128>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace, stream);
-    return launch_decode_t<uint16_t, 64>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace, stream);
+    if (D == 128)
+      return launch_decode_t<uint16_t, 128>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace,
+                                            row_index, state_index, stream);
+    return launch_decode_t<uint16_t, 64>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace,
+                                         row_index, state_index, stream);
   }
-  if (D == 128) return launch_decode_t<float, 128>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace, stream);
-  return launch_decode_t<float, 64>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace, stream);
+  if (D == 128)
+    return launch_decode_t<float, 128>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace,
+                                       row_index, state_index, stream);
+  return launch_decode_t<float, 64>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace,
+                                    row_index, state_index, stream);
+}
+
+// Mixed step: the one-token sequences of cu_seqlens (in sequence order) become the items
+// of a decode batch: item j gets the token row cu[s] and the state slot state_slot[s] of
+// the j-th such sequence.  One CTA; a block-wide prefix count per chunk of 1024 keeps the
+// order deterministic.
+__global__ void __launch_bounds__(1024) gather_single_token_kernel(const int* __restrict__ cu,
+                                                                     const int* __restrict__ state_slot, int n,
+                                                                     int* __restrict__ row_index,
+                                                                     int* __restrict__ state_index) {
+  __shared__ int warp_tot[32];
+  __shared__ int base;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) base = 0;
+  __syncthreads();
+  for (int s0 = 0; s0 < n; s0 += 1024) {
+    const int s = s0 + tid;
+    const bool one = s < n && (cu[s + 1] - cu[s]) == 1;
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, one);
+    const int before = __popc(m & ((1u << lane) - 1u));
+    if (lane == 0) warp_tot[warp] = __popc(m);
+    __syncthreads();
+    int off = base;
+    for (int w = 0; w < warp; ++w) off += warp_tot[w];
+    if (one) {
+      row_index[off + before] = cu[s];
+      state_index[off + before] = state_slot[s];
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int t = 0;
+      for (int w = 0; w < 32; ++w) t += warp_tot[w];
+      base += t;
+    }
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_gather_single_token(const int* cu, const int* state_slot, int n, int* row_index,
+                                       int* state_index, cudaStream_t stream) {
+  gather_single_token_kernel<<<1, 1024, 0, stream>>>(cu, state_slot, n, row_index, state_index);
+  return cudaGetLastError();
 }
 
 }  // namespace la

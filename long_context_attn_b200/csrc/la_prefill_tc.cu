@@ -118,6 +118,8 @@ struct TcParams {
   unsigned int* cnt;   // [nseq * max_tiles] arrivals per tile
   double* ss;          // [tokens] sum of squares over the head concatenation
   uint16_t* out;
+  const int* state_index;  // optional [nseq]: state slot of each sequence (else the index)
+  int skip_single;         // nonzero: one-token sequences belong to a decode step: skip them
 };
 
 // Shared-memory descriptor templates with start address 0; an operand at shared address a
@@ -144,7 +146,9 @@ __device__ __forceinline__ int pad_rows(int vr) { return vr <= 32 ? 32 : (vr <= 
 
 // Rows [row0, row0 + L) of sequence s.  Invalid cu_seqlens entries are reported and the
 // sequence is treated as empty (every role and every CTA reaches the same decision).
-__device__ __forceinline__ void seq_range(const TcParams& p, int s, int64_t& row0, int& L) {
+// Returns true for a sequence this call leaves alone entirely (a one-token sequence of a
+// mixed step, which the decode kernel handles): L = 0 and its state is not touched.
+__device__ __forceinline__ bool seq_range(const TcParams& p, int s, int64_t& row0, int& L) {
   if (p.cu) {
     const int a = __ldg(p.cu + s), b = __ldg(p.cu + s + 1);
     row0 = a;
@@ -153,10 +157,15 @@ __device__ __forceinline__ void seq_range(const TcParams& p, int s, int64_t& row
       if (threadIdx.x == 0) report(p.err, LA_ERR_DEVICE, SITE_VARLEN_CU, s, 0);
       L = 0;
     }
+    if (p.skip_single && L == 1) {
+      L = 0;
+      return true;
+    }
   } else {
     row0 = static_cast<int64_t>(s) * p.T;
     L = p.T;
   }
+  return false;
 }
 
 // The (sequence, tile) order every role walks; empty sequences have no tiles.
@@ -721,10 +730,11 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     for (int s = 0; s < p.nseq && ok; ++s) {
       int64_t row0;
       int L;
-      seq_range(p, s, row0, L);
+      if (seq_range(p, s, row0, L)) continue;   // a one-token sequence of a mixed step
       const int nt = (L + kTile - 1) / kTile;
       // Initial state: S0 (or zeros) into TMEM and the bf16 snapshot.
-      const int64_t st_row = ((static_cast<int64_t>(s) * p.H + h) * kD + wt) * kD + dvt * kDV;
+      const int64_t slot = p.state_index ? __ldg(p.state_index + s) : s;
+      const int64_t st_row = ((slot * p.H + h) * kD + wt) * kD + dvt * kDV;
       {
         // 16 columns at a time: TMEM copy (fp32) and snapshot chunks 2j, 2j + 1 (bf16).
 #pragma unroll
@@ -1051,6 +1061,8 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
   p.eps = a.eps;
   p.w = a.w;
   p.g = static_cast<const uint16_t*>(a.g);
+  p.state_index = a.state_index;
+  p.skip_single = a.skip_single;
   p.err = a.err;
   p.cnt = reinterpret_cast<unsigned int*>(a.ws);
   p.ss = reinterpret_cast<double*>(a.ws + cnt_bytes);

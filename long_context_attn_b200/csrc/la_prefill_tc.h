@@ -27,6 +27,8 @@ struct TcArgs {
   const float* w;
   ErrRec* err;
   char* ws;            // workspace after the error record
+  const int* state_index;  // optional [nseq] device: state slot of each sequence (else s)
+  int skip_single;         // nonzero: sequences of exactly one token are left alone entirely
 };
 
 // True when the tensor-core kernel handles this shape on a GPU with `num_sms` SMs.

@@ -20,7 +20,7 @@ LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT, LA_E
 LA_F32, LA_BF16 = 0, 1
 LA_OUT_RAW, LA_OUT_RMSNORM, LA_OUT_RMSNORM_GATE = 0, 1, 2
 LA_PHI_SILU, LA_PHI_IDENTITY = 0, 1
-LA_OP_PREFILL, LA_OP_PREFILL_VARLEN, LA_OP_DECODE = 0, 1, 2
+LA_OP_PREFILL, LA_OP_PREFILL_VARLEN, LA_OP_DECODE, LA_OP_MIXED = 0, 1, 2, 3
 
 # The symbols include/lightning_attn.h declares (checked by tests/test_abi.py).
 EXPORTED = (
@@ -28,6 +28,7 @@ EXPORTED = (
     "lightning_attn_prefill_varlen",
     "lightning_attn_decode_step",
     "lightning_attn_decode_step_noalloc",
+    "lightning_attn_mixed_step",
     "lightning_attn_workspace_size",
     "lightning_attn_check",
     "lightning_attn_status_string",
@@ -55,6 +56,8 @@ def _load():
                                                sz, vp]
     lib.lightning_attn_decode_step_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32,
                                                        vp, vp]
+    lib.lightning_attn_mixed_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                              f32, vp, vp, sz, vp, vp]
     lib.lightning_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
     lib.lightning_attn_workspace_size.restype = sz
     lib.lightning_attn_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint * 4)]
@@ -63,7 +66,7 @@ def _load():
     lib.lightning_attn_last_path.argtypes = []
     lib.lightning_attn_last_path.restype = ctypes.c_char_p
     for f in ("lightning_attn_prefill", "lightning_attn_prefill_varlen", "lightning_attn_decode_step",
-              "lightning_attn_decode_step_noalloc", "lightning_attn_check"):
+              "lightning_attn_decode_step_noalloc", "lightning_attn_mixed_step", "lightning_attn_check"):
         getattr(lib, f).restype = i32
     return lib
 
@@ -188,6 +191,29 @@ def lightning_attn_decode_step_noalloc(q, k, v, g, out, state, phi=LA_PHI_SILU, 
                                                  _ptr(_f32_or_none(norm_weight)), _stream(stream))
     if st != LA_OK:
         raise LightningAttnError(st, "lightning_attn_decode_step_noalloc")
+
+
+def lightning_attn_mixed_step(q, k, v, g, out, cu_seqlens, cu_seqlens_host, state_pool, state_slot,
+                              block_size=256, phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE, eps=1e-6, norm_weight=None,
+                              workspace=None, prefill_stream=None, decode_stream=None):
+    """One serving step over packed sequences: one-token sequences decode, longer ones prefill
+    from their state.  q, k, v [total, H, D]; g, out [total, H*D]; cu_seqlens int32 device
+    [N + 1] with the same values in `cu_seqlens_host` (a host sequence of ints); state_pool
+    fp32 [P, H, D, D] updated in place; state_slot int32 device [N] (distinct slots)."""
+    total, H, D = q.shape
+    _check_contig(q, k, v, g, out, cu_seqlens, state_pool, state_slot)
+    if cu_seqlens.dtype != torch.int32 or state_slot.dtype != torch.int32:
+        raise TypeError("cu_seqlens and state_slot must be int32")
+    n = cu_seqlens.numel() - 1
+    host = (ctypes.c_int * (n + 1))(*[int(x) for x in cu_seqlens_host])
+    st = _lib.lightning_attn_mixed_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(out), _ptr(cu_seqlens),
+                                        ctypes.cast(host, ctypes.c_void_p), _ptr(_f32_or_none(state_pool)),
+                                        _ptr(state_slot), n, H, D, block_size, _dtype(q), phi, mode, eps,
+                                        _ptr(_f32_or_none(norm_weight)), _ptr(workspace),
+                                        0 if workspace is None else workspace.numel(), _stream(prefill_stream),
+                                        _stream(decode_stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_mixed_step")
 
 
 def lightning_attn_check(workspace, stream=None, raise_on_error=True):

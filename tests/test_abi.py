@@ -89,3 +89,33 @@ def test_invalid_arguments_rejected_before_launch(lib):
              None) == 1  # missing state
     assert d(fake, fake, fake, fake, fake, fake, 4, 2, 128, 1, 0, 2, ctypes.c_float(1e-6), None, ws, 16,
              None) == 1  # workspace too small
+
+
+def test_mixed_step_host_checks(lib):
+    """The mixed step's split and argument checks happen on the host before any launch."""
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    f = lib.lightning_attn_mixed_step
+    f.argtypes = [vp] * 9 + [i32] * 7 + [ctypes.c_float, vp, vp, ctypes.c_size_t, vp, vp]
+    fake, ws = vp(0x1000), vp(0x100000)
+    good = (ctypes.c_int * 4)(0, 1, 5, 6)
+    bad = (ctypes.c_int * 4)(0, 3, 2, 6)        # decreasing offsets
+
+    def call(host, **kw):
+        a = dict(q=fake, k=fake, v=fake, g=fake, out=fake, cu=fake, pool=fake, slot=fake, n=3, H=2, D=128, C=256,
+                 dt=1, phi=0, mode=2, ws=ws)
+        a.update(kw)
+        return f(a["q"], a["k"], a["v"], a["g"], a["out"], a["cu"], ctypes.cast(host, vp), a["pool"], a["slot"],
+                 a["n"], a["H"], a["D"], a["C"], a["dt"], a["phi"], a["mode"], ctypes.c_float(1e-6), None, a["ws"],
+                 1 << 30, None, None)
+
+    assert call(bad) == 1                 # host cu_seqlens decrease
+    assert call(good, slot=None) == 1     # no slot map
+    assert call(good, pool=None) == 1     # no state pool
+    assert call(good, g=None) == 1        # gate required
+    assert call(good, D=96) == 1
+    assert call(good, ws=vp(0x100010)) == 1
+    lib.lightning_attn_workspace_size.restype = ctypes.c_size_t
+    # LA_OP_MIXED sizes: prefill part for the longest multi-token sequence + decode part for N.
+    n3 = lib.lightning_attn_workspace_size(3, 3, 4, 6, 2, 128, 256, 1, 2)
+    n_dec_only = lib.lightning_attn_workspace_size(3, 3, 0, 3, 2, 128, 256, 1, 2)
+    assert n3 > n_dec_only > 256
