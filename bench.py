@@ -346,12 +346,110 @@ class VarlenCase:
                 "l2": "inputs larger than L2 (%.1f GB per step), no flush" % (self.alg_bytes / 1e9)}
 
 
+class MixedCase:
+    """One serving step: 256 sequences decode a token each while 2 others prefill a 4096-token
+    chunk from their state; prefill and decode on two streams, states in a pool (slots in a
+    seeded shuffled order), updated in place step after step."""
+
+    def __init__(self, name, w, device, rank):
+        import torch
+        from long_context_attn_b200 import lightning_attn as la
+        self.la, self.w = la, w
+        H, D = w.H, w.D
+        self.lens = synth.mixed_lengths(w)
+        self.n = len(self.lens)
+        self.total = int(self.lens.sum())
+        t0 = time.time()
+        q, k, v, g = synth.prefill_inputs(w.seed + 1000 * rank, self.total, H, D, "bf16", w.qkv_scale, True)
+        pool = synth.decode_state(w.seed + 1000 * rank, self.n, H, D)
+        self.gen_s = time.time() - t0
+        perm = np.argsort(synth.uniform_int(w.seed, synth.STREAM_LEN, self.n, 0, 1 << 30), kind="stable")
+        self.slots_host = perm.astype(np.int32)
+
+        def pin(a):
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+        self.h_q, self.h_k, self.h_v, self.h_g = (pin(a) for a in (q, k, v, g))
+        del q, k, v, g
+        self.q = self.h_q.to(device).view(self.total, H, D)
+        self.k = self.h_k.to(device).view(self.total, H, D)
+        self.v = self.h_v.to(device).view(self.total, H, D)
+        self.g = self.h_g.to(device).view(self.total, H * D)
+        self.pool = torch.from_numpy(pool).to(device)
+        self.cu_host = synth.cu_seqlens_of(self.lens)
+        self.cu = torch.from_numpy(self.cu_host).to(device)
+        self.slots = torch.from_numpy(self.slots_host).to(device)
+        self.out = torch.empty((self.total, H * D), dtype=torch.bfloat16, device=device)
+        self.h_out = torch.empty((self.total, H * D), dtype=torch.bfloat16).pin_memory()
+        max_pre = int(self.lens[self.lens > 1].max()) if (self.lens > 1).any() else 0
+        self.ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_MIXED, self.n, max_pre, self.total, H, D,
+                                                                    w.block_size, la.LA_BF16, la.LA_OUT_RMSNORM_GATE),
+                                   device)
+        self.ps, self.ds = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        self.tokens = self.total
+        # this library's kernels per step: the prefill, the one-token gather and the decode
+        self.launches_per_step = int((self.lens > 1).any()) + 2 * int((self.lens == 1).any())
+        n_dec = int((self.lens == 1).sum())
+        n_pre_tok = int(self.lens[self.lens > 1].sum())
+        n_pre_seq = int((self.lens > 1).sum())
+        self.alg_bytes = (n_dec * H * (2 * D * D * 4 + 5 * D * 2) + n_pre_tok * _bytes_per_token(H, D) +
+                          n_pre_seq * H * D * D * 4 * 2)
+        algo_pt, issued_pt = _flops_per_token(H, D, w.block_size)
+        self.alg_flops = n_dec * H * 4 * D * D + n_pre_tok * algo_pt
+        self.issued_flops = n_dec * H * 4 * D * D + n_pre_tok * issued_pt
+        self.h2d = sum(t.numel() * t.element_size() for t in (self.h_q, self.h_k, self.h_v, self.h_g))
+        self.d2h = self.h_out.numel() * 2
+
+    def step(self):
+        import torch
+        cur = torch.cuda.current_stream()
+        self.ps.wait_stream(cur)
+        self.ds.wait_stream(cur)
+        self.la.lightning_attn_mixed_step(self.q, self.k, self.v, self.g, self.out, self.cu, self.cu_host.tolist(),
+                                          self.pool, self.slots, block_size=self.w.block_size, workspace=self.ws,
+                                          prefill_stream=self.ps, decode_stream=self.ds)
+        cur.wait_stream(self.ps)
+        cur.wait_stream(self.ds)
+
+    def e2e_step(self):
+        self.q.view(-1).copy_(self.h_q.view(-1), non_blocking=True)
+        self.k.view(-1).copy_(self.h_k.view(-1), non_blocking=True)
+        self.v.view(-1).copy_(self.h_v.view(-1), non_blocking=True)
+        self.g.view(-1).copy_(self.h_g.view(-1), non_blocking=True)
+        self.step()
+        self.h_out.copy_(self.out, non_blocking=True)
+
+    def check(self):
+        self.ps.synchronize()
+        self.ds.synchronize()
+        self.la.lightning_attn_check(self.ws)
+
+    def oracle_sample(self):
+        """fp64 oracle over the whole step (every sequence from its pooled state)."""
+        import oracle
+        w = self.w
+        q, k, v, g = synth.prefill_inputs(w.seed, self.total, w.H, w.D, "bf16", w.qkv_scale, True)
+        pool = synth.decode_state(w.seed, self.n, w.H, w.D)
+        t0 = time.perf_counter()
+        oracle.forward_packed(q, k, v, g, self.cu_host, w.H, w.D, state_in=pool[self.slots_host], store=False)
+        return time.perf_counter() - t0
+
+    def describe(self):
+        return {"workload": self.w.name, "decode_seqs": int((self.lens == 1).sum()),
+                "prefill_chunks": int((self.lens > 1).sum()), "chunk_tokens": self.w.T, "H": self.w.H,
+                "D": self.w.D, "block_size": self.w.block_size, "mode": "rmsnorm_gate",
+                "streams": "prefill and decode on two streams",
+                "l2": "state pool larger than L2 (%.2f GB per step), no flush" % (self.alg_bytes / 1e9)}
+
+
 def _make_case(name, device, rank):
     w = synth.WORKLOADS[name]
     if w.kind == "prefill" and w.dtype == "bf16":
         return PrefillCase(name, w, device, rank)
     if w.kind == "varlen":
         return VarlenCase(name, w, device, rank)
+    if w.kind == "mixed":
+        return MixedCase(name, w, device, rank)
     if w.kind == "decode":
         return DecodeCase(name, w, device, rank)
     raise SystemExit(f"workload {name} is not a bench workload")
@@ -460,7 +558,7 @@ def run_gpu(args):
                        "frac_issued": case.issued_flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
             "e2e": {"value": _job_value(case.tokens, args.steps, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": case.h2d, "d2h_bytes_per_step": case.d2h},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * getattr(case, "launches_per_step", 1),
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -508,6 +606,11 @@ def _cpu_baseline(case):
         return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
                 "sample": f"first {n} tokens of the {case.w.name} workload, all {case.H} heads, fp64, "
                           f"recurrence + norm + gate ({dt:.1f} s)"}
+    if isinstance(case, MixedCase):
+        dt = case.oracle_sample()
+        return {"value": case.total / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                "sample": f"the whole {case.w.name} step ({case.total} tokens, all {case.w.H} heads), fp64 "
+                          f"({dt:.1f} s)"}
     if isinstance(case, VarlenCase):
         dt, n = case.oracle_sample(131072)
         return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
@@ -526,7 +629,7 @@ def run_reference(args):
         return
     import oracle
     w = synth.WORKLOADS[args.workload]
-    if w.kind in ("prefill", "varlen"):
+    if w.kind in ("prefill", "varlen", "mixed"):
         n = 1024
         q, k, v, g = synth.prefill_inputs(w.seed, n, w.H, w.D, w.dtype, w.qkv_scale, True)
 
@@ -569,7 +672,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="prefill_128k",
-                    choices=["prefill_8k", "prefill_128k", "varlen_16", "decode_256"])
+                    choices=["prefill_8k", "prefill_128k", "varlen_16", "decode_256", "mixed_256"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     args = ap.parse_args()

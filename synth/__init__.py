@@ -114,7 +114,7 @@ def f32_to_bf16(a: np.ndarray) -> np.ndarray:
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str              # 'prefill' | 'varlen' | 'decode'
+    kind: str              # 'prefill' | 'varlen' | 'decode' | 'mixed'
     seed: int
     B: int                 # batch (prefill), number of sequences (varlen / decode)
     T: int                 # tokens per sequence (prefill); 0 otherwise
@@ -127,6 +127,7 @@ class Workload:
     len_lo: int = 0
     len_hi: int = 0
     eps: float = 1e-6
+    n_prefill: int = 0     # mixed: number of prefill chunks (of T tokens) among B decode sequences
 
 
 # The five workloads of the Lightning Attention forward (seed 1000 + k).
@@ -137,7 +138,24 @@ WORKLOADS = {
     "varlen_16": Workload("varlen_16", "varlen", 1004, 16, 0, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5,
                           len_lo=1000, len_hi=32768),
     "decode_256": Workload("decode_256", "decode", 1005, 256, 0, 64, 128, 0, "bf16", "rmsnorm_gate", 0.5),
+    # A serving step: 256 sequences decode one token each while 2 others prefill a 4096-token
+    # chunk from their state (chunked prefill), all packed into one batch.
+    "mixed_256": Workload("mixed_256", "mixed", 1006, 256, 4096, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5,
+                          n_prefill=2),
 }
+
+
+def mixed_lengths(w: Workload) -> np.ndarray:
+    """Sequence lengths of a mixed step: each prefill chunk is followed by its share of the
+    one-token (decode) sequences."""
+    lens = []
+    per = w.B // max(w.n_prefill, 1)
+    for i in range(w.n_prefill):
+        lens.append(w.T)
+        lens.extend([1] * (per if i < w.n_prefill - 1 else w.B - per * (w.n_prefill - 1)))
+    if w.n_prefill == 0:
+        lens.extend([1] * w.B)
+    return np.asarray(lens, dtype=np.int64)
 
 
 def varlen_lengths(w: Workload) -> np.ndarray:

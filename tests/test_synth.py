@@ -50,3 +50,6 @@ def test_workload_table():
     assert w["prefill_128k"].T == 131072 and w["prefill_128k"].H == 64 and w["prefill_128k"].D == 128
     lens = synth.varlen_lengths(w["varlen_16"])
     assert len(lens) == 16 and lens.min() >= 1000 and lens.max() <= 32768
+    mixed = w["mixed_256"]
+    ml = synth.mixed_lengths(mixed)
+    assert (ml == 1).sum() == 256 and (ml == 4096).sum() == 2 and len(ml) == 258 and mixed.seed == 1006
