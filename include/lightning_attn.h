@@ -207,6 +207,22 @@ LA_API la_status lightning_attn_mixed_step(const void* q, const void* k, const v
                                            la_stream_t prefill_stream, la_stream_t decode_stream);
 
 /*
+ * Sequence-parallel prefill ("MiniMax-01系列大模型：超长上下文与多模态能力深度解析与部署指南",
+ * section 2.1.3, LASP+): one sequence is split into contiguous chunks, one per rank.  The
+ * state is a plain sum, so the state entering chunk `rank` is state0 plus the sum of the
+ * states the earlier chunks reach from a zero state.  Given those chunk states gathered in
+ * rank order, this writes the prefix for `rank` (adding in rank order: deterministic).
+ *   gathered  fp32 device [world, H, D, D] (chunk states, rank order)
+ *   state0    fp32 device [H, D, D] or NULL (zero): the state before the whole sequence
+ *   out       fp32 device [H, D, D] (may not alias `gathered`)
+ * The host side of a sequence-parallel prefill is long_context_attn_b200.sequence_parallel:
+ * a raw-mode prefill of the chunk from a zero state, an all-gather of the chunk states,
+ * this prefix, then the chunk's prefill from the prefix.
+ */
+LA_API la_status lightning_attn_state_prefix(const float* gathered, int world, int rank, const float* state0,
+                                             float* out, int H, int D, la_stream_t stream);
+
+/*
  * Workspace bytes needed by one call (0 on invalid arguments).
  *   op == LA_OP_PREFILL:         B_or_N = B, T_or_max = T, total_tokens ignored.
  *   op == LA_OP_PREFILL_VARLEN:  B_or_N = N, T_or_max = max_seqlen, total_tokens.

@@ -29,6 +29,7 @@ EXPORTED = (
     "lightning_attn_decode_step",
     "lightning_attn_decode_step_noalloc",
     "lightning_attn_mixed_step",
+    "lightning_attn_state_prefix",
     "lightning_attn_workspace_size",
     "lightning_attn_check",
     "lightning_attn_status_string",
@@ -58,6 +59,7 @@ def _load():
                                                        vp, vp]
     lib.lightning_attn_mixed_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                               f32, vp, vp, sz, vp, vp]
+    lib.lightning_attn_state_prefix.argtypes = [vp, i32, i32, vp, vp, i32, i32, vp]
     lib.lightning_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
     lib.lightning_attn_workspace_size.restype = sz
     lib.lightning_attn_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint * 4)]
@@ -66,7 +68,8 @@ def _load():
     lib.lightning_attn_last_path.argtypes = []
     lib.lightning_attn_last_path.restype = ctypes.c_char_p
     for f in ("lightning_attn_prefill", "lightning_attn_prefill_varlen", "lightning_attn_decode_step",
-              "lightning_attn_decode_step_noalloc", "lightning_attn_mixed_step", "lightning_attn_check"):
+              "lightning_attn_decode_step_noalloc", "lightning_attn_mixed_step", "lightning_attn_state_prefix",
+              "lightning_attn_check"):
         getattr(lib, f).restype = i32
     return lib
 
@@ -214,6 +217,17 @@ def lightning_attn_mixed_step(q, k, v, g, out, cu_seqlens, cu_seqlens_host, stat
                                         _stream(decode_stream))
     if st != LA_OK:
         raise LightningAttnError(st, "lightning_attn_mixed_step")
+
+
+def lightning_attn_state_prefix(gathered, rank, out, state0=None, stream=None):
+    """out[H, D, D] = state0 + sum over ranks j < rank of gathered[j] (rank order)."""
+    world, H, D, _ = gathered.shape
+    _check_contig(gathered, out)
+    st = _lib.lightning_attn_state_prefix(_ptr(_f32_or_none(gathered)), world, int(rank),
+                                          _ptr(_f32_or_none(state0)), _ptr(_f32_or_none(out)), H, D,
+                                          _stream(stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_state_prefix")
 
 
 def lightning_attn_check(workspace, stream=None, raise_on_error=True):
