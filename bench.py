@@ -509,6 +509,10 @@ def run_gpu(args):
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        # A device-side spin ahead of the first event lets the host queue the first steps, so
+        # the events see the GPU's time and not the first call's marshalling; a host that
+        # cannot keep up in steady state still shows in the timing (and e2e has no hold).
+        torch.cuda._sleep(HOLD_CYCLES)
         e0.record(stream)
         for i in range(args.steps):
             starts[i].record(stream)
@@ -567,6 +571,8 @@ def run_gpu(args):
     if world > 1:
         dist.destroy_process_group()
 
+
+HOLD_CYCLES = 4_000_000   # about 2 ms at the B200's 1965 MHz SM clock
 
 # Source files each measured kernel is built from (a traffic figure is tied to their hash).
 KERNEL_SOURCES = {
