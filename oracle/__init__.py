@@ -15,7 +15,10 @@ computes, and which passage of the pages it follows, is documented there:
     ("MiniMax-Text-01 405B MoE模型架构与训练策略解析", section 2.1);
   * ``quadratic`` -- restatement R1, (phi(Q) phi(K)^T (.) M) V;
   * ``chunked``   -- restatement R2, block-wise intra + inter form for any block size;
-  * ``transform`` -- the output transform alone.
+  * ``transform`` -- the output transform alone;
+  * ``backward_packed`` / ``backward`` -- the gradients of the forward (chain rule through
+    the output transform, the recurrence and the feature map; pinned by finite differences
+    of ``forward_packed``).
 
 Parity pins for every function are in tests/test_oracle_pins.py.
 """
@@ -62,10 +65,12 @@ def _get():
         lib.oracle_quadratic.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
         lib.oracle_chunked.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
         lib.oracle_transform.argtypes = [vp, i64, i32, i32, i32, dbl, vp, vp, i32, vp]
+        lib.oracle_backward_packed.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, i32, i32, dbl,
+                                               vp, vp, vp, vp, vp, vp]
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         for f in (lib.oracle_forward_packed, lib.oracle_prefill, lib.oracle_decode,
-                  lib.oracle_quadratic, lib.oracle_chunked, lib.oracle_transform):
+                  lib.oracle_quadratic, lib.oracle_chunked, lib.oracle_transform, lib.oracle_backward_packed):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -186,3 +191,40 @@ def transform(y, mode, eps=1e-6, norm_weight=None, g=None):
     _get().oracle_transform(_ptr(y), tokens, H, D, mode, eps, _ptr(_c(norm_weight, np.float32)), _ptr(g),
                             dt, _ptr(out))
     return out
+
+
+def backward_packed(q, k, v, g, dout, cu_seqlens, H, D, state_in=None, phi=PHI_SILU, mode=MODE_RMSNORM_GATE,
+                    eps=1e-6, norm_weight=None):
+    """Gradients of forward_packed for the loss with output gradient dout [tokens, H*D].
+
+    q, k, v [tokens, H, D], g and dout [tokens, H*D] (bf16 bits or fp32, all one dtype).
+    Returns fp64 (dq, dk, dv [tokens, H, D], dg [tokens, H*D] or None, dstate [N, H, D, D]).
+    """
+    q, k, v, g, dout = _c(q), _c(k), _c(v), _c(g), _c(dout)
+    dt = _dtype_code(q)
+    cu = _c(cu_seqlens, np.int32)
+    N = cu.size - 1
+    tokens = int(cu[-1]) if N > 0 else 0
+    dq, dk, dv = (np.zeros((tokens, H, D), dtype=np.float64) for _ in range(3))
+    dg = np.zeros((tokens, H * D), dtype=np.float64) if mode == MODE_RMSNORM_GATE else None
+    dst = np.zeros((N, H, D, D), dtype=np.float64)
+    rc = _get().oracle_backward_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout), dt, _ptr(cu), N, H, D,
+                                       _ptr(_c(state_in, np.float32)), phi, mode, eps,
+                                       _ptr(_c(norm_weight, np.float32)), _ptr(dq), _ptr(dk), _ptr(dv),
+                                       _ptr(dg), _ptr(dst))
+    if rc != 0:
+        raise ValueError("oracle_backward_packed rejected its arguments")
+    return dq, dk, dv, dg, dst
+
+
+def backward(q, k, v, g, dout, state_in=None, phi=PHI_SILU, mode=MODE_RMSNORM_GATE, eps=1e-6,
+             norm_weight=None):
+    """Fixed-length batch: q, k, v [B, T, H, D]; g, dout [B, T, H*D]; state_in [B, H, D, D]."""
+    B, T, H, D = q.shape
+    cu = np.arange(B + 1, dtype=np.int32) * T
+    r = lambda a, s: None if a is None else np.reshape(a, s)
+    dq, dk, dv, dg, dst = backward_packed(r(q, (B * T, H, D)), r(k, (B * T, H, D)), r(v, (B * T, H, D)),
+                                          r(g, (B * T, H * D)), r(dout, (B * T, H * D)), cu, H, D, state_in,
+                                          phi, mode, eps, norm_weight)
+    return (dq.reshape(B, T, H, D), dk.reshape(B, T, H, D), dv.reshape(B, T, H, D),
+            None if dg is None else dg.reshape(B, T, H * D), dst)

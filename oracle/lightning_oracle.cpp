@@ -177,6 +177,102 @@ void write_stats(double* stats, const Cmp& o, const Cmp& s) {
   stats[7] = static_cast<double>(s.nonfinite);
 }
 
+// ---------------------------------------------------------------------------------------
+// Backward pass.  The pages print no gradient formulas (training used this operator, per
+// [Arch] section 2.1); what follows is the chain rule applied to the forward above, step
+// by step, in fp64.  For a loss L with dL/do = dO given:
+//
+//   output transform (per token, c over the H*D concatenation, s_c = sigmoid(g_c) with the
+//   gate and 1 without, r = 1/sqrt(mean(y^2) + eps), u_c = dO_c w_c s_c):
+//     RAW:            dy = dO
+//     RMSNORM(_GATE): dy_c = r u_c - r^3 y_c (sum_c' u_c' y_c') / (H*D)
+//     gate:           dg_c = dO_c y_c r w_c s_c (1 - s_c)
+//   recurrence (per head; S_t = S0 + sum_{i<=t} phi(k_i) v_i^T, y_t = S_t^T phi(q_t)):
+//     dphi(q_t) = S_t dy_t
+//     F_t = sum_{i>=t} phi(q_i) dy_i^T      (the same sum taken from the end)
+//     dphi(k_t) = F_t v_t,   dv_t = F_t^T phi(k_t),   dS0 = F_0
+//   feature map: dq = dphi(q) * phi'(q), phi'(x) = sigmoid(x) (1 + x (1 - sigmoid(x))) for
+//   SiLU and 1 for the identity; likewise dk.
+
+// d/dx [x * sigmoid(x)] = sigmoid(x) + x * sigmoid(x) * (1 - sigmoid(x)).
+inline double dfeature(double x, int phi) {
+  if (phi != PHI_SILU) return 1.0;
+  const double s = sigmoid(x);
+  return s * (1.0 + x * (1.0 - s));
+}
+
+// Backward of transform_token for one token: dy (H*D) and, with the gate, dg (H*D).
+void transform_token_backward(const double* y, const void* dout, const void* g, int dtype, int64_t grow,
+                              int HD, int mode, double eps, const float* w, double* dy, double* dg) {
+  if (mode == MODE_RAW) {
+    for (int c = 0; c < HD; ++c) dy[c] = widen(dout, dtype, grow * HD + c);
+    return;
+  }
+  double ss = 0.0;
+  for (int c = 0; c < HD; ++c) ss += y[c] * y[c];
+  const double r = 1.0 / std::sqrt(ss / HD + eps);
+  double dot = 0.0;
+  std::vector<double> u(HD);
+  for (int c = 0; c < HD; ++c) {
+    const double s = (mode == MODE_RMSNORM_GATE) ? sigmoid(widen(g, dtype, grow * HD + c)) : 1.0;
+    const double wc = w ? static_cast<double>(w[c]) : 1.0;
+    const double d = widen(dout, dtype, grow * HD + c);
+    u[c] = d * wc * s;
+    dot += u[c] * y[c];
+    if (mode == MODE_RMSNORM_GATE && dg) dg[c] = d * y[c] * r * wc * s * (1.0 - s);
+  }
+  for (int c = 0; c < HD; ++c) dy[c] = r * u[c] - r * r * r * y[c] * dot / HD;
+}
+
+// Recurrence backward for one head over rows [row0, row0 + n).  S enters as S0 (D x D);
+// dy is the fp64 [tokens, H, D] gradient of the raw output.  Writes dq, dk, dv at the
+// same packed positions and dS0 (D x D).  dy is indexed from the sequence's first row:
+// dy[(t * H + h) * D + j].
+void recur_head_backward(const void* q, const void* k, const void* v, int dtype, int64_t row0, int64_t n,
+                         int H, int D, int h, int phi, const double* S0, const double* dy, double* dq,
+                         double* dk, double* dv, double* dS0) {
+  std::vector<double> S(S0, S0 + static_cast<size_t>(D) * D);
+  std::vector<double> fk(D), vv(D);
+  // forward in time: dphi(q_t) = S_t dy_t, S_t including token t
+  for (int64_t t = 0; t < n; ++t) {
+    const int64_t base = ((row0 + t) * H + h) * static_cast<int64_t>(D);
+    for (int i = 0; i < D; ++i) {
+      fk[i] = feature(widen(k, dtype, base + i), phi);
+      vv[i] = widen(v, dtype, base + i);
+    }
+    for (int i = 0; i < D; ++i)
+      for (int j = 0; j < D; ++j) S[static_cast<size_t>(i) * D + j] += fk[i] * vv[j];
+    for (int i = 0; i < D; ++i) {
+      double a = 0.0;
+      for (int j = 0; j < D; ++j) a += S[static_cast<size_t>(i) * D + j] * dy[(t * H + h) * D + j];
+      dq[base + i] = a * dfeature(widen(q, dtype, base + i), phi);
+    }
+  }
+  // backward in time: F_t = sum_{i >= t} phi(q_i) dy_i^T
+  std::vector<double> F(static_cast<size_t>(D) * D, 0.0), fq(D);
+  for (int64_t t = n - 1; t >= 0; --t) {
+    const int64_t base = ((row0 + t) * H + h) * static_cast<int64_t>(D);
+    for (int i = 0; i < D; ++i) {
+      fq[i] = feature(widen(q, dtype, base + i), phi);
+      fk[i] = feature(widen(k, dtype, base + i), phi);
+      vv[i] = widen(v, dtype, base + i);
+    }
+    for (int i = 0; i < D; ++i)
+      for (int j = 0; j < D; ++j) F[static_cast<size_t>(i) * D + j] += fq[i] * dy[(t * H + h) * D + j];
+    for (int i = 0; i < D; ++i) {
+      double b = 0.0;
+      for (int j = 0; j < D; ++j) b += F[static_cast<size_t>(i) * D + j] * vv[j];
+      dk[base + i] = b * dfeature(widen(k, dtype, base + i), phi);
+    }
+    for (int j = 0; j < D; ++j) {
+      double c = 0.0;
+      for (int i = 0; i < D; ++i) c += F[static_cast<size_t>(i) * D + j] * fk[i];
+      dv[base + j] = c;
+    }
+  }
+  for (size_t i = 0; i < F.size(); ++i) dS0[i] = F[i];
+}
+
 }  // namespace
 
 extern "C" {
@@ -319,6 +415,46 @@ int oracle_transform(const double* y, int64_t tokens, int H, int D, int mode, do
   const int HD = H * D;
 #pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < tokens; ++t) transform_token(y + t * HD, HD, mode, eps, w, g, dtype, t, out + t * HD);
+  return 0;
+}
+
+// Backward of oracle_forward_packed for the loss whose output gradient is dout [tokens, H*D]
+// (same dtype as q).  Recomputes the raw forward y, applies the transform backward per
+// token, then the recurrence backward per head.  Outputs fp64: dq, dk, dv [tokens, H, D],
+// dg [tokens, H*D] (gate mode; may be null otherwise), dstate [N, H, D, D] (the gradient
+// of each sequence's initial state; may be null).
+int oracle_backward_packed(const void* q, const void* k, const void* v, const void* g, const void* dout,
+                           int dtype, const int32_t* cu, int N, int H, int D, const float* state_in, int phi,
+                           int mode, double eps, const float* w, double* dq, double* dk, double* dv,
+                           double* dg, double* dstate) {
+  if (N < 0 || H <= 0 || D <= 0 || !dout || !dq || !dk || !dv) return 1;
+  if (mode == MODE_RMSNORM_GATE && (!g || !dg)) return 1;
+  const int HD = H * D;
+  const int64_t nst = static_cast<int64_t>(H) * D * D;
+  for (int s = 0; s < N; ++s) {
+    const int64_t row0 = cu[s], L = static_cast<int64_t>(cu[s + 1]) - cu[s];
+    if (L < 0) return 1;
+    std::vector<double> S0(nst, 0.0);
+    if (state_in)
+      for (int64_t i = 0; i < nst; ++i) S0[i] = static_cast<double>(state_in[s * nst + i]);
+    // raw forward y, from S0
+    std::vector<double> st(S0), y(static_cast<size_t>(L) * HD), dy(static_cast<size_t>(L) * HD);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h)
+      recur_head(q, k, v, dtype, row0, L, H, D, h, phi, st.data() + static_cast<size_t>(h) * D * D, y.data());
+    // transform backward per token (dy indexed from the sequence's first row)
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < L; ++t)
+      transform_token_backward(y.data() + t * HD, dout, g, dtype, row0 + t, HD, mode, eps, w,
+                               dy.data() + t * HD, dg ? dg + (row0 + t) * HD : nullptr);
+    std::vector<double> dS0(nst);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h)
+      recur_head_backward(q, k, v, dtype, row0, L, H, D, h, phi, S0.data() + static_cast<size_t>(h) * D * D,
+                          dy.data(), dq, dk, dv, dS0.data() + static_cast<size_t>(h) * D * D);
+    if (dstate)
+      for (int64_t i = 0; i < nst; ++i) dstate[s * nst + i] = dS0[i];
+  }
   return 0;
 }
 
