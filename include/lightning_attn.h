@@ -70,7 +70,14 @@ typedef enum { LA_OUT_RAW = 0, LA_OUT_RMSNORM = 1, LA_OUT_RMSNORM_GATE = 2 } la_
 /* SILU: phi(x) = x * sigmoid(x) on q and k.  IDENTITY: phi(x) = x (exact-integer tests). */
 typedef enum { LA_PHI_SILU = 0, LA_PHI_IDENTITY = 1 } la_feature_map;
 
-typedef enum { LA_OP_PREFILL = 0, LA_OP_PREFILL_VARLEN = 1, LA_OP_DECODE = 2, LA_OP_MIXED = 3 } la_op;
+typedef enum {
+  LA_OP_PREFILL = 0,
+  LA_OP_PREFILL_VARLEN = 1,
+  LA_OP_DECODE = 2,
+  LA_OP_MIXED = 3,
+  LA_OP_BACKWARD = 4,
+  LA_OP_BACKWARD_VARLEN = 5
+} la_op;
 
 /*
  * Causal block-wise prefill of B sequences of T tokens each.
@@ -223,12 +230,61 @@ LA_API la_status lightning_attn_state_prefix(const float* gathered, int world, i
                                              float* out, int H, int D, la_stream_t stream);
 
 /*
+ * Backward pass of lightning_attn_prefill: the gradients of a loss with respect to q, k, v,
+ * the gate and the initial state, given the gradient `dout` of its output.  The pages give
+ * no gradient formulas ("MiniMax-Text-01 405B MoE模型架构与训练策略解析" section 2.1 names the
+ * operator as trained); they follow from the forward of "六十四：MiniMax-01" section 3 by the
+ * chain rule.  Per head, with dy the gradient of the raw output y (dy = dout in RAW mode;
+ * through RMSNorm * w * sigmoid(g) otherwise, recomputing y from q, k, v, state_in):
+ *   dphi(q_t) = sum_{i<=t} (dy_t . v_i) phi(k_i) + S0 dy_t
+ *   dphi(k_i) = sum_{t>=i} (v_i . dy_t) phi(q_t)
+ *   dv_i      = sum_{t>=i} (phi(k_i) . phi(q_t)) dy_t,      dS0 = sum_t phi(q_t) dy_t^T
+ * and dq = dphi(q) * phi'(q), dk = dphi(k) * phi'(k).  The three sums run as causal
+ * linear-attention passes of the prefill kernels (the last two on time-reversed copies).
+ *
+ *   q, k, v       [B, T, H, D] dtype, the forward's inputs; dout [B, T, H*D] dtype.
+ *   g             [B, T, H*D] dtype, required iff mode == LA_OUT_RMSNORM_GATE.
+ *   state_in      fp32 [B, H, D, D] the forward's initial states, or NULL (zeros).
+ *   dq, dk, dv    [B, T, H, D] dtype, written (none may alias an input or each other).
+ *   dg            [B, T, H*D] dtype, written iff mode == LA_OUT_RMSNORM_GATE (else ignored).
+ *   dstate_in     fp32 [B, H, D, D] gradient of the initial states, or NULL.
+ *   norm_weight   as the forward (its gradient is not computed).
+ *   workspace     >= lightning_attn_workspace_size(LA_OP_BACKWARD, B, T, 0, H, D, block_size,
+ *                 dtype, mode) bytes, 256-byte aligned; the error record as for the prefill.
+ * Other arguments as lightning_attn_prefill (block_size selects the passes' kernel the same
+ * way).  Returns LA_OK after enqueueing, or an error status with nothing enqueued.
+ */
+LA_API la_status lightning_attn_backward(const void* q, const void* k, const void* v, const void* g,
+                                         const void* dout, const float* state_in, void* dq, void* dk, void* dv,
+                                         void* dg, float* dstate_in, int B, int T, int H, int D, int block_size,
+                                         la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
+                                         const float* norm_weight, void* workspace, size_t workspace_bytes,
+                                         la_stream_t stream);
+
+/*
+ * Backward of lightning_attn_prefill_varlen: as lightning_attn_backward over N packed
+ * sequences (q, k, v, dq, dk, dv [total, H, D]; g, dout, dg [total, H*D]; cu_seqlens DEVICE
+ * int32 [N + 1] as for the forward; state_in, dstate_in [N, H, D, D] or NULL).  Time is
+ * reversed within each sequence.  Workspace: LA_OP_BACKWARD_VARLEN with N, max_seqlen,
+ * total_tokens.
+ */
+LA_API la_status lightning_attn_backward_varlen(const void* q, const void* k, const void* v, const void* g,
+                                                const void* dout, const float* state_in, void* dq, void* dk,
+                                                void* dv, void* dg, float* dstate_in, const int* cu_seqlens,
+                                                int num_seqs, int max_seqlen, int total_tokens, int H, int D,
+                                                int block_size, la_dtype dtype, la_feature_map phi,
+                                                la_out_mode mode, float eps, const float* norm_weight,
+                                                void* workspace, size_t workspace_bytes, la_stream_t stream);
+
+/*
  * Workspace bytes needed by one call (0 on invalid arguments).
  *   op == LA_OP_PREFILL:         B_or_N = B, T_or_max = T, total_tokens ignored.
  *   op == LA_OP_PREFILL_VARLEN:  B_or_N = N, T_or_max = max_seqlen, total_tokens.
  *   op == LA_OP_DECODE:          B_or_N = B, the rest ignored except H, D, dtype, mode.
  *   op == LA_OP_MIXED:           B_or_N = N, T_or_max = longest sequence with more than
  *                                one token (0 if none), total_tokens = all packed tokens.
+ *   op == LA_OP_BACKWARD:        as LA_OP_PREFILL.
+ *   op == LA_OP_BACKWARD_VARLEN: as LA_OP_PREFILL_VARLEN.
  * The size depends on the kernel the call will select (which depends on the device), so
  * query it with the target device current.
  */

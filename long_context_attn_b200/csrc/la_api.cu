@@ -21,6 +21,14 @@ cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, voi
                                 ErrRec* err, cudaStream_t stream);
 cudaError_t launch_norm_gate(const float* y, const void* g, void* out, int64_t tokens, int HD, int mode,
                              float eps, const float* w, la_dtype dt, cudaStream_t stream);
+cudaError_t launch_bwd_norm_gate(const void* y, const void* g, const void* dout, const float* w, void* dy, void* dg,
+                                 int64_t tokens, int HD, int gate, float eps, la_dtype dt, cudaStream_t stream);
+cudaError_t launch_bwd_prep(const void* q, const void* k, const void* v, const void* dy, void* fk, void* rv,
+                            void* rdy, void* rfq, void* rfk, const int* cu, int nseq, int T_fixed, int64_t tokens,
+                            int HD, int phi_identity, la_dtype dt, cudaStream_t stream);
+cudaError_t launch_bwd_post(const void* q, const void* k, void* dq, void* dk, void* dv, const int* cu, int nseq,
+                            int T_fixed, int64_t tokens, int HD, int phi_identity, la_dtype dt, cudaStream_t stream);
+cudaError_t launch_transpose_states(const float* in, float* out, int64_t nmat, int D, cudaStream_t stream);
 }  // namespace la
 
 namespace {
@@ -131,6 +139,84 @@ MixedLayout mixed_layout(int n, int max_pre, int64_t total, int H, int D, int C,
   return m;
 }
 
+// Backward workspace: [prefill part of the raw-mode passes (error record first)]
+// [6 token buffers: dy, phi(k), rho(v), rho(dy), rho(phi(q)), rho(phi(k))] [S0^T states].
+struct BwdLayout {
+  size_t pre, buf, st, total;
+};
+BwdLayout bwd_layout(int nseq, int max_len, int64_t tokens, int H, int D, int C, la_dtype dt) {
+  BwdLayout b{};
+  b.pre = prefill_ws_bytes(choose_path(dt, H, D, C, LA_OUT_RAW), nseq, max_len, tokens, H, D, C, LA_OUT_RAW);
+  b.buf = up256(static_cast<size_t>(tokens) * H * D * (dt == LA_BF16 ? 2 : 4));
+  b.st = up256(sizeof(float) * static_cast<size_t>(nseq) * H * D * D);
+  b.total = b.pre + 6 * b.buf + b.st;
+  return b;
+}
+
+// The backward as a sequence of launches on one stream (see la_backward.cu for the
+// derivation): [forward recompute of raw y, then dy/dg per token] -> prep -> three
+// raw-mode identity-feature passes of the prefill kernel -> post.
+la_status common_backward(const void* q, const void* k, const void* v, const void* g, const void* dout,
+                          const float* state_in, void* dq, void* dk, void* dv, void* dg, float* dstate,
+                          const int* cu, int nseq, int T_fixed, int max_len, int64_t tokens, int H, int D, int C,
+                          la_dtype dt, la_feature_map phi, la_out_mode mode, float eps, const float* w,
+                          void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!valid_enums(dt, phi, mode) || !valid_head(H, D, mode, eps)) return LA_ERR_INVALID_ARG;
+  if (C < 1 || C > 1024 || nseq < 1 || tokens < 0 || max_len < 0) return LA_ERR_INVALID_ARG;
+  if (tokens > 0) {
+    for (const void* p : {q, k, v, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv)})
+      if (!p || !aligned16(p)) return LA_ERR_INVALID_ARG;
+    if (mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g) || !dg || !aligned16(dg))) return LA_ERR_INVALID_ARG;
+  }
+  if ((state_in && !aligned16(state_in)) || (dstate && !aligned16(dstate)) || (w && !aligned16(w)))
+    return LA_ERR_INVALID_ARG;
+  if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;
+  const BwdLayout L = bwd_layout(nseq, max_len, tokens, H, D, C, dt);
+  if (ws_bytes < L.total) return LA_ERR_INVALID_ARG;
+
+  char* base = static_cast<char*>(workspace);
+  void* buf[6];
+  for (int i = 0; i < 6; ++i) buf[i] = base + L.pre + i * L.buf;
+  float* s0t = reinterpret_cast<float*>(base + L.pre + 6 * L.buf);
+  void *dybuf = buf[0], *fk = buf[1], *rv = buf[2], *rdy = buf[3], *rfq = buf[4], *rfk = buf[5];
+  const int HD = H * D;
+  const int phi_id = (phi == LA_PHI_IDENTITY) ? 1 : 0;
+  auto pass = [&](const void* qq, const void* kk, const void* vv, void* out, const float* sin,
+                  float* sout, la_feature_map f) {
+    return common_prefill(qq, kk, vv, nullptr, out, sin, sout, cu, nseq, T_fixed, max_len, tokens, H, D, C, dt, f,
+                          LA_OUT_RAW, eps, nullptr, workspace, L.pre, stream);
+  };
+  la_status st;
+  const void* dy = dout;
+  if (mode != LA_OUT_RAW) {
+    // raw y of the forward (from the same initial state), then dy (in place) and dg
+    if ((st = pass(q, k, v, dybuf, state_in, nullptr, phi)) != LA_OK) return st;
+    if (la::launch_bwd_norm_gate(dybuf, g, dout, w, dybuf, dg, tokens, HD, mode == LA_OUT_RMSNORM_GATE ? 1 : 0,
+                                 eps, dt, stream) != cudaSuccess)
+      return LA_ERR_CUDA;
+    dy = dybuf;
+  }
+  if (la::launch_bwd_prep(q, k, v, dy, fk, rv, rdy, rfq, rfk, cu, nseq, T_fixed, tokens, HD, phi_id, dt, stream) !=
+      cudaSuccess)
+    return LA_ERR_CUDA;
+  const float* s0 = nullptr;
+  if (state_in) {
+    if (la::launch_transpose_states(state_in, s0t, static_cast<int64_t>(nseq) * H, D, stream) != cudaSuccess)
+      return LA_ERR_CUDA;
+    s0 = s0t;
+  }
+  // dphi(q): queries dy, keys v, values phi(k), initial state S0^T
+  if ((st = pass(dy, v, fk, dq, s0, nullptr, LA_PHI_IDENTITY)) != LA_OK) return st;
+  // reversed dphi(k): queries rho(v), keys rho(dy), values rho(phi(q))
+  if ((st = pass(rv, rdy, rfq, dk, nullptr, nullptr, LA_PHI_IDENTITY)) != LA_OK) return st;
+  // reversed dv: queries rho(phi(k)), keys rho(phi(q)), values rho(dy); final state = dS0
+  if ((st = pass(rfk, rfq, rdy, dv, nullptr, dstate, LA_PHI_IDENTITY)) != LA_OK) return st;
+  if (la::launch_bwd_post(q, k, dq, dk, dv, cu, nseq, T_fixed, tokens, HD, phi_id, dt, stream) != cudaSuccess)
+    return LA_ERR_CUDA;
+  return LA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -146,6 +232,33 @@ la_status lightning_attn_prefill(const void* q, const void* k, const void* v, co
   return common_prefill(q, k, v, g, out, state_in, state_out, nullptr, B, T, T, tokens, H, D, block_size, dtype,
                         phi, mode, eps, norm_weight, workspace, workspace_bytes,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status lightning_attn_backward(const void* q, const void* k, const void* v, const void* g, const void* dout,
+                                  const float* state_in, void* dq, void* dk, void* dv, void* dg, float* dstate_in,
+                                  int B, int T, int H, int D, int block_size, la_dtype dtype, la_feature_map phi,
+                                  la_out_mode mode, float eps, const float* norm_weight, void* workspace,
+                                  size_t workspace_bytes, la_stream_t stream) {
+  if (B < 1 || T < 0) return LA_ERR_INVALID_ARG;
+  const int64_t tokens = static_cast<int64_t>(B) * T;
+  if (tokens > INT32_MAX) return LA_ERR_UNSUPPORTED;
+  return common_backward(q, k, v, g, dout, state_in, dq, dk, dv, dg, dstate_in, nullptr, B, T, T, tokens, H, D,
+                         block_size, dtype, phi, mode, eps, norm_weight, workspace, workspace_bytes,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status lightning_attn_backward_varlen(const void* q, const void* k, const void* v, const void* g,
+                                         const void* dout, const float* state_in, void* dq, void* dk, void* dv,
+                                         void* dg, float* dstate_in, const int* cu_seqlens, int num_seqs,
+                                         int max_seqlen, int total_tokens, int H, int D, int block_size,
+                                         la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
+                                         const float* norm_weight, void* workspace, size_t workspace_bytes,
+                                         la_stream_t stream) {
+  if (num_seqs < 1 || !cu_seqlens || !aligned16(cu_seqlens) || total_tokens < 0 || max_seqlen < 0)
+    return LA_ERR_INVALID_ARG;
+  return common_backward(q, k, v, g, dout, state_in, dq, dk, dv, dg, dstate_in, cu_seqlens, num_seqs, 0, max_seqlen,
+                         total_tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight, workspace,
+                         workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 la_status lightning_attn_prefill_varlen(const void* q, const void* k, const void* v, const void* g, void* out,
@@ -261,6 +374,12 @@ size_t lightning_attn_workspace_size(la_op op, int B_or_N, int T_or_max, int tot
   if (op == LA_OP_PREFILL_VARLEN) {
     if (total_tokens < 0) return 0;
     return prefill_ws_bytes(path, B_or_N, T_or_max, total_tokens, H, D, block_size, mode);
+  }
+  if (op == LA_OP_BACKWARD)
+    return bwd_layout(B_or_N, T_or_max, static_cast<int64_t>(B_or_N) * T_or_max, H, D, block_size, dtype).total;
+  if (op == LA_OP_BACKWARD_VARLEN) {
+    if (total_tokens < 0) return 0;
+    return bwd_layout(B_or_N, T_or_max, total_tokens, H, D, block_size, dtype).total;
   }
   return 0;
 }

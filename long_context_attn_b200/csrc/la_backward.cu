@@ -1,0 +1,302 @@
+// Backward pass of the Lightning Attention forward: the element-wise and per-token kernels
+// around three causal linear-attention passes (which run on the prefill kernels).
+//
+// The pages give no gradient formulas ("MiniMax-Text-01 405B MoE模型架构与训练策略解析",
+// section 2.1, names the operator used in training); the chain rule through the forward
+// of "六十四：MiniMax-01" section 3 (S_t = S0 + sum_{i<=t} phi(k_i) v_i^T, y_t = S_t^T phi(q_t))
+// gives, per head, with dy the gradient of the raw output:
+//   dphi(q_t) = sum_{i<=t} (dy_t . v_i) phi(k_i) + S0 dy_t
+//   dphi(k_i) = sum_{t>=i} (v_i . dy_t) phi(q_t)
+//   dv_i      = sum_{t>=i} (phi(k_i) . phi(q_t)) dy_t
+//   dS0       = sum_t phi(q_t) dy_t^T
+// Each line is a causal linear attention with the identity feature map: the first runs
+// forward in time (queries dy, keys v, values phi(k), initial state S0^T); the other two
+// run on the time-reversed sequences (queries rho(v), keys rho(dy), values rho(phi(q)); and
+// queries rho(phi(k)), keys rho(phi(q)), values rho(dy), whose final state is dS0).  The
+// kernels here supply what those passes take and finish what they give:
+//   bwd_norm_gate_kernel  dy and dg from dout through RMSNorm(y) * w * sigmoid(g) (per token)
+//   bwd_prep_kernel       phi(k) and the reversed copies rho(v), rho(dy), rho(phi(q)), rho(phi(k))
+//   bwd_post_kernel       dq = dphi(q) * phi'(q); un-reverses dk (times phi'(k)) and dv in place
+//   transpose_states      S0^T for the first pass
+// All of them are HBM-streaming kernels: 16-byte vectors, grid-stride loops over rows.
+#include "la_common.cuh"
+
+namespace la {
+namespace {
+
+constexpr int kVec = 8;   // elements per vector (16 bytes of bf16)
+
+template <typename T> struct Vec8;
+template <> struct Vec8<uint16_t> {
+  __device__ __forceinline__ static void load(const uint16_t* p, float* f) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = bf16_bits_to_f32(static_cast<uint16_t>(w[i] & 0xFFFFu));
+      f[2 * i + 1] = bf16_bits_to_f32(static_cast<uint16_t>(w[i] >> 16));
+    }
+  }
+  __device__ __forceinline__ static void store(uint16_t* p, const float* f) {
+    uint4 u;
+    u.x = pack_bf16x2(f[0], f[1]);
+    u.y = pack_bf16x2(f[2], f[3]);
+    u.z = pack_bf16x2(f[4], f[5]);
+    u.w = pack_bf16x2(f[6], f[7]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
+template <> struct Vec8<float> {
+  __device__ __forceinline__ static void load(const float* p, float* f) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+  __device__ __forceinline__ static void store(float* p, const float* f) {
+    *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<float4*>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
+  }
+};
+
+__device__ __forceinline__ float feature(float x, int phi_identity) {
+  return phi_identity ? x : silu_accurate(x);
+}
+// d/dx [x sigmoid(x)] = sigmoid(x) (1 + x (1 - sigmoid(x)))
+__device__ __forceinline__ float dfeature(float x, int phi_identity) {
+  if (phi_identity) return 1.0f;
+  const float s = sigmoid_accurate(x);
+  return s * (1.0f + x * (1.0f - s));
+}
+
+// Row `row` of the packed tokens: first row and one-past-last row of its sequence.
+__device__ __forceinline__ void seq_bounds(const int* cu, int nseq, int T_fixed, int64_t row, int64_t& lo,
+                                           int64_t& hi) {
+  if (!cu) {
+    const int64_t s = row / T_fixed;
+    lo = s * T_fixed;
+    hi = lo + T_fixed;
+    return;
+  }
+  int a = 0, b = nseq;   // largest s with cu[s] <= row; empty sequences are skipped
+  while (b - a > 1) {
+    const int m = (a + b) >> 1;
+    if (__ldg(cu + m) <= row) a = m; else b = m;
+  }
+  lo = __ldg(cu + a);
+  hi = __ldg(cu + a + 1);
+}
+
+// One CTA per token.  RAW is not launched (dy = dout).  With r = 1/sqrt(mean(y^2) + eps),
+// s = sigmoid(g) (1 without the gate) and u = dout * w * s:
+//   dy = r u - r^3 y (sum u y) / HD,    dg = dout * y * r * w * s * (1 - s).
+// y and dy may be the same buffer (each element is read by the thread that writes it).
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_norm_gate_kernel(const T* y, const T* __restrict__ g,
+                                                            const T* __restrict__ dout, const float* __restrict__ w,
+                                                            T* dy, T* __restrict__ dg, int HD, int gate, float eps) {
+  __shared__ float red[2][8];
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * HD;
+  float ss = 0.f, su = 0.f;
+  for (int c = threadIdx.x * kVec; c < HD; c += blockDim.x * kVec) {
+    float yv[kVec], dv[kVec], gv[kVec];
+    Vec8<T>::load(y + base + c, yv);
+    Vec8<T>::load(dout + base + c, dv);
+    if (gate) Vec8<T>::load(g + base + c, gv);
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+      const float s = gate ? sigmoid_accurate(gv[i]) : 1.0f;
+      const float u = dv[i] * (w ? __ldg(w + c + i) : 1.0f) * s;
+      ss = fmaf(yv[i], yv[i], ss);
+      su = fmaf(u, yv[i], su);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    su += __shfl_xor_sync(0xffffffffu, su, o);
+  }
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if ((threadIdx.x & 31) == 0) { red[0][warp] = ss; red[1][warp] = su; }
+  __syncthreads();
+  ss = 0.f; su = 0.f;
+  for (int i = 0; i < nw; ++i) { ss += red[0][i]; su += red[1][i]; }
+  const float r = 1.0f / sqrtf(ss / static_cast<float>(HD) + eps);
+  const float coef = r * r * r * su / static_cast<float>(HD);
+  for (int c = threadIdx.x * kVec; c < HD; c += blockDim.x * kVec) {
+    float yv[kVec], dv[kVec], gv[kVec], o[kVec], og[kVec];
+    Vec8<T>::load(y + base + c, yv);
+    Vec8<T>::load(dout + base + c, dv);
+    if (gate) Vec8<T>::load(g + base + c, gv);
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+      const float s = gate ? sigmoid_accurate(gv[i]) : 1.0f;
+      const float wc = w ? __ldg(w + c + i) : 1.0f;
+      o[i] = r * dv[i] * wc * s - coef * yv[i];
+      og[i] = dv[i] * yv[i] * r * wc * s * (1.0f - s);
+    }
+    Vec8<T>::store(dy + base + c, o);
+    if (gate) Vec8<T>::store(dg + base + c, og);
+  }
+}
+
+// Per 8-element vector of row `row`: fk[row] = phi(k); at the mirrored row m of the same
+// sequence, rv[m] = v, rdy[m] = dy, rfq[m] = phi(q), rfk[m] = phi(k).
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                       const T* __restrict__ v, const T* __restrict__ dy,
+                                                       T* __restrict__ fk, T* __restrict__ rv, T* __restrict__ rdy,
+                                                       T* __restrict__ rfq, T* __restrict__ rfk, const int* cu,
+                                                       int nseq, int T_fixed, int64_t tokens, int HD,
+                                                       int phi_identity) {
+  const int vpr = HD / kVec;
+  const int64_t n = tokens * vpr;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / vpr;
+    const int c = static_cast<int>(i - row * vpr) * kVec;
+    int64_t lo, hi;
+    seq_bounds(cu, nseq, T_fixed, row, lo, hi);
+    const int64_t m = lo + hi - 1 - row;
+    if (row < lo || row >= hi || m < 0 || m >= tokens) continue;   // malformed cu_seqlens (the passes report it)
+    const int64_t src = row * HD + c, dst = m * HD + c;
+    float a[kVec], b[kVec];
+    Vec8<T>::load(q + src, a);
+    Vec8<T>::load(k + src, b);
+#pragma unroll
+    for (int j = 0; j < kVec; ++j) { a[j] = feature(a[j], phi_identity); b[j] = feature(b[j], phi_identity); }
+    Vec8<T>::store(fk + src, b);
+    Vec8<T>::store(rfk + dst, b);
+    Vec8<T>::store(rfq + dst, a);
+    Vec8<T>::load(v + src, a);
+    Vec8<T>::store(rv + dst, a);
+    Vec8<T>::load(dy + src, a);
+    Vec8<T>::store(rdy + dst, a);
+  }
+}
+
+// dq *= phi'(q) in place.  dk and dv hold the reversed-time results: the thread of the
+// earlier row of each mirrored pair swaps the pair (dk times phi'(k) at its new row).
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_post_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                       T* __restrict__ dq, T* __restrict__ dk, T* __restrict__ dv,
+                                                       const int* cu, int nseq, int T_fixed, int64_t tokens,
+                                                       int HD, int phi_identity) {
+  const int vpr = HD / kVec;
+  const int64_t n = tokens * vpr;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / vpr;
+    const int c = static_cast<int>(i - row * vpr) * kVec;
+    int64_t lo, hi;
+    seq_bounds(cu, nseq, T_fixed, row, lo, hi);
+    const int64_t m = lo + hi - 1 - row;
+    if (row < lo || row >= hi || m < 0 || m >= tokens) continue;   // malformed cu_seqlens (the passes report it)
+    const int64_t a0 = row * HD + c, b0 = m * HD + c;
+    float x[kVec], d[kVec];
+    if (!phi_identity) {
+      Vec8<T>::load(q + a0, x);
+      Vec8<T>::load(dq + a0, d);
+#pragma unroll
+      for (int j = 0; j < kVec; ++j) d[j] *= dfeature(x[j], 0);
+      Vec8<T>::store(dq + a0, d);
+    }
+    if (row > m) continue;
+    float ka[kVec], kb[kVec], da[kVec], db[kVec];
+    Vec8<T>::load(dk + a0, da);
+    Vec8<T>::load(dk + b0, db);
+    if (!phi_identity) {
+      Vec8<T>::load(k + a0, ka);
+      Vec8<T>::load(k + b0, kb);
+#pragma unroll
+      for (int j = 0; j < kVec; ++j) { db[j] *= dfeature(ka[j], 0); da[j] *= dfeature(kb[j], 0); }
+    }
+    Vec8<T>::store(dk + a0, db);
+    if (row != m) Vec8<T>::store(dk + b0, da);
+    if (row != m) {
+      Vec8<T>::load(dv + a0, da);
+      Vec8<T>::load(dv + b0, db);
+      Vec8<T>::store(dv + a0, db);
+      Vec8<T>::store(dv + b0, da);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) transpose_states_kernel(const float* __restrict__ in, float* __restrict__ out,
+                                                               int64_t nmat, int D) {
+  const int64_t n = nmat * D * D;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t mtx = i / (static_cast<int64_t>(D) * D);
+    const int r = static_cast<int>((i / D) % D), c = static_cast<int>(i % D);
+    out[(mtx * D + c) * D + r] = in[i];
+  }
+}
+
+int grid_for(int64_t n) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = (n + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sms) * 8;   // 8 resident CTAs of 256 threads per SM
+  return static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_norm_gate(const void* y, const void* g, const void* dout, const float* w, void* dy, void* dg,
+                                 int64_t tokens, int HD, int gate, float eps, la_dtype dt, cudaStream_t stream) {
+  if (tokens == 0) return cudaSuccess;
+  if (dt == LA_BF16)
+    bwd_norm_gate_kernel<uint16_t><<<static_cast<unsigned>(tokens), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(y), static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(dout), w,
+        static_cast<uint16_t*>(dy), static_cast<uint16_t*>(dg), HD, gate, eps);
+  else
+    bwd_norm_gate_kernel<float><<<static_cast<unsigned>(tokens), 256, 0, stream>>>(
+        static_cast<const float*>(y), static_cast<const float*>(g), static_cast<const float*>(dout), w,
+        static_cast<float*>(dy), static_cast<float*>(dg), HD, gate, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_prep(const void* q, const void* k, const void* v, const void* dy, void* fk, void* rv,
+                            void* rdy, void* rfq, void* rfk, const int* cu, int nseq, int T_fixed, int64_t tokens,
+                            int HD, int phi_identity, la_dtype dt, cudaStream_t stream) {
+  const int64_t n = tokens * (HD / kVec);
+  if (n == 0) return cudaSuccess;
+  if (dt == LA_BF16)
+    bwd_prep_kernel<uint16_t><<<grid_for(n), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
+        static_cast<const uint16_t*>(dy), static_cast<uint16_t*>(fk), static_cast<uint16_t*>(rv),
+        static_cast<uint16_t*>(rdy), static_cast<uint16_t*>(rfq), static_cast<uint16_t*>(rfk), cu, nseq, T_fixed,
+        tokens, HD, phi_identity);
+  else
+    bwd_prep_kernel<float><<<grid_for(n), 256, 0, stream>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        static_cast<const float*>(dy), static_cast<float*>(fk), static_cast<float*>(rv), static_cast<float*>(rdy),
+        static_cast<float*>(rfq), static_cast<float*>(rfk), cu, nseq, T_fixed, tokens, HD, phi_identity);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_post(const void* q, const void* k, void* dq, void* dk, void* dv, const int* cu, int nseq,
+                            int T_fixed, int64_t tokens, int HD, int phi_identity, la_dtype dt, cudaStream_t stream) {
+  const int64_t n = tokens * (HD / kVec);
+  if (n == 0) return cudaSuccess;
+  if (dt == LA_BF16)
+    bwd_post_kernel<uint16_t><<<grid_for(n), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<uint16_t*>(dq),
+        static_cast<uint16_t*>(dk), static_cast<uint16_t*>(dv), cu, nseq, T_fixed, tokens, HD, phi_identity);
+  else
+    bwd_post_kernel<float><<<grid_for(n), 256, 0, stream>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<float*>(dq),
+        static_cast<float*>(dk), static_cast<float*>(dv), cu, nseq, T_fixed, tokens, HD, phi_identity);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_states(const float* in, float* out, int64_t nmat, int D, cudaStream_t stream) {
+  const int64_t n = nmat * D * D;
+  if (n == 0) return cudaSuccess;
+  transpose_states_kernel<<<grid_for(n), 256, 0, stream>>>(in, out, nmat, D);
+  return cudaGetLastError();
+}
+
+}  // namespace la

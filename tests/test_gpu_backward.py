@@ -1,0 +1,110 @@
+"""GPU parity of the backward pass against the oracle's fp64 gradients.
+
+Every gradient (dq, dk, dv, the gate's dg and the initial state's dS0) is compared element
+by element with the oracle (which finite differences of the forward pin) at the forward's
+tolerance: bf16 2e-2 * max|ref|, fp32 1e-4 * max|ref|.  Cases span several blocks with a
+ragged tail, both tensor-core block sizes, the three output modes, a norm weight, initial
+states, packed sequences with an empty and a one-token sequence, and the fp32 path.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests._helpers import assert_close, mode_code, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+def _la():
+    from long_context_attn_b200 import lightning_attn as la
+    return la
+
+
+def _run_fixed(B, T, H, D, C, dtype, mode, with_state, seed, expect=None):
+    import torch
+    la = _la()
+    m = mode_code(mode)
+    q, k, v, g = synth.prefill_inputs(seed, B * T, H, D, dtype, 0.5, True)
+    dout = synth.normal(seed, 21, (B * T, H * D), 1.0, dtype)
+    s0 = synth.normal(seed, 22, (B, H, D, D), 0.05, "f32") if with_state else None
+    w = (1.0 + 0.2 * synth.normal(seed, 23, (H * D,), 1.0, "f32")).astype(np.float32) if m else None
+    shp, gshp = (B, T, H, D), (B, T, H * D)
+    dq_, dk_, dv_, dg_ = (to_dev(a).reshape(shp if i < 3 else gshp) for i, a in enumerate((q, k, v, g)))
+    ddo = to_dev(dout).reshape(gshp)
+    gq, gk, gv = (torch.full_like(dq_, float("nan")) for _ in range(3))
+    gg = torch.full_like(dg_, float("nan")) if m == la.LA_OUT_RMSNORM_GATE else None
+    gs = torch.full((B, H, D, D), float("nan"), dtype=torch.float32, device="cuda")
+    ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD, B, T, 0, H, D, C, la._dtype(dq_), m))
+    la.lightning_attn_backward(dq_, dk_, dv_, dg_ if m == la.LA_OUT_RMSNORM_GATE else None, ddo, gq, gk, gv, dg=gg,
+                               state_in=None if s0 is None else to_dev(s0), dstate_in=gs, block_size=C, mode=m,
+                               norm_weight=None if w is None else to_dev(w), workspace=ws)
+    if expect:
+        assert la.lightning_attn_last_path() == expect
+    la.lightning_attn_check(ws)
+    r = lambda a, s: a.reshape(s)
+    ref = oracle.backward(r(q, shp), r(k, shp), r(v, shp), r(g, gshp) if m == la.LA_OUT_RMSNORM_GATE else None,
+                          r(dout, gshp), state_in=s0, mode=m, norm_weight=w)
+    assert_close(to_host(gq), ref[0], dtype, "dq")
+    assert_close(to_host(gk), ref[1], dtype, "dk")
+    assert_close(to_host(gv), ref[2], dtype, "dv")
+    if gg is not None:
+        assert_close(to_host(gg), ref[3], dtype, "dg")
+    assert_close(to_host(gs), ref[4], dtype, "dstate")
+
+
+@pytest.mark.parametrize("C", [128, 256])
+@pytest.mark.parametrize("mode", ["raw", "rmsnorm", "rmsnorm_gate"])
+def test_backward_tc_fixed(C, mode, cuda_device):
+    _run_fixed(2, 700, 8, 128, C, "bf16", mode, True, 3001 + C, expect="tcgen05")
+
+
+@pytest.mark.parametrize("T", [1, 33, 256, 1000])
+def test_backward_tc_lengths(T, cuda_device):
+    _run_fixed(1, T, 8, 128, 256, "bf16", "rmsnorm_gate", False, 3101 + T, expect="tcgen05")
+
+
+def test_backward_fp32_path(cuda_device):
+    _run_fixed(2, 150, 4, 64, 64, "f32", "rmsnorm_gate", True, 3201, expect="simt")
+
+
+@pytest.mark.parametrize("C", [128, 256])
+def test_backward_varlen(C, cuda_device):
+    import torch
+    la = _la()
+    H, D = 8, 128
+    lens = [300, 0, 257, 1, 31, 129]
+    tot = sum(lens)
+    cu = synth.cu_seqlens_of(lens)
+    n = len(lens)
+    q, k, v, g = synth.prefill_inputs(3301, tot, H, D, "bf16", 0.5, True)
+    dout = synth.normal(3301, 21, (tot, H * D), 1.0, "bf16")
+    s0 = synth.normal(3301, 22, (n, H, D, D), 0.05, "f32")
+    dq_, dk_, dv_, dg_, ddo = (to_dev(a) for a in (q, k, v, g, dout))
+    gq, gk, gv = (torch.full_like(dq_, float("nan")) for _ in range(3))
+    gg = torch.full_like(dg_, float("nan"))
+    gs = torch.full((n, H, D, D), float("nan"), dtype=torch.float32, device="cuda")
+    ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD_VARLEN, n, max(lens), tot, H, D, C,
+                                                           la.LA_BF16, la.LA_OUT_RMSNORM_GATE))
+    la.lightning_attn_backward_varlen(dq_, dk_, dv_, dg_, ddo, gq, gk, gv, torch.from_numpy(cu).cuda(), max(lens),
+                                      dg=gg, state_in=to_dev(s0), dstate_in=gs, block_size=C, workspace=ws)
+    assert la.lightning_attn_last_path() == "tcgen05"
+    la.lightning_attn_check(ws)
+    ref = oracle.backward_packed(q, k, v, g, dout, cu, H, D, state_in=s0)
+    for got, want, name in zip((gq, gk, gv, gg, gs), ref, ("dq", "dk", "dv", "dg", "dstate")):
+        assert_close(to_host(got), want, "bf16", name)
+
+
+def test_backward_rejects_bad_arguments(cuda_device):
+    import torch
+    la = _la()
+    B, T, H, D = 1, 64, 8, 128
+    x = torch.zeros((B, T, H, D), dtype=torch.bfloat16, device="cuda")
+    gx = torch.zeros((B, T, H * D), dtype=torch.bfloat16, device="cuda")
+    ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD, B, T, 0, H, D, 256, la.LA_BF16,
+                                                           la.LA_OUT_RMSNORM_GATE))
+    d = [torch.empty_like(x) for _ in range(3)]
+    with pytest.raises(la.LightningAttnError):       # gate mode without dg
+        la.lightning_attn_backward(x, x, x, gx, gx, *d, dg=None, workspace=ws)
+    with pytest.raises(la.LightningAttnError):       # workspace too small
+        la.lightning_attn_backward(x, x, x, gx, gx, *d, dg=torch.empty_like(gx), workspace=ws[:1024])
