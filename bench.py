@@ -346,6 +346,72 @@ class VarlenCase:
                 "l2": "inputs larger than L2 (%.1f GB per step), no flush" % (self.alg_bytes / 1e9)}
 
 
+class BackwardCase:
+    """The backward of one long prefill: gradients of q, k, v and the gate from dout."""
+
+    def __init__(self, name, w, device, rank):
+        import torch
+        from long_context_attn_b200 import lightning_attn as la
+        self.la, self.w = la, w
+        T, H, D, self.C = w.T, w.H, w.D, w.block_size
+        self.T, self.H, self.D = T, H, D
+        t0 = time.time()
+        q, k, v, g = synth.prefill_inputs(w.seed + 1000 * rank, T, H, D, "bf16", w.qkv_scale, True)
+        dout = synth.normal(w.seed + 1000 * rank, synth.STREAM_DOUT, (T, H * D), 1.0, "bf16")
+        self.gen_s = time.time() - t0
+
+        def pin(a):
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+        self.h_in = [pin(a) for a in (q, k, v, g, dout)]
+        del q, k, v, g, dout
+        shapes = [(1, T, H, D)] * 3 + [(1, T, H * D)] * 2
+        self.d_in = [h.to(device).view(s) for h, s in zip(self.h_in, shapes)]
+        self.d_out = [torch.empty(s, dtype=torch.bfloat16, device=device) for s in shapes[:4]]
+        self.h_out = [torch.empty(s, dtype=torch.bfloat16).pin_memory() for s in shapes[:4]]
+        nbytes = la.lightning_attn_workspace_size(la.LA_OP_BACKWARD, 1, T, 0, H, D, self.C, la.LA_BF16,
+                                                  la.LA_OUT_RMSNORM_GATE)
+        self.ws = la.new_workspace(nbytes, device)
+        self.tokens = T
+        # inputs q, k, v, g, dout read and dq, dk, dv, dg written once: the bytes any backward moves
+        self.alg_bytes = T * 9 * H * D * 2
+        # the forward recompute plus three passes of the same linear attention
+        self.alg_flops, self.issued_flops = (4 * x * T for x in _flops_per_token(H, D, self.C))
+        self.launches_per_step = 7      # recompute, norm/gate backward, prep, three passes, post
+        self.h2d = sum(t.numel() * 2 for t in self.h_in)
+        self.d2h = sum(t.numel() * 2 for t in self.h_out)
+
+    def step(self):
+        q, k, v, g, dout = self.d_in
+        dq, dk, dv, dg = self.d_out
+        self.la.lightning_attn_backward(q, k, v, g, dout, dq, dk, dv, dg=dg, block_size=self.C, workspace=self.ws)
+
+    def e2e_step(self):
+        for d, h in zip(self.d_in, self.h_in):
+            d.view(-1).copy_(h.view(-1), non_blocking=True)
+        self.step()
+        for h, d in zip(self.h_out, self.d_out):
+            h.copy_(d, non_blocking=True)
+
+    def check(self):
+        self.la.lightning_attn_check(self.ws)
+
+    def oracle_sample(self, tokens):
+        """fp64 oracle backward on the first `tokens` rows of the same workload (all heads)."""
+        import oracle
+        w = self.w
+        q, k, v, g = synth.prefill_inputs(w.seed, tokens, w.H, w.D, "bf16", w.qkv_scale, True)
+        dout = synth.normal(w.seed, synth.STREAM_DOUT, (tokens, w.H * w.D), 1.0, "bf16")
+        t0 = time.perf_counter()
+        oracle.backward(q[None], k[None], v[None], g[None], dout[None])
+        return time.perf_counter() - t0
+
+    def describe(self):
+        return {"workload": self.w.name, "B": 1, "T": self.T, "H": self.H, "D": self.D, "block_size": self.C,
+                "mode": "rmsnorm_gate", "grads": "dq, dk, dv, dg",
+                "l2": "inputs larger than L2 (%.1f GB per step), no flush" % (self.alg_bytes / 1e9)}
+
+
 class MixedCase:
     """One serving step: 256 sequences decode a token each while 2 others prefill a 4096-token
     chunk from their state; prefill and decode on two streams, states in a pool (slots in a
@@ -452,6 +518,8 @@ def _make_case(name, device, rank):
         return MixedCase(name, w, device, rank)
     if w.kind == "decode":
         return DecodeCase(name, w, device, rank)
+    if w.kind == "backward":
+        return BackwardCase(name, w, device, rank)
     raise SystemExit(f"workload {name} is not a bench workload")
 
 
@@ -551,10 +619,13 @@ def run_gpu(args):
             "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded SplitMix64/Box-Muller)",
             "config": dict(case.describe(), parallelism=f"replicas x{world} (independent sequences, no collective)"),
-            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": _traffic(args.workload),
-                         "peak_source": peaks["source"], "launch_ms": launch_ms,
-                         "algorithmic_bytes_per_launch": case.alg_bytes},
+            "roofline": dict({"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": _traffic(args.workload),
+                              "peak_source": peaks["source"], "launch_ms": launch_ms,
+                              "algorithmic_bytes_per_launch": case.alg_bytes},
+                             **({"scope": "one backward call (7 kernels); algorithmic bytes = its inputs "
+                                          "read and gradients written once"}
+                                if isinstance(case, BackwardCase) else {})),
             "tensor": {"algorithmic_tflops": case.alg_flops / (launch_ms / 1e3) / 1e12,
                        "issued_tflops": case.issued_flops / (launch_ms / 1e3) / 1e12,
                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -578,6 +649,7 @@ HOLD_CYCLES = 4_000_000   # about 2 ms at the B200's 1965 MHz SM clock
 KERNEL_SOURCES = {
     "prefill": ("la_prefill_tc.cu", "la_sm100.cuh", "la_common.cuh"),
     "decode": ("la_decode.cu", "la_common.cuh"),
+    "backward": ("la_backward.cu", "la_api.cu", "la_prefill_tc.cu", "la_sm100.cuh", "la_common.cuh"),
 }
 
 
@@ -598,7 +670,7 @@ def _traffic(workload):
     if not os.path.exists(path):
         return None
     entry = json.load(open(path)).get(workload)
-    kind = "decode" if workload.startswith("decode") else "prefill"
+    kind = next((k for k in ("decode", "backward") if workload.startswith(k)), "prefill")
     if not entry or entry.get("kernel_source_hash") != kernel_source_hash(kind):
         return None
     return entry["bytes_per_launch"]
@@ -617,6 +689,12 @@ def _cpu_baseline(case):
         return {"value": case.total / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
                 "sample": f"the whole {case.w.name} step ({case.total} tokens, all {case.w.H} heads), fp64 "
                           f"({dt:.1f} s)"}
+    if isinstance(case, BackwardCase):
+        n = min(16384, case.T)
+        dt = case.oracle_sample(n)
+        return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                "sample": f"first {n} tokens of the {case.w.name} workload, all {case.H} heads, fp64 backward "
+                          f"(forward recompute, norm/gate backward, both scans) ({dt:.1f} s)"}
     if isinstance(case, VarlenCase):
         dt, n = case.oracle_sample(131072)
         return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
@@ -635,7 +713,16 @@ def run_reference(args):
         return
     import oracle
     w = synth.WORKLOADS[args.workload]
-    if w.kind in ("prefill", "varlen", "mixed"):
+    if w.kind == "backward":
+        n = 512
+        q, k, v, g = synth.prefill_inputs(w.seed, n, w.H, w.D, w.dtype, w.qkv_scale, True)
+        dout = synth.normal(w.seed, synth.STREAM_DOUT, (n, w.H * w.D), 1.0, w.dtype)
+
+        def step():
+            oracle.backward(q[None], k[None], v[None], g[None], dout[None])
+        unit_per_step = n
+        sample = f"first {n} tokens of {w.name} (all {w.H} heads) per step, fp64 backward"
+    elif w.kind in ("prefill", "varlen", "mixed"):
         n = 1024
         q, k, v, g = synth.prefill_inputs(w.seed, n, w.H, w.D, w.dtype, w.qkv_scale, True)
 
@@ -678,7 +765,8 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="prefill_128k",
-                    choices=["prefill_8k", "prefill_128k", "varlen_16", "decode_256", "mixed_256"])
+                    choices=["prefill_8k", "prefill_128k", "varlen_16", "decode_256", "mixed_256", "backward_8k",
+                             "backward_128k"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     args = ap.parse_args()

@@ -3,14 +3,15 @@
 This module draws numbers only; it holds none of the attention arithmetic.  The
 generator itself is C (``synth.c``: SplitMix64 words + Box-Muller normals, a pure
 function of (seed, stream, element index)); this file loads it with ctypes and
-describes the five workloads (shapes, value distributions, seeds).
+describes the bench and test workloads (shapes, value distributions, seeds).
 
 Workload recipes (the Lightning Attention forward of MiniMax-01; the pages give
 no data, so every input is synthetic):
   * q, k, v ~ scale * N(0, 1), g ~ N(0, 1), rounded to the tensor dtype;
   * prior decode state S ~ N(0, 1) / sqrt(head_dim), fp32;
   * varlen lengths ~ U{1000..32768};
-  * config k uses seed 1000 + k; streams q=0, k=1, v=2, g=3, S=4, lengths=5.
+  * the backward's output gradient dout ~ N(0, 1) (bf16);
+  * config k uses seed 1000 + k; streams q=0, k=1, v=2, g=3, S=4, lengths=5, dout=6.
 """
 from __future__ import annotations
 
@@ -26,7 +27,7 @@ _SRC = os.path.join(_HERE, "synth.c")
 _LIB_PATH = os.path.join(_HERE, "libla_synth.so")
 _lib = None
 
-STREAM_Q, STREAM_K, STREAM_V, STREAM_G, STREAM_S, STREAM_LEN = 0, 1, 2, 3, 4, 5
+STREAM_Q, STREAM_K, STREAM_V, STREAM_G, STREAM_S, STREAM_LEN, STREAM_DOUT = 0, 1, 2, 3, 4, 5, 6
 
 
 def build(force: bool = False) -> str:
@@ -114,7 +115,7 @@ def f32_to_bf16(a: np.ndarray) -> np.ndarray:
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str              # 'prefill' | 'varlen' | 'decode' | 'mixed'
+    kind: str              # 'prefill' | 'varlen' | 'decode' | 'mixed' | 'backward'
     seed: int
     B: int                 # batch (prefill), number of sequences (varlen / decode)
     T: int                 # tokens per sequence (prefill); 0 otherwise
@@ -130,7 +131,7 @@ class Workload:
     n_prefill: int = 0     # mixed: number of prefill chunks (of T tokens) among B decode sequences
 
 
-# The five workloads of the Lightning Attention forward (seed 1000 + k).
+# The workloads of the Lightning Attention forward and its backward (seed 1000 + k).
 WORKLOADS = {
     "tiny_f32": Workload("tiny_f32", "prefill", 1001, 1, 512, 2, 64, 64, "f32", "raw", 1.0),
     "prefill_8k": Workload("prefill_8k", "prefill", 1002, 1, 8192, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5),
@@ -142,6 +143,11 @@ WORKLOADS = {
     # chunk from their state (chunked prefill), all packed into one batch.
     "mixed_256": Workload("mixed_256", "mixed", 1006, 256, 4096, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5,
                           n_prefill=2),
+    # The backward of the 128K prefill (gradients of q, k, v and the gate from dout ~ N(0, 1)),
+    # and an 8K version for captures.
+    "backward_128k": Workload("backward_128k", "backward", 1007, 1, 131072, 64, 128, 256, "bf16", "rmsnorm_gate",
+                              0.5),
+    "backward_8k": Workload("backward_8k", "backward", 1008, 1, 8192, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5),
 }
 
 

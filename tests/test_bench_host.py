@@ -4,6 +4,8 @@ import os
 import subprocess
 import sys
 
+import pytest
+
 import bench
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -28,9 +30,10 @@ def test_clock_summary_parses_nvidia_smi_csv():
     assert s["reasons"] == ["sw_power_cap"]
 
 
-def test_reference_arm_prints_one_json_line():
+@pytest.mark.parametrize("workload", ["prefill_8k", "backward_8k"])
+def test_reference_arm_prints_one_json_line(workload):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                        "--warmup", "0", "--workload", "prefill_8k"], capture_output=True, text=True, timeout=600)
+                        "--warmup", "0", "--workload", workload], capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr
     lines = [l for l in r.stdout.splitlines() if l.strip()]
     assert len(lines) == 1
@@ -45,7 +48,15 @@ def test_traffic_is_dropped_when_kernel_source_changes(tmp_path, monkeypatch):
     for wl, entry in t.items():
         if wl.startswith("_"):
             continue
-        kind = "decode" if wl.startswith("decode") else "prefill"
+        kind = next((k for k in ("decode", "backward") if wl.startswith(k)), "prefill")
         got = bench._traffic(wl)
         assert got == (entry["bytes_per_launch"] if entry["kernel_source_hash"] == bench.kernel_source_hash(kind)
                        else None)
+
+
+def test_backward_accounting():
+    w = bench.synth.WORKLOADS["backward_128k"]
+    assert w.kind == "backward" and w.T == 131072 and w.seed == 1007
+    # the kernel-source hash of the backward covers the prefill kernel its passes run on
+    assert "la_prefill_tc.cu" in bench.KERNEL_SOURCES["backward"]
+    assert "la_backward.cu" in bench.KERNEL_SOURCES["backward"]

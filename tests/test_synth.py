@@ -53,3 +53,4 @@ def test_workload_table():
     mixed = w["mixed_256"]
     ml = synth.mixed_lengths(mixed)
     assert (ml == 1).sum() == 256 and (ml == 4096).sum() == 2 and len(ml) == 258 and mixed.seed == 1006
+    assert w["backward_128k"].seed == 1007 and w["backward_8k"].seed == 1008 and w["backward_8k"].T == 8192
