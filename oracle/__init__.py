@@ -16,6 +16,8 @@ computes, and which passage of the pages it follows, is documented there:
   * ``quadratic`` -- restatement R1, (phi(Q) phi(K)^T (.) M) V;
   * ``chunked``   -- restatement R2, block-wise intra + inter form for any block size;
   * ``transform`` -- the output transform alone;
+  * ``forward_znorm_packed`` / ``prefill_znorm`` -- the normalised variant, y = phi(q)^T S /
+    (phi(q) . z) with z_t = z_{t-1} + phi(k_t) ("六十四：MiniMax-01", section 3);
   * ``backward_packed`` / ``backward`` -- the gradients of the forward (chain rule through
     the output transform, the recurrence and the feature map; pinned by finite differences
     of ``forward_packed``).
@@ -65,12 +67,15 @@ def _get():
         lib.oracle_quadratic.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
         lib.oracle_chunked.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
         lib.oracle_transform.argtypes = [vp, i64, i32, i32, i32, dbl, vp, vp, i32, vp]
+        lib.oracle_forward_znorm_packed.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, vp, i32, i32, dbl,
+                                                    vp, vp, vp, vp]
         lib.oracle_backward_packed.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, i32, i32, dbl,
                                                vp, vp, vp, vp, vp, vp]
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         for f in (lib.oracle_forward_packed, lib.oracle_prefill, lib.oracle_decode,
-                  lib.oracle_quadratic, lib.oracle_chunked, lib.oracle_transform, lib.oracle_backward_packed):
+                  lib.oracle_quadratic, lib.oracle_chunked, lib.oracle_transform, lib.oracle_backward_packed,
+                  lib.oracle_forward_znorm_packed):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -228,3 +233,36 @@ def backward(q, k, v, g, dout, state_in=None, phi=PHI_SILU, mode=MODE_RMSNORM_GA
                                           phi, mode, eps, norm_weight)
     return (dq.reshape(B, T, H, D), dk.reshape(B, T, H, D), dv.reshape(B, T, H, D),
             None if dg is None else dg.reshape(B, T, H * D), dst)
+
+
+def forward_znorm_packed(q, k, v, g, cu_seqlens, H, D, state_in=None, z_in=None, phi=PHI_SILU,
+                         mode=MODE_RMSNORM_GATE, eps=1e-6, norm_weight=None):
+    """Normalised variant over packed sequences: q, k, v [tokens, H, D]; g [tokens, H*D];
+    state_in [N, H, D, D], z_in [N, H, D] (fp32 or None).  Returns fp64 (out [tokens, H*D],
+    state [N, H, D, D], z [N, H, D])."""
+    q, k, v, g = _c(q), _c(k), _c(v), _c(g)
+    dt = _dtype_code(q)
+    cu = _c(cu_seqlens, np.int32)
+    N = cu.size - 1
+    tokens = int(cu[-1]) if N > 0 else 0
+    out = np.empty((tokens, H * D), dtype=np.float64)
+    st = np.empty((N, H, D, D), dtype=np.float64)
+    z = np.empty((N, H, D), dtype=np.float64)
+    rc = _get().oracle_forward_znorm_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), dt, _ptr(cu), N, H, D,
+                                            _ptr(_c(state_in, np.float32)), _ptr(_c(z_in, np.float32)), phi, mode,
+                                            eps, _ptr(_c(norm_weight, np.float32)), _ptr(out), _ptr(st), _ptr(z))
+    if rc != 0:
+        raise ValueError("oracle_forward_znorm_packed rejected its arguments")
+    return out, st, z
+
+
+def prefill_znorm(q, k, v, g=None, state_in=None, z_in=None, phi=PHI_SILU, mode=MODE_RMSNORM_GATE, eps=1e-6,
+                  norm_weight=None):
+    """Fixed-length batch of the normalised variant: q, k, v [B, T, H, D]; g [B, T, H*D]."""
+    B, T, H, D = q.shape
+    cu = np.arange(B + 1, dtype=np.int32) * T
+    out, st, z = forward_znorm_packed(np.reshape(q, (B * T, H, D)), np.reshape(k, (B * T, H, D)),
+                                      np.reshape(v, (B * T, H, D)),
+                                      None if g is None else np.reshape(g, (B * T, H * D)), cu, H, D, state_in,
+                                      z_in, phi, mode, eps, norm_weight)
+    return out.reshape(B, T, H * D), st, z

@@ -7,7 +7,9 @@
 // Sources (web pages; cited by title and section):
 //   [Tut64]  "六十四：MiniMax-01" (LLM tutorial, lesson 64), section 3 "Lightning Attention 的定位":
 //            linear attention as a running state, S_t = S_{t-1} + phi(k_t) v_t^T, and the
-//            output read from the state, phi(q_t)^T S_t (sum over i <= t: causal, inclusive).
+//            output read from the state, phi(q_t)^T S_t (sum over i <= t: causal, inclusive);
+//            in its normalised form also z_t = z_{t-1} + phi(k_t) and the division by
+//            phi(q_t)^T z_t.
 //   [Arch]   "MiniMax-Text-01 405B MoE模型架构与训练策略解析", section 2.1 "Lightning Attention-2":
 //            Q, K, V = SiLU(X);  Y = Q * (K^T * V);  output = RMSNorm(Y) * sigmoid(X).
 //   [Ops]    "MiniMax-01技术报告解读（二）计算优化", section 3: lightning_attention_chunk_size 256 and
@@ -273,6 +275,39 @@ void recur_head_backward(const void* q, const void* k, const void* v, int dtype,
   for (size_t i = 0; i < F.size(); ++i) dS0[i] = F[i];
 }
 
+// ---------------------------------------------------------------------------------------
+// Normalised variant ([Tut64] section 3, the linear-attention form before the deployment
+// drops the denominator): alongside S the recurrence carries z_t = z_{t-1} + phi(k_t), and
+//   y_t = phi(q_t)^T S_t / (phi(q_t) . z_t)
+// (the denominator is the normaliser that stands in for softmax's row sum).  The output
+// transform is then applied to y as in the plain form.  One head over rows [row0, row0+n);
+// S (D x D) and z (D) enter as the initial state and leave as the final one.
+void recur_head_znorm(const void* q, const void* k, const void* v, int dtype, int64_t row0, int64_t n, int H,
+                      int D, int h, int phi, double* S, double* z, double* y) {
+  std::vector<double> fq(D), fk(D), vv(D), acc(D);
+  for (int64_t t = 0; t < n; ++t) {
+    const int64_t base = ((row0 + t) * H + h) * static_cast<int64_t>(D);
+    for (int i = 0; i < D; ++i) {
+      fq[i] = feature(widen(q, dtype, base + i), phi);
+      fk[i] = feature(widen(k, dtype, base + i), phi);
+      vv[i] = widen(v, dtype, base + i);
+      acc[i] = 0.0;
+    }
+    double den = 0.0;
+    for (int i = 0; i < D; ++i) {
+      double* Si = S + static_cast<int64_t>(i) * D;
+      z[i] += fk[i];
+      den += fq[i] * z[i];
+      for (int j = 0; j < D; ++j) {
+        Si[j] += fk[i] * vv[j];
+        acc[j] += fq[i] * Si[j];
+      }
+    }
+    double* yt = y + (t * H + h) * static_cast<int64_t>(D);
+    for (int j = 0; j < D; ++j) yt[j] = acc[j] / den;
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -454,6 +489,40 @@ int oracle_backward_packed(const void* q, const void* k, const void* v, const vo
                           dy.data(), dq, dk, dv, dS0.data() + static_cast<size_t>(h) * D * D);
     if (dstate)
       for (int64_t i = 0; i < nst; ++i) dstate[s * nst + i] = dS0[i];
+  }
+  return 0;
+}
+
+// Packed-sequence forward of the normalised variant.  As oracle_forward_packed, plus the
+// normaliser state: z_in [N, H, D] (zeros if null) and z_out [N, H, D] (may be null).
+// out receives the transformed fp64 result [tokens, H*D].
+int oracle_forward_znorm_packed(const void* q, const void* k, const void* v, const void* g, int dtype,
+                                const int32_t* cu, int N, int H, int D, const float* state_in, const float* z_in,
+                                int phi, int mode, double eps, const float* w, double* out, double* state_out,
+                                double* z_out) {
+  if (N < 0 || H <= 0 || D <= 0 || !out) return 1;
+  if (mode == MODE_RMSNORM_GATE && !g) return 1;
+  const int HD = H * D;
+  const int64_t nst = static_cast<int64_t>(H) * D * D, nz = static_cast<int64_t>(H) * D;
+  for (int s = 0; s < N; ++s) {
+    const int64_t row0 = cu[s], L = static_cast<int64_t>(cu[s + 1]) - cu[s];
+    if (L < 0) return 1;
+    std::vector<double> S(nst, 0.0), z(nz, 0.0), y(static_cast<size_t>(L) * HD);
+    if (state_in)
+      for (int64_t i = 0; i < nst; ++i) S[i] = static_cast<double>(state_in[s * nst + i]);
+    if (z_in)
+      for (int64_t i = 0; i < nz; ++i) z[i] = static_cast<double>(z_in[s * nz + i]);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h)
+      recur_head_znorm(q, k, v, dtype, row0, L, H, D, h, phi, S.data() + static_cast<size_t>(h) * D * D,
+                       z.data() + static_cast<size_t>(h) * D, y.data());
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < L; ++t)
+      transform_token(y.data() + t * HD, HD, mode, eps, w, g, dtype, row0 + t, out + (row0 + t) * HD);
+    if (state_out)
+      for (int64_t i = 0; i < nst; ++i) state_out[s * nst + i] = S[i];
+    if (z_out)
+      for (int64_t i = 0; i < nz; ++i) z_out[s * nz + i] = z[i];
   }
   return 0;
 }
