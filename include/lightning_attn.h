@@ -76,7 +76,9 @@ typedef enum {
   LA_OP_DECODE = 2,
   LA_OP_MIXED = 3,
   LA_OP_BACKWARD = 4,
-  LA_OP_BACKWARD_VARLEN = 5
+  LA_OP_BACKWARD_VARLEN = 5,
+  LA_OP_PREFILL_ZNORM = 6,
+  LA_OP_PREFILL_ZNORM_VARLEN = 7
 } la_op;
 
 /*
@@ -230,6 +232,49 @@ LA_API la_status lightning_attn_state_prefix(const float* gathered, int world, i
                                              float* out, int H, int D, la_stream_t stream);
 
 /*
+ * Normalised variant of lightning_attn_prefill ("六十四：MiniMax-01" section 3, the linear-
+ * attention form with its normaliser): besides S each sequence carries z, the running sum
+ * of phi(k), and the raw output is divided by phi(q) . z before the output transform:
+ *   S_t = S_{t-1} + phi(k_t) v_t^T,  z_t = z_{t-1} + phi(k_t),
+ *   y_t = phi(q_t)^T S_t / (phi(q_t) . z_t),  out = transform(y) as lightning_attn_prefill.
+ * The denominator is not guarded: with phi = SiLU (which takes negative values) it can be
+ * zero or negative, and the result then is whatever the division gives.
+ *   z_in    fp32 [B, H, D] initial normaliser per sequence, or NULL (zeros).
+ *   z_out   fp32 [B, H, D] final normaliser, or NULL.  May equal z_in.
+ *   workspace  >= lightning_attn_workspace_size(LA_OP_PREFILL_ZNORM, B, T, 0, ...) bytes.
+ * Other arguments (state_in / state_out: the same S) as lightning_attn_prefill.
+ */
+LA_API la_status lightning_attn_prefill_znorm(const void* q, const void* k, const void* v, const void* g, void* out,
+                                              const float* state_in, const float* z_in, float* state_out,
+                                              float* z_out, int B, int T, int H, int D, int block_size,
+                                              la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
+                                              const float* norm_weight, void* workspace, size_t workspace_bytes,
+                                              la_stream_t stream);
+
+/*
+ * The normalised variant over N packed sequences (cu_seqlens as lightning_attn_prefill_varlen;
+ * z_in / z_out fp32 [N, H, D] or NULL).  Workspace: LA_OP_PREFILL_ZNORM_VARLEN.
+ */
+LA_API la_status lightning_attn_prefill_znorm_varlen(const void* q, const void* k, const void* v, const void* g,
+                                                     void* out, const float* state_in, const float* z_in,
+                                                     float* state_out, float* z_out, const int* cu_seqlens,
+                                                     int num_seqs, int max_seqlen, int total_tokens, int H, int D,
+                                                     int block_size, la_dtype dtype, la_feature_map phi,
+                                                     la_out_mode mode, float eps, const float* norm_weight,
+                                                     void* workspace, size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * One decode step of the normalised variant: as lightning_attn_decode_step, and z (fp32
+ * [B, H, D], required, updated in place) becomes z + phi(k); the raw output is divided by
+ * phi(q) . z before the output transform.  Workspace: LA_OP_DECODE.
+ */
+LA_API la_status lightning_attn_decode_step_znorm(const void* q, const void* k, const void* v, const void* g,
+                                                  void* out, float* state, float* z, int B, int H, int D,
+                                                  la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
+                                                  const float* norm_weight, void* workspace, size_t workspace_bytes,
+                                                  la_stream_t stream);
+
+/*
  * Backward pass of lightning_attn_prefill: the gradients of a loss with respect to q, k, v,
  * the gate and the initial state, given the gradient `dout` of its output.  The pages give
  * no gradient formulas ("MiniMax-Text-01 405B MoE模型架构与训练策略解析" section 2.1 names the
@@ -285,6 +330,8 @@ LA_API la_status lightning_attn_backward_varlen(const void* q, const void* k, co
  *                                one token (0 if none), total_tokens = all packed tokens.
  *   op == LA_OP_BACKWARD:        as LA_OP_PREFILL.
  *   op == LA_OP_BACKWARD_VARLEN: as LA_OP_PREFILL_VARLEN.
+ *   op == LA_OP_PREFILL_ZNORM:   as LA_OP_PREFILL.
+ *   op == LA_OP_PREFILL_ZNORM_VARLEN: as LA_OP_PREFILL_VARLEN.
  * The size depends on the kernel the call will select (which depends on the device), so
  * query it with the target device current.
  */

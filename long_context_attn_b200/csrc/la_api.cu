@@ -11,7 +11,8 @@ namespace la {
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, void* out, float* state,
                           int B, int H, int D, la_dtype dt, int phi_identity, int mode, float eps,
                           const float* w, void* workspace, cudaStream_t stream,
-                          const int* row_index = nullptr, const int* state_index = nullptr);
+                          const int* row_index = nullptr, const int* state_index = nullptr,
+                          float* z = nullptr);
 size_t decode_workspace_bytes(int B, int H, int D);
 cudaError_t launch_gather_single_token(const int* cu, const int* state_slot, int n, int* row_index,
                                        int* state_index, cudaStream_t stream);
@@ -29,6 +30,12 @@ cudaError_t launch_bwd_prep(const void* q, const void* k, const void* v, const v
 cudaError_t launch_bwd_post(const void* q, const void* k, void* dq, void* dk, void* dv, const int* cu, int nseq,
                             int T_fixed, int64_t tokens, int HD, int phi_identity, la_dtype dt, cudaStream_t stream);
 cudaError_t launch_transpose_states(const float* in, float* out, int64_t nmat, int D, cudaStream_t stream);
+int znorm_max_chunks(int max_len);
+cudaError_t launch_znorm_scan(const void* q, const void* k, const float* z_in, float* sums, float* den, float* z_out,
+                              const int* cu, int nseq, int T_fixed, int max_len, int64_t tokens, int H, int D,
+                              la_dtype dt, int phi_identity, cudaStream_t stream);
+cudaError_t launch_znorm_transform(void* io, const float* den, const void* g, const float* w, int64_t tokens, int H,
+                                   int D, int mode, float eps, la_dtype dt, cudaStream_t stream);
 }  // namespace la
 
 namespace {
@@ -217,6 +224,50 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
   return LA_OK;
 }
 
+// Normalised-variant workspace: [prefill part of the raw pass (error record first)]
+// [phi(k) chunk sums: nseq x H x chunks x D fp32] [denominators: tokens x H fp32].
+struct ZLayout {
+  size_t pre, sums, den, total;
+};
+ZLayout z_layout(int nseq, int max_len, int64_t tokens, int H, int D, int C, la_dtype dt) {
+  ZLayout z{};
+  z.pre = prefill_ws_bytes(choose_path(dt, H, D, C, LA_OUT_RAW), nseq, max_len, tokens, H, D, C, LA_OUT_RAW);
+  z.sums = up256(sizeof(float) * static_cast<size_t>(nseq) * H * la::znorm_max_chunks(max_len) * D);
+  z.den = up256(sizeof(float) * static_cast<size_t>(tokens) * H);
+  z.total = z.pre + z.sums + z.den;
+  return z;
+}
+
+// y = phi(q)^T S / (phi(q) . z): the raw prefill gives the numerators (and carries S), the
+// scan gives the denominators (and carries z), then y / den and the output transform.
+la_status common_prefill_znorm(const void* q, const void* k, const void* v, const void* g, void* out,
+                               const float* state_in, const float* z_in, float* state_out, float* z_out,
+                               const int* cu, int nseq, int T_fixed, int max_len, int64_t tokens, int H, int D,
+                               int C, la_dtype dt, la_feature_map phi, la_out_mode mode, float eps, const float* w,
+                               void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!valid_enums(dt, phi, mode) || !valid_head(H, D, mode, eps)) return LA_ERR_INVALID_ARG;
+  if (C < 1 || C > 1024 || nseq < 1 || nseq > 65535 || tokens < 0 || max_len < 0) return LA_ERR_INVALID_ARG;
+  if (tokens > 0 && mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g))) return LA_ERR_INVALID_ARG;
+  if ((z_in && !aligned16(z_in)) || (z_out && !aligned16(z_out))) return LA_ERR_INVALID_ARG;
+  if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;
+  const ZLayout L = z_layout(nseq, max_len, tokens, H, D, C, dt);
+  if (ws_bytes < L.total) return LA_ERR_INVALID_ARG;
+  char* base = static_cast<char*>(workspace);
+  float* sums = reinterpret_cast<float*>(base + L.pre);
+  float* den = reinterpret_cast<float*>(base + L.pre + L.sums);
+  la_status st = common_prefill(q, k, v, nullptr, out, state_in, state_out, cu, nseq, T_fixed, max_len, tokens, H,
+                                D, C, dt, phi, LA_OUT_RAW, eps, nullptr, workspace, L.pre, stream);
+  if (st != LA_OK) return st;
+  const int phi_id = (phi == LA_PHI_IDENTITY) ? 1 : 0;
+  if (la::launch_znorm_scan(q, k, z_in, sums, den, z_out, cu, nseq, T_fixed, max_len, tokens, H, D, dt, phi_id,
+                            stream) != cudaSuccess)
+    return LA_ERR_CUDA;
+  if (la::launch_znorm_transform(out, den, g, w, tokens, H, D, static_cast<int>(mode), eps, dt, stream) !=
+      cudaSuccess)
+    return LA_ERR_CUDA;
+  return LA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -259,6 +310,54 @@ la_status lightning_attn_backward_varlen(const void* q, const void* k, const voi
   return common_backward(q, k, v, g, dout, state_in, dq, dk, dv, dg, dstate_in, cu_seqlens, num_seqs, 0, max_seqlen,
                          total_tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight, workspace,
                          workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status lightning_attn_prefill_znorm(const void* q, const void* k, const void* v, const void* g, void* out,
+                                       const float* state_in, const float* z_in, float* state_out, float* z_out,
+                                       int B, int T, int H, int D, int block_size, la_dtype dtype,
+                                       la_feature_map phi, la_out_mode mode, float eps, const float* norm_weight,
+                                       void* workspace, size_t workspace_bytes, la_stream_t stream) {
+  if (B < 1 || T < 0) return LA_ERR_INVALID_ARG;
+  const int64_t tokens = static_cast<int64_t>(B) * T;
+  if (tokens > INT32_MAX) return LA_ERR_UNSUPPORTED;
+  return common_prefill_znorm(q, k, v, g, out, state_in, z_in, state_out, z_out, nullptr, B, T, T, tokens, H, D,
+                              block_size, dtype, phi, mode, eps, norm_weight, workspace, workspace_bytes,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status lightning_attn_prefill_znorm_varlen(const void* q, const void* k, const void* v, const void* g, void* out,
+                                              const float* state_in, const float* z_in, float* state_out,
+                                              float* z_out, const int* cu_seqlens, int num_seqs, int max_seqlen,
+                                              int total_tokens, int H, int D, int block_size, la_dtype dtype,
+                                              la_feature_map phi, la_out_mode mode, float eps,
+                                              const float* norm_weight, void* workspace, size_t workspace_bytes,
+                                              la_stream_t stream) {
+  if (num_seqs < 1 || !cu_seqlens || !aligned16(cu_seqlens) || total_tokens < 0 || max_seqlen < 0)
+    return LA_ERR_INVALID_ARG;
+  return common_prefill_znorm(q, k, v, g, out, state_in, z_in, state_out, z_out, cu_seqlens, num_seqs, 0,
+                              max_seqlen, total_tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight,
+                              workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status lightning_attn_decode_step_znorm(const void* q, const void* k, const void* v, const void* g, void* out,
+                                           float* state, float* z, int B, int H, int D, la_dtype dtype,
+                                           la_feature_map phi, la_out_mode mode, float eps, const float* norm_weight,
+                                           void* workspace, size_t workspace_bytes, la_stream_t stream) {
+  if (!z || !aligned16(z)) return LA_ERR_INVALID_ARG;
+  if (!valid_enums(dtype, phi, mode) || !valid_head(H, D, mode, eps) || B < 1) return LA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * H > INT32_MAX / 2) return LA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !out || !state) return LA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state))
+    return LA_ERR_INVALID_ARG;
+  if (mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g))) return LA_ERR_INVALID_ARG;
+  if (norm_weight && !aligned16(norm_weight)) return LA_ERR_INVALID_ARG;
+  if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;
+  if (workspace_bytes < la::decode_workspace_bytes(B, H, D)) return LA_ERR_INVALID_ARG;
+  cudaError_t e = la::launch_decode(q, k, v, g, out, state, B, H, D, dtype, phi == LA_PHI_IDENTITY ? 1 : 0,
+                                    static_cast<int>(mode), eps, norm_weight, workspace,
+                                    reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, z);
+  g_last_path = "decode";
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
 la_status lightning_attn_prefill_varlen(const void* q, const void* k, const void* v, const void* g, void* out,
@@ -374,6 +473,12 @@ size_t lightning_attn_workspace_size(la_op op, int B_or_N, int T_or_max, int tot
   if (op == LA_OP_PREFILL_VARLEN) {
     if (total_tokens < 0) return 0;
     return prefill_ws_bytes(path, B_or_N, T_or_max, total_tokens, H, D, block_size, mode);
+  }
+  if (op == LA_OP_PREFILL_ZNORM)
+    return z_layout(B_or_N, T_or_max, static_cast<int64_t>(B_or_N) * T_or_max, H, D, block_size, dtype).total;
+  if (op == LA_OP_PREFILL_ZNORM_VARLEN) {
+    if (total_tokens < 0) return 0;
+    return z_layout(B_or_N, T_or_max, total_tokens, H, D, block_size, dtype).total;
   }
   if (op == LA_OP_BACKWARD)
     return bwd_layout(B_or_N, T_or_max, static_cast<int64_t>(B_or_N) * T_or_max, H, D, block_size, dtype).total;

@@ -23,6 +23,7 @@ struct DecodeWs {
   float* part;     // [B, H] per-head sums of squares
   const int* row_index;    // optional [B]: token row of item b in q, k, v, g, out (else b)
   const int* state_index;  // optional [B]: state slot of item b (else b)
+  float* z;                // optional [slots, H, D]: normaliser of the normalised variant (in place)
 };
 
 template <typename T, int D>
@@ -90,6 +91,25 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     for (int r = 0; r < kRowsPerPass; ++r) y += s_red[r][tid];
   }
   const int HD = H * D;
+  if (ws.z) {
+    // Normalised variant ("六十四：MiniMax-01", section 3): z <- z + phi(k), y <- y / (phi(q) . z).
+    float zp = 0.f;
+    if (tid < D) {
+      float* zr = ws.z + (slot * H + h) * D;
+      const float zn = zr[tid] + s_fk[tid];
+      zr[tid] = zn;
+      zp = s_fq[tid] * zn;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) zp += __shfl_xor_sync(0xffffffffu, zp, o);
+    if ((tid & 31) == 0) s_ss[tid >> 5] = zp;
+    __syncthreads();
+    float den = 0.f;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) den += s_ss[w];
+    __syncthreads();   // s_ss is reused for the sum of squares below
+    y /= den;
+  }
   if (mode == LA_OUT_RAW) {
     if (tid < D) store_elem<T>(out, trow * HD + h * D + tid, y);
     return;
@@ -140,7 +160,7 @@ size_t decode_workspace_bytes(int B, int H, int D) {
 }
 
 static DecodeWs carve_decode_ws(void* workspace, int B, int H, int D, const int* row_index,
-                                const int* state_index) {
+                                const int* state_index, float* z) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   char* p = static_cast<char*>(workspace) + 256;
   DecodeWs ws;
@@ -151,6 +171,7 @@ static DecodeWs carve_decode_ws(void* workspace, int B, int H, int D, const int*
   ws.part = reinterpret_cast<float*>(p);
   ws.row_index = row_index;
   ws.state_index = state_index;
+  ws.z = z;
   return ws;
 }
 
@@ -158,8 +179,8 @@ template <typename T, int D>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* g, void* out,
                                    float* state, int B, int H, int phi_identity, int mode, float eps,
                                    const float* w, void* workspace, const int* row_index,
-                                   const int* state_index, cudaStream_t stream) {
-  DecodeWs ws = carve_decode_ws(workspace, B, H, D, row_index, state_index);
+                                   const int* state_index, float* z, cudaStream_t stream) {
+  DecodeWs ws = carve_decode_ws(workspace, B, H, D, row_index, state_index, z);
   decode_step_kernel<T, D><<<B * H, 256, 0, stream>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
       static_cast<const T*>(g), static_cast<T*>(out), state, B, H, phi_identity, mode, eps, w, ws);
@@ -169,19 +190,19 @@ static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, void* out, float* state,
                           int B, int H, int D, la_dtype dt, int phi_identity, int mode, float eps,
                           const float* w, void* workspace, cudaStream_t stream, const int* row_index,
-                          const int* state_index) {
+                          const int* state_index, float* z) {
   if (dt == LA_BF16) {
     if (D == 128)
       return launch_decode_t<uint16_t, 128>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace,
-                                            row_index, state_index, stream);
+                                            row_index, state_index, z, stream);
     return launch_decode_t<uint16_t, 64>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace,
-                                         row_index, state_index, stream);
+                                         row_index, state_index, z, stream);
   }
   if (D == 128)
     return launch_decode_t<float, 128>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace,
-                                       row_index, state_index, stream);
+                                       row_index, state_index, z, stream);
   return launch_decode_t<float, 64>(q, k, v, g, out, state, B, H, phi_identity, mode, eps, w, workspace,
-                                    row_index, state_index, stream);
+                                    row_index, state_index, z, stream);
 }
 
 // Mixed step: the one-token sequences of cu_seqlens (in sequence order) become the items

@@ -30,7 +30,8 @@ namespace la {
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, void* out, float* state,
                           int B, int H, int D, la_dtype dt, int phi_identity, int mode, float eps,
                           const float* w, void* workspace, cudaStream_t stream,
-                          const int* row_index = nullptr, const int* state_index = nullptr);
+                          const int* row_index = nullptr, const int* state_index = nullptr,
+                          float* z = nullptr);
 size_t decode_workspace_bytes(int B, int H, int D);
 }  // namespace la
 

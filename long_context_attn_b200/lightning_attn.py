@@ -20,14 +20,18 @@ LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT, LA_E
 LA_F32, LA_BF16 = 0, 1
 LA_OUT_RAW, LA_OUT_RMSNORM, LA_OUT_RMSNORM_GATE = 0, 1, 2
 LA_PHI_SILU, LA_PHI_IDENTITY = 0, 1
-LA_OP_PREFILL, LA_OP_PREFILL_VARLEN, LA_OP_DECODE, LA_OP_MIXED, LA_OP_BACKWARD, LA_OP_BACKWARD_VARLEN = range(6)
+(LA_OP_PREFILL, LA_OP_PREFILL_VARLEN, LA_OP_DECODE, LA_OP_MIXED, LA_OP_BACKWARD, LA_OP_BACKWARD_VARLEN,
+ LA_OP_PREFILL_ZNORM, LA_OP_PREFILL_ZNORM_VARLEN) = range(8)
 
 # The symbols include/lightning_attn.h declares (checked by tests/test_abi.py).
 EXPORTED = (
     "lightning_attn_prefill",
     "lightning_attn_prefill_varlen",
+    "lightning_attn_prefill_znorm",
+    "lightning_attn_prefill_znorm_varlen",
     "lightning_attn_backward",
     "lightning_attn_backward_varlen",
+    "lightning_attn_decode_step_znorm",
     "lightning_attn_decode_step",
     "lightning_attn_decode_step_noalloc",
     "lightning_attn_mixed_step",
@@ -55,6 +59,9 @@ def _load():
                                            f32, vp, vp, sz, vp]
     lib.lightning_attn_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                   i32, i32, i32, f32, vp, vp, sz, vp]
+    lib.lightning_attn_prefill_znorm.argtypes = [vp] * 9 + [i32] * 8 + [f32, vp, vp, sz, vp]
+    lib.lightning_attn_prefill_znorm_varlen.argtypes = [vp] * 10 + [i32] * 9 + [f32, vp, vp, sz, vp]
+    lib.lightning_attn_decode_step_znorm.argtypes = [vp] * 7 + [i32] * 6 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_backward.argtypes = [vp] * 11 + [i32] * 8 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_backward_varlen.argtypes = [vp] * 12 + [i32] * 9 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp,
@@ -72,7 +79,8 @@ def _load():
     lib.lightning_attn_last_path.argtypes = []
     lib.lightning_attn_last_path.restype = ctypes.c_char_p
     for f in ("lightning_attn_prefill", "lightning_attn_prefill_varlen", "lightning_attn_backward",
-              "lightning_attn_backward_varlen", "lightning_attn_decode_step",
+              "lightning_attn_backward_varlen", "lightning_attn_prefill_znorm", "lightning_attn_prefill_znorm_varlen",
+              "lightning_attn_decode_step_znorm", "lightning_attn_decode_step",
               "lightning_attn_decode_step_noalloc", "lightning_attn_mixed_step", "lightning_attn_state_prefix",
               "lightning_attn_check"):
         getattr(lib, f).restype = i32
@@ -169,6 +177,57 @@ def lightning_attn_prefill_varlen(q, k, v, g, out, cu_seqlens, max_seqlen, state
                                             0 if workspace is None else workspace.numel(), _stream(stream))
     if st != LA_OK:
         raise LightningAttnError(st, "lightning_attn_prefill_varlen")
+
+
+def lightning_attn_prefill_znorm(q, k, v, g, out, state_in=None, z_in=None, state_out=None, z_out=None,
+                                 block_size=256, phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE, eps=1e-6,
+                                 norm_weight=None, workspace=None, stream=None):
+    """Normalised variant: q, k, v [B, T, H, D]; g, out [B, T, H*D]; S fp32 [B, H, D, D]; z fp32 [B, H, D]."""
+    B, T, H, D = q.shape
+    _check_contig(q, k, v, g, out)
+    st = _lib.lightning_attn_prefill_znorm(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(out),
+                                           _ptr(_f32_or_none(state_in)), _ptr(_f32_or_none(z_in)),
+                                           _ptr(_f32_or_none(state_out)), _ptr(_f32_or_none(z_out)), B, T, H, D,
+                                           block_size, _dtype(q), phi, mode, eps, _ptr(_f32_or_none(norm_weight)),
+                                           _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                           _stream(stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_prefill_znorm")
+
+
+def lightning_attn_prefill_znorm_varlen(q, k, v, g, out, cu_seqlens, max_seqlen, state_in=None, z_in=None,
+                                        state_out=None, z_out=None, block_size=256, phi=LA_PHI_SILU,
+                                        mode=LA_OUT_RMSNORM_GATE, eps=1e-6, norm_weight=None, workspace=None,
+                                        stream=None):
+    """Normalised variant over packed sequences: q, k, v [total, H, D]; g, out [total, H*D]."""
+    total, H, D = q.shape
+    _check_contig(q, k, v, g, out, cu_seqlens)
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    n = cu_seqlens.numel() - 1
+    st = _lib.lightning_attn_prefill_znorm_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(out),
+                                                  _ptr(_f32_or_none(state_in)), _ptr(_f32_or_none(z_in)),
+                                                  _ptr(_f32_or_none(state_out)), _ptr(_f32_or_none(z_out)),
+                                                  _ptr(cu_seqlens), n, int(max_seqlen), total, H, D, block_size,
+                                                  _dtype(q), phi, mode, eps, _ptr(_f32_or_none(norm_weight)),
+                                                  _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                                  _stream(stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_prefill_znorm_varlen")
+
+
+def lightning_attn_decode_step_znorm(q, k, v, g, out, state, z, phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE,
+                                     eps=1e-6, norm_weight=None, workspace=None, stream=None):
+    """Normalised-variant decode: q, k, v [B, H, D]; g, out [B, H*D]; state [B, H, D, D] and z [B, H, D]
+    fp32, both updated in place."""
+    B, H, D = q.shape
+    _check_contig(q, k, v, g, out, state, z)
+    st = _lib.lightning_attn_decode_step_znorm(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(out),
+                                               _ptr(_f32_or_none(state)), _ptr(_f32_or_none(z)), B, H, D, _dtype(q),
+                                               phi, mode, eps, _ptr(_f32_or_none(norm_weight)), _ptr(workspace),
+                                               0 if workspace is None else workspace.numel(), _stream(stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_decode_step_znorm")
 
 
 def lightning_attn_backward(q, k, v, g, dout, dq, dk, dv, dg=None, state_in=None, dstate_in=None, block_size=256,
