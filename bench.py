@@ -346,6 +346,47 @@ class VarlenCase:
                 "l2": "inputs larger than L2 (%.1f GB per step), no flush" % (self.alg_bytes / 1e9)}
 
 
+class ZnormCase(PrefillCase):
+    """The normalised variant over the 128K prefill's shapes (q, k shifted so phi(q) . z > 0)."""
+
+    def __init__(self, name, w, device, rank):
+        super().__init__(name, w, device, rank)
+        import torch
+        T, H, D = self.T, self.H, self.D
+        for host, dev in ((self.h_q, self.q), (self.h_k, self.k)):
+            a = synth.shifted(host.view(torch.int16).numpy().view(np.uint16), w.qk_shift)
+            host.copy_(torch.from_numpy(a.view(np.int16)).view(torch.bfloat16))
+            dev.view(-1).copy_(host.view(-1))
+        self.z = torch.empty((1, H, D), dtype=torch.float32, device=device)
+        self.h_z = torch.empty((1, H, D), dtype=torch.float32).pin_memory()
+        nbytes = self.la.lightning_attn_workspace_size(self.la.LA_OP_PREFILL_ZNORM, 1, T, 0, H, D, self.C,
+                                                       self.la.LA_BF16, self.la.LA_OUT_RMSNORM_GATE)
+        self.ws = self.la.new_workspace(nbytes, device)
+        self.alg_bytes += H * D * 4
+        self.d2h += H * D * 4
+        self.launches_per_step = 5      # raw prefill, phi(k) chunk sums, their prefix, denominators, transform
+
+    def step(self):
+        self.la.lightning_attn_prefill_znorm(self.q, self.k, self.v, self.g, self.out, None, None, self.state, self.z,
+                                             block_size=self.C, workspace=self.ws)
+
+    def e2e_step(self):
+        super().e2e_step()
+        self.h_z.copy_(self.z, non_blocking=True)
+
+    def oracle_sample(self, tokens):
+        import oracle
+        w = self.w
+        q, k, v, g = synth.prefill_inputs(w.seed, tokens, w.H, w.D, "bf16", w.qkv_scale, True)
+        q, k = synth.shifted(q, w.qk_shift), synth.shifted(k, w.qk_shift)
+        t0 = time.perf_counter()
+        oracle.prefill_znorm(q[None], k[None], v[None], g[None])
+        return time.perf_counter() - t0
+
+    def describe(self):
+        return dict(super().describe(), variant="normalised (z-denominator)", qk_shift=self.w.qk_shift)
+
+
 class BackwardCase:
     """The backward of one long prefill: gradients of q, k, v and the gate from dout."""
 
@@ -520,6 +561,8 @@ def _make_case(name, device, rank):
         return DecodeCase(name, w, device, rank)
     if w.kind == "backward":
         return BackwardCase(name, w, device, rank)
+    if w.kind == "znorm":
+        return ZnormCase(name, w, device, rank)
     raise SystemExit(f"workload {name} is not a bench workload")
 
 
@@ -625,7 +668,10 @@ def run_gpu(args):
                               "algorithmic_bytes_per_launch": case.alg_bytes},
                              **({"scope": "one backward call (7 kernels); algorithmic bytes = its inputs "
                                           "read and gradients written once"}
-                                if isinstance(case, BackwardCase) else {})),
+                                if isinstance(case, BackwardCase) else
+                                {"scope": "one normalised-variant call (5 kernels); algorithmic bytes as the "
+                                          "prefill's plus z"}
+                                if isinstance(case, ZnormCase) else {})),
             "tensor": {"algorithmic_tflops": case.alg_flops / (launch_ms / 1e3) / 1e12,
                        "issued_tflops": case.issued_flops / (launch_ms / 1e3) / 1e12,
                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -678,6 +724,12 @@ def _traffic(workload):
 
 def _cpu_baseline(case):
     import oracle
+    if isinstance(case, ZnormCase):
+        n = min(16384, case.T)
+        dt = case.oracle_sample(n)
+        return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                "sample": f"first {n} tokens of the {case.w.name} workload, all {case.H} heads, fp64 normalised "
+                          f"recurrence + norm + gate ({dt:.1f} s)"}
     if isinstance(case, PrefillCase):
         n = min(131072, case.T)
         dt = case.oracle_sample(n)
@@ -713,7 +765,16 @@ def run_reference(args):
         return
     import oracle
     w = synth.WORKLOADS[args.workload]
-    if w.kind == "backward":
+    if w.kind == "znorm":
+        n = 1024
+        q, k, v, g = synth.prefill_inputs(w.seed, n, w.H, w.D, w.dtype, w.qkv_scale, True)
+        q, k = synth.shifted(q, w.qk_shift), synth.shifted(k, w.qk_shift)
+
+        def step():
+            oracle.prefill_znorm(q[None], k[None], v[None], g[None])
+        unit_per_step = n
+        sample = f"first {n} tokens of {w.name} (all {w.H} heads) per step, fp64 normalised recurrence + norm + gate"
+    elif w.kind == "backward":
         n = 512
         q, k, v, g = synth.prefill_inputs(w.seed, n, w.H, w.D, w.dtype, w.qkv_scale, True)
         dout = synth.normal(w.seed, synth.STREAM_DOUT, (n, w.H * w.D), 1.0, w.dtype)
@@ -766,7 +827,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="prefill_128k",
                     choices=["prefill_8k", "prefill_128k", "varlen_16", "decode_256", "mixed_256", "backward_8k",
-                             "backward_128k"])
+                             "backward_128k", "znorm_128k"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     args = ap.parse_args()

@@ -242,7 +242,8 @@ LA_API la_status lightning_attn_state_prefix(const float* gathered, int world, i
  *   z_in    fp32 [B, H, D] initial normaliser per sequence, or NULL (zeros).
  *   z_out   fp32 [B, H, D] final normaliser, or NULL.  May equal z_in.
  *   workspace  >= lightning_attn_workspace_size(LA_OP_PREFILL_ZNORM, B, T, 0, ...) bytes.
- * Other arguments (state_in / state_out: the same S) as lightning_attn_prefill.
+ * Needs H*D <= 16384 in every output mode (LA_ERR_UNSUPPORTED otherwise).  Other arguments
+ * (state_in / state_out: the same S) as lightning_attn_prefill.
  */
 LA_API la_status lightning_attn_prefill_znorm(const void* q, const void* k, const void* v, const void* g, void* out,
                                               const float* state_in, const float* z_in, float* state_out,

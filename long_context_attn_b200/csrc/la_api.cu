@@ -247,6 +247,7 @@ la_status common_prefill_znorm(const void* q, const void* k, const void* v, cons
                                void* workspace, size_t ws_bytes, cudaStream_t stream) {
   if (!valid_enums(dt, phi, mode) || !valid_head(H, D, mode, eps)) return LA_ERR_INVALID_ARG;
   if (C < 1 || C > 1024 || nseq < 1 || nseq > 65535 || tokens < 0 || max_len < 0) return LA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(H) * D > la::kMaxNormWidth) return LA_ERR_UNSUPPORTED;   // per-token reciprocals
   if (tokens > 0 && mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g))) return LA_ERR_INVALID_ARG;
   if ((z_in && !aligned16(z_in)) || (z_out && !aligned16(z_out))) return LA_ERR_INVALID_ARG;
   if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;

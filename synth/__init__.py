@@ -115,7 +115,7 @@ def f32_to_bf16(a: np.ndarray) -> np.ndarray:
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str              # 'prefill' | 'varlen' | 'decode' | 'mixed' | 'backward'
+    kind: str              # 'prefill' | 'varlen' | 'decode' | 'mixed' | 'backward' | 'znorm'
     seed: int
     B: int                 # batch (prefill), number of sequences (varlen / decode)
     T: int                 # tokens per sequence (prefill); 0 otherwise
@@ -129,6 +129,7 @@ class Workload:
     len_hi: int = 0
     eps: float = 1e-6
     n_prefill: int = 0     # mixed: number of prefill chunks (of T tokens) among B decode sequences
+    qk_shift: float = 0.0  # added to q and k (before rounding) to keep phi(q) . z away from zero
 
 
 # The workloads of the Lightning Attention forward and its backward (seed 1000 + k).
@@ -148,7 +149,20 @@ WORKLOADS = {
     "backward_128k": Workload("backward_128k", "backward", 1007, 1, 131072, 64, 128, 256, "bf16", "rmsnorm_gate",
                               0.5),
     "backward_8k": Workload("backward_8k", "backward", 1008, 1, 8192, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5),
+    # The normalised variant at the 128K prefill's shapes; q and k shifted by +1 so the
+    # denominators phi(q) . z stay positive.
+    "znorm_128k": Workload("znorm_128k", "znorm", 1009, 1, 131072, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5,
+                           qk_shift=1.0),
 }
+
+
+def shifted(a: np.ndarray, shift: float) -> np.ndarray:
+    """a + shift rounded back to a's dtype (bf16 bits or fp32); a itself if shift is 0."""
+    if shift == 0.0:
+        return a
+    if a.dtype == np.uint16:
+        return f32_to_bf16(bf16_to_f32(a) + np.float32(shift))
+    return (a + np.float32(shift)).astype(np.float32)
 
 
 def mixed_lengths(w: Workload) -> np.ndarray:
