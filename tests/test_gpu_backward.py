@@ -108,3 +108,44 @@ def test_backward_rejects_bad_arguments(cuda_device):
         la.lightning_attn_backward(x, x, x, gx, gx, *d, dg=None, workspace=ws)
     with pytest.raises(la.LightningAttnError):       # workspace too small
         la.lightning_attn_backward(x, x, x, gx, gx, *d, dg=torch.empty_like(gx), workspace=ws[:1024])
+
+
+@pytest.mark.parametrize("C", [128, 256])
+@pytest.mark.parametrize("T", [256, 700])
+def test_backward_exact_integers(C, T, cuda_device):
+    """Raw output, identity features, sparse ternary q, k, v, dout and an integer S0: every
+    score, state entry and gradient is an integer of magnitude <= 256 (checked on the
+    host), exact in bf16 and fp32, so the GPU gradients must equal the oracle's bit for bit
+    (a wrong row of the reversal, a transposed state or a shifted mask shows as a mismatch)."""
+    import torch
+    la = _la()
+    H, D = 4, 128
+    q, k, v, dout = (synth.ternary(3501 + T, s, (T, H, D), 0.06, "bf16") for s in range(4))
+    s0 = np.round(synth.normal(3501, 9, (1, H, D, D), 1.0, "f32")).astype(np.float32)
+    f = lambda a: synth.bf16_to_f32(a).astype(np.float64)
+    Q, K, V, dY = f(q), f(k), f(v), f(dout)
+    # every intermediate the three passes hold: running sums of v k^T (forward) and of
+    # dy q^T, q dy^T (from the end), plus the forward state itself
+    for a, b, rev in ((V, K, False), (dY, Q, True), (Q, dY, True), (K, V, False)):
+        outer = np.einsum("thi,thj->thij", a, b)
+        run = np.cumsum(outer[::-1] if rev else outer, axis=0)
+        assert np.abs(run).max() + np.abs(s0).max() <= 256
+    shp = (1, T, H, D)
+    dq_, dk_, dv_ = (to_dev(a).reshape(shp) for a in (q, k, v))
+    ddo = to_dev(dout).reshape(1, T, H * D)
+    gq, gk, gv = (torch.full_like(dq_, float("nan")) for _ in range(3))
+    gs = torch.full((1, H, D, D), float("nan"), dtype=torch.float32, device="cuda")
+    ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD, 1, T, 0, H, D, C, la.LA_BF16,
+                                                           la.LA_OUT_RAW))
+    la.lightning_attn_backward(dq_, dk_, dv_, None, ddo, gq, gk, gv, state_in=to_dev(s0), dstate_in=gs,
+                               block_size=C, phi=la.LA_PHI_IDENTITY, mode=la.LA_OUT_RAW, workspace=ws)
+    assert la.lightning_attn_last_path() == "tcgen05"
+    la.lightning_attn_check(ws)
+    ref = oracle.backward(q.reshape(shp), k.reshape(shp), v.reshape(shp), None, dout.reshape(1, T, H * D),
+                          state_in=s0, phi=oracle.PHI_IDENTITY, mode=oracle.MODE_RAW)
+    for got, want, name in zip((gq, gk, gv, gs), (ref[0], ref[1], ref[2], ref[4]), ("dq", "dk", "dv", "dstate")):
+        assert np.abs(want).max() <= 256, name
+        g64 = synth.bf16_to_f32(to_host(got)).astype(np.float64) if got.dtype == torch.bfloat16 \
+            else to_host(got).astype(np.float64)
+        bad = np.argwhere(g64.reshape(want.shape) != want)
+        assert bad.size == 0, f"{name}: {len(bad)} mismatches, first at {bad[:3].tolist()}"
