@@ -387,6 +387,58 @@ class ZnormCase(PrefillCase):
         return dict(super().describe(), variant="normalised (z-denominator)", qk_shift=self.w.qk_shift)
 
 
+class ChunkStateCase:
+    """Step 1 of the sequence-parallel prefill: the state of one 128K sequence from k and v."""
+
+    def __init__(self, name, w, device, rank):
+        import torch
+        from long_context_attn_b200 import lightning_attn as la
+        self.la, self.w = la, w
+        T, H, D = w.T, w.H, w.D
+        self.T, self.H, self.D = T, H, D
+        t0 = time.time()
+        _, k, v, _ = synth.prefill_inputs(w.seed + 1000 * rank, T, H, D, "bf16", w.qkv_scale, False)
+        self.gen_s = time.time() - t0
+        self.h_k, self.h_v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (k, v))
+        del k, v
+        self.k = self.h_k.to(device).view(1, T, H, D)
+        self.v = self.h_v.to(device).view(1, T, H, D)
+        self.state = torch.empty((1, H, D, D), dtype=torch.float32, device=device)
+        self.h_state = torch.empty((1, H, D, D), dtype=torch.float32).pin_memory()
+        self.ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_CHUNK_STATE, 1, T, 0, H, D, 0,
+                                                                    la.LA_BF16, 0), device)
+        self.tokens = T
+        self.alg_bytes = T * 2 * H * D * 2 + H * D * D * 4     # k, v read once; the state written
+        self.alg_flops = self.issued_flops = T * H * 2 * D * D
+        self.launches_per_step = 2                             # the state kernel and the split sum
+        self.h2d = 2 * T * H * D * 2
+        self.d2h = H * D * D * 4
+
+    def step(self):
+        self.la.lightning_attn_chunk_state(self.k, self.v, self.state, workspace=self.ws)
+
+    def e2e_step(self):
+        self.k.view(-1).copy_(self.h_k.view(-1), non_blocking=True)
+        self.v.view(-1).copy_(self.h_v.view(-1), non_blocking=True)
+        self.step()
+        self.h_state.copy_(self.state, non_blocking=True)
+
+    def check(self):
+        self.la.lightning_attn_check(self.ws)
+
+    def oracle_sample(self, tokens):
+        import oracle
+        w = self.w
+        q, k, v, _ = synth.prefill_inputs(w.seed, tokens, w.H, w.D, "bf16", w.qkv_scale, False)
+        t0 = time.perf_counter()
+        oracle.prefill(k[None], k[None], v[None], None, mode=oracle.MODE_RAW, store=False)
+        return time.perf_counter() - t0
+
+    def describe(self):
+        return {"workload": self.w.name, "B": 1, "T": self.T, "H": self.H, "D": self.D, "output": "final state only",
+                "l2": "inputs larger than L2 (%.1f GB per step), no flush" % (self.alg_bytes / 1e9)}
+
+
 class BackwardCase:
     """The backward of one long prefill: gradients of q, k, v and the gate from dout."""
 
@@ -563,6 +615,8 @@ def _make_case(name, device, rank):
         return BackwardCase(name, w, device, rank)
     if w.kind == "znorm":
         return ZnormCase(name, w, device, rank)
+    if w.kind == "chunk_state":
+        return ChunkStateCase(name, w, device, rank)
     raise SystemExit(f"workload {name} is not a bench workload")
 
 
@@ -671,7 +725,10 @@ def run_gpu(args):
                                 if isinstance(case, BackwardCase) else
                                 {"scope": "one normalised-variant call (5 kernels); algorithmic bytes as the "
                                           "prefill's plus z"}
-                                if isinstance(case, ZnormCase) else {})),
+                                if isinstance(case, ZnormCase) else
+                                {"scope": "one chunk-state call (state kernel + split sum); algorithmic bytes = k, "
+                                          "v read once + the state"}
+                                if isinstance(case, ChunkStateCase) else {})),
             "tensor": {"algorithmic_tflops": case.alg_flops / (launch_ms / 1e3) / 1e12,
                        "issued_tflops": case.issued_flops / (launch_ms / 1e3) / 1e12,
                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -741,6 +798,12 @@ def _cpu_baseline(case):
         return {"value": case.total / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
                 "sample": f"the whole {case.w.name} step ({case.total} tokens, all {case.w.H} heads), fp64 "
                           f"({dt:.1f} s)"}
+    if isinstance(case, ChunkStateCase):
+        n = min(32768, case.T)
+        dt = case.oracle_sample(n)
+        return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                "sample": f"first {n} tokens of the {case.w.name} workload, all {case.H} heads, fp64 recurrence "
+                          f"(final state) ({dt:.1f} s)"}
     if isinstance(case, BackwardCase):
         n = min(16384, case.T)
         dt = case.oracle_sample(n)
@@ -765,7 +828,15 @@ def run_reference(args):
         return
     import oracle
     w = synth.WORKLOADS[args.workload]
-    if w.kind == "znorm":
+    if w.kind == "chunk_state":
+        n = 1024
+        _, k, v, _ = synth.prefill_inputs(w.seed, n, w.H, w.D, w.dtype, w.qkv_scale, False)
+
+        def step():
+            oracle.prefill(k[None], k[None], v[None], None, mode=oracle.MODE_RAW, store=False)
+        unit_per_step = n
+        sample = f"first {n} tokens of {w.name} (all {w.H} heads) per step, fp64 recurrence (final state)"
+    elif w.kind == "znorm":
         n = 1024
         q, k, v, g = synth.prefill_inputs(w.seed, n, w.H, w.D, w.dtype, w.qkv_scale, True)
         q, k = synth.shifted(q, w.qk_shift), synth.shifted(k, w.qk_shift)
@@ -827,7 +898,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="prefill_128k",
                     choices=["prefill_8k", "prefill_128k", "varlen_16", "decode_256", "mixed_256", "backward_8k",
-                             "backward_128k", "znorm_128k"])
+                             "backward_128k", "znorm_128k", "chunk_state_128k"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     args = ap.parse_args()

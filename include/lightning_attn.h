@@ -78,7 +78,8 @@ typedef enum {
   LA_OP_BACKWARD = 4,
   LA_OP_BACKWARD_VARLEN = 5,
   LA_OP_PREFILL_ZNORM = 6,
-  LA_OP_PREFILL_ZNORM_VARLEN = 7
+  LA_OP_PREFILL_ZNORM_VARLEN = 7,
+  LA_OP_CHUNK_STATE = 8
 } la_op;
 
 /*
@@ -323,6 +324,26 @@ LA_API la_status lightning_attn_backward_varlen(const void* q, const void* k, co
                                                 void* workspace, size_t workspace_bytes, la_stream_t stream);
 
 /*
+ * The state lightning_attn_prefill would end with, without computing its outputs:
+ *   state_out[b] = state_in[b] + sum_t phi(k_t) v_t^T      ("六十四：MiniMax-01" section 3:
+ * the state is a plain sum over the sequence).  Step 1 of the sequence-parallel prefill
+ * ("MiniMax-01系列大模型：超长上下文与多模态能力深度解析与部署指南" section 2.1.3, LASP+): each
+ * rank's chunk state before the exchange.  Reads only k and v.
+ *   k, v        [B, T, H, D] dtype, device.
+ *   state_in    fp32 [B, H, D, D] or NULL (zeros).  state_out fp32 [B, H, D, D]; may equal
+ *               state_in.
+ *   workspace   >= lightning_attn_workspace_size(LA_OP_CHUNK_STATE, B, T, 0, H, D, 0, dtype, 0)
+ *               bytes, 256-byte aligned; error record as for the prefill.
+ * bf16 with D = 128 on sm_100a runs a tensor-core kernel (phi(K)^T V accumulated in TMEM,
+ * split over the tokens, the splits added in a fixed order); elsewhere a raw-mode prefill
+ * runs with its outputs written to the workspace.  The result equals the prefill's final
+ * state up to rounding order.
+ */
+LA_API la_status lightning_attn_chunk_state(const void* k, const void* v, const float* state_in, float* state_out,
+                                            int B, int T, int H, int D, la_dtype dtype, la_feature_map phi,
+                                            void* workspace, size_t workspace_bytes, la_stream_t stream);
+
+/*
  * Workspace bytes needed by one call (0 on invalid arguments).
  *   op == LA_OP_PREFILL:         B_or_N = B, T_or_max = T, total_tokens ignored.
  *   op == LA_OP_PREFILL_VARLEN:  B_or_N = N, T_or_max = max_seqlen, total_tokens.
@@ -333,6 +354,7 @@ LA_API la_status lightning_attn_backward_varlen(const void* q, const void* k, co
  *   op == LA_OP_BACKWARD_VARLEN: as LA_OP_PREFILL_VARLEN.
  *   op == LA_OP_PREFILL_ZNORM:   as LA_OP_PREFILL.
  *   op == LA_OP_PREFILL_ZNORM_VARLEN: as LA_OP_PREFILL_VARLEN.
+ *   op == LA_OP_CHUNK_STATE:     B_or_N = B, T_or_max = T (block_size and mode ignored).
  * The size depends on the kernel the call will select (which depends on the device), so
  * query it with the target device current.
  */

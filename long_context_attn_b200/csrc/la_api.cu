@@ -31,6 +31,10 @@ cudaError_t launch_bwd_post(const void* q, const void* k, void* dq, void* dk, vo
                             int T_fixed, int64_t tokens, int HD, int phi_identity, la_dtype dt, cudaStream_t stream);
 cudaError_t launch_transpose_states(const float* in, float* out, int64_t nmat, int D, cudaStream_t stream);
 int znorm_max_chunks(int max_len);
+int chunk_state_splits(int nseq, int H, int max_len, int num_sms);
+cudaError_t launch_chunk_state_tc(const void* k, const void* v, const float* state_in, float* state_out,
+                                  float* partial, const int* cu, int nseq, int T, int max_len, int64_t tokens, int H,
+                                  int phi_identity, int num_sms, ErrRec* err, cudaStream_t stream);
 cudaError_t launch_znorm_scan(const void* q, const void* k, const float* z_in, float* sums, float* den, float* z_out,
                               const int* cu, int nseq, int T_fixed, int max_len, int64_t tokens, int H, int D,
                               la_dtype dt, int phi_identity, cudaStream_t stream);
@@ -224,6 +228,21 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
   return LA_OK;
 }
 
+// Chunk state: the tensor-core kernel (bf16, D = 128, sm_100a) needs the error record and
+// one fp32 partial state per split; elsewhere a raw-mode prefill runs with its outputs
+// written to scratch (its prefill part, then the scratch outputs).
+bool chunk_state_tc(la_dtype dt, int D) { return dt == LA_BF16 && D == 128 && device_is_sm100(); }
+constexpr int kChunkFallbackC = 128;
+size_t chunk_state_ws_bytes(int nseq, int max_len, int64_t tokens, int H, int D, la_dtype dt) {
+  if (chunk_state_tc(dt, D)) {
+    const int sp = la::chunk_state_splits(nseq, H, max_len, current_sm_count());
+    return kErrBytes + up256(sizeof(float) * static_cast<size_t>(sp) * nseq * H * D * D);
+  }
+  const Path path = choose_path(dt, H, D, kChunkFallbackC, LA_OUT_RAW);
+  return prefill_ws_bytes(path, nseq, max_len, tokens, H, D, kChunkFallbackC, LA_OUT_RAW) +
+         up256(static_cast<size_t>(tokens) * H * D * (dt == LA_BF16 ? 2 : 4));
+}
+
 // Normalised-variant workspace: [prefill part of the raw pass (error record first)]
 // [phi(k) chunk sums: nseq x H x chunks x D fp32] [denominators: tokens x H fp32].
 struct ZLayout {
@@ -311,6 +330,35 @@ la_status lightning_attn_backward_varlen(const void* q, const void* k, const voi
   return common_backward(q, k, v, g, dout, state_in, dq, dk, dv, dg, dstate_in, cu_seqlens, num_seqs, 0, max_seqlen,
                          total_tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight, workspace,
                          workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status lightning_attn_chunk_state(const void* k, const void* v, const float* state_in, float* state_out, int B,
+                                     int T, int H, int D, la_dtype dtype, la_feature_map phi, void* workspace,
+                                     size_t workspace_bytes, la_stream_t stream) {
+  if (B < 1 || B > 65535 || T < 0 || H < 1 || H > 65535 || (D != 64 && D != 128)) return LA_ERR_INVALID_ARG;
+  if ((dtype != LA_F32 && dtype != LA_BF16) || (phi != LA_PHI_SILU && phi != LA_PHI_IDENTITY))
+    return LA_ERR_INVALID_ARG;
+  const int64_t tokens = static_cast<int64_t>(B) * T;
+  if (tokens > INT32_MAX) return LA_ERR_UNSUPPORTED;
+  if (!state_out || !aligned16(state_out) || (state_in && !aligned16(state_in))) return LA_ERR_INVALID_ARG;
+  if (tokens > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return LA_ERR_INVALID_ARG;
+  if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;
+  if (workspace_bytes < chunk_state_ws_bytes(B, T, tokens, H, D, dtype)) return LA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (chunk_state_tc(dtype, D)) {
+    la::ErrRec* err = static_cast<la::ErrRec*>(workspace);
+    float* partial = reinterpret_cast<float*>(static_cast<char*>(workspace) + kErrBytes);
+    const cudaError_t e = la::launch_chunk_state_tc(k, v, state_in, state_out, partial, nullptr, B, T, T, tokens, H,
+                                                    phi == LA_PHI_IDENTITY ? 1 : 0, current_sm_count(), err, st);
+    g_last_path = "tcgen05-state";
+    return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+  }
+  // Elsewhere: the raw prefill of (k, k, v) from state_in; its outputs go to scratch.
+  const Path path = choose_path(dtype, H, D, kChunkFallbackC, LA_OUT_RAW);
+  const size_t pre = prefill_ws_bytes(path, B, T, tokens, H, D, kChunkFallbackC, LA_OUT_RAW);
+  void* scratch = static_cast<char*>(workspace) + pre;
+  return common_prefill(k, k, v, nullptr, scratch, state_in, state_out, nullptr, B, T, T, tokens, H, D,
+                        kChunkFallbackC, dtype, phi, LA_OUT_RAW, 1e-6f, nullptr, workspace, pre, st);
 }
 
 la_status lightning_attn_prefill_znorm(const void* q, const void* k, const void* v, const void* g, void* out,
@@ -466,6 +514,8 @@ size_t lightning_attn_workspace_size(la_op op, int B_or_N, int T_or_max, int tot
     if (total_tokens < 0 || block_size < 1 || block_size > 1024) return 0;
     return mixed_layout(B_or_N, T_or_max, total_tokens, H, D, block_size, mode).total;
   }
+  if (op == LA_OP_CHUNK_STATE)   // no block size: the state does not depend on it
+    return chunk_state_ws_bytes(B_or_N, T_or_max, static_cast<int64_t>(B_or_N) * T_or_max, H, D, dtype);
   if (block_size < 1 || block_size > 1024) return 0;
   const Path path = choose_path(dtype, H, D, block_size, mode);
   if (op == LA_OP_PREFILL)

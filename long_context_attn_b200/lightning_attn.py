@@ -21,7 +21,7 @@ LA_F32, LA_BF16 = 0, 1
 LA_OUT_RAW, LA_OUT_RMSNORM, LA_OUT_RMSNORM_GATE = 0, 1, 2
 LA_PHI_SILU, LA_PHI_IDENTITY = 0, 1
 (LA_OP_PREFILL, LA_OP_PREFILL_VARLEN, LA_OP_DECODE, LA_OP_MIXED, LA_OP_BACKWARD, LA_OP_BACKWARD_VARLEN,
- LA_OP_PREFILL_ZNORM, LA_OP_PREFILL_ZNORM_VARLEN) = range(8)
+ LA_OP_PREFILL_ZNORM, LA_OP_PREFILL_ZNORM_VARLEN, LA_OP_CHUNK_STATE) = range(9)
 
 # The symbols include/lightning_attn.h declares (checked by tests/test_abi.py).
 EXPORTED = (
@@ -36,6 +36,7 @@ EXPORTED = (
     "lightning_attn_decode_step_noalloc",
     "lightning_attn_mixed_step",
     "lightning_attn_state_prefix",
+    "lightning_attn_chunk_state",
     "lightning_attn_workspace_size",
     "lightning_attn_check",
     "lightning_attn_status_string",
@@ -71,6 +72,7 @@ def _load():
     lib.lightning_attn_mixed_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                               f32, vp, vp, sz, vp, vp]
     lib.lightning_attn_state_prefix.argtypes = [vp, i32, i32, vp, vp, i32, i32, vp]
+    lib.lightning_attn_chunk_state.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, sz, vp]
     lib.lightning_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
     lib.lightning_attn_workspace_size.restype = sz
     lib.lightning_attn_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint * 4)]
@@ -81,7 +83,7 @@ def _load():
     for f in ("lightning_attn_prefill", "lightning_attn_prefill_varlen", "lightning_attn_backward",
               "lightning_attn_backward_varlen", "lightning_attn_prefill_znorm", "lightning_attn_prefill_znorm_varlen",
               "lightning_attn_decode_step_znorm", "lightning_attn_decode_step",
-              "lightning_attn_decode_step_noalloc", "lightning_attn_mixed_step", "lightning_attn_state_prefix",
+              "lightning_attn_decode_step_noalloc", "lightning_attn_mixed_step", "lightning_attn_state_prefix", "lightning_attn_chunk_state",
               "lightning_attn_check"):
         getattr(lib, f).restype = i32
     return lib
@@ -315,6 +317,17 @@ def lightning_attn_mixed_step(q, k, v, g, out, cu_seqlens, cu_seqlens_host, stat
                                         _stream(decode_stream))
     if st != LA_OK:
         raise LightningAttnError(st, "lightning_attn_mixed_step")
+
+
+def lightning_attn_chunk_state(k, v, state_out, state_in=None, phi=LA_PHI_SILU, workspace=None, stream=None):
+    """state_out = state_in + sum_t phi(k_t) v_t^T: k, v [B, T, H, D]; states fp32 [B, H, D, D]."""
+    B, T, H, D = k.shape
+    _check_contig(k, v, state_out, state_in)
+    st = _lib.lightning_attn_chunk_state(_ptr(k), _ptr(v), _ptr(_f32_or_none(state_in)),
+                                         _ptr(_f32_or_none(state_out)), B, T, H, D, _dtype(k), phi, _ptr(workspace),
+                                         0 if workspace is None else workspace.numel(), _stream(stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_chunk_state")
 
 
 def lightning_attn_state_prefix(gathered, rank, out, state0=None, stream=None):

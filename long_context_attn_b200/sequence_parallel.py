@@ -6,8 +6,8 @@ rests on is the state recurrence of "六十四：MiniMax-01" section 3: S_t = S0
 i <= t of phi(k_i) v_i^T is a plain sum, so rank r, holding the contiguous chunk r of the
 sequence, needs only the sum of the earlier chunks' states:
 
-  1. chunk_state: the state this chunk reaches from a zero state (a raw-mode prefill of the
-     chunk; its outputs go to the output buffer, which step 3 overwrites);
+  1. chunk_state: the state this chunk reaches from a zero state (lightning_attn_chunk_state:
+     phi(K)^T V accumulated on the tensor cores from k and v alone, no outputs);
   2. one all-gather of the [H, D, D] fp32 chunk states (NCCL over NVLink in a job);
   3. finish_chunk: the prefix state0 + sum_{j < r} state_j (lightning_attn_state_prefix, in
      rank order), then the chunk's prefill from that prefix with the requested output mode
@@ -24,20 +24,18 @@ from . import lightning_attn as la
 
 
 def workspace_for(T: int, H: int, D: int, block_size: int = 256, mode: int = la.LA_OUT_RMSNORM_GATE,
-                  device="cuda") -> torch.Tensor:
-    """One workspace that serves both prefill calls of a chunk of T tokens."""
-    n = max(la.lightning_attn_workspace_size(la.LA_OP_PREFILL, 1, T, 0, H, D, block_size, la.LA_BF16, m)
-            for m in (la.LA_OUT_RAW, mode))
+                  device="cuda", dtype: int = la.LA_BF16) -> torch.Tensor:
+    """One workspace that serves both steps of a chunk of T tokens (calls run one after another)."""
+    n = max(la.lightning_attn_workspace_size(la.LA_OP_PREFILL, 1, T, 0, H, D, block_size, dtype, mode),
+            la.lightning_attn_workspace_size(la.LA_OP_CHUNK_STATE, 1, T, 0, H, D, 0, dtype, 0))
     return la.new_workspace(n, device)
 
 
-def chunk_state(q, k, v, out, workspace, block_size: int = 256, phi: int = la.LA_PHI_SILU, stream=None):
-    """Step 1: the chunk's state from a zero state.  q, k, v [1, T, H, D]; `out` [1, T, H*D] is
-    used as scratch.  Returns fp32 [H, D, D]."""
-    _, T, H, D = q.shape
-    state = torch.empty((1, H, D, D), dtype=torch.float32, device=q.device)
-    la.lightning_attn_prefill(q, k, v, None, out, None, state, block_size=block_size, phi=phi, mode=la.LA_OUT_RAW,
-                              workspace=workspace, stream=stream)
+def chunk_state(k, v, workspace, phi: int = la.LA_PHI_SILU, stream=None):
+    """Step 1: the chunk's state from a zero state.  k, v [1, T, H, D].  Returns fp32 [H, D, D]."""
+    _, T, H, D = k.shape
+    state = torch.empty((1, H, D, D), dtype=torch.float32, device=k.device)
+    la.lightning_attn_chunk_state(k, v, state, phi=phi, workspace=workspace, stream=stream)
     return state[0]
 
 
@@ -76,8 +74,8 @@ def prefill_sequence_parallel(q, k, v, g, out, rank: int, all_gather=nccl_all_ga
     calls it with its own chunk, in the same order relative to other collectives."""
     _, T, H, D = q.shape
     if workspace is None:
-        workspace = workspace_for(T, H, D, block_size, mode, q.device)
-    local = chunk_state(q, k, v, out, workspace, block_size, phi, stream)
+        workspace = workspace_for(T, H, D, block_size, mode, q.device, la._dtype(q))
+    local = chunk_state(k, v, workspace, phi, stream)
     gathered = all_gather(local)
     finish_chunk(q, k, v, g, out, gathered, rank, workspace, state0, state_out, block_size, phi, mode, eps,
                  norm_weight, stream)

@@ -150,3 +150,18 @@ def test_backward_host_checks(lib):
     bwd_var = lib.lightning_attn_workspace_size(5, 2, 1000, 2000, 8, 128, 256, 1, 2)
     assert bwd >= fwd + 6 * 2000 * 8 * 128 * 2 + 2 * 8 * 128 * 128 * 4
     assert bwd_var == bwd
+
+
+def test_chunk_state_workspace_and_checks(lib):
+    """LA_OP_CHUNK_STATE needs no block size; bad arguments are rejected on the host."""
+    lib.lightning_attn_workspace_size.restype = ctypes.c_size_t
+    n = lib.lightning_attn_workspace_size(8, 1, 1000, 0, 8, 128, 0, 1, 0)
+    assert n > 256
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    f = lib.lightning_attn_chunk_state
+    f.argtypes = [vp, vp, vp, vp] + [i32] * 6 + [vp, ctypes.c_size_t, vp]
+    fake, ws = vp(0x1000), vp(0x100000)
+    assert f(fake, fake, None, None, 1, 64, 2, 128, 1, 0, ws, 1 << 30, None) == 1       # no state_out
+    assert f(fake, fake, None, fake, 1, 64, 2, 96, 1, 0, ws, 1 << 30, None) == 1        # D
+    assert f(fake, vp(0x1008), None, fake, 1, 64, 2, 128, 1, 0, ws, 1 << 30, None) == 1  # alignment
+    assert f(fake, fake, None, fake, 1, 64, 2, 128, 1, 0, ws, 16, None) == 1            # workspace too small

@@ -33,7 +33,7 @@ def test_emulated_ranks_match_one_prefill(C, chunks, mode, cuda_device):
         out = torch.empty((1, b - a, H * D), dtype=torch.bfloat16, device="cuda")
         parts.append((dq, dk, dv, dg, out, sp.workspace_for(b - a, H, D, C, m)))
     # step 1 on every "rank", step 2 as a stack, step 3 on every "rank"
-    local = [sp.chunk_state(dq, dk, dv, out, ws, C) for dq, dk, dv, dg, out, ws in parts]
+    local = [sp.chunk_state(dk, dv, ws) for dq, dk, dv, dg, out, ws in parts]
     gathered = torch.stack(local)
     final = torch.full((H, D, D), float("nan"), dtype=torch.float32, device="cuda")
     ds0 = to_dev(s0)

@@ -27,6 +27,10 @@ class _OracleBackend:
     """The three library calls sequence_parallel makes, on the CPU via the oracle."""
     LA_OUT_RAW, LA_OUT_RMSNORM_GATE, LA_PHI_SILU, LA_OP_PREFILL, LA_BF16 = 0, 2, 0, 0, 1
 
+    @staticmethod
+    def _dtype(t):
+        return 1
+
     def __init__(self):
         import oracle
         self.oracle = oracle
@@ -40,6 +44,13 @@ class _OracleBackend:
         out.copy_(torch.from_numpy(o))
         if state_out is not None:
             state_out.copy_(torch.from_numpy(st))
+
+    def lightning_attn_chunk_state(self, k, v, state_out, state_in=None, phi=0, workspace=None, stream=None):
+        import torch
+        q = k.numpy()   # the state does not depend on q
+        _, st, _ = self.oracle.prefill(q, k.numpy(), v.numpy(), None, state_in=None if state_in is None else
+                                       state_in.numpy(), phi=phi, mode=self.LA_OUT_RAW)
+        state_out.copy_(torch.from_numpy(st))
 
     def lightning_attn_state_prefix(self, gathered, rank, out, state0=None, stream=None):
         import torch
