@@ -149,3 +149,36 @@ def test_backward_exact_integers(C, T, cuda_device):
             else to_host(got).astype(np.float64)
         bad = np.argwhere(g64.reshape(want.shape) != want)
         assert bad.size == 0, f"{name}: {len(bad)} mismatches, first at {bad[:3].tolist()}"
+
+
+@pytest.mark.slow
+def test_backward_128k_full_size_samples(cuda_device):
+    """The backward at the bench's full size (T 131072, H 64, D 128, block 256) in raw mode,
+    where dy = dout needs no forward: dq of the first 4096 tokens depends only on them, and
+    dk, dv of the last 4096 tokens only on those (sums over t >= i), so both samples are
+    compared element by element with the oracle run on that prefix / suffix alone."""
+    import torch
+    la = _la()
+    w = synth.WORKLOADS["backward_128k"]
+    T, H, D, n = w.T, w.H, w.D, 4096
+    q, k, v, _ = synth.prefill_inputs(w.seed, T, H, D, "bf16", w.qkv_scale, False)
+    dout = synth.normal(w.seed, synth.STREAM_DOUT, (T, H * D), 1.0, "bf16")
+    shp = (1, T, H, D)
+    dq_, dk_, dv_ = (to_dev(a).reshape(shp) for a in (q, k, v))
+    ddo = to_dev(dout).reshape(1, T, H * D)
+    gq, gk, gv = (torch.empty_like(dq_) for _ in range(3))
+    ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD, 1, T, 0, H, D, w.block_size,
+                                                           la.LA_BF16, la.LA_OUT_RAW))
+    la.lightning_attn_backward(dq_, dk_, dv_, None, ddo, gq, gk, gv, block_size=w.block_size, mode=la.LA_OUT_RAW,
+                               workspace=ws)
+    assert la.lightning_attn_last_path() == "tcgen05"
+    la.lightning_attn_check(ws)
+    got_q = to_host(gq[0, :n])
+    got_k, got_v = to_host(gk[0, T - n:]), to_host(gv[0, T - n:])
+    del gq, gk, gv, dq_, dk_, dv_, ddo, ws
+    head = oracle.backward(q[None, :n], k[None, :n], v[None, :n], None, dout[None, :n], mode=oracle.MODE_RAW)
+    assert_close(got_q[None], head[0], "bf16", "dq (first 4096 tokens)")
+    tail = oracle.backward(q[None, T - n:], k[None, T - n:], v[None, T - n:], None, dout[None, T - n:],
+                           mode=oracle.MODE_RAW)
+    assert_close(got_k[None], tail[1], "bf16", "dk (last 4096 tokens)")
+    assert_close(got_v[None], tail[2], "bf16", "dv (last 4096 tokens)")

@@ -120,3 +120,31 @@ def test_decode_znorm(dtype, cuda_device):
     assert_close(to_host(out), ref, dtype)
     assert_close(to_host(dS), ref_S, dtype, "state")
     assert_close(to_host(dz), ref_z, "f32", "z")
+
+
+@pytest.mark.slow
+def test_znorm_128k_full_size_samples(cuda_device):
+    """The normalised variant at the bench's full size (znorm_128k): the outputs of the first
+    4096 tokens (causal: they depend on nothing later) against the oracle on that prefix, and
+    z_out against the fp64 sum of phi(k) over all 131072 tokens."""
+    import torch
+    la = _la()
+    w = synth.WORKLOADS["znorm_128k"]
+    T, H, D, n = w.T, w.H, w.D, 4096
+    q, k, v, g = synth.prefill_inputs(w.seed, T, H, D, "bf16", w.qkv_scale, True)
+    q, k = synth.shifted(q, w.qk_shift), synth.shifted(k, w.qk_shift)
+    out = torch.empty((1, T, H * D), dtype=torch.bfloat16, device="cuda")
+    zo = torch.empty((1, H, D), dtype=torch.float32, device="cuda")
+    ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_PREFILL_ZNORM, 1, T, 0, H, D, w.block_size,
+                                                           la.LA_BF16, la.LA_OUT_RMSNORM_GATE))
+    la.lightning_attn_prefill_znorm(*(to_dev(a).reshape(1, T, H, D) for a in (q, k, v)),
+                                    to_dev(g).reshape(1, T, H * D), out, z_out=zo, block_size=w.block_size,
+                                    workspace=ws)
+    la.lightning_attn_check(ws)
+    got = to_host(out[0, :n])
+    ref, _, _ = oracle.prefill_znorm(q[None, :n], k[None, :n], v[None, :n], g[None, :n])
+    assert_close(got[None], ref, "bf16")
+    kf = synth.bf16_to_f32(k).astype(np.float64)
+    z_ref = (kf / (1.0 + np.exp(-kf))).sum(axis=0)
+    # the scan's SiLU is the fast-intrinsic form (a few ulp) summed in fp32 over 131072 tokens
+    assert np.abs(to_host(zo)[0] - z_ref).max() <= 1e-4 * np.abs(z_ref).max()
