@@ -69,7 +69,7 @@ def _get():
         lib.oracle_transform.argtypes = [vp, i64, i32, i32, i32, dbl, vp, vp, i32, vp]
         lib.oracle_forward_znorm_packed.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, vp, i32, i32, dbl,
                                                     vp, vp, vp, vp]
-        lib.oracle_backward_packed.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, i32, i32, dbl,
+        lib.oracle_backward_packed.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, vp, i32, i32, dbl,
                                                vp, vp, vp, vp, vp, vp]
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -125,9 +125,10 @@ def forward_packed(q, k, v, g, cu_seqlens, H, D, state_in=None, phi=PHI_SILU, mo
     stats = np.zeros(8, dtype=np.float64) if (cand_out is not None or cand_state is not None) else None
     cand_out = _c(cand_out)
     cand_state = _c(cand_state, np.float32)
+    s_in, w = _c(state_in, np.float32), _c(norm_weight, np.float32)   # held until the call returns
     rc = _get().oracle_forward_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), dt, _ptr(cu), N, H, D,
-                                      _ptr(_c(state_in, np.float32)), phi, mode, eps,
-                                      _ptr(_c(norm_weight, np.float32)), _ptr(out), _ptr(st),
+                                      _ptr(s_in), phi, mode, eps,
+                                      _ptr(w), _ptr(out), _ptr(st),
                                       _ptr(cand_out), _ptr(cand_state), _ptr(stats))
     if rc != 0:
         raise ValueError("oracle_forward_packed rejected its arguments")
@@ -175,8 +176,9 @@ def chunked(q, k, v, C, phi=PHI_SILU, s0=None):
     T, H, D = q.shape
     y = np.empty((T, H, D), dtype=np.float64)
     st = np.empty((H, D, D), dtype=np.float64)
+    s0c = _c(s0, np.float64)   # held until the call returns
     if _get().oracle_chunked(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), T, H, D, C, phi,
-                             _ptr(_c(s0, np.float64)), _ptr(y), _ptr(st)) != 0:
+                             _ptr(s0c), _ptr(y), _ptr(st)) != 0:
         raise ValueError("oracle_chunked rejected its arguments")
     return y, st
 
@@ -193,14 +195,16 @@ def transform(y, mode, eps=1e-6, norm_weight=None, g=None):
     out = np.empty((tokens, H * D), dtype=np.float64)
     g = _c(g)
     dt = DT_F32 if g is None else _dtype_code(g)
-    _get().oracle_transform(_ptr(y), tokens, H, D, mode, eps, _ptr(_c(norm_weight, np.float32)), _ptr(g),
+    w = _c(norm_weight, np.float32)
+    _get().oracle_transform(_ptr(y), tokens, H, D, mode, eps, _ptr(w), _ptr(g),
                             dt, _ptr(out))
     return out
 
 
 def backward_packed(q, k, v, g, dout, cu_seqlens, H, D, state_in=None, phi=PHI_SILU, mode=MODE_RMSNORM_GATE,
-                    eps=1e-6, norm_weight=None):
-    """Gradients of forward_packed for the loss with output gradient dout [tokens, H*D].
+                    eps=1e-6, norm_weight=None, dstate_out=None):
+    """Gradients of forward_packed for the loss with output gradient dout [tokens, H*D] and
+    final-state gradient dstate_out [N, H, D, D] (fp32, or None for zero).
 
     q, k, v [tokens, H, D], g and dout [tokens, H*D] (bf16 bits or fp32, all one dtype).
     Returns fp64 (dq, dk, dv [tokens, H, D], dg [tokens, H*D] or None, dstate [N, H, D, D]).
@@ -213,24 +217,24 @@ def backward_packed(q, k, v, g, dout, cu_seqlens, H, D, state_in=None, phi=PHI_S
     dq, dk, dv = (np.zeros((tokens, H, D), dtype=np.float64) for _ in range(3))
     dg = np.zeros((tokens, H * D), dtype=np.float64) if mode == MODE_RMSNORM_GATE else None
     dst = np.zeros((N, H, D, D), dtype=np.float64)
+    s_in, ds_out, w = _c(state_in, np.float32), _c(dstate_out, np.float32), _c(norm_weight, np.float32)
     rc = _get().oracle_backward_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout), dt, _ptr(cu), N, H, D,
-                                       _ptr(_c(state_in, np.float32)), phi, mode, eps,
-                                       _ptr(_c(norm_weight, np.float32)), _ptr(dq), _ptr(dk), _ptr(dv),
-                                       _ptr(dg), _ptr(dst))
+                                       _ptr(s_in), _ptr(ds_out), phi, mode, eps, _ptr(w), _ptr(dq), _ptr(dk),
+                                       _ptr(dv), _ptr(dg), _ptr(dst))
     if rc != 0:
         raise ValueError("oracle_backward_packed rejected its arguments")
     return dq, dk, dv, dg, dst
 
 
 def backward(q, k, v, g, dout, state_in=None, phi=PHI_SILU, mode=MODE_RMSNORM_GATE, eps=1e-6,
-             norm_weight=None):
-    """Fixed-length batch: q, k, v [B, T, H, D]; g, dout [B, T, H*D]; state_in [B, H, D, D]."""
+             norm_weight=None, dstate_out=None):
+    """Fixed-length batch: q, k, v [B, T, H, D]; g, dout [B, T, H*D]; states [B, H, D, D]."""
     B, T, H, D = q.shape
     cu = np.arange(B + 1, dtype=np.int32) * T
     r = lambda a, s: None if a is None else np.reshape(a, s)
     dq, dk, dv, dg, dst = backward_packed(r(q, (B * T, H, D)), r(k, (B * T, H, D)), r(v, (B * T, H, D)),
                                           r(g, (B * T, H * D)), r(dout, (B * T, H * D)), cu, H, D, state_in,
-                                          phi, mode, eps, norm_weight)
+                                          phi, mode, eps, norm_weight, dstate_out)
     return (dq.reshape(B, T, H, D), dk.reshape(B, T, H, D), dv.reshape(B, T, H, D),
             None if dg is None else dg.reshape(B, T, H * D), dst)
 
@@ -248,9 +252,10 @@ def forward_znorm_packed(q, k, v, g, cu_seqlens, H, D, state_in=None, z_in=None,
     out = np.empty((tokens, H * D), dtype=np.float64)
     st = np.empty((N, H, D, D), dtype=np.float64)
     z = np.empty((N, H, D), dtype=np.float64)
+    s_in, zz, w = _c(state_in, np.float32), _c(z_in, np.float32), _c(norm_weight, np.float32)
     rc = _get().oracle_forward_znorm_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), dt, _ptr(cu), N, H, D,
-                                            _ptr(_c(state_in, np.float32)), _ptr(_c(z_in, np.float32)), phi, mode,
-                                            eps, _ptr(_c(norm_weight, np.float32)), _ptr(out), _ptr(st), _ptr(z))
+                                            _ptr(s_in), _ptr(zz), phi, mode, eps, _ptr(w), _ptr(out), _ptr(st),
+                                            _ptr(z))
     if rc != 0:
         raise ValueError("oracle_forward_znorm_packed rejected its arguments")
     return out, st, z

@@ -189,9 +189,10 @@ void write_stats(double* stats, const Cmp& o, const Cmp& s) {
 //     RAW:            dy = dO
 //     RMSNORM(_GATE): dy_c = r u_c - r^3 y_c (sum_c' u_c' y_c') / (H*D)
 //     gate:           dg_c = dO_c y_c r w_c s_c (1 - s_c)
-//   recurrence (per head; S_t = S0 + sum_{i<=t} phi(k_i) v_i^T, y_t = S_t^T phi(q_t)):
+//   recurrence (per head; S_t = S0 + sum_{i<=t} phi(k_i) v_i^T, y_t = S_t^T phi(q_t)), with
+//   dS_T the gradient reaching the final state (zero unless given):
 //     dphi(q_t) = S_t dy_t
-//     F_t = sum_{i>=t} phi(q_i) dy_i^T      (the same sum taken from the end)
+//     F_t = dS_T + sum_{i>=t} phi(q_i) dy_i^T      (the same sum taken from the end)
 //     dphi(k_t) = F_t v_t,   dv_t = F_t^T phi(k_t),   dS0 = F_0
 //   feature map: dq = dphi(q) * phi'(q), phi'(x) = sigmoid(x) (1 + x (1 - sigmoid(x))) for
 //   SiLU and 1 for the identity; likewise dk.
@@ -226,13 +227,14 @@ void transform_token_backward(const double* y, const void* dout, const void* g, 
   for (int c = 0; c < HD; ++c) dy[c] = r * u[c] - r * r * r * y[c] * dot / HD;
 }
 
-// Recurrence backward for one head over rows [row0, row0 + n).  S enters as S0 (D x D);
+// Recurrence backward for one head over rows [row0, row0 + n).  S enters as S0 (D x D) and
+// F as dST (D x D, the final state's gradient; null for zero);
 // dy is the fp64 [tokens, H, D] gradient of the raw output.  Writes dq, dk, dv at the
 // same packed positions and dS0 (D x D).  dy is indexed from the sequence's first row:
 // dy[(t * H + h) * D + j].
 void recur_head_backward(const void* q, const void* k, const void* v, int dtype, int64_t row0, int64_t n,
-                         int H, int D, int h, int phi, const double* S0, const double* dy, double* dq,
-                         double* dk, double* dv, double* dS0) {
+                         int H, int D, int h, int phi, const double* S0, const double* dST, const double* dy,
+                         double* dq, double* dk, double* dv, double* dS0) {
   std::vector<double> S(S0, S0 + static_cast<size_t>(D) * D);
   std::vector<double> fk(D), vv(D);
   // forward in time: dphi(q_t) = S_t dy_t, S_t including token t
@@ -250,8 +252,10 @@ void recur_head_backward(const void* q, const void* k, const void* v, int dtype,
       dq[base + i] = a * dfeature(widen(q, dtype, base + i), phi);
     }
   }
-  // backward in time: F_t = sum_{i >= t} phi(q_i) dy_i^T
+  // backward in time: F_t = dS_T + sum_{i >= t} phi(q_i) dy_i^T
   std::vector<double> F(static_cast<size_t>(D) * D, 0.0), fq(D);
+  if (dST)
+    for (size_t i = 0; i < F.size(); ++i) F[i] = dST[i];
   for (int64_t t = n - 1; t >= 0; --t) {
     const int64_t base = ((row0 + t) * H + h) * static_cast<int64_t>(D);
     for (int i = 0; i < D; ++i) {
@@ -454,14 +458,15 @@ int oracle_transform(const double* y, int64_t tokens, int H, int D, int mode, do
 }
 
 // Backward of oracle_forward_packed for the loss whose output gradient is dout [tokens, H*D]
-// (same dtype as q).  Recomputes the raw forward y, applies the transform backward per
-// token, then the recurrence backward per head.  Outputs fp64: dq, dk, dv [tokens, H, D],
-// dg [tokens, H*D] (gate mode; may be null otherwise), dstate [N, H, D, D] (the gradient
-// of each sequence's initial state; may be null).
+// (same dtype as q) and whose final-state gradient is dstate_out [N, H, D, D] fp32 (null for
+// zero).  Recomputes the raw forward y, applies the transform backward per token, then the
+// recurrence backward per head.  Outputs fp64: dq, dk, dv [tokens, H, D], dg [tokens, H*D]
+// (gate mode; may be null otherwise), dstate [N, H, D, D] (the gradient of each sequence's
+// initial state; may be null).
 int oracle_backward_packed(const void* q, const void* k, const void* v, const void* g, const void* dout,
-                           int dtype, const int32_t* cu, int N, int H, int D, const float* state_in, int phi,
-                           int mode, double eps, const float* w, double* dq, double* dk, double* dv,
-                           double* dg, double* dstate) {
+                           int dtype, const int32_t* cu, int N, int H, int D, const float* state_in,
+                           const float* dstate_out, int phi, int mode, double eps, const float* w, double* dq,
+                           double* dk, double* dv, double* dg, double* dstate) {
   if (N < 0 || H <= 0 || D <= 0 || !dout || !dq || !dk || !dv) return 1;
   if (mode == MODE_RMSNORM_GATE && (!g || !dg)) return 1;
   const int HD = H * D;
@@ -482,11 +487,16 @@ int oracle_backward_packed(const void* q, const void* k, const void* v, const vo
     for (int64_t t = 0; t < L; ++t)
       transform_token_backward(y.data() + t * HD, dout, g, dtype, row0 + t, HD, mode, eps, w,
                                dy.data() + t * HD, dg ? dg + (row0 + t) * HD : nullptr);
-    std::vector<double> dS0(nst);
+    std::vector<double> dS0(nst), dST;
+    if (dstate_out) {
+      dST.resize(nst);
+      for (int64_t i = 0; i < nst; ++i) dST[i] = static_cast<double>(dstate_out[s * nst + i]);
+    }
 #pragma omp parallel for schedule(dynamic, 1)
     for (int h = 0; h < H; ++h)
       recur_head_backward(q, k, v, dtype, row0, L, H, D, h, phi, S0.data() + static_cast<size_t>(h) * D * D,
-                          dy.data(), dq, dk, dv, dS0.data() + static_cast<size_t>(h) * D * D);
+                          dstate_out ? dST.data() + static_cast<size_t>(h) * D * D : nullptr, dy.data(), dq, dk,
+                          dv, dS0.data() + static_cast<size_t>(h) * D * D);
     if (dstate)
       for (int64_t i = 0; i < nst; ++i) dstate[s * nst + i] = dS0[i];
   }

@@ -105,3 +105,35 @@ def test_backward_matches_masked_matrix_form(phi):
         np.testing.assert_allclose(dk[:, h], (dA.T @ f(Q)) * df(K), rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(dv[:, h], A.T @ dY, rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(dst[0, h], f(Q).T @ dY, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_RAW, oracle.MODE_RMSNORM_GATE])
+def test_final_state_gradient_matches_finite_differences(mode):
+    """With a gradient dS_T reaching each sequence's final state, the loss is
+    sum(dout * o) + sum(dS_T * S_T); its finite differences pin the reverse sum's start."""
+    x, dout, w = _inputs(2171 + mode, mode)
+    dST = synth.normal(2171, 14, (len(CU) - 1, H, D, D), 0.5, "f32")
+    phi = oracle.PHI_SILU
+
+    def loss(xx):
+        out, st, _ = oracle.forward_packed(xx["q"], xx["k"], xx["v"], xx["g"], CU, H, D, state_in=xx["state_in"],
+                                           phi=phi, mode=mode, norm_weight=w)
+        return float(np.sum(out * dout.astype(np.float64)) + np.sum(st * dST.astype(np.float64)))
+
+    dq, dk, dv, dg, dst = oracle.backward_packed(x["q"], x["k"], x["v"], x["g"], dout, CU, H, D,
+                                                 state_in=x["state_in"], phi=phi, mode=mode, norm_weight=w,
+                                                 dstate_out=dST)
+    grads = {"q": dq, "k": dk, "v": dv, "state_in": dst}
+    rng = np.random.default_rng(2171)
+    eps = 1e-3
+    for name, grad in grads.items():
+        base = x[name]
+        delta = rng.standard_normal(base.shape)
+        plus, minus = dict(x), dict(x)
+        plus[name] = (base + eps * delta).astype(np.float32)
+        minus[name] = (base - eps * delta).astype(np.float32)
+        step = plus[name].astype(np.float64) - minus[name].astype(np.float64)
+        fd = loss(plus) - loss(minus)
+        pred = float(np.sum(grad.reshape(step.shape) * step))
+        scale = float(np.sum(np.abs(grad.reshape(step.shape) * step)))
+        assert abs(fd - pred) <= 1e-5 * scale, f"{name}: finite difference {fd:.9e} vs gradient {pred:.9e}"
