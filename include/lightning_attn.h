@@ -278,7 +278,8 @@ LA_API la_status lightning_attn_decode_step_znorm(const void* q, const void* k, 
 
 /*
  * Backward pass of lightning_attn_prefill: the gradients of a loss with respect to q, k, v,
- * the gate and the initial state, given the gradient `dout` of its output.  The pages give
+ * the gate and the initial state, given the gradient `dout` of its output and (optionally)
+ * the gradient `dstate_out` reaching its final state (a later chunk that continued from it).  The pages give
  * no gradient formulas ("MiniMax-Text-01 405B MoE模型架构与训练策略解析" section 2.1 names the
  * operator as trained); they follow from the forward of "六十四：MiniMax-01" section 3 by the
  * chain rule.  Per head, with dy the gradient of the raw output y (dy = dout in RAW mode;
@@ -286,12 +287,14 @@ LA_API la_status lightning_attn_decode_step_znorm(const void* q, const void* k, 
  *   dphi(q_t) = sum_{i<=t} (dy_t . v_i) phi(k_i) + S0 dy_t
  *   dphi(k_i) = sum_{t>=i} (v_i . dy_t) phi(q_t)
  *   dv_i      = sum_{t>=i} (phi(k_i) . phi(q_t)) dy_t,      dS0 = sum_t phi(q_t) dy_t^T
+ * plus, with dS_T = dstate_out:  dphi(k_i) += dS_T v_i,  dv_i += dS_T^T phi(k_i),  dS0 += dS_T
  * and dq = dphi(q) * phi'(q), dk = dphi(k) * phi'(k).  The three sums run as causal
  * linear-attention passes of the prefill kernels (the last two on time-reversed copies).
  *
  *   q, k, v       [B, T, H, D] dtype, the forward's inputs; dout [B, T, H*D] dtype.
  *   g             [B, T, H*D] dtype, required iff mode == LA_OUT_RMSNORM_GATE.
  *   state_in      fp32 [B, H, D, D] the forward's initial states, or NULL (zeros).
+ *   dstate_out    fp32 [B, H, D, D] gradient of the final states, or NULL (zeros).
  *   dq, dk, dv    [B, T, H, D] dtype, written (none may alias an input or each other).
  *   dg            [B, T, H*D] dtype, written iff mode == LA_OUT_RMSNORM_GATE (else ignored).
  *   dstate_in     fp32 [B, H, D, D] gradient of the initial states, or NULL.
@@ -302,8 +305,8 @@ LA_API la_status lightning_attn_decode_step_znorm(const void* q, const void* k, 
  * way).  Returns LA_OK after enqueueing, or an error status with nothing enqueued.
  */
 LA_API la_status lightning_attn_backward(const void* q, const void* k, const void* v, const void* g,
-                                         const void* dout, const float* state_in, void* dq, void* dk, void* dv,
-                                         void* dg, float* dstate_in, int B, int T, int H, int D, int block_size,
+                                         const void* dout, const float* state_in, const float* dstate_out,
+                                         void* dq, void* dk, void* dv, void* dg, float* dstate_in, int B, int T, int H, int D, int block_size,
                                          la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
                                          const float* norm_weight, void* workspace, size_t workspace_bytes,
                                          la_stream_t stream);
@@ -311,13 +314,13 @@ LA_API la_status lightning_attn_backward(const void* q, const void* k, const voi
 /*
  * Backward of lightning_attn_prefill_varlen: as lightning_attn_backward over N packed
  * sequences (q, k, v, dq, dk, dv [total, H, D]; g, dout, dg [total, H*D]; cu_seqlens DEVICE
- * int32 [N + 1] as for the forward; state_in, dstate_in [N, H, D, D] or NULL).  Time is
+ * int32 [N + 1] as for the forward; state_in, dstate_out, dstate_in [N, H, D, D] or NULL).  Time is
  * reversed within each sequence.  Workspace: LA_OP_BACKWARD_VARLEN with N, max_seqlen,
  * total_tokens.
  */
 LA_API la_status lightning_attn_backward_varlen(const void* q, const void* k, const void* v, const void* g,
-                                                const void* dout, const float* state_in, void* dq, void* dk,
-                                                void* dv, void* dg, float* dstate_in, const int* cu_seqlens,
+                                                const void* dout, const float* state_in, const float* dstate_out,
+                                                void* dq, void* dk, void* dv, void* dg, float* dstate_in, const int* cu_seqlens,
                                                 int num_seqs, int max_seqlen, int total_tokens, int H, int D,
                                                 int block_size, la_dtype dtype, la_feature_map phi,
                                                 la_out_mode mode, float eps, const float* norm_weight,

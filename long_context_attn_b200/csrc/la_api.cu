@@ -151,7 +151,7 @@ MixedLayout mixed_layout(int n, int max_pre, int64_t total, int H, int D, int C,
 }
 
 // Backward workspace: [prefill part of the raw-mode passes (error record first)]
-// [6 token buffers: dy, phi(k), rho(v), rho(dy), rho(phi(q)), rho(phi(k))] [S0^T states].
+// [6 token buffers: dy, phi(k), rho(v), rho(dy), rho(phi(q)), rho(phi(k))] [S0^T] [dS_T^T].
 struct BwdLayout {
   size_t pre, buf, st, total;
 };
@@ -160,7 +160,7 @@ BwdLayout bwd_layout(int nseq, int max_len, int64_t tokens, int H, int D, int C,
   b.pre = prefill_ws_bytes(choose_path(dt, H, D, C, LA_OUT_RAW), nseq, max_len, tokens, H, D, C, LA_OUT_RAW);
   b.buf = up256(static_cast<size_t>(tokens) * H * D * (dt == LA_BF16 ? 2 : 4));
   b.st = up256(sizeof(float) * static_cast<size_t>(nseq) * H * D * D);
-  b.total = b.pre + 6 * b.buf + b.st;
+  b.total = b.pre + 6 * b.buf + 2 * b.st;
   return b;
 }
 
@@ -168,7 +168,8 @@ BwdLayout bwd_layout(int nseq, int max_len, int64_t tokens, int H, int D, int C,
 // derivation): [forward recompute of raw y, then dy/dg per token] -> prep -> three
 // raw-mode identity-feature passes of the prefill kernel -> post.
 la_status common_backward(const void* q, const void* k, const void* v, const void* g, const void* dout,
-                          const float* state_in, void* dq, void* dk, void* dv, void* dg, float* dstate,
+                          const float* state_in, const float* dstate_out, void* dq, void* dk, void* dv, void* dg,
+                          float* dstate,
                           const int* cu, int nseq, int T_fixed, int max_len, int64_t tokens, int H, int D, int C,
                           la_dtype dt, la_feature_map phi, la_out_mode mode, float eps, const float* w,
                           void* workspace, size_t ws_bytes, cudaStream_t stream) {
@@ -180,7 +181,8 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
       if (!p || !aligned16(p)) return LA_ERR_INVALID_ARG;
     if (mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g) || !dg || !aligned16(dg))) return LA_ERR_INVALID_ARG;
   }
-  if ((state_in && !aligned16(state_in)) || (dstate && !aligned16(dstate)) || (w && !aligned16(w)))
+  if ((state_in && !aligned16(state_in)) || (dstate && !aligned16(dstate)) || (w && !aligned16(w)) ||
+      (dstate_out && !aligned16(dstate_out)))
     return LA_ERR_INVALID_ARG;
   if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(nseq, max_len, tokens, H, D, C, dt);
@@ -190,6 +192,7 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
   void* buf[6];
   for (int i = 0; i < 6; ++i) buf[i] = base + L.pre + i * L.buf;
   float* s0t = reinterpret_cast<float*>(base + L.pre + 6 * L.buf);
+  float* dstt = reinterpret_cast<float*>(base + L.pre + 6 * L.buf + L.st);
   void *dybuf = buf[0], *fk = buf[1], *rv = buf[2], *rdy = buf[3], *rfq = buf[4], *rfk = buf[5];
   const int HD = H * D;
   const int phi_id = (phi == LA_PHI_IDENTITY) ? 1 : 0;
@@ -219,10 +222,19 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
   }
   // dphi(q): queries dy, keys v, values phi(k), initial state S0^T
   if ((st = pass(dy, v, fk, dq, s0, nullptr, LA_PHI_IDENTITY)) != LA_OK) return st;
-  // reversed dphi(k): queries rho(v), keys rho(dy), values rho(phi(q))
-  if ((st = pass(rv, rdy, rfq, dk, nullptr, nullptr, LA_PHI_IDENTITY)) != LA_OK) return st;
-  // reversed dv: queries rho(phi(k)), keys rho(phi(q)), values rho(dy); final state = dS0
-  if ((st = pass(rfk, rfq, rdy, dv, nullptr, dstate, LA_PHI_IDENTITY)) != LA_OK) return st;
+  // A gradient reaching the final state starts the reverse sums: dphi(k) gets dS_T v, dv gets
+  // dS_T^T phi(k), dS0 includes dS_T.
+  const float* dsT_t = nullptr;
+  if (dstate_out) {
+    if (la::launch_transpose_states(dstate_out, dstt, static_cast<int64_t>(nseq) * H, D, stream) != cudaSuccess)
+      return LA_ERR_CUDA;
+    dsT_t = dstt;
+  }
+  // reversed dphi(k): queries rho(v), keys rho(dy), values rho(phi(q)), initial state dS_T^T
+  if ((st = pass(rv, rdy, rfq, dk, dsT_t, nullptr, LA_PHI_IDENTITY)) != LA_OK) return st;
+  // reversed dv: queries rho(phi(k)), keys rho(phi(q)), values rho(dy), initial state dS_T;
+  // its final state is dS0
+  if ((st = pass(rfk, rfq, rdy, dv, dstate_out, dstate, LA_PHI_IDENTITY)) != LA_OK) return st;
   if (la::launch_bwd_post(q, k, dq, dk, dv, cu, nseq, T_fixed, tokens, HD, phi_id, dt, stream) != cudaSuccess)
     return LA_ERR_CUDA;
   return LA_OK;
@@ -306,30 +318,31 @@ la_status lightning_attn_prefill(const void* q, const void* k, const void* v, co
 }
 
 la_status lightning_attn_backward(const void* q, const void* k, const void* v, const void* g, const void* dout,
-                                  const float* state_in, void* dq, void* dk, void* dv, void* dg, float* dstate_in,
+                                  const float* state_in, const float* dstate_out, void* dq, void* dk, void* dv,
+                                  void* dg, float* dstate_in,
                                   int B, int T, int H, int D, int block_size, la_dtype dtype, la_feature_map phi,
                                   la_out_mode mode, float eps, const float* norm_weight, void* workspace,
                                   size_t workspace_bytes, la_stream_t stream) {
   if (B < 1 || T < 0) return LA_ERR_INVALID_ARG;
   const int64_t tokens = static_cast<int64_t>(B) * T;
   if (tokens > INT32_MAX) return LA_ERR_UNSUPPORTED;
-  return common_backward(q, k, v, g, dout, state_in, dq, dk, dv, dg, dstate_in, nullptr, B, T, T, tokens, H, D,
-                         block_size, dtype, phi, mode, eps, norm_weight, workspace, workspace_bytes,
+  return common_backward(q, k, v, g, dout, state_in, dstate_out, dq, dk, dv, dg, dstate_in, nullptr, B, T, T,
+                         tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight, workspace, workspace_bytes,
                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 la_status lightning_attn_backward_varlen(const void* q, const void* k, const void* v, const void* g,
-                                         const void* dout, const float* state_in, void* dq, void* dk, void* dv,
-                                         void* dg, float* dstate_in, const int* cu_seqlens, int num_seqs,
+                                         const void* dout, const float* state_in, const float* dstate_out,
+                                         void* dq, void* dk, void* dv, void* dg, float* dstate_in, const int* cu_seqlens, int num_seqs,
                                          int max_seqlen, int total_tokens, int H, int D, int block_size,
                                          la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
                                          const float* norm_weight, void* workspace, size_t workspace_bytes,
                                          la_stream_t stream) {
   if (num_seqs < 1 || !cu_seqlens || !aligned16(cu_seqlens) || total_tokens < 0 || max_seqlen < 0)
     return LA_ERR_INVALID_ARG;
-  return common_backward(q, k, v, g, dout, state_in, dq, dk, dv, dg, dstate_in, cu_seqlens, num_seqs, 0, max_seqlen,
-                         total_tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight, workspace,
-                         workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+  return common_backward(q, k, v, g, dout, state_in, dstate_out, dq, dk, dv, dg, dstate_in, cu_seqlens, num_seqs,
+                         0, max_seqlen, total_tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight,
+                         workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 la_status lightning_attn_chunk_state(const void* k, const void* v, const float* state_in, float* state_out, int B,

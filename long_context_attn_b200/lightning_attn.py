@@ -63,8 +63,8 @@ def _load():
     lib.lightning_attn_prefill_znorm.argtypes = [vp] * 9 + [i32] * 8 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_prefill_znorm_varlen.argtypes = [vp] * 10 + [i32] * 9 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_decode_step_znorm.argtypes = [vp] * 7 + [i32] * 6 + [f32, vp, vp, sz, vp]
-    lib.lightning_attn_backward.argtypes = [vp] * 11 + [i32] * 8 + [f32, vp, vp, sz, vp]
-    lib.lightning_attn_backward_varlen.argtypes = [vp] * 12 + [i32] * 9 + [f32, vp, vp, sz, vp]
+    lib.lightning_attn_backward.argtypes = [vp] * 12 + [i32] * 8 + [f32, vp, vp, sz, vp]
+    lib.lightning_attn_backward_varlen.argtypes = [vp] * 13 + [i32] * 9 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp,
                                                sz, vp]
     lib.lightning_attn_decode_step_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32,
@@ -234,12 +234,14 @@ def lightning_attn_decode_step_znorm(q, k, v, g, out, state, z, phi=LA_PHI_SILU,
 
 def lightning_attn_backward(q, k, v, g, dout, dq, dk, dv, dg=None, state_in=None, dstate_in=None, block_size=256,
                             phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE, eps=1e-6, norm_weight=None, workspace=None,
-                            stream=None):
-    """q, k, v, dq, dk, dv [B, T, H, D]; g, dout, dg [B, T, H*D]; states fp32 [B, H, D, D]."""
+                            stream=None, dstate_out=None):
+    """q, k, v, dq, dk, dv [B, T, H, D]; g, dout, dg [B, T, H*D]; states fp32 [B, H, D, D]
+    (dstate_out: the gradient reaching the final states)."""
     B, T, H, D = q.shape
-    _check_contig(q, k, v, g, dout, dq, dk, dv, dg)
+    _check_contig(q, k, v, g, dout, dq, dk, dv, dg, dstate_out)
     st = _lib.lightning_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout), _ptr(_f32_or_none(state_in)),
-                                      _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(_f32_or_none(dstate_in)), B, T, H,
+                                      _ptr(_f32_or_none(dstate_out)), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+                                      _ptr(_f32_or_none(dstate_in)), B, T, H,
                                       D, block_size, _dtype(q), phi, mode, eps, _ptr(_f32_or_none(norm_weight)),
                                       _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                       _stream(stream))
@@ -249,15 +251,15 @@ def lightning_attn_backward(q, k, v, g, dout, dq, dk, dv, dg=None, state_in=None
 
 def lightning_attn_backward_varlen(q, k, v, g, dout, dq, dk, dv, cu_seqlens, max_seqlen, dg=None, state_in=None,
                                    dstate_in=None, block_size=256, phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE,
-                                   eps=1e-6, norm_weight=None, workspace=None, stream=None):
+                                   eps=1e-6, norm_weight=None, workspace=None, stream=None, dstate_out=None):
     """q, k, v, dq, dk, dv [total, H, D]; g, dout, dg [total, H*D]; cu_seqlens int32 device [N + 1]."""
     total, H, D = q.shape
-    _check_contig(q, k, v, g, dout, dq, dk, dv, dg, cu_seqlens)
+    _check_contig(q, k, v, g, dout, dq, dk, dv, dg, cu_seqlens, dstate_out)
     if cu_seqlens.dtype != torch.int32:
         raise TypeError("cu_seqlens must be int32")
     n = cu_seqlens.numel() - 1
     st = _lib.lightning_attn_backward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout),
-                                             _ptr(_f32_or_none(state_in)), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+                                             _ptr(_f32_or_none(state_in)), _ptr(_f32_or_none(dstate_out)), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
                                              _ptr(_f32_or_none(dstate_in)), _ptr(cu_seqlens), n, int(max_seqlen),
                                              total, H, D, block_size, _dtype(q), phi, mode, eps,
                                              _ptr(_f32_or_none(norm_weight)), _ptr(workspace),

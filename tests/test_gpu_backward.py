@@ -22,12 +22,14 @@ def _la():
 
 
 def _run_fixed(B, T, H, D, C, dtype, mode, with_state, seed, expect=None):
+    """with_state: an initial state S0 and a final-state gradient dS_T as well."""
     import torch
     la = _la()
     m = mode_code(mode)
     q, k, v, g = synth.prefill_inputs(seed, B * T, H, D, dtype, 0.5, True)
     dout = synth.normal(seed, 21, (B * T, H * D), 1.0, dtype)
     s0 = synth.normal(seed, 22, (B, H, D, D), 0.05, "f32") if with_state else None
+    dsT = synth.normal(seed, 24, (B, H, D, D), 0.05, "f32") if with_state else None
     w = (1.0 + 0.2 * synth.normal(seed, 23, (H * D,), 1.0, "f32")).astype(np.float32) if m else None
     shp, gshp = (B, T, H, D), (B, T, H * D)
     dq_, dk_, dv_, dg_ = (to_dev(a).reshape(shp if i < 3 else gshp) for i, a in enumerate((q, k, v, g)))
@@ -38,13 +40,14 @@ def _run_fixed(B, T, H, D, C, dtype, mode, with_state, seed, expect=None):
     ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD, B, T, 0, H, D, C, la._dtype(dq_), m))
     la.lightning_attn_backward(dq_, dk_, dv_, dg_ if m == la.LA_OUT_RMSNORM_GATE else None, ddo, gq, gk, gv, dg=gg,
                                state_in=None if s0 is None else to_dev(s0), dstate_in=gs, block_size=C, mode=m,
-                               norm_weight=None if w is None else to_dev(w), workspace=ws)
+                               norm_weight=None if w is None else to_dev(w), workspace=ws,
+                               dstate_out=None if dsT is None else to_dev(dsT))
     if expect:
         assert la.lightning_attn_last_path() == expect
     la.lightning_attn_check(ws)
     r = lambda a, s: a.reshape(s)
     ref = oracle.backward(r(q, shp), r(k, shp), r(v, shp), r(g, gshp) if m == la.LA_OUT_RMSNORM_GATE else None,
-                          r(dout, gshp), state_in=s0, mode=m, norm_weight=w)
+                          r(dout, gshp), state_in=s0, mode=m, norm_weight=w, dstate_out=dsT)
     assert_close(to_host(gq), ref[0], dtype, "dq")
     assert_close(to_host(gk), ref[1], dtype, "dk")
     assert_close(to_host(gv), ref[2], dtype, "dv")
@@ -80,6 +83,7 @@ def test_backward_varlen(C, cuda_device):
     q, k, v, g = synth.prefill_inputs(3301, tot, H, D, "bf16", 0.5, True)
     dout = synth.normal(3301, 21, (tot, H * D), 1.0, "bf16")
     s0 = synth.normal(3301, 22, (n, H, D, D), 0.05, "f32")
+    dsT = synth.normal(3301, 24, (n, H, D, D), 0.05, "f32")
     dq_, dk_, dv_, dg_, ddo = (to_dev(a) for a in (q, k, v, g, dout))
     gq, gk, gv = (torch.full_like(dq_, float("nan")) for _ in range(3))
     gg = torch.full_like(dg_, float("nan"))
@@ -87,10 +91,11 @@ def test_backward_varlen(C, cuda_device):
     ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD_VARLEN, n, max(lens), tot, H, D, C,
                                                            la.LA_BF16, la.LA_OUT_RMSNORM_GATE))
     la.lightning_attn_backward_varlen(dq_, dk_, dv_, dg_, ddo, gq, gk, gv, torch.from_numpy(cu).cuda(), max(lens),
-                                      dg=gg, state_in=to_dev(s0), dstate_in=gs, block_size=C, workspace=ws)
+                                      dg=gg, state_in=to_dev(s0), dstate_in=gs, block_size=C, workspace=ws,
+                                      dstate_out=to_dev(dsT))
     assert la.lightning_attn_last_path() == "tcgen05"
     la.lightning_attn_check(ws)
-    ref = oracle.backward_packed(q, k, v, g, dout, cu, H, D, state_in=s0)
+    ref = oracle.backward_packed(q, k, v, g, dout, cu, H, D, state_in=s0, dstate_out=dsT)
     for got, want, name in zip((gq, gk, gv, gg, gs), ref, ("dq", "dk", "dv", "dg", "dstate")):
         assert_close(to_host(got), want, "bf16", name)
 
@@ -122,6 +127,7 @@ def test_backward_exact_integers(C, T, cuda_device):
     H, D = 4, 128
     q, k, v, dout = (synth.ternary(3501 + T, s, (T, H, D), 0.06, "bf16") for s in range(4))
     s0 = np.round(synth.normal(3501, 9, (1, H, D, D), 1.0, "f32")).astype(np.float32)
+    dsT = np.round(synth.normal(3501, 10, (1, H, D, D), 1.0, "f32")).astype(np.float32)
     f = lambda a: synth.bf16_to_f32(a).astype(np.float64)
     Q, K, V, dY = f(q), f(k), f(v), f(dout)
     # every intermediate the three passes hold: running sums of v k^T (forward) and of
@@ -129,7 +135,7 @@ def test_backward_exact_integers(C, T, cuda_device):
     for a, b, rev in ((V, K, False), (dY, Q, True), (Q, dY, True), (K, V, False)):
         outer = np.einsum("thi,thj->thij", a, b)
         run = np.cumsum(outer[::-1] if rev else outer, axis=0)
-        assert np.abs(run).max() + np.abs(s0).max() <= 256
+        assert np.abs(run).max() + np.abs(s0).max() + np.abs(dsT).max() <= 256
     shp = (1, T, H, D)
     dq_, dk_, dv_ = (to_dev(a).reshape(shp) for a in (q, k, v))
     ddo = to_dev(dout).reshape(1, T, H * D)
@@ -138,11 +144,12 @@ def test_backward_exact_integers(C, T, cuda_device):
     ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD, 1, T, 0, H, D, C, la.LA_BF16,
                                                            la.LA_OUT_RAW))
     la.lightning_attn_backward(dq_, dk_, dv_, None, ddo, gq, gk, gv, state_in=to_dev(s0), dstate_in=gs,
-                               block_size=C, phi=la.LA_PHI_IDENTITY, mode=la.LA_OUT_RAW, workspace=ws)
+                               block_size=C, phi=la.LA_PHI_IDENTITY, mode=la.LA_OUT_RAW, workspace=ws,
+                               dstate_out=to_dev(dsT))
     assert la.lightning_attn_last_path() == "tcgen05"
     la.lightning_attn_check(ws)
     ref = oracle.backward(q.reshape(shp), k.reshape(shp), v.reshape(shp), None, dout.reshape(1, T, H * D),
-                          state_in=s0, phi=oracle.PHI_IDENTITY, mode=oracle.MODE_RAW)
+                          state_in=s0, phi=oracle.PHI_IDENTITY, mode=oracle.MODE_RAW, dstate_out=dsT)
     for got, want, name in zip((gq, gk, gv, gs), (ref[0], ref[1], ref[2], ref[4]), ("dq", "dk", "dv", "dstate")):
         assert np.abs(want).max() <= 256, name
         g64 = synth.bf16_to_f32(to_host(got)).astype(np.float64) if got.dtype == torch.bfloat16 \
