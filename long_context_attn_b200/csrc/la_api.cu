@@ -79,16 +79,22 @@ bool device_is_sm100() {
 }
 
 // Which prefill kernel a call takes.
-enum class Path { kTc, kSimt };
+// kTc: the tensor-core kernel with the norm fused (all of a tile's heads resident at once);
+// kTcSplit: more heads than fit at once in a norm mode -- the tensor-core kernel in raw
+// mode, then the norm and gate per token in place; kSimt: the CUDA-core kernel.
+enum class Path { kTc, kTcSplit, kSimt };
 
 Path choose_path(la_dtype dt, int H, int D, int C, la_out_mode mode) {
+  if (!device_is_sm100()) return Path::kSimt;
   la::TcShape s{H, D, C, dt == LA_BF16, static_cast<int>(mode)};
-  if (device_is_sm100() && la::tc_eligible(s, current_sm_count())) return Path::kTc;
+  if (la::tc_eligible(s, current_sm_count())) return Path::kTc;
+  la::TcShape raw{H, D, C, dt == LA_BF16, static_cast<int>(LA_OUT_RAW)};
+  if (mode != LA_OUT_RAW && la::tc_eligible(raw, current_sm_count())) return Path::kTcSplit;
   return Path::kSimt;
 }
 
 size_t prefill_ws_bytes(Path p, int nseq, int max_len, int64_t tokens, int H, int D, int C, la_out_mode mode) {
-  if (p == Path::kTc) return kErrBytes + la::tc_workspace_bytes(nseq, max_len, tokens, H, D, C);
+  if (p == Path::kTc || p == Path::kTcSplit) return kErrBytes + la::tc_workspace_bytes(nseq, max_len, tokens, H, D, C);
   size_t y = (mode == LA_OUT_RAW) ? 0 : up256(sizeof(float) * static_cast<size_t>(tokens) * H * D);
   return kErrBytes + y;
 }
@@ -116,15 +122,19 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
   char* ws = static_cast<char*>(workspace) + kErrBytes;
   const int phi_id = (phi == LA_PHI_IDENTITY) ? 1 : 0;
   cudaError_t e;
-  if (path == Path::kTc) {
+  if (path == Path::kTc || path == Path::kTcSplit) {
+    const bool split = path == Path::kTcSplit;
     la::TcArgs a{};
     a.q = q; a.k = k; a.v = v; a.g = g; a.out = out;
     a.state_in = state_in; a.state_out = state_out; a.cu = cu;
     a.nseq = nseq; a.T = T_fixed; a.max_len = max_len; a.tokens = tokens;
-    a.H = H; a.D = D; a.C = C; a.phi_identity = phi_id; a.mode = static_cast<int>(mode);
-    a.eps = eps; a.w = w; a.err = err; a.ws = ws;
+    a.H = H; a.D = D; a.C = C; a.phi_identity = phi_id;
+    a.mode = static_cast<int>(split ? LA_OUT_RAW : mode);
+    a.eps = eps; a.w = split ? nullptr : w; a.err = err; a.ws = ws;
     e = la::launch_tc_prefill(a, current_sm_count(), stream);
-    g_last_path = "tcgen05";
+    if (e == cudaSuccess && split)   // the norm (and gate) per token, over the raw output in place
+      e = la::launch_znorm_transform(out, nullptr, g, w, tokens, H, D, static_cast<int>(mode), eps, dt, stream);
+    g_last_path = split ? "tcgen05+norm" : "tcgen05";
   } else {
     float* y_ws = (mode == LA_OUT_RAW) ? nullptr : reinterpret_cast<float*>(ws);
     e = la::launch_simt_prefill(q, k, v, out, y_ws, state_in, state_out, cu, nseq, T_fixed, H, D, C, dt, phi_id,

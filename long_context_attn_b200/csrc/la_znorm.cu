@@ -171,6 +171,8 @@ __global__ void __launch_bounds__(256, 2) z_den_kernel(const T* __restrict__ q, 
 
 // One CTA per token: y / den per head, then RAW / RMSNORM / RMSNORM_GATE, in place on io.
 // 8-element vectors; the H reciprocals of the token's denominators sit in shared memory.
+// With den null it is the output transform alone (the prefill's norm when too many heads
+// for the fused exchange).
 template <typename T, int D>
 __global__ void __launch_bounds__(256) znorm_transform_kernel(T* io, const float* __restrict__ den,
                                                               const T* __restrict__ g, const float* __restrict__ w,
@@ -181,7 +183,7 @@ __global__ void __launch_bounds__(256) znorm_transform_kernel(T* io, const float
   const int64_t row = blockIdx.x;
   const int HD = H * D;
   T* y = io + row * HD;
-  for (int h = threadIdx.x; h < H; h += blockDim.x) rden[h] = 1.0f / den[row * H + h];
+  for (int h = threadIdx.x; h < H; h += blockDim.x) rden[h] = den ? 1.0f / den[row * H + h] : 1.0f;
   __syncthreads();
   float r = 1.0f;
   if (mode != LA_OUT_RAW) {

@@ -167,3 +167,19 @@ def test_tc_config_varlen16_full(cuda_device):
     assert stats["out_nonfinite"] == 0 and stats["state_nonfinite"] == 0
     assert stats["out_max_err"] <= 2e-2 * stats["out_max_ref"], stats
     assert stats["state_max_err"] <= 2e-2 * stats["state_max_ref"], stats
+
+
+@pytest.mark.parametrize("mode,expect", [("rmsnorm_gate", "tcgen05+norm"), ("rmsnorm", "tcgen05+norm"),
+                                         ("raw", "tcgen05")])
+def test_tc_more_heads_than_resident_pairs(mode, expect, cuda_device):
+    """H = 100: more CTA pairs than fit on the GPU at once.  The raw mode runs the tensor-core
+    kernel in waves; the norm modes run it raw and then the norm per token in place."""
+    H, D, T, C = 100, 128, 300, 256
+    q, k, v, g = synth.prefill_inputs(3801, T, H, D, "bf16", 0.5, True)
+    m = mode_code(mode)
+    o, st, _ = run_prefill(q[None], k[None], v[None], g[None] if m == oracle.MODE_RMSNORM_GATE else None, C, m,
+                           want_state=True, expect_path=expect)
+    ref, ref_st, _ = oracle.prefill(q[None], k[None], v[None], g[None] if m == oracle.MODE_RMSNORM_GATE else None,
+                                    mode=m)
+    assert_close(o, ref, "bf16")
+    assert_close(st, ref_st, "bf16", "state")
