@@ -505,6 +505,52 @@ class BackwardCase:
                 "l2": "inputs larger than L2 (%.1f GB per step), no flush" % (self.alg_bytes / 1e9)}
 
 
+class TrainCase(BackwardCase):
+    """A training step on one long sequence: the forward keeping its raw output y (prefill in
+    raw mode, then the norm and gate), and the backward from dout using that y."""
+
+    def __init__(self, name, w, device, rank):
+        super().__init__(name, w, device, rank)
+        import torch
+        T, H, D = self.T, self.H, self.D
+        self.y = torch.empty((1, T, H * D), dtype=torch.bfloat16, device=device)
+        self.out = torch.empty((1, T, H * D), dtype=torch.bfloat16, device=device)
+        self.h_out_fwd = torch.empty((1, T, H * D), dtype=torch.bfloat16).pin_memory()
+        # forward: q, k, v, g read + out written; backward: q, k, v, g, dout read + 4 gradients written
+        self.alg_bytes = T * 14 * H * D * 2
+        # the forward prefill plus the backward's three passes (the recompute is skipped)
+        self.alg_flops, self.issued_flops = (4 * x * T for x in _flops_per_token(H, D, self.C))
+        self.launches_per_step = 8    # prefill, transform, norm/gate backward, prep, three passes, post
+        self.d2h += self.h_out_fwd.numel() * 2
+
+    def step(self):
+        la = self.la
+        q, k, v, g, dout = self.d_in
+        dq, dk, dv, dg = self.d_out
+        B, T, H, D = q.shape
+        la.lightning_attn_prefill(q, k, v, None, self.y, None, None, block_size=self.C, mode=la.LA_OUT_RAW,
+                                  workspace=self.ws)
+        la.lightning_attn_output_transform(self.y.view(B, T, H, D), g, self.out)
+        la.lightning_attn_backward(q, k, v, g, dout, dq, dk, dv, dg=dg, block_size=self.C, workspace=self.ws, y=self.y)
+
+    def e2e_step(self):
+        super().e2e_step()
+        self.h_out_fwd.copy_(self.out, non_blocking=True)
+
+    def oracle_sample(self, tokens):
+        import oracle
+        w = self.w
+        q, k, v, g = synth.prefill_inputs(w.seed, tokens, w.H, w.D, "bf16", w.qkv_scale, True)
+        dout = synth.normal(w.seed, synth.STREAM_DOUT, (tokens, w.H * w.D), 1.0, "bf16")
+        t0 = time.perf_counter()
+        oracle.prefill(q[None], k[None], v[None], g[None], store=False)
+        oracle.backward(q[None], k[None], v[None], g[None], dout[None])
+        return time.perf_counter() - t0
+
+    def describe(self):
+        return dict(super().describe(), step="forward (raw prefill + norm/gate, y kept) + backward with y")
+
+
 class MixedCase:
     """One serving step: 256 sequences decode a token each while 2 others prefill a 4096-token
     chunk from their state; prefill and decode on two streams, states in a pool (slots in a
@@ -613,6 +659,8 @@ def _make_case(name, device, rank):
         return DecodeCase(name, w, device, rank)
     if w.kind == "backward":
         return BackwardCase(name, w, device, rank)
+    if w.kind == "train":
+        return TrainCase(name, w, device, rank)
     if w.kind == "znorm":
         return ZnormCase(name, w, device, rank)
     if w.kind == "chunk_state":
@@ -720,7 +768,10 @@ def run_gpu(args):
                               "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": _traffic(args.workload),
                               "peak_source": peaks["source"], "launch_ms": launch_ms,
                               "algorithmic_bytes_per_launch": case.alg_bytes},
-                             **({"scope": "one backward call (7 kernels); algorithmic bytes = its inputs "
+                             **({"scope": "one training step (forward + backward, 8 kernels); algorithmic "
+                                          "bytes = both calls' inputs read and outputs written once"}
+                                if isinstance(case, TrainCase) else
+                                {"scope": "one backward call (7 kernels); algorithmic bytes = its inputs "
                                           "read and gradients written once"}
                                 if isinstance(case, BackwardCase) else
                                 {"scope": "one normalised-variant call (5 kernels); algorithmic bytes as the "
@@ -807,9 +858,11 @@ def _cpu_baseline(case):
     if isinstance(case, BackwardCase):
         n = min(16384, case.T)
         dt = case.oracle_sample(n)
+        what = "forward + backward" if isinstance(case, TrainCase) else \
+            "backward (forward recompute, norm/gate backward, both scans)"
         return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-                "sample": f"first {n} tokens of the {case.w.name} workload, all {case.H} heads, fp64 backward "
-                          f"(forward recompute, norm/gate backward, both scans) ({dt:.1f} s)"}
+                "sample": f"first {n} tokens of the {case.w.name} workload, all {case.H} heads, fp64 {what} "
+                          f"({dt:.1f} s)"}
     if isinstance(case, VarlenCase):
         dt, n = case.oracle_sample(131072)
         return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
@@ -828,7 +881,17 @@ def run_reference(args):
         return
     import oracle
     w = synth.WORKLOADS[args.workload]
-    if w.kind == "chunk_state":
+    if w.kind == "train":
+        n = 512
+        q, k, v, g = synth.prefill_inputs(w.seed, n, w.H, w.D, w.dtype, w.qkv_scale, True)
+        dout = synth.normal(w.seed, synth.STREAM_DOUT, (n, w.H * w.D), 1.0, w.dtype)
+
+        def step():
+            oracle.prefill(q[None], k[None], v[None], g[None], store=False)
+            oracle.backward(q[None], k[None], v[None], g[None], dout[None])
+        unit_per_step = n
+        sample = f"first {n} tokens of {w.name} (all {w.H} heads) per step, fp64 forward + backward"
+    elif w.kind == "chunk_state":
         n = 1024
         _, k, v, _ = synth.prefill_inputs(w.seed, n, w.H, w.D, w.dtype, w.qkv_scale, False)
 
@@ -898,7 +961,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="prefill_128k",
                     choices=["prefill_8k", "prefill_128k", "varlen_16", "decode_256", "mixed_256", "backward_8k",
-                             "backward_128k", "znorm_128k", "chunk_state_128k"])
+                             "backward_128k", "train_128k", "znorm_128k", "chunk_state_128k"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     args = ap.parse_args()

@@ -295,6 +295,10 @@ LA_API la_status lightning_attn_decode_step_znorm(const void* q, const void* k, 
  *   g             [B, T, H*D] dtype, required iff mode == LA_OUT_RMSNORM_GATE.
  *   state_in      fp32 [B, H, D, D] the forward's initial states, or NULL (zeros).
  *   dstate_out    fp32 [B, H, D, D] gradient of the final states, or NULL (zeros).
+ *   y             [B, T, H*D] dtype: the forward's raw output (its y before the norm, as
+ *                 lightning_attn_prefill in LA_OUT_RAW mode gives it), or NULL.  In the norm
+ *                 modes the backward needs y; given, it is used, else it is recomputed (one
+ *                 more pass of the prefill kernel).  Ignored in LA_OUT_RAW mode.
  *   dq, dk, dv    [B, T, H, D] dtype, written (none may alias an input or each other).
  *   dg            [B, T, H*D] dtype, written iff mode == LA_OUT_RMSNORM_GATE (else ignored).
  *   dstate_in     fp32 [B, H, D, D] gradient of the initial states, or NULL.
@@ -306,7 +310,7 @@ LA_API la_status lightning_attn_decode_step_znorm(const void* q, const void* k, 
  */
 LA_API la_status lightning_attn_backward(const void* q, const void* k, const void* v, const void* g,
                                          const void* dout, const float* state_in, const float* dstate_out,
-                                         void* dq, void* dk, void* dv, void* dg, float* dstate_in, int B, int T, int H, int D, int block_size,
+                                         const void* y, void* dq, void* dk, void* dv, void* dg, float* dstate_in, int B, int T, int H, int D, int block_size,
                                          la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
                                          const float* norm_weight, void* workspace, size_t workspace_bytes,
                                          la_stream_t stream);
@@ -314,17 +318,33 @@ LA_API la_status lightning_attn_backward(const void* q, const void* k, const voi
 /*
  * Backward of lightning_attn_prefill_varlen: as lightning_attn_backward over N packed
  * sequences (q, k, v, dq, dk, dv [total, H, D]; g, dout, dg [total, H*D]; cu_seqlens DEVICE
- * int32 [N + 1] as for the forward; state_in, dstate_out, dstate_in [N, H, D, D] or NULL).  Time is
+ * int32 [N + 1] as for the forward; state_in, dstate_out, dstate_in [N, H, D, D] or NULL; y
+ * [total, H*D] or NULL).  Time is
  * reversed within each sequence.  Workspace: LA_OP_BACKWARD_VARLEN with N, max_seqlen,
  * total_tokens.
  */
 LA_API la_status lightning_attn_backward_varlen(const void* q, const void* k, const void* v, const void* g,
                                                 const void* dout, const float* state_in, const float* dstate_out,
-                                                void* dq, void* dk, void* dv, void* dg, float* dstate_in, const int* cu_seqlens,
+                                                const void* y, void* dq, void* dk, void* dv, void* dg,
+                                                float* dstate_in, const int* cu_seqlens,
                                                 int num_seqs, int max_seqlen, int total_tokens, int H, int D,
                                                 int block_size, la_dtype dtype, la_feature_map phi,
                                                 la_out_mode mode, float eps, const float* norm_weight,
                                                 void* workspace, size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * The output transform alone ("MiniMax-Text-01 405B MoE模型架构与训练策略解析" section 2.1), per
+ * token over the H*D concatenation:  RAW: out = y;  RMSNORM: out = y * r * w;
+ * RMSNORM_GATE: out = y * r * w * sigmoid(g), with r = 1 / sqrt(mean(y^2) + eps).
+ * With lightning_attn_prefill in LA_OUT_RAW mode it gives the normalised output while
+ * keeping y (for lightning_attn_backward's `y`).
+ *   y, out      [tokens, H*D] dtype, device; out may equal y (in place).
+ *   g           [tokens, H*D] dtype, required iff mode == LA_OUT_RMSNORM_GATE.
+ *   H*D <= 16384; norm_weight fp32 [H*D] or NULL (ones).
+ */
+LA_API la_status lightning_attn_output_transform(const void* y, const void* g, void* out, int tokens, int H, int D,
+                                                 la_dtype dtype, la_out_mode mode, float eps,
+                                                 const float* norm_weight, la_stream_t stream);
 
 /*
  * The state lightning_attn_prefill would end with, without computing its outputs:

@@ -3,9 +3,11 @@
 `lightning_attention(q, k, v, g, state_in=None, ...)` returns `(out, state_out)` like one
 `lightning_attn_prefill` call and is differentiable in q, k, v, g and state_in: its
 backward is one `lightning_attn_backward` call (the gradient reaching `state_out`, when the
-final state feeds later computation, is passed to it as dstate_out).  This module only
-orders the library calls and allocates their outputs; every computation runs in the
-library's kernels.
+final state feeds later computation, is passed to it as dstate_out).  When gradients are
+needed in a norm mode, the forward runs the prefill in raw mode and then the output
+transform, keeping the raw output y, which saves the backward its recompute of y.  This
+module only orders the library calls and allocates their outputs; every computation runs
+in the library's kernels.
 """
 from __future__ import annotations
 
@@ -22,19 +24,30 @@ class _LightningAttention(torch.autograd.Function):
         g = None if g is None else g.contiguous()
         out = torch.empty((B, T, H * D), dtype=q.dtype, device=q.device)
         state_out = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
-        ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_PREFILL, B, T, 0, H, D, block_size,
-                                                               la._dtype(q), mode), q.device)
         s_in = None if state_in is None else state_in.detach().contiguous()
-        la.lightning_attn_prefill(q, k, v, g, out, s_in, state_out, block_size=block_size, phi=phi, mode=mode,
-                                  eps=eps, norm_weight=norm_weight, workspace=ws)
-        ctx.save_for_backward(q, k, v, g, s_in, norm_weight)
+        keep_y = mode != la.LA_OUT_RAW and any(ctx.needs_input_grad[:5])
+        y = None
+        if keep_y:   # raw prefill, then the norm (and gate) from the kept y
+            y = torch.empty_like(out)
+            ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_PREFILL, B, T, 0, H, D, block_size,
+                                                                   la._dtype(q), la.LA_OUT_RAW), q.device)
+            la.lightning_attn_prefill(q, k, v, None, y, s_in, state_out, block_size=block_size, phi=phi,
+                                      mode=la.LA_OUT_RAW, workspace=ws)
+            la.lightning_attn_output_transform(y.view(B, T, H, D), g, out, mode=mode, eps=eps,
+                                               norm_weight=norm_weight)
+        else:        # the fused kernel
+            ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_PREFILL, B, T, 0, H, D, block_size,
+                                                                   la._dtype(q), mode), q.device)
+            la.lightning_attn_prefill(q, k, v, g, out, s_in, state_out, block_size=block_size, phi=phi, mode=mode,
+                                      eps=eps, norm_weight=norm_weight, workspace=ws)
+        ctx.save_for_backward(q, k, v, g, s_in, norm_weight, y)
         ctx.cfg = (block_size, phi, mode, eps)
         ctx.has_state = state_in is not None
         return out, state_out
 
     @staticmethod
     def backward(ctx, dout, dstate_out):
-        q, k, v, g, s_in, norm_weight = ctx.saved_tensors
+        q, k, v, g, s_in, norm_weight, y = ctx.saved_tensors
         block_size, phi, mode, eps = ctx.cfg
         B, T, H, D = q.shape
         if dout is None:
@@ -48,7 +61,7 @@ class _LightningAttention(torch.autograd.Function):
         la.lightning_attn_backward(q, k, v, g if mode == la.LA_OUT_RMSNORM_GATE else None, dout, dq, dk, dv, dg=dg,
                                    state_in=s_in, dstate_in=ds_in, block_size=block_size, phi=phi, mode=mode,
                                    eps=eps, norm_weight=norm_weight, workspace=ws,
-                                   dstate_out=None if dstate_out is None else dstate_out.float().contiguous())
+                                   dstate_out=None if dstate_out is None else dstate_out.float().contiguous(), y=y)
         return dq, dk, dv, dg, ds_in, None, None, None, None, None
 
 

@@ -40,6 +40,9 @@ cudaError_t launch_znorm_scan(const void* q, const void* k, const float* z_in, f
                               la_dtype dt, int phi_identity, cudaStream_t stream);
 cudaError_t launch_znorm_transform(void* io, const float* den, const void* g, const float* w, int64_t tokens, int H,
                                    int D, int mode, float eps, la_dtype dt, cudaStream_t stream);
+cudaError_t launch_output_transform(const void* src, void* dst, const float* den, const void* g, const float* w,
+                                    int64_t tokens, int H, int D, int mode, float eps, la_dtype dt,
+                                    cudaStream_t stream);
 }  // namespace la
 
 namespace {
@@ -178,8 +181,8 @@ BwdLayout bwd_layout(int nseq, int max_len, int64_t tokens, int H, int D, int C,
 // derivation): [forward recompute of raw y, then dy/dg per token] -> prep -> three
 // raw-mode identity-feature passes of the prefill kernel -> post.
 la_status common_backward(const void* q, const void* k, const void* v, const void* g, const void* dout,
-                          const float* state_in, const float* dstate_out, void* dq, void* dk, void* dv, void* dg,
-                          float* dstate,
+                          const float* state_in, const float* dstate_out, const void* y_saved, void* dq, void* dk,
+                          void* dv, void* dg, float* dstate,
                           const int* cu, int nseq, int T_fixed, int max_len, int64_t tokens, int H, int D, int C,
                           la_dtype dt, la_feature_map phi, la_out_mode mode, float eps, const float* w,
                           void* workspace, size_t ws_bytes, cudaStream_t stream) {
@@ -192,7 +195,7 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
     if (mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g) || !dg || !aligned16(dg))) return LA_ERR_INVALID_ARG;
   }
   if ((state_in && !aligned16(state_in)) || (dstate && !aligned16(dstate)) || (w && !aligned16(w)) ||
-      (dstate_out && !aligned16(dstate_out)))
+      (dstate_out && !aligned16(dstate_out)) || (y_saved && !aligned16(y_saved)))
     return LA_ERR_INVALID_ARG;
   if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(nseq, max_len, tokens, H, D, C, dt);
@@ -214,10 +217,15 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
   la_status st;
   const void* dy = dout;
   if (mode != LA_OUT_RAW) {
-    // raw y of the forward (from the same initial state), then dy (in place) and dg
-    if ((st = pass(q, k, v, dybuf, state_in, nullptr, phi)) != LA_OK) return st;
-    if (la::launch_bwd_norm_gate(dybuf, g, dout, w, dybuf, dg, tokens, HD, mode == LA_OUT_RMSNORM_GATE ? 1 : 0,
-                                 eps, dt, stream) != cudaSuccess)
+    // the forward's raw y (saved by the caller, else recomputed from the same initial
+    // state), then dy and dg
+    const void* yv = y_saved;
+    if (!yv) {
+      if ((st = pass(q, k, v, dybuf, state_in, nullptr, phi)) != LA_OK) return st;
+      yv = dybuf;
+    }
+    if (la::launch_bwd_norm_gate(yv, g, dout, w, dybuf, dg, tokens, HD, mode == LA_OUT_RMSNORM_GATE ? 1 : 0, eps, dt,
+                                 stream) != cudaSuccess)
       return LA_ERR_CUDA;
     dy = dybuf;
   }
@@ -328,31 +336,48 @@ la_status lightning_attn_prefill(const void* q, const void* k, const void* v, co
 }
 
 la_status lightning_attn_backward(const void* q, const void* k, const void* v, const void* g, const void* dout,
-                                  const float* state_in, const float* dstate_out, void* dq, void* dk, void* dv,
-                                  void* dg, float* dstate_in,
+                                  const float* state_in, const float* dstate_out, const void* y, void* dq, void* dk,
+                                  void* dv, void* dg, float* dstate_in,
                                   int B, int T, int H, int D, int block_size, la_dtype dtype, la_feature_map phi,
                                   la_out_mode mode, float eps, const float* norm_weight, void* workspace,
                                   size_t workspace_bytes, la_stream_t stream) {
   if (B < 1 || T < 0) return LA_ERR_INVALID_ARG;
   const int64_t tokens = static_cast<int64_t>(B) * T;
   if (tokens > INT32_MAX) return LA_ERR_UNSUPPORTED;
-  return common_backward(q, k, v, g, dout, state_in, dstate_out, dq, dk, dv, dg, dstate_in, nullptr, B, T, T,
+  return common_backward(q, k, v, g, dout, state_in, dstate_out, y, dq, dk, dv, dg, dstate_in, nullptr, B, T, T,
                          tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight, workspace, workspace_bytes,
                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 la_status lightning_attn_backward_varlen(const void* q, const void* k, const void* v, const void* g,
                                          const void* dout, const float* state_in, const float* dstate_out,
-                                         void* dq, void* dk, void* dv, void* dg, float* dstate_in, const int* cu_seqlens, int num_seqs,
+                                         const void* y, void* dq, void* dk, void* dv, void* dg, float* dstate_in, const int* cu_seqlens, int num_seqs,
                                          int max_seqlen, int total_tokens, int H, int D, int block_size,
                                          la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
                                          const float* norm_weight, void* workspace, size_t workspace_bytes,
                                          la_stream_t stream) {
   if (num_seqs < 1 || !cu_seqlens || !aligned16(cu_seqlens) || total_tokens < 0 || max_seqlen < 0)
     return LA_ERR_INVALID_ARG;
-  return common_backward(q, k, v, g, dout, state_in, dstate_out, dq, dk, dv, dg, dstate_in, cu_seqlens, num_seqs,
+  return common_backward(q, k, v, g, dout, state_in, dstate_out, y, dq, dk, dv, dg, dstate_in, cu_seqlens, num_seqs,
                          0, max_seqlen, total_tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight,
                          workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status lightning_attn_output_transform(const void* y, const void* g, void* out, int tokens, int H, int D,
+                                          la_dtype dtype, la_out_mode mode, float eps, const float* norm_weight,
+                                          la_stream_t stream) {
+  if (tokens < 0 || H < 1 || (D != 64 && D != 128) || static_cast<int64_t>(H) * D > la::kMaxNormWidth)
+    return LA_ERR_INVALID_ARG;
+  if (!valid_enums(dtype, LA_PHI_SILU, mode) || (mode != LA_OUT_RAW && !(eps > 0.0f))) return LA_ERR_INVALID_ARG;
+  if (tokens > 0) {
+    if (!y || !out || !aligned16(y) || !aligned16(out)) return LA_ERR_INVALID_ARG;
+    if (mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g))) return LA_ERR_INVALID_ARG;
+  }
+  if (norm_weight && !aligned16(norm_weight)) return LA_ERR_INVALID_ARG;
+  const cudaError_t e = la::launch_output_transform(y, out, nullptr, g, norm_weight, tokens, H, D,
+                                                    static_cast<int>(mode), eps, dtype,
+                                                    reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
 la_status lightning_attn_chunk_state(const void* k, const void* v, const float* state_in, float* state_out, int B,

@@ -12,7 +12,8 @@
 //   z_den_kernel         z entering the chunk (z0 + earlier chunks), then token by token
 //                        z_t += phi(k_t) and den_t = phi(q_t) . z_t; z_out from the last chunk
 //                        (8 dimensions per lane, the dot product reduced across a lane group)
-//   znorm_transform_kernel  per token: y / den per head, then the output transform, in place
+//   znorm_transform_kernel  per token: y / den per head, then the output transform (in place
+//                        or into another buffer)
 #include "la_common.cuh"
 #include "la_vec.cuh"
 
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(256, 2) z_den_kernel(const T* __restrict__ q, 
 // With den null it is the output transform alone (the prefill's norm when too many heads
 // for the fused exchange).
 template <typename T, int D>
-__global__ void __launch_bounds__(256) znorm_transform_kernel(T* io, const float* __restrict__ den,
+__global__ void __launch_bounds__(256) znorm_transform_kernel(const T* src, T* dst, const float* __restrict__ den,
                                                               const T* __restrict__ g, const float* __restrict__ w,
                                                               int H, int mode, float eps) {
   constexpr int kV = 8;
@@ -182,7 +183,8 @@ __global__ void __launch_bounds__(256) znorm_transform_kernel(T* io, const float
   __shared__ float red[8];
   const int64_t row = blockIdx.x;
   const int HD = H * D;
-  T* y = io + row * HD;
+  const T* y = src + row * HD;   // src and dst may be the same buffer (each element is read
+  T* yo = dst + row * HD;        // by the thread that writes it, after the row's reduction)
   for (int h = threadIdx.x; h < H; h += blockDim.x) rden[h] = den ? 1.0f / den[row * H + h] : 1.0f;
   __syncthreads();
   float r = 1.0f;
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(256) znorm_transform_kernel(T* io, const float
       if (mode == LA_OUT_RMSNORM_GATE) o *= sigmoid_accurate(gv[i]);
       x[i] = o;
     }
-    Vec8<T>::store(y + c, x);
+    Vec8<T>::store(yo + c, x);
   }
 }
 
@@ -255,22 +257,30 @@ cudaError_t launch_znorm_scan(const void* q, const void* k, const float* z_in, f
                                              phi_identity, stream);
 }
 
-cudaError_t launch_znorm_transform(void* io, const float* den, const void* g, const float* w, int64_t tokens, int H,
-                                   int D, int mode, float eps, la_dtype dt, cudaStream_t stream) {
+cudaError_t launch_output_transform(const void* src, void* dst, const float* den, const void* g, const float* w,
+                                    int64_t tokens, int H, int D, int mode, float eps, la_dtype dt,
+                                    cudaStream_t stream) {
   if (tokens == 0) return cudaSuccess;
   const unsigned n = static_cast<unsigned>(tokens);
   if (dt == LA_BF16) {
-    auto* y = static_cast<uint16_t*>(io);
+    auto* a = static_cast<const uint16_t*>(src);
+    auto* b = static_cast<uint16_t*>(dst);
     auto* gg = static_cast<const uint16_t*>(g);
-    if (D == 128) znorm_transform_kernel<uint16_t, 128><<<n, 256, 0, stream>>>(y, den, gg, w, H, mode, eps);
-    else znorm_transform_kernel<uint16_t, 64><<<n, 256, 0, stream>>>(y, den, gg, w, H, mode, eps);
+    if (D == 128) znorm_transform_kernel<uint16_t, 128><<<n, 256, 0, stream>>>(a, b, den, gg, w, H, mode, eps);
+    else znorm_transform_kernel<uint16_t, 64><<<n, 256, 0, stream>>>(a, b, den, gg, w, H, mode, eps);
   } else {
-    auto* y = static_cast<float*>(io);
+    auto* a = static_cast<const float*>(src);
+    auto* b = static_cast<float*>(dst);
     auto* gg = static_cast<const float*>(g);
-    if (D == 128) znorm_transform_kernel<float, 128><<<n, 256, 0, stream>>>(y, den, gg, w, H, mode, eps);
-    else znorm_transform_kernel<float, 64><<<n, 256, 0, stream>>>(y, den, gg, w, H, mode, eps);
+    if (D == 128) znorm_transform_kernel<float, 128><<<n, 256, 0, stream>>>(a, b, den, gg, w, H, mode, eps);
+    else znorm_transform_kernel<float, 64><<<n, 256, 0, stream>>>(a, b, den, gg, w, H, mode, eps);
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_znorm_transform(void* io, const float* den, const void* g, const float* w, int64_t tokens, int H,
+                                   int D, int mode, float eps, la_dtype dt, cudaStream_t stream) {
+  return launch_output_transform(io, io, den, g, w, tokens, H, D, mode, eps, dt, stream);
 }
 
 }  // namespace la

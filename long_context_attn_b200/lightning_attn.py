@@ -37,6 +37,7 @@ EXPORTED = (
     "lightning_attn_mixed_step",
     "lightning_attn_state_prefix",
     "lightning_attn_chunk_state",
+    "lightning_attn_output_transform",
     "lightning_attn_workspace_size",
     "lightning_attn_check",
     "lightning_attn_status_string",
@@ -63,8 +64,9 @@ def _load():
     lib.lightning_attn_prefill_znorm.argtypes = [vp] * 9 + [i32] * 8 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_prefill_znorm_varlen.argtypes = [vp] * 10 + [i32] * 9 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_decode_step_znorm.argtypes = [vp] * 7 + [i32] * 6 + [f32, vp, vp, sz, vp]
-    lib.lightning_attn_backward.argtypes = [vp] * 12 + [i32] * 8 + [f32, vp, vp, sz, vp]
-    lib.lightning_attn_backward_varlen.argtypes = [vp] * 13 + [i32] * 9 + [f32, vp, vp, sz, vp]
+    lib.lightning_attn_backward.argtypes = [vp] * 13 + [i32] * 8 + [f32, vp, vp, sz, vp]
+    lib.lightning_attn_backward_varlen.argtypes = [vp] * 14 + [i32] * 9 + [f32, vp, vp, sz, vp]
+    lib.lightning_attn_output_transform.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]
     lib.lightning_attn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp,
                                                sz, vp]
     lib.lightning_attn_decode_step_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32,
@@ -84,6 +86,7 @@ def _load():
               "lightning_attn_backward_varlen", "lightning_attn_prefill_znorm", "lightning_attn_prefill_znorm_varlen",
               "lightning_attn_decode_step_znorm", "lightning_attn_decode_step",
               "lightning_attn_decode_step_noalloc", "lightning_attn_mixed_step", "lightning_attn_state_prefix", "lightning_attn_chunk_state",
+              "lightning_attn_output_transform",
               "lightning_attn_check"):
         getattr(lib, f).restype = i32
     return lib
@@ -234,13 +237,13 @@ def lightning_attn_decode_step_znorm(q, k, v, g, out, state, z, phi=LA_PHI_SILU,
 
 def lightning_attn_backward(q, k, v, g, dout, dq, dk, dv, dg=None, state_in=None, dstate_in=None, block_size=256,
                             phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE, eps=1e-6, norm_weight=None, workspace=None,
-                            stream=None, dstate_out=None):
+                            stream=None, dstate_out=None, y=None):
     """q, k, v, dq, dk, dv [B, T, H, D]; g, dout, dg [B, T, H*D]; states fp32 [B, H, D, D]
-    (dstate_out: the gradient reaching the final states)."""
+    (dstate_out: the gradient reaching the final states; y: the forward's raw output, saved)."""
     B, T, H, D = q.shape
-    _check_contig(q, k, v, g, dout, dq, dk, dv, dg, dstate_out)
+    _check_contig(q, k, v, g, dout, dq, dk, dv, dg, dstate_out, y)
     st = _lib.lightning_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout), _ptr(_f32_or_none(state_in)),
-                                      _ptr(_f32_or_none(dstate_out)), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+                                      _ptr(_f32_or_none(dstate_out)), _ptr(y), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
                                       _ptr(_f32_or_none(dstate_in)), B, T, H,
                                       D, block_size, _dtype(q), phi, mode, eps, _ptr(_f32_or_none(norm_weight)),
                                       _ptr(workspace), 0 if workspace is None else workspace.numel(),
@@ -251,15 +254,17 @@ def lightning_attn_backward(q, k, v, g, dout, dq, dk, dv, dg=None, state_in=None
 
 def lightning_attn_backward_varlen(q, k, v, g, dout, dq, dk, dv, cu_seqlens, max_seqlen, dg=None, state_in=None,
                                    dstate_in=None, block_size=256, phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE,
-                                   eps=1e-6, norm_weight=None, workspace=None, stream=None, dstate_out=None):
+                                   eps=1e-6, norm_weight=None, workspace=None, stream=None, dstate_out=None,
+                                   y=None):
     """q, k, v, dq, dk, dv [total, H, D]; g, dout, dg [total, H*D]; cu_seqlens int32 device [N + 1]."""
     total, H, D = q.shape
-    _check_contig(q, k, v, g, dout, dq, dk, dv, dg, cu_seqlens, dstate_out)
+    _check_contig(q, k, v, g, dout, dq, dk, dv, dg, cu_seqlens, dstate_out, y)
     if cu_seqlens.dtype != torch.int32:
         raise TypeError("cu_seqlens must be int32")
     n = cu_seqlens.numel() - 1
     st = _lib.lightning_attn_backward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout),
-                                             _ptr(_f32_or_none(state_in)), _ptr(_f32_or_none(dstate_out)), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+                                             _ptr(_f32_or_none(state_in)), _ptr(_f32_or_none(dstate_out)), _ptr(y),
+                                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
                                              _ptr(_f32_or_none(dstate_in)), _ptr(cu_seqlens), n, int(max_seqlen),
                                              total, H, D, block_size, _dtype(q), phi, mode, eps,
                                              _ptr(_f32_or_none(norm_weight)), _ptr(workspace),
@@ -319,6 +324,20 @@ def lightning_attn_mixed_step(q, k, v, g, out, cu_seqlens, cu_seqlens_host, stat
                                         _stream(decode_stream))
     if st != LA_OK:
         raise LightningAttnError(st, "lightning_attn_mixed_step")
+
+
+def lightning_attn_output_transform(y, g, out, mode=LA_OUT_RMSNORM_GATE, eps=1e-6, norm_weight=None, stream=None):
+    """out = RMSNorm(y) * w (* sigmoid(g)) per token: y, g, out [..., H*D] with H*D the last axis;
+    H and D from y's last two dims when y is [..., H, D], else pass y as [tokens, H, D]."""
+    if y.dim() < 2:
+        raise ValueError("y must be [..., H, D]")
+    H, D = y.shape[-2], y.shape[-1]
+    tokens = y.numel() // (H * D)
+    _check_contig(y, g, out)
+    st = _lib.lightning_attn_output_transform(_ptr(y), _ptr(g), _ptr(out), tokens, H, D, _dtype(y), mode, eps,
+                                              _ptr(_f32_or_none(norm_weight)), _stream(stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_output_transform")
 
 
 def lightning_attn_chunk_state(k, v, state_out, state_in=None, phi=LA_PHI_SILU, workspace=None, stream=None):

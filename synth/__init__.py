@@ -115,7 +115,7 @@ def f32_to_bf16(a: np.ndarray) -> np.ndarray:
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str              # 'prefill' | 'varlen' | 'decode' | 'mixed' | 'backward' | 'znorm' | 'chunk_state'
+    kind: str              # prefill varlen decode mixed backward train znorm chunk_state
     seed: int
     B: int                 # batch (prefill), number of sequences (varlen / decode)
     T: int                 # tokens per sequence (prefill); 0 otherwise
@@ -153,6 +153,8 @@ WORKLOADS = {
     # denominators phi(q) . z stay positive.
     "znorm_128k": Workload("znorm_128k", "znorm", 1009, 1, 131072, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5,
                            qk_shift=1.0),
+    # A training step on the 128K prefill's shapes: forward (keeping y) and backward.
+    "train_128k": Workload("train_128k", "train", 1011, 1, 131072, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5),
     # Step 1 of the sequence-parallel prefill on the 128K prefill's shapes: the state from k, v.
     "chunk_state_128k": Workload("chunk_state_128k", "chunk_state", 1010, 1, 131072, 64, 128, 0, "bf16", "raw", 0.5),
 }

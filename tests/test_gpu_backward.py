@@ -189,3 +189,39 @@ def test_backward_128k_full_size_samples(cuda_device):
                            mode=oracle.MODE_RAW)
     assert_close(got_k[None], tail[1], "bf16", "dk (last 4096 tokens)")
     assert_close(got_v[None], tail[2], "bf16", "dv (last 4096 tokens)")
+
+
+@pytest.mark.parametrize("mode", ["rmsnorm", "rmsnorm_gate"])
+def test_backward_with_saved_y_equals_recompute(mode, cuda_device):
+    """Passing the forward's raw output y (prefill in raw mode) gives the same gradients as
+    letting the backward recompute it (the same kernel computes y either way)."""
+    import torch
+    la = _la()
+    m = mode_code(mode)
+    B, T, H, D, C = 1, 600, 8, 128, 256
+    q, k, v, g = synth.prefill_inputs(3901, T, H, D, "bf16", 0.5, True)
+    dout = synth.normal(3901, 21, (T, H * D), 1.0, "bf16")
+    shp, gshp = (B, T, H, D), (B, T, H * D)
+    dq_, dk_, dv_ = (to_dev(a).reshape(shp) for a in (q, k, v))
+    dg_, ddo = to_dev(g).reshape(gshp), to_dev(dout).reshape(gshp)
+    gate = dg_ if m == la.LA_OUT_RMSNORM_GATE else None
+    y = torch.empty(gshp, dtype=torch.bfloat16, device="cuda")
+    ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD, B, T, 0, H, D, C, la.LA_BF16, m))
+    la.lightning_attn_prefill(dq_, dk_, dv_, None, y, None, None, block_size=C, mode=la.LA_OUT_RAW, workspace=ws)
+    res = []
+    for yy in (None, y):
+        gq, gk, gv = (torch.empty_like(dq_) for _ in range(3))
+        gg = torch.empty_like(dg_) if gate is not None else None
+        la.lightning_attn_backward(dq_, dk_, dv_, gate, ddo, gq, gk, gv, dg=gg, block_size=C, mode=m, workspace=ws,
+                                   y=yy)
+        la.lightning_attn_check(ws)
+        res.append([to_host(t) for t in (gq, gk, gv) + ((gg,) if gg is not None else ())])
+    for a, b in zip(*res):
+        np.testing.assert_array_equal(a, b)
+    # and the output transform of the kept y is the fused forward's output (tolerance: y is
+    # rounded to bf16 before the norm here, the fused kernel normalises fp32 y)
+    out = torch.empty(gshp, dtype=torch.bfloat16, device="cuda")
+    la.lightning_attn_output_transform(y.view(B, T, H, D), gate, out, mode=m)
+    ref, _, _ = oracle.prefill(q.reshape(shp), k.reshape(shp), v.reshape(shp),
+                               g.reshape(gshp) if gate is not None else None, mode=m)
+    assert_close(to_host(out), ref, "bf16")

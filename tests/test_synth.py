@@ -56,6 +56,7 @@ def test_workload_table():
     assert w["backward_128k"].seed == 1007 and w["backward_8k"].seed == 1008 and w["backward_8k"].T == 8192
     assert w["znorm_128k"].seed == 1009 and w["znorm_128k"].qk_shift == 1.0
     assert w["chunk_state_128k"].seed == 1010 and w["chunk_state_128k"].kind == "chunk_state"
+    assert w["train_128k"].seed == 1011 and w["train_128k"].kind == "train"
     a = synth.normal(7, 0, (1000,), 0.5, "bf16")
     b = synth.shifted(a, 1.0)
     assert b.dtype == np.uint16 and np.allclose(synth.bf16_to_f32(b), synth.bf16_to_f32(a) + 1.0, atol=2 ** -7)
