@@ -168,3 +168,19 @@ def test_chunk_state_workspace_and_checks(lib):
     assert f(fake, fake, None, fake, 1, 64, 2, 96, 1, 0, ws, 1 << 30, None) == 1        # D
     assert f(fake, vp(0x1008), None, fake, 1, 64, 2, 128, 1, 0, ws, 1 << 30, None) == 1  # alignment
     assert f(fake, fake, None, fake, 1, 64, 2, 128, 1, 0, ws, 16, None) == 1            # workspace too small
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """The header compiles as C11 (no C++ in it) and every entry point it declares links
+    against the built library from a C program (compiled and linked with gcc, not run)."""
+    import subprocess
+    names = sorted(_declared())
+    src = tmp_path / "use_abi.c"
+    body = "\n".join(f"  (void *)&{n}," for n in names)
+    src.write_text('#include "lightning_attn.h"\n#include <stdio.h>\n'
+                   f"static void *const entry[] = {{\n{body}\n}};\n"
+                   "int main(void) { printf(\"%d\\n\", (int)(sizeof(entry) / sizeof(entry[0]))); return 0; }\n")
+    so = os.path.join(ROOT, "long_context_attn_b200", "liblightning_attn.so")
+    r = subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", HEADER_DIR, str(src), so,
+                        "-o", str(tmp_path / "use_abi")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
