@@ -30,6 +30,10 @@ cudaError_t launch_bwd_prep(const void* q, const void* k, const void* v, const v
 cudaError_t launch_bwd_post(const void* q, const void* k, void* dq, void* dk, void* dv, const int* cu, int nseq,
                             int T_fixed, int64_t tokens, int HD, int phi_identity, la_dtype dt, cudaStream_t stream);
 cudaError_t launch_transpose_states(const float* in, float* out, int64_t nmat, int D, cudaStream_t stream);
+cudaError_t launch_bwd_feat(const void* q, const void* k, void* fq, void* fk, int64_t elems, int phi_identity,
+                            la_dtype dt, cudaStream_t stream);
+cudaError_t launch_bwd_scale(const void* q, const void* k, void* dq, void* dk, int64_t elems, la_dtype dt,
+                             cudaStream_t stream);
 int znorm_max_chunks(int max_len);
 int chunk_state_splits(int nseq, int H, int max_len, int num_sms);
 cudaError_t launch_chunk_state_tc(const void* k, const void* v, const float* state_in, float* state_out,
@@ -106,7 +110,7 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
                          const float* state_in, float* state_out, const int* cu, int nseq, int T_fixed,
                          int max_len, int64_t tokens, int H, int D, int C, la_dtype dt, la_feature_map phi,
                          la_out_mode mode, float eps, const float* w, void* workspace, size_t ws_bytes,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, bool reverse = false) {
   if (!valid_enums(dt, phi, mode) || !valid_head(H, D, mode, eps)) return LA_ERR_INVALID_ARG;
   if (C < 1 || C > 1024 || nseq < 1 || tokens < 0 || max_len < 0) return LA_ERR_INVALID_ARG;
   if (tokens > 0) {
@@ -120,6 +124,7 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
   if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;
 
   const Path path = choose_path(dt, H, D, C, mode);
+  if (reverse && (path != Path::kTc || mode != LA_OUT_RAW)) return LA_ERR_UNSUPPORTED;   // internal use only
   if (ws_bytes < prefill_ws_bytes(path, nseq, max_len, tokens, H, D, C, mode)) return LA_ERR_INVALID_ARG;
   la::ErrRec* err = static_cast<la::ErrRec*>(workspace);
   char* ws = static_cast<char*>(workspace) + kErrBytes;
@@ -134,6 +139,7 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
     a.H = H; a.D = D; a.C = C; a.phi_identity = phi_id;
     a.mode = static_cast<int>(split ? LA_OUT_RAW : mode);
     a.eps = eps; a.w = split ? nullptr : w; a.err = err; a.ws = ws;
+    a.reverse = reverse ? 1 : 0;
     e = la::launch_tc_prefill(a, current_sm_count(), stream);
     if (e == cudaSuccess && split)   // the norm (and gate) per token, over the raw output in place
       e = la::launch_znorm_transform(out, nullptr, g, w, tokens, H, D, static_cast<int>(mode), eps, dt, stream);
@@ -163,17 +169,24 @@ MixedLayout mixed_layout(int n, int max_pre, int64_t total, int H, int D, int C,
   return m;
 }
 
-// Backward workspace: [prefill part of the raw-mode passes (error record first)]
-// [6 token buffers: dy, phi(k), rho(v), rho(dy), rho(phi(q)), rho(phi(k))] [S0^T] [dS_T^T].
+// Backward workspace: [prefill part of the raw-mode passes (error record first)] [token
+// buffers] [S0^T] [dS_T^T].  The token buffers are dy, phi(k), phi(q) when the tensor-core
+// kernel walks time backwards itself (rev), else dy, phi(k), rho(v), rho(dy), rho(phi(q)),
+// rho(phi(k)) (rho: each sequence reversed).
 struct BwdLayout {
+  bool rev;
+  int nbuf;
   size_t pre, buf, st, total;
 };
 BwdLayout bwd_layout(int nseq, int max_len, int64_t tokens, int H, int D, int C, la_dtype dt) {
   BwdLayout b{};
-  b.pre = prefill_ws_bytes(choose_path(dt, H, D, C, LA_OUT_RAW), nseq, max_len, tokens, H, D, C, LA_OUT_RAW);
+  const Path raw = choose_path(dt, H, D, C, LA_OUT_RAW);
+  b.rev = raw == Path::kTc;
+  b.nbuf = b.rev ? 3 : 6;
+  b.pre = prefill_ws_bytes(raw, nseq, max_len, tokens, H, D, C, LA_OUT_RAW);
   b.buf = up256(static_cast<size_t>(tokens) * H * D * (dt == LA_BF16 ? 2 : 4));
   b.st = up256(sizeof(float) * static_cast<size_t>(nseq) * H * D * D);
-  b.total = b.pre + 6 * b.buf + 2 * b.st;
+  b.total = b.pre + b.nbuf * b.buf + 2 * b.st;
   return b;
 }
 
@@ -202,17 +215,18 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
   if (ws_bytes < L.total) return LA_ERR_INVALID_ARG;
 
   char* base = static_cast<char*>(workspace);
-  void* buf[6];
-  for (int i = 0; i < 6; ++i) buf[i] = base + L.pre + i * L.buf;
-  float* s0t = reinterpret_cast<float*>(base + L.pre + 6 * L.buf);
-  float* dstt = reinterpret_cast<float*>(base + L.pre + 6 * L.buf + L.st);
+  void* buf[6] = {};
+  for (int i = 0; i < L.nbuf; ++i) buf[i] = base + L.pre + i * L.buf;
+  float* s0t = reinterpret_cast<float*>(base + L.pre + L.nbuf * L.buf);
+  float* dstt = reinterpret_cast<float*>(base + L.pre + L.nbuf * L.buf + L.st);
   void *dybuf = buf[0], *fk = buf[1], *rv = buf[2], *rdy = buf[3], *rfq = buf[4], *rfk = buf[5];
+  void* fq = buf[2];   // the reverse-time composition's third buffer
   const int HD = H * D;
   const int phi_id = (phi == LA_PHI_IDENTITY) ? 1 : 0;
   auto pass = [&](const void* qq, const void* kk, const void* vv, void* out, const float* sin,
-                  float* sout, la_feature_map f) {
+                  float* sout, la_feature_map f, bool rev = false) {
     return common_prefill(qq, kk, vv, nullptr, out, sin, sout, cu, nseq, T_fixed, max_len, tokens, H, D, C, dt, f,
-                          LA_OUT_RAW, eps, nullptr, workspace, L.pre, stream);
+                          LA_OUT_RAW, eps, nullptr, workspace, L.pre, stream, rev);
   };
   la_status st;
   const void* dy = dout;
@@ -229,17 +243,12 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
       return LA_ERR_CUDA;
     dy = dybuf;
   }
-  if (la::launch_bwd_prep(q, k, v, dy, fk, rv, rdy, rfq, rfk, cu, nseq, T_fixed, tokens, HD, phi_id, dt, stream) !=
-      cudaSuccess)
-    return LA_ERR_CUDA;
   const float* s0 = nullptr;
   if (state_in) {
     if (la::launch_transpose_states(state_in, s0t, static_cast<int64_t>(nseq) * H, D, stream) != cudaSuccess)
       return LA_ERR_CUDA;
     s0 = s0t;
   }
-  // dphi(q): queries dy, keys v, values phi(k), initial state S0^T
-  if ((st = pass(dy, v, fk, dq, s0, nullptr, LA_PHI_IDENTITY)) != LA_OK) return st;
   // A gradient reaching the final state starts the reverse sums: dphi(k) gets dS_T v, dv gets
   // dS_T^T phi(k), dS0 includes dS_T.
   const float* dsT_t = nullptr;
@@ -248,6 +257,24 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
       return LA_ERR_CUDA;
     dsT_t = dstt;
   }
+  if (L.rev) {
+    // The tensor-core kernel walks time backwards itself: no reversed copies.
+    if (la::launch_bwd_feat(q, k, fq, fk, tokens * HD, phi_id, dt, stream) != cudaSuccess) return LA_ERR_CUDA;
+    // dphi(q): queries dy, keys v, values phi(k), initial state S0^T, forward in time
+    if ((st = pass(dy, v, fk, dq, s0, nullptr, LA_PHI_IDENTITY)) != LA_OK) return st;
+    // dphi(k): queries v, keys dy, values phi(q), initial state dS_T^T, backward in time
+    if ((st = pass(v, dy, fq, dk, dsT_t, nullptr, LA_PHI_IDENTITY, true)) != LA_OK) return st;
+    // dv: queries phi(k), keys phi(q) (the kernel's feature map on the raw k and q), values
+    // dy, initial state dS_T, backward in time; its final state is dS0
+    if ((st = pass(k, q, dy, dv, dstate_out, dstate, phi, true)) != LA_OK) return st;
+    if (!phi_id && la::launch_bwd_scale(q, k, dq, dk, tokens * HD, dt, stream) != cudaSuccess) return LA_ERR_CUDA;
+    return LA_OK;
+  }
+  if (la::launch_bwd_prep(q, k, v, dy, fk, rv, rdy, rfq, rfk, cu, nseq, T_fixed, tokens, HD, phi_id, dt, stream) !=
+      cudaSuccess)
+    return LA_ERR_CUDA;
+  // dphi(q): queries dy, keys v, values phi(k), initial state S0^T
+  if ((st = pass(dy, v, fk, dq, s0, nullptr, LA_PHI_IDENTITY)) != LA_OK) return st;
   // reversed dphi(k): queries rho(v), keys rho(dy), values rho(phi(q)), initial state dS_T^T
   if ((st = pass(rv, rdy, rfq, dk, dsT_t, nullptr, LA_PHI_IDENTITY)) != LA_OK) return st;
   // reversed dv: queries rho(phi(k)), keys rho(phi(q)), values rho(dy), initial state dS_T;

@@ -18,6 +18,10 @@
 //   bwd_prep_kernel       phi(k) and the reversed copies rho(v), rho(dy), rho(phi(q)), rho(phi(k))
 //   bwd_post_kernel       dq = dphi(q) * phi'(q); un-reverses dk (times phi'(k)) and dv in place
 //   transpose_states      S0^T for the first pass
+// When the prefill kernel can walk time backwards itself (the tensor-core path), the
+// reversed copies are not needed: bwd_feat_kernel writes phi(q) and phi(k), the last two
+// passes run in reverse time (the third taking phi on the raw k and q in the kernel), and
+// bwd_scale_kernel multiplies dq and dk by phi'.
 // All of them are HBM-streaming kernels: 16-byte vectors, grid-stride loops over rows.
 #include "la_common.cuh"
 #include "la_vec.cuh"
@@ -190,6 +194,46 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const T* __restrict__ q, 
   }
 }
 
+// Reverse-time composition (the prefill kernel walks time backwards itself): phi(q) and
+// phi(k) in place of the reversed copies, 16-byte vectors.
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_feat_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                       T* __restrict__ fq, T* __restrict__ fk, int64_t n8,
+                                                       int phi_identity) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float a[kVec];
+    Vec8<T>::load(q + i * kVec, a);
+#pragma unroll
+    for (int j = 0; j < kVec; ++j) a[j] = feature(a[j], phi_identity);
+    Vec8<T>::store(fq + i * kVec, a);
+    Vec8<T>::load(k + i * kVec, a);
+#pragma unroll
+    for (int j = 0; j < kVec; ++j) a[j] = feature(a[j], phi_identity);
+    Vec8<T>::store(fk + i * kVec, a);
+  }
+}
+
+// ... and its finish: dq *= phi'(q), dk *= phi'(k), in place (dv needs nothing).
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_scale_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                        T* __restrict__ dq, T* __restrict__ dk, int64_t n8) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float x[kVec], d[kVec];
+    Vec8<T>::load(q + i * kVec, x);
+    Vec8<T>::load(dq + i * kVec, d);
+#pragma unroll
+    for (int j = 0; j < kVec; ++j) d[j] *= dfeature(x[j], 0);
+    Vec8<T>::store(dq + i * kVec, d);
+    Vec8<T>::load(k + i * kVec, x);
+    Vec8<T>::load(dk + i * kVec, d);
+#pragma unroll
+    for (int j = 0; j < kVec; ++j) d[j] *= dfeature(x[j], 0);
+    Vec8<T>::store(dk + i * kVec, d);
+  }
+}
+
 __global__ void __launch_bounds__(256) transpose_states_kernel(const float* __restrict__ in, float* __restrict__ out,
                                                                int64_t nmat, int D) {
   const int64_t n = nmat * D * D;
@@ -257,6 +301,36 @@ cudaError_t launch_bwd_post(const void* q, const void* k, void* dq, void* dk, vo
     bwd_post_kernel<float><<<grid_for(n), 256, 0, stream>>>(
         static_cast<const float*>(q), static_cast<const float*>(k), static_cast<float*>(dq),
         static_cast<float*>(dk), static_cast<float*>(dv), cu, nseq, T_fixed, tokens, HD, phi_identity);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_feat(const void* q, const void* k, void* fq, void* fk, int64_t elems, int phi_identity,
+                            la_dtype dt, cudaStream_t stream) {
+  const int64_t n8 = elems / kVec;
+  if (n8 == 0) return cudaSuccess;
+  if (dt == LA_BF16)
+    bwd_feat_kernel<uint16_t><<<grid_for(n8), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<uint16_t*>(fq),
+        static_cast<uint16_t*>(fk), n8, phi_identity);
+  else
+    bwd_feat_kernel<float><<<grid_for(n8), 256, 0, stream>>>(static_cast<const float*>(q),
+                                                             static_cast<const float*>(k), static_cast<float*>(fq),
+                                                             static_cast<float*>(fk), n8, phi_identity);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_scale(const void* q, const void* k, void* dq, void* dk, int64_t elems, la_dtype dt,
+                             cudaStream_t stream) {
+  const int64_t n8 = elems / kVec;
+  if (n8 == 0) return cudaSuccess;
+  if (dt == LA_BF16)
+    bwd_scale_kernel<uint16_t><<<grid_for(n8), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<uint16_t*>(dq),
+        static_cast<uint16_t*>(dk), n8);
+  else
+    bwd_scale_kernel<float><<<grid_for(n8), 256, 0, stream>>>(static_cast<const float*>(q),
+                                                              static_cast<const float*>(k), static_cast<float*>(dq),
+                                                              static_cast<float*>(dk), n8);
   return cudaGetLastError();
 }
 

@@ -46,6 +46,11 @@
 //    store each row's 128 bytes straight from registers.
 //  * Every wait is bounded (globaltimer); a wait that runs out records LA_ERR_TIMEOUT in
 //    the workspace and the CTA drains its async work, frees TMEM and exits.
+//  * Reverse time (raw mode, for the backward's sums over t >= i): each sequence's
+//    128-row tiles are walked from the last to the first and the diagonal tile keeps the
+//    keys at or after the query row.  The rows inside a tile keep their order, so the
+//    partial tile (now the first one walked) has its valid rows on top as before, and the
+//    block pairs simply start at the sequence end.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -207,8 +212,6 @@ __device__ __forceinline__ void tile_first(const TcParams& p, TileIter& it) {
   tile_next(p, it);
 }
 
-__device__ __forceinline__ bool aborted(Bars& B) { return *reinterpret_cast<volatile int*>(&B.abort_flag) != 0; }
-
 // Bounded wait for phase `parity` of an mbarrier.  Returns false (after recording a
 // timeout, or because another role already did) when the CTA is aborting.  The polling
 // loop is out of line: only the first test is inlined at each of the many wait sites,
@@ -325,7 +328,7 @@ __device__ __forceinline__ void red_add_f64(double* p, double v) {
 // ======================================================================================
 // One instantiation per output mode (la_out_mode) and block size (128 or 256 rows), so
 // that each variant's roles compile to straight-line code.
-template <int kMode, int kC>
+template <int kMode, int kC, bool kRev>
 __global__ void __launch_bounds__(kThreads, 1)
 lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -345,7 +348,11 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   constexpr int tpb = kC / kTile;        // tiles per block (1 or 2)
   constexpr bool norm = kMode != LA_OUT_RAW;
   constexpr bool gate = kMode == LA_OUT_RMSNORM_GATE;
+  static_assert(!kRev || kMode == LA_OUT_RAW, "reverse time is a raw-mode variant");
   const int W = p.H * kNdv * 4;          // reader warps contributing to one tile's norm
+  // Tile i of a sequence's processing order is physical tile i, or nt - 1 - i when time
+  // runs backwards (kRev: the sequence is walked from its end; see the header comment).
+  auto phys = [](int i, int nt) { return kRev ? nt - 1 - i : i; };
 
   if (tid == 0) {
     for (int i = 0; i < kNKV; ++i) {
@@ -420,7 +427,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             ok = false;
             break;
           }
-          const int32_t row = static_cast<int32_t>(row0 + static_cast<int64_t>(i) * kTile);
+          const int32_t row = static_cast<int32_t>(row0 + static_cast<int64_t>(phys(i, nt)) * kTile);
           if (is_q) {
             mbar_arrive_expect_tx(&B.full_q[sl], kBoxBytes);
             tma_load_2d(smem + OFF_Q + sl * kQBytes + dvt * kBoxBytes, &tm_q, h * kD + dvt * 64, row, &B.full_q[sl],
@@ -484,7 +491,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
           tc_fence_after();
         }
         const int u = it.i % tpb;
-        const int vr = min(kTile, it.L - it.i * kTile);
+        const int vr = min(kTile, it.L - phys(it.i, it.nt) * kTile);
         const uint32_t n = (kt == u) ? static_cast<uint32_t>(pad_rows(vr)) : 128u;
         const uint64_t qd = desc_at(kDescK, sbase + OFF_Q + (tt % kNQ) * kQBytes);
         const uint64_t kd = desc_at(kDescK, sbase + OFF_K + kv_slot(tt, u, kt) * kKBytes);
@@ -503,7 +510,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         const int u = cur.i % tpb;
         const int qs = t % kNQ, ks = t % kNKV;
         const int ob = t & 1;
-        const int vr = min(kTile, cur.L - cur.i * kTile);
+        const int vr = min(kTile, cur.L - phys(cur.i, cur.nt) * kTile);
         const int nk = pad_rows(vr);
         const uint32_t k0 = k;
         if (kp == k0) {  // P of this tile's first job was not issued ahead
@@ -625,7 +632,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     // Keys (and the zeroed tail of the values) of tile tt.
     auto xf_keys = [&](const TileIter& it, int tt) {
       const int ks = tt % kNKV;
-      const int vr = min(kTile, it.L - it.i * kTile);
+      const int vr = min(kTile, it.L - phys(it.i, it.nt) * kTile);
       xf_box(OFF_K + ks * kKBytes + dvt * kBoxBytes, vr);
       if (vr < kTile) {
         const uint32_t va = sbase + OFF_V + ks * kVBytes;
@@ -678,7 +685,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       const int nt = (L + kTile - 1) / kTile;
       for (int i = 0; i < nt && ok; ++i) {
         const int u = i % tpb;
-        const int vr = min(kTile, L - i * kTile);
+        const int vr = min(kTile, L - phys(i, nt) * kTile);
         const int nk = pad_rows(vr);
         for (int kt = 0; kt <= u; ++kt, ++k) {
           const uint32_t r = k & 1u;
@@ -696,9 +703,9 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             for (int e = 0; e < 16; ++e) {
               const int j = 32 * c + 2 * e;
               float a = __uint_as_float(x[2 * e]), b = __uint_as_float(x[2 * e + 1]);
-              if (diag) {
-                a = (j <= wt) ? a : 0.f;
-                b = (j + 1 <= wt) ? b : 0.f;
+              if (diag) {   // keys up to the query row; from it on when time runs backwards
+                a = (kRev ? j >= wt : j <= wt) ? a : 0.f;
+                b = (kRev ? j + 1 >= wt : j + 1 <= wt) ? b : 0.f;
               }
               pk[e] = pack_bf16x2(a, b);
             }
@@ -769,8 +776,8 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
         const int ob = t & 1;
         const int zs = t & 1;
         const int u = i % tpb;
-        const int vr = min(kTile, L - i * kTile);
-        const int64_t row = row0 + static_cast<int64_t>(i) * kTile;
+        const int vr = min(kTile, L - phys(i, nt) * kTile);
+        const int64_t row = row0 + static_cast<int64_t>(phys(i, nt)) * kTile;
         if (!wait_bar_warp(&B.o_full[ob], (t >> 1) & 1, B, p, SITE_TC_EPILOGUE, t)) { ok = false; break; }
         if (norm && t >= 2 && !wait_bar_warp(&B.z_free[zs][q], ((t >> 1) - 1) & 1, B, p, SITE_TC_EPILOGUE, t)) {
           ok = false;
@@ -891,9 +898,9 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       const int nt = (L + kTile - 1) / kTile;
       for (int i = 0; i < nt; ++i, ++t) {
         const int zs = t & 1;
-        const int vr = min(kTile, L - i * kTile);
+        const int vr = min(kTile, L - phys(i, nt) * kTile);
         const int r = kQuarterRows * q + lane;     // row of the tile
-        const int64_t row = row0 + static_cast<int64_t>(i) * kTile;
+        const int64_t row = row0 + static_cast<int64_t>(phys(i, nt)) * kTile;
         // This row's 64 gate values (bf16 pairs), loaded before the waits so that their
         // latency overlaps them; the producer has prefetched the tile into L2.
         uint32_t gq[32];
@@ -1000,7 +1007,7 @@ int max_active_clusters() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   std::lock_guard<std::mutex> lock(mu);
   if (cache[dev] == 0) {
-    if (cudaFuncSetAttribute(lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 256>,
+    if (cudaFuncSetAttribute(lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 256, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess)
       return 0;
@@ -1016,7 +1023,7 @@ int max_active_clusters() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 256>, &cfg) !=
+    if (cudaOccupancyMaxActiveClusters(&n, lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 256, false>, &cfg) !=
         cudaSuccess)
       n = -1;
     cache[dev] = n;
@@ -1083,10 +1090,18 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
   if (e != cudaSuccess) return e;
   using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, TcParams);
   static const Kernel kernels[3][2] = {
-      {lightning_prefill_tc_kernel<LA_OUT_RAW, 128>, lightning_prefill_tc_kernel<LA_OUT_RAW, 256>},
-      {lightning_prefill_tc_kernel<LA_OUT_RMSNORM, 128>, lightning_prefill_tc_kernel<LA_OUT_RMSNORM, 256>},
-      {lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 128>, lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 256>}};
-  const Kernel kernel = kernels[a.mode == LA_OUT_RAW ? 0 : (a.mode == LA_OUT_RMSNORM ? 1 : 2)][a.C == 256 ? 1 : 0];
+      {lightning_prefill_tc_kernel<LA_OUT_RAW, 128, false>, lightning_prefill_tc_kernel<LA_OUT_RAW, 256, false>},
+      {lightning_prefill_tc_kernel<LA_OUT_RMSNORM, 128, false>,
+       lightning_prefill_tc_kernel<LA_OUT_RMSNORM, 256, false>},
+      {lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 128, false>,
+       lightning_prefill_tc_kernel<LA_OUT_RMSNORM_GATE, 256, false>}};
+  // Time running backwards (raw mode only): the backward's reverse-time passes.
+  static const Kernel kernels_rev[2] = {lightning_prefill_tc_kernel<LA_OUT_RAW, 128, true>,
+                                        lightning_prefill_tc_kernel<LA_OUT_RAW, 256, true>};
+  if (a.reverse && a.mode != LA_OUT_RAW) return cudaErrorInvalidValue;
+  const Kernel kernel = a.reverse ? kernels_rev[a.C == 256 ? 1 : 0]
+                                  : kernels[a.mode == LA_OUT_RAW ? 0 : (a.mode == LA_OUT_RMSNORM ? 1 : 2)]
+                                           [a.C == 256 ? 1 : 0];
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};

@@ -23,6 +23,7 @@ struct TcArgs {
   int nseq, T, max_len;
   int64_t tokens;
   int H, D, C, phi_identity, mode;
+  int reverse;         // nonzero: time runs backwards (raw mode only)
   float eps;
   const float* w;
   ErrRec* err;
