@@ -31,13 +31,16 @@ namespace {
 
 constexpr int kVec = 8;   // elements per vector (16 bytes of bf16)
 
-__device__ __forceinline__ float feature(float x, int phi_identity) {
-  return phi_identity ? x : silu_accurate(x);
-}
+// sigmoid(x) = 1 / (1 + e^-x) from the CUDA fast intrinsics (__expf, __fdividef: a few ulp;
+// the exponent is clamped so the divisor stays below 2^126).  These streaming kernels
+// evaluate it once or twice per element; the accurate form (expf and an IEEE division)
+// left them instruction-bound below the HBM rate.
+__device__ __forceinline__ float sig(float x) { return __fdividef(1.0f, 1.0f + __expf(fminf(-x, 80.0f))); }
+__device__ __forceinline__ float feature(float x, int phi_identity) { return phi_identity ? x : x * sig(x); }
 // d/dx [x sigmoid(x)] = sigmoid(x) (1 + x (1 - sigmoid(x)))
 __device__ __forceinline__ float dfeature(float x, int phi_identity) {
   if (phi_identity) return 1.0f;
-  const float s = sigmoid_accurate(x);
+  const float s = sig(x);
   return s * (1.0f + x * (1.0f - s));
 }
 
@@ -77,7 +80,7 @@ __global__ void __launch_bounds__(256) bwd_norm_gate_kernel(const T* y, const T*
     if (gate) Vec8<T>::load(g + base + c, gv);
 #pragma unroll
     for (int i = 0; i < kVec; ++i) {
-      const float s = gate ? sigmoid_accurate(gv[i]) : 1.0f;
+      const float s = gate ? sig(gv[i]) : 1.0f;
       const float u = dv[i] * (w ? __ldg(w + c + i) : 1.0f) * s;
       ss = fmaf(yv[i], yv[i], ss);
       su = fmaf(u, yv[i], su);
@@ -102,7 +105,7 @@ __global__ void __launch_bounds__(256) bwd_norm_gate_kernel(const T* y, const T*
     if (gate) Vec8<T>::load(g + base + c, gv);
 #pragma unroll
     for (int i = 0; i < kVec; ++i) {
-      const float s = gate ? sigmoid_accurate(gv[i]) : 1.0f;
+      const float s = gate ? sig(gv[i]) : 1.0f;
       const float wc = w ? __ldg(w + c + i) : 1.0f;
       o[i] = r * dv[i] * wc * s - coef * yv[i];
       og[i] = dv[i] * yv[i] * r * wc * s * (1.0f - s);

@@ -173,7 +173,8 @@ __global__ void __launch_bounds__(256, 2) z_den_kernel(const T* __restrict__ q, 
 // One CTA per token: y / den per head, then RAW / RMSNORM / RMSNORM_GATE, in place on io.
 // 8-element vectors; the H reciprocals of the token's denominators sit in shared memory.
 // With den null it is the output transform alone (the prefill's norm when too many heads
-// for the fused exchange).
+// for the fused exchange).  sigmoid(g) from the fast intrinsics (a few ulp, exponent
+// clamped), as in the scan.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) znorm_transform_kernel(const T* src, T* dst, const float* __restrict__ den,
                                                               const T* __restrict__ g, const float* __restrict__ w,
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(256) znorm_transform_kernel(const T* src, T* d
     for (int i = 0; i < kV; ++i) {
       float o = x[i] * s;
       if (mode != LA_OUT_RAW && w) o *= __ldg(w + c + i);
-      if (mode == LA_OUT_RMSNORM_GATE) o *= sigmoid_accurate(gv[i]);
+      if (mode == LA_OUT_RMSNORM_GATE) o *= __fdividef(1.0f, 1.0f + __expf(fminf(-gv[i], 80.0f)));
       x[i] = o;
     }
     Vec8<T>::store(yo + c, x);
