@@ -9,8 +9,9 @@
 // followed by o = RMSNorm over the H*D head concatenation of a token times sigmoid(g).
 //
 // Design (B200, sm_100a):
-//  * One CTA owns one (head, 64-column slice of d_v) chain and walks all sequences.  With
-//    H = 64 that is 128 CTAs, one per SM, all resident at once.
+//  * One CTA owns one (head, 64-column slice of d_v) chain and walks all sequences of its
+//    group.  With H = 64 that is 128 CTAs, one per SM, all resident at once, and one group;
+//    with fewer heads several groups of CTA pairs split the sequences between them.
 //  * Work is tiled in 128-row tiles (the tcgen05 M).  C = 256 is two tiles per block: the
 //    second tile multiplies by the first tile's keys densely and by its own keys under the
 //    causal mask; the all-zero upper-right quarter of the 256 x 256 block is never issued.
@@ -53,6 +54,7 @@
 //    block pairs simply start at the sequence end.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "la_common.cuh"
@@ -125,6 +127,7 @@ struct TcParams {
   uint16_t* out;
   const int* state_index;  // optional [nseq]: state slot of each sequence (else the index)
   int skip_single;         // nonzero: one-token sequences belong to a decode step: skip them
+  int ngroups;             // sequence groups: the CTA pairs of group g take sequences g, g + G, ...
 };
 
 // Shared-memory descriptor templates with start address 0; an operand at shared address a
@@ -173,7 +176,8 @@ __device__ __forceinline__ bool seq_range(const TcParams& p, int s, int64_t& row
   return false;
 }
 
-// The (sequence, tile) order every role walks; empty sequences have no tiles.
+// The (sequence, tile) order every role walks: this CTA's group's sequences (every
+// p.ngroups-th from its group index), empty sequences have no tiles.
 struct TileIter {
   int s, i, nt, L;
   int64_t row0;
@@ -184,7 +188,7 @@ __device__ __forceinline__ void tile_next(const TcParams& p, TileIter& it) {
     ++it.i;
     return;
   }
-  for (int s = it.s + 1; s < p.nseq; ++s) {
+  for (int s = it.s + p.ngroups; s < p.nseq; s += p.ngroups) {
     int64_t r0;
     int L;
     seq_range(p, s, r0, L);
@@ -202,8 +206,8 @@ __device__ __forceinline__ void tile_next(const TcParams& p, TileIter& it) {
   it.s = p.nseq;
   it.valid = false;
 }
-__device__ __forceinline__ void tile_first(const TcParams& p, TileIter& it) {
-  it.s = -1;
+__device__ __forceinline__ void tile_first(const TcParams& p, TileIter& it, int grp) {
+  it.s = grp - p.ngroups;
   it.i = 0;
   it.nt = 0;
   it.L = 0;
@@ -342,7 +346,8 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int h = blockIdx.x / kNdv;
+  const int h = (blockIdx.x / kNdv) % p.H;
+  const int grp = blockIdx.x / (kNdv * p.H);             // sequence group
   const int dvt = static_cast<int>(cluster_ctarank());   // == blockIdx.x % 2 (cluster of 2)
   const uint32_t partner = static_cast<uint32_t>(dvt ^ 1);
   constexpr int tpb = kC / kTile;        // tiles per block (1 or 2)
@@ -415,7 +420,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       uint32_t uses[kNKV] = {0, 0, 0};
       int t = 0;
       bool ok = true;
-      for (int s = 0; s < p.nseq && ok; ++s) {
+      for (int s = grp; s < p.nseq && ok; s += p.ngroups) {
         int64_t row0;
         int L;
         seq_range(p, s, row0, L);
@@ -463,7 +468,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       int t = 0;
       bool ok = true;
       TileIter cur, nxt;
-      tile_first(p, cur);
+      tile_first(p, cur, grp);
       nxt = cur;
       tile_next(p, nxt);
 
@@ -641,7 +646,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
       }
     };
     TileIter cur, nxt;
-    tile_first(p, cur);
+    tile_first(p, cur, grp);
     nxt = cur;
     tile_next(p, nxt);
     int t = 0;
@@ -678,7 +683,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     const uint32_t lane_off = static_cast<uint32_t>(wt & ~31) << 16;
     uint32_t k = 0;
     bool ok = true;
-    for (int s = 0; s < p.nseq && ok; ++s) {
+    for (int s = grp; s < p.nseq && ok; s += p.ngroups) {
       int64_t row0;
       int L;
       seq_range(p, s, row0, L);
@@ -734,7 +739,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     bool ok = true;
     int t = 0;
     uint32_t blk = 0;
-    for (int s = 0; s < p.nseq && ok; ++s) {
+    for (int s = grp; s < p.nseq && ok; s += p.ngroups) {
       int64_t row0;
       int L;
       if (seq_range(p, s, row0, L)) continue;   // a one-token sequence of a mixed step
@@ -891,7 +896,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
     const float inv_hd = 1.0f / static_cast<float>(HD);
     bool ok = true;
     int t = 0;
-    for (int s = 0; s < p.nseq && ok; ++s) {
+    for (int s = grp; s < p.nseq && ok; s += p.ngroups) {
       int64_t row0;
       int L;
       seq_range(p, s, row0, L);
@@ -1104,8 +1109,13 @@ cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream)
                                            [a.C == 256 ? 1 : 0];
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
+  // Sequence groups: with few heads, the CTA pairs of several groups share the sequences
+  // (group g takes every G-th), as many as fit on the GPU at once (the norm exchange needs
+  // all pairs of a sequence's group resident; all groups together fit in one wave).
+  const int maxc = max_active_clusters();
+  p.ngroups = maxc > a.H ? std::max(1, std::min(a.nseq, maxc / a.H)) : 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.H * kNdv);
+  cfg.gridDim = dim3(a.H * kNdv * p.ngroups);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
