@@ -961,7 +961,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="prefill_128k",
                     choices=["prefill_8k", "prefill_128k", "varlen_16", "decode_256", "mixed_256", "backward_8k",
-                             "backward_128k", "train_128k", "znorm_128k", "chunk_state_128k"])
+                             "backward_128k", "train_128k", "znorm_128k", "chunk_state_128k", "prefill_128k_h8"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     args = ap.parse_args()

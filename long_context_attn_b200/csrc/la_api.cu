@@ -1,6 +1,7 @@
 // C ABI of the Lightning Attention library: argument validation, kernel selection,
 // workspace carving and the device error record.  Every compute step runs in the
 // kernels of la_decode.cu, la_simt.cu and la_prefill_tc.cu; there is no CPU path.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 
@@ -36,6 +37,9 @@ cudaError_t launch_bwd_scale(const void* q, const void* k, void* dq, void* dk, i
                              cudaStream_t stream);
 int znorm_max_chunks(int max_len);
 int chunk_state_splits(int nseq, int H, int max_len, int num_sms);
+cudaError_t launch_chunk_cu(int* cu, int B, int T, int Tc, int S, cudaStream_t stream);
+cudaError_t launch_chunk_prefix(const float* cs, const float* s0, float* prefix, float* out, int B, int S, int H,
+                                int num_sms, cudaStream_t stream);
 cudaError_t launch_chunk_state_tc(const void* k, const void* v, const float* state_in, float* state_out,
                                   float* partial, const int* cu, int nseq, int T, int max_len, int64_t tokens, int H,
                                   int phi_identity, int num_sms, ErrRec* err, cudaStream_t stream);
@@ -100,8 +104,51 @@ Path choose_path(la_dtype dt, int H, int D, int C, la_out_mode mode) {
   return Path::kSimt;
 }
 
+// Long sequences with few heads (tensor-core path, fixed length, forward time): each of the
+// B sequences is cut into S chunks of Tc tokens (a multiple of the tile) that run as
+// separate sequences in parallel CTA-pair groups, each chunk starting from the state the
+// chunks before it reach (their states from the chunk-state kernel, summed in order).
+constexpr int kSplitMinChunk = 1024;
+struct SplitPlan {
+  int S, Tc;
+};
+SplitPlan split_plan(int B, int T, int H, int D) {
+  SplitPlan sp{1, T};
+  if (D != 128 || B < 1 || H < 1 || T < 2 * kSplitMinChunk) return sp;
+  const int groups = la::max_active_clusters() / H;   // CTA-pair groups that fit at once
+  if (groups < 2 * B) return sp;
+  const int S = std::min(groups / B, T / kSplitMinChunk);
+  if (S < 2) return sp;
+  sp.Tc = ((T + S - 1) / S + 127) / 128 * 128;
+  sp.S = (T + sp.Tc - 1) / sp.Tc;
+  return sp;
+}
+// Workspace of a split call after the error record: [tensor-core part for the B * S chunks]
+// [chunk cu_seqlens] [chunk states] [chunk initial states] [chunk-state split partials].
+struct SplitLayout {
+  size_t tc, cu, st, part, total;
+};
+SplitLayout split_layout(const SplitPlan& sp, int B, int64_t tokens, int H, int D, int C) {
+  SplitLayout l{};
+  const int n = B * sp.S;
+  l.tc = la::tc_workspace_bytes(n, sp.Tc, tokens, H, D, C);
+  l.cu = up256(sizeof(int) * static_cast<size_t>(n + 1));
+  l.st = up256(sizeof(float) * static_cast<size_t>(n) * H * D * D);
+  l.part = up256(sizeof(float) * static_cast<size_t>(la::chunk_state_splits(n, H, sp.Tc, current_sm_count())) * n *
+                 H * D * D);
+  l.total = l.tc + l.cu + 2 * l.st + l.part;
+  return l;
+}
+
 size_t prefill_ws_bytes(Path p, int nseq, int max_len, int64_t tokens, int H, int D, int C, la_out_mode mode) {
-  if (p == Path::kTc || p == Path::kTcSplit) return kErrBytes + la::tc_workspace_bytes(nseq, max_len, tokens, H, D, C);
+  if (p == Path::kTc || p == Path::kTcSplit) {
+    // A fixed-length call may split (B = nseq, T = max_len); room for that is reserved here
+    // (a packed call never splits and at most over-reserves).
+    size_t n = la::tc_workspace_bytes(nseq, max_len, tokens, H, D, C);
+    const SplitPlan sp = split_plan(nseq, max_len, H, D);
+    if (sp.S > 1) n = std::max(n, split_layout(sp, nseq, tokens, H, D, C).total);
+    return kErrBytes + n;
+  }
   size_t y = (mode == LA_OUT_RAW) ? 0 : up256(sizeof(float) * static_cast<size_t>(tokens) * H * D);
   return kErrBytes + y;
 }
@@ -129,7 +176,7 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
   la::ErrRec* err = static_cast<la::ErrRec*>(workspace);
   char* ws = static_cast<char*>(workspace) + kErrBytes;
   const int phi_id = (phi == LA_PHI_IDENTITY) ? 1 : 0;
-  cudaError_t e;
+  cudaError_t e = cudaSuccess;
   if (path == Path::kTc || path == Path::kTcSplit) {
     const bool split = path == Path::kTcSplit;
     la::TcArgs a{};
@@ -140,10 +187,32 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
     a.mode = static_cast<int>(split ? LA_OUT_RAW : mode);
     a.eps = eps; a.w = split ? nullptr : w; a.err = err; a.ws = ws;
     a.reverse = reverse ? 1 : 0;
-    e = la::launch_tc_prefill(a, current_sm_count(), stream);
+    const SplitPlan sp = (!cu && T_fixed > 0 && !reverse) ? split_plan(nseq, T_fixed, H, D) : SplitPlan{1, T_fixed};
+    if (sp.S > 1) {
+      const SplitLayout sl = split_layout(sp, nseq, tokens, H, D, C);
+      char* x = ws + sl.tc;
+      int* ccu = reinterpret_cast<int*>(x);
+      float* cst = reinterpret_cast<float*>(x + sl.cu);
+      float* cin = reinterpret_cast<float*>(x + sl.cu + sl.st);
+      float* cpart = reinterpret_cast<float*>(x + sl.cu + 2 * sl.st);
+      const int n = nseq * sp.S;
+      e = la::launch_chunk_cu(ccu, nseq, T_fixed, sp.Tc, sp.S, stream);
+      if (e == cudaSuccess)
+        e = la::launch_chunk_state_tc(k, v, nullptr, cst, cpart, ccu, n, 0, sp.Tc, tokens, H, phi_id,
+                                      current_sm_count(), err, stream);
+      if (e == cudaSuccess)   // chunk initial states, and the sequences' final states
+        e = la::launch_chunk_prefix(cst, state_in, cin, state_out, nseq, sp.S, H, current_sm_count(), stream);
+      a.cu = ccu;
+      a.nseq = n;
+      a.T = 0;
+      a.max_len = sp.Tc;
+      a.state_in = cin;
+      a.state_out = nullptr;
+    }
+    if (e == cudaSuccess) e = la::launch_tc_prefill(a, current_sm_count(), stream);
     if (e == cudaSuccess && split)   // the norm (and gate) per token, over the raw output in place
       e = la::launch_znorm_transform(out, nullptr, g, w, tokens, H, D, static_cast<int>(mode), eps, dt, stream);
-    g_last_path = split ? "tcgen05+norm" : "tcgen05";
+    g_last_path = sp.S > 1 ? (split ? "tcgen05+norm+chunks" : "tcgen05+chunks") : (split ? "tcgen05+norm" : "tcgen05");
   } else {
     float* y_ws = (mode == LA_OUT_RAW) ? nullptr : reinterpret_cast<float*>(ws);
     e = la::launch_simt_prefill(q, k, v, out, y_ws, state_in, state_out, cu, nseq, T_fixed, H, D, C, dt, phi_id,

@@ -37,5 +37,7 @@ bool tc_eligible(const TcShape& s, int num_sms);
 // Workspace bytes after the 256-byte error record.
 size_t tc_workspace_bytes(int nseq, int max_len, int64_t tokens, int H, int D, int C);
 cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream);
+// CTA pairs (heads x groups) that fit on the current device at once.
+int max_active_clusters();
 
 }  // namespace la

@@ -296,6 +296,42 @@ __global__ void __launch_bounds__(256) state_reduce_kernel(const float4* __restr
   }
 }
 
+// Chunk boundaries of B sequences of T tokens cut into S chunks of Tc tokens (the last
+// chunks of a sequence may be shorter or empty): cu[b * S + c] = b * T + min(c * Tc, T).
+__global__ void chunk_cu_kernel(int* cu, int B, int T, int Tc, int S) {
+  const int n = B * S;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= n; i += gridDim.x * blockDim.x) {
+    if (i == n) {
+      cu[i] = B * T;
+    } else {
+      const int b = i / S, c = i % S;
+      const int64_t off = static_cast<int64_t>(c) * Tc;
+      cu[i] = b * T + static_cast<int>(off < T ? off : T);
+    }
+  }
+}
+
+// prefix[b, c] = S0[b] + sum_{c' < c} cs[b, c'] (in chunk order) and out[b] = S0[b] + all of
+// them: the initial state of every chunk of a sequence and its final state.
+__global__ void __launch_bounds__(256) chunk_prefix_kernel(const float4* __restrict__ cs,
+                                                           const float4* __restrict__ s0,
+                                                           float4* __restrict__ prefix, float4* __restrict__ out,
+                                                           int B, int S, int64_t n4) {
+  const int64_t total = static_cast<int64_t>(B) * n4;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = i / n4, e = i % n4;
+    float4 run = s0 ? s0[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < S; ++c) {
+      const int64_t at = (b * S + c) * n4 + e;
+      prefix[at] = run;
+      const float4 x = cs[at];
+      run.x += x.x; run.y += x.y; run.z += x.z; run.w += x.w;
+    }
+    if (out) out[i] = run;
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -364,6 +400,23 @@ cudaError_t launch_chunk_state_tc(const void* k, const void* v, const float* sta
   state_reduce_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(partial), splits,
                                                   reinterpret_cast<const float4*>(state_in),
                                                   reinterpret_cast<float4*>(state_out), n4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_cu(int* cu, int B, int T, int Tc, int S, cudaStream_t stream) {
+  chunk_cu_kernel<<<(B * S + 256) / 256, 256, 0, stream>>>(cu, B, T, Tc, S);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_prefix(const float* cs, const float* s0, float* prefix, float* out, int B, int S, int H,
+                                int num_sms, cudaStream_t stream) {
+  const int64_t n4 = static_cast<int64_t>(H) * kD * kD / 4;
+  const int64_t total = static_cast<int64_t>(B) * n4;
+  const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(num_sms) * 8));
+  chunk_prefix_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(cs),
+                                                  reinterpret_cast<const float4*>(s0),
+                                                  reinterpret_cast<float4*>(prefix), reinterpret_cast<float4*>(out),
+                                                  B, S, n4);
   return cudaGetLastError();
 }
 

@@ -153,6 +153,9 @@ WORKLOADS = {
     # denominators phi(q) . z stay positive.
     "znorm_128k": Workload("znorm_128k", "znorm", 1009, 1, 131072, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5,
                            qk_shift=1.0),
+    # One 128K sequence with 8 heads (a tensor-parallel shard of the 64): the few-heads case.
+    "prefill_128k_h8": Workload("prefill_128k_h8", "prefill", 1012, 1, 131072, 8, 128, 256, "bf16", "rmsnorm_gate",
+                                0.5),
     # A training step on the 128K prefill's shapes: forward (keeping y) and backward.
     "train_128k": Workload("train_128k", "train", 1011, 1, 131072, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5),
     # Step 1 of the sequence-parallel prefill on the 128K prefill's shapes: the state from k, v.

@@ -183,3 +183,21 @@ def test_tc_more_heads_than_resident_pairs(mode, expect, cuda_device):
                                     mode=m)
     assert_close(o, ref, "bf16")
     assert_close(st, ref_st, "bf16", "state")
+
+
+@pytest.mark.parametrize("B,T,H,mode,with_state", [(1, 8192, 8, "rmsnorm_gate", False), (2, 5000, 8, "raw", True),
+                                                   (1, 3000, 4, "rmsnorm", True), (1, 2048, 16, "rmsnorm_gate", True)])
+def test_tc_long_sequences_few_heads_split_into_chunks(B, T, H, mode, with_state, cuda_device):
+    """Few heads, long sequences: each sequence is cut into chunks that run as parallel
+    sequence groups, each starting from the state of the chunks before it (chunk-state
+    kernel + ordered prefix).  Output and final state against the oracle."""
+    D, C = 128, 256
+    m = mode_code(mode)
+    q, k, v, g = synth.prefill_inputs(3951 + T + H, B * T, H, D, "bf16", 0.5, True)
+    q, k, v = (a.reshape(B, T, H, D) for a in (q, k, v))
+    g = g.reshape(B, T, H * D) if m == oracle.MODE_RMSNORM_GATE else None
+    s0 = synth.normal(3951, 9, (B, H, D, D), 0.05, "f32") if with_state else None
+    o, st, _ = run_prefill(q, k, v, g, C, m, state_in=s0, want_state=True, expect_path="tcgen05+chunks")
+    ref, ref_st, _ = oracle.prefill(q, k, v, g, state_in=s0, mode=m)
+    assert_close(o, ref, "bf16")
+    assert_close(st, ref_st, "bf16", "state")

@@ -57,6 +57,7 @@ def test_workload_table():
     assert w["znorm_128k"].seed == 1009 and w["znorm_128k"].qk_shift == 1.0
     assert w["chunk_state_128k"].seed == 1010 and w["chunk_state_128k"].kind == "chunk_state"
     assert w["train_128k"].seed == 1011 and w["train_128k"].kind == "train"
+    assert w["prefill_128k_h8"].seed == 1012 and w["prefill_128k_h8"].H == 8
     a = synth.normal(7, 0, (1000,), 0.5, "bf16")
     b = synth.shifted(a, 1.0)
     assert b.dtype == np.uint16 and np.allclose(synth.bf16_to_f32(b), synth.bf16_to_f32(a) + 1.0, atol=2 ** -7)
