@@ -39,7 +39,7 @@ int znorm_max_chunks(int max_len);
 int chunk_state_splits(int nseq, int H, int max_len, int num_sms);
 cudaError_t launch_chunk_cu(int* cu, int B, int T, int Tc, int S, cudaStream_t stream);
 cudaError_t launch_chunk_prefix(const float* cs, const float* s0, float* prefix, float* out, int B, int S, int H,
-                                int num_sms, cudaStream_t stream);
+                                int reverse, int num_sms, cudaStream_t stream);
 cudaError_t launch_chunk_state_tc(const void* k, const void* v, const float* state_in, float* state_out,
                                   float* partial, const int* cu, int nseq, int T, int max_len, int64_t tokens, int H,
                                   int phi_identity, int num_sms, ErrRec* err, cudaStream_t stream);
@@ -104,10 +104,11 @@ Path choose_path(la_dtype dt, int H, int D, int C, la_out_mode mode) {
   return Path::kSimt;
 }
 
-// Long sequences with few heads (tensor-core path, fixed length, forward time): each of the
-// B sequences is cut into S chunks of Tc tokens (a multiple of the tile) that run as
-// separate sequences in parallel CTA-pair groups, each chunk starting from the state the
-// chunks before it reach (their states from the chunk-state kernel, summed in order).
+// Long sequences with few heads (tensor-core path, fixed length): each of the B sequences
+// is cut into S chunks of Tc tokens (a multiple of the tile) that run as separate
+// sequences in parallel CTA-pair groups, each chunk starting from the state the chunks
+// before it reach -- after it, when time runs backwards -- (their states from the
+// chunk-state kernel, summed in order).
 constexpr int kSplitMinChunk = 1024;
 struct SplitPlan {
   int S, Tc;
@@ -187,7 +188,7 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
     a.mode = static_cast<int>(split ? LA_OUT_RAW : mode);
     a.eps = eps; a.w = split ? nullptr : w; a.err = err; a.ws = ws;
     a.reverse = reverse ? 1 : 0;
-    const SplitPlan sp = (!cu && T_fixed > 0 && !reverse) ? split_plan(nseq, T_fixed, H, D) : SplitPlan{1, T_fixed};
+    const SplitPlan sp = (!cu && T_fixed > 0) ? split_plan(nseq, T_fixed, H, D) : SplitPlan{1, T_fixed};
     if (sp.S > 1) {
       const SplitLayout sl = split_layout(sp, nseq, tokens, H, D, C);
       char* x = ws + sl.tc;
@@ -201,7 +202,8 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
         e = la::launch_chunk_state_tc(k, v, nullptr, cst, cpart, ccu, n, 0, sp.Tc, tokens, H, phi_id,
                                       current_sm_count(), err, stream);
       if (e == cudaSuccess)   // chunk initial states, and the sequences' final states
-        e = la::launch_chunk_prefix(cst, state_in, cin, state_out, nseq, sp.S, H, current_sm_count(), stream);
+        e = la::launch_chunk_prefix(cst, state_in, cin, state_out, nseq, sp.S, H, reverse ? 1 : 0,
+                                    current_sm_count(), stream);
       a.cu = ccu;
       a.nseq = n;
       a.T = 0;

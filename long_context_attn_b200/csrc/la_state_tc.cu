@@ -312,17 +312,19 @@ __global__ void chunk_cu_kernel(int* cu, int B, int T, int Tc, int S) {
 }
 
 // prefix[b, c] = S0[b] + sum_{c' < c} cs[b, c'] (in chunk order) and out[b] = S0[b] + all of
-// them: the initial state of every chunk of a sequence and its final state.
+// them: the initial state of every chunk of a sequence and its final state.  With time
+// running backwards the chunks are taken from the last: prefix[b, c] = S0[b] + sum_{c' > c}.
 __global__ void __launch_bounds__(256) chunk_prefix_kernel(const float4* __restrict__ cs,
                                                            const float4* __restrict__ s0,
                                                            float4* __restrict__ prefix, float4* __restrict__ out,
-                                                           int B, int S, int64_t n4) {
+                                                           int B, int S, int64_t n4, int reverse) {
   const int64_t total = static_cast<int64_t>(B) * n4;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t b = i / n4, e = i % n4;
     float4 run = s0 ? s0[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = 0; c < S; ++c) {
+    for (int j = 0; j < S; ++j) {
+      const int c = reverse ? S - 1 - j : j;
       const int64_t at = (b * S + c) * n4 + e;
       prefix[at] = run;
       const float4 x = cs[at];
@@ -409,14 +411,14 @@ cudaError_t launch_chunk_cu(int* cu, int B, int T, int Tc, int S, cudaStream_t s
 }
 
 cudaError_t launch_chunk_prefix(const float* cs, const float* s0, float* prefix, float* out, int B, int S, int H,
-                                int num_sms, cudaStream_t stream) {
+                                int reverse, int num_sms, cudaStream_t stream) {
   const int64_t n4 = static_cast<int64_t>(H) * kD * kD / 4;
   const int64_t total = static_cast<int64_t>(B) * n4;
   const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(num_sms) * 8));
   chunk_prefix_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(cs),
                                                   reinterpret_cast<const float4*>(s0),
                                                   reinterpret_cast<float4*>(prefix), reinterpret_cast<float4*>(out),
-                                                  B, S, n4);
+                                                  B, S, n4, reverse);
   return cudaGetLastError();
 }
 

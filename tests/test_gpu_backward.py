@@ -225,3 +225,47 @@ def test_backward_with_saved_y_equals_recompute(mode, cuda_device):
     ref, _, _ = oracle.prefill(q.reshape(shp), k.reshape(shp), v.reshape(shp),
                                g.reshape(gshp) if gate is not None else None, mode=m)
     assert_close(to_host(out), ref, "bf16")
+
+
+def test_backward_long_sequence_few_heads_splits_every_pass(cuda_device):
+    """T = 4096 with 8 heads: every pass (forward and reverse time) is cut into chunks run
+    as parallel groups; gradients (with S0 and dS_T) against the oracle."""
+    _run_fixed(1, 4096, 8, 128, 256, "bf16", "rmsnorm_gate", True, 3961)
+
+
+@pytest.mark.parametrize("C", [128, 256])
+def test_backward_exact_integers_split(C, cuda_device):
+    """The split passes on integer inputs (identity features, ternary values, integer S0
+    and dS_T): bit-exact against the oracle, as for the unsplit passes."""
+    import torch
+    la = _la()
+    T, H, D = 4096, 4, 128
+    q, k, v, dout = (synth.ternary(3971, s, (T, H, D), 0.03, "bf16") for s in range(4))
+    s0 = np.round(synth.normal(3971, 9, (1, H, D, D), 1.0, "f32")).astype(np.float32)
+    dsT = np.round(synth.normal(3971, 10, (1, H, D, D), 1.0, "f32")).astype(np.float32)
+    f = lambda a: synth.bf16_to_f32(a).astype(np.float64)
+    Q, K, V, dY = f(q), f(k), f(v), f(dout)
+    for a, b, rev in ((V, K, False), (dY, Q, True), (Q, dY, True), (K, V, False)):
+        outer = np.einsum("thi,thj->thij", a, b)
+        run = np.cumsum(outer[::-1] if rev else outer, axis=0)
+        assert np.abs(run).max() + np.abs(s0).max() + np.abs(dsT).max() <= 256
+    shp = (1, T, H, D)
+    dq_, dk_, dv_ = (to_dev(a).reshape(shp) for a in (q, k, v))
+    ddo = to_dev(dout).reshape(1, T, H * D)
+    gq, gk, gv = (torch.full_like(dq_, float("nan")) for _ in range(3))
+    gs = torch.full((1, H, D, D), float("nan"), dtype=torch.float32, device="cuda")
+    ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD, 1, T, 0, H, D, C, la.LA_BF16,
+                                                           la.LA_OUT_RAW))
+    la.lightning_attn_backward(dq_, dk_, dv_, None, ddo, gq, gk, gv, state_in=to_dev(s0), dstate_in=gs,
+                               block_size=C, phi=la.LA_PHI_IDENTITY, mode=la.LA_OUT_RAW, workspace=ws,
+                               dstate_out=to_dev(dsT))
+    assert la.lightning_attn_last_path() == "tcgen05+chunks"
+    la.lightning_attn_check(ws)
+    ref = oracle.backward(q.reshape(shp), k.reshape(shp), v.reshape(shp), None, dout.reshape(1, T, H * D),
+                          state_in=s0, phi=oracle.PHI_IDENTITY, mode=oracle.MODE_RAW, dstate_out=dsT)
+    for got, want, name in zip((gq, gk, gv, gs), (ref[0], ref[1], ref[2], ref[4]), ("dq", "dk", "dv", "dstate")):
+        assert np.abs(want).max() <= 256, name
+        g64 = synth.bf16_to_f32(to_host(got)).astype(np.float64) if got.dtype == torch.bfloat16 \
+            else to_host(got).astype(np.float64)
+        bad = np.argwhere(g64.reshape(want.shape) != want)
+        assert bad.size == 0, f"{name}: {len(bad)} mismatches, first at {bad[:3].tolist()}"
