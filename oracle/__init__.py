@@ -70,7 +70,7 @@ def _get():
         lib.oracle_forward_znorm_packed.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, vp, i32, i32, dbl,
                                                     vp, vp, vp, vp]
         lib.oracle_backward_packed.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, vp, i32, i32, dbl,
-                                               vp, vp, vp, vp, vp, vp]
+                                               vp, vp, vp, vp, vp, vp, vp]
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         for f in (lib.oracle_forward_packed, lib.oracle_prefill, lib.oracle_decode,
@@ -207,7 +207,8 @@ def backward_packed(q, k, v, g, dout, cu_seqlens, H, D, state_in=None, phi=PHI_S
     final-state gradient dstate_out [N, H, D, D] (fp32, or None for zero).
 
     q, k, v [tokens, H, D], g and dout [tokens, H*D] (bf16 bits or fp32, all one dtype).
-    Returns fp64 (dq, dk, dv [tokens, H, D], dg [tokens, H*D] or None, dstate [N, H, D, D]).
+    Returns fp64 (dq, dk, dv [tokens, H, D], dg [tokens, H*D] or None, dstate [N, H, D, D],
+    dw [H*D] -- the norm weight's gradient, zeros in raw mode).
     """
     q, k, v, g, dout = _c(q), _c(k), _c(v), _c(g), _c(dout)
     dt = _dtype_code(q)
@@ -217,13 +218,14 @@ def backward_packed(q, k, v, g, dout, cu_seqlens, H, D, state_in=None, phi=PHI_S
     dq, dk, dv = (np.zeros((tokens, H, D), dtype=np.float64) for _ in range(3))
     dg = np.zeros((tokens, H * D), dtype=np.float64) if mode == MODE_RMSNORM_GATE else None
     dst = np.zeros((N, H, D, D), dtype=np.float64)
+    dw = np.zeros(H * D, dtype=np.float64)
     s_in, ds_out, w = _c(state_in, np.float32), _c(dstate_out, np.float32), _c(norm_weight, np.float32)
     rc = _get().oracle_backward_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout), dt, _ptr(cu), N, H, D,
                                        _ptr(s_in), _ptr(ds_out), phi, mode, eps, _ptr(w), _ptr(dq), _ptr(dk),
-                                       _ptr(dv), _ptr(dg), _ptr(dst))
+                                       _ptr(dv), _ptr(dg), _ptr(dst), _ptr(dw))
     if rc != 0:
         raise ValueError("oracle_backward_packed rejected its arguments")
-    return dq, dk, dv, dg, dst
+    return dq, dk, dv, dg, dst, dw
 
 
 def backward(q, k, v, g, dout, state_in=None, phi=PHI_SILU, mode=MODE_RMSNORM_GATE, eps=1e-6,
@@ -232,11 +234,11 @@ def backward(q, k, v, g, dout, state_in=None, phi=PHI_SILU, mode=MODE_RMSNORM_GA
     B, T, H, D = q.shape
     cu = np.arange(B + 1, dtype=np.int32) * T
     r = lambda a, s: None if a is None else np.reshape(a, s)
-    dq, dk, dv, dg, dst = backward_packed(r(q, (B * T, H, D)), r(k, (B * T, H, D)), r(v, (B * T, H, D)),
+    dq, dk, dv, dg, dst, dw = backward_packed(r(q, (B * T, H, D)), r(k, (B * T, H, D)), r(v, (B * T, H, D)),
                                           r(g, (B * T, H * D)), r(dout, (B * T, H * D)), cu, H, D, state_in,
                                           phi, mode, eps, norm_weight, dstate_out)
     return (dq.reshape(B, T, H, D), dk.reshape(B, T, H, D), dv.reshape(B, T, H, D),
-            None if dg is None else dg.reshape(B, T, H * D), dst)
+            None if dg is None else dg.reshape(B, T, H * D), dst, dw)
 
 
 def forward_znorm_packed(q, k, v, g, cu_seqlens, H, D, state_in=None, z_in=None, phi=PHI_SILU,

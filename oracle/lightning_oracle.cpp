@@ -189,6 +189,7 @@ void write_stats(double* stats, const Cmp& o, const Cmp& s) {
 //     RAW:            dy = dO
 //     RMSNORM(_GATE): dy_c = r u_c - r^3 y_c (sum_c' u_c' y_c') / (H*D)
 //     gate:           dg_c = dO_c y_c r w_c s_c (1 - s_c)
+//     norm weight:    dw_c = sum over tokens of dO_c y_c r s_c
 //   recurrence (per head; S_t = S0 + sum_{i<=t} phi(k_i) v_i^T, y_t = S_t^T phi(q_t)), with
 //   dS_T the gradient reaching the final state (zero unless given):
 //     dphi(q_t) = S_t dy_t
@@ -204,9 +205,11 @@ inline double dfeature(double x, int phi) {
   return s * (1.0 + x * (1.0 - s));
 }
 
-// Backward of transform_token for one token: dy (H*D) and, with the gate, dg (H*D).
+// Backward of transform_token for one token: dy (H*D), with the gate dg (H*D), and this
+// token's terms of dw (H*D, added into dwt if non-null).
 void transform_token_backward(const double* y, const void* dout, const void* g, int dtype, int64_t grow,
-                              int HD, int mode, double eps, const float* w, double* dy, double* dg) {
+                              int HD, int mode, double eps, const float* w, double* dy, double* dg,
+                              double* dwt) {
   if (mode == MODE_RAW) {
     for (int c = 0; c < HD; ++c) dy[c] = widen(dout, dtype, grow * HD + c);
     return;
@@ -223,6 +226,7 @@ void transform_token_backward(const double* y, const void* dout, const void* g, 
     u[c] = d * wc * s;
     dot += u[c] * y[c];
     if (mode == MODE_RMSNORM_GATE && dg) dg[c] = d * y[c] * r * wc * s * (1.0 - s);
+    if (dwt) dwt[c] = d * y[c] * r * s;
   }
   for (int c = 0; c < HD; ++c) dy[c] = r * u[c] - r * r * r * y[c] * dot / HD;
 }
@@ -462,14 +466,17 @@ int oracle_transform(const double* y, int64_t tokens, int H, int D, int mode, do
 // zero).  Recomputes the raw forward y, applies the transform backward per token, then the
 // recurrence backward per head.  Outputs fp64: dq, dk, dv [tokens, H, D], dg [tokens, H*D]
 // (gate mode; may be null otherwise), dstate [N, H, D, D] (the gradient of each sequence's
-// initial state; may be null).
+// initial state; may be null), dw [H*D] (the norm weight's gradient, zero in raw mode; may
+// be null).
 int oracle_backward_packed(const void* q, const void* k, const void* v, const void* g, const void* dout,
                            int dtype, const int32_t* cu, int N, int H, int D, const float* state_in,
                            const float* dstate_out, int phi, int mode, double eps, const float* w, double* dq,
-                           double* dk, double* dv, double* dg, double* dstate) {
+                           double* dk, double* dv, double* dg, double* dstate, double* dw) {
   if (N < 0 || H <= 0 || D <= 0 || !dout || !dq || !dk || !dv) return 1;
   if (mode == MODE_RMSNORM_GATE && (!g || !dg)) return 1;
   const int HD = H * D;
+  if (dw)
+    for (int c = 0; c < HD; ++c) dw[c] = 0.0;
   const int64_t nst = static_cast<int64_t>(H) * D * D;
   for (int s = 0; s < N; ++s) {
     const int64_t row0 = cu[s], L = static_cast<int64_t>(cu[s + 1]) - cu[s];
@@ -482,11 +489,18 @@ int oracle_backward_packed(const void* q, const void* k, const void* v, const vo
 #pragma omp parallel for schedule(dynamic, 1)
     for (int h = 0; h < H; ++h)
       recur_head(q, k, v, dtype, row0, L, H, D, h, phi, st.data() + static_cast<size_t>(h) * D * D, y.data());
-    // transform backward per token (dy indexed from the sequence's first row)
+    // transform backward per token (dy indexed from the sequence's first row); each token's
+    // dw terms kept apart and added afterwards in token order
+    const bool want_dw = dw && mode != MODE_RAW;
+    std::vector<double> dwt(want_dw ? static_cast<size_t>(L) * HD : 0);
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < L; ++t)
       transform_token_backward(y.data() + t * HD, dout, g, dtype, row0 + t, HD, mode, eps, w,
-                               dy.data() + t * HD, dg ? dg + (row0 + t) * HD : nullptr);
+                               dy.data() + t * HD, dg ? dg + (row0 + t) * HD : nullptr,
+                               want_dw ? dwt.data() + t * HD : nullptr);
+    if (want_dw)
+      for (int64_t t = 0; t < L; ++t)
+        for (int c = 0; c < HD; ++c) dw[c] += dwt[static_cast<size_t>(t) * HD + c];
     std::vector<double> dS0(nst), dST;
     if (dstate_out) {
       dST.resize(nst);

@@ -40,8 +40,8 @@ def _loss(x, dout, phi, mode, w):
 @pytest.mark.parametrize("mode", [oracle.MODE_RAW, oracle.MODE_RMSNORM, oracle.MODE_RMSNORM_GATE])
 def test_backward_matches_finite_differences(phi, mode):
     x, dout, w = _inputs(2101 + 7 * mode + phi, mode)
-    dq, dk, dv, dg, dst = oracle.backward_packed(x["q"], x["k"], x["v"], x["g"], dout, CU, H, D,
-                                                 state_in=x["state_in"], phi=phi, mode=mode, norm_weight=w)
+    dq, dk, dv, dg, dst, dw = oracle.backward_packed(x["q"], x["k"], x["v"], x["g"], dout, CU, H, D,
+                                                     state_in=x["state_in"], phi=phi, mode=mode, norm_weight=w)
     grads = {"q": dq, "k": dk, "v": dv, "state_in": dst}
     if mode == oracle.MODE_RMSNORM_GATE:
         grads["g"] = dg
@@ -67,7 +67,7 @@ def test_empty_sequence_gradient_of_state_is_zero_and_one_token_closed_form():
     dphi(q) = S_1 dy, dphi(k) = (dy.v) phi(q), dS0 = phi(q) dy^T (hand-derived)."""
     x, dout, w = _inputs(2151, oracle.MODE_RAW)
     phi = oracle.PHI_IDENTITY
-    dq, dk, dv, _, dst = oracle.backward_packed(x["q"], x["k"], x["v"], None, dout, CU, H, D,
+    dq, dk, dv, _, dst, _ = oracle.backward_packed(x["q"], x["k"], x["v"], None, dout, CU, H, D,
                                                 state_in=x["state_in"], phi=phi, mode=oracle.MODE_RAW)
     assert np.all(dst[1] == 0.0)
     t = int(CU[2])                      # the one-token sequence is sequence 2
@@ -89,7 +89,7 @@ def test_backward_matches_masked_matrix_form(phi):
     q, k, v, _ = synth.prefill_inputs(2161, T, Hh, Dd, "f32", 0.7, False)
     dout = synth.normal(2161, 11, (T, Hh * Dd), 1.0, "f32")
     s0 = synth.normal(2161, 12, (1, Hh, Dd, Dd), 0.3, "f32")
-    dq, dk, dv, _, dst = oracle.backward_packed(q, k, v, None, dout, [0, T], Hh, Dd, state_in=s0, phi=phi,
+    dq, dk, dv, _, dst, _ = oracle.backward_packed(q, k, v, None, dout, [0, T], Hh, Dd, state_in=s0, phi=phi,
                                                 mode=oracle.MODE_RAW)
     f = (lambda z: z / (1.0 + np.exp(-z))) if phi == oracle.PHI_SILU else (lambda z: z)
     df = (lambda z: (1 / (1 + np.exp(-z))) * (1 + z * (1 - 1 / (1 + np.exp(-z))))) if phi == oracle.PHI_SILU \
@@ -120,9 +120,9 @@ def test_final_state_gradient_matches_finite_differences(mode):
                                            phi=phi, mode=mode, norm_weight=w)
         return float(np.sum(out * dout.astype(np.float64)) + np.sum(st * dST.astype(np.float64)))
 
-    dq, dk, dv, dg, dst = oracle.backward_packed(x["q"], x["k"], x["v"], x["g"], dout, CU, H, D,
-                                                 state_in=x["state_in"], phi=phi, mode=mode, norm_weight=w,
-                                                 dstate_out=dST)
+    dq, dk, dv, dg, dst, _ = oracle.backward_packed(x["q"], x["k"], x["v"], x["g"], dout, CU, H, D,
+                                                    state_in=x["state_in"], phi=phi, mode=mode, norm_weight=w,
+                                                    dstate_out=dST)
     grads = {"q": dq, "k": dk, "v": dv, "state_in": dst}
     rng = np.random.default_rng(2171)
     eps = 1e-3
@@ -137,3 +137,22 @@ def test_final_state_gradient_matches_finite_differences(mode):
         pred = float(np.sum(grad.reshape(step.shape) * step))
         scale = float(np.sum(np.abs(grad.reshape(step.shape) * step)))
         assert abs(fd - pred) <= 1e-5 * scale, f"{name}: finite difference {fd:.9e} vs gradient {pred:.9e}"
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_RMSNORM, oracle.MODE_RMSNORM_GATE])
+def test_norm_weight_gradient_matches_finite_differences(mode):
+    """dw (the RMSNorm weight's gradient, summed over tokens) against central differences
+    of the forward in w; zero in raw mode."""
+    x, dout, w = _inputs(2181 + mode, mode)
+    *_, dw = oracle.backward_packed(x["q"], x["k"], x["v"], x["g"], dout, CU, H, D, state_in=x["state_in"],
+                                    mode=mode, norm_weight=w)
+    rng = np.random.default_rng(2181)
+    delta = rng.standard_normal(w.shape)
+    eps = 1e-3
+    wp, wm = (w + eps * delta).astype(np.float32), (w - eps * delta).astype(np.float32)
+    step = wp.astype(np.float64) - wm.astype(np.float64)
+    fd = _loss(x, dout, oracle.PHI_SILU, mode, wp) - _loss(x, dout, oracle.PHI_SILU, mode, wm)
+    pred = float(np.sum(dw * step))
+    assert abs(fd - pred) <= 1e-5 * float(np.sum(np.abs(dw * step))), (fd, pred)
+    *_, dw_raw = oracle.backward_packed(x["q"], x["k"], x["v"], None, dout, CU, H, D, mode=oracle.MODE_RAW)
+    assert np.all(dw_raw == 0.0)
