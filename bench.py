@@ -507,7 +507,8 @@ class BackwardCase:
 
 class TrainCase(BackwardCase):
     """A training step on one long sequence: the forward keeping its raw output y (prefill in
-    raw mode, then the norm and gate), and the backward from dout using that y."""
+    raw mode, then the norm and gate), and the backward from dout using that y, with the
+    norm weight's gradient as well (the norm weight is a trained parameter)."""
 
     def __init__(self, name, w, device, rank):
         super().__init__(name, w, device, rank)
@@ -516,12 +517,16 @@ class TrainCase(BackwardCase):
         self.y = torch.empty((1, T, H * D), dtype=torch.bfloat16, device=device)
         self.out = torch.empty((1, T, H * D), dtype=torch.bfloat16, device=device)
         self.h_out_fwd = torch.empty((1, T, H * D), dtype=torch.bfloat16).pin_memory()
+        self.nw = torch.ones((H * D,), dtype=torch.float32, device=device)
+        self.dw = torch.empty((H * D,), dtype=torch.float32, device=device)
+        self.h_dw = torch.empty((H * D,), dtype=torch.float32).pin_memory()
         # forward: q, k, v, g read + out written; backward: q, k, v, g, dout read + 4 gradients written
         self.alg_bytes = T * 14 * H * D * 2
         # the forward prefill plus the backward's three passes (the recompute is skipped)
         self.alg_flops, self.issued_flops = (4 * x * T for x in _flops_per_token(H, D, self.C))
-        self.launches_per_step = 8    # prefill, transform, norm/gate backward, prep, three passes, post
-        self.d2h += self.h_out_fwd.numel() * 2
+        # prefill, transform; backward: dw (two stages), norm/gate, features, three passes, scale
+        self.launches_per_step = 10
+        self.d2h += self.h_out_fwd.numel() * 2 + self.h_dw.numel() * 4
 
     def step(self):
         la = self.la
@@ -530,12 +535,14 @@ class TrainCase(BackwardCase):
         B, T, H, D = q.shape
         la.lightning_attn_prefill(q, k, v, None, self.y, None, None, block_size=self.C, mode=la.LA_OUT_RAW,
                                   workspace=self.ws)
-        la.lightning_attn_output_transform(self.y.view(B, T, H, D), g, self.out)
-        la.lightning_attn_backward(q, k, v, g, dout, dq, dk, dv, dg=dg, block_size=self.C, workspace=self.ws, y=self.y)
+        la.lightning_attn_output_transform(self.y.view(B, T, H, D), g, self.out, norm_weight=self.nw)
+        la.lightning_attn_backward(q, k, v, g, dout, dq, dk, dv, dg=dg, block_size=self.C, norm_weight=self.nw,
+                                   workspace=self.ws, y=self.y, dnorm_weight=self.dw)
 
     def e2e_step(self):
         super().e2e_step()
         self.h_out_fwd.copy_(self.out, non_blocking=True)
+        self.h_dw.copy_(self.dw, non_blocking=True)
 
     def oracle_sample(self, tokens):
         import oracle
@@ -548,7 +555,8 @@ class TrainCase(BackwardCase):
         return time.perf_counter() - t0
 
     def describe(self):
-        return dict(super().describe(), step="forward (raw prefill + norm/gate, y kept) + backward with y")
+        return dict(super().describe(), grads="dq, dk, dv, dg, dw",
+                    step="forward (raw prefill + norm/gate, y kept) + backward with y")
 
 
 class MixedCase:

@@ -307,7 +307,10 @@ LA_API la_status lightning_attn_decode_step_znorm(const void* q, const void* k, 
  *   dq, dk, dv    [B, T, H, D] dtype, written (none may alias an input or each other).
  *   dg            [B, T, H*D] dtype, written iff mode == LA_OUT_RMSNORM_GATE (else ignored).
  *   dstate_in     fp32 [B, H, D, D] gradient of the initial states, or NULL.
- *   norm_weight   as the forward (its gradient is not computed).
+ *   dnorm_weight  fp32 [H*D], written with the norm weight's gradient summed over all tokens
+ *                 (dw = sum_t dout_t * y_t * r_t [* sigmoid(g_t)], deterministic order), or
+ *                 NULL; zeros in LA_OUT_RAW mode.
+ *   norm_weight   as the forward.
  *   workspace     >= lightning_attn_workspace_size(LA_OP_BACKWARD, B, T, 0, H, D, block_size,
  *                 dtype, mode) bytes, 256-byte aligned; the error record as for the prefill.
  * Other arguments as lightning_attn_prefill (block_size selects the passes' kernel the same
@@ -315,7 +318,8 @@ LA_API la_status lightning_attn_decode_step_znorm(const void* q, const void* k, 
  */
 LA_API la_status lightning_attn_backward(const void* q, const void* k, const void* v, const void* g,
                                          const void* dout, const float* state_in, const float* dstate_out,
-                                         const void* y, void* dq, void* dk, void* dv, void* dg, float* dstate_in, int B, int T, int H, int D, int block_size,
+                                         const void* y, void* dq, void* dk, void* dv, void* dg, float* dstate_in,
+                                         float* dnorm_weight, int B, int T, int H, int D, int block_size,
                                          la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
                                          const float* norm_weight, void* workspace, size_t workspace_bytes,
                                          la_stream_t stream);
@@ -324,14 +328,13 @@ LA_API la_status lightning_attn_backward(const void* q, const void* k, const voi
  * Backward of lightning_attn_prefill_varlen: as lightning_attn_backward over N packed
  * sequences (q, k, v, dq, dk, dv [total, H, D]; g, dout, dg [total, H*D]; cu_seqlens DEVICE
  * int32 [N + 1] as for the forward; state_in, dstate_out, dstate_in [N, H, D, D] or NULL; y
- * [total, H*D] or NULL).  Time is
- * reversed within each sequence.  Workspace: LA_OP_BACKWARD_VARLEN with N, max_seqlen,
+ * [total, H*D] or NULL; dnorm_weight [H*D] or NULL).  Time is reversed within each sequence.  Workspace: LA_OP_BACKWARD_VARLEN with N, max_seqlen,
  * total_tokens.
  */
 LA_API la_status lightning_attn_backward_varlen(const void* q, const void* k, const void* v, const void* g,
                                                 const void* dout, const float* state_in, const float* dstate_out,
                                                 const void* y, void* dq, void* dk, void* dv, void* dg,
-                                                float* dstate_in, const int* cu_seqlens,
+                                                float* dstate_in, float* dnorm_weight, const int* cu_seqlens,
                                                 int num_seqs, int max_seqlen, int total_tokens, int H, int D,
                                                 int block_size, la_dtype dtype, la_feature_map phi,
                                                 la_out_mode mode, float eps, const float* norm_weight,

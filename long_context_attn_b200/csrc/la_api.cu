@@ -33,6 +33,9 @@ cudaError_t launch_bwd_post(const void* q, const void* k, void* dq, void* dk, vo
 cudaError_t launch_transpose_states(const float* in, float* out, int64_t nmat, int D, cudaStream_t stream);
 cudaError_t launch_bwd_feat(const void* q, const void* k, void* fq, void* fk, int64_t elems, int phi_identity,
                             la_dtype dt, cudaStream_t stream);
+int64_t norm_weight_partial_floats(int64_t tokens, int HD);
+cudaError_t launch_bwd_norm_weight(const void* y, const void* g, const void* dout, float* partial, float* dw,
+                                   int64_t tokens, int HD, int gate, float eps, la_dtype dt, cudaStream_t stream);
 cudaError_t launch_bwd_scale(const void* q, const void* k, void* dq, void* dk, int64_t elems, la_dtype dt,
                              cudaStream_t stream);
 int znorm_max_chunks(int max_len);
@@ -241,13 +244,13 @@ MixedLayout mixed_layout(int n, int max_pre, int64_t total, int H, int D, int C,
 }
 
 // Backward workspace: [prefill part of the raw-mode passes (error record first)] [token
-// buffers] [S0^T] [dS_T^T].  The token buffers are dy, phi(k), phi(q) when the tensor-core
+// buffers] [S0^T] [dS_T^T] [dw block partials].  The token buffers are dy, phi(k), phi(q) when the tensor-core
 // kernel walks time backwards itself (rev), else dy, phi(k), rho(v), rho(dy), rho(phi(q)),
 // rho(phi(k)) (rho: each sequence reversed).
 struct BwdLayout {
   bool rev;
   int nbuf;
-  size_t pre, buf, st, total;
+  size_t pre, buf, st, part, total;
 };
 BwdLayout bwd_layout(int nseq, int max_len, int64_t tokens, int H, int D, int C, la_dtype dt) {
   BwdLayout b{};
@@ -257,7 +260,8 @@ BwdLayout bwd_layout(int nseq, int max_len, int64_t tokens, int H, int D, int C,
   b.pre = prefill_ws_bytes(raw, nseq, max_len, tokens, H, D, C, LA_OUT_RAW);
   b.buf = up256(static_cast<size_t>(tokens) * H * D * (dt == LA_BF16 ? 2 : 4));
   b.st = up256(sizeof(float) * static_cast<size_t>(nseq) * H * D * D);
-  b.total = b.pre + b.nbuf * b.buf + 2 * b.st;
+  b.part = up256(sizeof(float) * static_cast<size_t>(la::norm_weight_partial_floats(tokens, H * D)));
+  b.total = b.pre + b.nbuf * b.buf + 2 * b.st + b.part;
   return b;
 }
 
@@ -266,7 +270,7 @@ BwdLayout bwd_layout(int nseq, int max_len, int64_t tokens, int H, int D, int C,
 // raw-mode identity-feature passes of the prefill kernel -> post.
 la_status common_backward(const void* q, const void* k, const void* v, const void* g, const void* dout,
                           const float* state_in, const float* dstate_out, const void* y_saved, void* dq, void* dk,
-                          void* dv, void* dg, float* dstate,
+                          void* dv, void* dg, float* dstate, float* dnorm_weight,
                           const int* cu, int nseq, int T_fixed, int max_len, int64_t tokens, int H, int D, int C,
                           la_dtype dt, la_feature_map phi, la_out_mode mode, float eps, const float* w,
                           void* workspace, size_t ws_bytes, cudaStream_t stream) {
@@ -279,7 +283,8 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
     if (mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g) || !dg || !aligned16(dg))) return LA_ERR_INVALID_ARG;
   }
   if ((state_in && !aligned16(state_in)) || (dstate && !aligned16(dstate)) || (w && !aligned16(w)) ||
-      (dstate_out && !aligned16(dstate_out)) || (y_saved && !aligned16(y_saved)))
+      (dstate_out && !aligned16(dstate_out)) || (y_saved && !aligned16(y_saved)) ||
+      (dnorm_weight && !aligned16(dnorm_weight)))
     return LA_ERR_INVALID_ARG;
   if (!workspace || !aligned256(workspace)) return LA_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(nseq, max_len, tokens, H, D, C, dt);
@@ -290,6 +295,7 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
   for (int i = 0; i < L.nbuf; ++i) buf[i] = base + L.pre + i * L.buf;
   float* s0t = reinterpret_cast<float*>(base + L.pre + L.nbuf * L.buf);
   float* dstt = reinterpret_cast<float*>(base + L.pre + L.nbuf * L.buf + L.st);
+  float* wpart = reinterpret_cast<float*>(base + L.pre + L.nbuf * L.buf + 2 * L.st);
   void *dybuf = buf[0], *fk = buf[1], *rv = buf[2], *rdy = buf[3], *rfq = buf[4], *rfk = buf[5];
   void* fq = buf[2];   // the reverse-time composition's third buffer
   const int HD = H * D;
@@ -301,6 +307,9 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
   };
   la_status st;
   const void* dy = dout;
+  if (dnorm_weight && mode == LA_OUT_RAW &&   // the raw output has no norm weight
+      cudaMemsetAsync(dnorm_weight, 0, sizeof(float) * static_cast<size_t>(HD), stream) != cudaSuccess)
+    return LA_ERR_CUDA;
   if (mode != LA_OUT_RAW) {
     // the forward's raw y (saved by the caller, else recomputed from the same initial
     // state), then dy and dg
@@ -309,6 +318,11 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
       if ((st = pass(q, k, v, dybuf, state_in, nullptr, phi)) != LA_OK) return st;
       yv = dybuf;
     }
+    // the norm weight's gradient reads y before dy may be written over it
+    if (dnorm_weight && la::launch_bwd_norm_weight(yv, g, dout, wpart, dnorm_weight, tokens, HD,
+                                                   mode == LA_OUT_RMSNORM_GATE ? 1 : 0, eps, dt,
+                                                   stream) != cudaSuccess)
+      return LA_ERR_CUDA;
     if (la::launch_bwd_norm_gate(yv, g, dout, w, dybuf, dg, tokens, HD, mode == LA_OUT_RMSNORM_GATE ? 1 : 0, eps, dt,
                                  stream) != cudaSuccess)
       return LA_ERR_CUDA;
@@ -435,30 +449,31 @@ la_status lightning_attn_prefill(const void* q, const void* k, const void* v, co
 
 la_status lightning_attn_backward(const void* q, const void* k, const void* v, const void* g, const void* dout,
                                   const float* state_in, const float* dstate_out, const void* y, void* dq, void* dk,
-                                  void* dv, void* dg, float* dstate_in,
+                                  void* dv, void* dg, float* dstate_in, float* dnorm_weight,
                                   int B, int T, int H, int D, int block_size, la_dtype dtype, la_feature_map phi,
                                   la_out_mode mode, float eps, const float* norm_weight, void* workspace,
                                   size_t workspace_bytes, la_stream_t stream) {
   if (B < 1 || T < 0) return LA_ERR_INVALID_ARG;
   const int64_t tokens = static_cast<int64_t>(B) * T;
   if (tokens > INT32_MAX) return LA_ERR_UNSUPPORTED;
-  return common_backward(q, k, v, g, dout, state_in, dstate_out, y, dq, dk, dv, dg, dstate_in, nullptr, B, T, T,
-                         tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight, workspace, workspace_bytes,
-                         reinterpret_cast<cudaStream_t>(stream));
+  return common_backward(q, k, v, g, dout, state_in, dstate_out, y, dq, dk, dv, dg, dstate_in, dnorm_weight, nullptr,
+                         B, T, T, tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight, workspace,
+                         workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 la_status lightning_attn_backward_varlen(const void* q, const void* k, const void* v, const void* g,
                                          const void* dout, const float* state_in, const float* dstate_out,
-                                         const void* y, void* dq, void* dk, void* dv, void* dg, float* dstate_in, const int* cu_seqlens, int num_seqs,
+                                         const void* y, void* dq, void* dk, void* dv, void* dg, float* dstate_in,
+                                         float* dnorm_weight, const int* cu_seqlens, int num_seqs,
                                          int max_seqlen, int total_tokens, int H, int D, int block_size,
                                          la_dtype dtype, la_feature_map phi, la_out_mode mode, float eps,
                                          const float* norm_weight, void* workspace, size_t workspace_bytes,
                                          la_stream_t stream) {
   if (num_seqs < 1 || !cu_seqlens || !aligned16(cu_seqlens) || total_tokens < 0 || max_seqlen < 0)
     return LA_ERR_INVALID_ARG;
-  return common_backward(q, k, v, g, dout, state_in, dstate_out, y, dq, dk, dv, dg, dstate_in, cu_seqlens, num_seqs,
-                         0, max_seqlen, total_tokens, H, D, block_size, dtype, phi, mode, eps, norm_weight,
-                         workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+  return common_backward(q, k, v, g, dout, state_in, dstate_out, y, dq, dk, dv, dg, dstate_in, dnorm_weight,
+                         cu_seqlens, num_seqs, 0, max_seqlen, total_tokens, H, D, block_size, dtype, phi, mode, eps,
+                         norm_weight, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 la_status lightning_attn_output_transform(const void* y, const void* g, void* out, int tokens, int H, int D,

@@ -115,6 +115,78 @@ __global__ void __launch_bounds__(256) bwd_norm_gate_kernel(const T* y, const T*
   }
 }
 
+// The norm weight's gradient dw_c = sum over tokens of dout_c * y_c * r * s_c, in two
+// deterministic stages.  Stage 1: one CTA per block of kNwTokens tokens, every column (kV
+// 8-element vectors per thread, H*D <= 256 * 8 * kV); per token r from the row's sum of
+// squares (block reduction), then each thread adds its columns' terms in registers; the
+// block's sums go to partial[block][c].  It reads y before the norm/gate backward, which
+// may overwrite y with dy.
+constexpr int kNwTokens = 256;
+template <typename T, int kV>
+__global__ void __launch_bounds__(256) bwd_norm_weight_kernel(const T* __restrict__ y, const T* __restrict__ g,
+                                                              const T* __restrict__ dout, float* __restrict__ partial,
+                                                              int64_t tokens, int HD, int gate, float eps) {
+  __shared__ float red[8];
+  float acc[kV][kVec];
+#pragma unroll
+  for (int i = 0; i < kV; ++i)
+#pragma unroll
+    for (int e = 0; e < kVec; ++e) acc[i][e] = 0.f;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kNwTokens;
+  const int64_t t1 = t0 + kNwTokens < tokens ? t0 + kNwTokens : tokens;
+  for (int64_t t = t0; t < t1; ++t) {
+    const int64_t base = t * HD;
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+      const int c = (threadIdx.x + i * 256) * kVec;
+      if (c < HD) {
+        float yv[kVec];
+        Vec8<T>::load(y + base + c, yv);
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) ss = fmaf(yv[e], yv[e], ss);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tot += red[i];
+    __syncthreads();   // red is rewritten for the next token
+    const float r = 1.0f / sqrtf(tot / static_cast<float>(HD) + eps);
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+      const int c = (threadIdx.x + i * 256) * kVec;
+      if (c < HD) {
+        float yv[kVec], dv[kVec], gv[kVec];
+        Vec8<T>::load(y + base + c, yv);
+        Vec8<T>::load(dout + base + c, dv);
+        if (gate) Vec8<T>::load(g + base + c, gv);
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) acc[i][e] = fmaf(dv[e] * yv[e] * r, gate ? sig(gv[e]) : 1.0f, acc[i][e]);
+      }
+    }
+  }
+  float* out = partial + static_cast<int64_t>(blockIdx.x) * HD;
+#pragma unroll
+  for (int i = 0; i < kV; ++i) {
+    const int c = (threadIdx.x + i * 256) * kVec;
+    if (c < HD) Vec8<float>::store(out + c, acc[i]);
+  }
+}
+
+// Stage 2: dw[c] = sum of the blocks' partials in block order.
+__global__ void __launch_bounds__(256) bwd_norm_weight_sum_kernel(const float* __restrict__ partial, int nblocks,
+                                                                  int HD, float* __restrict__ dw) {
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < HD; c += gridDim.x * blockDim.x) {
+    float a = 0.f;
+    for (int b = 0; b < nblocks; ++b) a += partial[static_cast<int64_t>(b) * HD + c];
+    dw[c] = a;
+  }
+}
+
 // Per 8-element vector of row `row`: fk[row] = phi(k); at the mirrored row m of the same
 // sequence, rv[m] = v, rdy[m] = dy, rfq[m] = phi(q), rfk[m] = phi(k).
 template <typename T>
@@ -304,6 +376,35 @@ cudaError_t launch_bwd_post(const void* q, const void* k, void* dq, void* dk, vo
     bwd_post_kernel<float><<<grid_for(n), 256, 0, stream>>>(
         static_cast<const float*>(q), static_cast<const float*>(k), static_cast<float*>(dq),
         static_cast<float*>(dk), static_cast<float*>(dv), cu, nseq, T_fixed, tokens, HD, phi_identity);
+  return cudaGetLastError();
+}
+
+int64_t norm_weight_partial_floats(int64_t tokens, int HD) {
+  return ((tokens + kNwTokens - 1) / kNwTokens) * HD;
+}
+
+cudaError_t launch_bwd_norm_weight(const void* y, const void* g, const void* dout, float* partial, float* dw,
+                                   int64_t tokens, int HD, int gate, float eps, la_dtype dt, cudaStream_t stream) {
+  const int nb = static_cast<int>((tokens + kNwTokens - 1) / kNwTokens);
+  if (nb > 0) {
+    const int kv = (HD + 256 * kVec - 1) / (256 * kVec);   // vectors per thread (H*D <= 16384: at most 8)
+    if (dt == LA_BF16) {
+      auto a = static_cast<const uint16_t*>(y);
+      auto b = static_cast<const uint16_t*>(g);
+      auto c = static_cast<const uint16_t*>(dout);
+      if (kv <= 4) bwd_norm_weight_kernel<uint16_t, 4><<<nb, 256, 0, stream>>>(a, b, c, partial, tokens, HD, gate, eps);
+      else bwd_norm_weight_kernel<uint16_t, 8><<<nb, 256, 0, stream>>>(a, b, c, partial, tokens, HD, gate, eps);
+    } else {
+      auto a = static_cast<const float*>(y);
+      auto b = static_cast<const float*>(g);
+      auto c = static_cast<const float*>(dout);
+      if (kv <= 4) bwd_norm_weight_kernel<float, 4><<<nb, 256, 0, stream>>>(a, b, c, partial, tokens, HD, gate, eps);
+      else bwd_norm_weight_kernel<float, 8><<<nb, 256, 0, stream>>>(a, b, c, partial, tokens, HD, gate, eps);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  bwd_norm_weight_sum_kernel<<<(HD + 255) / 256, 256, 0, stream>>>(partial, nb, HD, dw);
   return cudaGetLastError();
 }
 

@@ -64,8 +64,8 @@ def _load():
     lib.lightning_attn_prefill_znorm.argtypes = [vp] * 9 + [i32] * 8 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_prefill_znorm_varlen.argtypes = [vp] * 10 + [i32] * 9 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_decode_step_znorm.argtypes = [vp] * 7 + [i32] * 6 + [f32, vp, vp, sz, vp]
-    lib.lightning_attn_backward.argtypes = [vp] * 13 + [i32] * 8 + [f32, vp, vp, sz, vp]
-    lib.lightning_attn_backward_varlen.argtypes = [vp] * 14 + [i32] * 9 + [f32, vp, vp, sz, vp]
+    lib.lightning_attn_backward.argtypes = [vp] * 14 + [i32] * 8 + [f32, vp, vp, sz, vp]
+    lib.lightning_attn_backward_varlen.argtypes = [vp] * 15 + [i32] * 9 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_output_transform.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]
     lib.lightning_attn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp,
                                                sz, vp]
@@ -237,14 +237,15 @@ def lightning_attn_decode_step_znorm(q, k, v, g, out, state, z, phi=LA_PHI_SILU,
 
 def lightning_attn_backward(q, k, v, g, dout, dq, dk, dv, dg=None, state_in=None, dstate_in=None, block_size=256,
                             phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE, eps=1e-6, norm_weight=None, workspace=None,
-                            stream=None, dstate_out=None, y=None):
+                            stream=None, dstate_out=None, y=None, dnorm_weight=None):
     """q, k, v, dq, dk, dv [B, T, H, D]; g, dout, dg [B, T, H*D]; states fp32 [B, H, D, D]
-    (dstate_out: the gradient reaching the final states; y: the forward's raw output, saved)."""
+    (dstate_out: the gradient reaching the final states; y: the forward's raw output, saved;
+    dnorm_weight: fp32 [H*D] receiving the norm weight's gradient)."""
     B, T, H, D = q.shape
     _check_contig(q, k, v, g, dout, dq, dk, dv, dg, dstate_out, y)
     st = _lib.lightning_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout), _ptr(_f32_or_none(state_in)),
                                       _ptr(_f32_or_none(dstate_out)), _ptr(y), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
-                                      _ptr(_f32_or_none(dstate_in)), B, T, H,
+                                      _ptr(_f32_or_none(dstate_in)), _ptr(_f32_or_none(dnorm_weight)), B, T, H,
                                       D, block_size, _dtype(q), phi, mode, eps, _ptr(_f32_or_none(norm_weight)),
                                       _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                       _stream(stream))
@@ -255,7 +256,7 @@ def lightning_attn_backward(q, k, v, g, dout, dq, dk, dv, dg=None, state_in=None
 def lightning_attn_backward_varlen(q, k, v, g, dout, dq, dk, dv, cu_seqlens, max_seqlen, dg=None, state_in=None,
                                    dstate_in=None, block_size=256, phi=LA_PHI_SILU, mode=LA_OUT_RMSNORM_GATE,
                                    eps=1e-6, norm_weight=None, workspace=None, stream=None, dstate_out=None,
-                                   y=None):
+                                   y=None, dnorm_weight=None):
     """q, k, v, dq, dk, dv [total, H, D]; g, dout, dg [total, H*D]; cu_seqlens int32 device [N + 1]."""
     total, H, D = q.shape
     _check_contig(q, k, v, g, dout, dq, dk, dv, dg, cu_seqlens, dstate_out, y)
@@ -265,7 +266,8 @@ def lightning_attn_backward_varlen(q, k, v, g, dout, dq, dk, dv, cu_seqlens, max
     st = _lib.lightning_attn_backward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout),
                                              _ptr(_f32_or_none(state_in)), _ptr(_f32_or_none(dstate_out)), _ptr(y),
                                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
-                                             _ptr(_f32_or_none(dstate_in)), _ptr(cu_seqlens), n, int(max_seqlen),
+                                             _ptr(_f32_or_none(dstate_in)), _ptr(_f32_or_none(dnorm_weight)),
+                                             _ptr(cu_seqlens), n, int(max_seqlen),
                                              total, H, D, block_size, _dtype(q), phi, mode, eps,
                                              _ptr(_f32_or_none(norm_weight)), _ptr(workspace),
                                              0 if workspace is None else workspace.numel(), _stream(stream))

@@ -126,15 +126,15 @@ def test_backward_host_checks(lib):
     holds the raw-pass prefill part plus six token buffers and the transposed states."""
     vp, i32 = ctypes.c_void_p, ctypes.c_int
     f = lib.lightning_attn_backward
-    f.argtypes = [vp] * 13 + [i32] * 8 + [ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
+    f.argtypes = [vp] * 14 + [i32] * 8 + [ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
     fake, ws = vp(0x1000), vp(0x100000)
 
     def call(**kw):
         a = dict(q=fake, k=fake, v=fake, g=fake, dout=fake, s0=None, dsT=None, y=None, dq=fake, dk=fake, dv=fake,
-                 dg=fake, ds=None, B=1, T=64, H=2, D=128, C=256, dt=1, phi=0, mode=2, ws=ws, nbytes=1 << 40)
+                 dg=fake, ds=None, dw=None, B=1, T=64, H=2, D=128, C=256, dt=1, phi=0, mode=2, ws=ws, nbytes=1 << 40)
         a.update(kw)
         return f(a["q"], a["k"], a["v"], a["g"], a["dout"], a["s0"], a["dsT"], a["y"], a["dq"], a["dk"], a["dv"],
-                 a["dg"], a["ds"],
+                 a["dg"], a["ds"], a["dw"],
                  a["B"], a["T"], a["H"], a["D"], a["C"], a["dt"], a["phi"], a["mode"], ctypes.c_float(1e-6), None,
                  a["ws"], a["nbytes"], None)
 
@@ -147,6 +147,7 @@ def test_backward_host_checks(lib):
     assert call(nbytes=1024) == 1         # workspace too small
     assert call(dsT=vp(0x1008)) == 1      # misaligned final-state gradient
     assert call(y=vp(0x1008)) == 1        # misaligned saved output
+    assert call(dw=vp(0x1008)) == 1       # misaligned norm-weight gradient
     lib.lightning_attn_workspace_size.restype = ctypes.c_size_t
     fwd = lib.lightning_attn_workspace_size(0, 2, 1000, 0, 8, 128, 256, 1, 0)
     bwd = lib.lightning_attn_workspace_size(4, 2, 1000, 0, 8, 128, 256, 1, 2)

@@ -57,3 +57,23 @@ def test_autograd_through_the_carried_state(cuda_device):
     ref = oracle.backward(q[None], k[None], v[None], g[None], dout[None])
     for t, want, name in zip((tq, tk, tv, tg), ref, ("dq", "dk", "dv", "dg")):
         assert_close(to_host(t.grad), want.reshape(to_host(t.grad).shape), "bf16", name)
+
+
+def test_autograd_norm_weight_gradient(cuda_device):
+    """A norm weight that requires grad gets dw = sum_t dout_t * y_t * r_t * sigmoid(g_t)."""
+    import torch
+    from long_context_attn_b200.autograd import lightning_attention
+    B, T, H, D = 1, 520, 8, 128
+    q, k, v, g = synth.prefill_inputs(3721, T, H, D, "bf16", 0.5, True)
+    dout = synth.f32_to_bf16(synth.normal(3721, 21, (T, H * D), 1.0, "f32"))
+    w = (1.0 + 0.2 * synth.normal(3721, 23, (H * D,), 1.0, "f32")).astype(np.float32)
+    shp, gshp = (B, T, H, D), (B, T, H * D)
+    tq, tk, tv = (_leaf(a, shp) for a in (q, k, v))
+    tg = _leaf(g, gshp)
+    tw = torch.from_numpy(w).cuda().requires_grad_(True)
+    out, _ = lightning_attention(tq, tk, tv, tg, norm_weight=tw)
+    (out.float() * to_dev(dout).reshape(gshp).float()).sum().backward()
+    ref = oracle.backward(q.reshape(shp), k.reshape(shp), v.reshape(shp), g.reshape(gshp), dout.reshape(gshp),
+                          norm_weight=w)
+    for t, want, name in zip((tq, tk, tv, tg, tw), ref[:4] + ref[5:], ("dq", "dk", "dv", "dg", "dw")):
+        assert_close(to_host(t.grad), want.reshape(to_host(t.grad).shape), "bf16", name)

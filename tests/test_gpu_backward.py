@@ -1,7 +1,7 @@
 """GPU parity of the backward pass against the oracle's fp64 gradients.
 
-Every gradient (dq, dk, dv, the gate's dg and the initial state's dS0) is compared element
-by element with the oracle (which finite differences of the forward pin) at the forward's
+Every gradient (dq, dk, dv, the gate's dg, the initial state's dS0 and the norm weight's dw)
+is compared element by element with the oracle (which finite differences of the forward pin) at the forward's
 tolerance: bf16 2e-2 * max|ref|, fp32 1e-4 * max|ref|.  Cases span several blocks with a
 ragged tail, both tensor-core block sizes, the three output modes, a norm weight, initial
 states, packed sequences with an empty and a one-token sequence, and the fp32 path.
@@ -37,11 +37,12 @@ def _run_fixed(B, T, H, D, C, dtype, mode, with_state, seed, expect=None):
     gq, gk, gv = (torch.full_like(dq_, float("nan")) for _ in range(3))
     gg = torch.full_like(dg_, float("nan")) if m == la.LA_OUT_RMSNORM_GATE else None
     gs = torch.full((B, H, D, D), float("nan"), dtype=torch.float32, device="cuda")
+    gw = torch.full((H * D,), float("nan"), dtype=torch.float32, device="cuda")
     ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD, B, T, 0, H, D, C, la._dtype(dq_), m))
     la.lightning_attn_backward(dq_, dk_, dv_, dg_ if m == la.LA_OUT_RMSNORM_GATE else None, ddo, gq, gk, gv, dg=gg,
                                state_in=None if s0 is None else to_dev(s0), dstate_in=gs, block_size=C, mode=m,
                                norm_weight=None if w is None else to_dev(w), workspace=ws,
-                               dstate_out=None if dsT is None else to_dev(dsT))
+                               dstate_out=None if dsT is None else to_dev(dsT), dnorm_weight=gw)
     if expect:
         assert la.lightning_attn_last_path() == expect
     la.lightning_attn_check(ws)
@@ -54,6 +55,10 @@ def _run_fixed(B, T, H, D, C, dtype, mode, with_state, seed, expect=None):
     if gg is not None:
         assert_close(to_host(gg), ref[3], dtype, "dg")
     assert_close(to_host(gs), ref[4], dtype, "dstate")
+    if m == la.LA_OUT_RAW:
+        assert torch.all(gw == 0), "dw must be zero in raw mode"
+    else:
+        assert_close(to_host(gw), ref[5], dtype, "dw")
 
 
 @pytest.mark.parametrize("C", [128, 256])
@@ -88,15 +93,17 @@ def test_backward_varlen(C, cuda_device):
     gq, gk, gv = (torch.full_like(dq_, float("nan")) for _ in range(3))
     gg = torch.full_like(dg_, float("nan"))
     gs = torch.full((n, H, D, D), float("nan"), dtype=torch.float32, device="cuda")
+    gw = torch.full((H * D,), float("nan"), dtype=torch.float32, device="cuda")
+    w = (1.0 + 0.2 * synth.normal(3301, 23, (H * D,), 1.0, "f32")).astype(np.float32)
     ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_BACKWARD_VARLEN, n, max(lens), tot, H, D, C,
                                                            la.LA_BF16, la.LA_OUT_RMSNORM_GATE))
     la.lightning_attn_backward_varlen(dq_, dk_, dv_, dg_, ddo, gq, gk, gv, torch.from_numpy(cu).cuda(), max(lens),
                                       dg=gg, state_in=to_dev(s0), dstate_in=gs, block_size=C, workspace=ws,
-                                      dstate_out=to_dev(dsT))
+                                      dstate_out=to_dev(dsT), norm_weight=to_dev(w), dnorm_weight=gw)
     assert la.lightning_attn_last_path() == "tcgen05"
     la.lightning_attn_check(ws)
-    ref = oracle.backward_packed(q, k, v, g, dout, cu, H, D, state_in=s0, dstate_out=dsT)
-    for got, want, name in zip((gq, gk, gv, gg, gs), ref, ("dq", "dk", "dv", "dg", "dstate")):
+    ref = oracle.backward_packed(q, k, v, g, dout, cu, H, D, state_in=s0, dstate_out=dsT, norm_weight=w)
+    for got, want, name in zip((gq, gk, gv, gg, gs, gw), ref, ("dq", "dk", "dv", "dg", "dstate", "dw")):
         assert_close(to_host(got), want, "bf16", name)
 
 
@@ -212,10 +219,11 @@ def test_backward_with_saved_y_equals_recompute(mode, cuda_device):
     for yy in (None, y):
         gq, gk, gv = (torch.empty_like(dq_) for _ in range(3))
         gg = torch.empty_like(dg_) if gate is not None else None
+        gw = torch.empty((H * D,), dtype=torch.float32, device="cuda")
         la.lightning_attn_backward(dq_, dk_, dv_, gate, ddo, gq, gk, gv, dg=gg, block_size=C, mode=m, workspace=ws,
-                                   y=yy)
+                                   y=yy, dnorm_weight=gw)
         la.lightning_attn_check(ws)
-        res.append([to_host(t) for t in (gq, gk, gv) + ((gg,) if gg is not None else ())])
+        res.append([to_host(t) for t in (gq, gk, gv, gw) + ((gg,) if gg is not None else ())])
     for a, b in zip(*res):
         np.testing.assert_array_equal(a, b)
     # and the output transform of the kept y is the fused forward's output (tolerance: y is
@@ -225,6 +233,12 @@ def test_backward_with_saved_y_equals_recompute(mode, cuda_device):
     ref, _, _ = oracle.prefill(q.reshape(shp), k.reshape(shp), v.reshape(shp),
                                g.reshape(gshp) if gate is not None else None, mode=m)
     assert_close(to_host(out), ref, "bf16")
+
+
+def test_backward_wide_rows_norm_weight(cuda_device):
+    """H*D = 10240 (more than 4 vectors of 8 per thread in the norm-weight reduction) over
+    300 tokens (a full block of 256 tokens and a ragged one)."""
+    _run_fixed(1, 300, 80, 128, 256, "bf16", "rmsnorm_gate", False, 3951)
 
 
 def test_backward_long_sequence_few_heads_splits_every_pass(cuda_device):
