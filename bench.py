@@ -776,7 +776,7 @@ def run_gpu(args):
                               "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": _traffic(args.workload),
                               "peak_source": peaks["source"], "launch_ms": launch_ms,
                               "algorithmic_bytes_per_launch": case.alg_bytes},
-                             **({"scope": "one training step (forward + backward, 8 kernels); algorithmic "
+                             **({"scope": "one training step (forward + backward with dw, 10 kernels); algorithmic "
                                           "bytes = both calls' inputs read and outputs written once"}
                                 if isinstance(case, TrainCase) else
                                 {"scope": "one backward call (7 kernels); algorithmic bytes = its inputs "

@@ -24,7 +24,8 @@ cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, voi
 cudaError_t launch_norm_gate(const float* y, const void* g, void* out, int64_t tokens, int HD, int mode,
                              float eps, const float* w, la_dtype dt, cudaStream_t stream);
 cudaError_t launch_bwd_norm_gate(const void* y, const void* g, const void* dout, const float* w, void* dy, void* dg,
-                                 int64_t tokens, int HD, int gate, float eps, la_dtype dt, cudaStream_t stream);
+                                 float* partial, float* dw, int64_t tokens, int HD, int gate, float eps, la_dtype dt,
+                                 cudaStream_t stream);
 cudaError_t launch_bwd_prep(const void* q, const void* k, const void* v, const void* dy, void* fk, void* rv,
                             void* rdy, void* rfq, void* rfk, const int* cu, int nseq, int T_fixed, int64_t tokens,
                             int HD, int phi_identity, la_dtype dt, cudaStream_t stream);
@@ -34,8 +35,6 @@ cudaError_t launch_transpose_states(const float* in, float* out, int64_t nmat, i
 cudaError_t launch_bwd_feat(const void* q, const void* k, void* fq, void* fk, int64_t elems, int phi_identity,
                             la_dtype dt, cudaStream_t stream);
 int64_t norm_weight_partial_floats(int64_t tokens, int HD);
-cudaError_t launch_bwd_norm_weight(const void* y, const void* g, const void* dout, float* partial, float* dw,
-                                   int64_t tokens, int HD, int gate, float eps, la_dtype dt, cudaStream_t stream);
 cudaError_t launch_bwd_scale(const void* q, const void* k, void* dq, void* dk, int64_t elems, la_dtype dt,
                              cudaStream_t stream);
 int znorm_max_chunks(int max_len);
@@ -318,13 +317,9 @@ la_status common_backward(const void* q, const void* k, const void* v, const voi
       if ((st = pass(q, k, v, dybuf, state_in, nullptr, phi)) != LA_OK) return st;
       yv = dybuf;
     }
-    // the norm weight's gradient reads y before dy may be written over it
-    if (dnorm_weight && la::launch_bwd_norm_weight(yv, g, dout, wpart, dnorm_weight, tokens, HD,
-                                                   mode == LA_OUT_RMSNORM_GATE ? 1 : 0, eps, dt,
-                                                   stream) != cudaSuccess)
-      return LA_ERR_CUDA;
-    if (la::launch_bwd_norm_gate(yv, g, dout, w, dybuf, dg, tokens, HD, mode == LA_OUT_RMSNORM_GATE ? 1 : 0, eps, dt,
-                                 stream) != cudaSuccess)
+    // dy and dg, and the norm weight's gradient when asked for
+    if (la::launch_bwd_norm_gate(yv, g, dout, w, dybuf, dg, wpart, dnorm_weight, tokens, HD,
+                                 mode == LA_OUT_RMSNORM_GATE ? 1 : 0, eps, dt, stream) != cudaSuccess)
       return LA_ERR_CUDA;
     dy = dybuf;
   }

@@ -14,7 +14,8 @@
 // run on the time-reversed sequences (queries rho(v), keys rho(dy), values rho(phi(q)); and
 // queries rho(phi(k)), keys rho(phi(q)), values rho(dy), whose final state is dS0).  The
 // kernels here supply what those passes take and finish what they give:
-//   bwd_norm_gate_kernel  dy and dg from dout through RMSNorm(y) * w * sigmoid(g) (per token)
+//   bwd_norm_gate_token_kernel  dy and dg from dout through RMSNorm(y) * w * sigmoid(g)
+//   bwd_norm_gate_kernel  the same with the norm weight's gradient (CTAs over blocks of tokens)
 //   bwd_prep_kernel       phi(k) and the reversed copies rho(v), rho(dy), rho(phi(q)), rho(phi(k))
 //   bwd_post_kernel       dq = dphi(q) * phi'(q); un-reverses dk (times phi'(k)) and dv in place
 //   transpose_states      S0^T for the first pass
@@ -62,12 +63,12 @@ __device__ __forceinline__ void seq_bounds(const int* cu, int nseq, int T_fixed,
   hi = __ldg(cu + a + 1);
 }
 
-// One CTA per token.  RAW is not launched (dy = dout).  With r = 1/sqrt(mean(y^2) + eps),
-// s = sigmoid(g) (1 without the gate) and u = dout * w * s:
-//   dy = r u - r^3 y (sum u y) / HD,    dg = dout * y * r * w * s * (1 - s).
-// y and dy may be the same buffer (each element is read by the thread that writes it).
+// dy and dg alone (no dw), one CTA per token: many short CTAs per SM keep more rows in
+// flight than the token-blocked kernel below can, whose raw vectors fill the registers
+// (measured on the 128K-token, H*D = 8192 backward: 2.7 ms against 3.4 ms).  Same formulas;
+// the second loop re-reads the row (from L1/L2).
 template <typename T>
-__global__ void __launch_bounds__(256) bwd_norm_gate_kernel(const T* y, const T* __restrict__ g,
+__global__ void __launch_bounds__(256) bwd_norm_gate_token_kernel(const T* y, const T* __restrict__ g,
                                                             const T* __restrict__ dout, const float* __restrict__ w,
                                                             T* dy, T* __restrict__ dg, int HD, int gate, float eps) {
   __shared__ float red[2][8];
@@ -115,69 +116,113 @@ __global__ void __launch_bounds__(256) bwd_norm_gate_kernel(const T* y, const T*
   }
 }
 
-// The norm weight's gradient dw_c = sum over tokens of dout_c * y_c * r * s_c, in two
-// deterministic stages.  Stage 1: one CTA per block of kNwTokens tokens, every column (kV
-// 8-element vectors per thread, H*D <= 256 * 8 * kV); per token r from the row's sum of
-// squares (block reduction), then each thread adds its columns' terms in registers; the
-// block's sums go to partial[block][c].  It reads y before the norm/gate backward, which
-// may overwrite y with dy.
-constexpr int kNwTokens = 256;
+// The norm/gate backward with the norm weight's gradient, in one pass over the tokens.  RAW
+// is not launched (dy = dout).  With r = 1/sqrt(mean(y^2) + eps), s = sigmoid(g) (1 without
+// the gate) and u = dout * w * s, per token:
+//   dy = r u - r^3 y (sum u y) / HD,    dg = dout * y * r * w * s * (1 - s),
+// and per column dw_c = sum over tokens of dout_c * y_c * r * s_c.
+// CTA b takes the contiguous tokens [b * per, min((b + 1) * per, tokens)); thread j owns the
+// columns (j + i * blockDim.x) * 8 .. + 7, i < kV.  Per token each thread loads its vectors of
+// y, dout and g once (kept raw in registers), the CTA reduces sum(y^2) and sum(u y), and the
+// thread writes dy and dg and adds its dw terms in registers.  Several CTAs per SM keep
+// enough loads in flight; the reduction buffer alternates between two halves by token
+// parity, so one barrier per token suffices.  With `partial` set, the CTA's dw column sums
+// go to partial[b] (summed over b in order by bwd_norm_weight_sum_kernel: deterministic).
+// y and dy may be the same buffer (each element is read by the thread that writes it).
 template <typename T, int kV>
-__global__ void __launch_bounds__(256) bwd_norm_weight_kernel(const T* __restrict__ y, const T* __restrict__ g,
-                                                              const T* __restrict__ dout, float* __restrict__ partial,
-                                                              int64_t tokens, int HD, int gate, float eps) {
-  __shared__ float red[8];
+__global__ void __launch_bounds__(512) bwd_norm_gate_kernel(const T* y, const T* __restrict__ g,
+                                                            const T* __restrict__ dout, const float* __restrict__ w,
+                                                            T* dy, T* __restrict__ dg, float* __restrict__ partial,
+                                                            int64_t tokens, int64_t per, int HD, int gate, float eps) {
+  using Raw = typename Vec8<T>::Raw;
+  __shared__ float2 red[2][16];
+  const int nwarp = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * per;
+  const int64_t t1 = t0 + per < tokens ? t0 + per : tokens;
+  const float inv_hd = 1.0f / static_cast<float>(HD);
   float acc[kV][kVec];
 #pragma unroll
   for (int i = 0; i < kV; ++i)
 #pragma unroll
     for (int e = 0; e < kVec; ++e) acc[i][e] = 0.f;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kNwTokens;
-  const int64_t t1 = t0 + kNwTokens < tokens ? t0 + kNwTokens : tokens;
-  for (int64_t t = t0; t < t1; ++t) {
+  int par = 0;
+  for (int64_t t = t0; t < t1; ++t, par ^= 1) {
     const int64_t base = t * HD;
-    float ss = 0.f;
+    Raw ry[kV], rd[kV], rg[kV];
 #pragma unroll
     for (int i = 0; i < kV; ++i) {
-      const int c = (threadIdx.x + i * 256) * kVec;
+      const int c = (threadIdx.x + i * blockDim.x) * kVec;
       if (c < HD) {
-        float yv[kVec];
-        Vec8<T>::load(y + base + c, yv);
+        ry[i] = Vec8<T>::load_raw(y + base + c);
+        rd[i] = Vec8<T>::load_raw(dout + base + c);
+        if (gate) rg[i] = Vec8<T>::load_raw(g + base + c);
+      }
+    }
+    float ss = 0.f, su = 0.f;
 #pragma unroll
-        for (int e = 0; e < kVec; ++e) ss = fmaf(yv[e], yv[e], ss);
+    for (int i = 0; i < kV; ++i) {
+      const int c = (threadIdx.x + i * blockDim.x) * kVec;
+      if (c < HD) {
+        float yv[kVec], dv[kVec], gv[kVec];
+        Vec8<T>::unpack(ry[i], yv);
+        Vec8<T>::unpack(rd[i], dv);
+        if (gate) Vec8<T>::unpack(rg[i], gv);
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) {
+          const float u = dv[e] * (w ? __ldg(w + c + e) : 1.0f) * (gate ? sig(gv[e]) : 1.0f);
+          ss = fmaf(yv[e], yv[e], ss);
+          su = fmaf(u, yv[e], su);
+        }
       }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    for (int o = 16; o > 0; o >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      su += __shfl_xor_sync(0xffffffffu, su, o);
+    }
+    if (lane == 0) red[par][warp] = make_float2(ss, su);
     __syncthreads();
-    float tot = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) tot += red[i];
-    __syncthreads();   // red is rewritten for the next token
-    const float r = 1.0f / sqrtf(tot / static_cast<float>(HD) + eps);
+    ss = 0.f;
+    su = 0.f;
+    for (int i = 0; i < nwarp; ++i) {
+      const float2 x = red[par][i];
+      ss += x.x;
+      su += x.y;
+    }
+    const float r = 1.0f / sqrtf(ss * inv_hd + eps);
+    const float coef = r * r * r * su * inv_hd;
 #pragma unroll
     for (int i = 0; i < kV; ++i) {
-      const int c = (threadIdx.x + i * 256) * kVec;
+      const int c = (threadIdx.x + i * blockDim.x) * kVec;
       if (c < HD) {
-        float yv[kVec], dv[kVec], gv[kVec];
-        Vec8<T>::load(y + base + c, yv);
-        Vec8<T>::load(dout + base + c, dv);
-        if (gate) Vec8<T>::load(g + base + c, gv);
+        float yv[kVec], dv[kVec], gv[kVec], o[kVec], og[kVec];
+        Vec8<T>::unpack(ry[i], yv);
+        Vec8<T>::unpack(rd[i], dv);
+        if (gate) Vec8<T>::unpack(rg[i], gv);
 #pragma unroll
-        for (int e = 0; e < kVec; ++e) acc[i][e] = fmaf(dv[e] * yv[e] * r, gate ? sig(gv[e]) : 1.0f, acc[i][e]);
+        for (int e = 0; e < kVec; ++e) {
+          const float sg = gate ? sig(gv[e]) : 1.0f;
+          const float wc = w ? __ldg(w + c + e) : 1.0f;
+          const float n = dv[e] * yv[e] * r * sg;   // dout * y * r * s: dw's term
+          o[e] = r * dv[e] * wc * sg - coef * yv[e];
+          og[e] = n * wc * (1.0f - sg);
+          acc[i][e] += n;
+        }
+        Vec8<T>::store(dy + base + c, o);
+        if (gate) Vec8<T>::store(dg + base + c, og);
       }
     }
   }
+  if (!partial) return;
   float* out = partial + static_cast<int64_t>(blockIdx.x) * HD;
 #pragma unroll
   for (int i = 0; i < kV; ++i) {
-    const int c = (threadIdx.x + i * 256) * kVec;
+    const int c = (threadIdx.x + i * blockDim.x) * kVec;
     if (c < HD) Vec8<float>::store(out + c, acc[i]);
   }
 }
 
-// Stage 2: dw[c] = sum of the blocks' partials in block order.
+// dw[c] = sum of the CTAs' partial sums in CTA order.
 __global__ void __launch_bounds__(256) bwd_norm_weight_sum_kernel(const float* __restrict__ partial, int nblocks,
                                                                   int HD, float* __restrict__ dw) {
   for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < HD; c += gridDim.x * blockDim.x) {
@@ -329,20 +374,88 @@ int grid_for(int64_t n) {
   return static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
 }
 
+// The norm/gate kernel's launch shape: kvmax vectors of 8 per thread at most (4 of bf16, 2
+// of fp32: the raw vectors stay in registers), threads a multiple of 32 (<= 512), kV = the
+// vectors each thread takes; CTAs = the resident CTAs of the whole GPU (at most
+// kNormGateMaxBlocks, at most one per token).
+constexpr int kNormGateMaxBlocks = 1024;
+struct NormGateShape {
+  int threads, kv;
+};
+NormGateShape norm_gate_shape(int HD, int kvmax) {
+  const int vecs = HD / kVec;
+  int threads = (vecs + kvmax - 1) / kvmax;
+  threads = ((threads + 31) / 32) * 32;
+  if (threads > 512) threads = 512;
+  return {threads, (vecs + threads - 1) / threads};
+}
+
+}  // namespace
+
+int64_t norm_weight_partial_floats(int64_t tokens, int HD) {
+  const int64_t nb = tokens < kNormGateMaxBlocks ? tokens : kNormGateMaxBlocks;
+  return nb * HD;
+}
+
+namespace {
+template <typename T, int kV>
+cudaError_t launch_norm_gate_t(const void* y, const void* g, const void* dout, const float* w, void* dy, void* dg,
+                               float* partial, float* dw, int64_t tokens, int threads, int HD, int gate, float eps,
+                               cudaStream_t stream) {
+  auto kern = bwd_norm_gate_kernel<T, kV>;
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
+  if (e != cudaSuccess) return e;
+  int64_t nb = static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1);
+  if (nb > kNormGateMaxBlocks) nb = kNormGateMaxBlocks;
+  if (nb > tokens) nb = tokens;
+  const int64_t per = (tokens + nb - 1) / nb;
+  nb = (tokens + per - 1) / per;
+  kern<<<static_cast<unsigned>(nb), threads, 0, stream>>>(static_cast<const T*>(y), static_cast<const T*>(g),
+                                                          static_cast<const T*>(dout), w, static_cast<T*>(dy),
+                                                          static_cast<T*>(dg), dw ? partial : nullptr, tokens, per,
+                                                          HD, gate, eps);
+  if ((e = cudaGetLastError()) != cudaSuccess || !dw) return e;
+  bwd_norm_weight_sum_kernel<<<(HD + 255) / 256, 256, 0, stream>>>(partial, static_cast<int>(nb), HD, dw);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_norm_gate_dt(const void* y, const void* g, const void* dout, const float* w, void* dy, void* dg,
+                                float* partial, float* dw, int64_t tokens, int HD, int gate, float eps,
+                                cudaStream_t stream) {
+  const NormGateShape sh = norm_gate_shape(HD, sizeof(T) == 2 ? 4 : 2);
+  switch (sh.kv) {
+    case 1: return launch_norm_gate_t<T, 1>(y, g, dout, w, dy, dg, partial, dw, tokens, sh.threads, HD, gate, eps, stream);
+    case 2: return launch_norm_gate_t<T, 2>(y, g, dout, w, dy, dg, partial, dw, tokens, sh.threads, HD, gate, eps, stream);
+    case 3: return launch_norm_gate_t<T, 3>(y, g, dout, w, dy, dg, partial, dw, tokens, sh.threads, HD, gate, eps, stream);
+    default: return launch_norm_gate_t<T, 4>(y, g, dout, w, dy, dg, partial, dw, tokens, sh.threads, HD, gate, eps, stream);
+  }
+}
 }  // namespace
 
 cudaError_t launch_bwd_norm_gate(const void* y, const void* g, const void* dout, const float* w, void* dy, void* dg,
-                                 int64_t tokens, int HD, int gate, float eps, la_dtype dt, cudaStream_t stream) {
-  if (tokens == 0) return cudaSuccess;
-  if (dt == LA_BF16)
-    bwd_norm_gate_kernel<uint16_t><<<static_cast<unsigned>(tokens), 256, 0, stream>>>(
-        static_cast<const uint16_t*>(y), static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(dout), w,
-        static_cast<uint16_t*>(dy), static_cast<uint16_t*>(dg), HD, gate, eps);
-  else
-    bwd_norm_gate_kernel<float><<<static_cast<unsigned>(tokens), 256, 0, stream>>>(
-        static_cast<const float*>(y), static_cast<const float*>(g), static_cast<const float*>(dout), w,
-        static_cast<float*>(dy), static_cast<float*>(dg), HD, gate, eps);
-  return cudaGetLastError();
+                                 float* partial, float* dw, int64_t tokens, int HD, int gate, float eps, la_dtype dt,
+                                 cudaStream_t stream) {
+  if (tokens == 0) {   // no tokens: the gradient of the norm weight is zero
+    if (dw) bwd_norm_weight_sum_kernel<<<(HD + 255) / 256, 256, 0, stream>>>(partial, 0, HD, dw);
+    return cudaGetLastError();
+  }
+  if (!dw) {
+    if (dt == LA_BF16)
+      bwd_norm_gate_token_kernel<uint16_t><<<static_cast<unsigned>(tokens), 256, 0, stream>>>(
+          static_cast<const uint16_t*>(y), static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(dout), w,
+          static_cast<uint16_t*>(dy), static_cast<uint16_t*>(dg), HD, gate, eps);
+    else
+      bwd_norm_gate_token_kernel<float><<<static_cast<unsigned>(tokens), 256, 0, stream>>>(
+          static_cast<const float*>(y), static_cast<const float*>(g), static_cast<const float*>(dout), w,
+          static_cast<float*>(dy), static_cast<float*>(dg), HD, gate, eps);
+    return cudaGetLastError();
+  }
+  if (dt == LA_BF16) return launch_norm_gate_dt<uint16_t>(y, g, dout, w, dy, dg, partial, dw, tokens, HD, gate, eps, stream);
+  return launch_norm_gate_dt<float>(y, g, dout, w, dy, dg, partial, dw, tokens, HD, gate, eps, stream);
 }
 
 cudaError_t launch_bwd_prep(const void* q, const void* k, const void* v, const void* dy, void* fk, void* rv,
@@ -376,35 +489,6 @@ cudaError_t launch_bwd_post(const void* q, const void* k, void* dq, void* dk, vo
     bwd_post_kernel<float><<<grid_for(n), 256, 0, stream>>>(
         static_cast<const float*>(q), static_cast<const float*>(k), static_cast<float*>(dq),
         static_cast<float*>(dk), static_cast<float*>(dv), cu, nseq, T_fixed, tokens, HD, phi_identity);
-  return cudaGetLastError();
-}
-
-int64_t norm_weight_partial_floats(int64_t tokens, int HD) {
-  return ((tokens + kNwTokens - 1) / kNwTokens) * HD;
-}
-
-cudaError_t launch_bwd_norm_weight(const void* y, const void* g, const void* dout, float* partial, float* dw,
-                                   int64_t tokens, int HD, int gate, float eps, la_dtype dt, cudaStream_t stream) {
-  const int nb = static_cast<int>((tokens + kNwTokens - 1) / kNwTokens);
-  if (nb > 0) {
-    const int kv = (HD + 256 * kVec - 1) / (256 * kVec);   // vectors per thread (H*D <= 16384: at most 8)
-    if (dt == LA_BF16) {
-      auto a = static_cast<const uint16_t*>(y);
-      auto b = static_cast<const uint16_t*>(g);
-      auto c = static_cast<const uint16_t*>(dout);
-      if (kv <= 4) bwd_norm_weight_kernel<uint16_t, 4><<<nb, 256, 0, stream>>>(a, b, c, partial, tokens, HD, gate, eps);
-      else bwd_norm_weight_kernel<uint16_t, 8><<<nb, 256, 0, stream>>>(a, b, c, partial, tokens, HD, gate, eps);
-    } else {
-      auto a = static_cast<const float*>(y);
-      auto b = static_cast<const float*>(g);
-      auto c = static_cast<const float*>(dout);
-      if (kv <= 4) bwd_norm_weight_kernel<float, 4><<<nb, 256, 0, stream>>>(a, b, c, partial, tokens, HD, gate, eps);
-      else bwd_norm_weight_kernel<float, 8><<<nb, 256, 0, stream>>>(a, b, c, partial, tokens, HD, gate, eps);
-    }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  bwd_norm_weight_sum_kernel<<<(HD + 255) / 256, 256, 0, stream>>>(partial, nb, HD, dw);
   return cudaGetLastError();
 }
 

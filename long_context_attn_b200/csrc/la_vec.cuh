@@ -6,9 +6,12 @@
 namespace la {
 
 template <typename T> struct Vec8;
+// Raw: the vector as loaded (kept in registers until it is needed as floats).
 template <> struct Vec8<uint16_t> {
-  __device__ __forceinline__ static void load(const uint16_t* p, float* f) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
+  using Raw = uint4;
+  __device__ __forceinline__ static Raw load_raw(const uint16_t* p) { return *reinterpret_cast<const uint4*>(p); }
+  __device__ __forceinline__ static void load(const uint16_t* p, float* f) { unpack(load_raw(p), f); }
+  __device__ __forceinline__ static void unpack(const Raw& u, float* f) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -26,11 +29,16 @@ template <> struct Vec8<uint16_t> {
   }
 };
 template <> struct Vec8<float> {
-  __device__ __forceinline__ static void load(const float* p, float* f) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    const float4 b = *reinterpret_cast<const float4*>(p + 4);
-    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  struct Raw {
+    float4 a, b;
+  };
+  __device__ __forceinline__ static Raw load_raw(const float* p) {
+    return Raw{*reinterpret_cast<const float4*>(p), *reinterpret_cast<const float4*>(p + 4)};
+  }
+  __device__ __forceinline__ static void load(const float* p, float* f) { unpack(load_raw(p), f); }
+  __device__ __forceinline__ static void unpack(const Raw& r, float* f) {
+    f[0] = r.a.x; f[1] = r.a.y; f[2] = r.a.z; f[3] = r.a.w;
+    f[4] = r.b.x; f[5] = r.b.y; f[6] = r.b.z; f[7] = r.b.w;
   }
   __device__ __forceinline__ static void store(float* p, const float* f) {
     *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
