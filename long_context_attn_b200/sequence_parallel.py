@@ -13,11 +13,29 @@ sequence, needs only the sum of the earlier chunks' states:
      rank order), then the chunk's prefill from that prefix with the requested output mode
      (the RMSNorm over the head concatenation is per token, so it needs no exchange).
 
-The last rank's state_out is the state after the whole sequence.  Every compute step runs
-in the library's kernels; this module only orders the calls and the collective.
+The last rank's state_out is the state after the whole sequence.
+
+The same section's variable-length batches (sequences of different lengths handed along
+the ranks like a relay) take the same three steps over a packed batch: the token stream of
+N sequences (cu_seqlens) is cut into contiguous rank slices (`bounds`), so a sequence may
+start on one rank and end several ranks later.  Each rank's slice holds pieces of
+consecutive sequences; only its first piece can continue a sequence from earlier ranks and
+only its last piece can continue onto later ones.  Step 1 is the state that last piece
+reaches from a zero state (zero when its sequence ends on this rank); step 2 the same
+all-gather; in step 3 the first piece starts from state0 of its sequence plus the gathered
+states of the ranks from the one where that sequence starts up to this one (in rank order),
+and the slice runs as one varlen prefill with a state per piece.  The relay is one
+collective step, not a chain of hops, because every rank's contribution is computed from a
+zero state.
+
+Every compute step runs in the library's kernels; this module only orders the calls and
+the collective (and allocates or slices the state buffers).
 """
 from __future__ import annotations
 
+from dataclasses import dataclass
+
+import numpy as np
 import torch
 
 from . import lightning_attn as la
@@ -79,3 +97,150 @@ def prefill_sequence_parallel(q, k, v, g, out, rank: int, all_gather=nccl_all_ga
     gathered = all_gather(local)
     finish_chunk(q, k, v, g, out, gathered, rank, workspace, state0, state_out, block_size, phi, mode, eps,
                  norm_weight, stream)
+
+
+@dataclass
+class VarlenSlice:
+    """One rank's share of a packed batch cut into contiguous rank slices.
+
+    lo, hi        the slice's tokens [lo, hi) of the packed stream
+    seq           the sequences with a piece here (consecutive indices, in order)
+    local_cu      int32 [len(seq) + 1]: the pieces' boundaries relative to lo
+    max_len       the longest piece
+    first_from    the rank where the first piece's sequence starts, when that is an earlier
+                  rank (the piece continues it), else None
+    carries       True when the last piece's sequence goes on past hi
+    final         per piece: its sequence ends on this rank (its state after the piece is
+                  the sequence's final state)
+    """
+    lo: int
+    hi: int
+    seq: list
+    local_cu: np.ndarray
+    max_len: int
+    first_from: int | None
+    carries: bool
+    final: list
+
+
+def varlen_slice_plan(cu_seqlens, bounds, rank: int) -> VarlenSlice:
+    """Host-side plan of rank `rank`'s slice.  cu_seqlens [N + 1] (host, non-decreasing from
+    0) packs N sequences; bounds [world + 1] (non-decreasing from 0 to cu_seqlens[-1]) gives
+    rank r the tokens [bounds[r], bounds[r + 1]).  An empty sequence belongs to the rank whose
+    slice holds its position (the last rank when it sits at the end of the stream)."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    b = np.asarray(bounds, dtype=np.int64)
+    if cu.ndim != 1 or cu.size < 1 or cu[0] != 0 or np.any(np.diff(cu) < 0):
+        raise ValueError("cu_seqlens must be non-decreasing from 0")
+    if b.ndim != 1 or b.size < 2 or b[0] != 0 or b[-1] != cu[-1] or np.any(np.diff(b) < 0):
+        raise ValueError("bounds must be non-decreasing from 0 to the total token count")
+    world = b.size - 1
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    lo, hi = int(b[rank]), int(b[rank + 1])
+
+    def owner(pos):   # the rank whose slice holds token position pos
+        return min(int(np.searchsorted(b, pos, side="right")) - 1, world - 1)
+
+    seq, edges, final = [], [], []
+    first_from, carries = None, False
+    for s in range(cu.size - 1):
+        a, e = int(cu[s]), int(cu[s + 1])
+        if a == e:
+            if owner(a) == rank:
+                seq.append(s)
+                edges.append((a, a))
+                final.append(True)
+            continue
+        x, y = max(a, lo), min(e, hi)
+        if x >= y:
+            continue
+        if not seq and a < lo:
+            first_from = owner(a)
+        seq.append(s)
+        edges.append((x, y))
+        final.append(e <= hi)
+    if seq and not final[-1]:
+        carries = True
+    local_cu = np.array([0] + [y - lo for _, y in edges], dtype=np.int32)
+    max_len = max([y - x for x, y in edges], default=0)
+    return VarlenSlice(lo, hi, seq, local_cu, max_len, first_from, carries, final)
+
+
+def varlen_workspace_for(plan: VarlenSlice, H: int, D: int, block_size: int = 256,
+                         mode: int = la.LA_OUT_RMSNORM_GATE, device="cuda", dtype: int = la.LA_BF16):
+    """One workspace for the slice's chunk-state call and its varlen prefill."""
+    n = 256
+    if plan.seq:
+        n = max(n, la.lightning_attn_workspace_size(la.LA_OP_PREFILL_VARLEN, len(plan.seq), plan.max_len,
+                                                    plan.hi - plan.lo, H, D, block_size, dtype, mode))
+    if plan.carries:
+        last = int(plan.local_cu[-1] - plan.local_cu[-2])
+        n = max(n, la.lightning_attn_workspace_size(la.LA_OP_CHUNK_STATE, 1, last, 0, H, D, 0, dtype, 0))
+    return la.new_workspace(n, device)
+
+
+def varlen_carry(k, v, plan: VarlenSlice, workspace, phi: int = la.LA_PHI_SILU, stream=None):
+    """Step 1: the state the slice's last piece reaches from a zero state when its sequence
+    continues on a later rank, else zero.  k, v [L, H, D] (this slice).  Returns fp32 [H, D, D]."""
+    _, H, D = k.shape
+    state = torch.zeros((1, H, D, D), dtype=torch.float32, device=k.device)
+    if plan.carries:
+        a, e = int(plan.local_cu[-2]), int(plan.local_cu[-1])
+        la.lightning_attn_chunk_state(k[a:e][None], v[a:e][None], state, phi=phi, workspace=workspace,
+                                      stream=stream)
+    return state[0]
+
+
+def varlen_finish(q, k, v, g, out, gathered, plan: VarlenSlice, rank: int, workspace, state0=None,
+                  block_size: int = 256, phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE,
+                  eps: float = 1e-6, norm_weight=None, stream=None):
+    """Step 3: the slice's varlen prefill, its first piece starting from state0 of its sequence
+    plus the gathered states [world, H, D, D] of the ranks from the one where that sequence
+    starts up to this one.  q, k, v [L, H, D]; g, out [L, H*D]; state0 fp32 [N, H, D, D] (all
+    sequences; None: zero).  Returns the states after each piece, fp32 [len(plan.seq), H, D, D]
+    (the sequences' final states where plan.final)."""
+    _, H, D = q.shape
+    m = len(plan.seq)
+    st_out = torch.empty((m, H, D, D), dtype=torch.float32, device=q.device)
+    if m == 0:
+        return st_out
+    s0 = plan.seq[0]
+    st_in = None if state0 is None else state0[s0:s0 + m]
+    if plan.first_from is not None:
+        st_in = (torch.zeros((m, H, D, D), dtype=torch.float32, device=q.device) if st_in is None
+                 else st_in.clone())
+        r0 = plan.first_from
+        la.lightning_attn_state_prefix(gathered[r0:rank + 1], rank - r0, st_in[0],
+                                       state0=None if state0 is None else state0[s0], stream=stream)
+    if plan.hi == plan.lo:   # only empty sequences: each keeps its initial state
+        if st_in is None:
+            st_out.zero_()
+        else:
+            st_out.copy_(st_in)
+        return st_out
+    cu = torch.from_numpy(plan.local_cu).to(q.device)
+    la.lightning_attn_prefill_varlen(q, k, v, g, out, cu, plan.max_len, state_in=st_in, state_out=st_out,
+                                     block_size=block_size, phi=phi, mode=mode, eps=eps, norm_weight=norm_weight,
+                                     workspace=workspace, stream=stream)
+    return st_out
+
+
+def prefill_varlen_sequence_parallel(q, k, v, g, out, cu_seqlens, bounds, rank: int, all_gather=nccl_all_gather,
+                                     state0=None, block_size: int = 256, phi: int = la.LA_PHI_SILU,
+                                     mode: int = la.LA_OUT_RMSNORM_GATE, eps: float = 1e-6, norm_weight=None,
+                                     workspace=None, stream=None):
+    """This rank's part of a sequence-parallel prefill of a packed batch (steps 1-3).
+    cu_seqlens and bounds are host arrays, the same on every rank; q, k, v [L, H, D] and g,
+    out [L, H*D] hold this rank's slice.  Returns (plan, states after each piece)."""
+    _, H, D = q.shape
+    plan = varlen_slice_plan(cu_seqlens, bounds, rank)
+    if q.shape[0] != plan.hi - plan.lo:
+        raise ValueError("q holds %d tokens, the slice %d" % (q.shape[0], plan.hi - plan.lo))
+    if workspace is None:
+        workspace = varlen_workspace_for(plan, H, D, block_size, mode, q.device, la._dtype(q))
+    carry = varlen_carry(k, v, plan, workspace, phi, stream)
+    gathered = all_gather(carry)
+    st = varlen_finish(q, k, v, g, out, gathered, plan, rank, workspace, state0, block_size, phi, mode, eps,
+                       norm_weight, stream)
+    return plan, st

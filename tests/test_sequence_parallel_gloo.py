@@ -24,7 +24,9 @@ def _free_port():
 
 
 class _OracleBackend:
-    """The three library calls sequence_parallel makes, on the CPU via the oracle."""
+    """The library calls sequence_parallel makes, on the CPU via the oracle.  Each call is
+    first bound to the real binding's signature, so a call the real library would reject
+    for its arguments fails here too."""
     LA_OUT_RAW, LA_OUT_RMSNORM_GATE, LA_PHI_SILU, LA_OP_PREFILL, LA_BF16 = 0, 2, 0, 0, 1
 
     @staticmethod
@@ -33,7 +35,31 @@ class _OracleBackend:
 
     def __init__(self):
         import oracle
+        from long_context_attn_b200 import lightning_attn as real
         self.oracle = oracle
+        self.real = real
+
+    def _bind(self, name, *args, **kw):
+        import inspect
+        inspect.signature(getattr(self.real, name)).bind(*args, **kw)
+
+    def lightning_attn_prefill_varlen(self, q, k, v, g, out, cu_seqlens, max_seqlen, state_in=None, state_out=None,
+                                      block_size=256, phi=0, mode=2, eps=1e-6, norm_weight=None, workspace=None,
+                                      stream=None):
+        import torch
+        self._bind("lightning_attn_prefill_varlen", q, k, v, g, out, cu_seqlens, max_seqlen, state_in=state_in,
+                   state_out=state_out, block_size=block_size, phi=phi, mode=mode, eps=eps, norm_weight=norm_weight,
+                   workspace=workspace, stream=stream)
+        cu = cu_seqlens.numpy()
+        assert cu.dtype == np.int32 and int(max_seqlen) >= int(np.diff(cu).max())
+        assert state_in is None or (state_in.dtype == torch.float32 and state_in.is_contiguous())
+        assert state_out.dtype == torch.float32 and state_out.shape[0] == cu.size - 1
+        _, H, D = q.shape
+        o, st, _ = self.oracle.forward_packed(q.numpy(), k.numpy(), v.numpy(), None if g is None else g.numpy(), cu,
+                                              H, D, state_in=None if state_in is None else state_in.numpy(),
+                                              phi=phi, mode=mode, eps=eps)
+        out.copy_(torch.from_numpy(o))
+        state_out.copy_(torch.from_numpy(st))
 
     def lightning_attn_prefill(self, q, k, v, g, out, state_in, state_out, block_size=256, phi=0, mode=2,
                                eps=1e-6, norm_weight=None, workspace=None, stream=None):
@@ -47,6 +73,9 @@ class _OracleBackend:
 
     def lightning_attn_chunk_state(self, k, v, state_out, state_in=None, phi=0, workspace=None, stream=None):
         import torch
+        self._bind("lightning_attn_chunk_state", k, v, state_out, state_in=state_in, phi=phi, workspace=workspace,
+                   stream=stream)
+        assert k.is_contiguous() and v.is_contiguous() and k.dim() == 4
         q = k.numpy()   # the state does not depend on q
         _, st, _ = self.oracle.prefill(q, k.numpy(), v.numpy(), None, state_in=None if state_in is None else
                                        state_in.numpy(), phi=phi, mode=self.LA_OUT_RAW)
@@ -54,6 +83,8 @@ class _OracleBackend:
 
     def lightning_attn_state_prefix(self, gathered, rank, out, state0=None, stream=None):
         import torch
+        self._bind("lightning_attn_state_prefix", gathered, rank, out, state0=state0, stream=stream)
+        assert 0 <= rank < gathered.shape[0] and gathered.is_contiguous() and out.is_contiguous()
         acc = np.zeros(out.shape) if state0 is None else state0.numpy().astype(np.float64)
         for r in range(rank):
             acc = acc + gathered[r].numpy()
@@ -104,3 +135,106 @@ def test_two_gloo_ranks_match_one_prefill(tmp_path):
     # while a wrong prefix (a chunk missed, counted twice or taken out of order) is O(1)
     np.testing.assert_allclose(got, ref[0], rtol=0, atol=1e-5 * np.abs(ref).max())
     np.testing.assert_allclose(np.load(tmp_path / "final.npy"), ref_st[0], rtol=0, atol=1e-5 * np.abs(ref_st).max())
+
+
+# A packed batch over five ranks: sequence 2 starts on rank 0, passes over rank 1 (an empty
+# slice) and ends exactly on rank 2's upper boundary; sequence 4 spans ranks 3-4; empty
+# sequences inside a slice and at the very end of the stream.
+VL_LENS = [20, 0, 45, 15, 60, 0, 26, 0]
+VL_BOUNDS = [0, 30, 30, 65, 100, 166]
+
+
+def _varlen_main(rank, world, port, out_dir):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import synth
+    from long_context_attn_b200 import sequence_parallel as sp
+    sp.la = _OracleBackend()
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        cu = synth.cu_seqlens_of(VL_LENS)
+        tot = int(cu[-1])
+        q, k, v, g = synth.prefill_inputs(1511, tot, H, D, "f32", 0.5, True)
+        s0 = synth.normal(1511, 9, (len(VL_LENS), H, D, D), 0.1, "f32")
+        a, b = VL_BOUNDS[rank], VL_BOUNDS[rank + 1]
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+        out = torch.zeros((b - a, H * D), dtype=torch.float64)
+        plan, st = sp.prefill_varlen_sequence_parallel(t(q[a:b]), t(k[a:b]), t(v[a:b]), t(g[a:b]), out, cu,
+                                                       VL_BOUNDS, rank, state0=t(s0), mode=2, workspace=object())
+        np.save(os.path.join(out_dir, f"vout{rank}.npy"), out.numpy())
+        fin = {int(s): st[i].numpy() for i, s in enumerate(plan.seq) if plan.final[i]}
+        np.save(os.path.join(out_dir, f"vfin{rank}.npy"), fin, allow_pickle=True)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_varlen_batch_over_five_gloo_ranks_matches_one_packed_prefill(tmp_path):
+    """Every token's output and every sequence's final state (from the rank where it ends)
+    against one oracle prefill of the whole packed batch."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    import synth
+    world = len(VL_BOUNDS) - 1
+    mp.start_processes(_varlen_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    cu = synth.cu_seqlens_of(VL_LENS)
+    tot = int(cu[-1])
+    q, k, v, g = synth.prefill_inputs(1511, tot, H, D, "f32", 0.5, True)
+    s0 = synth.normal(1511, 9, (len(VL_LENS), H, D, D), 0.1, "f32")
+    ref, ref_st, _ = oracle.forward_packed(q, k, v, g, cu, H, D, state_in=s0)
+    got = np.concatenate([np.load(tmp_path / f"vout{r}.npy") for r in range(world)])
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-5 * np.abs(ref).max())
+    fins = {}
+    for r in range(world):
+        part = np.load(tmp_path / f"vfin{r}.npy", allow_pickle=True).item()
+        assert not set(part) & set(fins), "a sequence's final state came from two ranks"
+        fins.update(part)
+    assert sorted(fins) == list(range(len(VL_LENS)))
+    for s, st in fins.items():
+        np.testing.assert_allclose(st, ref_st[s], rtol=0, atol=1e-5 * np.abs(ref_st).max(), err_msg=f"seq {s}")
+
+
+def test_varlen_slice_plans_partition_the_batch():
+    """Host planning alone, over seeded random batches and cuts: the pieces of all ranks tile
+    the stream in order; each sequence ends (final) on exactly one rank, empty ones included;
+    a continued first piece names the rank where its sequence starts, which carries it, as
+    does every rank in between whose slice is non-empty."""
+    sys.path.insert(0, ROOT)
+    from long_context_attn_b200.sequence_parallel import varlen_slice_plan
+    rng = np.random.default_rng(1521)
+    for _ in range(300):
+        n = int(rng.integers(1, 8))
+        lens = rng.integers(0, 40, size=n) * (rng.random(n) > 0.25)
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+        tot = int(cu[-1])
+        world = int(rng.integers(1, 6))
+        bounds = np.concatenate([[0], np.sort(rng.integers(0, tot + 1, size=world - 1)), [tot]])
+        plans = [varlen_slice_plan(cu, bounds, r) for r in range(world)]
+        pos, finals = 0, []
+        for r, p in enumerate(plans):
+            assert (p.lo, p.hi) == (bounds[r], bounds[r + 1])
+            assert p.seq == list(range(p.seq[0], p.seq[0] + len(p.seq))) if p.seq else True
+            assert p.local_cu[0] == 0 and p.local_cu[-1] == p.hi - p.lo and np.all(np.diff(p.local_cu) >= 0)
+            pos += p.hi - p.lo
+            for i, s in enumerate(p.seq):
+                a, e = p.lo + p.local_cu[i], p.lo + p.local_cu[i + 1]
+                assert cu[s] <= a <= e <= cu[s + 1]
+                assert p.final[i] == (e == cu[s + 1])
+                if p.final[i]:
+                    finals.append(s)
+            if p.first_from is not None:
+                s = p.seq[0]
+                r0 = p.first_from
+                assert r0 < r and bounds[r0] <= cu[s] < bounds[r0 + 1]
+                for j in range(r0, r):
+                    if bounds[j] < bounds[j + 1]:
+                        assert plans[j].carries and plans[j].seq[-1] == s
+            if p.carries:
+                nxt = next(j for j in range(r + 1, world) if bounds[j] < bounds[j + 1])
+                assert plans[nxt].first_from is not None and plans[nxt].seq[0] == p.seq[-1]
+        assert pos == tot
+        assert sorted(finals) == list(range(n))
