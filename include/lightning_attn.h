@@ -56,7 +56,7 @@ typedef struct CUstream_st* la_stream_t;
 typedef enum {
   LA_OK = 0,
   LA_ERR_INVALID_ARG = 1,  /* a pointer, size, alignment or enum value is invalid          */
-  LA_ERR_UNSUPPORTED = 2,  /* valid, but no kernel of this build handles the combination   */
+  LA_ERR_UNSUPPORTED = 2,  /* valid, but no kernel of the library handles the combination */
   LA_ERR_CUDA = 3,         /* a CUDA runtime/driver call or a kernel launch failed         */
   LA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out (reported by _check)      */
   LA_ERR_DEVICE = 5        /* a device-side argument check failed (reported by _check)     */
