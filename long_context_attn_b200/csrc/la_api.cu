@@ -382,15 +382,18 @@ size_t chunk_state_ws_bytes(int nseq, int max_len, int64_t tokens, int H, int D,
 
 // Normalised-variant workspace: [prefill part of the raw pass (error record first)]
 // [phi(k) chunk sums: nseq x H x chunks x D fp32] [denominators: tokens x H fp32].
+// Normalised-variant workspace: [raw prefill part] [chunk sums of phi(k)] [denominators]
+// [a copy of z_in, used when z_out overlaps it].
 struct ZLayout {
-  size_t pre, sums, den, total;
+  size_t pre, sums, den, zin, total;
 };
 ZLayout z_layout(int nseq, int max_len, int64_t tokens, int H, int D, int C, la_dtype dt) {
   ZLayout z{};
   z.pre = prefill_ws_bytes(choose_path(dt, H, D, C, LA_OUT_RAW), nseq, max_len, tokens, H, D, C, LA_OUT_RAW);
   z.sums = up256(sizeof(float) * static_cast<size_t>(nseq) * H * la::znorm_max_chunks(max_len) * D);
   z.den = up256(sizeof(float) * static_cast<size_t>(tokens) * H);
-  z.total = z.pre + z.sums + z.den;
+  z.zin = up256(sizeof(float) * static_cast<size_t>(nseq) * H * D);
+  z.total = z.pre + z.sums + z.den + z.zin;
   return z;
 }
 
@@ -416,6 +419,15 @@ la_status common_prefill_znorm(const void* q, const void* k, const void* v, cons
                                 D, C, dt, phi, LA_OUT_RAW, eps, nullptr, workspace, L.pre, stream);
   if (st != LA_OK) return st;
   const int phi_id = (phi == LA_PHI_IDENTITY) ? 1 : 0;
+  // z_out may be z_in (in place), but the scan's chunk items of a sequence all read z_in
+  // while its last item writes z_out, with no order between them: read a copy then.
+  const size_t zbytes = sizeof(float) * static_cast<size_t>(nseq) * H * D;
+  const uintptr_t zi = reinterpret_cast<uintptr_t>(z_in), zo = reinterpret_cast<uintptr_t>(z_out);
+  if (z_in && z_out && zi < zo + zbytes && zo < zi + zbytes) {
+    float* zcopy = reinterpret_cast<float*>(base + L.pre + L.sums + L.den);
+    if (cudaMemcpyAsync(zcopy, z_in, zbytes, cudaMemcpyDeviceToDevice, stream) != cudaSuccess) return LA_ERR_CUDA;
+    z_in = zcopy;
+  }
   if (la::launch_znorm_scan(q, k, z_in, sums, den, z_out, cu, nseq, T_fixed, max_len, tokens, H, D, dt, phi_id,
                             stream) != cudaSuccess)
     return LA_ERR_CUDA;

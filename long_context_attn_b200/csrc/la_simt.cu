@@ -44,8 +44,8 @@ __device__ __forceinline__ void load_rows(float (*dst)[D + 1], const T* src, int
 template <typename T, int D>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_prefill_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                    T* __restrict__ out, float* __restrict__ y_ws, const float* __restrict__ state_in,
-                    float* __restrict__ state_out, const int* __restrict__ cu, int T_fixed, int H,
+                    T* __restrict__ out, float* __restrict__ y_ws, const float* state_in,
+                    float* state_out, const int* __restrict__ cu, int T_fixed, int H,
                     int C, int phi_identity, int64_t total_rows, ErrRec* err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SimtSmem<D>& sm = *reinterpret_cast<SimtSmem<D>*>(smem_raw);

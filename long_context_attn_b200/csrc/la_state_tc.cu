@@ -281,10 +281,10 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
   if (warp == 1) tmem_dealloc<kTmemCols>(tmem);
 }
 
-// out = state_in (or zeros) + the split partials, added in split order.
+// out = state_in (or zeros) + the split partials, added in split order.  state_in and out
+// may be the same buffer (each element is read once by the thread that writes it).
 __global__ void __launch_bounds__(256) state_reduce_kernel(const float4* __restrict__ partial, int splits,
-                                                           const float4* __restrict__ state_in,
-                                                           float4* __restrict__ out, int64_t n4) {
+                                                           const float4* state_in, float4* out, int64_t n4) {
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
     float4 a = state_in ? state_in[i] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -314,9 +314,10 @@ __global__ void chunk_cu_kernel(int* cu, int B, int T, int Tc, int S) {
 // prefix[b, c] = S0[b] + sum_{c' < c} cs[b, c'] (in chunk order) and out[b] = S0[b] + all of
 // them: the initial state of every chunk of a sequence and its final state.  With time
 // running backwards the chunks are taken from the last: prefix[b, c] = S0[b] + sum_{c' > c}.
-__global__ void __launch_bounds__(256) chunk_prefix_kernel(const float4* __restrict__ cs,
-                                                           const float4* __restrict__ s0,
-                                                           float4* __restrict__ prefix, float4* __restrict__ out,
+// s0 and out may be the same buffer (a call's state_in and state_out): each element is read
+// once, by the thread that later writes it, so neither is declared __restrict__.
+__global__ void __launch_bounds__(256) chunk_prefix_kernel(const float4* __restrict__ cs, const float4* s0,
+                                                           float4* __restrict__ prefix, float4* out,
                                                            int B, int S, int64_t n4, int reverse) {
   const int64_t total = static_cast<int64_t>(B) * n4;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
