@@ -45,45 +45,3 @@ def test_emulated_ranks_match_one_prefill(C, chunks, mode, cuda_device):
     ref, ref_st, _ = oracle.prefill(q[None], k[None], v[None], g[None], state_in=s0[None], mode=m)
     assert_close(got[None], ref, "bf16")
     assert_close(to_host(final)[None], ref_st, "bf16", "final state")
-
-
-def test_emulated_ranks_varlen_batch_match_one_packed_prefill(cuda_device):
-    """A packed batch cut into five rank slices (one empty; sequences spanning two and three
-    ranks; empty sequences; a sequence ending on a slice boundary), the ranks emulated one
-    after another: every token's output and every sequence's final state against one
-    oracle prefill of the whole batch from the same initial states."""
-    import torch
-    from long_context_attn_b200 import lightning_attn as la
-    from long_context_attn_b200 import sequence_parallel as sp
-    H, D, C = 8, 128, 256
-    lens = [300, 0, 900, 129, 1000, 0, 257, 0]
-    bounds = [0, 500, 500, 1200, 1700, 2586]
-    cu = synth.cu_seqlens_of(lens)
-    tot = int(cu[-1])
-    assert tot == bounds[-1]
-    q, k, v, g = synth.prefill_inputs(1411, tot, H, D, "bf16", 0.5, True)
-    s0 = synth.normal(1411, 9, (len(lens), H, D, D), 0.05, "f32")
-    ds0 = to_dev(s0)
-    world = len(bounds) - 1
-    ranks = []
-    for r in range(world):
-        a, b = bounds[r], bounds[r + 1]
-        plan = sp.varlen_slice_plan(cu, bounds, r)
-        dq, dk, dv, dg = (to_dev(x[a:b]) for x in (q, k, v, g))
-        out = torch.full((b - a, H * D), float("nan"), dtype=torch.bfloat16, device="cuda")
-        ranks.append((plan, dq, dk, dv, dg, out, sp.varlen_workspace_for(plan, H, D, C)))
-    carries = [sp.varlen_carry(dk, dv, plan, ws) for plan, dq, dk, dv, dg, out, ws in ranks]
-    gathered = torch.stack(carries)
-    finals = {}
-    for r, (plan, dq, dk, dv, dg, out, ws) in enumerate(ranks):
-        st = sp.varlen_finish(dq, dk, dv, dg, out, gathered, plan, r, ws, state0=ds0, block_size=C)
-        la.lightning_attn_check(ws)
-        for i, s in enumerate(plan.seq):
-            if plan.final[i]:
-                assert s not in finals
-                finals[s] = to_host(st[i])
-    assert sorted(finals) == list(range(len(lens)))
-    got = np.concatenate([to_host(p[5]) for p in ranks])
-    ref, ref_st, _ = oracle.forward_packed(q, k, v, g, cu, H, D, state_in=s0)
-    assert_close(got, ref, "bf16")
-    assert_close(np.stack([finals[s] for s in range(len(lens))]), ref_st, "bf16", "final states")

@@ -100,36 +100,6 @@ def test_prefill_znorm_fp32_path(cuda_device):
     assert_close(to_host(zo), ref_z, "f32", "z")
 
 
-def test_prefill_znorm_continuation_in_place(cuda_device):
-    """A 10000-token sequence as two calls, the second continuing from the first with the
-    state and z updated in place (state_out = state_in, z_out = z_in; 20 scan chunks, so the
-    chunk items span several blocks): output and final state and z against one oracle run."""
-    import torch
-    la = _la()
-    H, D, C, T1, T2 = 8, 128, 256, 4880, 5120
-    T = T1 + T2
-    q, k, v, g = _inputs(3441, T, H, D, "bf16")
-    S = torch.empty((1, H, D, D), dtype=torch.float32, device="cuda")
-    z = torch.empty((1, H, D), dtype=torch.float32, device="cuda")
-    outs = []
-    for a, b, first in ((0, T1, True), (T1, T, False)):
-        shp, gshp = (1, b - a, H, D), (1, b - a, H * D)
-        out = torch.empty(gshp, dtype=torch.bfloat16, device="cuda")
-        ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_PREFILL_ZNORM, 1, b - a, 0, H, D, C,
-                                                               la.LA_BF16, la.LA_OUT_RMSNORM_GATE))
-        la.lightning_attn_prefill_znorm(*(to_dev(x[a:b]).reshape(shp) for x in (q, k, v)),
-                                        to_dev(g[a:b]).reshape(gshp), out, state_in=None if first else S,
-                                        z_in=None if first else z, state_out=S, z_out=z, block_size=C,
-                                        workspace=ws)
-        la.lightning_attn_check(ws)
-        outs.append(to_host(out)[0])
-    shp, gshp = (1, T, H, D), (1, T, H * D)
-    ref, ref_S, ref_z = oracle.prefill_znorm(q.reshape(shp), k.reshape(shp), v.reshape(shp), g.reshape(gshp))
-    assert_close(np.concatenate(outs)[None], ref, "bf16")
-    assert_close(to_host(S), ref_S, "bf16", "state")
-    assert_close(to_host(z), ref_z, "f32", "z")
-
-
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_decode_znorm(dtype, cuda_device):
     la = _la()
