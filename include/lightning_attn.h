@@ -79,7 +79,8 @@ typedef enum {
   LA_OP_BACKWARD_VARLEN = 5,
   LA_OP_PREFILL_ZNORM = 6,
   LA_OP_PREFILL_ZNORM_VARLEN = 7,
-  LA_OP_CHUNK_STATE = 8
+  LA_OP_CHUNK_STATE = 8,
+  LA_OP_OUTPUT_TRANSFORM_BACKWARD = 9
 } la_op;
 
 /*
@@ -355,6 +356,32 @@ LA_API la_status lightning_attn_output_transform(const void* y, const void* g, v
                                                  const float* norm_weight, la_stream_t stream);
 
 /*
+ * Backward of lightning_attn_output_transform: given the gradient dout of its output, the
+ * gradient dy of the raw output y, the gate's gradient dg and the norm weight's gradient
+ * (the chain rule through the transform of "MiniMax-Text-01 405B MoE模型架构与训练策略解析"
+ * section 2.1, as inside lightning_attn_backward).  Per token, with r = 1/sqrt(mean(y^2) +
+ * eps), s = sigmoid(g) (1 without the gate) and u = dout * w * s:
+ *   dy = r u - r^3 y (sum over the row of u y) / (H*D),   dg = dout * y * r * w * s * (1 - s),
+ *   dnorm_weight = sum over tokens of dout * y * r * s.
+ * RAW: dy = dout (copied), dnorm_weight zeros.  It is the first step of a backward whose
+ * linear-attention part runs elsewhere (lightning_attn_backward in LA_OUT_RAW mode given dy,
+ * e.g. each rank of a sequence-parallel backward).
+ *   y, g, dout    [tokens, H*D] dtype, device (y ignored in RAW; g iff RMSNORM_GATE).
+ *   dy            [tokens, H*D] dtype, written; may equal y, not dout or g.
+ *   dg            [tokens, H*D] dtype, written iff RMSNORM_GATE; distinct from the others.
+ *   dnorm_weight  fp32 [H*D] or NULL; summed in a fixed order (deterministic).
+ *   workspace     needed iff dnorm_weight is given in a norm mode: >= lightning_attn_workspace_size(
+ *                 LA_OP_OUTPUT_TRANSFORM_BACKWARD, tokens, 0, 0, H, D, 0, dtype, mode) bytes,
+ *                 256-byte aligned.
+ * H*D <= 16384.  Returns LA_OK after enqueueing, or an error status with nothing enqueued.
+ */
+LA_API la_status lightning_attn_output_transform_backward(const void* y, const void* g, const void* dout, void* dy,
+                                                          void* dg, float* dnorm_weight, int tokens, int H, int D,
+                                                          la_dtype dtype, la_out_mode mode, float eps,
+                                                          const float* norm_weight, void* workspace,
+                                                          size_t workspace_bytes, la_stream_t stream);
+
+/*
  * The state lightning_attn_prefill would end with, without computing its outputs:
  *   state_out[b] = state_in[b] + sum_t phi(k_t) v_t^T      ("六十四：MiniMax-01" section 3:
  * the state is a plain sum over the sequence).  Step 1 of the sequence-parallel prefill
@@ -386,6 +413,7 @@ LA_API la_status lightning_attn_chunk_state(const void* k, const void* v, const 
  *   op == LA_OP_PREFILL_ZNORM:   as LA_OP_PREFILL.
  *   op == LA_OP_PREFILL_ZNORM_VARLEN: as LA_OP_PREFILL_VARLEN.
  *   op == LA_OP_CHUNK_STATE:     B_or_N = B, T_or_max = T (block_size and mode ignored).
+ *   op == LA_OP_OUTPUT_TRANSFORM_BACKWARD: B_or_N = tokens (>= 0), H, D; the rest ignored.
  * The size depends on the kernel the call will select (which depends on the device), so
  * query it with the target device current.
  */

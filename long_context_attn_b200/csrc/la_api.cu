@@ -437,6 +437,11 @@ la_status common_prefill_znorm(const void* q, const void* k, const void* v, cons
   return LA_OK;
 }
 
+// The output transform's backward: the norm weight's gradient as per-CTA partial rows.
+size_t output_transform_backward_ws_bytes(int64_t tokens, int HD) {
+  return std::max<size_t>(256, up256(sizeof(float) * static_cast<size_t>(la::norm_weight_partial_floats(tokens, HD))));
+}
+
 }  // namespace
 
 extern "C" {
@@ -497,6 +502,41 @@ la_status lightning_attn_output_transform(const void* y, const void* g, void* ou
   const cudaError_t e = la::launch_output_transform(y, out, nullptr, g, norm_weight, tokens, H, D,
                                                     static_cast<int>(mode), eps, dtype,
                                                     reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status lightning_attn_output_transform_backward(const void* y, const void* g, const void* dout, void* dy, void* dg,
+                                                   float* dnorm_weight, int tokens, int H, int D, la_dtype dtype,
+                                                   la_out_mode mode, float eps, const float* norm_weight,
+                                                   void* workspace, size_t workspace_bytes, la_stream_t stream) {
+  if (tokens < 0 || H < 1 || (D != 64 && D != 128) || static_cast<int64_t>(H) * D > la::kMaxNormWidth)
+    return LA_ERR_INVALID_ARG;
+  if (!valid_enums(dtype, LA_PHI_SILU, mode) || (mode != LA_OUT_RAW && !(eps > 0.0f))) return LA_ERR_INVALID_ARG;
+  if (tokens > 0) {
+    if (!dout || !dy || !aligned16(dout) || !aligned16(dy)) return LA_ERR_INVALID_ARG;
+    if (mode != LA_OUT_RAW && (!y || !aligned16(y))) return LA_ERR_INVALID_ARG;
+    if (mode == LA_OUT_RMSNORM_GATE && (!g || !aligned16(g) || !dg || !aligned16(dg))) return LA_ERR_INVALID_ARG;
+    if (dy == dout || (mode == LA_OUT_RMSNORM_GATE && (dy == g || dg == y || dg == dout || dg == dy)))
+      return LA_ERR_INVALID_ARG;
+  }
+  if ((norm_weight && !aligned16(norm_weight)) || (dnorm_weight && !aligned16(dnorm_weight)))
+    return LA_ERR_INVALID_ARG;
+  const int HD = H * D;
+  const bool want_dw = dnorm_weight && mode != LA_OUT_RAW;
+  if (want_dw && (!workspace || !aligned256(workspace) ||
+                  workspace_bytes < output_transform_backward_ws_bytes(tokens, HD)))
+    return LA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (mode == LA_OUT_RAW) {   // dy = dout; the raw output has no norm weight
+    const size_t bytes = static_cast<size_t>(tokens) * HD * (dtype == LA_BF16 ? 2 : 4);
+    if (bytes && cudaMemcpyAsync(dy, dout, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return LA_ERR_CUDA;
+    if (dnorm_weight && cudaMemsetAsync(dnorm_weight, 0, sizeof(float) * HD, st) != cudaSuccess) return LA_ERR_CUDA;
+    return LA_OK;
+  }
+  const cudaError_t e = la::launch_bwd_norm_gate(y, g, dout, norm_weight, dy, dg,
+                                                 want_dw ? static_cast<float*>(workspace) : nullptr,
+                                                 want_dw ? dnorm_weight : nullptr, tokens, HD,
+                                                 mode == LA_OUT_RMSNORM_GATE ? 1 : 0, eps, dtype, st);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
@@ -676,6 +716,10 @@ la_status lightning_attn_mixed_step(const void* q, const void* k, const void* v,
 
 size_t lightning_attn_workspace_size(la_op op, int B_or_N, int T_or_max, int total_tokens, int H, int D,
                                      int block_size, la_dtype dtype, la_out_mode mode) {
+  if (op == LA_OP_OUTPUT_TRANSFORM_BACKWARD) {   // B_or_N = tokens
+    if (B_or_N < 0 || H < 1 || (D != 64 && D != 128)) return 0;
+    return output_transform_backward_ws_bytes(B_or_N, H * D);
+  }
   if (B_or_N < 1 || T_or_max < 0 || H < 1 || (D != 64 && D != 128)) return 0;
   if (op == LA_OP_DECODE) return la::decode_workspace_bytes(B_or_N, H, D);
   if (op == LA_OP_MIXED) {

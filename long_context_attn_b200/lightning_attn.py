@@ -21,7 +21,7 @@ LA_F32, LA_BF16 = 0, 1
 LA_OUT_RAW, LA_OUT_RMSNORM, LA_OUT_RMSNORM_GATE = 0, 1, 2
 LA_PHI_SILU, LA_PHI_IDENTITY = 0, 1
 (LA_OP_PREFILL, LA_OP_PREFILL_VARLEN, LA_OP_DECODE, LA_OP_MIXED, LA_OP_BACKWARD, LA_OP_BACKWARD_VARLEN,
- LA_OP_PREFILL_ZNORM, LA_OP_PREFILL_ZNORM_VARLEN, LA_OP_CHUNK_STATE) = range(9)
+ LA_OP_PREFILL_ZNORM, LA_OP_PREFILL_ZNORM_VARLEN, LA_OP_CHUNK_STATE, LA_OP_OUTPUT_TRANSFORM_BACKWARD) = range(10)
 
 # The symbols include/lightning_attn.h declares (checked by tests/test_abi.py).
 EXPORTED = (
@@ -38,6 +38,7 @@ EXPORTED = (
     "lightning_attn_state_prefix",
     "lightning_attn_chunk_state",
     "lightning_attn_output_transform",
+    "lightning_attn_output_transform_backward",
     "lightning_attn_workspace_size",
     "lightning_attn_check",
     "lightning_attn_status_string",
@@ -67,6 +68,7 @@ def _load():
     lib.lightning_attn_backward.argtypes = [vp] * 14 + [i32] * 8 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_backward_varlen.argtypes = [vp] * 15 + [i32] * 9 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_output_transform.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]
+    lib.lightning_attn_output_transform_backward.argtypes = [vp] * 6 + [i32] * 5 + [f32, vp, vp, sz, vp]
     lib.lightning_attn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp,
                                                sz, vp]
     lib.lightning_attn_decode_step_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32,
@@ -86,7 +88,7 @@ def _load():
               "lightning_attn_backward_varlen", "lightning_attn_prefill_znorm", "lightning_attn_prefill_znorm_varlen",
               "lightning_attn_decode_step_znorm", "lightning_attn_decode_step",
               "lightning_attn_decode_step_noalloc", "lightning_attn_mixed_step", "lightning_attn_state_prefix", "lightning_attn_chunk_state",
-              "lightning_attn_output_transform",
+              "lightning_attn_output_transform", "lightning_attn_output_transform_backward",
               "lightning_attn_check"):
         getattr(lib, f).restype = i32
     return lib
@@ -340,6 +342,26 @@ def lightning_attn_output_transform(y, g, out, mode=LA_OUT_RMSNORM_GATE, eps=1e-
                                               _ptr(_f32_or_none(norm_weight)), _stream(stream))
     if st != LA_OK:
         raise LightningAttnError(st, "lightning_attn_output_transform")
+
+
+def lightning_attn_output_transform_backward(y, g, dout, dy, dg=None, dnorm_weight=None, mode=LA_OUT_RMSNORM_GATE,
+                                            eps=1e-6, norm_weight=None, workspace=None, stream=None):
+    """dy, dg (and the norm weight's gradient) from dout through the output transform of y:
+    y, g, dout, dy, dg hold tokens * H * D elements each, H and D taken from the last two dims
+    of y viewed as [..., H, D] (of dout when y is None, in raw mode); dnorm_weight fp32 [H*D]."""
+    src = y if y is not None else dout
+    if src.dim() < 2:
+        raise ValueError("y (or dout) must be [..., H, D]")
+    H, D = src.shape[-2], src.shape[-1]
+    tokens = src.numel() // (H * D)
+    _check_contig(y, g, dout, dy, dg)
+    st = _lib.lightning_attn_output_transform_backward(_ptr(y), _ptr(g), _ptr(dout), _ptr(dy), _ptr(dg),
+                                                       _ptr(_f32_or_none(dnorm_weight)), tokens, H, D, _dtype(dout),
+                                                       mode, eps, _ptr(_f32_or_none(norm_weight)), _ptr(workspace),
+                                                       0 if workspace is None else workspace.numel(),
+                                                       _stream(stream))
+    if st != LA_OK:
+        raise LightningAttnError(st, "lightning_attn_output_transform_backward")
 
 
 def lightning_attn_chunk_state(k, v, state_out, state_in=None, phi=LA_PHI_SILU, workspace=None, stream=None):

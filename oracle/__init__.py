@@ -71,11 +71,12 @@ def _get():
                                                     vp, vp, vp, vp]
         lib.oracle_backward_packed.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, vp, i32, i32, dbl,
                                                vp, vp, vp, vp, vp, vp, vp]
+        lib.oracle_transform_backward.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, dbl, vp, vp, vp, vp]
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         for f in (lib.oracle_forward_packed, lib.oracle_prefill, lib.oracle_decode,
                   lib.oracle_quadratic, lib.oracle_chunked, lib.oracle_transform, lib.oracle_backward_packed,
-                  lib.oracle_forward_znorm_packed):
+                  lib.oracle_forward_znorm_packed, lib.oracle_transform_backward):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -199,6 +200,24 @@ def transform(y, mode, eps=1e-6, norm_weight=None, g=None):
     _get().oracle_transform(_ptr(y), tokens, H, D, mode, eps, _ptr(w), _ptr(g),
                             dt, _ptr(out))
     return out
+
+
+def transform_backward(y, dout, mode, eps=1e-6, norm_weight=None, g=None):
+    """Backward of `transform`: y fp64 [tokens, H, D]; dout, g [tokens, H*D] (bf16 bits or
+    fp32, one dtype).  Returns fp64 (dy [tokens, H*D], dg [tokens, H*D] or None, dw [H*D])."""
+    y = _c(y, np.float64)
+    tokens, H, D = y.shape
+    dout, g = _c(dout), _c(g)
+    dt = _dtype_code(dout)
+    w = _c(norm_weight, np.float32)
+    dy = np.empty((tokens, H * D), dtype=np.float64)
+    dg = np.empty((tokens, H * D), dtype=np.float64) if mode == MODE_RMSNORM_GATE else None
+    dw = np.empty(H * D, dtype=np.float64)
+    rc = _get().oracle_transform_backward(_ptr(y), _ptr(dout), _ptr(g), dt, tokens, H, D, mode, eps, _ptr(w),
+                                          _ptr(dy), _ptr(dg), _ptr(dw))
+    if rc != 0:
+        raise ValueError("oracle_transform_backward rejected its arguments")
+    return dy, dg, dw
 
 
 def backward_packed(q, k, v, g, dout, cu_seqlens, H, D, state_in=None, phi=PHI_SILU, mode=MODE_RMSNORM_GATE,

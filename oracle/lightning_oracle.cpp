@@ -461,6 +461,32 @@ int oracle_transform(const double* y, int64_t tokens, int H, int D, int mode, do
   return 0;
 }
 
+// The output transform's backward alone ([Arch] 2.1, by the chain rule), for tests of a
+// backward whose first step it is: per token, dy (fp64 [tokens, H*D]) from the raw output y
+// (fp64 [tokens, H*D]) and dout (dtype), dg in gate mode, and dw [H*D] summed over the tokens
+// in token order (zero in raw mode).  dg and dw may be null.
+int oracle_transform_backward(const double* y, const void* dout, const void* g, int dtype, int64_t tokens, int H,
+                              int D, int mode, double eps, const float* w, double* dy, double* dg, double* dw) {
+  if (tokens < 0 || H <= 0 || D <= 0 || !dout || !dy) return 1;
+  if (mode != MODE_RAW && !y) return 1;
+  if (mode == MODE_RMSNORM_GATE && !g) return 1;
+  const int HD = H * D;
+  const bool want_dw = dw && mode != MODE_RAW;
+  std::vector<double> dwt(want_dw ? static_cast<size_t>(tokens) * HD : 0);
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < tokens; ++t)
+    transform_token_backward(mode == MODE_RAW ? nullptr : y + t * HD, dout, g, dtype, t, HD, mode, eps, w,
+                             dy + t * HD, (mode == MODE_RMSNORM_GATE && dg) ? dg + t * HD : nullptr,
+                             want_dw ? dwt.data() + t * HD : nullptr);
+  if (dw) {
+    for (int c = 0; c < HD; ++c) dw[c] = 0.0;
+    if (want_dw)
+      for (int64_t t = 0; t < tokens; ++t)
+        for (int c = 0; c < HD; ++c) dw[c] += dwt[static_cast<size_t>(t) * HD + c];
+  }
+  return 0;
+}
+
 // Backward of oracle_forward_packed for the loss whose output gradient is dout [tokens, H*D]
 // (same dtype as q) and whose final-state gradient is dstate_out [N, H, D, D] fp32 (null for
 // zero).  Recomputes the raw forward y, applies the transform backward per token, then the

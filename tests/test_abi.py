@@ -185,3 +185,41 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
     r = subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", HEADER_DIR, str(src), so,
                         "-o", str(tmp_path / "use_abi")], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_output_transform_backward_host_checks(lib):
+    """lightning_attn_output_transform_backward rejects bad arguments on the host; its
+    workspace (the norm weight's gradient as partial rows) is sized from the token count."""
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    lib.lightning_attn_workspace_size.restype = ctypes.c_size_t
+    n0 = lib.lightning_attn_workspace_size(9, 0, 0, 0, 8, 128, 0, 1, 2)
+    n1 = lib.lightning_attn_workspace_size(9, 100, 0, 0, 8, 128, 0, 1, 2)
+    n2 = lib.lightning_attn_workspace_size(9, 100000, 0, 0, 8, 128, 0, 1, 2)
+    assert n0 >= 256 and n1 >= 100 * 8 * 128 * 4 and n2 >= 1024 * 8 * 128 * 4 and n2 < 2 * 1024 * 8 * 128 * 4
+    assert lib.lightning_attn_workspace_size(9, 100, 0, 0, 8, 96, 0, 1, 2) == 0
+    f = lib.lightning_attn_output_transform_backward
+    f.argtypes = [vp] * 6 + [i32] * 5 + [ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
+    y, g, d, dy, dg = (vp(0x1000 * (i + 1)) for i in range(5))
+    ws = vp(0x100000)
+
+    def call(**kw):
+        a = dict(y=y, g=g, d=d, dy=dy, dg=dg, dw=None, tokens=10, H=8, D=128, dt=1, mode=2, eps=1e-6, w=None, ws=None,
+                 nbytes=0)
+        a.update(kw)
+        return f(a["y"], a["g"], a["d"], a["dy"], a["dg"], a["dw"], a["tokens"], a["H"], a["D"], a["dt"], a["mode"],
+                 ctypes.c_float(a["eps"]), a["w"], a["ws"], a["nbytes"], None)
+
+    assert call(dg=None) == 1                     # gate mode needs dg
+    assert call(y=None) == 1                      # norm modes need y
+    assert call(dy=vp(0x1008)) == 1               # 16-byte alignment
+    assert call(dy=d) == 1                        # dy may not be dout
+    assert call(dg=dy) == 1                       # dg distinct
+    assert call(D=96) == 1
+    assert call(H=200) == 1                       # H*D > 16384
+    assert call(eps=0.0) == 1
+    assert call(mode=5) == 1
+    assert call(tokens=-1) == 1
+    assert call(dw=vp(0x2000)) == 1               # dw without a workspace
+    assert call(dw=vp(0x2000), ws=vp(0x100010), nbytes=1 << 30) == 1   # misaligned workspace
+    assert call(dw=vp(0x2000), ws=ws, nbytes=256) == 1                 # workspace too small
+    assert call(dw=vp(0x2004), ws=ws, nbytes=1 << 30) == 1             # misaligned dw

@@ -156,3 +156,40 @@ def test_norm_weight_gradient_matches_finite_differences(mode):
     assert abs(fd - pred) <= 1e-5 * float(np.sum(np.abs(dw * step))), (fd, pred)
     *_, dw_raw = oracle.backward_packed(x["q"], x["k"], x["v"], None, dout, CU, H, D, mode=oracle.MODE_RAW)
     assert np.all(dw_raw == 0.0)
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_RAW, oracle.MODE_RMSNORM, oracle.MODE_RMSNORM_GATE])
+def test_transform_backward_matches_finite_differences(mode):
+    """oracle.transform_backward (the output transform's backward alone) against central
+    differences of oracle.transform in y, in the gate and in the norm weight, each along a
+    random direction; in raw mode dy = dout and dw = 0."""
+    tokens = 7
+    rng = np.random.default_rng(2191 + mode)
+    y = rng.standard_normal((tokens, H, D))
+    g = synth.normal(2191, 3, (tokens, H * D), 1.0, "f32") if mode == oracle.MODE_RMSNORM_GATE else None
+    w = (1.0 + 0.25 * synth.normal(2191, 13, (H * D,), 1.0, "f32")).astype(np.float32)
+    dout = synth.normal(2191, 11, (tokens, H * D), 1.0, "f32")
+    dy, dg, dw = oracle.transform_backward(y, dout, mode, norm_weight=w, g=g)
+    loss = lambda yy, gg, ww: float(np.sum(oracle.transform(yy, mode, norm_weight=ww, g=gg) * dout.astype(np.float64)))
+    e = 1e-4
+    d = rng.standard_normal(y.shape)
+    fd = (loss(y + e * d, g, w) - loss(y - e * d, g, w)) / (2 * e)
+    pred = float(np.sum(dy * d.reshape(tokens, H * D)))
+    assert abs(fd - pred) <= 1e-7 * float(np.sum(np.abs(dy * d.reshape(tokens, H * D)))), ("y", fd, pred)
+    if mode == oracle.MODE_RAW:
+        np.testing.assert_array_equal(dy, dout.astype(np.float64))
+        assert np.all(dw == 0.0) and dg is None
+        return
+    dlt = rng.standard_normal(w.shape)
+    wp, wm = (w + 1e-3 * dlt).astype(np.float32), (w - 1e-3 * dlt).astype(np.float32)
+    step = wp.astype(np.float64) - wm.astype(np.float64)
+    fd = loss(y, g, wp) - loss(y, g, wm)
+    pred = float(np.sum(dw * step))
+    assert abs(fd - pred) <= 1e-5 * float(np.sum(np.abs(dw * step))), ("w", fd, pred)
+    if mode == oracle.MODE_RMSNORM_GATE:
+        dlt = rng.standard_normal(g.shape)
+        gp, gm = (g + 1e-3 * dlt).astype(np.float32), (g - 1e-3 * dlt).astype(np.float32)
+        step = gp.astype(np.float64) - gm.astype(np.float64)
+        fd = loss(y, gp, w) - loss(y, gm, w)
+        pred = float(np.sum(dg * step))
+        assert abs(fd - pred) <= 1e-5 * float(np.sum(np.abs(dg * step))), ("g", fd, pred)
