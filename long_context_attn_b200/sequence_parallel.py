@@ -28,6 +28,12 @@ and the slice runs as one varlen prefill with a state per piece.  The relay is o
 collective step, not a chain of hops, because every rank's contribution is computed from a
 zero state.
 
+The backward (training used LASP+ as well) needs one exchange too: the gradient reaching
+the end of chunk r is the final-state gradient plus, for each later chunk, the sum over
+its tokens of phi(q_t) dy_t^T, which every rank computes from its own chunk (the chunk-state
+kernel with q as keys and dy as values); after one all-gather each rank adds the later
+ranks' sums and runs its chunk's backward (backward_sequence_parallel).
+
 Every compute step runs in the library's kernels; this module only orders the calls and
 the collective (and allocates or slices the state buffers).
 """
@@ -61,7 +67,8 @@ def finish_chunk(q, k, v, g, out, gathered, rank: int, workspace, state0=None, s
                  block_size: int = 256, phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE,
                  eps: float = 1e-6, norm_weight=None, stream=None):
     """Step 3: prefix the gathered chunk states [world, H, D, D] for `rank` and prefill the chunk
-    from it.  state0 [H, D, D] is the state before the whole sequence (None: zero)."""
+    from it.  state0 [H, D, D] is the state before the whole sequence (None: zero).  Returns the
+    prefix (fp32 [H, D, D], the state the chunk started from; the backward takes it)."""
     _, T, H, D = q.shape
     prefix = torch.empty((H, D, D), dtype=torch.float32, device=q.device)
     la.lightning_attn_state_prefix(gathered, rank, prefix, state0=state0, stream=stream)
@@ -69,6 +76,7 @@ def finish_chunk(q, k, v, g, out, gathered, rank: int, workspace, state0=None, s
                               None if state_out is None else state_out.view(1, H, D, D), block_size=block_size,
                               phi=phi, mode=mode, eps=eps, norm_weight=norm_weight, workspace=workspace,
                               stream=stream)
+    return prefix
 
 
 def nccl_all_gather(state: torch.Tensor, group=None) -> torch.Tensor:
@@ -89,14 +97,94 @@ def prefill_sequence_parallel(q, k, v, g, out, rank: int, all_gather=nccl_all_ga
                               mode: int = la.LA_OUT_RMSNORM_GATE, eps: float = 1e-6, norm_weight=None,
                               workspace=None, stream=None):
     """This rank's part of a sequence-parallel prefill (steps 1-3).  Every rank of the group
-    calls it with its own chunk, in the same order relative to other collectives."""
+    calls it with its own chunk, in the same order relative to other collectives.  Returns the
+    state the chunk started from (fp32 [H, D, D])."""
     _, T, H, D = q.shape
     if workspace is None:
         workspace = workspace_for(T, H, D, block_size, mode, q.device, la._dtype(q))
     local = chunk_state(k, v, workspace, phi, stream)
     gathered = all_gather(local)
-    finish_chunk(q, k, v, g, out, gathered, rank, workspace, state0, state_out, block_size, phi, mode, eps,
-                 norm_weight, stream)
+    return finish_chunk(q, k, v, g, out, gathered, rank, workspace, state0, state_out, block_size, phi, mode, eps,
+                        norm_weight, stream)
+
+
+def backward_workspace_for(T: int, H: int, D: int, block_size: int = 256, mode: int = la.LA_OUT_RMSNORM_GATE,
+                           device="cuda", dtype: int = la.LA_BF16) -> torch.Tensor:
+    """One workspace for every call of backward_sequence_parallel on a chunk of T tokens."""
+    n = max(la.lightning_attn_workspace_size(la.LA_OP_PREFILL, 1, T, 0, H, D, block_size, dtype, la.LA_OUT_RAW),
+            la.lightning_attn_workspace_size(la.LA_OP_CHUNK_STATE, 1, T, 0, H, D, 0, dtype, 0),
+            la.lightning_attn_workspace_size(la.LA_OP_BACKWARD, 1, T, 0, H, D, block_size, dtype, la.LA_OUT_RAW),
+            la.lightning_attn_workspace_size(la.LA_OP_OUTPUT_TRANSFORM_BACKWARD, T, 0, 0, H, D, 0, dtype, mode))
+    return la.new_workspace(n, device)
+
+
+def backward_local(q, k, v, g, dout, prefix, workspace, y=None, dg=None, dnorm_weight=None, block_size: int = 256,
+                   phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE, eps: float = 1e-6,
+                   norm_weight=None, stream=None):
+    """Backward steps 1-2 on this rank's chunk: dy (and dg, this chunk's terms of dw) from dout
+    through the output transform of the chunk's raw output y (given, or recomputed from
+    `prefix`), then G = sum over the chunk of phi(q_t) dy_t^T (the chunk-state kernel with q
+    as the keys and dy as the values).  Returns (dy [1, T, H*D], G fp32 [H, D, D])."""
+    _, T, H, D = q.shape
+    if mode == la.LA_OUT_RAW:
+        dy = dout
+        if dnorm_weight is not None:
+            dnorm_weight.zero_()
+    else:
+        if y is None:
+            y = torch.empty_like(dout)
+            la.lightning_attn_prefill(q, k, v, None, y, prefix.view(1, H, D, D), None, block_size=block_size, phi=phi,
+                                      mode=la.LA_OUT_RAW, workspace=workspace, stream=stream)
+        dy = torch.empty_like(dout)
+        la.lightning_attn_output_transform_backward(y.view(1, T, H, D), g, dout, dy, dg=dg, dnorm_weight=dnorm_weight,
+                                                    mode=mode, eps=eps, norm_weight=norm_weight, workspace=workspace,
+                                                    stream=stream)
+    G = torch.empty((1, H, D, D), dtype=torch.float32, device=q.device)
+    la.lightning_attn_chunk_state(q, dy.view(1, T, H, D), G, phi=phi, workspace=workspace, stream=stream)
+    return dy, G[0]
+
+
+def backward_finish(q, k, v, dy, dq, dk, dv, gathered, rank: int, prefix, workspace, dstate_out=None,
+                    dstate_in=None, block_size: int = 256, phi: int = la.LA_PHI_SILU, stream=None):
+    """Backward steps 3-4: the gradient reaching the end of the chunk, dS_T + sum_{j > rank} of
+    the gathered G_j [world, H, D, D] (added from the last rank down), then the chunk's
+    backward in raw mode from dy with its initial state `prefix`."""
+    _, T, H, D = q.shape
+    world = gathered.shape[0]
+    later_first = torch.flip(gathered, dims=[0]).contiguous()   # rank world-1 first
+    ds_end = torch.empty((H, D, D), dtype=torch.float32, device=q.device)
+    la.lightning_attn_state_prefix(later_first, world - 1 - rank, ds_end, state0=dstate_out, stream=stream)
+    st = lambda x: None if x is None else x.view(1, H, D, D)
+    la.lightning_attn_backward(q, k, v, None, dy, dq, dk, dv, state_in=st(prefix), dstate_in=st(dstate_in),
+                               block_size=block_size, phi=phi, mode=la.LA_OUT_RAW, workspace=workspace,
+                               stream=stream, dstate_out=st(ds_end))
+
+
+def backward_sequence_parallel(q, k, v, g, dout, dq, dk, dv, rank: int, prefix, all_gather=nccl_all_gather,
+                               dstate_out=None, y=None, dg=None, dnorm_weight=None, dstate_in=None,
+                               block_size: int = 256, phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE,
+                               eps: float = 1e-6, norm_weight=None, workspace=None, stream=None):
+    """This rank's part of the backward of prefill_sequence_parallel.
+
+    The gradient reaching the end of chunk r is the sequence's final-state gradient dS_T
+    plus, for every later chunk j, G_j = sum over its tokens of phi(q_t) dy_t^T (the part of
+    chunk j's initial-state gradient that its own tokens give), so after one all-gather of
+    the G_j every rank runs its chunk's backward on its own (backward_local, the all-gather,
+    backward_finish).
+    q, k, v, dq, dk, dv [1, T, H, D]; g, dout, dg [1, T, H*D]; prefix (the state the chunk
+    started from, as prefill_sequence_parallel returns it), dstate_out, dstate_in fp32
+    [H, D, D] (dstate_out: the same tensor on every rank, None for zero; rank 0's dstate_in
+    is the gradient of the sequence's initial state); y: the chunk's raw output if kept;
+    dnorm_weight fp32 [H*D] receives this chunk's part of the norm weight's gradient (sum it
+    over the ranks)."""
+    _, T, H, D = q.shape
+    if workspace is None:
+        workspace = backward_workspace_for(T, H, D, block_size, mode, q.device, la._dtype(q))
+    dy, G = backward_local(q, k, v, g, dout, prefix, workspace, y, dg, dnorm_weight, block_size, phi, mode, eps,
+                           norm_weight, stream)
+    gathered = all_gather(G)
+    backward_finish(q, k, v, dy, dq, dk, dv, gathered, rank, prefix, workspace, dstate_out, dstate_in, block_size,
+                    phi, stream)
 
 
 @dataclass

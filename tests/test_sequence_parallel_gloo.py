@@ -71,6 +71,41 @@ class _OracleBackend:
         if state_out is not None:
             state_out.copy_(torch.from_numpy(st))
 
+    def lightning_attn_output_transform_backward(self, y, g, dout, dy, dg=None, dnorm_weight=None, mode=2, eps=1e-6,
+                                                 norm_weight=None, workspace=None, stream=None):
+        import torch
+        self._bind("lightning_attn_output_transform_backward", y, g, dout, dy, dg=dg, dnorm_weight=dnorm_weight,
+                   mode=mode, eps=eps, norm_weight=norm_weight, workspace=workspace, stream=stream)
+        H, D = y.shape[-2], y.shape[-1]
+        n = y.numel() // (H * D)
+        r = lambda t: None if t is None else t.numpy().reshape(n, H * D)
+        dyy, dgg, dw = self.oracle.transform_backward(y.numpy().reshape(n, H, D), r(dout), mode, eps=eps,
+                                                      norm_weight=None if norm_weight is None else norm_weight.numpy(),
+                                                      g=r(g))
+        dy.copy_(torch.from_numpy(dyy).view(dy.shape))
+        if dg is not None:
+            dg.copy_(torch.from_numpy(dgg).view(dg.shape))
+        if dnorm_weight is not None:
+            dnorm_weight.copy_(torch.from_numpy(dw))
+
+    def lightning_attn_backward(self, q, k, v, g, dout, dq, dk, dv, dg=None, state_in=None, dstate_in=None,
+                                block_size=256, phi=0, mode=2, eps=1e-6, norm_weight=None, workspace=None, stream=None,
+                                dstate_out=None, y=None, dnorm_weight=None):
+        import torch
+        self._bind("lightning_attn_backward", q, k, v, g, dout, dq, dk, dv, dg=dg, state_in=state_in,
+                   dstate_in=dstate_in, block_size=block_size, phi=phi, mode=mode, eps=eps, norm_weight=norm_weight,
+                   workspace=workspace, stream=stream, dstate_out=dstate_out, y=y, dnorm_weight=dnorm_weight)
+        assert q.dim() == 4 and dout.shape == (q.shape[0], q.shape[1], q.shape[2] * q.shape[3])
+        npy = lambda t: None if t is None else t.numpy()
+        ref = self.oracle.backward(q.numpy(), k.numpy(), v.numpy(), npy(g), dout.numpy(), state_in=npy(state_in),
+                                   phi=phi, mode=mode, eps=eps, norm_weight=npy(norm_weight),
+                                   dstate_out=npy(dstate_out))
+        for t, r in zip((dq, dk, dv, dg, dstate_in), ref):
+            if t is not None:
+                t.copy_(torch.from_numpy(r).view(t.shape))
+        if dnorm_weight is not None:
+            dnorm_weight.copy_(torch.from_numpy(ref[5]))
+
     def lightning_attn_chunk_state(self, k, v, state_out, state_in=None, phi=0, workspace=None, stream=None):
         import torch
         self._bind("lightning_attn_chunk_state", k, v, state_out, state_in=state_in, phi=phi, workspace=workspace,
@@ -238,3 +273,76 @@ def test_varlen_slice_plans_partition_the_batch():
                 assert plans[nxt].first_from is not None and plans[nxt].seq[0] == p.seq[-1]
         assert pos == tot
         assert sorted(finals) == list(range(n))
+
+
+# The backward over three ranks (a one-token chunk in the middle), with a final-state
+# gradient, an initial state, a trained norm weight and the gate.
+BW_CHUNKS = [40, 1, 55]
+
+
+def _backward_main(rank, world, port, out_dir):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import synth
+    from long_context_attn_b200 import sequence_parallel as sp
+    sp.la = _OracleBackend()
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        Tt = sum(BW_CHUNKS)
+        q, k, v, g = synth.prefill_inputs(1531, Tt, H, D, "f32", 0.5, True)
+        dout = synth.normal(1531, 11, (Tt, H * D), 1.0, "f32")
+        s0 = synth.normal(1531, 9, (H, D, D), 0.1, "f32")
+        dsT = synth.normal(1531, 10, (H, D, D), 0.1, "f32")
+        w = (1.0 + 0.2 * synth.normal(1531, 13, (H * D,), 1.0, "f32")).astype(np.float32)
+        a = sum(BW_CHUNKS[:rank])
+        b = a + BW_CHUNKS[rank]
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+        cq, ck, cv = (t(x[a:b])[None] for x in (q, k, v))
+        cg, cd = t(g[a:b])[None], t(dout[a:b])[None]
+        out = torch.zeros((1, b - a, H * D), dtype=torch.float64)
+        prefix = sp.prefill_sequence_parallel(cq, ck, cv, cg, out, rank, state0=t(s0), mode=2, norm_weight=t(w),
+                                              workspace=object())
+        dq, dk, dv = (torch.zeros((1, b - a, H, D), dtype=torch.float32) for _ in range(3))
+        dg = torch.zeros((1, b - a, H * D), dtype=torch.float32)
+        dw = torch.zeros((H * D,), dtype=torch.float32)
+        ds0 = torch.zeros((H, D, D), dtype=torch.float32)
+        sp.backward_sequence_parallel(cq, ck, cv, cg, cd, dq, dk, dv, rank, prefix, dstate_out=t(dsT), dg=dg,
+                                      dnorm_weight=dw, dstate_in=ds0, mode=2, norm_weight=t(w), workspace=object())
+        np.savez(os.path.join(out_dir, f"bw{rank}.npz"), dq=dq.numpy()[0], dk=dk.numpy()[0], dv=dv.numpy()[0],
+                 dg=dg.numpy()[0], dw=dw.numpy(), ds0=ds0.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_backward_over_three_gloo_ranks_matches_one_backward(tmp_path):
+    """Each rank's dq, dk, dv, dg, the ranks' dw summed and rank 0's initial-state gradient
+    against one oracle backward of the whole sequence (with S0, dS_T and a norm weight)."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    import synth
+    world = len(BW_CHUNKS)
+    mp.start_processes(_backward_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    Tt = sum(BW_CHUNKS)
+    q, k, v, g = synth.prefill_inputs(1531, Tt, H, D, "f32", 0.5, True)
+    dout = synth.normal(1531, 11, (Tt, H * D), 1.0, "f32")
+    s0 = synth.normal(1531, 9, (H, D, D), 0.1, "f32")
+    dsT = synth.normal(1531, 10, (H, D, D), 0.1, "f32")
+    w = (1.0 + 0.2 * synth.normal(1531, 13, (H * D,), 1.0, "f32")).astype(np.float32)
+    ref = oracle.backward(q[None], k[None], v[None], g[None], dout[None], state_in=s0[None], norm_weight=w,
+                          dstate_out=dsT[None])
+    parts = [np.load(tmp_path / f"bw{r}.npz") for r in range(world)]
+    # states, dy and the partial sums pass through fp32 between the steps: 1e-5 of the largest
+    # value covers that, while a missing or misplaced later-chunk sum is O(1)
+    for i, name in enumerate(("dq", "dk", "dv", "dg")):
+        got = np.concatenate([p[name] for p in parts])
+        want = ref[i][0]
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-5 * np.abs(want).max(), err_msg=name)
+    np.testing.assert_allclose(sum(p["dw"].astype(np.float64) for p in parts), ref[5], rtol=0,
+                               atol=1e-5 * np.abs(ref[5]).max(), err_msg="dw")
+    np.testing.assert_allclose(parts[0]["ds0"], ref[4][0], rtol=0, atol=1e-5 * np.abs(ref[4]).max(),
+                               err_msg="dS0")

@@ -89,3 +89,97 @@ def test_prefill_znorm_continuation_in_place(cuda_device):
     assert_close(np.concatenate(outs)[None], ref, "bf16")
     assert_close(to_host(S), ref_S, "bf16", "state")
     assert_close(to_host(z), ref_z, "f32", "z")
+
+
+@pytest.mark.parametrize("mode", ["raw", "rmsnorm", "rmsnorm_gate"])
+def test_output_transform_backward_matches_oracle(mode, cuda_device):
+    """lightning_attn_output_transform_backward (the norm/gate backward kernels behind their own
+    entry point): dy, dg and dw against the oracle's transform backward over 700 tokens."""
+    import torch
+    from long_context_attn_b200 import lightning_attn as la
+    from tests._helpers import mode_code
+    m = mode_code(mode)
+    tokens, H, D = 700, 8, 128
+    y = synth.normal(3451, 1, (tokens, H * D), 1.0, "bf16")
+    g = synth.normal(3451, 2, (tokens, H * D), 1.0, "bf16")
+    dout = synth.normal(3451, 3, (tokens, H * D), 1.0, "bf16")
+    w = (1.0 + 0.2 * synth.normal(3451, 4, (H * D,), 1.0, "f32")).astype(np.float32)
+    gate = m == la.LA_OUT_RMSNORM_GATE
+    dy = torch.full((tokens, H * D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    dg = torch.full((tokens, H * D), float("nan"), dtype=torch.bfloat16, device="cuda") if gate else None
+    dw = torch.full((H * D,), float("nan"), dtype=torch.float32, device="cuda")
+    ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_OUTPUT_TRANSFORM_BACKWARD, tokens, 0, 0, H, D, 0,
+                                                           la.LA_BF16, m))
+    la.lightning_attn_output_transform_backward(to_dev(y).view(tokens, H, D), to_dev(g) if gate else None,
+                                                to_dev(dout), dy, dg=dg, dnorm_weight=dw, mode=m,
+                                                norm_weight=to_dev(w), workspace=ws)
+    torch.cuda.synchronize()
+    yf = synth.bf16_to_f32(y).astype(np.float64).reshape(tokens, H, D)
+    rdy, rdg, rdw = oracle.transform_backward(yf, dout, m, norm_weight=w, g=g if gate else None)
+    assert_close(to_host(dy), rdy, "bf16", "dy")
+    if gate:
+        assert_close(to_host(dg), rdg, "bf16", "dg")
+    if m == la.LA_OUT_RAW:
+        assert torch.all(dw == 0)
+    else:
+        assert_close(to_host(dw), rdw, "bf16", "dw")
+
+
+def test_emulated_ranks_backward_match_one_backward(cuda_device):
+    """The sequence-parallel backward over three chunks (a one-token chunk in the middle), the
+    ranks emulated one after another (backward_local on every rank, a stack for the
+    all-gather, backward_finish on every rank), with an initial state, a final-state
+    gradient, a norm weight and the gate: every chunk's dq, dk, dv, dg, the chunks' dw summed
+    and the first chunk's initial-state gradient against one oracle backward."""
+    import torch
+    from long_context_attn_b200 import sequence_parallel as sp
+    H, D, C = 8, 128, 256
+    chunks = [700, 1, 333]
+    T = sum(chunks)
+    q, k, v, g = synth.prefill_inputs(1421, T, H, D, "bf16", 0.5, True)
+    dout = synth.normal(1421, 11, (T, H * D), 1.0, "bf16")
+    s0 = synth.normal(1421, 9, (H, D, D), 0.05, "f32")
+    dsT = synth.normal(1421, 10, (H, D, D), 0.05, "f32")
+    w = (1.0 + 0.2 * synth.normal(1421, 13, (H * D,), 1.0, "f32")).astype(np.float32)
+    bounds = np.cumsum([0] + chunks)
+    dw_, ds0_, dsT_ = to_dev(w), to_dev(s0), to_dev(dsT)
+    ranks = []
+    for r in range(len(chunks)):
+        a, b = bounds[r], bounds[r + 1]
+        dq, dk, dv = (to_dev(x[a:b])[None] for x in (q, k, v))
+        ranks.append((dq, dk, dv, to_dev(g[a:b])[None], to_dev(dout[a:b])[None],
+                      sp.backward_workspace_for(b - a, H, D, C)))
+    # forward steps (for each chunk's initial state)
+    fws = [sp.workspace_for(b - a, H, D, C) for a, b in zip(bounds[:-1], bounds[1:])]
+    local = [sp.chunk_state(p[1], p[2], ws) for p, ws in zip(ranks, fws)]
+    gathered = torch.stack(local)
+    prefixes = []
+    for r, (dq, dk, dv, dg, dd, _) in enumerate(ranks):
+        out = torch.empty((1, dq.shape[1], H * D), dtype=torch.bfloat16, device="cuda")
+        prefixes.append(sp.finish_chunk(dq, dk, dv, dg, out, gathered, r, fws[r], state0=ds0_, block_size=C,
+                                        norm_weight=dw_))
+    # backward steps
+    grads, dys, Gs = [], [], []
+    for r, (dq, dk, dv, dg, dd, ws) in enumerate(ranks):
+        gq, gk, gv = (torch.full_like(dq, float("nan")) for _ in range(3))
+        gg = torch.full_like(dg, float("nan"))
+        gw = torch.full((H * D,), float("nan"), dtype=torch.float32, device="cuda")
+        gs = torch.full((H, D, D), float("nan"), dtype=torch.float32, device="cuda")
+        dy, G = sp.backward_local(dq, dk, dv, dg, dd, prefixes[r], ws, dg=gg, dnorm_weight=gw, block_size=C,
+                                  norm_weight=dw_)
+        grads.append((gq, gk, gv, gg, gw, gs))
+        dys.append(dy)
+        Gs.append(G)
+    gathered = torch.stack(Gs)
+    for r, (dq, dk, dv, dg, dd, ws) in enumerate(ranks):
+        gq, gk, gv, gg, gw, gs = grads[r]
+        sp.backward_finish(dq, dk, dv, dys[r], gq, gk, gv, gathered, r, prefixes[r], ws, dstate_out=dsT_,
+                           dstate_in=gs, block_size=C)
+    torch.cuda.synchronize()
+    ref = oracle.backward(q[None], k[None], v[None], g[None], dout[None], state_in=s0[None], norm_weight=w,
+                          dstate_out=dsT[None])
+    for i, name in enumerate(("dq", "dk", "dv", "dg")):
+        got = np.concatenate([to_host(grads[r][i])[0] for r in range(len(chunks))])
+        assert_close(got[None], ref[i], "bf16", name)
+    assert_close(sum(to_host(grads[r][4]).astype(np.float64) for r in range(len(chunks))), ref[5], "bf16", "dw")
+    assert_close(to_host(grads[0][5]), ref[4][0], "bf16", "dS0")
