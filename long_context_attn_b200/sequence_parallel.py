@@ -280,38 +280,50 @@ def varlen_carry(k, v, plan: VarlenSlice, workspace, phi: int = la.LA_PHI_SILU, 
     return state[0]
 
 
-def varlen_finish(q, k, v, g, out, gathered, plan: VarlenSlice, rank: int, workspace, state0=None,
-                  block_size: int = 256, phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE,
-                  eps: float = 1e-6, norm_weight=None, stream=None):
-    """Step 3: the slice's varlen prefill, its first piece starting from state0 of its sequence
+def varlen_initial_states(plan: VarlenSlice, gathered, rank: int, state0=None, device="cuda", stream=None):
+    """The initial state of every piece of the slice, fp32 [len(plan.seq), H, D, D] (None when
+    all are zero): state0 of its sequence, and for a first piece that continues a sequence,
     plus the gathered states [world, H, D, D] of the ranks from the one where that sequence
-    starts up to this one.  q, k, v [L, H, D]; g, out [L, H*D]; state0 fp32 [N, H, D, D] (all
-    sequences; None: zero).  Returns the states after each piece, fp32 [len(plan.seq), H, D, D]
-    (the sequences' final states where plan.final)."""
-    _, H, D = q.shape
+    starts up to this one."""
     m = len(plan.seq)
-    st_out = torch.empty((m, H, D, D), dtype=torch.float32, device=q.device)
     if m == 0:
-        return st_out
+        return None
+    _, H, D, _ = gathered.shape
     s0 = plan.seq[0]
     st_in = None if state0 is None else state0[s0:s0 + m]
     if plan.first_from is not None:
-        st_in = (torch.zeros((m, H, D, D), dtype=torch.float32, device=q.device) if st_in is None
+        st_in = (torch.zeros((m, H, D, D), dtype=torch.float32, device=device) if st_in is None
                  else st_in.clone())
         r0 = plan.first_from
         la.lightning_attn_state_prefix(gathered[r0:rank + 1], rank - r0, st_in[0],
                                        state0=None if state0 is None else state0[s0], stream=stream)
+    return st_in
+
+
+def varlen_finish(q, k, v, g, out, gathered, plan: VarlenSlice, rank: int, workspace, state0=None,
+                  block_size: int = 256, phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE,
+                  eps: float = 1e-6, norm_weight=None, stream=None):
+    """Step 3: the slice's varlen prefill, every piece from its initial state
+    (varlen_initial_states).  q, k, v [L, H, D]; g, out [L, H*D]; state0 fp32 [N, H, D, D] (all
+    sequences; None: zero).  Returns (the states after each piece, fp32 [len(plan.seq), H, D, D]
+    -- the sequences' final states where plan.final --, the pieces' initial states or None)."""
+    _, H, D = q.shape
+    m = len(plan.seq)
+    st_out = torch.empty((m, H, D, D), dtype=torch.float32, device=q.device)
+    if m == 0:
+        return st_out, None
+    st_in = varlen_initial_states(plan, gathered, rank, state0, q.device, stream)
     if plan.hi == plan.lo:   # only empty sequences: each keeps its initial state
         if st_in is None:
             st_out.zero_()
         else:
             st_out.copy_(st_in)
-        return st_out
+        return st_out, st_in
     cu = torch.from_numpy(plan.local_cu).to(q.device)
     la.lightning_attn_prefill_varlen(q, k, v, g, out, cu, plan.max_len, state_in=st_in, state_out=st_out,
                                      block_size=block_size, phi=phi, mode=mode, eps=eps, norm_weight=norm_weight,
                                      workspace=workspace, stream=stream)
-    return st_out
+    return st_out, st_in
 
 
 def prefill_varlen_sequence_parallel(q, k, v, g, out, cu_seqlens, bounds, rank: int, all_gather=nccl_all_gather,
@@ -320,7 +332,8 @@ def prefill_varlen_sequence_parallel(q, k, v, g, out, cu_seqlens, bounds, rank: 
                                      workspace=None, stream=None):
     """This rank's part of a sequence-parallel prefill of a packed batch (steps 1-3).
     cu_seqlens and bounds are host arrays, the same on every rank; q, k, v [L, H, D] and g,
-    out [L, H*D] hold this rank's slice.  Returns (plan, states after each piece)."""
+    out [L, H*D] hold this rank's slice.  Returns (plan, the states after each piece, the
+    pieces' initial states or None -- the backward takes them)."""
     _, H, D = q.shape
     plan = varlen_slice_plan(cu_seqlens, bounds, rank)
     if q.shape[0] != plan.hi - plan.lo:
@@ -329,6 +342,120 @@ def prefill_varlen_sequence_parallel(q, k, v, g, out, cu_seqlens, bounds, rank: 
         workspace = varlen_workspace_for(plan, H, D, block_size, mode, q.device, la._dtype(q))
     carry = varlen_carry(k, v, plan, workspace, phi, stream)
     gathered = all_gather(carry)
-    st = varlen_finish(q, k, v, g, out, gathered, plan, rank, workspace, state0, block_size, phi, mode, eps,
-                       norm_weight, stream)
-    return plan, st
+    st_out, st_in = varlen_finish(q, k, v, g, out, gathered, plan, rank, workspace, state0, block_size, phi, mode,
+                                  eps, norm_weight, stream)
+    return plan, st_out, st_in
+
+
+def varlen_backward_workspace_for(plan: VarlenSlice, H: int, D: int, block_size: int = 256,
+                                  mode: int = la.LA_OUT_RMSNORM_GATE, device="cuda", dtype: int = la.LA_BF16):
+    """One workspace for every call of the packed-batch backward on this slice."""
+    n, L, m = 256, plan.hi - plan.lo, len(plan.seq)
+    if m:
+        n = max(n, la.lightning_attn_workspace_size(la.LA_OP_PREFILL_VARLEN, m, plan.max_len, L, H, D, block_size,
+                                                    dtype, la.LA_OUT_RAW),
+                la.lightning_attn_workspace_size(la.LA_OP_BACKWARD_VARLEN, m, plan.max_len, L, H, D, block_size,
+                                                 dtype, la.LA_OUT_RAW),
+                la.lightning_attn_workspace_size(la.LA_OP_OUTPUT_TRANSFORM_BACKWARD, L, 0, 0, H, D, 0, dtype, mode))
+    if plan.first_from is not None:
+        first = int(plan.local_cu[1])
+        n = max(n, la.lightning_attn_workspace_size(la.LA_OP_CHUNK_STATE, 1, first, 0, H, D, 0, dtype, 0))
+    return la.new_workspace(n, device)
+
+
+def varlen_backward_local(q, k, v, g, dout, plan: VarlenSlice, st_in, workspace, y=None, dg=None, dnorm_weight=None,
+                          block_size: int = 256, phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE,
+                          eps: float = 1e-6, norm_weight=None, stream=None):
+    """Backward steps 1-2 on this rank's slice of a packed batch: dy (and dg, the slice's terms
+    of dw) through the output transform of the slice's raw output y (given, or recomputed from
+    the pieces' initial states st_in), then G = sum of phi(q_t) dy_t^T over the first piece
+    when it continues a sequence from an earlier rank (zero otherwise: the sums that later
+    ranks need only come from pieces that continue a sequence).  q, k, v [L, H, D]; g, dout
+    [L, H*D].  Returns (dy [L, H*D], G fp32 [H, D, D])."""
+    L, H, D = q.shape
+    if mode == la.LA_OUT_RAW:
+        dy = dout
+        if dnorm_weight is not None:
+            dnorm_weight.zero_()
+    else:
+        if y is None:
+            y = torch.empty_like(dout)
+            if L:
+                cu = torch.from_numpy(plan.local_cu).to(q.device)
+                la.lightning_attn_prefill_varlen(q, k, v, None, y, cu, plan.max_len, state_in=st_in,
+                                                 block_size=block_size, phi=phi, mode=la.LA_OUT_RAW,
+                                                 workspace=workspace, stream=stream)
+        dy = torch.empty_like(dout)
+        la.lightning_attn_output_transform_backward(y.view(L, H, D), g, dout, dy, dg=dg, dnorm_weight=dnorm_weight,
+                                                    mode=mode, eps=eps, norm_weight=norm_weight, workspace=workspace,
+                                                    stream=stream)
+    G = torch.zeros((1, H, D, D), dtype=torch.float32, device=q.device)
+    if plan.first_from is not None:
+        e = int(plan.local_cu[1])
+        la.lightning_attn_chunk_state(q[:e][None], dy[:e].view(1, e, H, D), G, phi=phi, workspace=workspace,
+                                      stream=stream)
+    return dy, G[0]
+
+
+def varlen_backward_finish(q, k, v, dy, dq, dk, dv, gathered, plan: VarlenSlice, cu_seqlens, bounds, rank: int, st_in,
+                           workspace, dstate_out=None, dstate_in=None, block_size: int = 256,
+                           phi: int = la.LA_PHI_SILU, stream=None):
+    """Backward steps 3-4: each piece's end-of-piece gradient -- dstate_out of its sequence
+    (fp32 [N, H, D, D] for all sequences, None: zero), plus, for a last piece whose sequence
+    goes on, the gathered sums [world, H, D, D] of the later ranks up to the one holding the
+    sequence's last token -- then the slice's backward in raw mode from dy with the pieces'
+    initial states st_in.  dstate_in (fp32 [len(plan.seq), H, D, D] or None) receives each
+    piece's initial-state gradient (for a piece that starts its sequence, the gradient of
+    that sequence's initial state)."""
+    L, H, D = q.shape
+    m = len(plan.seq)
+    if m == 0:
+        return
+    s0 = plan.seq[0]
+    ds_end = None if dstate_out is None else dstate_out[s0:s0 + m]
+    if plan.carries:
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+        b = np.asarray(bounds, dtype=np.int64)
+        s_last = plan.seq[-1]
+        r_end = int(np.searchsorted(b, cu[s_last + 1] - 1, side="right")) - 1   # holds the last token
+        later = gathered[rank + 1:r_end + 1]
+        ds_end = (torch.zeros((m, H, D, D), dtype=torch.float32, device=q.device) if ds_end is None
+                  else ds_end.clone())
+        pad = torch.cat([later, torch.zeros((1, H, D, D), dtype=torch.float32, device=q.device)])
+        la.lightning_attn_state_prefix(pad, later.shape[0], ds_end[m - 1],
+                                       state0=None if dstate_out is None else dstate_out[s_last], stream=stream)
+    if L == 0:   # only empty sequences: the initial-state gradient is the final one
+        if dstate_in is not None:
+            if ds_end is None:
+                dstate_in.zero_()
+            else:
+                dstate_in.copy_(ds_end)
+        return
+    cu_local = torch.from_numpy(plan.local_cu).to(q.device)
+    la.lightning_attn_backward_varlen(q, k, v, None, dy, dq, dk, dv, cu_local, plan.max_len, state_in=st_in,
+                                      dstate_in=dstate_in, block_size=block_size, phi=phi, mode=la.LA_OUT_RAW,
+                                      workspace=workspace, stream=stream, dstate_out=ds_end)
+
+
+def backward_varlen_sequence_parallel(q, k, v, g, dout, dq, dk, dv, cu_seqlens, bounds, rank: int, st_in,
+                                      all_gather=nccl_all_gather, dstate_out=None, y=None, dg=None,
+                                      dnorm_weight=None, dstate_in=None, block_size: int = 256,
+                                      phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE,
+                                      eps: float = 1e-6, norm_weight=None, workspace=None, stream=None):
+    """This rank's part of the backward of prefill_varlen_sequence_parallel: st_in is the
+    pieces' initial states it returned; dstate_out fp32 [N, H, D, D] (all sequences, the same
+    on every rank) or None; dstate_in fp32 [len(plan.seq), H, D, D] or None; dnorm_weight
+    receives this slice's part of the norm weight's gradient (sum it over the ranks).
+    Returns the plan."""
+    L, H, D = q.shape
+    plan = varlen_slice_plan(cu_seqlens, bounds, rank)
+    if L != plan.hi - plan.lo:
+        raise ValueError("q holds %d tokens, the slice %d" % (L, plan.hi - plan.lo))
+    if workspace is None:
+        workspace = varlen_backward_workspace_for(plan, H, D, block_size, mode, q.device, la._dtype(q))
+    dy, G = varlen_backward_local(q, k, v, g, dout, plan, st_in, workspace, y, dg, dnorm_weight, block_size, phi,
+                                  mode, eps, norm_weight, stream)
+    gathered = all_gather(G)
+    varlen_backward_finish(q, k, v, dy, dq, dk, dv, gathered, plan, cu_seqlens, bounds, rank, st_in, workspace,
+                           dstate_out, dstate_in, block_size, phi, stream)
+    return plan

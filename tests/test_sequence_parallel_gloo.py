@@ -53,13 +53,14 @@ class _OracleBackend:
         cu = cu_seqlens.numpy()
         assert cu.dtype == np.int32 and int(max_seqlen) >= int(np.diff(cu).max())
         assert state_in is None or (state_in.dtype == torch.float32 and state_in.is_contiguous())
-        assert state_out.dtype == torch.float32 and state_out.shape[0] == cu.size - 1
+        assert state_out is None or (state_out.dtype == torch.float32 and state_out.shape[0] == cu.size - 1)
         _, H, D = q.shape
         o, st, _ = self.oracle.forward_packed(q.numpy(), k.numpy(), v.numpy(), None if g is None else g.numpy(), cu,
                                               H, D, state_in=None if state_in is None else state_in.numpy(),
                                               phi=phi, mode=mode, eps=eps)
         out.copy_(torch.from_numpy(o))
-        state_out.copy_(torch.from_numpy(st))
+        if state_out is not None:
+            state_out.copy_(torch.from_numpy(st))
 
     def lightning_attn_prefill(self, q, k, v, g, out, state_in, state_out, block_size=256, phi=0, mode=2,
                                eps=1e-6, norm_weight=None, workspace=None, stream=None):
@@ -100,6 +101,28 @@ class _OracleBackend:
         ref = self.oracle.backward(q.numpy(), k.numpy(), v.numpy(), npy(g), dout.numpy(), state_in=npy(state_in),
                                    phi=phi, mode=mode, eps=eps, norm_weight=npy(norm_weight),
                                    dstate_out=npy(dstate_out))
+        for t, r in zip((dq, dk, dv, dg, dstate_in), ref):
+            if t is not None:
+                t.copy_(torch.from_numpy(r).view(t.shape))
+        if dnorm_weight is not None:
+            dnorm_weight.copy_(torch.from_numpy(ref[5]))
+
+    def lightning_attn_backward_varlen(self, q, k, v, g, dout, dq, dk, dv, cu_seqlens, max_seqlen, dg=None,
+                                       state_in=None, dstate_in=None, block_size=256, phi=0, mode=2, eps=1e-6,
+                                       norm_weight=None, workspace=None, stream=None, dstate_out=None, y=None,
+                                       dnorm_weight=None):
+        import torch
+        self._bind("lightning_attn_backward_varlen", q, k, v, g, dout, dq, dk, dv, cu_seqlens, max_seqlen, dg=dg,
+                   state_in=state_in, dstate_in=dstate_in, block_size=block_size, phi=phi, mode=mode, eps=eps,
+                   norm_weight=norm_weight, workspace=workspace, stream=stream, dstate_out=dstate_out, y=y,
+                   dnorm_weight=dnorm_weight)
+        cu = cu_seqlens.numpy()
+        assert cu.dtype == np.int32 and int(max_seqlen) >= int(np.diff(cu).max()) and q.dim() == 3
+        _, H, D = q.shape
+        npy = lambda t: None if t is None else t.numpy()
+        ref = self.oracle.backward_packed(q.numpy(), k.numpy(), v.numpy(), npy(g), dout.numpy(), cu, H, D,
+                                          state_in=npy(state_in), phi=phi, mode=mode, eps=eps,
+                                          norm_weight=npy(norm_weight), dstate_out=npy(dstate_out))
         for t, r in zip((dq, dk, dv, dg, dstate_in), ref):
             if t is not None:
                 t.copy_(torch.from_numpy(r).view(t.shape))
@@ -198,7 +221,7 @@ def _varlen_main(rank, world, port, out_dir):
         a, b = VL_BOUNDS[rank], VL_BOUNDS[rank + 1]
         t = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
         out = torch.zeros((b - a, H * D), dtype=torch.float64)
-        plan, st = sp.prefill_varlen_sequence_parallel(t(q[a:b]), t(k[a:b]), t(v[a:b]), t(g[a:b]), out, cu,
+        plan, st, _ = sp.prefill_varlen_sequence_parallel(t(q[a:b]), t(k[a:b]), t(v[a:b]), t(g[a:b]), out, cu,
                                                        VL_BOUNDS, rank, state0=t(s0), mode=2, workspace=object())
         np.save(os.path.join(out_dir, f"vout{rank}.npy"), out.numpy())
         fin = {int(s): st[i].numpy() for i, s in enumerate(plan.seq) if plan.final[i]}
@@ -346,3 +369,79 @@ def test_backward_over_three_gloo_ranks_matches_one_backward(tmp_path):
                                atol=1e-5 * np.abs(ref[5]).max(), err_msg="dw")
     np.testing.assert_allclose(parts[0]["ds0"], ref[4][0], rtol=0, atol=1e-5 * np.abs(ref[4]).max(),
                                err_msg="dS0")
+
+
+
+def _varlen_backward_main(rank, world, port, out_dir):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import synth
+    from long_context_attn_b200 import sequence_parallel as sp
+    sp.la = _OracleBackend()
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        cu = synth.cu_seqlens_of(VL_LENS)
+        tot, n = int(cu[-1]), len(VL_LENS)
+        q, k, v, g = synth.prefill_inputs(1541, tot, H, D, "f32", 0.5, True)
+        dout = synth.normal(1541, 11, (tot, H * D), 1.0, "f32")
+        s0 = synth.normal(1541, 9, (n, H, D, D), 0.1, "f32")
+        dsT = synth.normal(1541, 10, (n, H, D, D), 0.1, "f32")
+        w = (1.0 + 0.2 * synth.normal(1541, 13, (H * D,), 1.0, "f32")).astype(np.float32)
+        a, b = VL_BOUNDS[rank], VL_BOUNDS[rank + 1]
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+        cq, ck, cv, cg, cd = (t(x[a:b]) for x in (q, k, v, g, dout))
+        out = torch.zeros((b - a, H * D), dtype=torch.float32)
+        plan, _, st_in = sp.prefill_varlen_sequence_parallel(cq, ck, cv, cg, out, cu, VL_BOUNDS, rank, state0=t(s0),
+                                                             mode=2, norm_weight=t(w), workspace=object())
+        dq, dk, dv = (torch.zeros((b - a, H, D), dtype=torch.float32) for _ in range(3))
+        dg = torch.zeros((b - a, H * D), dtype=torch.float32)
+        dw = torch.zeros((H * D,), dtype=torch.float32)
+        ds_in = torch.zeros((len(plan.seq), H, D, D), dtype=torch.float32)
+        sp.backward_varlen_sequence_parallel(cq, ck, cv, cg, cd, dq, dk, dv, cu, VL_BOUNDS, rank, st_in,
+                                             dstate_out=t(dsT), dg=dg, dnorm_weight=dw, dstate_in=ds_in, mode=2,
+                                             norm_weight=t(w), workspace=object())
+        starts = {int(s): ds_in[i].numpy() for i, s in enumerate(plan.seq) if not (i == 0 and plan.first_from is not None)}
+        np.savez(os.path.join(out_dir, f"vbw{rank}.npz"), dq=dq.numpy(), dk=dk.numpy(), dv=dv.numpy(), dg=dg.numpy(),
+                 dw=dw.numpy())
+        np.save(os.path.join(out_dir, f"vbs{rank}.npy"), starts, allow_pickle=True)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_varlen_backward_over_five_gloo_ranks_matches_one_packed_backward(tmp_path):
+    """The packed batch and cuts of the varlen forward test, backwards: every token's dq, dk,
+    dv, dg, the ranks' dw summed and every sequence's initial-state gradient (from the rank
+    where the sequence starts) against one oracle backward of the whole batch with initial
+    states, final-state gradients and a norm weight."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    import synth
+    world = len(VL_BOUNDS) - 1
+    mp.start_processes(_varlen_backward_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    cu = synth.cu_seqlens_of(VL_LENS)
+    tot, n = int(cu[-1]), len(VL_LENS)
+    q, k, v, g = synth.prefill_inputs(1541, tot, H, D, "f32", 0.5, True)
+    dout = synth.normal(1541, 11, (tot, H * D), 1.0, "f32")
+    s0 = synth.normal(1541, 9, (n, H, D, D), 0.1, "f32")
+    dsT = synth.normal(1541, 10, (n, H, D, D), 0.1, "f32")
+    w = (1.0 + 0.2 * synth.normal(1541, 13, (H * D,), 1.0, "f32")).astype(np.float32)
+    ref = oracle.backward_packed(q, k, v, g, dout, cu, H, D, state_in=s0, norm_weight=w, dstate_out=dsT)
+    parts = [np.load(tmp_path / f"vbw{r}.npz") for r in range(world)]
+    for i, name in enumerate(("dq", "dk", "dv", "dg")):
+        got = np.concatenate([p[name] for p in parts])
+        np.testing.assert_allclose(got, ref[i], rtol=0, atol=1e-5 * np.abs(ref[i]).max(), err_msg=name)
+    np.testing.assert_allclose(sum(p["dw"].astype(np.float64) for p in parts), ref[5], rtol=0,
+                               atol=1e-5 * np.abs(ref[5]).max(), err_msg="dw")
+    starts = {}
+    for r in range(world):
+        part = np.load(tmp_path / f"vbs{r}.npy", allow_pickle=True).item()
+        assert not set(part) & set(starts)
+        starts.update(part)
+    assert sorted(starts) == list(range(n))
+    for s, ds in starts.items():
+        np.testing.assert_allclose(ds, ref[4][s], rtol=0, atol=1e-5 * np.abs(ref[4]).max(), err_msg=f"dS0 {s}")

@@ -47,7 +47,7 @@ def test_emulated_ranks_varlen_batch_match_one_packed_prefill(cuda_device):
     gathered = torch.stack(carries)
     finals = {}
     for r, (plan, dq, dk, dv, dg, out, ws) in enumerate(ranks):
-        st = sp.varlen_finish(dq, dk, dv, dg, out, gathered, plan, r, ws, state0=ds0, block_size=C)
+        st, _ = sp.varlen_finish(dq, dk, dv, dg, out, gathered, plan, r, ws, state0=ds0, block_size=C)
         la.lightning_attn_check(ws)
         for i, s in enumerate(plan.seq):
             if plan.final[i]:
@@ -183,3 +183,69 @@ def test_emulated_ranks_backward_match_one_backward(cuda_device):
         assert_close(got[None], ref[i], "bf16", name)
     assert_close(sum(to_host(grads[r][4]).astype(np.float64) for r in range(len(chunks))), ref[5], "bf16", "dw")
     assert_close(to_host(grads[0][5]), ref[4][0], "bf16", "dS0")
+
+
+def test_emulated_ranks_varlen_backward_match_one_packed_backward(cuda_device):
+    """The packed batch and cuts of the varlen forward test above, backwards, the ranks emulated
+    one after another (varlen_backward_local on every rank, a stack for the all-gather,
+    varlen_backward_finish on every rank): every token's dq, dk, dv, dg, the ranks' dw summed
+    and every sequence's initial-state gradient against one oracle backward of the batch."""
+    import torch
+    from long_context_attn_b200 import sequence_parallel as sp
+    H, D, C = 8, 128, 256
+    lens = [300, 0, 900, 129, 1000, 0, 257, 0]
+    bounds = [0, 500, 500, 1200, 1700, 2586]
+    cu = synth.cu_seqlens_of(lens)
+    tot, n = int(cu[-1]), len(lens)
+    q, k, v, g = synth.prefill_inputs(1431, tot, H, D, "bf16", 0.5, True)
+    dout = synth.normal(1431, 11, (tot, H * D), 1.0, "bf16")
+    s0 = synth.normal(1431, 9, (n, H, D, D), 0.05, "f32")
+    dsT = synth.normal(1431, 10, (n, H, D, D), 0.05, "f32")
+    w = (1.0 + 0.2 * synth.normal(1431, 13, (H * D,), 1.0, "f32")).astype(np.float32)
+    ds0_, dsT_, dw_ = to_dev(s0), to_dev(dsT), to_dev(w)
+    world = len(bounds) - 1
+    ranks = []
+    for r in range(world):
+        a, b = bounds[r], bounds[r + 1]
+        plan = sp.varlen_slice_plan(cu, bounds, r)
+        ranks.append((plan, *(to_dev(x[a:b]) for x in (q, k, v, g, dout)),
+                      sp.varlen_workspace_for(plan, H, D, C), sp.varlen_backward_workspace_for(plan, H, D, C)))
+    # forward: the pieces' initial states
+    carries = [sp.varlen_carry(dk, dv, plan, fws) for plan, dq, dk, dv, dg, dd, fws, bws in ranks]
+    gathered = torch.stack(carries)
+    st_ins = []
+    for r, (plan, dq, dk, dv, dg, dd, fws, bws) in enumerate(ranks):
+        out = torch.empty((plan.hi - plan.lo, H * D), dtype=torch.bfloat16, device="cuda")
+        _, st_in = sp.varlen_finish(dq, dk, dv, dg, out, gathered, plan, r, fws, state0=ds0_, block_size=C,
+                                    norm_weight=dw_)
+        st_ins.append(st_in)
+    # backward
+    grads, dys, Gs = [], [], []
+    for r, (plan, dq, dk, dv, dg, dd, fws, bws) in enumerate(ranks):
+        gq, gk, gv = (torch.full_like(dq, float("nan")) for _ in range(3))
+        gg = torch.full_like(dg, float("nan"))
+        gw = torch.full((H * D,), float("nan"), dtype=torch.float32, device="cuda")
+        gs = torch.full((len(plan.seq), H, D, D), float("nan"), dtype=torch.float32, device="cuda")
+        dy, G = sp.varlen_backward_local(dq, dk, dv, dg, dd, plan, st_ins[r], bws, dg=gg, dnorm_weight=gw,
+                                         block_size=C, norm_weight=dw_)
+        grads.append((gq, gk, gv, gg, gw, gs))
+        dys.append(dy)
+        Gs.append(G)
+    gathered = torch.stack(Gs)
+    starts = {}
+    for r, (plan, dq, dk, dv, dg, dd, fws, bws) in enumerate(ranks):
+        gq, gk, gv, gg, gw, gs = grads[r]
+        sp.varlen_backward_finish(dq, dk, dv, dys[r], gq, gk, gv, gathered, plan, cu, bounds, r, st_ins[r], bws,
+                                  dstate_out=dsT_, dstate_in=gs, block_size=C)
+        for i, s in enumerate(plan.seq):
+            if not (i == 0 and plan.first_from is not None):
+                assert s not in starts
+                starts[s] = gs[i]
+    torch.cuda.synchronize()
+    assert sorted(starts) == list(range(n))
+    ref = oracle.backward_packed(q, k, v, g, dout, cu, H, D, state_in=s0, norm_weight=w, dstate_out=dsT)
+    for i, name in enumerate(("dq", "dk", "dv", "dg")):
+        got = np.concatenate([to_host(grads[r][i]) for r in range(world)])
+        assert_close(got, ref[i], "bf16", name)
+    assert_close(sum(to_host(grads[r][4]).astype(np.float64) for r in range(world)), ref[5], "bf16", "dw")
+    assert_close(np.stack([to_host(starts[s]) for s in range(n)]), ref[4], "bf16", "dS0")
