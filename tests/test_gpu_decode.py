@@ -4,7 +4,7 @@ import pytest
 
 import oracle
 import synth
-from tests._helpers import TOL, as_f64, assert_close, mode_code, rel_err, to_dev, to_host
+from tests._helpers import as_f64, assert_close, mode_code, rel_err, to_dev, to_host
 
 pytestmark = pytest.mark.gpu
 

@@ -6,7 +6,6 @@ out (a flag that nothing sets).  With a 50 ms limit written into the workspace, 
 must report LA_ERR_TIMEOUT through lightning_attn_check, the kernel must end on its own,
 and the context must stay usable: a normal call right after gives the oracle's result.
 """
-import numpy as np
 import pytest
 
 import oracle

@@ -14,7 +14,7 @@ import pytest
 
 import oracle
 import synth
-from tests._helpers import as_f64, assert_close, mode_code, rel_err, to_dev, to_host
+from tests._helpers import as_f64, assert_close, mode_code
 from tests.test_gpu_prefill_simt import run_prefill, run_varlen
 
 pytestmark = pytest.mark.gpu

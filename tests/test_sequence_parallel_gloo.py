@@ -4,7 +4,6 @@ The kernels are replaced by the fp64 oracle (this checks the ordering of the cal
 real all-gather over the process group and the prefix arithmetic, not the GPU code):
 rank r's chunk output and the last rank's state must equal one oracle prefill of the whole
 sequence."""
-import json
 import os
 import socket
 import sys
