@@ -249,3 +249,27 @@ def test_emulated_ranks_varlen_backward_match_one_packed_backward(cuda_device):
         assert_close(got, ref[i], "bf16", name)
     assert_close(sum(to_host(grads[r][4]).astype(np.float64) for r in range(world)), ref[5], "bf16", "dw")
     assert_close(np.stack([to_host(starts[s]) for s in range(n)]), ref[4], "bf16", "dS0")
+
+
+@pytest.mark.parametrize("chunk", [4096, 20000])
+def test_host_prefill_pipeline_matches_one_prefill(chunk, cuda_device):
+    """HostPrefill: a 10000-token sequence in pinned host memory, chunks pipelined over three
+    streams (4096: three chunks with a ragged last one; 20000: one chunk), from an initial
+    state: the host output and the final state against one oracle prefill."""
+    import torch
+    from long_context_attn_b200.host_stream import HostPrefill
+    H, D, T = 8, 128, 10000
+    q, k, v, g = synth.prefill_inputs(1441, T, H, D, "bf16", 0.5, True)
+    s0 = synth.normal(1441, 9, (H, D, D), 0.05, "f32")
+    pin = lambda a, shape: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).reshape(shape).pin_memory()
+    hq, hk, hv = (pin(a, (T, H, D)) for a in (q, k, v))
+    hg = pin(g, (T, H * D))
+    hout = torch.full((T, H * D), float("nan"), dtype=torch.bfloat16).pin_memory()
+    st = torch.full((H, D, D), float("nan"), dtype=torch.float32, device="cuda")
+    hp = HostPrefill(H, D, chunk_tokens=chunk)
+    hp(hq, hk, hv, hg, hout, state_in=to_dev(s0), state_out=st)
+    torch.cuda.current_stream().synchronize()
+    hp.check()
+    ref, ref_st, _ = oracle.prefill(q[None], k[None], v[None], g[None], state_in=s0[None])
+    assert_close(hout.float().numpy()[None], ref, "bf16")
+    assert_close(to_host(st)[None], ref_st, "bf16", "final state")
