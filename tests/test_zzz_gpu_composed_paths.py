@@ -2,7 +2,8 @@
 the sequence-parallel prefill of a packed variable-length batch (ranks emulated one after
 another on one GPU: a stack stands in for the all-gather, no kernel waits on another) and
 the normalised variant continued in place (state_out = state_in, z_out = z_in).  Collected
-after the per-kernel files, so a failure here never hides theirs."""
+after every other file (the per-kernel ones and the workspace-free decode), so a
+failure here never hides theirs."""
 import numpy as np
 import pytest
 
