@@ -1,9 +1,10 @@
 """GPU tests of paths composed from calls that the per-kernel files test on their own:
-the sequence-parallel prefill of a packed variable-length batch (ranks emulated one after
-another on one GPU: a stack stands in for the all-gather, no kernel waits on another) and
-the normalised variant continued in place (state_out = state_in, z_out = z_in).  Collected
-after every other file (the per-kernel ones and the workspace-free decode), so a
-failure here never hides theirs."""
+the sequence-parallel prefill and backward (one sequence or a packed variable-length batch;
+ranks emulated one after another on one GPU: a stack stands in for the all-gather, no
+kernel waits on another), the output transform's backward as its own entry point, the
+normalised variant continued in place (state_out = state_in, z_out = z_in) and the
+host-memory prefill with overlapped copies.  Collected after every other file (the
+per-kernel ones and the workspace-free decode), so a failure here never hides theirs."""
 import numpy as np
 import pytest
 
