@@ -15,6 +15,7 @@ from __future__ import annotations
 import torch
 
 from . import lightning_attn as la
+from . import sequence_parallel as sp
 
 
 class _LightningAttention(torch.autograd.Function):
@@ -76,3 +77,69 @@ def lightning_attention(q, k, v, g=None, state_in=None, block_size: int = 256, p
     if norm_weight is not None:
         norm_weight = norm_weight.float().contiguous()
     return _LightningAttention.apply(q, k, v, g, state_in, block_size, phi, mode, eps, norm_weight)
+
+
+class _SequenceParallelLightningAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, g, state0, norm_weight, rank, all_gather, block_size, phi, mode, eps):
+        _, T, H, D = q.shape
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        g = None if g is None else g.contiguous()
+        s0 = None if state0 is None else state0.detach().contiguous()
+        w = None if norm_weight is None else norm_weight.detach().contiguous()
+        out = torch.empty((1, T, H * D), dtype=q.dtype, device=q.device)
+        state_end = torch.empty((H, D, D), dtype=torch.float32, device=q.device)
+        ws = sp.workspace_for(T, H, D, block_size, mode, q.device, la._dtype(q))
+        y = None
+        if mode != la.LA_OUT_RAW and any(ctx.needs_input_grad[:6]):   # keep the raw output for the backward
+            y = torch.empty_like(out)
+            prefix = sp.prefill_sequence_parallel(q, k, v, None, y, rank, all_gather, state0=s0, state_out=state_end,
+                                                  block_size=block_size, phi=phi, mode=la.LA_OUT_RAW, workspace=ws)
+            la.lightning_attn_output_transform(y.view(1, T, H, D), g, out, mode=mode, eps=eps, norm_weight=w)
+        else:
+            prefix = sp.prefill_sequence_parallel(q, k, v, g, out, rank, all_gather, state0=s0, state_out=state_end,
+                                                  block_size=block_size, phi=phi, mode=mode, eps=eps, norm_weight=w,
+                                                  workspace=ws)
+        ctx.save_for_backward(q, k, v, g, prefix, w, y)
+        ctx.cfg = (rank, all_gather, block_size, phi, mode, eps, state0 is not None)
+        return out, state_end
+
+    @staticmethod
+    def backward(ctx, dout, dstate_end):
+        q, k, v, g, prefix, w, y = ctx.saved_tensors
+        rank, all_gather, block_size, phi, mode, eps, has_s0 = ctx.cfg
+        _, T, H, D = q.shape
+        if dout is None:
+            dout = torch.zeros((1, T, H * D), dtype=q.dtype, device=q.device)
+        dout = dout.to(q.dtype).contiguous()
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        dg = torch.empty_like(g) if mode == la.LA_OUT_RMSNORM_GATE else None
+        dw = torch.empty((H * D,), dtype=torch.float32, device=q.device) if ctx.needs_input_grad[5] else None
+        ds_in = torch.empty((H, D, D), dtype=torch.float32, device=q.device) if has_s0 else None
+        sp.backward_sequence_parallel(q, k, v, g, dout, dq, dk, dv, rank, prefix, all_gather,
+                                      dstate_end=None if dstate_end is None else dstate_end.float().contiguous(),
+                                      y=y, dg=dg, dnorm_weight=dw, dstate_in=ds_in, block_size=block_size, phi=phi,
+                                      mode=mode, eps=eps, norm_weight=w)
+        # state0 is the same tensor on every rank: rank 0 returns its whole gradient and the
+        # others zero, so that adding the ranks' gradients (as for the norm weight's per-chunk
+        # parts) gives the total
+        if ds_in is not None and rank != 0:
+            ds_in.zero_()
+        return dq, dk, dv, dg, ds_in, dw, None, None, None, None, None, None
+
+
+def lightning_attention_sequence_parallel(q, k, v, g=None, state0=None, norm_weight=None, rank: int = 0,
+                                          all_gather=sp.nccl_all_gather, block_size: int = 256,
+                                          phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE,
+                                          eps: float = 1e-6):
+    """Differentiable sequence-parallel prefill: this rank's contiguous chunk q, k, v
+    [1, T, H, D] (g [1, T, H*D]) of one sequence split across the group's ranks in order.
+    Returns (out [1, T, H*D], the state at the end of this chunk fp32 [H, D, D]: on the last
+    rank the sequence's final state).  One all-gather in the forward and one in the backward,
+    so every rank must call it in the same order and back-propagate through its output.
+    Gradients of state0 and the norm weight (the same tensors on every rank) come as per-rank
+    parts to be added over the ranks, as data-parallel gradients are."""
+    if norm_weight is not None:
+        norm_weight = norm_weight.float().contiguous()
+    return _SequenceParallelLightningAttention.apply(q, k, v, g, state0, norm_weight, rank, all_gather, block_size,
+                                                     phi, mode, eps)

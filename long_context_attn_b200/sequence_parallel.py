@@ -118,13 +118,15 @@ def backward_workspace_for(T: int, H: int, D: int, block_size: int = 256, mode: 
     return la.new_workspace(n, device)
 
 
-def backward_local(q, k, v, g, dout, prefix, workspace, y=None, dg=None, dnorm_weight=None, block_size: int = 256,
-                   phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE, eps: float = 1e-6,
-                   norm_weight=None, stream=None):
+def backward_local(q, k, v, g, dout, prefix, workspace, y=None, dg=None, dnorm_weight=None, dstate_end=None,
+                   block_size: int = 256, phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE,
+                   eps: float = 1e-6, norm_weight=None, stream=None):
     """Backward steps 1-2 on this rank's chunk: dy (and dg, this chunk's terms of dw) from dout
     through the output transform of the chunk's raw output y (given, or recomputed from
-    `prefix`), then G = sum over the chunk of phi(q_t) dy_t^T (the chunk-state kernel with q
-    as the keys and dy as the values).  Returns (dy [1, T, H*D], G fp32 [H, D, D])."""
+    `prefix`), then this rank's contribution to the earlier ranks' end-of-chunk gradients:
+    G = dstate_end + sum over the chunk of phi(q_t) dy_t^T (the chunk-state kernel with q as
+    the keys, dy as the values and dstate_end, the gradient of the state at the end of this
+    chunk from outside, as its initial state).  Returns (dy [1, T, H*D], G fp32 [H, D, D])."""
     _, T, H, D = q.shape
     if mode == la.LA_OUT_RAW:
         dy = dout
@@ -140,20 +142,21 @@ def backward_local(q, k, v, g, dout, prefix, workspace, y=None, dg=None, dnorm_w
                                                     mode=mode, eps=eps, norm_weight=norm_weight, workspace=workspace,
                                                     stream=stream)
     G = torch.empty((1, H, D, D), dtype=torch.float32, device=q.device)
-    la.lightning_attn_chunk_state(q, dy.view(1, T, H, D), G, phi=phi, workspace=workspace, stream=stream)
+    la.lightning_attn_chunk_state(q, dy.view(1, T, H, D), G, None if dstate_end is None else dstate_end.view(1, H, D, D),
+                                  phi=phi, workspace=workspace, stream=stream)
     return dy, G[0]
 
 
-def backward_finish(q, k, v, dy, dq, dk, dv, gathered, rank: int, prefix, workspace, dstate_out=None,
+def backward_finish(q, k, v, dy, dq, dk, dv, gathered, rank: int, prefix, workspace, dstate_end=None,
                     dstate_in=None, block_size: int = 256, phi: int = la.LA_PHI_SILU, stream=None):
-    """Backward steps 3-4: the gradient reaching the end of the chunk, dS_T + sum_{j > rank} of
-    the gathered G_j [world, H, D, D] (added from the last rank down), then the chunk's
+    """Backward steps 3-4: the gradient reaching the end of the chunk, dstate_end + sum_{j > rank}
+    of the gathered G_j [world, H, D, D] (added from the last rank down), then the chunk's
     backward in raw mode from dy with its initial state `prefix`."""
     _, T, H, D = q.shape
     world = gathered.shape[0]
     later_first = torch.flip(gathered, dims=[0]).contiguous()   # rank world-1 first
     ds_end = torch.empty((H, D, D), dtype=torch.float32, device=q.device)
-    la.lightning_attn_state_prefix(later_first, world - 1 - rank, ds_end, state0=dstate_out, stream=stream)
+    la.lightning_attn_state_prefix(later_first, world - 1 - rank, ds_end, state0=dstate_end, stream=stream)
     st = lambda x: None if x is None else x.view(1, H, D, D)
     la.lightning_attn_backward(q, k, v, None, dy, dq, dk, dv, state_in=st(prefix), dstate_in=st(dstate_in),
                                block_size=block_size, phi=phi, mode=la.LA_OUT_RAW, workspace=workspace,
@@ -161,29 +164,29 @@ def backward_finish(q, k, v, dy, dq, dk, dv, gathered, rank: int, prefix, worksp
 
 
 def backward_sequence_parallel(q, k, v, g, dout, dq, dk, dv, rank: int, prefix, all_gather=nccl_all_gather,
-                               dstate_out=None, y=None, dg=None, dnorm_weight=None, dstate_in=None,
+                               dstate_end=None, y=None, dg=None, dnorm_weight=None, dstate_in=None,
                                block_size: int = 256, phi: int = la.LA_PHI_SILU, mode: int = la.LA_OUT_RMSNORM_GATE,
                                eps: float = 1e-6, norm_weight=None, workspace=None, stream=None):
     """This rank's part of the backward of prefill_sequence_parallel.
 
-    The gradient reaching the end of chunk r is the sequence's final-state gradient dS_T
-    plus, for every later chunk j, G_j = sum over its tokens of phi(q_t) dy_t^T (the part of
-    chunk j's initial-state gradient that its own tokens give), so after one all-gather of
-    the G_j every rank runs its chunk's backward on its own (backward_local, the all-gather,
-    backward_finish).
+    With X_j the gradient that reaches the state at the end of chunk j from outside (on the
+    last rank the gradient of the sequence's final state; elsewhere zero unless the caller
+    used that state) and G_j = sum over chunk j of phi(q_t) dy_t^T (the part of chunk j's
+    initial-state gradient that its own tokens give), the gradient reaching the end of
+    chunk r is X_r + sum_{j > r} (G_j + X_j): after one all-gather of the G_j + X_j every rank
+    runs its chunk's backward on its own (backward_local, the all-gather, backward_finish).
     q, k, v, dq, dk, dv [1, T, H, D]; g, dout, dg [1, T, H*D]; prefix (the state the chunk
-    started from, as prefill_sequence_parallel returns it), dstate_out, dstate_in fp32
-    [H, D, D] (dstate_out: the same tensor on every rank, None for zero; rank 0's dstate_in
-    is the gradient of the sequence's initial state); y: the chunk's raw output if kept;
-    dnorm_weight fp32 [H*D] receives this chunk's part of the norm weight's gradient (sum it
-    over the ranks)."""
+    started from, as prefill_sequence_parallel returns it), dstate_end (X_r, None for zero),
+    dstate_in fp32 [H, D, D] (rank 0's dstate_in is the gradient of the sequence's initial
+    state); y: the chunk's raw output if kept; dnorm_weight fp32 [H*D] receives this chunk's
+    part of the norm weight's gradient (sum it over the ranks)."""
     _, T, H, D = q.shape
     if workspace is None:
         workspace = backward_workspace_for(T, H, D, block_size, mode, q.device, la._dtype(q))
-    dy, G = backward_local(q, k, v, g, dout, prefix, workspace, y, dg, dnorm_weight, block_size, phi, mode, eps,
-                           norm_weight, stream)
+    dy, G = backward_local(q, k, v, g, dout, prefix, workspace, y, dg, dnorm_weight, dstate_end, block_size, phi,
+                           mode, eps, norm_weight, stream)
     gathered = all_gather(G)
-    backward_finish(q, k, v, dy, dq, dk, dv, gathered, rank, prefix, workspace, dstate_out, dstate_in, block_size,
+    backward_finish(q, k, v, dy, dq, dk, dv, gathered, rank, prefix, workspace, dstate_end, dstate_in, block_size,
                     phi, stream)
 
 

@@ -71,6 +71,17 @@ class _OracleBackend:
         if state_out is not None:
             state_out.copy_(torch.from_numpy(st))
 
+    def lightning_attn_output_transform(self, y, g, out, mode=2, eps=1e-6, norm_weight=None, stream=None):
+        import torch
+        self._bind("lightning_attn_output_transform", y, g, out, mode=mode, eps=eps, norm_weight=norm_weight,
+                   stream=stream)
+        H, D = y.shape[-2], y.shape[-1]
+        n = y.numel() // (H * D)
+        o = self.oracle.transform(y.detach().numpy().reshape(n, H, D), mode, eps=eps,
+                                  norm_weight=None if norm_weight is None else norm_weight.numpy(),
+                                  g=None if g is None else g.detach().numpy().reshape(n, H * D))
+        out.copy_(torch.from_numpy(o).view(out.shape))
+
     def lightning_attn_output_transform_backward(self, y, g, dout, dy, dg=None, dnorm_weight=None, mode=2, eps=1e-6,
                                                  norm_weight=None, workspace=None, stream=None):
         import torch
@@ -298,7 +309,8 @@ def test_varlen_slice_plans_partition_the_batch():
 
 
 # The backward over three ranks (a one-token chunk in the middle), with a final-state
-# gradient, an initial state, a trained norm weight and the gate.
+# gradient, a gradient on the state at the end of the middle chunk too, an initial state, a
+# trained norm weight and the gate.
 BW_CHUNKS = [40, 1, 55]
 
 
@@ -319,6 +331,7 @@ def _backward_main(rank, world, port, out_dir):
         dout = synth.normal(1531, 11, (Tt, H * D), 1.0, "f32")
         s0 = synth.normal(1531, 9, (H, D, D), 0.1, "f32")
         dsT = synth.normal(1531, 10, (H, D, D), 0.1, "f32")
+        dsM = synth.normal(1531, 14, (H, D, D), 0.1, "f32")
         w = (1.0 + 0.2 * synth.normal(1531, 13, (H * D,), 1.0, "f32")).astype(np.float32)
         a = sum(BW_CHUNKS[:rank])
         b = a + BW_CHUNKS[rank]
@@ -332,8 +345,10 @@ def _backward_main(rank, world, port, out_dir):
         dg = torch.zeros((1, b - a, H * D), dtype=torch.float32)
         dw = torch.zeros((H * D,), dtype=torch.float32)
         ds0 = torch.zeros((H, D, D), dtype=torch.float32)
-        sp.backward_sequence_parallel(cq, ck, cv, cg, cd, dq, dk, dv, rank, prefix, dstate_out=t(dsT), dg=dg,
-                                      dnorm_weight=dw, dstate_in=ds0, mode=2, norm_weight=t(w), workspace=object())
+        end = {world - 1: dsT, 1: dsM}.get(rank)
+        sp.backward_sequence_parallel(cq, ck, cv, cg, cd, dq, dk, dv, rank, prefix,
+                                      dstate_end=None if end is None else t(end), dg=dg, dnorm_weight=dw,
+                                      dstate_in=ds0, mode=2, norm_weight=t(w), workspace=object())
         np.savez(os.path.join(out_dir, f"bw{rank}.npz"), dq=dq.numpy()[0], dk=dk.numpy()[0], dv=dv.numpy()[0],
                  dg=dg.numpy()[0], dw=dw.numpy(), ds0=ds0.numpy())
     finally:
@@ -342,7 +357,9 @@ def _backward_main(rank, world, port, out_dir):
 
 def test_backward_over_three_gloo_ranks_matches_one_backward(tmp_path):
     """Each rank's dq, dk, dv, dg, the ranks' dw summed and rank 0's initial-state gradient
-    against one oracle backward of the whole sequence (with S0, dS_T and a norm weight)."""
+    against the oracle: one backward of the whole sequence (with S0, dS_T and a norm weight)
+    plus, the backward being linear in its output gradients, one of the tokens up to the
+    middle chunk's end with no output gradient and that state's gradient as the final one."""
     sys.path.insert(0, ROOT)
     import oracle
     import synth
@@ -354,9 +371,16 @@ def test_backward_over_three_gloo_ranks_matches_one_backward(tmp_path):
     dout = synth.normal(1531, 11, (Tt, H * D), 1.0, "f32")
     s0 = synth.normal(1531, 9, (H, D, D), 0.1, "f32")
     dsT = synth.normal(1531, 10, (H, D, D), 0.1, "f32")
+    dsM = synth.normal(1531, 14, (H, D, D), 0.1, "f32")
     w = (1.0 + 0.2 * synth.normal(1531, 13, (H * D,), 1.0, "f32")).astype(np.float32)
-    ref = oracle.backward(q[None], k[None], v[None], g[None], dout[None], state_in=s0[None], norm_weight=w,
-                          dstate_out=dsT[None])
+    ref = list(oracle.backward(q[None], k[None], v[None], g[None], dout[None], state_in=s0[None], norm_weight=w,
+                               dstate_out=dsT[None]))
+    m = BW_CHUNKS[0] + BW_CHUNKS[1]
+    mid = oracle.backward(q[None, :m], k[None, :m], v[None, :m], g[None, :m], np.zeros_like(dout[None, :m]),
+                          state_in=s0[None], norm_weight=w, dstate_out=dsM[None])
+    for i in range(3):
+        ref[i][:, :m] += mid[i]
+    ref[4] = ref[4] + mid[4]   # dg and dw get nothing from a state gradient
     parts = [np.load(tmp_path / f"bw{r}.npz") for r in range(world)]
     # states, dy and the partial sums pass through fp32 between the steps: 1e-5 of the largest
     # value covers that, while a missing or misplaced later-chunk sum is O(1)
@@ -444,3 +468,82 @@ def test_varlen_backward_over_five_gloo_ranks_matches_one_packed_backward(tmp_pa
     assert sorted(starts) == list(range(n))
     for s, ds in starts.items():
         np.testing.assert_allclose(ds, ref[4][s], rtol=0, atol=1e-5 * np.abs(ref[4]).max(), err_msg=f"dS0 {s}")
+
+
+
+def _autograd_main(rank, world, port, out_dir):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import synth
+    from long_context_attn_b200 import autograd as ag
+    from long_context_attn_b200 import sequence_parallel as sp
+    fake = _OracleBackend()
+    fake.lightning_attn_workspace_size = lambda *a: 256
+    fake.new_workspace = lambda n, device=None: torch.zeros(n, dtype=torch.uint8)
+    for name in ("LA_OP_CHUNK_STATE", "LA_OP_BACKWARD", "LA_OP_OUTPUT_TRANSFORM_BACKWARD"):
+        setattr(fake, name, 0)
+    sp.la = ag.la = fake
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        Tt = sum(BW_CHUNKS)
+        q, k, v, g = synth.prefill_inputs(1531, Tt, H, D, "f32", 0.5, True)
+        dout = synth.normal(1531, 11, (Tt, H * D), 1.0, "f32")
+        s0 = synth.normal(1531, 9, (H, D, D), 0.1, "f32")
+        dsT = synth.normal(1531, 10, (H, D, D), 0.1, "f32")
+        dsM = synth.normal(1531, 14, (H, D, D), 0.1, "f32")
+        w = (1.0 + 0.2 * synth.normal(1531, 13, (H * D,), 1.0, "f32")).astype(np.float32)
+        a = sum(BW_CHUNKS[:rank])
+        b = a + BW_CHUNKS[rank]
+        leaf = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).requires_grad_(True)
+        cq, ck, cv = (leaf(x[a:b][None]) for x in (q, k, v))
+        cg, ts0, tw = leaf(g[a:b][None]), leaf(s0), leaf(w)
+        out, st_end = ag.lightning_attention_sequence_parallel(cq, ck, cv, cg, state0=ts0, norm_weight=tw, rank=rank)
+        loss = (out * torch.from_numpy(dout[a:b][None])).sum()
+        end = {world - 1: dsT, 1: dsM}.get(rank)
+        if end is not None:
+            loss = loss + (st_end * torch.from_numpy(end)).sum()
+        loss.backward()
+        np.savez(os.path.join(out_dir, f"ag{rank}.npz"), dq=cq.grad.numpy()[0], dk=ck.grad.numpy()[0],
+                 dv=cv.grad.numpy()[0], dg=cg.grad.numpy()[0], dw=tw.grad.numpy(), ds0=ts0.grad.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_autograd_over_three_gloo_ranks_matches_one_backward(tmp_path):
+    """lightning_attention_sequence_parallel under loss.backward() on three gloo ranks (the
+    middle chunk's end state and the last one's in the loss too): the chunks' input gradients
+    and the ranks' state0 and norm-weight gradients added up, against the oracle as in the
+    test above."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    import synth
+    world = len(BW_CHUNKS)
+    mp.start_processes(_autograd_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    Tt = sum(BW_CHUNKS)
+    q, k, v, g = synth.prefill_inputs(1531, Tt, H, D, "f32", 0.5, True)
+    dout = synth.normal(1531, 11, (Tt, H * D), 1.0, "f32")
+    s0 = synth.normal(1531, 9, (H, D, D), 0.1, "f32")
+    dsT = synth.normal(1531, 10, (H, D, D), 0.1, "f32")
+    dsM = synth.normal(1531, 14, (H, D, D), 0.1, "f32")
+    w = (1.0 + 0.2 * synth.normal(1531, 13, (H * D,), 1.0, "f32")).astype(np.float32)
+    ref = list(oracle.backward(q[None], k[None], v[None], g[None], dout[None], state_in=s0[None], norm_weight=w,
+                               dstate_out=dsT[None]))
+    m = BW_CHUNKS[0] + BW_CHUNKS[1]
+    mid = oracle.backward(q[None, :m], k[None, :m], v[None, :m], g[None, :m], np.zeros_like(dout[None, :m]),
+                          state_in=s0[None], norm_weight=w, dstate_out=dsM[None])
+    for i in range(3):
+        ref[i][:, :m] += mid[i]
+    ref[4] = ref[4] + mid[4]
+    parts = [np.load(tmp_path / f"ag{r}.npz") for r in range(world)]
+    for i, name in enumerate(("dq", "dk", "dv", "dg")):
+        got = np.concatenate([p[name] for p in parts])
+        np.testing.assert_allclose(got, ref[i][0], rtol=0, atol=1e-5 * np.abs(ref[i]).max(), err_msg=name)
+    np.testing.assert_allclose(sum(p["dw"].astype(np.float64) for p in parts), ref[5], rtol=0,
+                               atol=1e-5 * np.abs(ref[5]).max(), err_msg="dw")
+    np.testing.assert_allclose(sum(p["ds0"].astype(np.float64) for p in parts), ref[4][0], rtol=0,
+                               atol=1e-5 * np.abs(ref[4]).max(), err_msg="dS0")

@@ -167,16 +167,16 @@ def test_emulated_ranks_backward_match_one_backward(cuda_device):
         gg = torch.full_like(dg, float("nan"))
         gw = torch.full((H * D,), float("nan"), dtype=torch.float32, device="cuda")
         gs = torch.full((H, D, D), float("nan"), dtype=torch.float32, device="cuda")
-        dy, G = sp.backward_local(dq, dk, dv, dg, dd, prefixes[r], ws, dg=gg, dnorm_weight=gw, block_size=C,
-                                  norm_weight=dw_)
+        dy, G = sp.backward_local(dq, dk, dv, dg, dd, prefixes[r], ws, dg=gg, dnorm_weight=gw,
+                                  dstate_end=dsT_ if r == len(chunks) - 1 else None, block_size=C, norm_weight=dw_)
         grads.append((gq, gk, gv, gg, gw, gs))
         dys.append(dy)
         Gs.append(G)
     gathered = torch.stack(Gs)
     for r, (dq, dk, dv, dg, dd, ws) in enumerate(ranks):
         gq, gk, gv, gg, gw, gs = grads[r]
-        sp.backward_finish(dq, dk, dv, dys[r], gq, gk, gv, gathered, r, prefixes[r], ws, dstate_out=dsT_,
-                           dstate_in=gs, block_size=C)
+        sp.backward_finish(dq, dk, dv, dys[r], gq, gk, gv, gathered, r, prefixes[r], ws,
+                           dstate_end=dsT_ if r == len(chunks) - 1 else None, dstate_in=gs, block_size=C)
     torch.cuda.synchronize()
     ref = oracle.backward(q[None], k[None], v[None], g[None], dout[None], state_in=s0[None], norm_weight=w,
                           dstate_out=dsT[None])
@@ -275,3 +275,32 @@ def test_host_prefill_pipeline_matches_one_prefill(chunk, cuda_device):
     ref, ref_st, _ = oracle.prefill(q[None], k[None], v[None], g[None], state_in=s0[None])
     assert_close(hout.float().numpy()[None], ref, "bf16")
     assert_close(to_host(st)[None], ref_st, "bf16", "final state")
+
+
+def test_sequence_parallel_autograd_single_rank(cuda_device):
+    """lightning_attention_sequence_parallel with a group of one (the all-gather a stack of one):
+    out, the end state and, under loss.backward(), every input's gradient against the oracle."""
+    import torch
+    from long_context_attn_b200.autograd import lightning_attention_sequence_parallel
+    H, D, T = 8, 128, 700
+    q, k, v, g = synth.prefill_inputs(1451, T, H, D, "bf16", 0.5, True)
+    dout = synth.f32_to_bf16(synth.normal(1451, 11, (T, H * D), 1.0, "f32"))
+    s0 = synth.normal(1451, 9, (H, D, D), 0.05, "f32")
+    dsT = synth.normal(1451, 10, (H, D, D), 0.05, "f32")
+    w = (1.0 + 0.2 * synth.normal(1451, 13, (H * D,), 1.0, "f32")).astype(np.float32)
+    leaf = lambda a, shape: to_dev(a).reshape(shape).clone().requires_grad_(True)
+    tq, tk, tv = (leaf(a, (1, T, H, D)) for a in (q, k, v))
+    tg, ts0, tw = leaf(g, (1, T, H * D)), leaf(s0, (H, D, D)), leaf(w, (H * D,))
+    out, st = lightning_attention_sequence_parallel(tq, tk, tv, tg, state0=ts0, norm_weight=tw, rank=0,
+                                                    all_gather=lambda x: x[None])
+    loss = (out.float() * to_dev(dout).reshape(1, T, H * D).float()).sum() + (st * to_dev(dsT)).sum()
+    loss.backward()
+    ref_o, ref_s, _ = oracle.prefill(q[None], k[None], v[None], g[None], state_in=s0[None], norm_weight=w)
+    assert_close(to_host(out.detach()), ref_o, "bf16")
+    assert_close(to_host(st.detach())[None], ref_s, "bf16", "end state")
+    ref = oracle.backward(q[None], k[None], v[None], g[None], dout[None], state_in=s0[None], norm_weight=w,
+                          dstate_out=dsT[None])
+    for t, want, name in zip((tq, tk, tv, tg), ref[:4], ("dq", "dk", "dv", "dg")):
+        assert_close(to_host(t.grad), want, "bf16", name)
+    assert_close(to_host(ts0.grad)[None], ref[4], "bf16", "dS0")
+    assert_close(to_host(tw.grad), ref[5], "bf16", "dw")
