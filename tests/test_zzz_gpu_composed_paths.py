@@ -304,3 +304,29 @@ def test_sequence_parallel_autograd_single_rank(cuda_device):
         assert_close(to_host(t.grad), want, "bf16", name)
     assert_close(to_host(ts0.grad)[None], ref[4], "bf16", "dS0")
     assert_close(to_host(tw.grad), ref[5], "bf16", "dw")
+
+
+def test_varlen_autograd_matches_oracle(cuda_device):
+    """lightning_attention_varlen under loss.backward(): packed sequences (an empty and a
+    one-token one among them) with initial states, final-state gradients, a trained norm
+    weight and the gate, against the oracle's packed backward."""
+    import torch
+    from long_context_attn_b200.autograd import lightning_attention_varlen
+    H, D = 8, 128
+    lens = [300, 0, 257, 1, 129]
+    cu = synth.cu_seqlens_of(lens)
+    tot, n = int(cu[-1]), len(lens)
+    q, k, v, g = synth.prefill_inputs(1461, tot, H, D, "bf16", 0.5, True)
+    dout = synth.f32_to_bf16(synth.normal(1461, 11, (tot, H * D), 1.0, "f32"))
+    s0 = synth.normal(1461, 9, (n, H, D, D), 0.05, "f32")
+    dsT = synth.normal(1461, 10, (n, H, D, D), 0.05, "f32")
+    w = (1.0 + 0.2 * synth.normal(1461, 13, (H * D,), 1.0, "f32")).astype(np.float32)
+    leaf = lambda a: to_dev(a).clone().requires_grad_(True)
+    tq, tk, tv, tg, ts0, tw = (leaf(a) for a in (q, k, v, g, s0, w))
+    out, st = lightning_attention_varlen(tq, tk, tv, torch.from_numpy(cu).cuda(), max(lens), g=tg, state_in=ts0,
+                                         norm_weight=tw)
+    loss = (out.float() * to_dev(dout).float()).sum() + (st * to_dev(dsT)).sum()
+    loss.backward()
+    ref = oracle.backward_packed(q, k, v, g, dout, cu, H, D, state_in=s0, norm_weight=w, dstate_out=dsT)
+    for t, want, name in zip((tq, tk, tv, tg, ts0, tw), ref, ("dq", "dk", "dv", "dg", "dS0", "dw")):
+        assert_close(to_host(t.grad), want, "bf16", name)
