@@ -72,11 +72,13 @@ def _get():
         lib.oracle_backward_packed.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, vp, i32, i32, dbl,
                                                vp, vp, vp, vp, vp, vp, vp]
         lib.oracle_transform_backward.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, dbl, vp, vp, vp, vp]
+        lib.oracle_backward_znorm_packed.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, vp, vp, vp, i32,
+                                                     i32, dbl, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         for f in (lib.oracle_forward_packed, lib.oracle_prefill, lib.oracle_decode,
                   lib.oracle_quadratic, lib.oracle_chunked, lib.oracle_transform, lib.oracle_backward_packed,
-                  lib.oracle_forward_znorm_packed, lib.oracle_transform_backward):
+                  lib.oracle_forward_znorm_packed, lib.oracle_transform_backward, lib.oracle_backward_znorm_packed):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -280,6 +282,32 @@ def forward_znorm_packed(q, k, v, g, cu_seqlens, H, D, state_in=None, z_in=None,
     if rc != 0:
         raise ValueError("oracle_forward_znorm_packed rejected its arguments")
     return out, st, z
+
+
+def backward_znorm_packed(q, k, v, g, dout, cu_seqlens, H, D, state_in=None, z_in=None, phi=PHI_SILU,
+                          mode=MODE_RMSNORM_GATE, eps=1e-6, norm_weight=None, dstate_out=None, dz_out=None):
+    """Gradients of forward_znorm_packed for the loss with output gradient dout [tokens, H*D]
+    and final-state gradients dstate_out [N, H, D, D], dz_out [N, H, D] (fp32 or None).
+    Returns fp64 (dq, dk, dv [tokens, H, D], dg [tokens, H*D] or None, dstate [N, H, D, D],
+    dz [N, H, D], dw [H*D])."""
+    q, k, v, g, dout = _c(q), _c(k), _c(v), _c(g), _c(dout)
+    dt = _dtype_code(q)
+    cu = _c(cu_seqlens, np.int32)
+    N = cu.size - 1
+    tokens = int(cu[-1]) if N > 0 else 0
+    dq, dk, dv = (np.zeros((tokens, H, D), dtype=np.float64) for _ in range(3))
+    dg = np.zeros((tokens, H * D), dtype=np.float64) if mode == MODE_RMSNORM_GATE else None
+    dst = np.zeros((N, H, D, D), dtype=np.float64)
+    dz = np.zeros((N, H, D), dtype=np.float64)
+    dw = np.zeros(H * D, dtype=np.float64)
+    s_in, z0, w = _c(state_in, np.float32), _c(z_in, np.float32), _c(norm_weight, np.float32)
+    ds_out, dz_o = _c(dstate_out, np.float32), _c(dz_out, np.float32)
+    rc = _get().oracle_backward_znorm_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout), dt, _ptr(cu), N, H, D,
+                                             _ptr(s_in), _ptr(z0), _ptr(ds_out), _ptr(dz_o), phi, mode, eps, _ptr(w),
+                                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dst), _ptr(dz), _ptr(dw))
+    if rc != 0:
+        raise ValueError("oracle_backward_znorm_packed rejected its arguments")
+    return dq, dk, dv, dg, dst, dz, dw
 
 
 def prefill_znorm(q, k, v, g=None, state_in=None, z_in=None, phi=PHI_SILU, mode=MODE_RMSNORM_GATE, eps=1e-6,

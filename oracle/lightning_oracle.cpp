@@ -291,7 +291,7 @@ void recur_head_backward(const void* q, const void* k, const void* v, int dtype,
 // transform is then applied to y as in the plain form.  One head over rows [row0, row0+n);
 // S (D x D) and z (D) enter as the initial state and leave as the final one.
 void recur_head_znorm(const void* q, const void* k, const void* v, int dtype, int64_t row0, int64_t n, int H,
-                      int D, int h, int phi, double* S, double* z, double* y) {
+                      int D, int h, int phi, double* S, double* z, double* y, double* dens = nullptr) {
   std::vector<double> fq(D), fk(D), vv(D), acc(D);
   for (int64_t t = 0; t < n; ++t) {
     const int64_t base = ((row0 + t) * H + h) * static_cast<int64_t>(D);
@@ -313,7 +313,39 @@ void recur_head_znorm(const void* q, const void* k, const void* v, int dtype, in
     }
     double* yt = y + (t * H + h) * static_cast<int64_t>(D);
     for (int j = 0; j < D; ++j) yt[j] = acc[j] / den;
+    if (dens) dens[t * H + h] = den;
   }
+}
+
+// Backward of the normalised variant's denominator for one head, after the numerator's
+// part has gone through recur_head_backward (which assigned dq, dk).  With d_t = phi(q_t) . z_t
+// and dd_t the gradient reaching d_t (for y_t = n_t / d_t: dd_t = -(dy_t . y_t) / d_t):
+//   dphi(q_t) += dd_t z_t           (z_t including token t)
+//   dphi(k_i) += dz_T + sum_{t >= i} dd_t phi(q_t),    dz0 = dz_T + sum_t dd_t phi(q_t)
+// through phi' as in the plain backward.  dd is indexed [t * H + h] from the sequence's
+// first row; z0 and dzT (nullable) are this head's D-vectors; dz0 receives D values.
+void znorm_head_backward_den(const void* q, const void* k, int dtype, int64_t row0, int64_t n, int H, int D, int h,
+                             int phi, const double* z0, const double* dzT, const double* dd, double* dq, double* dk,
+                             double* dz0) {
+  std::vector<double> z(z0, z0 + D);
+  for (int64_t t = 0; t < n; ++t) {
+    const int64_t base = ((row0 + t) * H + h) * static_cast<int64_t>(D);
+    for (int i = 0; i < D; ++i) {
+      z[i] += feature(widen(k, dtype, base + i), phi);
+      dq[base + i] += dd[t * H + h] * z[i] * dfeature(widen(q, dtype, base + i), phi);
+    }
+  }
+  std::vector<double> acc(D, 0.0);
+  if (dzT)
+    for (int i = 0; i < D; ++i) acc[i] = dzT[i];
+  for (int64_t t = n - 1; t >= 0; --t) {
+    const int64_t base = ((row0 + t) * H + h) * static_cast<int64_t>(D);
+    for (int i = 0; i < D; ++i) {
+      acc[i] += dd[t * H + h] * feature(widen(q, dtype, base + i), phi);
+      dk[base + i] += acc[i] * dfeature(widen(k, dtype, base + i), phi);
+    }
+  }
+  for (int i = 0; i < D; ++i) dz0[i] = acc[i];
 }
 
 }  // namespace
@@ -573,6 +605,88 @@ int oracle_forward_znorm_packed(const void* q, const void* k, const void* v, con
       for (int64_t i = 0; i < nst; ++i) state_out[s * nst + i] = S[i];
     if (z_out)
       for (int64_t i = 0; i < nz; ++i) z_out[s * nz + i] = z[i];
+  }
+  return 0;
+}
+
+// Backward of oracle_forward_znorm_packed for the loss with output gradient dout [tokens, H*D]
+// (dtype of q) and final-state gradients dstate_out [N, H, D, D], dz_out [N, H, D] (fp32, null
+// for zero).  Recomputes the forward (y and each token's denominators), applies the transform
+// backward per token, splits each head's raw-output gradient into the numerator's
+// dn_t = dy_t / d_t and the denominator's dd_t = -(dy_t . y_t) / d_t, runs the plain recurrence
+// backward on dn and adds the denominator's terms.  Outputs fp64: dq, dk, dv [tokens, H, D],
+// dg [tokens, H*D] (gate mode), dstate [N, H, D, D], dz [N, H, D], dw [H*D] (may be null
+// but dq, dk, dv).
+int oracle_backward_znorm_packed(const void* q, const void* k, const void* v, const void* g, const void* dout,
+                                 int dtype, const int32_t* cu, int N, int H, int D, const float* state_in,
+                                 const float* z_in, const float* dstate_out, const float* dz_out, int phi, int mode,
+                                 double eps, const float* w, double* dq, double* dk, double* dv, double* dg,
+                                 double* dstate, double* dz, double* dw) {
+  if (N < 0 || H <= 0 || D <= 0 || !dout || !dq || !dk || !dv) return 1;
+  if (mode == MODE_RMSNORM_GATE && (!g || !dg)) return 1;
+  const int HD = H * D;
+  if (dw)
+    for (int c = 0; c < HD; ++c) dw[c] = 0.0;
+  const int64_t nst = static_cast<int64_t>(H) * D * D, nz = static_cast<int64_t>(H) * D;
+  for (int s = 0; s < N; ++s) {
+    const int64_t row0 = cu[s], L = static_cast<int64_t>(cu[s + 1]) - cu[s];
+    if (L < 0) return 1;
+    std::vector<double> S0(nst, 0.0), z0(nz, 0.0), dST, dzT;
+    if (state_in)
+      for (int64_t i = 0; i < nst; ++i) S0[i] = static_cast<double>(state_in[s * nst + i]);
+    if (z_in)
+      for (int64_t i = 0; i < nz; ++i) z0[i] = static_cast<double>(z_in[s * nz + i]);
+    if (dstate_out) {
+      dST.resize(nst);
+      for (int64_t i = 0; i < nst; ++i) dST[i] = static_cast<double>(dstate_out[s * nst + i]);
+    }
+    if (dz_out) {
+      dzT.resize(nz);
+      for (int64_t i = 0; i < nz; ++i) dzT[i] = static_cast<double>(dz_out[s * nz + i]);
+    }
+    // forward recompute: y and the denominators
+    std::vector<double> S(S0), z(z0), y(static_cast<size_t>(L) * HD), den(static_cast<size_t>(L) * H);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h)
+      recur_head_znorm(q, k, v, dtype, row0, L, H, D, h, phi, S.data() + static_cast<size_t>(h) * D * D,
+                       z.data() + static_cast<size_t>(h) * D, y.data(), den.data());
+    // transform backward per token (dw terms kept per token, added in token order)
+    const bool want_dw = dw && mode != MODE_RAW;
+    std::vector<double> dy(static_cast<size_t>(L) * HD), dwt(want_dw ? static_cast<size_t>(L) * HD : 0);
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < L; ++t)
+      transform_token_backward(y.data() + t * HD, dout, g, dtype, row0 + t, HD, mode, eps, w, dy.data() + t * HD,
+                               dg ? dg + (row0 + t) * HD : nullptr, want_dw ? dwt.data() + t * HD : nullptr);
+    if (want_dw)
+      for (int64_t t = 0; t < L; ++t)
+        for (int c = 0; c < HD; ++c) dw[c] += dwt[static_cast<size_t>(t) * HD + c];
+    // numerator and denominator parts of each head's raw-output gradient
+    std::vector<double> dn(static_cast<size_t>(L) * HD), dd(static_cast<size_t>(L) * H);
+    for (int64_t t = 0; t < L; ++t)
+      for (int h = 0; h < H; ++h) {
+        const double d = den[t * H + h];
+        double dot = 0.0;
+        for (int j = 0; j < D; ++j) {
+          const int64_t at = (t * H + h) * static_cast<int64_t>(D) + j;
+          dot += dy[at] * y[at];
+          dn[at] = dy[at] / d;
+        }
+        dd[t * H + h] = -dot / d;
+      }
+    std::vector<double> dS0(nst), dz0(nz);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+      recur_head_backward(q, k, v, dtype, row0, L, H, D, h, phi, S0.data() + static_cast<size_t>(h) * D * D,
+                          dstate_out ? dST.data() + static_cast<size_t>(h) * D * D : nullptr, dn.data(), dq, dk, dv,
+                          dS0.data() + static_cast<size_t>(h) * D * D);
+      znorm_head_backward_den(q, k, dtype, row0, L, H, D, h, phi, z0.data() + static_cast<size_t>(h) * D,
+                              dz_out ? dzT.data() + static_cast<size_t>(h) * D : nullptr, dd.data(), dq, dk,
+                              dz0.data() + static_cast<size_t>(h) * D);
+    }
+    if (dstate)
+      for (int64_t i = 0; i < nst; ++i) dstate[s * nst + i] = dS0[i];
+    if (dz)
+      for (int64_t i = 0; i < nz; ++i) dz[s * nz + i] = dz0[i];
   }
   return 0;
 }
