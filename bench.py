@@ -173,7 +173,21 @@ class PrefillCase:
         self.la.lightning_attn_prefill(self.q, self.k, self.v, self.g, self.out, None, self.state,
                                        block_size=self.C, workspace=self.ws)
 
+    def enable_host_pipeline(self, chunk_tokens):
+        """e2e through HostPrefill: the copies in and out overlapped over chunks of the sequence."""
+        from long_context_attn_b200.host_stream import HostPrefill
+        self.host = HostPrefill(self.H, self.D, chunk_tokens=chunk_tokens, block_size=self.C,
+                                device=self.q.device)
+        self.host_chunk = chunk_tokens
+
     def e2e_step(self):
+        host = getattr(self, "host", None)
+        if host is not None:
+            T, H, D = self.T, self.H, self.D
+            host(self.h_q.view(T, H, D), self.h_k.view(T, H, D), self.h_v.view(T, H, D), self.h_g.view(T, H * D),
+                 self.h_out.view(T, H * D), state_out=self.state.view(H, D, D))
+            self.h_state.copy_(self.state, non_blocking=True)
+            return
         self.q.view(-1).copy_(self.h_q.view(-1), non_blocking=True)
         self.k.view(-1).copy_(self.h_k.view(-1), non_blocking=True)
         self.v.view(-1).copy_(self.h_v.view(-1), non_blocking=True)
@@ -184,6 +198,8 @@ class PrefillCase:
 
     def check(self):
         self.la.lightning_attn_check(self.ws)
+        if getattr(self, "host", None) is not None:
+            self.host.check()
 
     def oracle_sample(self, tokens):
         """fp64 oracle on the first `tokens` rows of the same workload (all heads)."""
@@ -717,6 +733,10 @@ def run_gpu(args):
             dist.barrier()
 
     case = _make_case(args.workload, device, rank)
+    if args.e2e_chunk:
+        if not hasattr(case, "enable_host_pipeline"):
+            raise SystemExit(f"--e2e-chunk applies to the single-sequence prefill workloads, not {args.workload}")
+        case.enable_host_pipeline(args.e2e_chunk)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         case.step()
@@ -793,8 +813,9 @@ def run_gpu(args):
                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                        "frac_algorithmic": case.alg_flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
                        "frac_issued": case.issued_flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
-            "e2e": {"value": _job_value(case.tokens, args.steps, world, e2e_ms), "unit": "tokens/s",
-                    "h2d_bytes_per_step": case.h2d, "d2h_bytes_per_step": case.d2h},
+            "e2e": dict({"value": _job_value(case.tokens, args.steps, world, e2e_ms), "unit": "tokens/s",
+                         "h2d_bytes_per_step": case.h2d, "d2h_bytes_per_step": case.d2h},
+                        **({"pipeline": f"HostPrefill, chunks of {args.e2e_chunk} tokens"} if args.e2e_chunk else {})),
             "gpu_launches": args.steps * getattr(case, "launches_per_step", 1),
             "clocks": clk.summary(),
         }
@@ -972,6 +993,8 @@ def main():
                              "backward_128k", "train_128k", "znorm_128k", "chunk_state_128k", "prefill_128k_h8"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--e2e-chunk", type=int, default=0,
+                    help="e2e through HostPrefill with chunks of this many tokens (0: copy in, step, copy out)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         print("note: fewer than 3 warm-up steps; this run is not a valid bench line", file=sys.stderr)
