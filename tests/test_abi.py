@@ -223,3 +223,25 @@ def test_output_transform_backward_host_checks(lib):
     assert call(dw=vp(0x2000), ws=vp(0x100010), nbytes=1 << 30) == 1   # misaligned workspace
     assert call(dw=vp(0x2000), ws=ws, nbytes=256) == 1                 # workspace too small
     assert call(dw=vp(0x2004), ws=ws, nbytes=1 << 30) == 1             # misaligned dw
+
+
+def test_binding_constants_match_header_enums(lib):
+    """Every LA_* enumerator the header defines has the same value in the Python binding, and
+    the binding defines no LA_* status, dtype, mode, feature-map or op constant the header
+    lacks."""
+    from long_context_attn_b200 import lightning_attn as la
+    src = open(os.path.join(HEADER_DIR, "lightning_attn.h")).read()
+    enums = {}
+    for body in re.findall(r"typedef\s+enum\s*\{(.*?)\}", src, flags=re.S):
+        body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+        for name, value in re.findall(r"\b(LA_\w+)\s*=\s*(\d+)", body):
+            enums[name] = int(value)
+    assert {"LA_OK", "LA_BF16", "LA_OUT_RMSNORM_GATE", "LA_PHI_SILU", "LA_OP_OUTPUT_TRANSFORM_BACKWARD"} <= set(enums)
+    for name, value in enums.items():
+        if hasattr(la, name):
+            assert getattr(la, name) == value, name
+    prefixes = ("LA_OK", "LA_ERR_", "LA_F32", "LA_BF16", "LA_OUT_", "LA_PHI_", "LA_OP_")
+    py = {n for n in dir(la) if n.startswith(prefixes)}
+    assert py <= set(enums), py - set(enums)
+    missing = {n for n in enums if n.startswith("LA_OP_")} - py
+    assert not missing, missing
