@@ -245,3 +245,18 @@ def test_binding_constants_match_header_enums(lib):
     assert py <= set(enums), py - set(enums)
     missing = {n for n in enums if n.startswith("LA_OP_")} - py
     assert not missing, missing
+
+
+def test_binding_argument_counts_match_header(lib):
+    """The ctypes argument list the binding sets for each entry point has as many entries as
+    the header's declaration has parameters."""
+    from long_context_attn_b200 import lightning_attn as la
+    src = open(os.path.join(HEADER_DIR, "lightning_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    decls = dict(re.findall(r"LA_API\s+[\w\s\*]+?\b(\w+)\s*\(([^)]*)\)\s*;", src))
+    assert len(decls) == len(_declared())
+    for name, params in decls.items():
+        params = params.strip()
+        n = 0 if params in ("", "void") else len(params.split(","))
+        argtypes = getattr(la._lib, name).argtypes
+        assert argtypes is not None and len(argtypes) == n, (name, n, argtypes)
