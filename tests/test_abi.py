@@ -260,3 +260,17 @@ def test_binding_argument_counts_match_header(lib):
         n = 0 if params in ("", "void") else len(params.split(","))
         argtypes = getattr(la._lib, name).argtypes
         assert argtypes is not None and len(argtypes) == n, (name, n, argtypes)
+
+
+def test_every_workspace_op_has_a_size(lib):
+    """lightning_attn_workspace_size answers every LA_OP_* with a positive size for valid
+    arguments and 0 for an invalid head size (host-only query)."""
+    from long_context_attn_b200 import lightning_attn as la
+    lib.lightning_attn_workspace_size.restype = ctypes.c_size_t
+    ops = sorted(getattr(la, n) for n in dir(la) if n.startswith("LA_OP_"))
+    assert ops == list(range(len(ops)))
+    for op in ops:
+        n = lib.lightning_attn_workspace_size(op, 2, 300, 600, 8, 128, 256, la.LA_BF16, la.LA_OUT_RMSNORM_GATE)
+        assert n >= 256, op
+        assert lib.lightning_attn_workspace_size(op, 2, 300, 600, 8, 100, 256, la.LA_BF16,
+                                                 la.LA_OUT_RMSNORM_GATE) == 0, op
