@@ -162,9 +162,10 @@ LA_API la_status lightning_attn_decode_step(const void* q, const void* k, const 
                                      la_stream_t stream);
 
 /* Size of the scratch array compiled into the library for
- * lightning_attn_decode_step_noalloc (8.25 MiB: enough for B*H*D up to 2^21, e.g. 256
- * sequences x 64 heads x 128). */
-#define LA_DECODE_NOALLOC_SCRATCH_BYTES 8650752u
+ * lightning_attn_decode_step_noalloc: 8.25 MiB + 256 bytes, which holds the decode scratch
+ * of every batch with B*H*D <= 2^21 (e.g. 256 sequences x 64 heads x 128, or 32768
+ * sequences x 1 head x 64): 256 + 4B + 4*B*H*D + 4*B*H bytes, each part rounded up to 256. */
+#define LA_DECODE_NOALLOC_SCRATCH_BYTES 8651008u
 
 /*
  * Decode step that allocates nothing and takes no workspace (the pages have no
@@ -185,6 +186,15 @@ LA_API la_status lightning_attn_decode_step(const void* q, const void* k, const 
  *   - Batches whose scratch would exceed the array (decode_workspace bytes > the size above)
  *     return LA_ERR_UNSUPPORTED with nothing enqueued.
  *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - The error record sits in the library's array, where lightning_attn_check cannot
+ *     reach it: device-side errors of this call are not reported to the caller (the decode
+ *     kernel has no bounded waits, so the only such errors would be the CUDA launch errors
+ *     that the return status already carries).
+ *   - The array's address is kept per device for the life of the process; after a
+ *     cudaDeviceReset (or any other teardown of the device's primary context) this entry
+ *     point must not be called again in that process.
+ *   - q, k, v, g, out, state and norm_weight must live on the current device.
+ * On success lightning_attn_last_path() returns "decode".
  */
 LA_API la_status lightning_attn_decode_step_noalloc(const void* q, const void* k, const void* v, const void* g,
                                                     void* out, float* state, int B, int H, int D, la_dtype dtype,

@@ -126,6 +126,24 @@ SplitPlan split_plan(int B, int T, int H, int D) {
   sp.S = (T + sp.Tc - 1) / sp.Tc;
   return sp;
 }
+// Forward time (pair kernel): 2G workers per head, each owning whole sequences.  With fewer
+// sequences than workers, each sequence is cut into S chunks (whole blocks of C rows) so
+// that every worker has one: chunk c starts from S0 plus the states of the chunks before it
+// (chunk-state kernel over all but the last chunk, then the ordered prefix), and the last
+// chunk's final state is the sequence's.
+SplitPlan forward_split_plan(int B, int T, int H, int D, int C) {
+  SplitPlan sp{1, T};
+  if (D != 128 || B < 1 || H < 1 || T < 2 * kSplitMinChunk) return sp;
+  const int workers = 2 * std::max(1, la::pair_max_active_clusters() / H);
+  if (B >= workers) return sp;
+  const int S = std::min((workers + B - 1) / B, T / kSplitMinChunk);
+  if (S < 2) return sp;
+  const int align = C > 128 ? C : 128;
+  sp.Tc = ((T + S - 1) / S + align - 1) / align * align;
+  sp.S = (T + sp.Tc - 1) / sp.Tc;
+  if (sp.S < 2) return SplitPlan{1, T};
+  return sp;
+}
 // Workspace of a split call after the error record: [tensor-core part for the B * S chunks]
 // [chunk cu_seqlens] [chunk states] [chunk initial states] [chunk-state split partials].
 struct SplitLayout {
@@ -150,6 +168,8 @@ size_t prefill_ws_bytes(Path p, int nseq, int max_len, int64_t tokens, int H, in
     size_t n = la::tc_workspace_bytes(nseq, max_len, tokens, H, D, C);
     const SplitPlan sp = split_plan(nseq, max_len, H, D);
     if (sp.S > 1) n = std::max(n, split_layout(sp, nseq, tokens, H, D, C).total);
+    const SplitPlan fp = forward_split_plan(nseq, max_len, H, D, C);
+    if (fp.S > 1) n = std::max(n, split_layout(fp, nseq, tokens, H, D, C).total);
     return kErrBytes + n;
   }
   size_t y = (mode == LA_OUT_RAW) ? 0 : up256(sizeof(float) * static_cast<size_t>(tokens) * H * D);
@@ -190,7 +210,9 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
     a.mode = static_cast<int>(split ? LA_OUT_RAW : mode);
     a.eps = eps; a.w = split ? nullptr : w; a.err = err; a.ws = ws;
     a.reverse = reverse ? 1 : 0;
-    const SplitPlan sp = (!cu && T_fixed > 0) ? split_plan(nseq, T_fixed, H, D) : SplitPlan{1, T_fixed};
+    const bool fixed = !cu && T_fixed > 0;
+    const SplitPlan sp = !fixed ? SplitPlan{1, T_fixed}
+                                : (reverse ? split_plan(nseq, T_fixed, H, D) : forward_split_plan(nseq, T_fixed, H, D, C));
     if (sp.S > 1) {
       const SplitLayout sl = split_layout(sp, nseq, tokens, H, D, C);
       char* x = ws + sl.tc;
@@ -200,18 +222,26 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
       float* cpart = reinterpret_cast<float*>(x + sl.cu + 2 * sl.st);
       const int n = nseq * sp.S;
       e = la::launch_chunk_cu(ccu, nseq, T_fixed, sp.Tc, sp.S, stream);
+      // Forward time with one sequence: the last chunk's state is never needed (the kernel
+      // ends that chunk with the sequence's final state), and the first S - 1 chunks are
+      // contiguous, so only they are summed.
+      const bool skip_last = !reverse && nseq == 1;
       if (e == cudaSuccess)
-        e = la::launch_chunk_state_tc(k, v, nullptr, cst, cpart, ccu, n, 0, sp.Tc, tokens, H, phi_id,
-                                      current_sm_count(), err, stream);
-      if (e == cudaSuccess)   // chunk initial states, and the sequences' final states
-        e = la::launch_chunk_prefix(cst, state_in, cin, state_out, nseq, sp.S, H, reverse ? 1 : 0,
-                                    current_sm_count(), stream);
+        e = la::launch_chunk_state_tc(k, v, nullptr, cst, cpart, ccu, skip_last ? n - 1 : n, 0, sp.Tc, tokens, H,
+                                      phi_id, current_sm_count(), err, stream);
+      if (e == cudaSuccess)   // chunk initial states (and, reverse time, the sequences' final states)
+        e = la::launch_chunk_prefix(cst, state_in, cin, reverse ? state_out : nullptr, nseq, sp.S, H,
+                                    reverse ? 1 : 0, current_sm_count(), stream);
       a.cu = ccu;
       a.nseq = n;
       a.T = 0;
       a.max_len = sp.Tc;
       a.state_in = cin;
-      a.state_out = nullptr;
+      if (reverse) {
+        a.state_out = nullptr;
+      } else {
+        a.chunk_div = sp.S;   // the kernel writes each sequence's final state from its last chunk
+      }
     }
     if (e == cudaSuccess) e = la::launch_tc_prefill(a, current_sm_count(), stream);
     if (e == cudaSuccess && split)   // the norm (and gate) per token, over the raw output in place
@@ -443,6 +473,11 @@ size_t output_transform_backward_ws_bytes(int64_t tokens, int HD) {
 }
 
 }  // namespace
+
+namespace la {
+// Lets entry points defined in other files record their path (the workspace-free decode).
+void set_last_path(const char* path) { g_last_path = path; }
+}  // namespace la
 
 extern "C" {
 

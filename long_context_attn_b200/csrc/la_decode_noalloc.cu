@@ -22,6 +22,11 @@
 //    or different host threads without ordering) race on the array.
 //  * Sizes whose scratch would not fit are rejected with LA_ERR_UNSUPPORTED before anything
 //    is enqueued.  Nothing here calls cudaMalloc, cudaFree or an allocating library routine.
+//  * The address is cached per device index for the life of the process: a device reset
+//    (cudaDeviceReset) unmaps the array and makes the cached address stale, so the entry
+//    point must not be called again after one.
+//  * The error record lives in the array and is not visible to lightning_attn_check; the
+//    decode kernel has no bounded waits, so the launch status is the whole error report.
 #include <mutex>
 
 #include "la_common.cuh"
@@ -33,6 +38,7 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const voi
                           const int* row_index = nullptr, const int* state_index = nullptr,
                           float* z = nullptr);
 size_t decode_workspace_bytes(int B, int H, int D);
+void set_last_path(const char* path);
 }  // namespace la
 
 namespace {
@@ -90,5 +96,7 @@ extern "C" la_status lightning_attn_decode_step_noalloc(const void* q, const voi
     return LA_ERR_CUDA;
   const cudaError_t e = la::launch_decode(q, k, v, g, out, state, B, H, D, dtype, phi == LA_PHI_IDENTITY ? 1 : 0,
                                           static_cast<int>(mode), eps, norm_weight, scratch, s);
-  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+  if (e != cudaSuccess) return LA_ERR_CUDA;
+  la::set_last_path("decode");
+  return LA_OK;
 }

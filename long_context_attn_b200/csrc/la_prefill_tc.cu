@@ -16,8 +16,8 @@
 //    second tile multiplies by the first tile's keys densely and by its own keys under the
 //    causal mask; the all-zero upper-right quarter of the 256 x 256 block is never issued.
 //  * The two CTAs of a head form a cluster.  Each loads (TMA, 128-byte swizzle) its own
-//    64-column box of the Q and K tiles plus its V slice, applies SiLU to its boxes with
-//    six transform warps, and writes the result both into its own shared memory and into
+//    64-column box of the Q and K tiles plus its V slice, applies SiLU (packed bf16x2
+//    arithmetic) to its boxes with six transform warps, and writes the result both into its own shared memory and into
 //    its partner's (distributed shared memory), so each SiLU is computed once per head and
 //    both CTAs end up with the full phi(Q), phi(K) tiles.  Q tiles use a two-slot ring and
 //    K/V tiles a three-slot ring, so the next block's first tile loads while the second
@@ -60,6 +60,7 @@
 #include "la_common.cuh"
 #include "la_prefill_tc.h"
 #include "la_sm100.cuh"
+#include "la_tc_util.cuh"
 
 namespace la {
 using namespace sm100;
@@ -225,8 +226,8 @@ __device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, int* 
   const uint64_t t0 = globaltimer_ns();
   const uint64_t lim = wait_limit_ns(err);
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 31u) == 0) {
+    if (mbar_try_wait_sleep(bar, parity, 20000)) return true;   // suspends: no issue slots used
+    if ((n & 3u) == 0) {
       if (*reinterpret_cast<volatile int*>(abort_flag) != 0) return false;
       if (globaltimer_ns() - t0 > lim) {
         report(err, LA_ERR_TIMEOUT, site, index, parity);
@@ -248,7 +249,8 @@ __device__ __noinline__ bool poll_count_slow(unsigned int* c, uint32_t W, int* a
                                              uint32_t index) {
   const uint64_t t0 = globaltimer_ns();
   const uint64_t lim = wait_limit_ns(err);
-  while (ld_acquire_gpu(c) < W) {
+  for (uint32_t ns = 32; ld_acquire_gpu(c) < W; ns = ns < 256 ? 2 * ns : ns) {
+    __nanosleep(ns);
     if (*reinterpret_cast<volatile int*>(abort_flag) != 0) return false;
     if (globaltimer_ns() - t0 > lim) {
       report(err, LA_ERR_TIMEOUT, SITE_TC_NORM_WAIT, index, ld_acquire_gpu(c));
@@ -273,17 +275,6 @@ __device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, Ba
                                               uint32_t site, uint32_t index) {
   const bool ok = wait_bar(bar, parity, B, p, site, index);
   return __all_sync(0xFFFFFFFFu, ok);
-}
-
-// SiLU of two packed bf16 values in packed bf16 arithmetic, from sigmoid(x) =
-// (1 + tanh(x/2)) / 2:  h = x/2 (exact), t = tanh(h) (one MUFU op for both halves),
-// SiLU(x) = h + h t (one fused multiply-add, rounded once to bf16).
-__device__ __forceinline__ uint32_t silu_bf16x2(uint32_t x) {
-  uint32_t h, t, r;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(h) : "r"(x), "r"(0x3F003F00u));
-  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(h));
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(h), "r"(t), "r"(h));
-  return r;
 }
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v);
@@ -626,7 +617,7 @@ lightning_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __gr
             if ((c >> 3) >= zero_from) {
               x = make_uint4(0, 0, 0, 0);
             } else if (!p.phi_identity) {
-              x.x = silu_bf16x2(x.x); x.y = silu_bf16x2(x.y); x.z = silu_bf16x2(x.z); x.w = silu_bf16x2(x.w);
+              x = tcu::silu8(x);
             }
             sts128(sbase + off0 + 16u * c, x);
             st_cluster128(remote + off0 + 16u * c, x);
@@ -1033,7 +1024,8 @@ int max_active_clusters() {
       n = -1;
     cache[dev] = n;
   }
-  return cache[dev];
+  const int pairs = pair_max_active_clusters();
+  return std::min(cache[dev], pairs);
 }
 
 bool tc_eligible(const TcShape& s, int num_sms) {
@@ -1047,14 +1039,16 @@ bool tc_eligible(const TcShape& s, int num_sms) {
 size_t tc_workspace_bytes(int nseq, int max_len, int64_t tokens, int H, int D, int C) {
   (void)D;
   (void)C;
-  (void)H;
   const size_t max_tiles = (static_cast<size_t>(max_len) + kTile - 1) / kTile;
-  return up256(sizeof(unsigned int) * static_cast<size_t>(nseq) * (max_tiles ? max_tiles : 1)) +
-         up256(sizeof(double) * static_cast<size_t>(tokens > 0 ? tokens : 1));
+  const size_t own = up256(sizeof(unsigned int) * static_cast<size_t>(nseq) * (max_tiles ? max_tiles : 1)) +
+                     up256(sizeof(double) * static_cast<size_t>(tokens > 0 ? tokens : 1));
+  return std::max(own, pair_workspace_bytes(nseq, max_len, tokens, H));
 }
 
 cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream) {
   (void)num_sms;
+  // Forward time runs on the pair kernel; this kernel serves the reverse-time passes.
+  if (!a.reverse) return launch_pair_prefill(a, stream);
   const int max_tiles = (a.max_len + kTile - 1) / kTile;
   const size_t cnt_bytes = up256(sizeof(unsigned int) * static_cast<size_t>(a.nseq) * (max_tiles ? max_tiles : 1));
   const size_t ss_bytes = up256(sizeof(double) * static_cast<size_t>(a.tokens > 0 ? a.tokens : 1));

@@ -30,6 +30,8 @@ struct TcArgs {
   char* ws;            // workspace after the error record
   const int* state_index;  // optional [nseq] device: state slot of each sequence (else s)
   int skip_single;         // nonzero: sequences of exactly one token are left alone entirely
+  int chunk_div;           // > 1 (forward only): sequence s is chunk s % chunk_div of sequence
+                           // s / chunk_div; only a last chunk writes state_out (at s / chunk_div)
 };
 
 // True when the tensor-core kernel handles this shape on a GPU with `num_sms` SMs.
@@ -37,7 +39,16 @@ bool tc_eligible(const TcShape& s, int num_sms);
 // Workspace bytes after the 256-byte error record.
 size_t tc_workspace_bytes(int nseq, int max_len, int64_t tokens, int H, int D, int C);
 cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream);
-// CTA pairs (heads x groups) that fit on the current device at once.
+// CTA pairs (heads x groups) that fit on the current device at once (the smaller count of
+// the two tensor-core prefill kernels).
 int max_active_clusters();
+
+// The forward-time prefill (la_prefill_pair.cu): one head per CTA pair, blocks alternating
+// between the two CTAs, the state handed over through a per-pair buffer in the workspace.
+cudaError_t launch_pair_prefill(const TcArgs& a, cudaStream_t stream);
+size_t pair_workspace_bytes(int nseq, int max_len, int64_t tokens, int H);
+int pair_max_active_clusters();
+// Sequence groups of the pair kernel for a call (2 workers per head and group).
+int pair_groups(int nseq, int H);
 
 }  // namespace la

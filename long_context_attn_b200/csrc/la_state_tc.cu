@@ -15,7 +15,7 @@
 //    depend on timing.
 //  * Warp 0 (one lane) streams K (two 64-column boxes) and V (two boxes) of each tile with
 //    TMA (128-byte swizzle) into a three-stage ring; warps 4-11 apply SiLU to the K boxes in
-//    place (the same packed-bf16 form as the tensor-core prefill, so both give the same
+//    place (the same packed-bf16 SiLU as the tensor-core prefill, so both give the same
 //    state) and zero the rows past the sequence end in K and V; warp 1 (one lane) issues,
 //    per tile, 8 k-steps x 2 MMAs  S[:, 0:64] += phi(K)^T V[:, 0:64],  S[:, 64:128] += ...
 //    (both operands MN-major, M = d_k = 128, N = 64, K = 16 tokens); warps 0-3 (one per
@@ -28,6 +28,7 @@
 
 #include "la_common.cuh"
 #include "la_sm100.cuh"
+#include "la_tc_util.cuh"
 
 namespace la {
 using namespace sm100;
@@ -79,24 +80,14 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
 }
-// SiLU of two packed bf16 values: h = x/2, SiLU(x) = h + h * tanh(h) (sigmoid(x) =
-// (1 + tanh(x/2)) / 2), in packed bf16 arithmetic with one MUFU op for both halves.
-__device__ __forceinline__ uint32_t silu_bf16x2(uint32_t x) {
-  uint32_t h, t, r;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(h) : "r"(x), "r"(0x3F003F00u));
-  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(h));
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(h), "r"(t), "r"(h));
-  return r;
-}
-
 // Bounded wait; false once the CTA is aborting (this wait ran out, or another role's did).
 __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, int* abort_flag, ErrRec* err, uint32_t site,
                                        uint32_t index) {
   const uint64_t t0 = globaltimer_ns();
   const uint64_t lim = wait_limit_ns(err);
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 31u) == 0) {
+    if (mbar_try_wait_sleep(bar, parity, 20000)) return true;   // suspends: no issue slots used
+    if ((n & 3u) == 0) {
       if (*reinterpret_cast<volatile int*>(abort_flag) != 0) return false;
       if (globaltimer_ns() - t0 > lim) {
         report(err, LA_ERR_TIMEOUT, site, index, parity);
@@ -235,7 +226,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             if ((c >> 3) >= vr) {
               y = make_uint4(0, 0, 0, 0);
             } else if (!p.phi_identity) {
-              y.x = silu_bf16x2(y.x); y.y = silu_bf16x2(y.y); y.z = silu_bf16x2(y.z); y.w = silu_bf16x2(y.w);
+              y = tcu::silu8(y);
             }
             sts128(box + 16u * c, y);
           }

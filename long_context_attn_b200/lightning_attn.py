@@ -300,6 +300,10 @@ def lightning_attn_decode_step_noalloc(q, k, v, g, out, state, phi=LA_PHI_SILU, 
     """
     B, H, D = q.shape
     _check_contig(q, k, v, g, out, state)
+    dev = torch.cuda.current_device()
+    for t in (q, k, v, g, out, state, norm_weight):
+        if t is not None and (t.device.type != "cuda" or t.device.index != dev):
+            raise ValueError(f"tensors must be on the current CUDA device cuda:{dev}, got {t.device}")
     st = _lib.lightning_attn_decode_step_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(out),
                                                  _ptr(_f32_or_none(state)), B, H, D, _dtype(q), phi, mode, eps,
                                                  _ptr(_f32_or_none(norm_weight)), _stream(stream))

@@ -19,3 +19,11 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.fail("GPU test selected but torch.cuda.is_available() is False")
     return torch.device("cuda:0")
+
+
+def pytest_terminal_summary(terminalreporter):
+    from tests._helpers import MARGINS
+    if MARGINS:
+        terminalreporter.write_sep("-", "parity margins (max|err| / max|ref|; tolerance 2e-2 bf16, 1e-4 fp32)")
+        for name, text in MARGINS:
+            terminalreporter.write_line(f"{name}: {text}")

@@ -4,7 +4,7 @@ import pytest
 
 import oracle
 import synth
-from tests._helpers import as_f64, assert_close, mode_code, rel_err, to_dev, to_host
+from tests._helpers import as_f64, assert_close, mode_code, record_margin, rel_err, to_dev, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -91,5 +91,7 @@ def test_decode_full_config_16_steps(cuda_device):
         ref_S = ref_S64.astype(np.float32)
         if step in (0, 15):
             la.lightning_attn_check(ws)
-            assert_close(to_host(out), ref_o, "bf16", f"decode output after step {step + 1}")
-            assert rel_err(to_host(dS), ref_S64) <= 1e-5
+            e_o = assert_close(to_host(out), ref_o, "bf16", f"decode output after step {step + 1}")
+            e_s = rel_err(to_host(dS), ref_S64)
+            assert e_s <= 1e-5
+            record_margin(f"test_decode_full_config_16_steps step {step + 1}", out=e_o, state=e_s)

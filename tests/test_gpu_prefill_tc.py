@@ -14,7 +14,7 @@ import pytest
 
 import oracle
 import synth
-from tests._helpers import as_f64, assert_close, mode_code
+from tests._helpers import as_f64, assert_close, mode_code, record_margin
 from tests.test_gpu_prefill_simt import run_prefill, run_varlen
 
 pytestmark = pytest.mark.gpu
@@ -131,11 +131,13 @@ def test_tc_config_8k(cuda_device):
     w = synth.WORKLOADS["prefill_8k"]
     q, k, v, g = synth.prefill_inputs(w.seed, w.T, w.H, w.D, "bf16", w.qkv_scale, True)
     o, st, _ = run_prefill(q[None], k[None], v[None], g[None], w.block_size, oracle.MODE_RMSNORM_GATE,
-                           want_state=True, expect_path="tcgen05")
+                           want_state=True, expect_path="tcgen05+chunks")
     _, _, stats = oracle.prefill(q[None], k[None], v[None], g[None], store=False, cand_out=o, cand_state=st)
     assert stats["out_nonfinite"] == 0 and stats["state_nonfinite"] == 0
     assert stats["out_max_err"] <= 2e-2 * stats["out_max_ref"], stats
     assert stats["state_max_err"] <= 2e-2 * stats["state_max_ref"], stats
+    record_margin("test_tc_config_8k", out=stats["out_max_err"] / stats["out_max_ref"],
+                  state=stats["state_max_err"] / stats["state_max_ref"])
 
 
 @pytest.mark.slow
@@ -145,11 +147,13 @@ def test_tc_config_128k_full(cuda_device):
     w = synth.WORKLOADS["prefill_128k"]
     q, k, v, g = synth.prefill_inputs(w.seed, w.T, w.H, w.D, "bf16", w.qkv_scale, True)
     o, st, _ = run_prefill(q[None], k[None], v[None], g[None], w.block_size, oracle.MODE_RMSNORM_GATE,
-                           want_state=True, expect_path="tcgen05")
+                           want_state=True, expect_path="tcgen05+chunks")
     _, _, stats = oracle.prefill(q[None], k[None], v[None], g[None], store=False, cand_out=o, cand_state=st)
     assert stats["out_nonfinite"] == 0 and stats["state_nonfinite"] == 0
     assert stats["out_max_err"] <= 2e-2 * stats["out_max_ref"], stats
     assert stats["state_max_err"] <= 2e-2 * stats["state_max_ref"], stats
+    record_margin("test_tc_config_128k_full", out=stats["out_max_err"] / stats["out_max_ref"],
+                  state=stats["state_max_err"] / stats["state_max_ref"])
 
 
 @pytest.mark.slow
@@ -167,6 +171,8 @@ def test_tc_config_varlen16_full(cuda_device):
     assert stats["out_nonfinite"] == 0 and stats["state_nonfinite"] == 0
     assert stats["out_max_err"] <= 2e-2 * stats["out_max_ref"], stats
     assert stats["state_max_err"] <= 2e-2 * stats["state_max_ref"], stats
+    record_margin("test_tc_config_varlen16_full", out=stats["out_max_err"] / stats["out_max_ref"],
+                  state=stats["state_max_err"] / stats["state_max_ref"])
 
 
 @pytest.mark.parametrize("mode,expect", [("rmsnorm_gate", "tcgen05+norm"), ("rmsnorm", "tcgen05+norm"),
