@@ -155,8 +155,12 @@ SplitLayout split_layout(const SplitPlan& sp, int B, int64_t tokens, int H, int 
   l.tc = la::tc_workspace_bytes(n, sp.Tc, tokens, H, D, C);
   l.cu = up256(sizeof(int) * static_cast<size_t>(n + 1));
   l.st = up256(sizeof(float) * static_cast<size_t>(n) * H * D * D);
-  l.part = up256(sizeof(float) * static_cast<size_t>(la::chunk_state_splits(n, H, sp.Tc, current_sm_count())) * n *
-                 H * D * D);
+  // Chunk-state partials: the launch covers n chunks, or n - 1 when a single forward-time
+  // sequence skips its last chunk, and fewer chunks may take more splits each.
+  const int sms = current_sm_count();
+  size_t units = static_cast<size_t>(la::chunk_state_splits(n, H, sp.Tc, sms)) * n;
+  if (n > 1) units = std::max(units, static_cast<size_t>(la::chunk_state_splits(n - 1, H, sp.Tc, sms)) * (n - 1));
+  l.part = up256(sizeof(float) * units * H * D * D);
   l.total = l.tc + l.cu + 2 * l.st + l.part;
   return l;
 }
