@@ -21,19 +21,25 @@
 //    extents of 32, 64 or 128 rows (`lightning_attention_pad_options`) with zeroed tail rows
 //    of K and V.  The inter product phi(Q_b) S_{b-1} uses a bf16 snapshot of the state that
 //    the state warps take after the previous block's last state update.
-//  * Roles (24 warps): warp 0 streams Q tiles (lane 0) and K/V tiles (lane 1) with TMA into
-//    two-slot rings; warp 1 issues every MMA; warps 2-7 apply SiLU (packed bf16x2
-//    arithmetic) to Q and K in place; warps 8-11 turn score tiles into masked bf16 in TMEM;
-//    warps 12-15 own the state (S0 in, the snapshot, the final state out); warps 16-23 read
-//    the output accumulators (each warp 64 of the 128 columns of its TMEM lane quarter),
-//    publish the rows' sums of squares and, once all heads of the tile have published,
-//    read the accumulator again and store o = y w rsqrt(mean(y^2) + eps) sigmoid(g).
-//  * TMEM (512 columns): S (128), two output accumulators (2 x 128), one score region (128).
-//  * Cross-head RMSNorm: every epilogue thread adds its row's partial sum of squares into an
-//    fp64 per-token total (red.add; exact and order-independent while a token's partials
-//    span less than 2^22), and each warp bumps the tile's arrival counter after a fence.
-//    The same worker of every head processes the same tiles in the same order, and all CTAs
-//    are resident at once (checked on the host).
+//  * Roles (32 warps): warp 0 streams Q, K and V tiles with TMA into two-slot rings (one
+//    lane per ring); warp 1 issues every MMA; warps 2, 3 and 24-31 apply SiLU (packed
+//    bf16x2 arithmetic) to K in place; warps 4-7 turn score tiles into masked bf16 in TMEM;
+//    warps 8-11 apply SiLU to Q on its way into TMEM; warps 12-15 own the state (S0 in, the
+//    snapshot, the final state out) and the output accumulator (each row read once,
+//    written out and, in the norm modes, its sum of squares published); warps 16-23, once
+//    all heads of a tile have published, rescale its rows in place:
+//    o = z rsqrt(mean(y^2) + eps) sigmoid(g) with z = bf16(y w).
+//  * TMEM (512 columns): S (128), the output accumulator (128), one score region (128),
+//    phi(Q) of two tiles (2 x 64, the A operand of the score and inter MMAs).  The three
+//    score jobs of a block go through the one region back to back: MMAs of one thread run
+//    in issue order, so each job is issued right after the previous job's PV.
+//  * Cross-head RMSNorm: every drain thread adds its row's sum of squares into an fp64
+//    per-token total (red.add; exact and order-independent while a token's partials span
+//    less than 2^22), and each warp bumps the tile's arrival counter after a fence.  The
+//    same worker of every head processes the same tiles in the same order, and all CTAs are
+//    resident at once (checked on the host).  A CTA's Q loads wait until every head has
+//    published the tile kThrottle tiles back, so the rows waiting for their rescale stay
+//    few enough to remain in L2.
 //  * Every wait is bounded (globaltimer); a wait that runs out records LA_ERR_TIMEOUT in
 //    the workspace, raises the CTA's abort flag and the CTA drains its async work, frees
 //    TMEM and exits.
@@ -57,32 +63,49 @@ namespace {
 
 constexpr int kD = 128;           // head dim (d_k = d_v)
 constexpr int kTile = 128;        // rows per tile (MMA M)
-constexpr int kThreads = 768;     // 24 warps
-constexpr int kConvWarp0 = 4;     // warps 4..7: score conversion, the state, the rows' sums of squares
-constexpr int kXfThreads = 320;   // transform: warps 2, 3 and 8..15
-constexpr int kXfIlp = 8;         // 16-byte chunks in flight per transform thread
-constexpr int kEpiWarp0 = 16;     // warps 16..23: the output stores
+constexpr int kThreads = 1024;    // 32 warps
+constexpr int kConvWarp0 = 4;     // warps 4..7: score conversion
+constexpr int kQxfWarp0 = 8;      // warps 8..11: SiLU of Q into TMEM (one TMEM lane quarter each)
+constexpr int kStateWarp0 = 12;   // warps 12..15: the state and the rows' sums of squares
+constexpr int kXfThreads = 320;   // warps 2, 3, 24..31: SiLU of K in place
+constexpr int kXfIlp = 4;         // 16-byte chunks in flight per K-transform thread
+constexpr int kEpiWarp0 = 16;     // warps 16..23: the normalised output (norm modes)
 constexpr int kEpiWarps = 8;
+constexpr int kXfWarp1 = 24;      // first of the K-transform warps after the output warps
 constexpr int kPubWarps = 4;      // arrivals per CTA that publish a tile's sums
+// Norm modes: the Q loads of own tile t wait until every head has published the sums of own
+// tile t - kThrottle, so that no CTA runs far ahead of the slowest head.  The rows each CTA
+// has written but not yet rescaled then stay few enough to remain in L2 until the final
+// warps read them back.
+constexpr int kThrottle = 6;
 
 constexpr uint32_t kBoxBytes = kTile * 64 * 2;    // one 128-row x 64-column bf16 box (16 KiB)
 constexpr uint32_t kTileBytes = 2 * kBoxBytes;    // a 128 x 128 tile: two boxes (32 KiB)
-constexpr uint32_t OFF_Q = 0;                     // 2 slots
-constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;
+constexpr uint32_t OFF_Q = 0;                     // 2 slots (landing only: phi(Q) moves to TMEM)
+constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;   // 2 slots
 constexpr uint32_t OFF_V = OFF_K + 2 * kTileBytes;
 constexpr uint32_t OFF_SNAP = OFF_V + 2 * kTileBytes;
 constexpr uint32_t OFF_BARS = OFF_SNAP + kTileBytes;
 
+// Norm exchange in global memory: one 128-byte line per token sum and per tile counter, so
+// that the 64 heads' additions to one tile's sums spread over many L2 slices instead of
+// queueing on the eight lines 128 packed fp64 values would share.
+constexpr int kSsStride = 16;    // doubles per token
+constexpr int kCntStride = 32;   // counters per tile
+
 constexpr uint32_t TM_S = 0;      // S, 128 columns (lanes = d_k, columns = d_v)
-constexpr uint32_t TM_O = 128;    // two output accumulators, 128 columns each
-constexpr uint32_t TM_P = 384;    // score region, 128 columns
+constexpr uint32_t TM_O = 128;    // the output accumulator, 128 columns
+constexpr uint32_t TM_P = 256;    // the score region, 128 columns
+constexpr uint32_t TM_Q = 384;    // phi(Q) of two tiles, 64 columns each (bf16 pairs; MMA A operand)
 constexpr uint32_t kTmemCols = 512;
 
 struct Bars {
-  uint64_t full_q[2], xf_q[2], q_empty[2];
-  uint64_t full_kv[2], xf_kv[2], kv_empty[2];
-  uint64_t p_full, p_conv, pv_done;
-  uint64_t o_full[2], o_empty[2];
+  uint64_t full_q[2], q_empty[2];      // Q landing slots (freed once phi(Q) is in TMEM)
+  uint64_t qt_ready[2], qt_free[2];    // phi(Q) tiles in TMEM
+  uint64_t full_k[2], xf_k[2], k_empty[2];
+  uint64_t full_v[2], v_empty[2];
+  uint64_t p_full, p_conv;
+  uint64_t o_full, o_empty;
   uint64_t s_ready;     // S in TMEM may take the block's state update (S0 written / S_{b-1} read)
   uint64_t snap_ready;  // bf16 snapshot of S_{b-1} written
   uint64_t su_done;     // the block's state update (and its inter products) completed
@@ -282,18 +305,20 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&B.qt_ready[i], 4);
+      mbar_init(&B.qt_free[i], 1);
       mbar_init(&B.full_q[i], 1);
-      mbar_init(&B.xf_q[i], kXfThreads);
-      mbar_init(&B.q_empty[i], 1);
-      mbar_init(&B.full_kv[i], 1);
-      mbar_init(&B.xf_kv[i], kXfThreads);
-      mbar_init(&B.kv_empty[i], 1);
-      mbar_init(&B.o_full[i], 1);
-      mbar_init(&B.o_empty[i], kEpiWarps);
+      mbar_init(&B.q_empty[i], 4);   // the Q-transform warps
+      mbar_init(&B.full_k[i], 1);
+      mbar_init(&B.xf_k[i], kXfThreads);
+      mbar_init(&B.k_empty[i], 1);
+      mbar_init(&B.full_v[i], 1);
+      mbar_init(&B.v_empty[i], 1);
     }
     mbar_init(&B.p_full, 1);
     mbar_init(&B.p_conv, 128);
-    mbar_init(&B.pv_done, 1);
+    mbar_init(&B.o_full, 1);
+    mbar_init(&B.o_empty, 4);   // the four drain warps
     mbar_init(&B.s_ready, 128);
     mbar_init(&B.snap_ready, 128);
     mbar_init(&B.su_done, 1);
@@ -313,76 +338,69 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
   const uint32_t tmem = B.tmem_base;
 
   // ------------------------------------------------------------------------------------
-  // Warp 0: TMA producers.  Lane 0: Q tiles of this CTA's blocks into Q slot (own tile % 2);
-  // lane 1: K and V tiles into K/V slot (own tile % 2), and the gate tile prefetched into
-  // L2 for the epilogue.  Own tiles are numbered in walk order; both rings use that number.
+  // Warp 0: TMA producers, one lane per two-slot ring: lane 0 Q tiles, lane 1 K tiles (and
+  // the gate tile prefetched into L2 for the output), lane 2 V tiles.  Own tiles are numbered
+  // in walk order and every ring uses that number: tile t goes to slot t % 2.  Each tile of
+  // the next block is also prefetched into L2 when its load is issued.
   // ------------------------------------------------------------------------------------
   if (warp == 0) {
-    if (lane < 2) {
-      const bool is_q = lane == 0;
-      if (is_q) {
-        prefetch_tmap(&tm_q);
-      } else {
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_v);
-        if (gate) prefetch_tmap(&tm_g);
-      }
+    if (lane < 3) {
+      const CUtensorMap* map = lane == 0 ? &tm_q : (lane == 1 ? &tm_k : &tm_v);
+      prefetch_tmap(map);
+      if (lane == 1 && gate) prefetch_tmap(&tm_g);
+      uint64_t* full = lane == 0 ? B.full_q : (lane == 1 ? B.full_k : B.full_v);
+      uint64_t* empty = lane == 0 ? B.q_empty : (lane == 1 ? B.k_empty : B.v_empty);
+      const uint32_t off = lane == 0 ? OFF_Q : (lane == 1 ? OFF_K : OFF_V);
+      constexpr uint32_t sh = 1;   // log2 of the slots per ring
       const uint64_t pol = policy_evict_first();
       uint32_t ot = 0;
       bool ok = true;
+      unsigned int* hist[kThrottle];   // norm counters of the last kThrottle own tiles (Q lane)
+#pragma unroll
+      for (int j = 0; j < kThrottle; ++j) hist[j] = nullptr;
       BlkIter it;
       blk_first<tpb>(p, it, wk);
       for (; it.valid && ok; blk_next<tpb>(p, it, wk)) {
         int vr0, vr1;
         const int n = blk_tiles<tpb>(it, vr0, vr1);
         for (int u = 0; u < n; ++u, ++ot) {
-          const uint32_t sl = ot & 1u;
-          uint64_t* empty = is_q ? &B.q_empty[sl] : &B.kv_empty[sl];
-          if (ot >= 2 && !tcu::wait(empty, ((ot >> 1) - 1) & 1u, abort_flag, err, SITE_TC_PRODUCER, ot)) {
+          if (norm && lane == 0) {
+            unsigned int* c = hist[kThrottle - 1];
+            if (c && ld_acquire_gpu(c) < W && !tcu::poll_count(c, W, abort_flag, err, ot)) {
+              ok = false;
+              break;
+            }
+#pragma unroll
+            for (int j = kThrottle - 1; j > 0; --j) hist[j] = hist[j - 1];
+            hist[0] = p.cnt + (static_cast<int64_t>(it.s) * p.max_tiles + it.jb * tpb + u) * kCntStride;
+          }
+          const uint32_t sl = ot & sh, use = ot >> sh;   // slot, and the loads into it before
+          if (use >= 1 && !tcu::wait(&empty[sl], (use - 1) & 1u, abort_flag, err, SITE_TC_PRODUCER, ot)) {
             ok = false;
             break;
           }
           const int32_t row = static_cast<int32_t>(it.row0 + static_cast<int64_t>(it.jb * tpb + u) * kTile);
           const int32_t col = h * kD;
-          // The same tile of the next block, into L2: the demand on DRAM runs a block ahead
-          // of the two-slot rings.
-          const bool ahead = (it.jb * tpb + u + tpb) < it.nt;
-          if (is_q) {
-            if (ahead) {
-              tma_prefetch_l2_2d(&tm_q, col, row + kC);
-              tma_prefetch_l2_2d(&tm_q, col + 64, row + kC);
-            }
-            uint8_t* dst = smem + OFF_Q + sl * kTileBytes;
-            mbar_arrive_expect_tx(&B.full_q[sl], kTileBytes);
-            tma_load_2d(dst, &tm_q, col, row, &B.full_q[sl], pol);
-            tma_load_2d(dst + kBoxBytes, &tm_q, col + 64, row, &B.full_q[sl], pol);
-          } else {
-            if (ahead) {
-              tma_prefetch_l2_2d(&tm_k, col, row + kC);
-              tma_prefetch_l2_2d(&tm_k, col + 64, row + kC);
-              tma_prefetch_l2_2d(&tm_v, col, row + kC);
-              tma_prefetch_l2_2d(&tm_v, col + 64, row + kC);
-            }
-            uint8_t* dk = smem + OFF_K + sl * kTileBytes;
-            uint8_t* dv = smem + OFF_V + sl * kTileBytes;
-            mbar_arrive_expect_tx(&B.full_kv[sl], 2 * kTileBytes);
-            tma_load_2d(dk, &tm_k, col, row, &B.full_kv[sl], pol);
-            tma_load_2d(dk + kBoxBytes, &tm_k, col + 64, row, &B.full_kv[sl], pol);
-            tma_load_2d(dv, &tm_v, col, row, &B.full_kv[sl], pol);
-            tma_load_2d(dv + kBoxBytes, &tm_v, col + 64, row, &B.full_kv[sl], pol);
-            if (gate) {
-              tma_prefetch_l2_2d(&tm_g, col, row);
-              tma_prefetch_l2_2d(&tm_g, col + 64, row);
-            }
+          if ((it.jb * tpb + u + tpb) < it.nt) {
+            tma_prefetch_l2_2d(map, col, row + kC);
+            tma_prefetch_l2_2d(map, col + 64, row + kC);
+          }
+          uint8_t* dst = smem + off + sl * kTileBytes;
+          mbar_arrive_expect_tx(&full[sl], kTileBytes);
+          tma_load_2d(dst, map, col, row, &full[sl], pol);
+          tma_load_2d(dst + kBoxBytes, map, col + 64, row, &full[sl], pol);
+          if (lane == 1 && gate) {
+            tma_prefetch_l2_2d(&tm_g, col, row);
+            tma_prefetch_l2_2d(&tm_g, col + 64, row);
           }
         }
       }
       // Drain: every issued load must land before the CTA may exit (the last load into
-      // each slot is own tile ot - 1 or ot - 2).
-      for (uint32_t sl = 0; sl < 2; ++sl) {
+      // each slot is own tile ot - 1, or ot - 2 for the other slot of a two-slot ring).
+      for (uint32_t sl = 0; sl <= sh; ++sl) {
         if (ot <= sl) continue;
-        const uint32_t t = ((ot - 1) & 1u) == sl ? ot - 1 : ot - 2;
-        tcu::drain(is_q ? &B.full_q[sl] : &B.full_kv[sl], (t >> 1) & 1u);
+        const uint32_t t = ((ot - 1) & sh) == sl ? ot - 1 : ot - 2;
+        tcu::drain(&full[sl], (t >> sh) & 1u);
       }
     }
   }
@@ -391,7 +409,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
   // ------------------------------------------------------------------------------------
   else if (warp == 1) {
     if (lane == 0) {
-      uint32_t ot = 0, jb = 0, nb = 0;
+      uint32_t ot = 0, nb = 0, jb = 0;
       bool ok = true;
       BlkIter it;
       blk_first<tpb>(p, it, wk);
@@ -400,25 +418,23 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
         tc_fence_after();
         return true;
       };
-      // Score job into the region (after the previous job's PV has completed).
-      auto issue_p = [&](uint32_t qs, uint32_t ks, uint32_t n) -> bool {
-        if (jb > 0 && !mw(&B.pv_done, (jb - 1) & 1u, jb)) return false;
-        const uint64_t qd = desc_at(kDescK, sbase + OFF_Q + qs * kTileBytes);
+      // Score job phi(Q) K^T (A = phi(Q) of Q tile qs in TMEM) into the score region.  MMAs
+      // issued by one thread execute in issue order, so the job may follow the previous job's
+      // PV (which reads the converted scores there) without waiting for it to complete.
+      auto issue_p = [&](uint32_t qs, uint32_t ks, uint32_t n) {
         const uint64_t kd = desc_at(kDescK, sbase + OFF_K + ks * kTileBytes);
         const uint32_t idesc = make_idesc_bf16(128, n, 0, 0);
 #pragma unroll 1
-        for (int kk = 0; kk < 8; ++kk) mma_ss(tmem + TM_P, qd + kstep_k(kk), kd + kstep_k(kk), idesc, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) mma_ts(tmem + TM_P, tmem + TM_Q + 64 * qs + 8 * kk, kd + kstep_k(kk), idesc, kk > 0);
         mma_commit(&B.p_full);
-        return true;
       };
-      // PV of the current job into accumulator od over ksteps key steps.
-      auto issue_pv = [&](uint32_t od, uint32_t vs, int ksteps, bool acc) -> bool {
+      // PV of the converted scores into the accumulator over ksteps key steps.
+      auto issue_pv = [&](uint32_t vs, int ksteps, bool acc) -> bool {
         if (!mw(&B.p_conv, jb & 1u, jb)) return false;
         const uint64_t vd = desc_at(kDescMN, sbase + OFF_V + vs * kTileBytes);
 #pragma unroll 1
         for (int kk = 0; kk < ksteps; ++kk)
-          mma_ts(od, tmem + TM_P + 8 * kk, vd + 128 * kk, kIdesc128MN, (acc || kk > 0) ? 1u : 0u);
-        mma_commit(&B.pv_done);
+          mma_ts(tmem + TM_O, tmem + TM_P + 8 * kk, vd + 128 * kk, kIdesc128MN, (acc || kk > 0) ? 1u : 0u);
         ++jb;
         return true;
       };
@@ -427,176 +443,268 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
         const uint64_t kd = desc_at(kDescMN, sbase + OFF_K + ks * kTileBytes);
         const uint64_t vd = desc_at(kDescMN, sbase + OFF_V + ks * kTileBytes);
 #pragma unroll 1
-        for (int kk = 0; kk < ksteps; ++kk)
-          mma_ss(tmem + TM_S, kd + 128 * kk, vd + 128 * kk, kIdescSU, 1u);
+        for (int kk = 0; kk < ksteps; ++kk) mma_ss(tmem + TM_S, kd + 128 * kk, vd + 128 * kk, kIdescSU, 1u);
       };
-      auto issue_qs = [&](uint32_t od, uint32_t qs) {
-        const uint64_t qd = desc_at(kDescK, sbase + OFF_Q + qs * kTileBytes);
+      // O += phi(Q) S_{b-1} (A = phi(Q) in TMEM, B = the bf16 snapshot).
+      auto issue_qs = [&](uint32_t qs) {
         const uint64_t sd = desc_at(kDescMN, sbase + OFF_SNAP);
 #pragma unroll 1
-        for (int kk = 0; kk < 8; ++kk) mma_ss(od, qd + kstep_k(kk), sd + 128 * kk, kIdesc128MN, 1u);
+        for (int kk = 0; kk < 8; ++kk) mma_ts(tmem + TM_O, tmem + TM_Q + 64 * qs + 8 * kk, sd + 128 * kk, kIdesc128MN, 1u);
       };
 
-      // Per block: the score jobs (A = Q0 K0^T masked, B = Q1 K0^T dense, C = Q1 K1^T
-      // masked) through the single score region, each followed by its PV; the inter
-      // products with the snapshot of S_{b-1}; the state update over both tiles' keys after
-      // the inter products (so that su_done also covers them and the snapshot area is free
-      // once the state warps see it).
+      // Per block, score jobs A = Q0 K0^T (masked), B = Q1 K0^T (dense), C = Q1 K1^T (masked)
+      // run back to back through the one score region: each job is issued right after the
+      // previous job's PV, so the conversion warps always have the next job in flight, and
+      // the inter products and state updates fill the tensor pipe while they convert.  Tile
+      // 0's accumulator is PV_A + Q0 S_{b-1}; tile 1's is PV_B + PV_C + Q1 S_{b-1}.  Each
+      // operand is released after its last use: K0 after B and the state update over tile 0,
+      // V0 after PV_B, K1 after C and the update over tile 1, V1 after PV_C.  su_done comes
+      // after both inter products, so the snapshot area is free once the state warps see it.
       for (; it.valid && ok; blk_next<tpb>(p, it, wk)) {
         int vr0, vr1;
         const int n = blk_tiles<tpb>(it, vr0, vr1);
-        const uint32_t s0 = ot & 1u, s1 = (ot + 1) & 1u;            // slots (and accumulators)
+        const uint32_t s0 = ot & 1u, s1 = (ot + 1) & 1u;            // slots (and phi(Q) tiles)
         const uint32_t ph0 = (ot >> 1) & 1u, ph1 = ((ot + 1) >> 1) & 1u;
         const int pad0 = pad_rows(vr0), pad1 = n > 1 ? pad_rows(vr1) : 0;
-        const uint32_t od0 = tmem + TM_O + 128 * s0, od1 = tmem + TM_O + 128 * s1;
-        // job A: Q0 K0^T (masked) -> PV into accumulator s0, then Q0 S_{b-1}
-        if (!mw(&B.xf_kv[s0], ph0, ot) || !mw(&B.xf_q[s0], ph0, ot)) break;
-        if (!issue_p(s0, s0, static_cast<uint32_t>(pad0))) break;
-        if (ot >= 2 && !mw(&B.o_empty[s0], ((ot >> 1) - 1) & 1u, ot)) break;
-        if (!issue_pv(od0, s0, pad0 / 16, false)) break;
-        if (!mw(&B.snap_ready, nb & 1u, nb)) break;
-        issue_qs(od0, s0);
-        mma_commit(&B.o_full[s0]);
-        mma_commit(&B.q_empty[s0]);
+        if (!mw(&B.xf_k[s0], ph0, ot) || !mw(&B.qt_ready[s0], ph0, ot)) break;
+        issue_p(s0, s0, static_cast<uint32_t>(pad0));                                   // A
+        if (!mw(&B.full_v[s0], ph0, ot)) break;
+        if (ot >= 1 && !mw(&B.o_empty, (ot - 1) & 1u, ot)) break;
+        if (!issue_pv(s0, pad0 / 16, false)) break;                                     // PV_A
         if (n > 1) {
-          // job B: Q1 K0^T (dense) -> PV into accumulator s1, then Q1 S_{b-1}
-          if (!mw(&B.xf_q[s1], ph1, ot + 1)) break;
-          if (!issue_p(s1, s0, 128u)) break;
-          if (ot + 1 >= 2 && !mw(&B.o_empty[s1], (((ot + 1) >> 1) - 1) & 1u, ot + 1)) break;
-          if (!issue_pv(od1, s0, 8, false)) break;
-          issue_qs(od1, s1);
-          // state update over tile 0's and tile 1's keys
-          if (!mw(&B.s_ready, nb & 1u, nb)) break;
-          issue_su(s0, pad0 / 16);
-          mma_commit(&B.kv_empty[s0]);   // tile 0's keys and values: A, B, S all issued
-          if (!mw(&B.xf_kv[s1], ph1, ot + 1)) break;
-          issue_su(s1, pad1 / 16);
-          mma_commit(&B.su_done);
-          // job C: Q1 K1^T (masked) -> PV into accumulator s1
-          if (!issue_p(s1, s1, static_cast<uint32_t>(pad1))) break;
-          if (!issue_pv(od1, s1, pad1 / 16, true)) break;
-          mma_commit(&B.o_full[s1]);
-          mma_commit(&B.q_empty[s1]);
-          mma_commit(&B.kv_empty[s1]);
-        } else {
-          if (!mw(&B.s_ready, nb & 1u, nb)) break;
-          issue_su(s0, pad0 / 16);
-          mma_commit(&B.su_done);
-          mma_commit(&B.kv_empty[s0]);
+          if (!mw(&B.qt_ready[s1], ph1, ot + 1)) break;
+          issue_p(s1, s0, 128u);                                                         // B
         }
+        if (!mw(&B.snap_ready, nb & 1u, nb)) break;
+        issue_qs(s0);
+        mma_commit(&B.o_full);
+        mma_commit(&B.qt_free[s0]);
+        if (!mw(&B.s_ready, nb & 1u, nb)) break;
+        issue_su(s0, pad0 / 16);
+        mma_commit(&B.k_empty[s0]);
+        if (n > 1) {
+          if (!mw(&B.o_empty, ot & 1u, ot + 1)) break;   // the drain warps have read tile 0
+          if (!issue_pv(s0, 8, false)) break;                                           // PV_B
+          mma_commit(&B.v_empty[s0]);
+          if (!mw(&B.xf_k[s1], ph1, ot + 1)) break;
+          issue_p(s1, s1, static_cast<uint32_t>(pad1));                                 // C
+          if (!mw(&B.full_v[s1], ph1, ot + 1)) break;
+          issue_su(s1, pad1 / 16);
+          mma_commit(&B.k_empty[s1]);
+          if (!issue_pv(s1, pad1 / 16, true)) break;                                    // PV_C
+          mma_commit(&B.v_empty[s1]);
+          issue_qs(s1);
+          mma_commit(&B.o_full);
+          mma_commit(&B.qt_free[s1]);
+        } else {
+          mma_commit(&B.v_empty[s0]);
+        }
+        mma_commit(&B.su_done);
         ot += n;
         ++nb;
       }
-      (void)ok;
       // Drain: all MMAs complete before TMEM is released.
       mma_commit(&B.final_bar);
       tcu::drain(&B.final_bar, 0);
     }
   }
   // ------------------------------------------------------------------------------------
-  // Warps 2, 3, 8-15: SiLU of this CTA's K and Q tiles in place, in the order the MMAs need them
-  // (K0, Q0, Q1, K1 of each block); tail rows of K and V zeroed.
+  // Warps 2, 3, 24-31: SiLU of this CTA's K tiles in place (tail rows of K zeroed, and of V once it
+  // has landed).
   // ------------------------------------------------------------------------------------
-  else if (warp == 2 || warp == 3 || (warp >= 8 && warp < 16)) {
-    const int wt = warp < 4 ? tid - 64 : tid - 192;   // 0..63, then 64..319
+  else if (warp == 2 || warp == 3 || warp >= kXfWarp1) {
+    const int wt = warp < kXfWarp1 ? tid - 64 : tid - 32 * kXfWarp1 + 64;
     const bool silu = !p.phi_identity;
     uint32_t ot = 0;
     BlkIter it;
     blk_first<tpb>(p, it, wk);
-    auto do_k = [&](uint32_t t, int vr) -> bool {
-      const uint32_t sl = t & 1u;
-      if (!tcu::wait_warp(&B.full_kv[sl], (t >> 1) & 1u, abort_flag, err, SITE_TC_TRANSFORM, t)) return false;
-      xf_tile(sbase + OFF_K + sl * kTileBytes, vr, silu, wt);
-      if (vr < kTile) zero_tail(sbase + OFF_V + sl * kTileBytes, vr, wt);
-      fence_proxy_async_smem();
-      mbar_arrive(&B.xf_kv[sl]);
-      return true;
-    };
-    auto do_q = [&](uint32_t t) -> bool {
-      const uint32_t sl = t & 1u;
-      if (!tcu::wait_warp(&B.full_q[sl], (t >> 1) & 1u, abort_flag, err, SITE_TC_TRANSFORM, t)) return false;
-      xf_tile(sbase + OFF_Q + sl * kTileBytes, kTile, silu, wt);
-      fence_proxy_async_smem();
-      mbar_arrive(&B.xf_q[sl]);
-      return true;
-    };
     for (; it.valid; blk_next<tpb>(p, it, wk)) {
       int vr0, vr1;
       const int n = blk_tiles<tpb>(it, vr0, vr1);
-      if (!do_k(ot, vr0) || !do_q(ot)) break;
-      if (n > 1 && (!do_q(ot + 1) || !do_k(ot + 1, vr1))) break;
+      bool ok = true;
+      for (int u = 0; u < n && ok; ++u) {
+        const uint32_t t = ot + u, sl = t & 1u;
+        const int vr = u == 0 ? vr0 : vr1;
+        ok = tcu::wait_warp(&B.full_k[sl], (t >> 1) & 1u, abort_flag, err, SITE_TC_TRANSFORM, t);
+        if (!ok) break;
+        xf_tile(sbase + OFF_K + sl * kTileBytes, vr, silu, wt);
+        if (vr < kTile) {
+          ok = tcu::wait_warp(&B.full_v[sl], (t >> 1) & 1u, abort_flag, err, SITE_TC_TRANSFORM, t);
+          if (!ok) break;
+          zero_tail(sbase + OFF_V + sl * kTileBytes, vr, wt);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&B.xf_k[sl]);
+      }
+      if (!ok) break;
       ot += n;
     }
   }
   // ------------------------------------------------------------------------------------
-  // Warps 4-7 (one per TMEM lane quarter; thread r owns row r of every TMEM tile):
-  //  * score conversion (fp32 -> masked bf16 in place), job by job;
-  //  * the state: S0 into TMEM and the bf16 snapshot at a sequence start; after each
-  //    block's state update, S_b once: into the snapshot for the next block's inter
-  //    products, or to state_out after the sequence's last block;
-  //  * norm modes: each tile's sums of squares over the head's 128 columns of a row, added
-  //    into the fp64 per-token total, then one arrival per warp on the tile's counter.
-  // Per block: conversions A and B, the sums of tile 0, conversion C, the state, the sums of
-  // tile 1 -- the order in which the MMA warp makes them ready.
+  // Warps 8-11: SiLU of this CTA's Q tiles into TMEM (the A operand of the score and inter
+  // MMAs); thread r converts row r of the tile (16 swizzled 16-byte chunks) and writes its
+  // 64 columns of bf16 pairs.  The landing slot is free once read.
+  // ------------------------------------------------------------------------------------
+  else if (warp >= kQxfWarp0 && warp < kQxfWarp0 + 4) {
+    const int r = tid - 32 * kQxfWarp0;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(r & ~31) << 16) + TM_Q;
+    const bool silu = !p.phi_identity;
+    uint32_t ot = 0;
+    BlkIter it;
+    blk_first<tpb>(p, it, wk);
+    bool ok = true;
+    for (; it.valid && ok; blk_next<tpb>(p, it, wk)) {
+      int vr0, vr1;
+      const int n = blk_tiles<tpb>(it, vr0, vr1);
+      for (int u = 0; u < n; ++u) {
+        const uint32_t t = ot + u, sl = t & 1u;   // landing slot and phi(Q) tile in TMEM
+        if (!tcu::wait_warp(&B.full_q[sl], (t >> 1) & 1u, abort_flag, err, SITE_TC_TRANSFORM, t) ||
+            (t >= 2 && !tcu::wait_warp(&B.qt_free[sl], ((t >> 1) - 1) & 1u, abort_flag, err, SITE_TC_TRANSFORM, t))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t src = sbase + OFF_Q + sl * kTileBytes;
+#pragma unroll 1
+        for (int g = 0; g < 4; ++g) {   // 32 columns of d_k: chunks 4g .. 4g + 3 of the row
+          uint32_t x[16];
+#pragma unroll
+          for (int m4 = 0; m4 < 4; ++m4) {
+            const int m = 4 * g + m4;   // 8-column chunk of the row (box m / 8)
+            uint4 v = lds128(src + (m >> 3) * kBoxBytes + sw128_offset(r, m & 7));
+            if (silu) v = tcu::silu8(v);
+            x[4 * m4] = v.x; x[4 * m4 + 1] = v.y; x[4 * m4 + 2] = v.z; x[4 * m4 + 3] = v.w;
+          }
+          tmem_st16(tq + 64 * sl + 16 * g, x);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if ((r & 31) == 0) {
+          mbar_arrive(&B.q_empty[sl]);
+          mbar_arrive(&B.qt_ready[sl]);
+        }
+      }
+      ot += n;
+    }
+  }
+  // ------------------------------------------------------------------------------------
+  // Warps 4-7: score conversion (fp32 -> masked bf16 in place in TMEM), job by job; thread
+  // r owns row r of the score tile.
   // ------------------------------------------------------------------------------------
   else if (warp >= kConvWarp0 && warp < kConvWarp0 + 4) {
-    const int r = tid - 32 * kConvWarp0;           // TMEM lane: row of a tile, or d_k row of S
-    const uint32_t lane_off = static_cast<uint32_t>(r & ~31) << 16;
-    const uint32_t tP = tmem + lane_off + TM_P;
-    const uint32_t tS = tmem + lane_off + TM_S;
-    const uint32_t snap = sbase + OFF_SNAP;
-    const bool skip_publish = (err->inject == INJECT_SKIP_PUBLISH) && blockIdx.x == 0;
-    uint32_t jb = 0, nb = 0, ot = 0;
+    const int r = tid - 32 * kConvWarp0;
+    const uint32_t lane_t = tmem + (static_cast<uint32_t>(r & ~31) << 16);
+    uint32_t uc = 0;   // score jobs converted
     bool ok = true;
     auto conv = [&](int ncols, bool diag) -> bool {
-      if (!tcu::wait_warp(&B.p_full, jb & 1u, abort_flag, err, SITE_TC_CONVERT, jb)) return false;
+      const uint32_t tP = lane_t + TM_P;
+      if (!tcu::wait_warp(&B.p_full, uc & 1u, abort_flag, err, SITE_TC_CONVERT, uc)) return false;
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < ncols / 16; ++c) {
-        uint32_t x[16];
-        tmem_ld16(tP + 16 * c, x);
+      for (int c = 0; c < ncols / 32; ++c) {
+        uint32_t x[32];
+        tmem_ld32(tP + 32 * c, x);
         tmem_ld_wait();
-        uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int j = 16 * c + 2 * e;
-          float a = __uint_as_float(x[2 * e]), b = __uint_as_float(x[2 * e + 1]);
-          if (diag) {   // keys up to the query row
-            a = (j <= r) ? a : 0.f;
-            b = (j + 1 <= r) ? b : 0.f;
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int j = 32 * c + 16 * hh + 2 * e;
+            float a = __uint_as_float(x[16 * hh + 2 * e]), b = __uint_as_float(x[16 * hh + 2 * e + 1]);
+            if (diag) {   // keys up to the query row
+              a = (j <= r) ? a : 0.f;
+              b = (j + 1 <= r) ? b : 0.f;
+            }
+            pk[e] = pack_bf16x2(a, b);
           }
-          pk[e] = pack_bf16x2(a, b);
+          tmem_st8(tP + 16 * c + 8 * hh, pk);
         }
-        tmem_st8(tP + 8 * c, pk);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&B.p_conv);
-      ++jb;
+      ++uc;
       return true;
     };
-    // Sum of squares of row r of own tile t (tile i of sequence s, rows from row0).
-    auto publish = [&](uint32_t t, const BlkIter& bi, int u, int vr) -> bool {
-      const uint32_t sa = t & 1u;
-      if (!tcu::wait_warp(&B.o_full[sa], (t >> 1) & 1u, abort_flag, err, SITE_TC_EPILOGUE, t)) return false;
+    BlkIter it;
+    blk_first<tpb>(p, it, wk);
+    for (; it.valid && ok; blk_next<tpb>(p, it, wk)) {
+      int vr0, vr1;
+      const int n = blk_tiles<tpb>(it, vr0, vr1);
+      // jobs A (tile 0, masked), then for two tiles B (dense) and C (tile 1, masked)
+#pragma unroll 1
+      for (int j = 0; j < 2 * n - 1 && ok; ++j) ok = conv(j == 0 ? pad_rows(vr0) : (j == 1 ? 128 : pad_rows(vr1)), j != 1);
+    }
+  }
+  // ------------------------------------------------------------------------------------
+  // Warps 12-15 (one per TMEM lane quarter; thread r owns row r of every TMEM tile):
+  //  * the state: S0 into TMEM and the bf16 snapshot at a sequence start; after each
+  //    block's state update, S_b once: into the snapshot for the next block's inter
+  //    products, or to state_out after the sequence's last block;
+  //  * the output accumulators: each tile's rows read once and written out (y, or z for the
+  //    final warps to rescale), and in the norm modes the rows' sums of squares published.
+  // Per block: tile 0 (read, then published), tile 1 (read), the state, tile 1's sums -- the
+  // order in which the MMA warp makes them ready, reads that free the accumulator first.
+  // ------------------------------------------------------------------------------------
+  else if (warp >= kStateWarp0 && warp < kStateWarp0 + 4) {
+    const int r = tid - 32 * kStateWarp0;          // TMEM lane: row of a tile, or d_k row of S
+    const uint32_t lane_off = static_cast<uint32_t>(r & ~31) << 16;
+    const uint32_t tS = tmem + lane_off + TM_S;
+    const uint32_t snap = sbase + OFF_SNAP;
+    const bool skip_publish = (err->inject == INJECT_SKIP_PUBLISH) && blockIdx.x == 0;
+    uint32_t nb = 0, ot = 0;
+    bool ok = true;
+    // Drain own tile t (tile i of the block's sequence): read row r of the accumulator once,
+    // free it, and write the row to the output -- y in raw mode, z = bf16(y w) in the norm
+    // modes, where the final warps rescale it in place -- then publish the row's sum of
+    // squares (fp64 add into the token's total, fence, one arrival per warp).
+    const int64_t HD = static_cast<int64_t>(p.H) * kD;
+    // drain() reads tile t's row r and frees the accumulator; publish() then adds the row's
+    // sum of squares (kept in ss_row) and makes the warp's arrival.
+    float ss_row = 0.f;
+    auto drain = [&](uint32_t t, const BlkIter& bi, int u, int vr) -> bool {
+      if (!tcu::wait_warp(&B.o_full, t & 1u, abort_flag, err, SITE_TC_EPILOGUE, t)) return false;
       tc_fence_after();
+      const int i = bi.jb * tpb + u;
+      const int64_t row = bi.row0 + static_cast<int64_t>(i) * kTile + r;
+      const bool valid = r < vr;
+      uint16_t* dst = p.out + row * HD + h * kD;
       float ss = 0.f;
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         uint32_t x[16];
-        tmem_ld16(tmem + lane_off + TM_O + 128 * sa + 16 * c, x);
+        tmem_ld16(tmem + lane_off + TM_O + 16 * c, x);
         tmem_ld_wait();
+        uint32_t z[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) ss = fmaf(__uint_as_float(x[e]), __uint_as_float(x[e]), ss);
+        for (int e = 0; e < 8; ++e) {
+          float a = __uint_as_float(x[2 * e]), b = __uint_as_float(x[2 * e + 1]);
+          ss = fmaf(a, a, ss);
+          ss = fmaf(b, b, ss);
+          if (norm) {
+            a *= B.w[16 * c + 2 * e];
+            b *= B.w[16 * c + 2 * e + 1];
+          }
+          z[e] = pack_bf16x2(a, b);
+        }
+        if (valid) tcu::st_na_v8(dst + 16 * c, z);
       }
       tc_fence_before();
+      __syncwarp();
+      if ((r & 31) == 0) mbar_arrive(&B.o_empty);   // done reading the accumulator
+      ss_row = ss;
+      return true;
+    };
+    auto publish = [&](const BlkIter& bi, int u, int vr) {
+      if (!norm) return;
       const int i = bi.jb * tpb + u;
-      if (r < vr) tcu::red_add_f64(p.ss + bi.row0 + static_cast<int64_t>(i) * kTile + r, static_cast<double>(ss));
+      const int64_t row = bi.row0 + static_cast<int64_t>(i) * kTile + r;
+      if (r < vr) tcu::red_add_f64(p.ss + row * kSsStride, static_cast<double>(ss_row));
       tcu::fence_acq_rel_gpu();
       __syncwarp();
       if ((r & 31) == 0 && !skip_publish)
-        tcu::red_add_relaxed_u32(p.cnt + static_cast<int64_t>(bi.s) * p.max_tiles + i, 1u);
-      return true;
+        tcu::red_add_relaxed_u32(p.cnt + (static_cast<int64_t>(bi.s) * p.max_tiles + i) * kCntStride, 1u);
     };
     // Columns 16c .. 16c + 15 of row r of S into the snapshot (two 16-byte bf16 chunks).
     auto snap16 = [&](int c, const uint32_t (&x)[16]) {
@@ -672,10 +780,9 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
         mbar_arrive(&B.snap_ready);
         mbar_arrive(&B.s_ready);
       }
-      if (!conv(pad_rows(vr0), true)) break;
-      if (n > 1 && !conv(128, false)) break;
-      if (norm && !publish(ot, it, 0, vr0)) break;
-      if (n > 1 && !conv(pad_rows(vr1), true)) break;
+      if (!drain(ot, it, 0, vr0)) break;
+      publish(it, 0, vr0);
+      if (n > 1 && !drain(ot + 1, it, 1, vr1)) break;
       // S_b, once the block's state update is done
       if (!tcu::wait_warp(&B.su_done, nb & 1u, abort_flag, err, SITE_TC_EPILOGUE, nb)) break;
       tc_fence_after();
@@ -702,25 +809,23 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
         mbar_arrive(&B.s_ready);
       }
       ++nb;
-      if (norm && n > 1 && !publish(ot + 1, it, 1, vr1)) break;
+      if (n > 1) publish(it, 1, vr1);
       ot += n;
     }
   }
   // ------------------------------------------------------------------------------------
-  // Warps 16-23: output stores.  Warp e owns TMEM lane quarter e % 4 (32 rows of every
-  // tile) and columns 64 * (e / 4 - 4) .. +63 of the head.  Raw mode stores y.  The norm
-  // modes wait until every head has published the tile's sums, then store
-  // o = bf16(y w) rsqrt(mean(y^2) + eps) [sigmoid(g)], 32 bytes per access; the
-  // accumulator is freed after its last read.
+  // Warps 16-23 (norm modes): the normalised output.  Once every head has published a
+  // tile's sums, its rows (z = bf16(y w), written by the drain warps) are rescaled in place:
+  // o = z rsqrt(mean(y^2) + eps) [sigmoid(g)].  No TMEM access: warp e takes rows
+  // 16e .. 16e + 15 of the tile, each half-warp one row's 256 bytes of this head per step,
+  // so every access is a full 512-byte line pair.
   // ------------------------------------------------------------------------------------
-  else if (warp >= kEpiWarp0) {
-    const int q = warp & 3;
-    const int half = (warp - kEpiWarp0) >> 2;
-    const int rr = 32 * q + lane;                     // row of the tile
-    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+  else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiWarps && norm) {
+    const int e = warp - kEpiWarp0;
+    const int half = lane >> 4;                       // which row of the pair
+    const int cl = (lane & 15) * 8;                   // this lane's 8 columns of the head
     const int64_t HD = static_cast<int64_t>(p.H) * kD;
     const float inv_hd = 1.0f / static_cast<float>(HD);
-    const int col0 = h * kD + 64 * half;
     uint32_t ot = 0;
     bool ok = true;
     BlkIter it;
@@ -729,72 +834,55 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
       int vr0, vr1;
       const int n = blk_tiles<tpb>(it, vr0, vr1);
       for (int u = 0; u < n && ok; ++u, ++ot) {
-        const uint32_t sa = ot & 1u;
         const int i = it.jb * tpb + u;                 // tile of the sequence
         const int vr = u == 0 ? vr0 : vr1;
-        const int64_t row = it.row0 + static_cast<int64_t>(i) * kTile + rr;
-        const bool valid = rr < vr;
-        uint16_t* dst = p.out + row * HD + col0;
-        const uint32_t oacc = tmem + lane_off + TM_O + 128 * sa + 64 * half;
-        float rn = 1.f;
-        uint32_t g0[8], g1[8];   // gate values of columns 0..15 and 16..31 of the current 32
-        if (norm) {
-          const uint16_t* gsrc = p.g + row * HD + col0;
-          if (gate && valid) {   // in flight during the waits
-            tcu::ld_nc_v8(gsrc, g0);
-            tcu::ld_nc_v8(gsrc + 16, g1);
-          }
-          unsigned int* cnt = p.cnt + static_cast<int64_t>(it.s) * p.max_tiles + i;
-          int go = 1;
-          if (lane == 0 && ld_acquire_gpu(cnt) < W)
-            go = tcu::poll_count(cnt, W, abort_flag, err, static_cast<uint32_t>(it.s * p.max_tiles + i)) ? 1 : 0;
-          if (!__shfl_sync(0xFFFFFFFFu, go, 0)) {
-            ok = false;
-            break;
-          }
-          (void)ld_acquire_gpu(cnt);
-          if (valid) rn = 1.0f / sqrtf(static_cast<float>(tcu::ld_cg_f64(p.ss + row)) * inv_hd + p.eps);
-        }
-        // The counter covers the accumulator's completion (its publisher waited for it); the
-        // wait here orders this warp's TMEM reads after the MMAs.
-        if (!tcu::wait_warp(&B.o_full[sa], (ot >> 1) & 1u, abort_flag, err, SITE_TC_EPILOGUE, ot)) {
+        unsigned int* cnt = p.cnt + (static_cast<int64_t>(it.s) * p.max_tiles + i) * kCntStride;
+        int go = 1;
+        if (lane == 0 && ld_acquire_gpu(cnt) < W)
+          go = tcu::poll_count(cnt, W, abort_flag, err, static_cast<uint32_t>(it.s * p.max_tiles + i)) ? 1 : 0;
+        if (!__shfl_sync(0xFFFFFFFFu, go, 0)) {
           ok = false;
           break;
         }
-        tc_fence_after();
+        (void)ld_acquire_gpu(cnt);
+        const int64_t base = it.row0 + static_cast<int64_t>(i) * kTile;
+        // Lane l holds the norm factor of row 16e + (l & 15).
+        const int myrt = 16 * e + (lane & 15);
+        const double myss = myrt < vr ? tcu::ld_cg_f64(p.ss + (base + myrt) * kSsStride) : 0.0;
+        const float myrn = 1.0f / sqrtf(static_cast<float>(myss) * inv_hd + p.eps);
+        const uint16_t* zrow = p.out + (base + 16 * e + half) * HD + h * kD + cl;   // row pair 0
+        const uint16_t* grow = gate ? p.g + (base + 16 * e + half) * HD + h * kD + cl : nullptr;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {   // 16 columns at a time
-          if (gate && valid && c == 2) {
-            tcu::ld_nc_v8(p.g + row * HD + col0 + 32, g0);
-            tcu::ld_nc_v8(p.g + row * HD + col0 + 48, g1);
-          }
-          uint32_t x[16];
-          tmem_ld16(oacc + 16 * c, x);
-          tmem_ld_wait();
-          if (c == 3) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&B.o_empty[sa]);
-          }
-          uint32_t o[8];
+        for (int k0 = 0; k0 < 8; k0 += 2) {           // 2 row pairs at a time
+          uint4 zv[2], gv[2];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int col = 64 * half + 16 * c + 2 * e;
-            float a = __uint_as_float(x[2 * e]), b = __uint_as_float(x[2 * e + 1]);
-            if (norm) {
-              // z = bf16(y w): the unnormalised output is rounded before the scale
-              const uint32_t zz = pack_bf16x2(a * B.w[col], b * B.w[col + 1]);
-              a = __uint_as_float(zz << 16) * rn;
-              b = __uint_as_float(zz & 0xFFFF0000u) * rn;
-              if (gate) {
-                const uint32_t gg = (c & 1) ? g1[e] : g0[e];
-                a *= sigmoid_fast(__uint_as_float(gg << 16));
-                b *= sigmoid_fast(__uint_as_float(gg & 0xFFFF0000u));
-              }
-            }
-            o[e] = pack_bf16x2(a, b);
+          for (int k = 0; k < 2; ++k) {
+            const int rt = 16 * e + 2 * (k0 + k) + half;   // row of the tile
+            const bool valid = rt < vr;
+            const int64_t off = static_cast<int64_t>(2 * (k0 + k)) * HD;
+            zv[k] = valid ? tcu::ld_cg_u4(zrow + off) : make_uint4(0, 0, 0, 0);
+            gv[k] = (gate && valid) ? tcu::ld_nc_u4(grow + off) : make_uint4(0, 0, 0, 0);
           }
-          if (valid) tcu::st_na_v8(dst + 16 * c, o);
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int rt = 16 * e + 2 * (k0 + k) + half;
+            const float rn = __shfl_sync(0xFFFFFFFFu, myrn, 2 * (k0 + k) + half);
+            if (rt >= vr) continue;
+            const uint32_t zw[4] = {zv[k].x, zv[k].y, zv[k].z, zv[k].w};
+            const uint32_t gw[4] = {gv[k].x, gv[k].y, gv[k].z, gv[k].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float a = __uint_as_float(zw[q] << 16) * rn, b = __uint_as_float(zw[q] & 0xFFFF0000u) * rn;
+              if (gate) {
+                a *= sigmoid_fast(__uint_as_float(gw[q] << 16));
+                b *= sigmoid_fast(__uint_as_float(gw[q] & 0xFFFF0000u));
+              }
+              o[q] = pack_bf16x2(a, b);
+            }
+            tcu::st_global_na(const_cast<uint16_t*>(zrow) + static_cast<int64_t>(2 * (k0 + k)) * HD,
+                              make_uint4(o[0], o[1], o[2], o[3]));
+          }
         }
       }
     }
@@ -980,16 +1068,17 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
 size_t pair_workspace_bytes(int nseq, int max_len, int64_t tokens, int H) {
   const size_t max_tiles = (static_cast<size_t>(max_len) + kTile - 1) / kTile;
   const size_t nw = 2 * static_cast<size_t>(pair_groups(nseq, H));
-  return up256(sizeof(unsigned int) * static_cast<size_t>(nseq) * (max_tiles ? max_tiles : 1)) +
-         up256(sizeof(double) * static_cast<size_t>(tokens > 0 ? tokens : 1)) +
+  return up256(sizeof(unsigned int) * kCntStride * static_cast<size_t>(nseq) * (max_tiles ? max_tiles : 1)) +
+         up256(sizeof(double) * kSsStride * static_cast<size_t>(tokens > 0 ? tokens : 1)) +
          up256(sizeof(int) * static_cast<size_t>(nseq)) + up256(sizeof(int) * (nw + 1));
 }
 
 cudaError_t launch_pair_prefill(const TcArgs& a, cudaStream_t stream) {
   if (a.reverse || a.D != kD || (a.C != 128 && a.C != 256)) return cudaErrorInvalidValue;
   const int max_tiles = (a.max_len + kTile - 1) / kTile;
-  const size_t cnt_bytes = up256(sizeof(unsigned int) * static_cast<size_t>(a.nseq) * (max_tiles ? max_tiles : 1));
-  const size_t ss_bytes = up256(sizeof(double) * static_cast<size_t>(a.tokens > 0 ? a.tokens : 1));
+  const size_t cnt_bytes =
+      up256(sizeof(unsigned int) * kCntStride * static_cast<size_t>(a.nseq) * (max_tiles ? max_tiles : 1));
+  const size_t ss_bytes = up256(sizeof(double) * kSsStride * static_cast<size_t>(a.tokens > 0 ? a.tokens : 1));
   const size_t sched_bytes = up256(sizeof(int) * static_cast<size_t>(a.nseq));
   PairParams p{};
   p.state_in = a.state_in;
