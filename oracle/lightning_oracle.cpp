@@ -15,7 +15,7 @@
 //   [Ops]    "MiniMax-01技术报告解读（二）计算优化", section 3: lightning_attention_chunk_size 256 and
 //            lightning_attention_pad_options [32, 64, 128] (block size and tail padding).
 //
-// Readings taken where the pages are silent or disagree (each is listed in the design doc):
+// Readings taken where the pages are silent or disagree (each is listed with the design notes):
 //   * phi = SiLU on q and k only; v is used raw (the workload statement applies SiLU to Q, K).
 //   * No normaliser z and no denominator: [Arch] feeds Y straight into RMSNorm.
 //   * No decay factor and no 1/sqrt(d) scaling (neither appears in the linear form).
