@@ -120,15 +120,15 @@ def _flops_per_token(H, D, C):
     algorithmic: 2 d (C + 1) for the masked intra block (averaged over a block) plus 4 d^2
     for the inter read phi(q)^T S and the state carry phi(k) v^T.
     issued by the tensor-core kernel: 128-row tiles; a query tile multiplies by the key
-    tiles of its block up to the diagonal (the zero quarter of a 256-block is skipped),
-    and the two CTAs of a head (64 columns of d_v each) both compute the scores.
+    tiles of its block up to the diagonal (the zero quarter of a 256-block is skipped);
+    each CTA computes a head's full width, so every score is computed once.  The chunk-state
+    pass that lets a long sequence run as parallel chunks is not counted.
     """
     algo = H * (2 * D * (C + 1) + 4 * D * D)
     tiles = C // 128
     keys = 128 * (tiles + 1) / 2          # mean keys per query row multiplied
-    n_dv = 2
-    issued = H * (2 * keys * D * n_dv     # P = phi(Q) phi(K)^T, once per d_v slice
-                  + 2 * keys * D          # O += P V over both slices
+    issued = H * (2 * keys * D            # P = phi(Q) phi(K)^T
+                  + 2 * keys * D          # O += P V
                   + 2 * D * D             # O += phi(Q) S
                   + 2 * D * D)            # S += phi(K)^T V
     return algo, issued
@@ -172,6 +172,12 @@ class PrefillCase:
     def step(self):
         self.la.lightning_attn_prefill(self.q, self.k, self.v, self.g, self.out, None, self.state,
                                        block_size=self.C, workspace=self.ws)
+
+    @property
+    def launches_per_step(self):
+        # a sequence run as parallel chunks: chunk bounds, chunk states, their split sum, the
+        # prefix of initial states and the prefill kernel; else the prefill kernel alone
+        return 5 if self.la.lightning_attn_last_path().endswith("+chunks") else 1
 
     def enable_host_pipeline(self, chunk_tokens):
         """e2e through HostPrefill: the copies in and out overlapped over chunks of the sequence."""
@@ -283,6 +289,8 @@ class VarlenCase:
     """16 packed sequences (lengths ~ U{1000..32768}), cu_seqlens on the device, block 256
     with 32/64/128 tail pads, gated concat RMSNorm, per-sequence final states."""
 
+    launches_per_step = 2   # the longest-first work plan and the prefill kernel
+
     def __init__(self, name, w, device, rank):
         import torch
         from long_context_attn_b200 import lightning_attn as la
@@ -365,6 +373,8 @@ class VarlenCase:
 class ZnormCase(PrefillCase):
     """The normalised variant over the 128K prefill's shapes (q, k shifted so phi(q) . z > 0)."""
 
+    launches_per_step = 5   # raw prefill, phi(k) chunk sums, their prefix, denominators, transform
+
     def __init__(self, name, w, device, rank):
         super().__init__(name, w, device, rank)
         import torch
@@ -380,7 +390,6 @@ class ZnormCase(PrefillCase):
         self.ws = self.la.new_workspace(nbytes, device)
         self.alg_bytes += H * D * 4
         self.d2h += H * D * 4
-        self.launches_per_step = 5      # raw prefill, phi(k) chunk sums, their prefix, denominators, transform
 
     def step(self):
         self.la.lightning_attn_prefill_znorm(self.q, self.k, self.v, self.g, self.out, None, None, self.state, self.z,
@@ -401,6 +410,49 @@ class ZnormCase(PrefillCase):
 
     def describe(self):
         return dict(super().describe(), variant="normalised (z-denominator)", qk_shift=self.w.qk_shift)
+
+
+class TinyCase:
+    """The small fp32 check: 1 x 512 tokens x 2 heads x d 64, block 64, raw output.  Its
+    inputs fit in L2, so each timed step follows a write of a buffer larger than L2 and is
+    timed alone."""
+
+    def __init__(self, name, w, device, rank):
+        import torch
+        from long_context_attn_b200 import lightning_attn as la
+        self.la, self.w = la, w
+        T, H, D = w.T, w.H, w.D
+        q, k, v, _ = synth.prefill_inputs(w.seed + 1000 * rank, T, H, D, "f32", w.qkv_scale, False)
+        self.q, self.k, self.v = (torch.from_numpy(a).to(device).view(1, T, H, D) for a in (q, k, v))
+        self.out = torch.empty((1, T, H * D), dtype=torch.float32, device=device)
+        self.state = torch.empty((1, H, D, D), dtype=torch.float32, device=device)
+        self.ws = la.new_workspace(la.lightning_attn_workspace_size(la.LA_OP_PREFILL, 1, T, 0, H, D, w.block_size,
+                                                                    la.LA_F32, la.LA_OUT_RAW), device)
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        self.tokens = T
+        self.alg_bytes = T * 4 * H * D * 4 + H * D * D * 4   # q, k, v read + out written, fp32; the state
+        self.alg_flops, self.issued_flops = (x * T for x in _flops_per_token(H, D, w.block_size))
+        self.launches_per_step = 1
+
+    def step(self):
+        self.la.lightning_attn_prefill(self.q, self.k, self.v, None, self.out, None, self.state,
+                                       block_size=self.w.block_size, mode=self.la.LA_OUT_RAW, workspace=self.ws)
+
+    def check(self):
+        self.la.lightning_attn_check(self.ws)
+
+    def oracle_sample(self):
+        import oracle
+        w = self.w
+        q, k, v, _ = synth.prefill_inputs(w.seed, w.T, w.H, w.D, "f32", w.qkv_scale, False)
+        t0 = time.perf_counter()
+        oracle.prefill(q[None], k[None], v[None], None, mode=oracle.MODE_RAW, store=False)
+        return time.perf_counter() - t0
+
+    def describe(self):
+        w = self.w
+        return {"workload": w.name, "B": 1, "T": w.T, "H": w.H, "D": w.D, "block_size": w.block_size,
+                "dtype": "f32", "mode": "raw", "l2": "inputs fit in L2: a 256 MiB write before each timed step"}
 
 
 class ChunkStateCase:
@@ -689,6 +741,8 @@ def _make_case(name, device, rank):
         return ZnormCase(name, w, device, rank)
     if w.kind == "chunk_state":
         return ChunkStateCase(name, w, device, rank)
+    if w.kind == "prefill" and w.dtype == "f32":
+        return TinyCase(name, w, device, rank)
     raise SystemExit(f"workload {name} is not a bench workload")
 
 
@@ -821,6 +875,11 @@ def run_gpu(args):
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = _cpu_baseline(case)
+        if world == 1 and args.workload == "prefill_128k" and not args.no_secondary:
+            del case
+            torch.cuda.empty_cache()
+            for name in SECONDARY_STEPS:
+                line[name] = _measure_secondary(name, device, peaks)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -828,11 +887,65 @@ def run_gpu(args):
 
 HOLD_CYCLES = 4_000_000   # about 2 ms at the B200's 1965 MHz SM clock
 
+# The other configurations, measured in the same process after the headline (one GPU) and
+# reported as keys of the same line: steps timed per configuration.
+SECONDARY_STEPS = {"decode_256": 1000, "varlen_16": 10, "prefill_8k": 50, "tiny_f32": 200}
+
+
+def _measure_secondary(name, device, peaks):
+    """ms per step, tokens/s, the HBM roofline fraction and the clocks of one configuration."""
+    import torch
+    case = _make_case(name, device, 0)
+    steps = SECONDARY_STEPS[name]
+    for _ in range(3):
+        case.step()
+    case.check()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    per_step = isinstance(case, TinyCase)   # inputs inside L2: flush, then time each step alone
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        if per_step:
+            total = 0.0
+            for _ in range(steps):
+                case.flush.fill_(1)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                case.step()
+                b.record(stream)
+                torch.cuda.synchronize()
+                total += a.elapsed_time(b)
+            ms = total / steps
+        else:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda._sleep(HOLD_CYCLES)
+            a.record(stream)
+            for _ in range(steps):
+                case.step()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / steps
+    case.check()
+    gbs = case.alg_bytes / (ms / 1e3) / 1e9
+    out = {"ms_per_step": ms, "tokens_per_s": case.tokens / (ms / 1e3), "steps": steps,
+           "config": case.describe(),
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_step": case.alg_bytes},
+           "tensor": {"algorithmic_tflops": case.alg_flops / (ms / 1e3) / 1e12,
+                      "frac_algorithmic": case.alg_flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
+           "gpu_launches": steps * case.launches_per_step if hasattr(case, "launches_per_step") else steps,
+           "clocks": clk.summary()}
+    if hasattr(case, "lens"):
+        out["path"] = case.la.lightning_attn_last_path()
+    del case
+    torch.cuda.empty_cache()
+    return out
+
 # Source files each measured kernel is built from (a traffic figure is tied to their hash).
 KERNEL_SOURCES = {
-    "prefill": ("la_prefill_tc.cu", "la_sm100.cuh", "la_common.cuh"),
+    "prefill": ("la_prefill_pair.cu", "la_state_tc.cu", "la_tc_util.cuh", "la_sm100.cuh", "la_common.cuh"),
     "decode": ("la_decode.cu", "la_common.cuh"),
-    "backward": ("la_backward.cu", "la_api.cu", "la_prefill_tc.cu", "la_sm100.cuh", "la_common.cuh"),
+    "backward": ("la_backward.cu", "la_api.cu", "la_prefill_tc.cu", "la_prefill_pair.cu", "la_state_tc.cu",
+                 "la_tc_util.cuh", "la_sm100.cuh", "la_common.cuh"),
 }
 
 
@@ -873,6 +986,11 @@ def _cpu_baseline(case):
         return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
                 "sample": f"first {n} tokens of the {case.w.name} workload, all {case.H} heads, fp64, "
                           f"recurrence + norm + gate ({dt:.1f} s)"}
+    if isinstance(case, TinyCase):
+        dt = case.oracle_sample()
+        return {"value": case.tokens / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                "sample": f"the whole {case.w.name} workload ({case.tokens} tokens, {case.w.H} heads), fp64 raw "
+                          f"recurrence ({dt:.2f} s)"}
     if isinstance(case, MixedCase):
         dt = case.oracle_sample()
         return {"value": case.total / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
@@ -989,10 +1107,13 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="prefill_128k",
-                    choices=["prefill_8k", "prefill_128k", "varlen_16", "decode_256", "mixed_256", "backward_8k",
+                    choices=["prefill_8k", "prefill_32k", "prefill_128k", "varlen_16", "decode_256", "mixed_256",
+                             "backward_8k", "tiny_f32",
                              "backward_128k", "train_128k", "znorm_128k", "chunk_state_128k", "prefill_128k_h8"])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other configurations after the headline (profiling runs)")
     ap.add_argument("--e2e-chunk", type=int, default=0,
                     help="e2e through HostPrefill with chunks of this many tokens (0: copy in, step, copy out)")
     args = ap.parse_args()

@@ -1116,8 +1116,9 @@ cudaError_t launch_pair_prefill(const TcArgs& a, cudaStream_t stream) {
   // Arrival counters and the fp64 sums start at zero on every call.
   cudaError_t e = cudaMemsetAsync(a.ws, 0, cnt_bytes + (a.mode != LA_OUT_RAW ? ss_bytes : 0), stream);
   if (e != cudaSuccess) return e;
-  // Packed batches of several sequences: the longest-first worker plan.
-  if (a.cu && a.nseq > 1 && a.nseq <= kPlanMaxSeqs && nw <= 256) {
+  // Packed batches with more sequences than workers: the longest-first worker plan (with
+  // at most one sequence per worker the round-robin order is already that plan).
+  if (a.cu && a.nseq > nw && a.nseq <= kPlanMaxSeqs && nw <= 256) {
     int* sched = reinterpret_cast<int*>(a.ws + cnt_bytes + ss_bytes);
     int* wstart = reinterpret_cast<int*>(a.ws + cnt_bytes + ss_bytes + sched_bytes);
     plan_kernel<<<1, kPlanThreads, 0, stream>>>(a.cu, a.nseq, nw, a.skip_single, sched, wstart);

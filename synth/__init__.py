@@ -153,6 +153,9 @@ WORKLOADS = {
     # denominators phi(q) . z stay positive.
     "znorm_128k": Workload("znorm_128k", "znorm", 1009, 1, 131072, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5,
                            qk_shift=1.0),
+    # The 128K prefill's shapes at 32K tokens: inputs four times L2, small enough for DRAM
+    # counter captures of every kernel of one call.
+    "prefill_32k": Workload("prefill_32k", "prefill", 1013, 1, 32768, 64, 128, 256, "bf16", "rmsnorm_gate", 0.5),
     # One 128K sequence with 8 heads (a tensor-parallel shard of the 64): the few-heads case.
     "prefill_128k_h8": Workload("prefill_128k_h8", "prefill", 1012, 1, 131072, 8, 128, 256, "bf16", "rmsnorm_gate",
                                 0.5),

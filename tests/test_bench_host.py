@@ -14,8 +14,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def test_per_token_accounting():
     algo, issued = bench._flops_per_token(64, 128, 256)
     assert algo / 64 == 2 * 128 * 257 + 4 * 128 * 128 == 131328
-    # two d_v slices recompute the scores; a 256-block multiplies 192 keys per row on average
-    assert issued / 64 == 2 * 192 * 128 * 2 + 2 * 192 * 128 + 4 * 128 * 128
+    # scores once per head (full d_v per CTA); a 256-block multiplies 192 keys per row on average
+    assert issued / 64 == 2 * 192 * 128 + 2 * 192 * 128 + 4 * 128 * 128
     assert bench._bytes_per_token(64, 128) == 81920
 
 
