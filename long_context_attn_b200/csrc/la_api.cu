@@ -216,7 +216,7 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
     a.reverse = reverse ? 1 : 0;
     const bool fixed = !cu && T_fixed > 0;
     const SplitPlan sp = !fixed ? SplitPlan{1, T_fixed}
-                                : (reverse ? split_plan(nseq, T_fixed, H, D) : forward_split_plan(nseq, T_fixed, H, D, C));
+                                : forward_split_plan(nseq, T_fixed, H, D, C);
     if (sp.S > 1) {
       const SplitLayout sl = split_layout(sp, nseq, tokens, H, D, C);
       char* x = ws + sl.tc;

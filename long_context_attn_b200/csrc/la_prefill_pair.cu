@@ -233,13 +233,19 @@ __device__ __forceinline__ void blk_next(const PairParams& p, BlkIter& it, int w
   ++it.k;
   blk_seek<tpb>(p, it, w);
 }
+// The tile of a sequence that walk position i covers: time forwards walks tiles 0 .. nt - 1,
+// time backwards nt - 1 .. 0 (rows keep their order inside a tile).
+template <bool rev>
+__device__ __forceinline__ int phys_tile(int i, int nt) {
+  return rev ? nt - 1 - i : i;
+}
 // Tiles of the current block and the valid rows of each.
-template <int tpb>
+template <int tpb, bool rev>
 __device__ __forceinline__ int blk_tiles(const BlkIter& it, int& vr0, int& vr1) {
   const int t0 = it.jb * tpb;
   const int n = min(tpb, it.nt - t0);
-  vr0 = min(kTile, it.L - t0 * kTile);
-  vr1 = n > 1 ? min(kTile, it.L - (t0 + 1) * kTile) : 0;
+  vr0 = min(kTile, it.L - phys_tile<rev>(t0, it.nt) * kTile);
+  vr1 = n > 1 ? min(kTile, it.L - phys_tile<rev>(t0 + 1, it.nt) * kTile) : 0;
   return n;
 }
 
@@ -278,7 +284,7 @@ __device__ __forceinline__ void zero_tail(uint32_t base, int vr, int wt) {
 // ======================================================================================
 // The kernel (one instantiation per output mode and block size)
 // ======================================================================================
-template <int kMode, int kC>
+template <int kMode, int kC, bool kRev>
 __global__ void __launch_bounds__(kThreads, 1)
 lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -292,6 +298,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
   constexpr int tpb = kC / kTile;
   constexpr bool norm = kMode != LA_OUT_RAW;
   constexpr bool gate = kMode == LA_OUT_RMSNORM_GATE;
+  static_assert(!kRev || kMode == LA_OUT_RAW, "time runs backwards in the raw mode only");
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -362,7 +369,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
       blk_first<tpb>(p, it, wk);
       for (; it.valid && ok; blk_next<tpb>(p, it, wk)) {
         int vr0, vr1;
-        const int n = blk_tiles<tpb>(it, vr0, vr1);
+        const int n = blk_tiles<tpb, kRev>(it, vr0, vr1);
         for (int u = 0; u < n; ++u, ++ot) {
           if (norm && lane == 0) {
             unsigned int* c = hist[kThrottle - 1];
@@ -379,11 +386,14 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
             ok = false;
             break;
           }
-          const int32_t row = static_cast<int32_t>(it.row0 + static_cast<int64_t>(it.jb * tpb + u) * kTile);
+          const int wi = it.jb * tpb + u;   // walk position of the tile
+          const int32_t row = static_cast<int32_t>(it.row0 + static_cast<int64_t>(phys_tile<kRev>(wi, it.nt)) * kTile);
           const int32_t col = h * kD;
-          if ((it.jb * tpb + u + tpb) < it.nt) {
-            tma_prefetch_l2_2d(map, col, row + kC);
-            tma_prefetch_l2_2d(map, col + 64, row + kC);
+          if (wi + tpb < it.nt) {   // the same tile of the next block
+            const int32_t nrow =
+                static_cast<int32_t>(it.row0 + static_cast<int64_t>(phys_tile<kRev>(wi + tpb, it.nt)) * kTile);
+            tma_prefetch_l2_2d(map, col, nrow);
+            tma_prefetch_l2_2d(map, col + 64, nrow);
           }
           uint8_t* dst = smem + off + sl * kTileBytes;
           mbar_arrive_expect_tx(&full[sl], kTileBytes);
@@ -462,7 +472,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
       // after both inter products, so the snapshot area is free once the state warps see it.
       for (; it.valid && ok; blk_next<tpb>(p, it, wk)) {
         int vr0, vr1;
-        const int n = blk_tiles<tpb>(it, vr0, vr1);
+        const int n = blk_tiles<tpb, kRev>(it, vr0, vr1);
         const uint32_t s0 = ot & 1u, s1 = (ot + 1) & 1u;            // slots (and phi(Q) tiles)
         const uint32_t ph0 = (ot >> 1) & 1u, ph1 = ((ot + 1) >> 1) & 1u;
         const int pad0 = pad_rows(vr0), pad1 = n > 1 ? pad_rows(vr1) : 0;
@@ -473,7 +483,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
         if (!issue_pv(s0, pad0 / 16, false)) break;                                     // PV_A
         if (n > 1) {
           if (!mw(&B.qt_ready[s1], ph1, ot + 1)) break;
-          issue_p(s1, s0, 128u);                                                         // B
+          issue_p(s1, s0, static_cast<uint32_t>(pad0));                                 // B
         }
         if (!mw(&B.snap_ready, nb & 1u, nb)) break;
         issue_qs(s0);
@@ -484,7 +494,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
         mma_commit(&B.k_empty[s0]);
         if (n > 1) {
           if (!mw(&B.o_empty, ot & 1u, ot + 1)) break;   // the drain warps have read tile 0
-          if (!issue_pv(s0, 8, false)) break;                                           // PV_B
+          if (!issue_pv(s0, pad0 / 16, false)) break;                                   // PV_B
           mma_commit(&B.v_empty[s0]);
           if (!mw(&B.xf_k[s1], ph1, ot + 1)) break;
           issue_p(s1, s1, static_cast<uint32_t>(pad1));                                 // C
@@ -520,7 +530,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
     blk_first<tpb>(p, it, wk);
     for (; it.valid; blk_next<tpb>(p, it, wk)) {
       int vr0, vr1;
-      const int n = blk_tiles<tpb>(it, vr0, vr1);
+      const int n = blk_tiles<tpb, kRev>(it, vr0, vr1);
       bool ok = true;
       for (int u = 0; u < n && ok; ++u) {
         const uint32_t t = ot + u, sl = t & 1u;
@@ -555,7 +565,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
     bool ok = true;
     for (; it.valid && ok; blk_next<tpb>(p, it, wk)) {
       int vr0, vr1;
-      const int n = blk_tiles<tpb>(it, vr0, vr1);
+      const int n = blk_tiles<tpb, kRev>(it, vr0, vr1);
       for (int u = 0; u < n; ++u) {
         const uint32_t t = ot + u, sl = t & 1u;   // landing slot and phi(Q) tile in TMEM
         if (!tcu::wait_warp(&B.full_q[sl], (t >> 1) & 1u, abort_flag, err, SITE_TC_TRANSFORM, t) ||
@@ -612,9 +622,9 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
           for (int e = 0; e < 8; ++e) {
             const int j = 32 * c + 16 * hh + 2 * e;
             float a = __uint_as_float(x[16 * hh + 2 * e]), b = __uint_as_float(x[16 * hh + 2 * e + 1]);
-            if (diag) {   // keys up to the query row
-              a = (j <= r) ? a : 0.f;
-              b = (j + 1 <= r) ? b : 0.f;
+            if (diag) {   // keys up to the query row; from it on when time runs backwards
+              a = (kRev ? j >= r : j <= r) ? a : 0.f;
+              b = (kRev ? j + 1 >= r : j + 1 <= r) ? b : 0.f;
             }
             pk[e] = pack_bf16x2(a, b);
           }
@@ -631,10 +641,11 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
     blk_first<tpb>(p, it, wk);
     for (; it.valid && ok; blk_next<tpb>(p, it, wk)) {
       int vr0, vr1;
-      const int n = blk_tiles<tpb>(it, vr0, vr1);
-      // jobs A (tile 0, masked), then for two tiles B (dense) and C (tile 1, masked)
+      const int n = blk_tiles<tpb, kRev>(it, vr0, vr1);
+      // jobs A (tile 0, masked), then for two tiles B (dense, over tile 0's keys) and C (tile
+      // 1, masked); going backwards in time tile 0 may be the sequence's partial tile
 #pragma unroll 1
-      for (int j = 0; j < 2 * n - 1 && ok; ++j) ok = conv(j == 0 ? pad_rows(vr0) : (j == 1 ? 128 : pad_rows(vr1)), j != 1);
+      for (int j = 0; j < 2 * n - 1 && ok; ++j) ok = conv(j == 1 ? pad_rows(vr0) : pad_rows(j == 0 ? vr0 : vr1), j != 1);
     }
   }
   // ------------------------------------------------------------------------------------
@@ -667,7 +678,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
       if (!tcu::wait_warp(&B.o_full, t & 1u, abort_flag, err, SITE_TC_EPILOGUE, t)) return false;
       tc_fence_after();
       const int i = bi.jb * tpb + u;
-      const int64_t row = bi.row0 + static_cast<int64_t>(i) * kTile + r;
+      const int64_t row = bi.row0 + static_cast<int64_t>(phys_tile<kRev>(i, bi.nt)) * kTile + r;
       const bool valid = r < vr;
       uint16_t* dst = p.out + row * HD + h * kD;
       float ss = 0.f;
@@ -699,7 +710,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
     auto publish = [&](const BlkIter& bi, int u, int vr) {
       if (!norm) return;
       const int i = bi.jb * tpb + u;
-      const int64_t row = bi.row0 + static_cast<int64_t>(i) * kTile + r;
+      const int64_t row = bi.row0 + static_cast<int64_t>(phys_tile<kRev>(i, bi.nt)) * kTile + r;
       if (r < vr) tcu::red_add_f64(p.ss + row * kSsStride, static_cast<double>(ss_row));
       tcu::fence_acq_rel_gpu();
       __syncwarp();
@@ -757,7 +768,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
     blk_first<tpb>(p, it, wk);
     for (; it.valid && ok; blk_next<tpb>(p, it, wk)) {
       int vr0, vr1;
-      const int n = blk_tiles<tpb>(it, vr0, vr1);
+      const int n = blk_tiles<tpb, kRev>(it, vr0, vr1);
       const bool first = it.jb == 0, last = it.jb == it.nblk - 1;
       if (first) {   // S0 into TMEM and the snapshot
         const int64_t ir = in_row(it.s);
@@ -832,7 +843,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
     blk_first<tpb>(p, it, wk);
     for (; it.valid && ok; blk_next<tpb>(p, it, wk)) {
       int vr0, vr1;
-      const int n = blk_tiles<tpb>(it, vr0, vr1);
+      const int n = blk_tiles<tpb, kRev>(it, vr0, vr1);
       for (int u = 0; u < n && ok; ++u, ++ot) {
         const int i = it.jb * tpb + u;                 // tile of the sequence
         const int vr = u == 0 ? vr0 : vr1;
@@ -845,7 +856,7 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
           break;
         }
         (void)ld_acquire_gpu(cnt);
-        const int64_t base = it.row0 + static_cast<int64_t>(i) * kTile;
+        const int64_t base = it.row0 + static_cast<int64_t>(phys_tile<kRev>(i, it.nt)) * kTile;
         // Lane l holds the norm factor of row 16e + (l & 15).
         const int myrt = 16 * e + (lane & 15);
         const double myss = myrt < vr ? tcu::ld_cg_f64(p.ss + (base + myrt) * kSsStride) : 0.0;
@@ -931,13 +942,16 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
 inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 using PairKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, PairParams);
-PairKernel pair_kernel(int mode, int C) {
-  static const PairKernel k[3][2] = {
-      {lightning_prefill_pair_kernel<LA_OUT_RAW, 128>, lightning_prefill_pair_kernel<LA_OUT_RAW, 256>},
-      {lightning_prefill_pair_kernel<LA_OUT_RMSNORM, 128>, lightning_prefill_pair_kernel<LA_OUT_RMSNORM, 256>},
-      {lightning_prefill_pair_kernel<LA_OUT_RMSNORM_GATE, 128>,
-       lightning_prefill_pair_kernel<LA_OUT_RMSNORM_GATE, 256>}};
-  return k[mode == LA_OUT_RAW ? 0 : (mode == LA_OUT_RMSNORM ? 1 : 2)][C == 256 ? 1 : 0];
+PairKernel pair_kernel(int mode, int C, bool rev) {
+  static const PairKernel k[4][2] = {
+      {lightning_prefill_pair_kernel<LA_OUT_RAW, 128, false>, lightning_prefill_pair_kernel<LA_OUT_RAW, 256, false>},
+      {lightning_prefill_pair_kernel<LA_OUT_RMSNORM, 128, false>,
+       lightning_prefill_pair_kernel<LA_OUT_RMSNORM, 256, false>},
+      {lightning_prefill_pair_kernel<LA_OUT_RMSNORM_GATE, 128, false>,
+       lightning_prefill_pair_kernel<LA_OUT_RMSNORM_GATE, 256, false>},
+      {lightning_prefill_pair_kernel<LA_OUT_RAW, 128, true>, lightning_prefill_pair_kernel<LA_OUT_RAW, 256, true>}};
+  const int m = rev ? 3 : (mode == LA_OUT_RAW ? 0 : (mode == LA_OUT_RMSNORM ? 1 : 2));
+  return k[m][C == 256 ? 1 : 0];
 }
 
 }  // namespace
@@ -950,7 +964,7 @@ int pair_max_active_clusters() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   std::lock_guard<std::mutex> lock(mu);
   if (cache[dev] == 0) {
-    PairKernel kern = pair_kernel(LA_OUT_RMSNORM_GATE, 256);
+    PairKernel kern = pair_kernel(LA_OUT_RMSNORM_GATE, 256, false);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes)) !=
         cudaSuccess)
       return 0;
@@ -1074,7 +1088,7 @@ size_t pair_workspace_bytes(int nseq, int max_len, int64_t tokens, int H) {
 }
 
 cudaError_t launch_pair_prefill(const TcArgs& a, cudaStream_t stream) {
-  if (a.reverse || a.D != kD || (a.C != 128 && a.C != 256)) return cudaErrorInvalidValue;
+  if (a.D != kD || (a.C != 128 && a.C != 256) || (a.reverse && a.mode != LA_OUT_RAW)) return cudaErrorInvalidValue;
   const int max_tiles = (a.max_len + kTile - 1) / kTile;
   const size_t cnt_bytes =
       up256(sizeof(unsigned int) * kCntStride * static_cast<size_t>(a.nseq) * (max_tiles ? max_tiles : 1));
@@ -1126,7 +1140,7 @@ cudaError_t launch_pair_prefill(const TcArgs& a, cudaStream_t stream) {
     p.sched = sched;
     p.wstart = wstart;
   }
-  const PairKernel kernel = pair_kernel(a.mode, a.C);
+  const PairKernel kernel = pair_kernel(a.mode, a.C, a.reverse != 0);
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};

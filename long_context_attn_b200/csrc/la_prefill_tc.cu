@@ -1047,8 +1047,8 @@ size_t tc_workspace_bytes(int nseq, int max_len, int64_t tokens, int H, int D, i
 
 cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream) {
   (void)num_sms;
-  // Forward time runs on the pair kernel; this kernel serves the reverse-time passes.
-  if (!a.reverse) return launch_pair_prefill(a, stream);
+  // Both directions of time run on the pair kernel.
+  return launch_pair_prefill(a, stream);
   const int max_tiles = (a.max_len + kTile - 1) / kTile;
   const size_t cnt_bytes = up256(sizeof(unsigned int) * static_cast<size_t>(a.nseq) * (max_tiles ? max_tiles : 1));
   const size_t ss_bytes = up256(sizeof(double) * static_cast<size_t>(a.tokens > 0 ? a.tokens : 1));

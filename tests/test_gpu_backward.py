@@ -189,7 +189,8 @@ def test_backward_128k_full_size_samples(cuda_device):
                                                            la.LA_BF16, la.LA_OUT_RAW))
     la.lightning_attn_backward(dq_, dk_, dv_, None, ddo, gq, gk, gv, block_size=w.block_size, mode=la.LA_OUT_RAW,
                                workspace=ws)
-    assert la.lightning_attn_last_path() == "tcgen05"
+    # every pass (forward and reverse time) runs the 64 heads' sequence as two parallel chunks
+    assert la.lightning_attn_last_path() == "tcgen05+chunks"
     la.lightning_attn_check(ws)
     got_q = to_host(gq[0, :n])
     got_k, got_v = to_host(gk[0, T - n:]), to_host(gv[0, T - n:])
