@@ -944,8 +944,8 @@ def _measure_secondary(name, device, peaks):
 KERNEL_SOURCES = {
     "prefill": ("la_prefill_pair.cu", "la_state_tc.cu", "la_tc_util.cuh", "la_sm100.cuh", "la_common.cuh"),
     "decode": ("la_decode.cu", "la_common.cuh"),
-    "backward": ("la_backward.cu", "la_api.cu", "la_prefill_tc.cu", "la_prefill_pair.cu", "la_state_tc.cu",
-                 "la_tc_util.cuh", "la_sm100.cuh", "la_common.cuh"),
+    "backward": ("la_backward.cu", "la_api.cu", "la_prefill_pair.cu", "la_state_tc.cu", "la_tc_util.cuh",
+                 "la_sm100.cuh", "la_common.cuh"),
 }
 
 

@@ -1,6 +1,6 @@
 // C ABI of the Lightning Attention library: argument validation, kernel selection,
 // workspace carving and the device error record.  Every compute step runs in the
-// kernels of la_decode.cu, la_simt.cu and la_prefill_tc.cu; there is no CPU path.
+// kernels of la_decode.cu, la_simt.cu and la_prefill_pair.cu; there is no CPU path.
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
@@ -115,23 +115,12 @@ constexpr int kSplitMinChunk = 1024;
 struct SplitPlan {
   int S, Tc;
 };
-SplitPlan split_plan(int B, int T, int H, int D) {
-  SplitPlan sp{1, T};
-  if (D != 128 || B < 1 || H < 1 || T < 2 * kSplitMinChunk) return sp;
-  const int groups = la::max_active_clusters() / H;   // CTA-pair groups that fit at once
-  if (groups < 2 * B) return sp;
-  const int S = std::min(groups / B, T / kSplitMinChunk);
-  if (S < 2) return sp;
-  sp.Tc = ((T + S - 1) / S + 127) / 128 * 128;
-  sp.S = (T + sp.Tc - 1) / sp.Tc;
-  return sp;
-}
-// Forward time (pair kernel): 2G workers per head, each owning whole sequences.  With fewer
-// sequences than workers, each sequence is cut into S chunks (whole blocks of C rows) so
-// that every worker has one: chunk c starts from S0 plus the states of the chunks before it
-// (chunk-state kernel over all but the last chunk, then the ordered prefix), and the last
-// chunk's final state is the sequence's.
-SplitPlan forward_split_plan(int B, int T, int H, int D, int C) {
+// 2G workers per head, each owning whole sequences.  With fewer sequences than workers,
+// each sequence is cut into S chunks (whole blocks of C rows) so that every worker has one:
+// chunk c starts from S0 plus the states of the chunks before it (after it, when time runs
+// backwards) -- the chunk-state kernel, then the ordered prefix -- and the sequence's final
+// state comes from its last chunk (backwards: from the prefix).
+SplitPlan chunk_plan(int B, int T, int H, int D, int C) {
   SplitPlan sp{1, T};
   if (D != 128 || B < 1 || H < 1 || T < 2 * kSplitMinChunk) return sp;
   const int workers = 2 * std::max(1, la::pair_max_active_clusters() / H);
@@ -170,9 +159,7 @@ size_t prefill_ws_bytes(Path p, int nseq, int max_len, int64_t tokens, int H, in
     // A fixed-length call may split (B = nseq, T = max_len); room for that is reserved here
     // (a packed call never splits and at most over-reserves).
     size_t n = la::tc_workspace_bytes(nseq, max_len, tokens, H, D, C);
-    const SplitPlan sp = split_plan(nseq, max_len, H, D);
-    if (sp.S > 1) n = std::max(n, split_layout(sp, nseq, tokens, H, D, C).total);
-    const SplitPlan fp = forward_split_plan(nseq, max_len, H, D, C);
+    const SplitPlan fp = chunk_plan(nseq, max_len, H, D, C);
     if (fp.S > 1) n = std::max(n, split_layout(fp, nseq, tokens, H, D, C).total);
     return kErrBytes + n;
   }
@@ -216,7 +203,7 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
     a.reverse = reverse ? 1 : 0;
     const bool fixed = !cu && T_fixed > 0;
     const SplitPlan sp = !fixed ? SplitPlan{1, T_fixed}
-                                : forward_split_plan(nseq, T_fixed, H, D, C);
+                                : chunk_plan(nseq, T_fixed, H, D, C);
     if (sp.S > 1) {
       const SplitLayout sl = split_layout(sp, nseq, tokens, H, D, C);
       char* x = ws + sl.tc;

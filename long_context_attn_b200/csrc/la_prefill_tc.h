@@ -39,12 +39,11 @@ bool tc_eligible(const TcShape& s, int num_sms);
 // Workspace bytes after the 256-byte error record.
 size_t tc_workspace_bytes(int nseq, int max_len, int64_t tokens, int H, int D, int C);
 cudaError_t launch_tc_prefill(const TcArgs& a, int num_sms, cudaStream_t stream);
-// CTA pairs (heads x groups) that fit on the current device at once (the smaller count of
-// the two tensor-core prefill kernels).
+// CTA pairs (heads x groups) that fit on the current device at once.
 int max_active_clusters();
 
-// The forward-time prefill (la_prefill_pair.cu): one head per CTA pair, blocks alternating
-// between the two CTAs, the state handed over through a per-pair buffer in the workspace.
+// The kernel (la_prefill_pair.cu): each CTA of a head's pair is a worker that owns whole
+// sequences (or chunks of one) with the state in its TMEM; time runs either way.
 cudaError_t launch_pair_prefill(const TcArgs& a, cudaStream_t stream);
 size_t pair_workspace_bytes(int nseq, int max_len, int64_t tokens, int H);
 int pair_max_active_clusters();

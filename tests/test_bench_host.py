@@ -58,5 +58,5 @@ def test_backward_accounting():
     w = bench.synth.WORKLOADS["backward_128k"]
     assert w.kind == "backward" and w.T == 131072 and w.seed == 1007
     # the kernel-source hash of the backward covers the prefill kernel its passes run on
-    assert "la_prefill_tc.cu" in bench.KERNEL_SOURCES["backward"]
+    assert "la_prefill_pair.cu" in bench.KERNEL_SOURCES["backward"]
     assert "la_backward.cu" in bench.KERNEL_SOURCES["backward"]
