@@ -213,25 +213,27 @@ la_status common_prefill(const void* q, const void* k, const void* v, const void
       float* cpart = reinterpret_cast<float*>(x + sl.cu + 2 * sl.st);
       const int n = nseq * sp.S;
       e = la::launch_chunk_cu(ccu, nseq, T_fixed, sp.Tc, sp.S, stream);
-      // Forward time with one sequence: the last chunk's state is never needed (the kernel
-      // ends that chunk with the sequence's final state), and the first S - 1 chunks are
-      // contiguous, so only they are summed.
-      const bool skip_last = !reverse && nseq == 1;
+      // One sequence: the state of the chunk that ends the walk (the last, or the first when
+      // time runs backwards) is never needed -- the kernel ends that chunk with the sequence's
+      // final state -- and the other S - 1 chunks are contiguous, so only they are summed.
+      const bool skip_one = nseq == 1;
+      const size_t chunk_floats = static_cast<size_t>(H) * D * D;
       if (e == cudaSuccess)
-        e = la::launch_chunk_state_tc(k, v, nullptr, cst, cpart, ccu, skip_last ? n - 1 : n, 0, sp.Tc, tokens, H,
-                                      phi_id, current_sm_count(), err, stream);
-      if (e == cudaSuccess)   // chunk initial states (and, reverse time, the sequences' final states)
-        e = la::launch_chunk_prefix(cst, state_in, cin, reverse ? state_out : nullptr, nseq, sp.S, H,
+        e = la::launch_chunk_state_tc(k, v, nullptr, (skip_one && reverse) ? cst + chunk_floats : cst, cpart,
+                                      (skip_one && reverse) ? ccu + 1 : ccu, skip_one ? n - 1 : n, 0, sp.Tc, tokens,
+                                      H, phi_id, current_sm_count(), err, stream);
+      if (e == cudaSuccess)   // chunk initial states (and, reverse time with several sequences, their final states)
+        e = la::launch_chunk_prefix(cst, state_in, cin, (reverse && !skip_one) ? state_out : nullptr, nseq, sp.S, H,
                                     reverse ? 1 : 0, current_sm_count(), stream);
       a.cu = ccu;
       a.nseq = n;
       a.T = 0;
       a.max_len = sp.Tc;
       a.state_in = cin;
-      if (reverse) {
+      if (reverse && !skip_one) {
         a.state_out = nullptr;
       } else {
-        a.chunk_div = sp.S;   // the kernel writes each sequence's final state from its last chunk
+        a.chunk_div = sp.S;   // the kernel writes the sequence's final state from the chunk ending the walk
       }
     }
     if (e == cudaSuccess) e = la::launch_tc_prefill(a, current_sm_count(), stream);

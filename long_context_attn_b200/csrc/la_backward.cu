@@ -116,6 +116,73 @@ __global__ void __launch_bounds__(256) bwd_norm_gate_token_kernel(const T* y, co
   }
 }
 
+// The same for bf16 rows of exactly 2048 VPT elements (H * D = 8192 at 64 heads of 128):
+// each thread keeps its VPT vectors of y, dout and g, and the gate's sigmoid, in registers
+// between the two sums and the outputs, so every row is read from memory once.
+template <int VPT>
+__global__ void __launch_bounds__(256) bwd_norm_gate_row_kernel(const uint16_t* y, const uint16_t* __restrict__ g,
+                                                          const uint16_t* __restrict__ dout,
+                                                          const float* __restrict__ w, uint16_t* dy,
+                                                          uint16_t* __restrict__ dg, int gate, float eps) {
+  constexpr int HD = 256 * kVec * VPT;
+  __shared__ float red[2][8];
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * HD;
+  uint4 yr[VPT], dr[VPT], gr[VPT];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int c = (threadIdx.x + 256 * j) * kVec;
+    yr[j] = Vec8<uint16_t>::load_raw(y + base + c);
+    dr[j] = Vec8<uint16_t>::load_raw(dout + base + c);
+    gr[j] = gate ? Vec8<uint16_t>::load_raw(g + base + c) : make_uint4(0, 0, 0, 0);
+  }
+  float sg[VPT][kVec];
+  float ss = 0.f, su = 0.f;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int c = (threadIdx.x + 256 * j) * kVec;
+    float yv[kVec], dv[kVec], gv[kVec];
+    Vec8<uint16_t>::unpack(yr[j], yv);
+    Vec8<uint16_t>::unpack(dr[j], dv);
+    Vec8<uint16_t>::unpack(gr[j], gv);
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+      sg[j][i] = gate ? sig(gv[i]) : 1.0f;
+      const float u = dv[i] * (w ? __ldg(w + c + i) : 1.0f) * sg[j][i];
+      ss = fmaf(yv[i], yv[i], ss);
+      su = fmaf(u, yv[i], su);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    su += __shfl_xor_sync(0xffffffffu, su, o);
+  }
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) { red[0][warp] = ss; red[1][warp] = su; }
+  __syncthreads();
+  ss = 0.f; su = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) { ss += red[0][i]; su += red[1][i]; }
+  const float r = 1.0f / sqrtf(ss / static_cast<float>(HD) + eps);
+  const float coef = r * r * r * su / static_cast<float>(HD);
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int c = (threadIdx.x + 256 * j) * kVec;
+    float yv[kVec], dv[kVec], o[kVec], og[kVec];
+    Vec8<uint16_t>::unpack(yr[j], yv);
+    Vec8<uint16_t>::unpack(dr[j], dv);
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+      const float s = sg[j][i];
+      const float wc = w ? __ldg(w + c + i) : 1.0f;
+      o[i] = r * dv[i] * wc * s - coef * yv[i];
+      og[i] = dv[i] * yv[i] * r * wc * s * (1.0f - s);
+    }
+    Vec8<uint16_t>::store(dy + base + c, o);
+    if (gate) Vec8<uint16_t>::store(dg + base + c, og);
+  }
+}
+
 // The norm/gate backward with the norm weight's gradient, in one pass over the tokens.  RAW
 // is not launched (dy = dout).  With r = 1/sqrt(mean(y^2) + eps), s = sigmoid(g) (1 without
 // the gate) and u = dout * w * s, per token:
@@ -444,7 +511,17 @@ cudaError_t launch_bwd_norm_gate(const void* y, const void* g, const void* dout,
     return cudaGetLastError();
   }
   if (!dw) {
-    if (dt == LA_BF16)
+    if (dt == LA_BF16 && (HD == 4096 || HD == 8192)) {
+      const auto yb = static_cast<const uint16_t*>(y), gb = static_cast<const uint16_t*>(g),
+                 db = static_cast<const uint16_t*>(dout);
+      auto dyb = static_cast<uint16_t*>(dy), dgb = static_cast<uint16_t*>(dg);
+      if (HD == 8192)
+        bwd_norm_gate_row_kernel<4><<<static_cast<unsigned>(tokens), 256, 0, stream>>>(yb, gb, db, w, dyb, dgb, gate,
+                                                                                        eps);
+      else
+        bwd_norm_gate_row_kernel<2><<<static_cast<unsigned>(tokens), 256, 0, stream>>>(yb, gb, db, w, dyb, dgb, gate,
+                                                                                        eps);
+    } else if (dt == LA_BF16)
       bwd_norm_gate_token_kernel<uint16_t><<<static_cast<unsigned>(tokens), 256, 0, stream>>>(
           static_cast<const uint16_t*>(y), static_cast<const uint16_t*>(g), static_cast<const uint16_t*>(dout), w,
           static_cast<uint16_t*>(dy), static_cast<uint16_t*>(dg), HD, gate, eps);

@@ -740,8 +740,8 @@ lightning_prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __
       if (!p.state_out) return -1;
       int64_t slot = s;
       if (p.state_index) slot = __ldg(p.state_index + s);
-      else if (p.chunk_div > 1) {
-        if (s % p.chunk_div != p.chunk_div - 1) return -1;
+      else if (p.chunk_div > 1) {   // the chunk that ends the walk holds the sequence's final state
+        if (s % p.chunk_div != (kRev ? 0 : p.chunk_div - 1)) return -1;
         slot = s / p.chunk_div;
       }
       return ((slot * p.H + h) * kD + r) * kD;

@@ -30,8 +30,9 @@ struct TcArgs {
   char* ws;            // workspace after the error record
   const int* state_index;  // optional [nseq] device: state slot of each sequence (else s)
   int skip_single;         // nonzero: sequences of exactly one token are left alone entirely
-  int chunk_div;           // > 1 (forward only): sequence s is chunk s % chunk_div of sequence
-                           // s / chunk_div; only a last chunk writes state_out (at s / chunk_div)
+  int chunk_div;           // > 1: sequence s is chunk s % chunk_div of sequence s / chunk_div;
+                           // only the chunk that ends the walk (the last one, or the first when
+                           // time runs backwards) writes state_out (at s / chunk_div)
 };
 
 // True when the tensor-core kernel handles this shape on a GPU with `num_sms` SMs.

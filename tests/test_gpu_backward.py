@@ -76,6 +76,13 @@ def test_backward_tc_lengths(T, cuda_device):
     _run_fixed(1, T, 8, 128, 256, "bf16", "rmsnorm_gate", False, 3101 + T, expect="tcgen05", want_dw=T >= 256)
 
 
+@pytest.mark.parametrize("H", [32, 64])
+def test_backward_wide_rows_gated(H, cuda_device):
+    """H * D = 4096 and 8192 without the norm weight's gradient: the norm/gate backward keeps
+    each token's row in registers (one read of y, dout and g)."""
+    _run_fixed(1, 300, H, 128, 256, "bf16", "rmsnorm_gate", True, 3601 + H, expect="tcgen05", want_dw=False)
+
+
 def test_backward_fp32_path(cuda_device):
     _run_fixed(2, 150, 4, 64, 64, "f32", "rmsnorm_gate", True, 3201, expect="simt")
 
