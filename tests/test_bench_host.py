@@ -30,7 +30,7 @@ def test_clock_summary_parses_nvidia_smi_csv():
     assert s["reasons"] == ["sw_power_cap"]
 
 
-@pytest.mark.parametrize("workload", ["prefill_8k", "backward_8k"])
+@pytest.mark.parametrize("workload", ["prefill_8k", "backward_8k", "tiny_f32"])
 def test_reference_arm_prints_one_json_line(workload):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
                         "--warmup", "0", "--workload", workload], capture_output=True, text=True, timeout=600)
@@ -60,3 +60,13 @@ def test_backward_accounting():
     # the kernel-source hash of the backward covers the prefill kernel its passes run on
     assert "la_prefill_pair.cu" in bench.KERNEL_SOURCES["backward"]
     assert "la_backward.cu" in bench.KERNEL_SOURCES["backward"]
+
+
+def test_secondary_configs_are_bench_workloads():
+    """The default line's extra keys: each a workload the bench can build a case for."""
+    assert set(bench.SECONDARY_STEPS) == {"decode_256", "varlen_16", "prefill_8k", "tiny_f32"}
+    for name, steps in bench.SECONDARY_STEPS.items():
+        w = bench.synth.WORKLOADS[name]
+        assert steps >= 10
+        assert w.kind in ("prefill", "varlen", "decode")
+    assert bench.synth.WORKLOADS["tiny_f32"].dtype == "f32"
