@@ -99,11 +99,13 @@ typedef enum {
  *   block_size   the block (chunk) size C, 1..1024.  bf16 with D = 128 and C in {128, 256} runs
  *                on the tcgen05 tensor-core kernel; every other valid combination runs on the
  *                CUDA-core kernel (fp32 arithmetic).  lightning_attn_last_path() names the one used.
- *                On the tensor-core kernel: with few heads, groups of CTA pairs share the
- *                sequences, and a long sequence (T >= 2048) may be cut into chunks that run in
- *                parallel from the states of the chunks before them ("tcgen05+chunks"); in a
- *                norm mode with more heads than CTA pairs fit at once, the norm runs as a
- *                second per-token pass ("tcgen05+norm").  The result is the same up to rounding.
+ *                On the tensor-core kernel each CTA of a head's pair is a worker that owns
+ *                whole sequences (with few heads, several groups of pairs share them); when a
+ *                call has fewer sequences than workers per head, a sequence of T >= 2048 is
+ *                cut into chunks that run in parallel from the states of the chunks before
+ *                them ("tcgen05+chunks": at 64 heads, two chunks); in a norm mode with more
+ *                heads than CTA pairs fit at once, the norm runs as a second per-token pass
+ *                ("tcgen05+norm").  The result is the same up to rounding.
  *   eps          RMSNorm epsilon (> 0 for the norm modes).
  *   norm_weight  fp32 [H*D] RMSNorm weight, or NULL for ones.
  *   workspace    device scratch of >= lightning_attn_workspace_size(LA_OP_PREFILL, ...)
